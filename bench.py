@@ -1,0 +1,349 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200.
+
+Headline: chunkwise prefill tokens/s on B=8, H=32, T=8192, dk=dv=128 (bf16
+q/k/v, fp32 gates and state), one prefill call per step, inputs resident in
+HBM (2.7 GB of inputs: larger than the 126 MB L2, so no flush is needed).
+Beside it: the recurrent decode (256 sequences x 32 heads, in-place fp32
+state, one token per step) as state GB/s, the roofline fractions, the fp64
+CPU oracle timed on this host's cores, and an end-to-end figure through the
+public host-buffer API (pinned host -> device copies, prefill, copies back).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched with torch.distributed.run): every rank processes its own
+full batch (weak scaling; units are independent, no data-path collective);
+timing is the max over ranks of CUDA-event time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_workloads as W  # noqa: E402
+
+METRIC = "KDA prefill tokens/s (B8 H32 T8192 d128) + decode state GB/s, % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# Algorithmic work per token-head at dk = dv = 128, C = 64 (minimum traffic:
+# q, k, v bf16 + g fp32 + beta fp32 + o bf16; flops of the dense chunk
+# contractions A, P, W, U, P.E, W.S, Q.S, K^T.E).
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 256 + 512 + 4 + 256
+PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * 128 * 128 + 2 * 64 * (3 * 128 + 2 * 128)
+STATE_BYTES = 128 * 128 * 4
+# decode: state read + write, q, k, v, o bf16, g fp32, beta fp32 per head-step
+DECODE_BYTES_PER_HEAD_STEP = 2 * STATE_BYTES + 3 * 256 + 512 + 4 + 256
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling during the timed region (clocks and throttle reasons)."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, f in enumerate(fl) if f.lower() == "active"})
+        loaded = [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": reasons}
+
+
+def dist_setup(n_gpus):
+    if n_gpus <= 1 or "RANK" not in os.environ:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    rank, world = dist.get_rank(), dist.get_world_size()
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_baseline(w, target_s=15.0):
+    """Time the fp64 CPU oracle on a bounded sample of workload ``w``: whole
+    (sequence, head) units of the full length T, enough of them for about
+    ``target_s`` seconds of work on this host's cores."""
+    import oracle
+    cores = oracle.max_threads()
+    cal = W.make_prefill(1, 512, 2, w.dk, w.dv, w.dtype, w.g_mu, w.g_sigma, 0.0, seed=w.seed + 1)
+    t0 = time.perf_counter()
+    oracle.recurrent(cal["q"], cal["k"], cal["v"], cal["g"], cal["beta"], num_threads=cores)
+    rate = 1024 / max(time.perf_counter() - t0, 1e-6)  # token-heads/s (rough)
+    units = max(cores, int(target_s * rate / w.T))
+    units = min(units, w.B * w.H)
+    # the sample: `units` heads of the first sequence(s), full length, same recipe
+    sample = W.make_prefill(1, w.T, units, w.dk, w.dv, w.dtype, w.g_mu, w.g_sigma, w.s0_std,
+                            seed=w.seed)
+    t0 = time.perf_counter()
+    oracle.recurrent(sample["q"], sample["k"], sample["v"], sample["g"], sample["beta"],
+                     sample["S0"], num_threads=cores)
+    dt = time.perf_counter() - t0
+    token_heads = units * w.T
+    return {"value": token_heads / dt / w.H, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{units} (sequence, head) units x {w.T} tokens of the {w.name} recipe "
+                      f"({token_heads} token-heads, fp64 token-by-token recurrence, {dt:.1f} s); "
+                      f"tokens/s = token-heads/s / H"}, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.PREFILL_B8
+    import oracle  # noqa: F401  (built on import of the first call)
+    values = []
+    total = 0.0
+    base = None
+    for i in range(args.warmup + args.steps):
+        base, dt = oracle_baseline(w, target_s=max(2.0, 60.0 / max(args.steps + args.warmup, 1)))
+        if i >= args.warmup:
+            values.append(base["value"])
+            total += dt
+    value = statistics.median(values)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / max(args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                       "chunk": w.chunk},
+            "cpu_baseline": dict(base, value=value),
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def time_launches(fn, steps, stream):
+    """CUDA-event time of `steps` calls of fn() on `stream` (ms per call)."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / steps
+
+
+def run_ours(args):
+    import kimi_delta_attention_31_b200 as kda
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    w = W.PREFILL_B8
+
+    # ---------------- prefill (headline) ----------------
+    inp = W.make_workload(w, dev)
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    ws_bytes = kda.workspace_size(B, T, H, dk, dv, 0, w.chunk, torch.bfloat16)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    launches_per_prefill = kda.launches_per_chunk_fwd(dk, dv, w.chunk, torch.bfloat16)
+
+    def prefill():
+        kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], None, w.chunk,
+                      o=o, S_out=S_out, workspace=ws)
+
+    for _ in range(args.warmup):
+        prefill()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = time_launches(prefill, args.steps, stream)
+        # per-kernel breakdown of the same calls (events between the launches)
+        kernel_ms = kda.profile_chunk_fwd(prefill, stream, repeats=max(1, min(args.steps, 5)),
+                                          dk=dk, dv=dv, chunk_size=w.chunk)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_max = max_over_ranks(ms, world, dev)
+    tokens = B * T
+    value = world * tokens / (ms_max * 1e-3)
+    clocks = clk.summary()
+
+    token_heads = B * T * H
+    alg_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + B * H * STATE_BYTES  # S_out
+    alg_flops = token_heads * PREFILL_FLOPS_PER_TOKEN_HEAD
+    dom_name, dom_ms = max(kernel_ms.items(), key=lambda kv: kv[1])
+    dom_bytes = kda.algorithmic_bytes_per_launch(dom_name, token_heads, B * H, d=dk)
+    achieved_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom_name, "achieved": achieved_gbs,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
+                "traffic": None, "peak_source": f"{peak_src} HBM copy bandwidth",
+                "kernel_ms": kernel_ms,
+                "whole_call": {"alg_bytes": alg_bytes, "achieved_gbs": alg_bytes / (ms * 1e-3) / 1e9,
+                               "hbm_frac": alg_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                               "alg_tflops": alg_flops / (ms * 1e-3) / 1e12,
+                               "tensor_frac_of_burst": alg_flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}}
+    del inp, o, S_out, ws
+    torch.cuda.empty_cache()
+
+    # ---------------- end to end through the host-buffer API ----------------
+    host = W.make_workload(w, "cpu")
+    host = {n: (t.pin_memory() if t is not None else None) for n, t in host.items()}
+    runner = kda.HostPrefill(host, dev, w.chunk)
+    e2e_steps = max(1, min(args.steps, 3))
+    runner(host)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = time_launches(lambda: runner(host), e2e_steps, stream)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    e2e = {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": runner.h2d_bytes(host), "d2h_bytes_per_step": runner.d2h_bytes(),
+           "ms_per_step": e2e_ms}
+    del runner, host
+    torch.cuda.empty_cache()
+
+    # ---------------- decode: 256 x 32 heads, 1024 steps, in place ----------------
+    dw = W.DECODE
+    N, Hd, dd = dw.B, dw.H, dw.dk
+    S = W.make_decode_state(N, Hd, dd, dd, dw.s0_std, seed=dw.seed, device=dev)
+    nsteps = dw.T
+    xs = W.make_decode_steps(N, Hd, dd, dd, nsteps, dw.dtype, dw.g_mu, dw.g_sigma, seed=dw.seed,
+                             device=dev)
+    od = torch.empty((N, Hd, dd), dtype=torch.bfloat16, device=dev)
+    step = [0]
+
+    def decode_step():
+        t = step[0] % nsteps
+        kda.recurrent_step(xs["q"][t], xs["k"][t], xs["v"][t], xs["g"][t], xs["beta"][t], S, o=od)
+        step[0] += 1
+
+    for _ in range(16):
+        decode_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    dec_ms = time_launches(decode_step, nsteps, stream)
+    dec_ms = max_over_ranks(dec_ms, world, dev)
+    heads = N * Hd
+    state_gbs = world * heads * 2 * STATE_BYTES / (dec_ms * 1e-3) / 1e9
+    dec_alg_gbs = heads * DECODE_BYTES_PER_HEAD_STEP / (dec_ms * 1e-3) / 1e9
+    decode = {"workload": dw.name, "value": state_gbs, "unit": "GB/s (state read+write)",
+              "us_per_step": dec_ms * 1e3, "steps": nsteps,
+              "roofline": {"bound": "hbm", "achieved": dec_alg_gbs, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": dec_alg_gbs / peaks["hbm_gbs"], "traffic": None,
+                           "kernel": "kda_decode_step_kernel"}}
+    del S, xs, od
+    torch.cuda.empty_cache()
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1 only) ----------------
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu, _ = oracle_baseline(w)
+
+    gpu_launches = args.steps * launches_per_prefill
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+                       "chunk": w.chunk, "g": f"-softplus(N({w.g_mu},{w.g_sigma}))",
+                       "l2": "inputs (2.7 GB) larger than L2; no flush",
+                       "parallelism": f"dp{world} (independent batches per GPU)"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+            "gpu_launches": gpu_launches, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

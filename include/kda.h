@@ -1,0 +1,147 @@
+/*
+ * kda.h -- C ABI of libkda: the Kimi Delta Attention (KDA) recurrence on one
+ * NVIDIA B200 (sm_100a), in its two schedules.
+ *
+ * The operation (sources are web pages, cited by title and section):
+ *   per token t, per (sequence, head), with the state S in R^{dk x dv}
+ *   (row = key channel, column = value channel), g_t = log(alpha_t) in R^dk,
+ *   beta_t in (0, 1]:
+ *     S~  = Diag(alpha_t) S_{t-1}        decay per key channel
+ *     v^  = S~^T k_t                     prediction from the key
+ *     e_t = beta_t (v_t - v^)            error
+ *     S_t = S~ + k_t e_t^T               write along the key
+ *     o_t = S_t^T q_t                    read with the query
+ *   "Kimi K3 notes 1: KDA" section 4 (projection form of the update) and
+ *   section 5 (boxed summary, decay then delta correction); "Deriving Kimi
+ *   Delta Attention from scratch" sections 3-5 (predict, error, write) and
+ *   section 6 (the fused recurrent mode for decode and the chunked mode for
+ *   prefill are two schedules of this one formula).  No output scale and no
+ *   normaliser are applied; q and k are used as given (a caller that wants
+ *   L2-normalised q, k or a 1/sqrt(dk) scale applies it beforehand).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers, row-major, densely packed, with
+ *     16-byte aligned bases.  The caller owns every buffer and the stream; the
+ *     library never allocates, frees or synchronises (except
+ *     kda_device_error, which synchronises the given stream by design).
+ *   - Calls are asynchronous on `stream`.  The return value reports argument
+ *     errors and launch errors; execution errors appear at the caller's next
+ *     synchronisation.  On any non-KDA_OK return, kda_last_error() holds a
+ *     message for the calling thread.
+ *   - dtype selects the element type of q, k, v and o (bf16 or fp32).  g, beta
+ *     and the state are always fp32.
+ *   - Supported head sizes: dk == dv in {32, 64, 128}; anything else returns
+ *     KDA_ERR_UNSUPPORTED.
+ *   - Thread safety: no global mutable state is shared between calls apart
+ *     from a device-side error word (see kda_device_error).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,    /* null pointer, negative size, bad cu_seqlens */
+  KDA_ERR_UNSUPPORTED = 2,    /* head size / chunk size / dtype not built   */
+  KDA_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned           */
+  KDA_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
+  KDA_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed       */
+  KDA_ERR_DEVICE_TIMEOUT = 6  /* a bounded device-side wait gave up         */
+} kda_status_t;
+
+typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype_t;
+
+/*
+ * Bytes of device workspace kda_chunk_fwd needs for these sizes (0 is a
+ * valid answer).  For packed inputs (num_seqs > 0) the bound assumes T total
+ * tokens split into num_seqs sequences.  Arguments as for kda_chunk_fwd.
+ */
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                    int chunk_size, kda_dtype_t dtype);
+
+/*
+ * Chunkwise-parallel prefill ("Deriving Kimi Delta Attention from scratch"
+ * section 6, chunked mode; "Linear / sparse attention" tutorial section 6.2
+ * chunk skeleton and section 5.3 WY representation): C tokens per chunk
+ * become dense matrix products plus one unit-lower-triangular solve that
+ * corrects each token's provisional error; the dk x dv fp32 state is carried
+ * from chunk to chunk.  The result equals the token-by-token recurrence up to
+ * rounding and does not depend on chunk_size.
+ *
+ *   q, k  : [B, T, H, dk]  (dtype)          g : [B, T, H, dk] fp32, log alpha <= 0
+ *   v     : [B, T, H, dv]  (dtype)       beta : [B, T, H]     fp32
+ *   S0    : [N, H, dk, dv] fp32, or NULL for a zero initial state
+ *   o     : [B, T, H, dv]  (dtype), written; must not alias an input
+ *   S_out : [N, H, dk, dv] fp32, or NULL; may alias S0
+ *   cu_seqlens : device int32 [num_seqs + 1] (packed varlen layout, B == 1,
+ *           T == total tokens, cu_seqlens[0] == 0, non-decreasing,
+ *           cu_seqlens[num_seqs] == T; the library trusts these values) or
+ *           NULL, in which case num_seqs must be 0 and N = B.
+ *   chunk_size : 16, 32 or 64.  The tensor-core path (bf16, dk == dv == 128)
+ *           runs with 64; other combinations run the fp32-arithmetic path.
+ *   workspace : device buffer of at least kda_chunk_fwd_workspace_size(...)
+ *           bytes (may be NULL when that size is 0); contents are scratch.
+ * Numerics: the tensor-core path takes bf16 operands with fp32 accumulation
+ * and an fp32 state; it is exact (no overflow) as long as every key channel's
+ * log-decay over any 16 consecutive tokens of a chunk is >= -80 (implied by
+ * per-token log alpha >= -5).  The fp32 path has no such restriction.
+ */
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* S0, void* o, float* S_out,
+                           const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
+                           int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Fused recurrent step, one token for each of N sequences ("Deriving Kimi
+ * Delta Attention from scratch" section 6, recurrent mode for decode): each
+ * (sequence, head) state is read once and written once, in place.
+ *
+ *   q, k : [N, H, dk] (dtype)    v : [N, H, dv] (dtype)
+ *   g    : [N, H, dk] fp32       beta : [N, H] fp32
+ *   S    : [N, H, dk, dv] fp32, updated in place
+ *   o    : [N, H, dv] (dtype), written
+ */
+kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, float* S, void* o, int N, int H, int dk,
+                                int dv, kda_dtype_t dtype, cudaStream_t stream);
+
+/* Message describing the calling thread's last failure ("" if none). */
+const char* kda_last_error(void);
+
+/*
+ * Reads and clears the device-side error word that bounded waits inside the
+ * kernels set when they give up (KDA_ERR_DEVICE_TIMEOUT).  Synchronises
+ * `stream` first.  *code receives 0 when no wait gave up.
+ */
+kda_status_t kda_device_error(int* code, cudaStream_t stream);
+
+/*
+ * Number of kernels one kda_chunk_fwd call with these arguments launches
+ * (1 for the fp32-arithmetic path, more for the tensor-core path).
+ */
+int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype);
+
+/*
+ * Measurement hook.  While set (events != NULL), each later kda_chunk_fwd
+ * call made by the calling thread records events[0] before its first kernel
+ * launch and events[i] after its i-th launch, on the call's stream; count
+ * must be at least kda_chunk_fwd_launches(...) + 1 or the call fails with
+ * KDA_ERR_INVALID_ARG.  The caller owns the events.  Pass NULL, 0 to stop.
+ */
+kda_status_t kda_profile_events(cudaEvent_t* events, int count);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H_ */

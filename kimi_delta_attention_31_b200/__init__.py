@@ -1,0 +1,289 @@
+"""KDA (Kimi Delta Attention) on NVIDIA B200: Python binding of libkda.
+
+Argument marshalling only: every step of the recurrence runs in the CUDA
+kernels of ``libkda.so`` (declared in ``include/kda.h``).  PyTorch supplies
+device memory and the current stream.  There is no CPU fallback: if the
+library is missing, importing the binding's functions raises.
+
+Public API
+----------
+chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, ...)
+    chunkwise prefill -> (o, S_out)
+recurrent_step(q, k, v, g, beta, S, o=None)
+    one decode token per sequence, S updated in place -> o
+chunk_fwd_host(...)
+    chunk_fwd for pinned host tensors: copies in, runs, copies results out
+workspace_size(...), last_error(), device_error(), lib_path()
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libkda.so")
+_lock = threading.Lock()
+_lib = None
+
+KDA_OK = 0
+_STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_ALIGNMENT",
+           4: "KDA_ERR_WORKSPACE", 5: "KDA_ERR_CUDA", 6: "KDA_ERR_DEVICE_TIMEOUT"}
+KDA_BF16, KDA_F32 = 0, 1
+
+# Every symbol include/kda.h declares (checked by the CPU test-suite).
+EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
+            "kda_last_error", "kda_device_error", "kda_chunk_fwd_launches", "kda_profile_events",
+            "kda_version")
+
+# Kernels of one kda_chunk_fwd call, in launch order, per path.
+KERNELS_SIMT = ("kda_chunk_simt_kernel",)
+KERNELS_TC = ("kda_tc_chunk_local_kernel", "kda_tc_state_pass_kernel")
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libkda.so (building it first if the sources are newer).  Raises if
+    it cannot be built or loaded: there is deliberately no fallback."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        from . import build as _build
+        if _build.needs_build():
+            _build.build()
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"libkda.so not found at {_LIB_PATH}; run "
+                              "python -m kimi_delta_attention_31_b200.build")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, i32, szt = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        lib.kda_chunk_fwd_workspace_size.argtypes = [i32] * 7 + [i32]
+        lib.kda_chunk_fwd_workspace_size.restype = szt
+        lib.kda_chunk_fwd.argtypes = [vp] * 9 + [i32] * 7 + [i32, vp, szt, vp]
+        lib.kda_chunk_fwd.restype = i32
+        lib.kda_recurrent_step.argtypes = [vp] * 7 + [i32] * 5 + [vp]
+        lib.kda_recurrent_step.restype = i32
+        lib.kda_last_error.argtypes = []
+        lib.kda_last_error.restype = ctypes.c_char_p
+        lib.kda_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), vp]
+        lib.kda_device_error.restype = i32
+        lib.kda_chunk_fwd_launches.argtypes = [i32] * 4
+        lib.kda_chunk_fwd_launches.restype = i32
+        lib.kda_profile_events.argtypes = [vp, i32]
+        lib.kda_profile_events.restype = i32
+        lib.kda_version.argtypes = []
+        lib.kda_version.restype = i32
+        _lib = lib
+        return lib
+
+
+def _check(st):
+    if st != KDA_OK:
+        raise KDAError(st, load_library().kda_last_error().decode())
+
+
+def last_error() -> str:
+    return load_library().kda_last_error().decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must be on a CUDA device (use chunk_fwd_host for host buffers)")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def workspace_size(B, T, H, dk, dv, num_seqs=0, chunk_size=64, dtype=torch.bfloat16) -> int:
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(load_library().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, code))
+
+
+def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, output_final_state=True,
+              o=None, S_out=None, workspace=None):
+    """Chunkwise KDA prefill.  q, k, g: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H];
+    S0: [N,H,dk,dv] fp32 or None; cu_seqlens: int32 [N+1] (B == 1) or None.
+    Returns (o, S_out) with S_out None when output_final_state is False."""
+    lib = load_library()
+    _need_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_out, workspace)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = num_seqs if cu_seqlens is not None else B
+    if g.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("g and beta must be float32")
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_out is None and output_final_state:
+        S_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    ws_need = workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, q.dtype)
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                           _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
+                           _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(q.device))
+    _check(st)
+    return o, S_out
+
+
+def recurrent_step(q, k, v, g, beta, S, o=None):
+    """One decode token per sequence: q, k, g [N,H,dk]; v [N,H,dv]; beta [N,H];
+    S [N,H,dk,dv] fp32 updated in place.  Returns o [N,H,dv]."""
+    lib = load_library()
+    _need_cuda(q, k, v, g, beta, S, o)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if S.dtype != torch.float32 or g.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("S, g and beta must be float32")
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    st = lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                N, H, dk, dv, _dtype_code(q), _stream_handle(q.device))
+    _check(st)
+    return o
+
+
+class HostPrefill:
+    """chunk_fwd over pinned HOST tensors: each call copies the inputs to the
+    device, runs the prefill and copies o and S_out back into pinned host
+    buffers (all on the current stream).  Device buffers are allocated once."""
+
+    def __init__(self, like: dict, device="cuda", chunk_size=64):
+        self.device = torch.device(device)
+        self.chunk_size = chunk_size
+        self.dev = {n: torch.empty_like(t, device=self.device) for n, t in like.items() if t is not None}
+        q, v = like["q"], like["v"]
+        B, T, H, dk = q.shape
+        cu = like.get("cu_seqlens")
+        N = cu.numel() - 1 if cu is not None else B
+        self.o_host = torch.empty((B, T, H, v.shape[-1]), dtype=q.dtype, pin_memory=True)
+        self.S_host = torch.empty((N, H, dk, v.shape[-1]), dtype=torch.float32, pin_memory=True)
+        self.o_dev = torch.empty_like(self.o_host, device=self.device)
+        self.S_dev = torch.empty_like(self.S_host, device=self.device)
+        num_seqs = 0 if cu is None else N
+        ws = workspace_size(B, T, H, dk, v.shape[-1], num_seqs, chunk_size, q.dtype)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=self.device) if ws else None
+
+    def h2d_bytes(self, host: dict) -> int:
+        return int(sum(t.numel() * t.element_size() for n, t in host.items() if t is not None and n in self.dev))
+
+    def d2h_bytes(self) -> int:
+        return int(self.o_host.numel() * self.o_host.element_size() + self.S_host.numel() * 4)
+
+    def __call__(self, host: dict):
+        for n, t in host.items():
+            if t is not None and n in self.dev:
+                self.dev[n].copy_(t, non_blocking=True)
+        d = self.dev
+        chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("S0"), d.get("cu_seqlens"),
+                  self.chunk_size, o=self.o_dev, S_out=self.S_dev, workspace=self.ws)
+        self.o_host.copy_(self.o_dev, non_blocking=True)
+        self.S_host.copy_(self.S_dev, non_blocking=True)
+        return self.o_host, self.S_host
+
+
+def chunk_fwd_host(host: dict, chunk_size=64, device="cuda"):
+    """One-shot host-buffer prefill (see HostPrefill); synchronises before returning."""
+    runner = HostPrefill(host, device, chunk_size)
+    o, S = runner(host)
+    torch.cuda.current_stream(runner.device).synchronize()
+    return o, S
+
+
+def device_error(device=None) -> int:
+    """Read-and-clear the device error word set by bounded waits (synchronises)."""
+    lib = load_library()
+    code = ctypes.c_int(0)
+    _check(lib.kda_device_error(ctypes.byref(code), _stream_handle(device)))
+    return code.value
+
+
+def launches_per_chunk_fwd(dk, dv, chunk_size, dtype=torch.bfloat16) -> int:
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(load_library().kda_chunk_fwd_launches(dk, dv, chunk_size, code))
+
+
+def kernel_names(dk, dv, chunk_size, dtype=torch.bfloat16):
+    n = launches_per_chunk_fwd(dk, dv, chunk_size, dtype)
+    return KERNELS_SIMT if n == 1 else KERNELS_TC[:n]
+
+
+def profile_chunk_fwd(call, stream, repeats=3, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16):
+    """Run ``call()`` (one chunk_fwd call) ``repeats`` times with the library's
+    event hook set and return {kernel name: mean ms per launch}."""
+    lib = load_library()
+    names = kernel_names(dk, dv, chunk_size, dtype)
+    n = len(names)
+    events = [torch.cuda.Event(enable_timing=True) for _ in range((n + 1) * repeats)]
+    totals = [0.0] * n
+    for r in range(repeats):
+        evs = events[r * (n + 1):(r + 1) * (n + 1)]
+        arr = (ctypes.c_void_p * (n + 1))(*[ctypes.c_void_p(e.cuda_event) for e in evs])
+        _check(lib.kda_profile_events(arr, n + 1))
+        try:
+            call()
+        finally:
+            lib.kda_profile_events(None, 0)
+        evs[-1].synchronize()
+        for i in range(n):
+            totals[i] += evs[i].elapsed_time(evs[i + 1])
+    return {name: t / repeats for name, t in zip(names, totals)}
+
+
+# Algorithmic bytes per launch, per kernel, for dk = dv = 128 (see the design
+# notes): the prefill's minimum traffic is q, k, v (bf16), g (fp32), beta, o
+# (bf16) = 1540 B per token-head plus the fp32 initial/final state per unit.
+# In the two-kernel tensor-core path the chunk-local kernel also writes, and
+# the state pass reads, the per-chunk WY image (1160 B per token-head).
+TC_IMAGE_BYTES_PER_TOKEN_HEAD = 1160
+
+
+def algorithmic_bytes_per_launch(kernel, token_heads, units, d=128, with_state_in=False):
+    state = d * d * 4 * units
+    if kernel == "kda_chunk_simt_kernel":
+        return token_heads * (3 * 2 * d + 4 * d + 4 + 2 * d) + state * (2 if with_state_in else 1)
+    if kernel == "kda_tc_chunk_local_kernel":
+        return token_heads * (3 * 2 * d + 4 * d + 4 + TC_IMAGE_BYTES_PER_TOKEN_HEAD)
+    if kernel == "kda_tc_state_pass_kernel":
+        return token_heads * (TC_IMAGE_BYTES_PER_TOKEN_HEAD + 2 * d) + state * (2 if with_state_in else 1)
+    raise KeyError(kernel)
+
+
+def version() -> int:
+    return int(load_library().kda_version())
+
+
+__all__ = ["chunk_fwd", "recurrent_step", "chunk_fwd_host", "HostPrefill", "workspace_size",
+           "launches_per_chunk_fwd", "kernel_names", "profile_chunk_fwd", "algorithmic_bytes_per_launch",
+           "last_error", "device_error", "version", "load_library", "lib_path", "KDAError", "EXPORTED"]

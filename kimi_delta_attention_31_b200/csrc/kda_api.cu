@@ -1,0 +1,200 @@
+// kda_api.cu -- the C ABI of libkda (declared in include/kda.h): argument
+// validation, workspace sizing, dispatch to the kernels, error reporting.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/kda.h"
+#include "kda_chunk_simt.cuh"
+#include "kda_chunk_tc.cuh"
+#include "kda_common.cuh"
+#include "kda_decode.cuh"
+
+namespace {
+
+thread_local char t_err[512] = "";
+thread_local cudaEvent_t* t_prof_events = nullptr;
+thread_local int t_prof_count = 0;
+
+kda_status_t fail(kda_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_err, sizeof(t_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+kda_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(KDA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_head(int dk, int dv) { return dk == dv && (dk == 32 || dk == 64 || dk == 128); }
+
+bool use_tensor_core_path(int dk, int dv, int chunk_size, kda_dtype_t dt) {
+  return kda::kTcPathBuilt && dt == KDA_BF16 && dk == 128 && dv == 128 && chunk_size == 64;
+}
+
+long long max_chunks(int B, int T, int num_seqs, int chunk_size) {
+  if (num_seqs > 0) return (long long)T / chunk_size + num_seqs;
+  return (long long)B * ((T + chunk_size - 1) / chunk_size);
+}
+
+template <typename TIn>
+cudaError_t dispatch_chunk_simt(int dk, int C, const void* q, const void* k, const void* v,
+                                const float* g, const float* beta, const float* S0, void* o,
+                                float* S_out, const int32_t* cu, int N, int T, int H, int dv,
+                                cudaStream_t st) {
+#define KDA_SIMT_CASE(D, CC)                                                                  \
+  if (dk == D && C == CC)                                                                     \
+    return kda::launch_chunk_simt<TIn, D, CC>(q, k, v, g, beta, S0, o, S_out, cu, N, T, H, dv, \
+                                               st);
+  KDA_SIMT_CASE(32, 16) KDA_SIMT_CASE(32, 32) KDA_SIMT_CASE(32, 64)
+  KDA_SIMT_CASE(64, 16) KDA_SIMT_CASE(64, 32) KDA_SIMT_CASE(64, 64)
+  KDA_SIMT_CASE(128, 16) KDA_SIMT_CASE(128, 32) KDA_SIMT_CASE(128, 64)
+#undef KDA_SIMT_CASE
+  return cudaErrorInvalidValue;
+}
+
+template <typename TIn>
+cudaError_t dispatch_decode(int dk, const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, float* S, void* o, int N, int H,
+                            cudaStream_t st) {
+  if (dk == 32) return kda::launch_decode_step<TIn, 32, 32>(q, k, v, g, beta, S, o, N, H, st);
+  if (dk == 64) return kda::launch_decode_step<TIn, 64, 64>(q, k, v, g, beta, S, o, N, H, st);
+  if (dk == 128) return kda::launch_decode_step<TIn, 128, 128>(q, k, v, g, beta, S, o, N, H, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_last_error(void) { return t_err; }
+
+int kda_version(void) { return 100; }
+
+int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype) {
+  return use_tensor_core_path(dk, dv, chunk_size, dtype) ? kda::kTcLaunches : 1;
+}
+
+kda_status_t kda_profile_events(cudaEvent_t* events, int count) {
+  t_err[0] = 0;
+  if (events && count <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_profile_events: count=%d", count);
+  t_prof_events = events;
+  t_prof_count = events ? count : 0;
+  return KDA_OK;
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                    int chunk_size, kda_dtype_t dtype) {
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || chunk_size <= 0) return 0;
+  if (!use_tensor_core_path(dk, dv, chunk_size, dtype)) return 0;
+  const int N = num_seqs > 0 ? num_seqs : B;
+  return kda::tc_workspace_bytes(max_chunks(B, T, num_seqs, chunk_size), H, N);
+}
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* S0, void* o, float* S_out,
+                           const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
+                           int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  t_err[0] = 0;
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0)
+    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: bad sizes B=%d T=%d H=%d num_seqs=%d", B,
+                T, H, num_seqs);
+  if (dtype != KDA_BF16 && dtype != KDA_F32)
+    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd: unknown dtype %d", (int)dtype);
+  if (!supported_head(dk, dv))
+    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd: dk=%d dv=%d (need dk == dv in {32,64,128})",
+                dk, dv);
+  if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64)
+    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd: chunk_size=%d (need 16, 32 or 64)",
+                chunk_size);
+  if (cu_seqlens) {
+    if (B != 1) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: packed inputs need B == 1");
+    if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: cu_seqlens needs num_seqs >= 1");
+  } else if (num_seqs != 0) {
+    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: num_seqs=%d without cu_seqlens", num_seqs);
+  }
+  const int N = cu_seqlens ? num_seqs : B;
+  const long long tokens = (long long)B * T;
+  if (N == 0) return KDA_OK;
+  if (tokens > 0 && (!q || !k || !v || !g || !beta || !o))
+    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: null input/output pointer");
+  const void* ptrs[] = {q, k, v, g, beta, S0, o, S_out, cu_seqlens, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(KDA_ERR_ALIGNMENT, "kda_chunk_fwd: pointer %p is not 16-byte aligned", p);
+  if (S_out && o && (const void*)S_out == (const void*)o)
+    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: o aliases S_out");
+
+  const int launches = kda_chunk_fwd_launches(dk, dv, chunk_size, dtype);
+  cudaEvent_t* ev = t_prof_events;
+  if (ev && t_prof_count < launches + 1)
+    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: %d profiling events, need %d", t_prof_count,
+                launches + 1);
+  cudaError_t e;
+  if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return cuda_fail(e, "event record");
+  if (use_tensor_core_path(dk, dv, chunk_size, dtype)) {
+    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
+    if (need && (!workspace || workspace_bytes < need))
+      return fail(KDA_ERR_WORKSPACE, "kda_chunk_fwd: workspace %zu bytes, need %zu", workspace_bytes,
+                  need);
+    e = kda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
+                             static_cast<const __nv_bfloat16*>(k),
+                             static_cast<const __nv_bfloat16*>(v), g, beta, S0,
+                             static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H,
+                             max_chunks(B, T, num_seqs, chunk_size), workspace, ev, stream);
+  } else if (dtype == KDA_F32) {
+    e = dispatch_chunk_simt<float>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, T,
+                                   H, dv, stream);
+  } else {
+    e = dispatch_chunk_simt<__nv_bfloat16>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out,
+                                           cu_seqlens, N, T, H, dv, stream);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd launch");
+  if (ev && launches == 1 && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess)
+    return cuda_fail(e, "event record");
+  return KDA_OK;
+}
+
+kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, float* S, void* o, int N, int H, int dk,
+                                int dv, kda_dtype_t dtype, cudaStream_t stream) {
+  t_err[0] = 0;
+  if (N < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_step: bad sizes N=%d H=%d", N, H);
+  if (dtype != KDA_BF16 && dtype != KDA_F32)
+    return fail(KDA_ERR_UNSUPPORTED, "kda_recurrent_step: unknown dtype %d", (int)dtype);
+  if (!supported_head(dk, dv))
+    return fail(KDA_ERR_UNSUPPORTED,
+                "kda_recurrent_step: dk=%d dv=%d (need dk == dv in {32,64,128})", dk, dv);
+  if (N == 0) return KDA_OK;
+  if (!q || !k || !v || !g || !beta || !S || !o)
+    return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_step: null pointer");
+  const void* ptrs[] = {q, k, v, g, beta, S, o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(KDA_ERR_ALIGNMENT, "kda_recurrent_step: pointer %p is not 16-byte aligned", p);
+  cudaError_t e = dtype == KDA_F32
+                      ? dispatch_decode<float>(dk, q, k, v, g, beta, S, o, N, H, stream)
+                      : dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, N, H, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_step launch");
+  return KDA_OK;
+}
+
+kda_status_t kda_device_error(int* code, cudaStream_t stream) {
+  t_err[0] = 0;
+  if (!code) return fail(KDA_ERR_INVALID_ARG, "kda_device_error: null code");
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_device_error: synchronize");
+  int h = 0;
+  e = cudaMemcpyFromSymbol(&h, kda::g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "kda_device_error: read");
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(kda::g_device_error, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "kda_device_error: clear");
+  *code = h;
+  return KDA_OK;
+}
+
+}  // extern "C"

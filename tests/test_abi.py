@@ -1,0 +1,96 @@
+"""CPU-side checks of the C ABI: libkda.so loads, exports every function that
+include/kda.h declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kimi_delta_attention_31_b200 as kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_header_symbols():
+    lib = kda.load_library()
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    assert set(names) == set(kda.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert kda.version() == 100
+
+
+def _null():
+    return ctypes.c_void_p(0)
+
+
+def _fake(addr=0x1000):
+    return ctypes.c_void_p(addr)
+
+
+def test_recurrent_step_rejects_bad_arguments():
+    lib = kda.load_library()
+    f = _fake()
+    # unsupported head size
+    st = lib.kda_recurrent_step(f, f, f, f, f, f, f, 4, 2, 96, 96, kda.KDA_BF16, None)
+    assert st == 2 and "dk=96" in kda.last_error()
+    # dk != dv
+    st = lib.kda_recurrent_step(f, f, f, f, f, f, f, 4, 2, 128, 64, kda.KDA_BF16, None)
+    assert st == 2
+    # null pointer
+    st = lib.kda_recurrent_step(f, f, _null(), f, f, f, f, 4, 2, 128, 128, kda.KDA_BF16, None)
+    assert st == 1
+    # misaligned pointer
+    st = lib.kda_recurrent_step(f, f, _fake(0x1004), f, f, f, f, 4, 2, 64, 64, kda.KDA_F32, None)
+    assert st == 3
+    # bad dtype, bad sizes
+    assert lib.kda_recurrent_step(f, f, f, f, f, f, f, 4, 2, 64, 64, 7, None) == 2
+    assert lib.kda_recurrent_step(f, f, f, f, f, f, f, -1, 2, 64, 64, 0, None) == 1
+    # nothing to do: N == 0 succeeds without launching
+    assert lib.kda_recurrent_step(f, f, f, f, f, f, f, 0, 2, 64, 64, 0, None) == 0
+
+
+def test_chunk_fwd_rejects_bad_arguments():
+    lib = kda.load_library()
+    f = _fake()
+    args = lambda **kw: dict(dict(num_seqs=0, B=1, T=64, H=2, dk=128, dv=128, C=64, dt=0, cu=None,
+                                  o=f, ws=None, wsb=0), **kw)
+
+    def call(a):
+        return lib.kda_chunk_fwd(f, f, f, f, f, None, a["o"], f, a["cu"], a["num_seqs"], a["B"], a["T"],
+                                 a["H"], a["dk"], a["dv"], a["C"], a["dt"], a["ws"], a["wsb"], None)
+
+    assert call(args(C=48)) == 2
+    assert call(args(dk=80, dv=80)) == 2
+    assert call(args(num_seqs=3)) == 1              # num_seqs without cu_seqlens
+    assert call(args(cu=f, num_seqs=2, B=2)) == 1   # packed needs B == 1
+    assert call(args(cu=f, num_seqs=0)) == 1
+    assert call(args(o=_null())) == 1
+    assert call(args(o=_fake(0x1008))) == 3
+    assert call(args(H=0)) == 1
+    assert call(args(dt=5)) == 2
+    assert call(args(B=0)) == 0  # no sequences: nothing to do
+
+
+def test_workspace_size_is_consistent():
+    lib = kda.load_library()
+    # fp32 arithmetic path needs no workspace
+    assert lib.kda_chunk_fwd_workspace_size(1, 256, 2, 32, 32, 0, 16, kda.KDA_F32) == 0
+    a = lib.kda_chunk_fwd_workspace_size(8, 8192, 32, 128, 128, 0, 64, kda.KDA_BF16)
+    b = lib.kda_chunk_fwd_workspace_size(8, 8193, 32, 128, 128, 0, 64, kda.KDA_BF16)
+    assert b >= a
+    assert lib.kda_chunk_fwd_workspace_size(-1, 8, 2, 128, 128, 0, 64, kda.KDA_BF16) == 0
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 32)
+    with pytest.raises(ValueError):
+        kda.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
