@@ -141,11 +141,11 @@ def oracle_baseline(w, target_s=15.0):
     ``target_s`` seconds of work on this host's cores."""
     import oracle
     cores = oracle.max_threads()
-    cal = W.make_prefill(1, 512, 2, w.dk, w.dv, w.dtype, w.g_mu, w.g_sigma, 0.0, seed=w.seed + 1)
+    cal = W.make_prefill(1, 512, cores, w.dk, w.dv, w.dtype, w.g_mu, w.g_sigma, 0.0, seed=w.seed + 1)
     t0 = time.perf_counter()
     oracle.recurrent(cal["q"], cal["k"], cal["v"], cal["g"], cal["beta"], num_threads=cores)
-    rate = 1024 / max(time.perf_counter() - t0, 1e-6)  # token-heads/s (rough)
-    units = max(cores, int(target_s * rate / w.T))
+    rate = 512 * cores / max(time.perf_counter() - t0, 1e-6)  # token-heads/s on all cores
+    units = max(cores, int(target_s * rate / w.T) // cores * cores)
     units = min(units, w.B * w.H)
     # the sample: `units` heads of the first sequence(s), full length, same recipe
     sample = W.make_prefill(1, w.T, units, w.dk, w.dv, w.dtype, w.g_mu, w.g_sigma, w.s0_std,

@@ -20,8 +20,10 @@
  *   L2-normalised q, k or a 1/sqrt(dk) scale applies it beforehand).
  *
  * Conventions shared by every entry point:
- *   - All tensor pointers are DEVICE pointers, row-major, densely packed, with
- *     16-byte aligned bases.  The caller owns every buffer and the stream; the
+ *   - All tensor pointers are DEVICE pointers, row-major, densely packed.
+ *     Alignment: kda_chunk_fwd needs 16-byte aligned q, k, v, g, o, S0, S_out
+ *     and workspace and 4-byte aligned beta and cu_seqlens; kda_recurrent_step
+ *     needs a 16-byte aligned S and element-aligned q, k, v, o, g, beta.  The caller owns every buffer and the stream; the
  *     library never allocates, frees or synchronises (except
  *     kda_device_error, which synchronises the given stream by design).
  *   - Calls are asynchronous on `stream`.  The return value reports argument

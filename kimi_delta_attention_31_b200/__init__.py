@@ -246,6 +246,8 @@ def profile_chunk_fwd(call, stream, repeats=3, dk=128, dv=128, chunk_size=64, dt
     names = kernel_names(dk, dv, chunk_size, dtype)
     n = len(names)
     events = [torch.cuda.Event(enable_timing=True) for _ in range((n + 1) * repeats)]
+    for e in events:  # torch creates the underlying event lazily, at its first record
+        e.record(stream)
     totals = [0.0] * n
     for r in range(repeats):
         evs = events[r * (n + 1):(r + 1) * (n + 1)]

@@ -29,6 +29,7 @@ kda_status_t cuda_fail(cudaError_t e, const char* where) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1u)) == 0; }
 
 bool supported_head(int dk, int dv) { return dk == dv && (dk == 32 || dk == 64 || dk == 128); }
 
@@ -123,9 +124,11 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
   if (N == 0) return KDA_OK;
   if (tokens > 0 && (!q || !k || !v || !g || !beta || !o))
     return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: null input/output pointer");
-  const void* ptrs[] = {q, k, v, g, beta, S0, o, S_out, cu_seqlens, workspace};
+  const void* ptrs[] = {q, k, v, g, S0, o, S_out, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(KDA_ERR_ALIGNMENT, "kda_chunk_fwd: pointer %p is not 16-byte aligned", p);
+  if ((beta && !aligned_to(beta, 4)) || (cu_seqlens && !aligned_to(cu_seqlens, 4)))
+    return fail(KDA_ERR_ALIGNMENT, "kda_chunk_fwd: beta / cu_seqlens not 4-byte aligned");
   if (S_out && o && (const void*)S_out == (const void*)o)
     return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: o aliases S_out");
 
@@ -172,9 +175,13 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, con
   if (N == 0) return KDA_OK;
   if (!q || !k || !v || !g || !beta || !S || !o)
     return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_step: null pointer");
-  const void* ptrs[] = {q, k, v, g, beta, S, o};
-  for (const void* p : ptrs)
-    if (!aligned16(p)) return fail(KDA_ERR_ALIGNMENT, "kda_recurrent_step: pointer %p is not 16-byte aligned", p);
+  const unsigned esz = dtype == KDA_F32 ? 4u : 2u;
+  if (!aligned16(S)) return fail(KDA_ERR_ALIGNMENT, "kda_recurrent_step: S %p is not 16-byte aligned", (const void*)S);
+  const void* elem[] = {q, k, v, o};
+  for (const void* p : elem)
+    if (!aligned_to(p, esz)) return fail(KDA_ERR_ALIGNMENT, "kda_recurrent_step: pointer %p is misaligned", p);
+  if (!aligned_to(g, 4) || !aligned_to(beta, 4))
+    return fail(KDA_ERR_ALIGNMENT, "kda_recurrent_step: g / beta not 4-byte aligned");
   cudaError_t e = dtype == KDA_F32
                       ? dispatch_decode<float>(dk, q, k, v, g, beta, S, o, N, H, stream)
                       : dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, N, H, stream);

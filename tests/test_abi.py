@@ -47,8 +47,10 @@ def test_recurrent_step_rejects_bad_arguments():
     # null pointer
     st = lib.kda_recurrent_step(f, f, _null(), f, f, f, f, 4, 2, 128, 128, kda.KDA_BF16, None)
     assert st == 1
-    # misaligned pointer
-    st = lib.kda_recurrent_step(f, f, _fake(0x1004), f, f, f, f, 4, 2, 64, 64, kda.KDA_F32, None)
+    # misaligned pointers: the state must be 16-byte aligned, fp32 inputs 4-byte
+    st = lib.kda_recurrent_step(f, f, f, f, f, _fake(0x1004), f, 4, 2, 64, 64, kda.KDA_F32, None)
+    assert st == 3
+    st = lib.kda_recurrent_step(f, f, _fake(0x1002), f, f, f, f, 4, 2, 64, 64, kda.KDA_F32, None)
     assert st == 3
     # bad dtype, bad sizes
     assert lib.kda_recurrent_step(f, f, f, f, f, f, f, 4, 2, 64, 64, 7, None) == 2
