@@ -62,7 +62,7 @@ constexpr uint32_t IMG_BYTES = 74240;
 // chunk-local kernel shared memory (dynamic, 1024-aligned base)
 constexpr uint32_t KA_L3 = 0;       // [K a; Q a]  K-major [128][128] (2 K-panels)  32768
 constexpr uint32_t KA_RB = 32768;   // right operands K-major [160][128]          40960
-constexpr uint32_t KA_AS = 0;       // after the first MMA: A fp32 [64][65]       16640
+constexpr uint32_t KA_AS = 0;       // after the first MMA: A fp32 [64][68]       17408
 constexpr uint32_t KA_PT = 17408;   //                      P bf16 K-major          8192
 constexpr uint32_t KA_TT = 25600;   //                      T bf16 K-major          8192
 constexpr uint32_t KA_WT = 0;       // after the solve:     W^T bf16 K-major       16384
@@ -79,9 +79,12 @@ constexpr uint32_t KB_E = KB_SB + 32768;    // E bf16 MN-major 2 panels [64][64]
 constexpr uint32_t KB_BYTES = KB_E + 16384;
 constexpr uint32_t KB_DYN = KB_BYTES + 1024;
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~(uintptr_t)1023);
-}
+// 1024-byte aligned start inside the dynamic shared buffer.  Offsetting the
+// array (not casting through an integer) keeps the pointer in the shared
+// address space, so the compiler emits st.shared/ld.shared and can reorder
+// global loads around them.
+#define KDA_ALIGNED_DSMEM(name, raw) \
+  uint8_t* name = (raw) + ((1024u - (ptx::smem_u32(raw) & 1023u)) & 1023u)
 __device__ __forceinline__ void st_bf16(uint8_t* p, float x) {
   *reinterpret_cast<bf16*>(p) = __float2bfloat16_rn(x);
 }
@@ -151,23 +154,36 @@ __device__ __forceinline__ float sel4(int i, float a0, float a1, float a2, float
 
 // ---------------------------------------------------------------------------
 // Kernel 1: chunk-local work, one CTA (256 threads) per (chunk, head).
-// Thread t handles key channel c = t mod 128 for the rows of its half
-// (rows 32 * (t / 128) ... + 31) during the gate preparation.
+// Operand building: thread t owns channels 8 (t mod 16) .. + 7 of rows
+// 4 (t / 16) .. + 3, so every global load and shared store moves 16 bytes.
 // ---------------------------------------------------------------------------
+constexpr uint32_t KA_TS = 33792;  // after the first MMA: T fp32 [64][68]          17408
+constexpr uint32_t KA_MT = 51200;  //                      block products [3][16][16] 3072
+constexpr int AS_LD = 68;          // row stride (floats) of A and T in fp32
+
+__device__ __forceinline__ void unpack8(uint4 w, float* x) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(p[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+
 __global__ void __launch_bounds__(256, 2)
     kda_tc_chunk_local_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                               const bf16* __restrict__ v, const float* __restrict__ g,
                               const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                               int num_seqs, int T, int H, uint8_t* __restrict__ ws) {
   __shared__ float s_beta[C];
-  __shared__ float s_Ge[4][D];
-  __shared__ float s_tot[D];
+  __shared__ __align__(16) float s_Ge[4][D];  // G at the end of each 16-token block
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ uint32_t s_tmem;
   __shared__ long long s_loc_s;
   __shared__ int s_loc_n;
-  extern __shared__ uint8_t dsm_raw[];
-  uint8_t* sm = align1024(dsm_raw);
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
+  KDA_ALIGNED_DSMEM(sm, dsm_raw);
   const uint32_t sb = ptx::smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -198,8 +214,7 @@ __global__ void __launch_bounds__(256, 2)
   if (Cn <= 0) return;  // uniform across the CTA
 
   uint8_t* img = ws + ((size_t)ci * H + h) * IMG_BYTES;
-  const int c = tid & 127, half = tid >> 7, r0 = half * 32;
-  const uint32_t kp = c >> 6, ce = c & 63;
+  const size_t rs = (size_t)H * D;  // elements between consecutive tokens
 
   if (warp == 0) {
     ptx::tmem_alloc(&s_tmem, 256);
@@ -211,76 +226,122 @@ __global__ void __launch_bounds__(256, 2)
   }
   if (tid < C) s_beta[tid] = tid < Cn ? beta[(size_t)(s0 + tid) * H + h] : 0.f;
 
-  // ---- 1. cumulative log-decay (fp32), rows >= Cn contribute g = 0
-  const size_t rs = (size_t)H * D;
-  const size_t base = ((size_t)s0 * H + h) * D + c;
-  float G[32];
-  {
-    float acc = 0.f;
+  // ---- 1. cumulative log-decay G (fp32); rows >= Cn contribute g = 0
+  const int co = tid & 15, rg = tid >> 4, J = rg >> 2;  // channel octet, row group, 16-token block
+  const int c0 = 8 * co;
+  const uint32_t kp = co >> 3, ck = co & 7;  // K-panel and 16-byte chunk of the channels
+  const size_t base8 = ((size_t)s0 * H + h) * D + c0;
+  float G[4][8];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float x = (r0 + i) < Cn ? g[base + (size_t)(r0 + i) * rs] : 0.f;
-      acc += x;
-      G[i] = acc;
+  for (int u = 0; u < 4; ++u) {
+    const int r = 4 * rg + u;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (r < Cn) {
+      const float4* gp = reinterpret_cast<const float4*>(g + base8 + (size_t)r * rs);
+      a = gp[0];
+      b = gp[1];
     }
-    if (half == 0) s_tot[c] = acc;
+    const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) G[u][e] = (u ? G[u - 1][e] : 0.f) + x[e];
   }
+  float* s_tot = reinterpret_cast<float*>(sm + KA_XK);  // [16][128] row-group totals (XK is built later)
+  reinterpret_cast<float4*>(s_tot + rg * D + c0)[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+  reinterpret_cast<float4*>(s_tot + rg * D + c0)[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = s_tmem;
-  if (half == 1) {
-    const float b0 = s_tot[c];
+  {
+    float off[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < 32; ++i) G[i] += b0;
-  }
-  s_Ge[2 * half][c] = G[15];
-  s_Ge[2 * half + 1][c] = G[31];
-  __syncthreads();
-  const float Ge0 = s_Ge[0][c], Ge1 = s_Ge[1][c], Ge2 = s_Ge[2][c], Ge3 = s_Ge[3][c];
-
-  // ---- 2. decay-scaled bf16 operands
-#pragma unroll
-  for (int bi = 0; bi < 2; ++bi) {
-    const int J = 2 * half + bi;
-    const float Gb = J == 0 ? 0.f : sel4(J - 1, Ge0, Ge1, Ge2, Ge3);
-    const float GeJ = sel4(J, Ge0, Ge1, Ge2, Ge3);
-    const float eGb = expf(Gb);           // e^{G} at the block start
-    const float invD = expf(Gb - GeJ);    // 1 / (block decay), >= 1
-    const float lam = expf(Ge3 - GeJ);    // decay from block end to chunk end
-    // right-operand scale for row block I = J + 1 + t: e^{G_end(I-1) - G_end(J)}
-    const float sig1 = J <= 1 ? expf(sel4(J + 1, Ge0, Ge1, Ge2, Ge3) - GeJ) : 0.f;
-    const float sig2 = J == 0 ? expf(Ge2 - GeJ) : 0.f;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int i = 16 * bi + e;
-      const int r = r0 + i;  // == 16 J + e
-      float kv = 0.f, qv = 0.f, vv = 0.f;
-      if (r < Cn) {
-        const size_t off = base + (size_t)r * rs;
-        kv = __bfloat162float(k[off]);
-        qv = __bfloat162float(q[off]);
-        vv = __bfloat162float(v[off]);
+    for (int q2 = 0; q2 < 15; ++q2) {
+      if (q2 < rg) {
+        const float4 t0 = reinterpret_cast<const float4*>(s_tot + q2 * D + c0)[0];
+        const float4 t1 = reinterpret_cast<const float4*>(s_tot + q2 * D + c0)[1];
+        off[0] += t0.x; off[1] += t0.y; off[2] += t0.z; off[3] += t0.w;
+        off[4] += t1.x; off[5] += t1.y; off[6] += t1.z; off[7] += t1.w;
       }
-      const float a = __expf(G[i] - Gb);
-      const float b = __expf(GeJ - G[i]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) G[u][e] += off[e];
+  }
+  if ((rg & 3) == 3) {
+    reinterpret_cast<float4*>(&s_Ge[J][c0])[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+    reinterpret_cast<float4*>(&s_Ge[J][c0])[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
+  }
+  __syncthreads();
+
+  // ---- 2. decay-scaled bf16 operands, 16-byte stores
+  {
+    float Gb[8], GeJ[8], eGb[8], invD[8], lam[8], sig1[8], sig2[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = c0 + e;
+      GeJ[e] = s_Ge[J][c];
+      Gb[e] = J ? s_Ge[J - 1][c] : 0.f;
+      eGb[e] = __expf(Gb[e]);                        // e^{G} at the block start
+      invD[e] = __expf(Gb[e] - GeJ[e]);              // 1 / (block decay), >= 1
+      lam[e] = __expf(s_Ge[3][c] - GeJ[e]);          // block end -> chunk end
+      sig1[e] = J <= 1 ? __expf(s_Ge[J + 1][c] - GeJ[e]) : 0.f;  // for row block J + 2
+      sig2[e] = J == 0 ? __expf(s_Ge[2][c] - GeJ[e]) : 0.f;      // for row block 3
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = 4 * rg + u, e16 = r & 15;
+      uint4 kw = make_uint4(0, 0, 0, 0), qw = kw, vw = kw;
+      if (r < Cn) {
+        const size_t off = base8 + (size_t)r * rs;
+        kw = *reinterpret_cast<const uint4*>(k + off);
+        qw = *reinterpret_cast<const uint4*>(q + off);
+        vw = *reinterpret_cast<const uint4*>(v + off);
+      }
+      float kv[8], qv[8], vv[8];
+      unpack8(kw, kv);
+      unpack8(qw, qv);
+      unpack8(vw, vv);
       const float br = s_beta[r];
-      const float ka = kv * a, kb = kv * b;
-      st_bf16(sm + KA_L3 + kp * 16384 + ptx::sw128(r, ce), ka);
-      st_bf16(sm + KA_L3 + kp * 16384 + ptx::sw128(64 + r, ce), qv * a);
-      // right operands: rows 16 * (I (I - 1) / 2 + J) + e for I = J+1..3, diag at 96 + r
-      if (J <= 2) st_bf16(sm + KA_RB + kp * 20480 + ptx::sw128(16 * ((J + 1) * J / 2 + J) + e, ce), kb);
-      if (J <= 1) st_bf16(sm + KA_RB + kp * 20480 + ptx::sw128(16 * ((J + 2) * (J + 1) / 2 + J) + e, ce), kb * sig1);
-      if (J == 0) st_bf16(sm + KA_RB + kp * 20480 + ptx::sw128(16 * 3 + e, ce), kb * sig2);
-      st_bf16(sm + KA_RB + kp * 20480 + ptx::sw128(96 + r, ce), kb * invD);
-      // Kbar = K o e^{G_last - G}  (image, MN-major, panel = c / 64, row = token)
-      st_bf16(img + IMG_KB + kp * 8192 + ptx::sw128(r, ce), kb * lam);
-      // beta K o e^{G} and beta V (MN-major A operands of the WY products)
-      st_bf16(sm + KA_XK + kp * 8192 + ptx::sw128(r, ce), br * ka * eGb);
-      st_bf16(sm + KA_BV + kp * 8192 + ptx::sw128(r, ce), br * vv);
+      float o_lk[8], o_lq[8], o_r0[8], o_r1[8], o_r2[8], o_rd[8], o_kb[8], o_xk[8], o_bv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float a = __expf(G[u][e] - Gb[e]);   // (0, 1]
+        const float b = __expf(GeJ[e] - G[u][e]);  // (0, 1]
+        const float ka = kv[e] * a, kb = kv[e] * b;
+        o_lk[e] = ka;
+        o_lq[e] = qv[e] * a;
+        o_r0[e] = kb;
+        o_r1[e] = kb * sig1[e];
+        o_r2[e] = kb * sig2[e];
+        o_rd[e] = kb * invD[e];
+        o_kb[e] = kb * lam[e];
+        o_xk[e] = br * ka * eGb[e];
+        o_bv[e] = br * vv[e];
+      }
+      uint8_t* l3 = sm + KA_L3 + kp * 16384;
+      uint8_t* rb = sm + KA_RB + kp * 20480;
+      *reinterpret_cast<uint4*>(l3 + ptx::sw128_chunk(r, ck)) = pack8(o_lk);
+      *reinterpret_cast<uint4*>(l3 + ptx::sw128_chunk(64 + r, ck)) = pack8(o_lq);
+      // right operands: rows 16 (I (I - 1) / 2 + J) + e16 for row block I = J+1..3; diagonal at 96 + r
+      if (J <= 2) *reinterpret_cast<uint4*>(rb + ptx::sw128_chunk(16 * ((J + 1) * J / 2 + J) + e16, ck)) = pack8(o_r0);
+      if (J <= 1) *reinterpret_cast<uint4*>(rb + ptx::sw128_chunk(16 * ((J + 2) * (J + 1) / 2 + J) + e16, ck)) = pack8(o_r1);
+      if (J == 0) *reinterpret_cast<uint4*>(rb + ptx::sw128_chunk(48 + e16, ck)) = pack8(o_r2);
+      *reinterpret_cast<uint4*>(rb + ptx::sw128_chunk(96 + r, ck)) = pack8(o_rd);
+      // Kbar = K o e^{G_last - G} (image, MN-major panel = channel / 64, row = token)
+      *reinterpret_cast<uint4*>(img + IMG_KB + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_kb);
+      // beta K o e^G and beta V: MN-major A operands of the WY products
+      *reinterpret_cast<uint4*>(sm + KA_XK + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_xk);
+      *reinterpret_cast<uint4*>(sm + KA_BV + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_bv);
     }
   }
-  if (half == 0) reinterpret_cast<float*>(img + IMG_G)[c] = expf(Ge3);
+  if (rg == 0) {
+    float gm[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) gm[e] = expf(s_Ge[3][c0 + e]);
+    reinterpret_cast<float4*>(img + IMG_G)[2 * co] = make_float4(gm[0], gm[1], gm[2], gm[3]);
+    reinterpret_cast<float4*>(img + IMG_G)[2 * co + 1] = make_float4(gm[4], gm[5], gm[6], gm[7]);
+  }
 
   // ---- 3. [A'; P'] = [K a; Q a] (right operands)^T : M=128, N=160, K=128
   ptx::fence_proxy_async_smem();
@@ -300,13 +361,7 @@ __global__ void __launch_bounds__(256, 2)
   ptx::mbar_wait_bounded(&s_bar, 0);
   ptx::tc_fence_after();
 
-  // ---- 4. gather A (fp32, beta-scaled, strictly lower) and P (bf16, lower)
-  {
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int i = tid; i < 1040; i += 256) reinterpret_cast<uint4*>(sm + KA_AS)[i] = z;
-    for (int i = tid; i < 512; i += 256) reinterpret_cast<uint4*>(sm + KA_PT)[i] = z;
-  }
-  __syncthreads();
+  // ---- 4. scatter A (fp32, beta-scaled) and P (bf16, lower incl. diagonal, zero above)
   {
     const int qd = warp & 3, ch = warp >> 2;
     const int rho = 32 * qd + lane;
@@ -320,9 +375,9 @@ __global__ void __launch_bounds__(256, 2)
       float x[16];
       ptx::tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + col0, x);
       ptx::tmem_wait_ld();
+      const bool diag = col0 >= 96;
       int Jb;
       bool use;
-      const bool diag = col0 >= 96;
       if (!diag) {
         const int seg = col0 >> 4;
         const int Is = seg == 0 ? 1 : (seg < 3 ? 2 : 3);
@@ -332,42 +387,100 @@ __global__ void __launch_bounds__(256, 2)
         Jb = (col0 - 96) >> 4;
         use = Jb == I;
       }
-      if (use) {
+      if (isK) {
+        if (use) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int j = 16 * Jb + e;
-          if (isK) {
-            if (!diag || j < r) As[r * 65 + j] = br * x[e];
-          } else {
-            if (!diag || j <= r) st_bf16(sm + KA_PT + ptx::sw128(r, j), x[e]);
-          }
+          for (int e = 0; e < 16; ++e) x[e] = (!diag || 16 * Jb + e < r) ? br * x[e] : 0.f;
+          float4* dst = reinterpret_cast<float4*>(As + r * AS_LD + 16 * Jb);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_float4(x[4 * v4], x[4 * v4 + 1], x[4 * v4 + 2], x[4 * v4 + 3]);
         }
+      } else if (use || (diag && Jb > I)) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = (!diag || (Jb == I && 16 * Jb + e <= r)) ? x[e] : 0.f;
+        *reinterpret_cast<uint4*>(sm + KA_PT + ptx::sw128_chunk(r, 2 * Jb)) = pack8(x);
+        *reinterpret_cast<uint4*>(sm + KA_PT + ptx::sw128_chunk(r, 2 * Jb + 1)) = pack8(x + 8);
       }
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
 
-  // ---- 5. T = (I + A)^{-1} by forward substitution in fp32.
-  // Column j of T is owned by 4 lanes; lane `part` keeps rows i = 4 m + part.
+  // ---- 5. T = (I + A)^{-1} in fp32, blocked by 16: invert the diagonal blocks,
+  //         then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ by distance below the diagonal.
   {
     const float* As = reinterpret_cast<const float*>(sm + KA_AS);
-    const int j = tid >> 2, part = tid & 3;
-    float x[16];
+    float* Ts = reinterpret_cast<float*>(sm + KA_TS);
+    float* Mt = reinterpret_cast<float*>(sm + KA_MT);
+    if (tid < 64) {  // column jj of diagonal block Ib, forward substitution
+      const int Ib = tid >> 4, jj = tid & 15, o = 16 * Ib;
+      float x[16];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) x[m] = (4 * m + part == j) ? 1.f : 0.f;
+      for (int i = 0; i < 16; ++i) x[i] = (i == jj) ? 1.f : 0.f;
 #pragma unroll
-    for (int i = 1; i < 64; ++i) {
-      float acc = 0.f;
+      for (int i = 1; i < 16; ++i) {
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int m = 0; m < 16; ++m)
-        if (4 * m < i) acc = fmaf(As[i * 65 + 4 * m + part], x[m], acc);  // A[i][>=i] == 0
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      if ((i & 3) == part) x[i >> 2] = (i == j ? 1.f : 0.f) - acc;
+        for (int m = 0; m < i; ++m) a4[m & 3] = fmaf(As[(o + i) * AS_LD + o + m], x[m], a4[m & 3]);
+        const float val = -((a4[0] + a4[1]) + (a4[2] + a4[3]));
+        if (i > jj) x[i] = val;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) Ts[(o + i) * AS_LD + o + jj] = x[i];
     }
+    __syncthreads();
+    const int blk = tid >> 6, tt = tid & 63, i = tt >> 2, j4 = tt & 3;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) st_bf16(sm + KA_TT + ptx::sw128(4 * m + part, j), x[m]);
+    for (int dist = 1; dist <= 3; ++dist) {
+      const bool act = blk < 4 - dist;
+      const int Jc = blk, Ir = blk + dist;
+      if (act) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int kk = 0; kk < dist; ++kk) {
+          const int K = Jc + kk;
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const float a = As[(16 * Ir + i) * AS_LD + 16 * K + m];
+            const float4 t = *reinterpret_cast<const float4*>(Ts + (16 * K + m) * AS_LD + 16 * Jc + 4 * j4);
+            acc.x = fmaf(a, t.x, acc.x);
+            acc.y = fmaf(a, t.y, acc.y);
+            acc.z = fmaf(a, t.z, acc.z);
+            acc.w = fmaf(a, t.w, acc.w);
+          }
+        }
+        *reinterpret_cast<float4*>(Mt + blk * 256 + i * 16 + 4 * j4) = acc;
+      }
+      __syncthreads();
+      if (act) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float a = Ts[(16 * Ir + i) * AS_LD + 16 * Ir + m];  // T_II, zero above its diagonal
+          const float4 t = *reinterpret_cast<const float4*>(Mt + blk * 256 + m * 16 + 4 * j4);
+          acc.x = fmaf(a, t.x, acc.x);
+          acc.y = fmaf(a, t.y, acc.y);
+          acc.z = fmaf(a, t.z, acc.z);
+          acc.w = fmaf(a, t.w, acc.w);
+        }
+        *reinterpret_cast<float4*>(Ts + (16 * Ir + i) * AS_LD + 16 * Jc + 4 * j4) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+      }
+      __syncthreads();
+    }
+    // bf16 T (K-major [64 r][64 j]); blocks above the diagonal are zero
+    for (int idx = tid; idx < 512; idx += 256) {
+      const int rr = idx >> 3, k8 = idx & 7;
+      float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if ((k8 >> 1) <= (rr >> 4)) {
+        const float4 t0 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8);
+        const float4 t1 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8 + 4);
+        y[0] = t0.x; y[1] = t0.y; y[2] = t0.z; y[3] = t0.w;
+        y[4] = t1.x; y[5] = t1.y; y[6] = t1.z; y[7] = t1.w;
+      }
+      *reinterpret_cast<uint4*>(sm + KA_TT + ptx::sw128_chunk(rr, k8)) = pack8(y);
+    }
   }
 
   // ---- 6. W^T = (beta K e^G)^T T^T, U^T = (beta V)^T T^T : M=128, N=64, K=64
@@ -385,8 +498,8 @@ __global__ void __launch_bounds__(256, 2)
     }
     ptx::mma_commit(&s_bar);
   }
-  for (int i = tid; i < 512; i += 256)
-    reinterpret_cast<uint4*>(img + IMG_P)[i] = reinterpret_cast<const uint4*>(sm + KA_PT)[i];
+  for (int i2 = tid; i2 < 512; i2 += 256)
+    reinterpret_cast<uint4*>(img + IMG_P)[i2] = reinterpret_cast<const uint4*>(sm + KA_PT)[i2];
   ptx::mbar_wait_bounded(&s_bar, 1);
   ptx::tc_fence_after();
   {
@@ -413,7 +526,7 @@ __global__ void __launch_bounds__(256, 2)
     }
   }
 
-  // ---- 7. (P W)^T = W^T P^T : M=128, N=64, K=64; then Q'^T = (Q e^G)^T - (P W)^T
+  // ---- 7. (P W)^T = W^T P^T : M=128, N=64, K=64; then Q'^T = (Q o e^G)^T - (P W)^T
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
@@ -426,10 +539,27 @@ __global__ void __launch_bounds__(256, 2)
                     ptx::sdesc_sw128(sb + KA_PT + kk * 32, 16, 1024), id, kk > 0);
     ptx::mma_commit(&s_bar);
   }
-  ptx::mbar_wait_bounded(&s_bar, 0);
-  ptx::tc_fence_after();
   {
-    const int qd = warp & 3;  // row c = 32 qd + lane == tid mod 128; tokens r0 .. r0 + 31
+    // thread = (channel c = tid mod 128, tokens 32 (tid / 128) + [0, 32)): re-read g and q
+    // (L2-resident) while the MMA runs; G restarts from the block-1 end for the upper half.
+    const int qd = warp & 3, half = warp >> 2;
+    const int c = 32 * qd + lane, r0 = 32 * half;
+    const size_t base1 = ((size_t)s0 * H + h) * D + c;
+    float gr[32], qr[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int r = r0 + i;
+      gr[i] = r < Cn ? g[base1 + (size_t)r * rs] : 0.f;
+      qr[i] = r < Cn ? __bfloat162float(q[base1 + (size_t)r * rs]) : 0.f;
+    }
+    float acc = half ? s_Ge[1][c] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      acc += gr[i];
+      qr[i] *= __expf(acc);
+    }
+    ptx::mbar_wait_bounded(&s_bar, 0);
+    ptx::tc_fence_after();
     float x[32];
     const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + r0;
     ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
@@ -439,11 +569,7 @@ __global__ void __launch_bounds__(256, 2)
     for (int k8 = 0; k8 < 4; ++k8) {
       float y[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int i = 8 * k8 + e, r = r0 + i;
-        const float qv = r < Cn ? __bfloat162float(q[base + (size_t)r * rs]) : 0.f;
-        y[e] = qv * __expf(G[i]) - x[i];
-      }
+      for (int e = 0; e < 8; ++e) y[e] = qr[8 * k8 + e] - x[8 * k8 + e];
       *reinterpret_cast<uint4*>(img + IMG_A1 + 16384 + ptx::sw128_chunk(c, 4 * half + k8)) = pack8(y);
     }
   }
@@ -473,8 +599,8 @@ __global__ void __launch_bounds__(256, 1)
   __shared__ long long s_u_first, s_u_start;
   __shared__ int s_u_len;
   __shared__ int s_abort;
-  extern __shared__ uint8_t dsm_raw[];
-  uint8_t* sm = align1024(dsm_raw);
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
+  KDA_ALIGNED_DSMEM(sm, dsm_raw);
   const uint32_t sb = ptx::smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
