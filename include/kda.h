@@ -115,6 +115,32 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, con
                                 const float* beta, float* S, void* o, int N, int H, int dk,
                                 int dv, kda_dtype_t dtype, cudaStream_t stream);
 
+/*
+ * kda_chunk_fwd for callers that cannot allocate device memory: the same
+ * prefill, same arguments minus the workspace.  (Library plumbing: the pages
+ * have no counterpart.)  Some callers get only input and output pointers
+ * from a host framework that owns the whole device memory pool, or must not
+ * call cudaMalloc because it synchronises the device; this entry point needs
+ * no allocation from them and makes none itself.
+ *
+ * Its scratch is a fixed array inside the library, KDA_NOALLOC_SCRATCH_BYTES
+ * bytes on every GPU that loads the library, held until process exit.  Sizes
+ * whose kda_chunk_fwd_workspace_size(...) exceeds it are rejected with
+ * KDA_ERR_WORKSPACE (64 MiB holds 903 (chunk, head) pairs of the tensor-core
+ * path, e.g. B=1, H=8, T=7168; the fp32-arithmetic path needs none).
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array: calls whose executions overlap on the GPU
+ * (other streams, other threads) race and corrupt each other's results.
+ * Nothing in it has to start at zero: each call writes every byte it reads.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* S0, void* o, float* S_out,
+                                   const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
+                                   int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                                   cudaStream_t stream);
+
 /* Message describing the calling thread's last failure ("" if none). */
 const char* kda_last_error(void);
 

@@ -36,7 +36,8 @@ KDA_BF16, KDA_F32 = 0, 1
 # Every symbol include/kda.h declares (checked by the CPU test-suite).
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_last_error", "kda_device_error", "kda_chunk_fwd_launches", "kda_profile_events",
-            "kda_version")
+            "kda_version", "kda_chunk_fwd_noalloc")
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
 KERNELS_SIMT = ("kda_chunk_simt_kernel",)
@@ -82,6 +83,8 @@ def load_library():
         lib.kda_chunk_fwd_launches.restype = i32
         lib.kda_profile_events.argtypes = [vp, i32]
         lib.kda_profile_events.restype = i32
+        lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 9 + [i32] * 7 + [i32, vp]
+        lib.kda_chunk_fwd_noalloc.restype = i32
         lib.kda_version.argtypes = []
         lib.kda_version.restype = i32
         _lib = lib
@@ -153,6 +156,27 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, output_
     st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
                            _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
                            _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(q.device))
+    _check(st)
+    return o, S_out
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, o=None, S_out=None):
+    """chunk_fwd through kda_chunk_fwd_noalloc: no workspace is passed or
+    allocated (the library's built-in scratch array is used; o and S_out are
+    allocated here only when not given).  Returns (o, S_out)."""
+    lib = load_library()
+    _need_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_out)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = num_seqs if cu_seqlens is not None else B
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_out is None:
+        S_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                   _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
+                                   _dtype_code(q), _stream_handle(q.device))
     _check(st)
     return o, S_out
 
@@ -286,6 +310,6 @@ def version() -> int:
     return int(load_library().kda_version())
 
 
-__all__ = ["chunk_fwd", "recurrent_step", "chunk_fwd_host", "HostPrefill", "workspace_size",
+__all__ = ["chunk_fwd", "chunk_fwd_noalloc", "recurrent_step", "chunk_fwd_host", "HostPrefill", "workspace_size",
            "launches_per_chunk_fwd", "kernel_names", "profile_chunk_fwd", "algorithmic_bytes_per_launch",
            "last_error", "device_error", "version", "load_library", "lib_path", "KDAError", "EXPORTED"]

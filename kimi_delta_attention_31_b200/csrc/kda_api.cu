@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/kda.h"
 #include "kda_chunk_simt.cuh"
@@ -187,6 +188,65 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, con
                       : dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, N, H, stream);
   if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_step launch");
   return KDA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Prefill without any caller-provided workspace.
+//
+// Some callers cannot allocate device memory: a plug-in that receives only
+// input and output pointers from a host framework that owns the whole device
+// memory pool, or code that must not call cudaMalloc because it implicitly
+// synchronises the device.  For them the scratch the tensor-core prefill
+// needs (its per-chunk operand images) lives in this file-scope device array
+// instead.  Every GPU that loads the library keeps it until process exit.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[256] = {};  // device address of g_noalloc_scratch, per device ordinal
+
+// Host code only ever sees a host-side stand-in for g_noalloc_scratch, so the
+// real device address is looked up once per device, with that device current.
+kda_status_t noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= 256) return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_noalloc: device %d", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetSymbolAddress");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return KDA_OK;
+}
+}  // namespace
+
+kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* S0, void* o, float* S_out,
+                                   const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
+                                   int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                                   cudaStream_t stream) {
+  t_err[0] = 0;
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || chunk_size <= 0)
+    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_noalloc: bad sizes B=%d T=%d H=%d num_seqs=%d", B, T,
+                H, num_seqs);
+  const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
+  if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES)
+    return fail(KDA_ERR_WORKSPACE,
+                "kda_chunk_fwd_noalloc: these sizes need %zu bytes of scratch, more than the built-in "
+                "%zu-byte array; use kda_chunk_fwd with a caller-provided workspace",
+                need, (size_t)KDA_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if (need > 0) {
+    const kda_status_t st = noalloc_scratch(&scratch);
+    if (st != KDA_OK) return st;
+  }
+  return kda_chunk_fwd(q, k, v, g, beta, S0, o, S_out, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                       chunk_size, dtype, scratch, need, stream);
 }
 
 kda_status_t kda_device_error(int* code, cudaStream_t stream) {
