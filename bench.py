@@ -46,6 +46,30 @@ STATE_BYTES = 128 * 128 * 4
 DECODE_BYTES_PER_HEAD_STEP = 2 * STATE_BYTES + 3 * 256 + 512 + 4 + 256
 
 
+def profiled_traffic(kernel, unit_key):
+    """DRAM bytes per unit (token-head or head-step) for `kernel` from its ncu
+    summary under profiles/, or None when there is none or when the kernel's
+    source file changed since the counters were taken (sha1 recorded there)."""
+    import glob
+    import hashlib
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*.md"))):
+        fields = {}
+        for line in open(path):
+            if ":" in line and not line.startswith(("|", " ", "#")):
+                key, _, val = line.partition(":")
+                fields[key.strip()] = val.strip()
+        src, sha, per = fields.get("source_file"), fields.get("source_sha1"), fields.get(unit_key)
+        if not (src and sha and per):
+            continue
+        try:
+            cur = hashlib.sha1(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+        except OSError:
+            continue
+        if cur == sha:
+            return float(per), os.path.basename(path)
+    return None, None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -247,9 +271,14 @@ def run_ours(args):
     dom_name, dom_ms = max(kernel_ms.items(), key=lambda kv: kv[1])
     dom_bytes = kda.algorithmic_bytes_per_launch(dom_name, token_heads, B * H, d=dk)
     achieved_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
+    per_unit, prof_file = profiled_traffic(dom_name, "traffic_bytes_per_token_head")
     roofline = {"bound": "hbm", "kernel": dom_name, "achieved": achieved_gbs,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
-                "traffic": None, "peak_source": f"{peak_src} HBM copy bandwidth",
+                "traffic": None if per_unit is None else per_unit * token_heads,
+                "traffic_source": None if per_unit is None else
+                f"profiles/{prof_file}: DRAM bytes per token-head of a smaller launch x {token_heads} token-heads",
+                "alg_bytes_per_launch": dom_bytes,
+                "peak_source": f"{peak_src} HBM copy bandwidth",
                 "kernel_ms": kernel_ms,
                 "whole_call": {"alg_bytes": alg_bytes, "achieved_gbs": alg_bytes / (ms * 1e-3) / 1e9,
                                "hbm_frac": alg_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -298,10 +327,15 @@ def run_ours(args):
     heads = N * Hd
     state_gbs = world * heads * 2 * STATE_BYTES / (dec_ms * 1e-3) / 1e9
     dec_alg_gbs = heads * DECODE_BYTES_PER_HEAD_STEP / (dec_ms * 1e-3) / 1e9
+    dec_unit, dec_prof = profiled_traffic("kda_decode_step_kernel", "traffic_bytes_per_head_step")
     decode = {"workload": dw.name, "value": state_gbs, "unit": "GB/s (state read+write)",
               "us_per_step": dec_ms * 1e3, "steps": nsteps,
               "roofline": {"bound": "hbm", "achieved": dec_alg_gbs, "peak": peaks["hbm_gbs"],
-                           "unit": "GB/s", "frac": dec_alg_gbs / peaks["hbm_gbs"], "traffic": None,
+                           "unit": "GB/s", "frac": dec_alg_gbs / peaks["hbm_gbs"],
+                           "traffic": None if dec_unit is None else dec_unit * heads,
+                           "traffic_source": None if dec_unit is None else
+                           f"profiles/{dec_prof}: DRAM bytes per head-step x {heads} head-steps",
+                           "alg_bytes_per_launch": heads * DECODE_BYTES_PER_HEAD_STEP,
                            "kernel": "kda_decode_step_kernel"}}
     del S, xs, od
     torch.cuda.empty_cache()
