@@ -8,7 +8,7 @@
 //   A_rj = beta_r sum_c k_rc k_jc e^{G_rc - G_jc}  (j < r),
 //   P_rj =        sum_c q_rc k_jc e^{G_rc - G_jc}  (j <= r),
 //   T = (I + A)^{-1},  W = T diag(beta) (K o e^G),  U = T diag(beta) V,
-//   E = U - W S,  O = (Q o e^G) S + P E = Q' S + P U  with Q' = Q o e^G - P W,
+//   E = U - W S,  O = (Q o e^G) S + P E,
 //   S <- Diag(e^{G_last}) S + (K o e^{G_last - G})^T E.
 // Everything left of "S" is chunk-local and parallel over chunks; only the
 // last three lines carry the state.  Two kernels:
@@ -16,15 +16,15 @@
 //  1. kda_tc_chunk_local_kernel -- one CTA per (chunk, head), all chunks in
 //     parallel.  Builds the decay-scaled bf16 operands in shared memory,
 //     computes [A; P] with one tcgen05 MMA (M=128, N=160, K=128) into TMEM,
-//     inverts I + A by fp32 forward substitution (warp shuffles), forms
-//     W^T, U^T (two MMAs) and (P W)^T (one MMA), and writes a 74,240-byte
-//     per-chunk image already laid out as the state pass's MMA operands.
+//     inverts I + A in fp32 (blocked by 16), forms W^T and U^T (two MMAs),
+//     and writes a 74,240-byte per-chunk image already laid out as the
+//     state pass's MMA operands.
 //  2. kda_tc_state_pass_kernel -- persistent, one CTA per SM, one (sequence,
 //     head) unit at a time, chunks in order.  The fp32 state lives in
 //     registers (thread = state row x 64 columns); per chunk one bulk copy
 //     brings the image in (double-buffered) and two MMA groups run:
-//       X = [-I; P] U + [W; Q'] S_bf16   -> rows 0..63 = -E, rows 64..127 = O
-//       Y = Kbar^T E                     -> S <- gamma o S + Y.
+//       X = [-I; 0] U + [W; Q e^G] S_bf16  -> rows 0..63 = -E, rows 64..127 = Q e^G S
+//       Y = Kbar^T E,  X += [*; P] E       -> S <- gamma o S + Y,  O = rows 64..127 of X.
 //
 // Overflow-free decay factors: A and P are never formed from e^{G} and
 // e^{-G} over the whole chunk.  The chunk is split into four 16-token blocks;
@@ -54,7 +54,7 @@ constexpr int D = 128;  // dk = dv
 // piece by the state pass.  Offsets in bytes; every piece 1024-aligned.
 constexpr uint32_t IMG_P = 0;       // P     K-major [64 r][64 j]                 8192
 constexpr uint32_t IMG_U = 8192;    // U^T   K-major [128 dv][64 j]               16384
-constexpr uint32_t IMG_A1 = 24576;  // [W;Q'] MN-major: 2 panels [128 dk][64 tok] 32768
+constexpr uint32_t IMG_A1 = 24576;  // [W;Q e^G] MN-major: 2 panels [128 dk][64 tok] 32768
 constexpr uint32_t IMG_KB = 57344;  // Kbar  MN-major: 2 panels [64 tok][64 dk]   16384
 constexpr uint32_t IMG_G = 73728;   // gamma = e^{G_last}, fp32 [128]             512
 constexpr uint32_t IMG_BYTES = 74240;
@@ -65,17 +65,20 @@ constexpr uint32_t KA_RB = 32768;   // right operands K-major [160][128]        
 constexpr uint32_t KA_AS = 0;       // after the first MMA: A fp32 [64][68]       17408
 constexpr uint32_t KA_PT = 17408;   //                      P bf16 K-major          8192
 constexpr uint32_t KA_TT = 25600;   //                      T bf16 K-major          8192
-constexpr uint32_t KA_WT = 0;       // after the solve:     W^T bf16 K-major       16384
 constexpr uint32_t KA_XK = 73728;   // beta K e^G  MN-major 2 panels [64][64]       16384
 constexpr uint32_t KA_BV = 90112;   // beta V      MN-major 2 panels [64][64]       16384
 constexpr uint32_t KA_BYTES = 106496;
 constexpr uint32_t KA_DYN = KA_BYTES + 1024;
 
-// state-pass kernel shared memory
-constexpr uint32_t KB_STAGE = 82944;        // -I (8192) + image (74240) + pad
-constexpr uint32_t KB_IMG = 8192;           // image offset inside a stage
-constexpr uint32_t KB_SB = 2 * KB_STAGE;    // S bf16 MN-major 2 panels [128][64]  32768
-constexpr uint32_t KB_E = KB_SB + 32768;    // E bf16 MN-major 2 panels [64][64]   16384
+// state-pass kernel shared memory.  [-I; 0] is a constant K-major [128][64]
+// operand; the two image stages follow it, so that the 8 KB in front of each
+// stage's P (the zero half, or the tail of stage 0) can serve as the unused
+// upper half of the [*; P] operand.
+constexpr uint32_t KB_NEGI = 0;             // [-I; 0] K-major [128 rows][64 K]        16384
+constexpr uint32_t KB_STAGE0 = 16384;       // image stages                     2 x 75776
+constexpr uint32_t KB_STAGE = 75776;
+constexpr uint32_t KB_SB = KB_STAGE0 + 2 * KB_STAGE;  // S bf16 MN-major 2 panels [128][64] 32768
+constexpr uint32_t KB_E = KB_SB + 32768;    // E bf16 MN-major 2 panels [64][64]         16384
 constexpr uint32_t KB_BYTES = KB_E + 16384;
 constexpr uint32_t KB_DYN = KB_BYTES + 1024;
 
@@ -288,6 +291,8 @@ __global__ void __launch_bounds__(256, 2)
       sig1[e] = J <= 1 ? __expf(s_Ge[J + 1][c] - GeJ[e]) : 0.f;  // for row block J + 2
       sig2[e] = J == 0 ? __expf(s_Ge[2][c] - GeJ[e]) : 0.f;      // for row block 3
     }
+    uint32_t qgp[2][8];  // Q o e^G of this thread's 4 tokens, bf16 pairs per channel
+    float qg_prev[8];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int r = 4 * rg + u, e16 = r & 15;
@@ -311,6 +316,10 @@ __global__ void __launch_bounds__(256, 2)
         const float ka = kv[e] * a, kb = kv[e] * b;
         o_lk[e] = ka;
         o_lq[e] = qv[e] * a;
+        // Q o e^G for the state pass, packed over token pairs (u, u+1)
+        const float qg = o_lq[e] * eGb[e];
+        if (u & 1) qgp[u >> 1][e] = ptx::pack_bf16x2(qg_prev[e], qg);
+        else qg_prev[e] = qg;
         o_r0[e] = kb;
         o_r1[e] = kb * sig1[e];
         o_r2[e] = kb * sig2[e];
@@ -333,6 +342,14 @@ __global__ void __launch_bounds__(256, 2)
       // beta K o e^G and beta V: MN-major A operands of the WY products
       *reinterpret_cast<uint4*>(sm + KA_XK + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_xk);
       *reinterpret_cast<uint4*>(sm + KA_BV + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_bv);
+    }
+    // Q o e^G into the lower panel of the [W; Q e^G] image (MN-major, row = channel,
+    // 64 tokens per 128-byte row): this thread's 4 tokens are 8 contiguous bytes
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = c0 + e;
+      *reinterpret_cast<uint2*>(img + IMG_A1 + 16384 + c * 128 + ((((4 * rg) >> 3) ^ c) & 7) * 16 +
+                                8 * (rg & 1)) = make_uint2(qgp[0][e], qgp[1][e]);
     }
   }
   if (rg == 0) {
@@ -369,12 +386,15 @@ __global__ void __launch_bounds__(256, 2)
     const int r = rho & 63, I = r >> 4;
     const float br = s_beta[r];
     float* As = reinterpret_cast<float*>(sm + KA_AS);
+    float xs[5][16];
+#pragma unroll
+    for (int grp = 0; grp < 5; ++grp)
+      ptx::tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + 80 * ch + 16 * grp, xs[grp]);
+    ptx::tmem_wait_ld();
 #pragma unroll
     for (int grp = 0; grp < 5; ++grp) {
       const int col0 = 80 * ch + 16 * grp;
-      float x[16];
-      ptx::tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + col0, x);
-      ptx::tmem_wait_ld();
+      float* x = xs[grp];
       const bool diag = col0 >= 96;
       int Jb;
       bool use;
@@ -518,7 +538,6 @@ __global__ void __launch_bounds__(256, 2)
         const uint32_t off = ptx::sw128_chunk(row, 4 * hh + k8);
         if (ch == 0) {
           *reinterpret_cast<uint4*>(img + IMG_A1 + off) = pk;
-          *reinterpret_cast<uint4*>(sm + KA_WT + off) = pk;
         } else {
           *reinterpret_cast<uint4*>(img + IMG_U + off) = pk;
         }
@@ -526,53 +545,6 @@ __global__ void __launch_bounds__(256, 2)
     }
   }
 
-  // ---- 7. (P W)^T = W^T P^T : M=128, N=64, K=64; then Q'^T = (Q o e^G)^T - (P W)^T
-  ptx::fence_proxy_async_smem();
-  ptx::tc_fence_before();
-  __syncthreads();
-  if (tid == 0) {
-    ptx::tc_fence_after();
-    constexpr uint32_t id = ptx::idesc_bf16(128, 64, false, false);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      ptx::mma_bf16(tmem, ptx::sdesc_sw128(sb + KA_WT + kk * 32, 16, 1024),
-                    ptx::sdesc_sw128(sb + KA_PT + kk * 32, 16, 1024), id, kk > 0);
-    ptx::mma_commit(&s_bar);
-  }
-  {
-    // thread = (channel c = tid mod 128, tokens 32 (tid / 128) + [0, 32)): re-read g and q
-    // (L2-resident) while the MMA runs; G restarts from the block-1 end for the upper half.
-    const int qd = warp & 3, half = warp >> 2;
-    const int c = 32 * qd + lane, r0 = 32 * half;
-    const size_t base1 = ((size_t)s0 * H + h) * D + c;
-    float gr[32], qr[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int r = r0 + i;
-      gr[i] = r < Cn ? g[base1 + (size_t)r * rs] : 0.f;
-      qr[i] = r < Cn ? __bfloat162float(q[base1 + (size_t)r * rs]) : 0.f;
-    }
-    float acc = half ? s_Ge[1][c] : 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      acc += gr[i];
-      qr[i] *= __expf(acc);
-    }
-    ptx::mbar_wait_bounded(&s_bar, 0);
-    ptx::tc_fence_after();
-    float x[32];
-    const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + r0;
-    ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
-    ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
-    ptx::tmem_wait_ld();
-#pragma unroll
-    for (int k8 = 0; k8 < 4; ++k8) {
-      float y[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = qr[8 * k8 + e] - x[8 * k8 + e];
-      *reinterpret_cast<uint4*>(img + IMG_A1 + 16384 + ptx::sw128_chunk(c, 4 * half + k8)) = pack8(y);
-    }
-  }
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) ptx::tmem_dealloc(tmem, 256);
@@ -620,16 +592,15 @@ __global__ void __launch_bounds__(256, 1)
     ptx::tmem_alloc(&s_tmem, 256);
     ptx::tmem_relinquish();
   }
-  // rows 0..63 of each stage's [-I; P] operand: -I (bf16 -1.0 = 0xBF80)
+  // constant [-I; 0] operand (K-major [128 rows][64 K]; bf16 -1.0 = 0xBF80)
   for (int idx = tid; idx < 1024; idx += 256) {
-    const int stg = idx >> 9, row = (idx >> 3) & 63, chunk = idx & 7;
+    const int row = idx >> 3, chunk = idx & 7;
     uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if ((row >> 3) == chunk) {
+    if (row < 64 && (row >> 3) == chunk) {
       const int e = row & 7;
       w[e >> 1] = (e & 1) ? 0xBF800000u : 0x0000BF80u;
     }
-    *reinterpret_cast<uint4*>(sm + stg * KB_STAGE + ptx::sw128_chunk(row, chunk)) =
-        make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(sm + KB_NEGI + ptx::sw128_chunk(row, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
@@ -686,7 +657,7 @@ __global__ void __launch_bounds__(256, 1)
 
     auto issue = [&](long long chunk_idx, int stage) {
       ptx::mbar_arrive_expect_tx(&s_full[stage], IMG_BYTES);
-      ptx::bulk_g2s(sm + stage * KB_STAGE + KB_IMG, ws + ((size_t)chunk_idx * H + h) * IMG_BYTES,
+      ptx::bulk_g2s(sm + KB_STAGE0 + stage * KB_STAGE, ws + ((size_t)chunk_idx * H + h) * IMG_BYTES,
                     IMG_BYTES, &s_full[stage]);
     };
     if (tid == 0 && nc > 0) {
@@ -695,8 +666,8 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int cc = 0; cc < nc; ++cc, ++it) {
       const int st = it & 1;
-      uint8_t* stage = sm + st * KB_STAGE;
-      const uint32_t sst = sb + st * KB_STAGE;
+      uint8_t* stage = sm + KB_STAGE0 + st * KB_STAGE;
+      const uint32_t sst = sb + KB_STAGE0 + st * KB_STAGE;
       const long long s = start + (long long)cc * C;
       const int Cn = min(C, len - cc * C);
       if (tid == 0) {
@@ -704,45 +675,38 @@ __global__ void __launch_bounds__(256, 1)
         if (!ptx::mbar_wait_bounded(&s_full[st], (it >> 1) & 1)) s_abort = 1;
         pending_stage = (cc + 1 < nc) ? (st ^ 1) : -1;
         ptx::tc_fence_after();
-        // X = [-I; P] U  (M=128, N=128, K=64, both K-major)
+        // X = [-I; 0] U  (M=128, N=128, K=64, both K-major)
         constexpr uint32_t id0 = ptx::idesc_bf16(128, 128, false, false);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + kk * 32, 16, 1024),
-                        ptx::sdesc_sw128(sst + KB_IMG + IMG_U + kk * 32, 16, 1024), id0, kk > 0);
-        // X += [W; Q'] S  (M=128, N=128, K=128, both MN-major)
+          ptx::mma_bf16(tX, ptx::sdesc_sw128(sb + KB_NEGI + kk * 32, 16, 1024),
+                        ptx::sdesc_sw128(sst + IMG_U + kk * 32, 16, 1024), id0, kk > 0);
+        // X += [W; Q e^G] S  (M=128, N=128, K=128, both MN-major)
         constexpr uint32_t id1 = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + KB_IMG + IMG_A1 + kk * 2048, 16384, 1024),
+          ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + IMG_A1 + kk * 2048, 16384, 1024),
                         ptx::sdesc_sw128(sb + KB_SB + kk * 2048, 16384, 1024), id1, 1);
         ptx::mma_commit(&s_xbar);
       }
       if (!ptx::mbar_wait_bounded(&s_xbar, it & 1)) s_abort = 1;
       ptx::tc_fence_after();
-      const float gam = reinterpret_cast<const float*>(stage + KB_IMG + IMG_G)[c];
-      // epilogue 1: rows 0..63 -> E = -X (bf16 operand), rows 64..127 -> O
+      const float gam = reinterpret_cast<const float*>(stage + IMG_G)[c];
+      // epilogue 1: rows 0..63 -> E = -X (bf16 operand)
+      if (qd < 2) {
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float x[32];
-        const uint32_t ta = tX + lane_off + 64 * ch + 32 * hh;
-        ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
-        ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
-        ptx::tmem_wait_ld();
-        if (qd < 2) {
+        for (int hh = 0; hh < 2; ++hh) {
+          float x[32];
+          const uint32_t ta = tX + lane_off + 64 * ch + 32 * hh;
+          ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
+          ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+          ptx::tmem_wait_ld();
 #pragma unroll
           for (int k8 = 0; k8 < 4; ++k8) {
             float y[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) y[e] = -x[8 * k8 + e];
             *reinterpret_cast<uint4*>(sm + KB_E + ch * 8192 + ptx::sw128_chunk(c, 4 * hh + k8)) = pack8(y);
-          }
-        } else {
-          const int r = c - 64;
-          if (r < Cn) {
-            bf16* dst = o + ((size_t)(s + r) * H + h) * D + 64 * ch + 32 * hh;
-#pragma unroll
-            for (int k8 = 0; k8 < 4; ++k8) reinterpret_cast<uint4*>(dst)[k8] = pack8(x + 8 * k8);
           }
         }
       }
@@ -755,8 +719,15 @@ __global__ void __launch_bounds__(256, 1)
         constexpr uint32_t id2 = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_bf16(tY, ptx::sdesc_sw128(sst + KB_IMG + IMG_KB + kk * 2048, 8192, 1024),
+          ptx::mma_bf16(tY, ptx::sdesc_sw128(sst + IMG_KB + kk * 2048, 8192, 1024),
                         ptx::sdesc_sw128(sb + KB_E + kk * 2048, 8192, 1024), id2, kk > 0);
+        // X += [*; P] E: rows 64..127 become O = Q e^G S + P E (rows 0..63 are dead);
+        // A = the 8 KB in front of P (unused rows) followed by P, K-major [128][64]
+        constexpr uint32_t id3 = ptx::idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + IMG_P - 8192 + kk * 32, 16, 1024),
+                        ptx::sdesc_sw128(sb + KB_E + kk * 2048, 8192, 1024), id3, 1);
         ptx::mma_commit(&s_ybar);
       }
       if (!ptx::mbar_wait_bounded(&s_ybar, it & 1)) s_abort = 1;
@@ -772,6 +743,23 @@ __global__ void __launch_bounds__(256, 1)
         for (int e = 0; e < 32; ++e) S[32 * hh + e] = fmaf(gam, S[32 * hh + e], y[e]);
       }
       store_state_bf16(sm, c, ch, S);
+      // rows 64..127 of X: the chunk's outputs
+      if (qd >= 2) {
+        const int r = c - 64;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float x[32];
+          const uint32_t ta = tX + lane_off + 64 * ch + 32 * hh;
+          ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
+          ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+          ptx::tmem_wait_ld();
+          if (r < Cn) {
+            bf16* dst = o + ((size_t)(s + r) * H + h) * D + 64 * ch + 32 * hh;
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) reinterpret_cast<uint4*>(dst)[k8] = pack8(x + 8 * k8);
+          }
+        }
+      }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
