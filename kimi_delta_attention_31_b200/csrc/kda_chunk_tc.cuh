@@ -161,8 +161,38 @@ __device__ __forceinline__ float sel4(int i, float a0, float a1, float a2, float
 // 4 (t / 16) .. + 3, so every global load and shared store moves 16 bytes.
 // ---------------------------------------------------------------------------
 constexpr uint32_t KA_TS = 33792;  // after the first MMA: T fp32 [64][68]          17408
-constexpr uint32_t KA_MT = 51200;  //                      block products [3][16][16] 3072
+constexpr uint32_t KA_MT = 51200;  //                      block products [3][16][20] 3840
+constexpr int MT_LD = 20;          // row stride (floats) of a block product
 constexpr int AS_LD = 68;          // row stride (floats) of A and T in fp32
+
+// acc (16 x 16 as two m16n8 halves) += X (16 x 16, fp32, row stride ldx) * Y (16 x 16,
+// row stride ldy), one warp, TF32 operands with fp32 accumulation.
+__device__ __forceinline__ void warp_gemm16(float (&acc)[2][4], const float* xp, int ldx, const float* yp,
+                                            int ldy, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int kh = 0; kh < 2; ++kh) {
+    const uint32_t a[4] = {ptx::to_tf32(xp[g * ldx + 8 * kh + t]), ptx::to_tf32(xp[(g + 8) * ldx + 8 * kh + t]),
+                           ptx::to_tf32(xp[g * ldx + 8 * kh + t + 4]),
+                           ptx::to_tf32(xp[(g + 8) * ldx + 8 * kh + t + 4])};
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+      const uint32_t b[2] = {ptx::to_tf32(yp[(8 * kh + t) * ldy + 8 * nh + g]),
+                             ptx::to_tf32(yp[(8 * kh + t + 4) * ldy + 8 * nh + g])};
+      ptx::mma_tf32_m16n8k8(acc[nh], a, b);
+    }
+  }
+}
+__device__ __forceinline__ void warp_store16(float* dp, int ldd, const float (&acc)[2][4], float scale, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nh = 0; nh < 2; ++nh) {
+    dp[g * ldd + 8 * nh + 2 * t] = scale * acc[nh][0];
+    dp[g * ldd + 8 * nh + 2 * t + 1] = scale * acc[nh][1];
+    dp[(g + 8) * ldd + 8 * nh + 2 * t] = scale * acc[nh][2];
+    dp[(g + 8) * ldd + 8 * nh + 2 * t + 1] = scale * acc[nh][3];
+  }
+}
 
 __device__ __forceinline__ void unpack8(uint4 w, float* x) {
   const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&w);
@@ -178,7 +208,7 @@ __global__ void __launch_bounds__(256, 2)
     kda_tc_chunk_local_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                               const bf16* __restrict__ v, const float* __restrict__ g,
                               const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
-                              int num_seqs, int T, int H, uint8_t* __restrict__ ws) {
+                              int num_seqs, int T, int H, int prefetch_dist, uint8_t* __restrict__ ws) {
   __shared__ float s_beta[C];
   __shared__ __align__(16) float s_Ge[4][D];  // G at the end of each 16-token block
   __shared__ __align__(8) uint64_t s_bar;
@@ -219,6 +249,28 @@ __global__ void __launch_bounds__(256, 2)
   uint8_t* img = ws + ((size_t)ci * H + h) * IMG_BYTES;
   const size_t rs = (size_t)H * D;  // elements between consecutive tokens
 
+  // L2 hint for the (chunk, head) that will start about one residency wave
+  // later (grid index + prefetch_dist): its q, k, v, g rows, one line per lane.
+  if (!cu_seqlens && prefetch_dist > 0 && blockIdx.x + (long long)prefetch_dist < gridDim.x) {
+    const long long nb = blockIdx.x + (long long)prefetch_dist;
+    const int nh = (int)(nb % H);
+    const long long ncps = (T + C - 1) / C, nci = nb / H, ncc = nci % ncps;
+    const long long ns = (nci / ncps) * T + ncc * C;
+    const int ncn = (int)min((long long)C, (long long)T - ncc * C);
+    // per token row: k, q, v 2 lines each, g 4 lines: 10 lines x 64 rows
+    for (int idx = tid; idx < 10 * C; idx += 256) {
+      const int r = idx / 10, l = idx % 10;
+      if (r < ncn) {
+        const size_t off = ((size_t)(ns + r) * H + nh) * D;
+        const void* p = l < 2 ? (const void*)(k + off + 64 * l)
+                      : l < 4 ? (const void*)(q + off + 64 * (l - 2))
+                      : l < 6 ? (const void*)(v + off + 64 * (l - 4))
+                              : (const void*)(g + off + 32 * (l - 6));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+      }
+    }
+  }
+
   if (warp == 0) {
     ptx::tmem_alloc(&s_tmem, 256);
     ptx::tmem_relinquish();
@@ -229,11 +281,28 @@ __global__ void __launch_bounds__(256, 2)
   }
   if (tid < C) s_beta[tid] = tid < Cn ? beta[(size_t)(s0 + tid) * H + h] : 0.f;
 
-  // ---- 1. cumulative log-decay G (fp32); rows >= Cn contribute g = 0
+  // ---- 1. loads; cumulative log-decay G (fp32); rows >= Cn contribute g = 0.
+  // The k, q, v rows are loaded here, together with g, and parked in TMEM
+  // columns (idle until the first MMA) so that their latency overlaps g's.
   const int co = tid & 15, rg = tid >> 4, J = rg >> 2;  // channel octet, row group, 16-token block
   const int c0 = 8 * co;
   const uint32_t kp = co >> 3, ck = co & 7;  // K-panel and 16-byte chunk of the channels
   const size_t base8 = ((size_t)s0 * H + h) * D + c0;
+  uint32_t kst[16], qst[16], vst[16];  // [row u][4 words]: 8 bf16 per row
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int r = 4 * rg + u;
+    uint4 kw = make_uint4(0, 0, 0, 0), qw = kw, vw = kw;
+    if (r < Cn) {
+      const size_t off = base8 + (size_t)r * rs;
+      kw = *reinterpret_cast<const uint4*>(k + off);
+      qw = *reinterpret_cast<const uint4*>(q + off);
+      vw = *reinterpret_cast<const uint4*>(v + off);
+    }
+    kst[4 * u] = kw.x; kst[4 * u + 1] = kw.y; kst[4 * u + 2] = kw.z; kst[4 * u + 3] = kw.w;
+    qst[4 * u] = qw.x; qst[4 * u + 1] = qw.y; qst[4 * u + 2] = qw.z; qst[4 * u + 3] = qw.w;
+    vst[4 * u] = vw.x; vst[4 * u + 1] = vw.y; vst[4 * u + 2] = vw.z; vst[4 * u + 3] = vw.w;
+  }
   float G[4][8];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -255,6 +324,12 @@ __global__ void __launch_bounds__(256, 2)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = s_tmem;
+  // stash: warp w uses lanes 32 (w mod 4) .., columns 48 (w / 4) + [k 0..15 | q 16..31 | v 32..47]
+  const uint32_t stash = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 48 * (warp >> 2);
+  ptx::tmem_st16u(stash, kst);
+  ptx::tmem_st16u(stash + 16, qst);
+  ptx::tmem_st16u(stash + 32, vst);
+  ptx::tmem_wait_st();
   {
     float off[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -296,13 +371,14 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int r = 4 * rg + u, e16 = r & 15;
-      uint4 kw = make_uint4(0, 0, 0, 0), qw = kw, vw = kw;
-      if (r < Cn) {
-        const size_t off = base8 + (size_t)r * rs;
-        kw = *reinterpret_cast<const uint4*>(k + off);
-        qw = *reinterpret_cast<const uint4*>(q + off);
-        vw = *reinterpret_cast<const uint4*>(v + off);
-      }
+      uint32_t kr4[4], qr4[4], vr4[4];
+      ptx::tmem_ld4u(stash + 4 * u, kr4);
+      ptx::tmem_ld4u(stash + 16 + 4 * u, qr4);
+      ptx::tmem_ld4u(stash + 32 + 4 * u, vr4);
+      ptx::tmem_wait_ld();
+      const uint4 kw = make_uint4(kr4[0], kr4[1], kr4[2], kr4[3]);
+      const uint4 qw = make_uint4(qr4[0], qr4[1], qr4[2], qr4[3]);
+      const uint4 vw = make_uint4(vr4[0], vr4[1], vr4[2], vr4[3]);
       float kv[8], qv[8], vv[8];
       unpack8(kw, kv);
       unpack8(qw, qv);
@@ -427,65 +503,50 @@ __global__ void __launch_bounds__(256, 2)
   ptx::tc_fence_before();
   __syncthreads();
 
-  // ---- 5. T = (I + A)^{-1} in fp32, blocked by 16: invert the diagonal blocks,
-  //         then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ by distance below the diagonal.
+  // ---- 5. T = (I + A)^{-1}, blocked by 16.  Diagonal blocks: forward
+  //         substitution in fp32, one column per 4 lanes (warp shuffles).
+  //         Then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ by distance below the
+  //         diagonal, one warp per block, TF32 warp MMAs with fp32 accumulation.
   {
     const float* As = reinterpret_cast<const float*>(sm + KA_AS);
     float* Ts = reinterpret_cast<float*>(sm + KA_TS);
     float* Mt = reinterpret_cast<float*>(sm + KA_MT);
-    if (tid < 64) {  // column jj of diagonal block Ib, forward substitution
-      const int Ib = tid >> 4, jj = tid & 15, o = 16 * Ib;
-      float x[16];
+    {
+      const int j = tid >> 2, part = tid & 3;  // column j of T; this lane keeps rows 4 m + part
+      const int Ib = j >> 4, jj = j & 15, o = 16 * Ib;
+      float x[4];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = (i == jj) ? 1.f : 0.f;
+      for (int m = 0; m < 4; ++m) x[m] = (4 * m + part == jj) ? 1.f : 0.f;
 #pragma unroll
       for (int i = 1; i < 16; ++i) {
-        float a4[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc = 0.f;
 #pragma unroll
-        for (int m = 0; m < i; ++m) a4[m & 3] = fmaf(As[(o + i) * AS_LD + o + m], x[m], a4[m & 3]);
-        const float val = -((a4[0] + a4[1]) + (a4[2] + a4[3]));
-        if (i > jj) x[i] = val;
+        for (int m = 0; m < 4; ++m)
+          if (4 * m < i) acc = fmaf(As[(o + i) * AS_LD + o + 4 * m + part], x[m], acc);  // A[i][>=i] == 0
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if ((i & 3) == part && i > jj) x[i >> 2] = -acc;
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) Ts[(o + i) * AS_LD + o + jj] = x[i];
+      for (int m = 0; m < 4; ++m) Ts[(o + 4 * m + part) * AS_LD + o + jj] = x[m];
     }
     __syncthreads();
-    const int blk = tid >> 6, tt = tid & 63, i = tt >> 2, j4 = tt & 3;
 #pragma unroll
     for (int dist = 1; dist <= 3; ++dist) {
-      const bool act = blk < 4 - dist;
-      const int Jc = blk, Ir = blk + dist;
-      if (act) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (warp < 4 - dist) {
+        const int Jc = warp, Ir = warp + dist;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int kk = 0; kk < dist; ++kk) {
           const int K = Jc + kk;
-#pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const float a = As[(16 * Ir + i) * AS_LD + 16 * K + m];
-            const float4 t = *reinterpret_cast<const float4*>(Ts + (16 * K + m) * AS_LD + 16 * Jc + 4 * j4);
-            acc.x = fmaf(a, t.x, acc.x);
-            acc.y = fmaf(a, t.y, acc.y);
-            acc.z = fmaf(a, t.z, acc.z);
-            acc.w = fmaf(a, t.w, acc.w);
-          }
+          warp_gemm16(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
         }
-        *reinterpret_cast<float4*>(Mt + blk * 256 + i * 16 + 4 * j4) = acc;
-      }
-      __syncthreads();
-      if (act) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const float a = Ts[(16 * Ir + i) * AS_LD + 16 * Ir + m];  // T_II, zero above its diagonal
-          const float4 t = *reinterpret_cast<const float4*>(Mt + blk * 256 + m * 16 + 4 * j4);
-          acc.x = fmaf(a, t.x, acc.x);
-          acc.y = fmaf(a, t.y, acc.y);
-          acc.z = fmaf(a, t.z, acc.z);
-          acc.w = fmaf(a, t.w, acc.w);
-        }
-        *reinterpret_cast<float4*>(Ts + (16 * Ir + i) * AS_LD + 16 * Jc + 4 * j4) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        float* mt = Mt + warp * 16 * MT_LD;
+        warp_store16(mt, MT_LD, acc, 1.f, lane);
+        __syncwarp();
+        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        warp_gemm16(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
+        warp_store16(Ts + 16 * Ir * AS_LD + 16 * Jc, AS_LD, acc2, -1.f, lane);
       }
       __syncthreads();
     }
@@ -820,7 +881,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   if (gridA > 0x7fffffffLL) return cudaErrorInvalidValue;
   if (gridA > 0) {
     tc::kda_tc_chunk_local_kernel<<<(unsigned)gridA, 256, tc::KA_DYN, stream>>>(
-        q, k, v, g, beta, cu_seqlens, num_seqs, T, H, ws);
+        q, k, v, g, beta, cu_seqlens, num_seqs, T, H, 2 * s_sms, ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
