@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(256, 2)
     kda_tc_chunk_local_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                               const bf16* __restrict__ v, const float* __restrict__ g,
                               const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
-                              int num_seqs, int T, int H, int prefetch_dist, uint8_t* __restrict__ ws) {
+                              int num_seqs, int T, int H, long long num_items, uint8_t* __restrict__ ws) {
   __shared__ float s_beta[C];
   __shared__ __align__(16) float s_Ge[4][D];  // G at the end of each 16-token block
   __shared__ __align__(8) uint64_t s_bar;
@@ -220,8 +220,26 @@ __global__ void __launch_bounds__(256, 2)
   const uint32_t sb = ptx::smem_u32(sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.x % H;
-  const long long ci = blockIdx.x / H;
+  const size_t rs = (size_t)H * D;  // elements between consecutive tokens
+
+  if (warp == 0) {
+    ptx::tmem_alloc(&s_tmem, 256);
+    ptx::tmem_relinquish();
+  }
+  if (tid == 0) {
+    ptx::mbar_init(&s_bar, 1);
+    ptx::fence_mbar_init();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  // Persistent: this CTA handles items (chunk * H + head) blockIdx.x, + gridDim.x, ...
+  // Each processed item completes s_bar twice (parities 0 then 1).
+  for (long long item = blockIdx.x; item < num_items; item += gridDim.x) {
+  const int h = (int)(item % H);
+  const long long ci = item / H;
 
   long long s0;
   int Cn;
@@ -244,40 +262,32 @@ __global__ void __launch_bounds__(256, 2)
     s0 = (ci / cps) * T + cc * C;
     Cn = (int)min((long long)C, (long long)T - cc * C);
   }
-  if (Cn <= 0) return;  // uniform across the CTA
+  if (Cn <= 0) {  // uniform across the CTA: past the last chunk of a packed batch
+    __syncthreads();  // everyone has read s_loc before warp 0 rewrites it
+    continue;
+  }
 
   uint8_t* img = ws + ((size_t)ci * H + h) * IMG_BYTES;
-  const size_t rs = (size_t)H * D;  // elements between consecutive tokens
 
-  // L2 hint for the (chunk, head) that will start about one residency wave
-  // later (grid index + prefetch_dist): its q, k, v, g rows, one line per lane.
-  if (!cu_seqlens && prefetch_dist > 0 && blockIdx.x + (long long)prefetch_dist < gridDim.x) {
-    const long long nb = blockIdx.x + (long long)prefetch_dist;
+  // L2 hint for this CTA's next item (packed-free layout only): its q, k, v, g
+  // rows, one 128-byte line per lane.
+  if (!cu_seqlens && item + gridDim.x < num_items) {
+    const long long nb = item + gridDim.x;
     const int nh = (int)(nb % H);
     const long long ncps = (T + C - 1) / C, nci = nb / H, ncc = nci % ncps;
     const long long ns = (nci / ncps) * T + ncc * C;
     const int ncn = (int)min((long long)C, (long long)T - ncc * C);
-    // per token row: k, q, v 2 lines each, g 4 lines: 10 lines x 64 rows
     for (int idx = tid; idx < 10 * C; idx += 256) {
       const int r = idx / 10, l = idx % 10;
       if (r < ncn) {
         const size_t off = ((size_t)(ns + r) * H + nh) * D;
-        const void* p = l < 2 ? (const void*)(k + off + 64 * l)
-                      : l < 4 ? (const void*)(q + off + 64 * (l - 2))
-                      : l < 6 ? (const void*)(v + off + 64 * (l - 4))
-                              : (const void*)(g + off + 32 * (l - 6));
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+        const void* pp = l < 2 ? (const void*)(k + off + 64 * l)
+                       : l < 4 ? (const void*)(q + off + 64 * (l - 2))
+                       : l < 6 ? (const void*)(v + off + 64 * (l - 4))
+                               : (const void*)(g + off + 32 * (l - 6));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(pp));
       }
     }
-  }
-
-  if (warp == 0) {
-    ptx::tmem_alloc(&s_tmem, 256);
-    ptx::tmem_relinquish();
-  }
-  if (tid == 0) {
-    ptx::mbar_init(&s_bar, 1);
-    ptx::fence_mbar_init();
   }
   if (tid < C) s_beta[tid] = tid < Cn ? beta[(size_t)(s0 + tid) * H + h] : 0.f;
 
@@ -323,7 +333,6 @@ __global__ void __launch_bounds__(256, 2)
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tmem = s_tmem;
   // stash: warp w uses lanes 32 (w mod 4) .., columns 48 (w / 4) + [k 0..15 | q 16..31 | v 32..47]
   const uint32_t stash = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 48 * (warp >> 2);
   ptx::tmem_st16u(stash, kst);
@@ -451,7 +460,7 @@ __global__ void __launch_bounds__(256, 2)
     }
     ptx::mma_commit(&s_bar);
   }
-  ptx::mbar_wait_bounded(&s_bar, 0);
+  ptx::mbar_wait_bounded(&s_bar, 0);  // first completion of this item
   ptx::tc_fence_after();
 
   // ---- 4. scatter A (fp32, beta-scaled) and P (bf16, lower incl. diagonal, zero above)
@@ -581,7 +590,7 @@ __global__ void __launch_bounds__(256, 2)
   }
   for (int i2 = tid; i2 < 512; i2 += 256)
     reinterpret_cast<uint4*>(img + IMG_P)[i2] = reinterpret_cast<const uint4*>(sm + KA_PT)[i2];
-  ptx::mbar_wait_bounded(&s_bar, 1);
+  ptx::mbar_wait_bounded(&s_bar, 1);  // second completion of this item
   ptx::tc_fence_after();
   {
     const int qd = warp & 3, ch = warp >> 2;
@@ -607,7 +616,8 @@ __global__ void __launch_bounds__(256, 2)
   }
 
   ptx::tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // every TMEM read of this item is done before the next item's stash
+  }  // item loop
   if (warp == 0) ptx::tmem_dealloc(tmem, 256);
 }
 
@@ -877,11 +887,11 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int num_seqs = cu_seqlens ? N : 0;
-  const long long gridA = max_chunks * H;
-  if (gridA > 0x7fffffffLL) return cudaErrorInvalidValue;
-  if (gridA > 0) {
-    tc::kda_tc_chunk_local_kernel<<<(unsigned)gridA, 256, tc::KA_DYN, stream>>>(
-        q, k, v, g, beta, cu_seqlens, num_seqs, T, H, 2 * s_sms, ws);
+  const long long items = max_chunks * H;
+  if (items > 0) {
+    const int gridA = (int)(items < 2LL * s_sms ? items : 2LL * s_sms);
+    tc::kda_tc_chunk_local_kernel<<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens,
+                                                                        num_seqs, T, H, items, ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
