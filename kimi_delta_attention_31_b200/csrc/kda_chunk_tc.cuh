@@ -60,13 +60,15 @@ constexpr uint32_t IMG_G = 73728;   // gamma = e^{G_last}, fp32 [128]           
 constexpr uint32_t IMG_BYTES = 74240;
 
 // chunk-local kernel shared memory (dynamic, 1024-aligned base)
+// L3 is two K-panels of 128 rows: rows 0..63 (the K part) of each panel are
+// bytes [0, 8K) and [16K, 24K); the Q part fills [8K, 16K) and [24K, 32K).
 constexpr uint32_t KA_L3 = 0;       // [K a; Q a]  K-major [128][128] (2 K-panels)  32768
 constexpr uint32_t KA_RB = 32768;   // right operands K-major [160][128]          40960
-constexpr uint32_t KA_AS = 0;       // after the first MMA: A fp32 [64][68]       17408
-constexpr uint32_t KA_PT = 17408;   //                      P bf16 K-major          8192
-constexpr uint32_t KA_TT = 25600;   //                      T bf16 K-major          8192
-constexpr uint32_t KA_XK = 73728;   // beta K e^G  MN-major 2 panels [64][64]       16384
-constexpr uint32_t KA_BV = 90112;   // beta V      MN-major 2 panels [64][64]       16384
+constexpr uint32_t KA_PT = 8192;    // after the first MMA: P bf16 K-major (Q part of panel 0) 8192
+constexpr uint32_t KA_TT = 24576;   //                      T diag(beta) bf16 (Q part of panel 1) 8192
+constexpr uint32_t KA_AS = 32768;   //                      A fp32 [64][68] (over RB)  17408
+constexpr uint32_t KA_XK = 73728;   // K o e^G  MN-major 2 panels [64][64] (block path) 16384
+constexpr uint32_t KA_BV = 90112;   // V        MN-major 2 panels [64][64]       16384
 constexpr uint32_t KA_BYTES = 106496;
 constexpr uint32_t KA_DYN = KA_BYTES + 1024;
 
@@ -160,8 +162,12 @@ __device__ __forceinline__ float sel4(int i, float a0, float a1, float a2, float
 // Operand building: thread t owns channels 8 (t mod 16) .. + 7 of rows
 // 4 (t / 16) .. + 3, so every global load and shared store moves 16 bytes.
 // ---------------------------------------------------------------------------
-constexpr uint32_t KA_TS = 33792;  // after the first MMA: T fp32 [64][68]          17408
-constexpr uint32_t KA_MT = 51200;  //                      block products [3][16][20] 3840
+constexpr uint32_t KA_TS = 50176;  // after the first MMA: T fp32 [64][68] (over RB) 17408
+constexpr uint32_t KA_MT = 67584;  //                      block products [3][16][20] 3840
+// A chunk whose every channel keeps its log-decay over the whole chunk above
+// this bound takes the single-reference form (left K o e^{G}, right K o e^{-G}):
+// both factors and every product stay inside the fp32 / bf16 exponent range.
+constexpr float kChunkRefMinG = -80.f;
 constexpr int MT_LD = 20;          // row stride (floats) of a block product
 constexpr int AS_LD = 68;          // row stride (floats) of A and T in fp32
 
@@ -209,7 +215,7 @@ __global__ void __launch_bounds__(256, 2)
                               const bf16* __restrict__ v, const float* __restrict__ g,
                               const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                               int num_seqs, int T, int H, long long num_items, uint8_t* __restrict__ ws) {
-  __shared__ float s_beta[C];
+  __shared__ __align__(16) float s_beta[C];
   __shared__ __align__(16) float s_Ge[4][D];  // G at the end of each 16-token block
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ uint32_t s_tmem;
@@ -355,14 +361,57 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
       for (int e = 0; e < 8; ++e) G[u][e] += off[e];
   }
+  bool steep = false;  // some channel decays below the single-reference range
   if ((rg & 3) == 3) {
     reinterpret_cast<float4*>(&s_Ge[J][c0])[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
     reinterpret_cast<float4*>(&s_Ge[J][c0])[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) steep |= (J == 3) && !(G[3][e] >= kChunkRefMinG);
   }
-  __syncthreads();
+  // G is non-increasing (g <= 0), so G at the chunk's last row is each channel's minimum.
+  const bool fast = !__syncthreads_or(steep);
 
   // ---- 2. decay-scaled bf16 operands, 16-byte stores
-  {
+  uint32_t qgp[2][8];  // Q o e^G of this thread's 4 tokens, bf16 pairs per channel
+  if (fast) {
+    // Single reference (chunk start): a = e^{G} <= 1, rho = e^{-G} >= 1.
+    float gam[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) gam[e] = __expf(s_Ge[3][c0 + e]);
+    float qg_prev[8];
+    uint8_t* l3 = sm + KA_L3 + kp * 16384;
+    uint8_t* rb = sm + KA_RB + kp * 20480;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = 4 * rg + u;
+      uint32_t kr4[4], qr4[4], vr4[4];
+      ptx::tmem_ld4u(stash + 4 * u, kr4);
+      ptx::tmem_ld4u(stash + 16 + 4 * u, qr4);
+      ptx::tmem_ld4u(stash + 32 + 4 * u, vr4);
+      ptx::tmem_wait_ld();
+      float kv[8], qv[8];
+      unpack8(make_uint4(kr4[0], kr4[1], kr4[2], kr4[3]), kv);
+      unpack8(make_uint4(qr4[0], qr4[1], qr4[2], qr4[3]), qv);
+      float o_ka[8], o_qa[8], o_kr[8], o_kb[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float a = __expf(G[u][e]);     // (0, 1]
+        const float rho = __expf(-G[u][e]);  // [1, e^80]
+        o_ka[e] = kv[e] * a;
+        o_qa[e] = qv[e] * a;
+        o_kr[e] = kv[e] * rho;
+        o_kb[e] = o_kr[e] * gam[e];          // K o e^{G_last - G}
+        if (u & 1) qgp[u >> 1][e] = ptx::pack_bf16x2(qg_prev[e], o_qa[e]);
+        else qg_prev[e] = o_qa[e];
+      }
+      *reinterpret_cast<uint4*>(l3 + ptx::sw128_chunk(r, ck)) = pack8(o_ka);
+      *reinterpret_cast<uint4*>(l3 + ptx::sw128_chunk(64 + r, ck)) = pack8(o_qa);
+      *reinterpret_cast<uint4*>(rb + ptx::sw128_chunk(r, ck)) = pack8(o_kr);
+      *reinterpret_cast<uint4*>(img + IMG_KB + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_kb);
+      *reinterpret_cast<uint4*>(sm + KA_BV + kp * 8192 + ptx::sw128_chunk(r, ck)) =
+          make_uint4(vr4[0], vr4[1], vr4[2], vr4[3]);
+    }
+  } else {
     float Gb[8], GeJ[8], eGb[8], invD[8], lam[8], sig1[8], sig2[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -375,7 +424,6 @@ __global__ void __launch_bounds__(256, 2)
       sig1[e] = J <= 1 ? __expf(s_Ge[J + 1][c] - GeJ[e]) : 0.f;  // for row block J + 2
       sig2[e] = J == 0 ? __expf(s_Ge[2][c] - GeJ[e]) : 0.f;      // for row block 3
     }
-    uint32_t qgp[2][8];  // Q o e^G of this thread's 4 tokens, bf16 pairs per channel
     float qg_prev[8];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -388,12 +436,10 @@ __global__ void __launch_bounds__(256, 2)
       const uint4 kw = make_uint4(kr4[0], kr4[1], kr4[2], kr4[3]);
       const uint4 qw = make_uint4(qr4[0], qr4[1], qr4[2], qr4[3]);
       const uint4 vw = make_uint4(vr4[0], vr4[1], vr4[2], vr4[3]);
-      float kv[8], qv[8], vv[8];
+      float kv[8], qv[8];
       unpack8(kw, kv);
       unpack8(qw, qv);
-      unpack8(vw, vv);
-      const float br = s_beta[r];
-      float o_lk[8], o_lq[8], o_r0[8], o_r1[8], o_r2[8], o_rd[8], o_kb[8], o_xk[8], o_bv[8];
+      float o_lk[8], o_lq[8], o_r0[8], o_r1[8], o_r2[8], o_rd[8], o_kb[8], o_xk[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float a = __expf(G[u][e] - Gb[e]);   // (0, 1]
@@ -410,8 +456,7 @@ __global__ void __launch_bounds__(256, 2)
         o_r2[e] = kb * sig2[e];
         o_rd[e] = kb * invD[e];
         o_kb[e] = kb * lam[e];
-        o_xk[e] = br * ka * eGb[e];
-        o_bv[e] = br * vv[e];
+        o_xk[e] = ka * eGb[e];
       }
       uint8_t* l3 = sm + KA_L3 + kp * 16384;
       uint8_t* rb = sm + KA_RB + kp * 20480;
@@ -424,10 +469,12 @@ __global__ void __launch_bounds__(256, 2)
       *reinterpret_cast<uint4*>(rb + ptx::sw128_chunk(96 + r, ck)) = pack8(o_rd);
       // Kbar = K o e^{G_last - G} (image, MN-major panel = channel / 64, row = token)
       *reinterpret_cast<uint4*>(img + IMG_KB + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_kb);
-      // beta K o e^G and beta V: MN-major A operands of the WY products
+      // K o e^G and V: MN-major A operands of the WY products (beta is folded into T)
       *reinterpret_cast<uint4*>(sm + KA_XK + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_xk);
-      *reinterpret_cast<uint4*>(sm + KA_BV + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_bv);
+      *reinterpret_cast<uint4*>(sm + KA_BV + kp * 8192 + ptx::sw128_chunk(r, ck)) = vw;
     }
+  }
+  {
     // Q o e^G into the lower panel of the [W; Q e^G] image (MN-major, row = channel,
     // 64 tokens per 128-byte row): this thread's 4 tokens are 8 contiguous bytes
 #pragma unroll
@@ -445,13 +492,14 @@ __global__ void __launch_bounds__(256, 2)
     reinterpret_cast<float4*>(img + IMG_G)[2 * co + 1] = make_float4(gm[4], gm[5], gm[6], gm[7]);
   }
 
-  // ---- 3. [A'; P'] = [K a; Q a] (right operands)^T : M=128, N=160, K=128
+  // ---- 3. [A'; P'] = [K a; Q a] (right operands)^T : M=128, K=128,
+  //         N=64 (single reference) or 160 (block references)
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   if (tid == 0) {
     ptx::tc_fence_after();
-    constexpr uint32_t id = ptx::idesc_bf16(128, 160, false, false);
+    const uint32_t id = fast ? ptx::idesc_bf16(128, 64, false, false) : ptx::idesc_bf16(128, 160, false, false);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const uint64_t ad = ptx::sdesc_sw128(sb + KA_L3 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
@@ -464,7 +512,29 @@ __global__ void __launch_bounds__(256, 2)
   ptx::tc_fence_after();
 
   // ---- 4. scatter A (fp32, beta-scaled) and P (bf16, lower incl. diagonal, zero above)
-  {
+  if (fast) {  // TMEM columns 0..63 hold whole rows; warp half ch takes columns 32 ch ..
+    const int qd = warp & 3, ch = warp >> 2;
+    const int rho = 32 * qd + lane, r = rho & 63, j0 = 32 * ch;
+    float x[32];
+    const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + j0;
+    ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
+    ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+    ptx::tmem_wait_ld();
+    if (rho < 64) {  // warp-uniform
+      const float br = s_beta[r];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = (j0 + e < r) ? br * x[e] : 0.f;
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(sm + KA_AS) + r * AS_LD + j0);
+#pragma unroll
+      for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(x[4 * v4], x[4 * v4 + 1], x[4 * v4 + 2], x[4 * v4 + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = (j0 + e <= r) ? x[e] : 0.f;
+#pragma unroll
+      for (int k8 = 0; k8 < 4; ++k8)
+        *reinterpret_cast<uint4*>(sm + KA_PT + ptx::sw128_chunk(r, 4 * ch + k8)) = pack8(x + 8 * k8);
+    }
+  } else {
     const int qd = warp & 3, ch = warp >> 2;
     const int rho = 32 * qd + lane;
     const bool isK = rho < 64;
@@ -559,21 +629,23 @@ __global__ void __launch_bounds__(256, 2)
       }
       __syncthreads();
     }
-    // bf16 T (K-major [64 r][64 j]); blocks above the diagonal are zero
+    // bf16 T diag(beta) (K-major [64 r][64 j]); blocks above the diagonal are zero
     for (int idx = tid; idx < 512; idx += 256) {
       const int rr = idx >> 3, k8 = idx & 7;
       float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if ((k8 >> 1) <= (rr >> 4)) {
         const float4 t0 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8);
         const float4 t1 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8 + 4);
-        y[0] = t0.x; y[1] = t0.y; y[2] = t0.z; y[3] = t0.w;
-        y[4] = t1.x; y[5] = t1.y; y[6] = t1.z; y[7] = t1.w;
+        const float4 b0 = *reinterpret_cast<const float4*>(s_beta + 8 * k8);
+        const float4 b1 = *reinterpret_cast<const float4*>(s_beta + 8 * k8 + 4);
+        y[0] = t0.x * b0.x; y[1] = t0.y * b0.y; y[2] = t0.z * b0.z; y[3] = t0.w * b0.w;
+        y[4] = t1.x * b1.x; y[5] = t1.y * b1.y; y[6] = t1.z * b1.z; y[7] = t1.w * b1.w;
       }
       *reinterpret_cast<uint4*>(sm + KA_TT + ptx::sw128_chunk(rr, k8)) = pack8(y);
     }
   }
 
-  // ---- 6. W^T = (beta K e^G)^T T^T, U^T = (beta V)^T T^T : M=128, N=64, K=64
+  // ---- 6. W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
@@ -583,7 +655,10 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       const uint64_t bd = ptx::sdesc_sw128(sb + KA_TT + kk * 32, 16, 1024);
-      ptx::mma_bf16(tmem + 0, ptx::sdesc_sw128(sb + KA_XK + kk * 2048, 8192, 1024), bd, id, kk > 0);
+      // K o e^G: the K part of L3 (panel stride 16 KB) on the single-reference path
+      const uint64_t xd = fast ? ptx::sdesc_sw128(sb + KA_L3 + kk * 2048, 16384, 1024)
+                               : ptx::sdesc_sw128(sb + KA_XK + kk * 2048, 8192, 1024);
+      ptx::mma_bf16(tmem + 0, xd, bd, id, kk > 0);
       ptx::mma_bf16(tmem + 64, ptx::sdesc_sw128(sb + KA_BV + kk * 2048, 8192, 1024), bd, id, kk > 0);
     }
     ptx::mma_commit(&s_bar);

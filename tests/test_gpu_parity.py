@@ -94,6 +94,34 @@ def test_prefill_split_invariance(cuda_device):
     compare_units(inp, o, S, [(0, h) for h in range(4)], 1e-2)
 
 
+@pytest.mark.parametrize("g_rate", [1.2, 1.3])
+def test_prefill_tc_chunk_decay_range_edges(cuda_device, g_rate):
+    """Per-token log-decay close to -g_rate on every channel: a full 64-token
+    chunk decays by about -76.8 (inside the single-reference range of the
+    tensor-core path, factors up to e^76.8) or -83.2 (outside it: the chunk
+    takes the 16-token block references).  T = 200 ends in an 8-token chunk
+    that decays by ~-10, so the -83.2 case mixes both forms in one launch."""
+    inp = W.make_prefill(2, 200, 4, 128, 128, "bf16", -3.0, 1.0, 0.05, seed=21, device=cuda_device)
+    gen = torch.Generator(device=cuda_device).manual_seed(22)
+    u = torch.rand(inp["g"].shape, generator=gen, device=cuda_device)
+    inp["g"] = (-g_rate * (1.0 - 0.005 * u)).contiguous()
+    o, S = _run_prefill(inp, 64)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    compare_units(inp, o, S, [(n, h) for n in range(2) for h in range(4)], 1e-2)
+
+
+def test_prefill_tc_steep_random_decay(cuda_device):
+    """Random steep gates (log-decay about -2 per token, up to -2.7): every
+    full chunk of the tensor-core path takes the block-reference form."""
+    inp = W.make_prefill(2, 300, 4, 128, 128, "bf16", 1.8, 0.2, 0.05, seed=23, device=cuda_device)
+    assert float(inp["g"].min()) > -5.0
+    o, S = _run_prefill(inp, 64)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    compare_units(inp, o, S, [(n, h) for n in range(2) for h in range(4)], 1e-2)
+
+
 # ------------------------------------------------------------ prefill, full size
 def test_prefill_h16_full(cuda_device):
     """bf16 B1 H16 T4096 d128, random initial state: all 16 units."""
