@@ -64,8 +64,11 @@ constexpr uint32_t IMG_BYTES = 74240;
 // bytes [0, 8K) and [16K, 24K); the Q part fills [8K, 16K) and [24K, 32K).
 constexpr uint32_t KA_L3 = 0;       // [K a; Q a]  K-major [128][128] (2 K-panels)  32768
 constexpr uint32_t KA_RB = 32768;   // right operands K-major [160][128]          40960
-constexpr uint32_t KA_PT = 8192;    // after the first MMA: P bf16 K-major (Q part of panel 0) 8192
-constexpr uint32_t KA_TT = 24576;   //                      T diag(beta) bf16 (Q part of panel 1) 8192
+constexpr uint32_t KA_TT = 8192;    // after the first MMA: T diag(beta) bf16 (Q part of panel 0) 8192
+constexpr uint32_t KA_PT = 24576;   //                      P bf16 K-major (Q part of panel 1)  8192
+// P, U^T and W^T are staged at KA_PT .. KA_PT + 40960 (U^T and W^T over A and T,
+// after the second MMA) in image order and leave in one bulk store.
+constexpr uint32_t KA_IMG_STAGE = KA_PT;
 constexpr uint32_t KA_AS = 32768;   //                      A fp32 [64][68] (over RB)  17408
 constexpr uint32_t KA_XK = 73728;   // K o e^G  MN-major 2 panels [64][64] (block path) 16384
 constexpr uint32_t KA_BV = 90112;   // V        MN-major 2 panels [64][64]       16384
@@ -368,6 +371,9 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
     for (int e = 0; e < 8; ++e) steep |= (J == 3) && !(G[3][e] >= kChunkRefMinG);
   }
+  // The previous item's image bulk store has read its staging area before the
+  // builder below overwrites it.
+  if (tid == 0) ptx::bulk_wait_read0();
   // G is non-increasing (g <= 0), so G at the chunk's last row is each channel's minimum.
   const bool fast = !__syncthreads_or(steep);
 
@@ -382,13 +388,21 @@ __global__ void __launch_bounds__(256, 2)
     uint8_t* l3 = sm + KA_L3 + kp * 16384;
     uint8_t* rb = sm + KA_RB + kp * 20480;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int r = 4 * rg + u;
-      uint32_t kr4[4], qr4[4], vr4[4];
-      ptx::tmem_ld4u(stash + 4 * u, kr4);
-      ptx::tmem_ld4u(stash + 16 + 4 * u, qr4);
-      ptx::tmem_ld4u(stash + 32 + 4 * u, vr4);
+    for (int up = 0; up < 2; ++up) {  // two rows per TMEM round trip
+      uint32_t kr2[2][4], qr2[2][4], vr2[2][4];
+#pragma unroll
+      for (int uu = 0; uu < 2; ++uu) {
+        ptx::tmem_ld4u(stash + 4 * (2 * up + uu), kr2[uu]);
+        ptx::tmem_ld4u(stash + 16 + 4 * (2 * up + uu), qr2[uu]);
+        ptx::tmem_ld4u(stash + 32 + 4 * (2 * up + uu), vr2[uu]);
+      }
       ptx::tmem_wait_ld();
+#pragma unroll
+      for (int uu = 0; uu < 2; ++uu) {
+      const int u = 2 * up + uu, r = 4 * rg + u;
+      const uint32_t* kr4 = kr2[uu];
+      const uint32_t* qr4 = qr2[uu];
+      const uint32_t* vr4 = vr2[uu];
       float kv[8], qv[8];
       unpack8(make_uint4(kr4[0], kr4[1], kr4[2], kr4[3]), kv);
       unpack8(make_uint4(qr4[0], qr4[1], qr4[2], qr4[3]), qv);
@@ -410,6 +424,7 @@ __global__ void __launch_bounds__(256, 2)
       *reinterpret_cast<uint4*>(img + IMG_KB + kp * 8192 + ptx::sw128_chunk(r, ck)) = pack8(o_kb);
       *reinterpret_cast<uint4*>(sm + KA_BV + kp * 8192 + ptx::sw128_chunk(r, ck)) =
           make_uint4(vr4[0], vr4[1], vr4[2], vr4[3]);
+      }
     }
   } else {
     float Gb[8], GeJ[8], eGb[8], invD[8], lam[8], sig1[8], sig2[8];
@@ -663,8 +678,6 @@ __global__ void __launch_bounds__(256, 2)
     }
     ptx::mma_commit(&s_bar);
   }
-  for (int i2 = tid; i2 < 512; i2 += 256)
-    reinterpret_cast<uint4*>(img + IMG_P)[i2] = reinterpret_cast<const uint4*>(sm + KA_PT)[i2];
   ptx::mbar_wait_bounded(&s_bar, 1);  // second completion of this item
   ptx::tc_fence_after();
   {
@@ -681,18 +694,20 @@ __global__ void __launch_bounds__(256, 2)
       for (int k8 = 0; k8 < 4; ++k8) {
         const uint4 pk = pack8(x + 8 * k8);
         const uint32_t off = ptx::sw128_chunk(row, 4 * hh + k8);
-        if (ch == 0) {
-          *reinterpret_cast<uint4*>(img + IMG_A1 + off) = pk;
-        } else {
-          *reinterpret_cast<uint4*>(img + IMG_U + off) = pk;
-        }
+        *reinterpret_cast<uint4*>(sm + KA_IMG_STAGE + (ch == 0 ? IMG_A1 : IMG_U) + off) = pk;
       }
     }
   }
 
+  ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();  // every TMEM read of this item is done before the next item's stash
+  if (tid == 0) {
+    ptx::bulk_s2g(img + IMG_P, sm + KA_IMG_STAGE, IMG_A1 + 16384 - IMG_P);
+    ptx::bulk_commit();
+  }
   }  // item loop
+  if (tid == 0) ptx::bulk_wait0();
   if (warp == 0) ptx::tmem_dealloc(tmem, 256);
 }
 
