@@ -5,7 +5,8 @@ Headline: chunkwise prefill tokens/s on B=8, H=32, T=8192, dk=dv=128 (bf16
 q/k/v, fp32 gates and state), one prefill call per step, inputs resident in
 HBM (2.7 GB of inputs: larger than the 126 MB L2, so no flush is needed).
 Beside it: the recurrent decode (256 sequences x 32 heads, in-place fp32
-state, one token per step) as state GB/s, the roofline fractions, the fp64
+state, one token per step) as state GB/s, the Gated DeltaNet variant (one
+gate per token and head) on both shapes, the roofline fractions, the fp64
 CPU oracle timed on this host's cores, and an end-to-end figure through the
 public host-buffer API (pinned host -> device copies, prefill, copies back).
 
@@ -44,6 +45,9 @@ PREFILL_FLOPS_PER_TOKEN_HEAD = 6 * 128 * 128 + 2 * 64 * (3 * 128 + 2 * 128)
 STATE_BYTES = 128 * 128 * 4
 # decode: state read + write, q, k, v, o bf16, g fp32, beta fp32 per head-step
 DECODE_BYTES_PER_HEAD_STEP = 2 * STATE_BYTES + 3 * 256 + 512 + 4 + 256
+# Gated DeltaNet (one fp32 gate per token-head instead of dk)
+GDN_PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 256 + 4 + 4 + 256
+GDN_DECODE_BYTES_PER_HEAD_STEP = 2 * STATE_BYTES + 3 * 256 + 4 + 4 + 256
 
 
 def profiled_traffic(kernel, unit_key):
@@ -226,6 +230,70 @@ def time_launches(fn, steps, stream):
     return start.elapsed_time(end) / steps
 
 
+def gdn_leg(kda, args, world, dev, stream, peaks):
+    """Gated DeltaNet on the headline prefill shape and the decode shape."""
+    w = W.GDN_PREFILL_B8
+    inp = W.make_workload(w, dev)
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(kda.workspace_size(B, T, H, dk, dv, 0, w.chunk, torch.bfloat16), 1),
+                     dtype=torch.uint8, device=dev)
+
+    def prefill():
+        kda.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], None, w.chunk,
+                          o=o, S_out=S_out, workspace=ws)
+
+    for _ in range(args.warmup):
+        prefill()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(time_launches(prefill, args.steps, stream), world, dev)
+    kernel_ms = kda.profile_chunk_fwd(prefill, stream, repeats=max(1, min(args.steps, 5)), dk=dk, dv=dv,
+                                      chunk_size=w.chunk)
+    token_heads = B * T * H
+    dom_name, dom_ms = max(kernel_ms.items(), key=lambda kv: kv[1])
+    dom_bytes = kda.algorithmic_bytes_per_launch(dom_name, token_heads, B * H, d=dk, gate_per_channel=False)
+    dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
+    alg_bytes = token_heads * GDN_PREFILL_BYTES_PER_TOKEN_HEAD + B * H * STATE_BYTES
+    prefill_line = {"workload": w.name, "value": world * B * T / (ms * 1e-3), "unit": "tokens/s",
+                    "ms_per_step": ms, "kernel_ms": kernel_ms,
+                    "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": dom_gbs,
+                                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dom_gbs / peaks["hbm_gbs"],
+                                 "alg_bytes_per_launch": dom_bytes, "traffic": None},
+                    "whole_call_hbm_frac": alg_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del inp, o, S_out, ws
+    torch.cuda.empty_cache()
+
+    dw = W.GDN_DECODE
+    N, Hd, dd = dw.B, dw.H, dw.dk
+    S = W.make_decode_state(N, Hd, dd, dd, dw.s0_std, seed=dw.seed, device=dev)
+    xs = W.make_decode_steps(N, Hd, dd, dd, dw.T, dw.dtype, dw.g_mu, dw.g_sigma, seed=dw.seed,
+                             device=dev, scalar_gate=True)
+    od = torch.empty((N, Hd, dd), dtype=torch.bfloat16, device=dev)
+    step = [0]
+
+    def decode_step():
+        t = step[0] % dw.T
+        kda.gdn_recurrent_step(xs["q"][t], xs["k"][t], xs["v"][t], xs["g"][t], xs["beta"][t], S, o=od)
+        step[0] += 1
+
+    for _ in range(16):
+        decode_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    dec_ms = max_over_ranks(time_launches(decode_step, dw.T, stream), world, dev)
+    heads = N * Hd
+    dec_gbs = heads * GDN_DECODE_BYTES_PER_HEAD_STEP / (dec_ms * 1e-3) / 1e9
+    decode_line = {"workload": dw.name, "value": world * heads * 2 * STATE_BYTES / (dec_ms * 1e-3) / 1e9,
+                   "unit": "GB/s (state read+write)", "us_per_step": dec_ms * 1e3,
+                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": dec_gbs / peaks["hbm_gbs"], "kernel": "kda_decode_step_kernel"}}
+    del S, xs, od
+    torch.cuda.empty_cache()
+    return {"prefill": prefill_line, "decode": decode_line}
+
+
 def run_ours(args):
     import kimi_delta_attention_31_b200 as kda
     rank, world, local = dist_setup(args.gpus)
@@ -340,6 +408,9 @@ def run_ours(args):
     del S, xs, od
     torch.cuda.empty_cache()
 
+    # ---------------- Gated DeltaNet (scalar gate) ----------------
+    gdn = gdn_leg(kda, args, world, dev, stream, peaks)
+
     # ---------------- CPU oracle baseline (rank 0, N = 1 only) ----------------
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -354,7 +425,7 @@ def run_ours(args):
                        "chunk": w.chunk, "g": f"-softplus(N({w.g_mu},{w.g_sigma}))",
                        "l2": "inputs (2.7 GB) larger than L2; no flush",
                        "parallelism": f"dp{world} (independent batches per GPU)"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "gdn": gdn,
             "gpu_launches": gpu_launches, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)

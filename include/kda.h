@@ -22,8 +22,10 @@
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers, row-major, densely packed.
  *     Alignment: kda_chunk_fwd needs 16-byte aligned q, k, v, g, o, S0, S_out
- *     and workspace and 4-byte aligned beta and cu_seqlens; kda_recurrent_step
- *     needs a 16-byte aligned S and element-aligned q, k, v, o, g, beta.  The caller owns every buffer and the stream; the
+ *     and workspace and 4-byte aligned beta and cu_seqlens (kda_gdn_chunk_fwd:
+ *     the same, with a 4-byte aligned g); kda_recurrent_step and
+ *     kda_gdn_recurrent_step need a 16-byte aligned S and element-aligned q, k,
+ *     v, o, g, beta.  The caller owns every buffer and the stream; the
  *     library never allocates, frees or synchronises (except
  *     kda_device_error, which synchronises the given stream by design).
  *   - Calls are asynchronous on `stream`.  The return value reports argument
@@ -93,7 +95,10 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
  * Numerics: the tensor-core path takes bf16 operands with fp32 accumulation
  * and an fp32 state; it is exact (no overflow) as long as every key channel's
  * log-decay over any 16 consecutive tokens of a chunk is >= -80 (implied by
- * per-token log alpha >= -5).  The fp32 path has no such restriction.
+ * per-token log alpha >= -5).  Chunks whose every channel decays by no more
+ * than 80 over the whole chunk use one decay reference per chunk, the others
+ * one per 16-token block; both give the same result up to rounding.  The fp32
+ * path has no such restriction.
  */
 kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, const float* S0, void* o, float* S_out,
@@ -114,6 +119,29 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
 kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, float* S, void* o, int N, int H, int dk,
                                 int dv, kda_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * Gated DeltaNet: the same recurrence with one decay per token and head
+ * instead of one per key channel, alpha_t a scalar ("Kimi K3 notes 1: KDA"
+ * section 3; "Linear / sparse attention" tutorial section 5.2).  It is KDA
+ * with every key channel's gate equal, and runs the same kernels with g
+ * broadcast over dk.
+ *
+ * kda_gdn_chunk_fwd: arguments as kda_chunk_fwd except
+ *   g : [B, T, H] fp32, log alpha <= 0, 4-byte aligned.
+ * It takes the same workspace (kda_chunk_fwd_workspace_size), chunk sizes,
+ * paths and exactness domain (log alpha over any 16 tokens >= -80).
+ * kda_gdn_recurrent_step: arguments as kda_recurrent_step except
+ *   g : [N, H] fp32.
+ */
+kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* S0, void* o, float* S_out,
+                               const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
+                               int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+kda_status_t kda_gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                                    const float* beta, float* S, void* o, int N, int H, int dk,
+                                    int dv, kda_dtype_t dtype, cudaStream_t stream);
 
 /*
  * kda_chunk_fwd for callers that cannot allocate device memory: the same
@@ -158,8 +186,8 @@ kda_status_t kda_device_error(int* code, cudaStream_t stream);
 int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype);
 
 /*
- * Measurement hook.  While set (events != NULL), each later kda_chunk_fwd
- * call made by the calling thread records events[0] before its first kernel
+ * Measurement hook.  While set (events != NULL), each later kda_chunk_fwd or
+ * kda_gdn_chunk_fwd call made by the calling thread records events[0] before its first kernel
  * launch and events[i] after its i-th launch, on the call's stream; count
  * must be at least kda_chunk_fwd_launches(...) + 1 or the call fails with
  * KDA_ERR_INVALID_ARG.  The caller owns the events.  Pass NULL, 0 to stop.

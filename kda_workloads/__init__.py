@@ -10,7 +10,8 @@ each workload's definition, not of the method) is:
   vectors), then rounded to the workload dtype;
 * v ~ N(0, 1), rounded to the workload dtype;
 * beta = sigmoid(N(0, 1)) in fp32 (a write strength in (0, 1));
-* g = log(alpha) = -softplus(N(mu, sigma)) in fp32 (alpha in (0, 1));
+* g = log(alpha) = -softplus(N(mu, sigma)) in fp32 (alpha in (0, 1)), one per
+  key channel, or one per token and head for the Gated DeltaNet workloads;
 * S0 ~ N(0, s0_std^2) in fp32, or zeros.
 
 Draw order is q, k, v, beta-logit, alpha-logit, S0 from one torch generator
@@ -42,6 +43,7 @@ class Workload:
     chunk: int
     seed: int
     lengths: Optional[tuple] = None  # packed varlen sequence lengths (B == 1)
+    scalar_gate: bool = False  # Gated DeltaNet: g is [B, T, H] (one gate per token and head)
 
     @property
     def tokens(self) -> int:
@@ -79,8 +81,14 @@ PREFILL_VARLEN = Workload("kda_prefill_varlen_bf16_16seq_H32_d128", 1, sum(_VL),
                           -4.0, 1.0, 0.0, 64, 1003, lengths=_VL)
 DECODE = Workload("kda_decode_bf16_N256_H32_d128_1024steps", 256, 1024, 32, 128, 128, "bf16",
                   -3.0, 1.0, 0.02, 1, 1004)
+# Gated DeltaNet (scalar gate) on the shapes of the prefill headline and of decode.
+GDN_PREFILL_B8 = Workload("gdn_prefill_bf16_B8_H32_T8192_d128", 8, 8192, 32, 128, 128, "bf16",
+                          -5.0, 1.5, 0.0, 64, 1005, scalar_gate=True)
+GDN_DECODE = Workload("gdn_decode_bf16_N256_H32_d128_1024steps", 256, 1024, 32, 128, 128, "bf16",
+                      -3.0, 1.0, 0.02, 1, 1006, scalar_gate=True)
 
-WORKLOADS = {w.name: w for w in (ORACLE_SMALL, PREFILL_H16, PREFILL_B8, PREFILL_VARLEN, DECODE)}
+WORKLOADS = {w.name: w for w in (ORACLE_SMALL, PREFILL_H16, PREFILL_B8, PREFILL_VARLEN, DECODE,
+                                 GDN_PREFILL_B8, GDN_DECODE)}
 
 
 def cu_seqlens_of(lengths, device="cpu") -> torch.Tensor:
@@ -96,9 +104,10 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
 
 
 def make_prefill(B, T, H, dk, dv, dtype="bf16", g_mu=-4.0, g_sigma=1.0, s0_std=0.0,
-                 seed=0, device="cpu", lengths=None, normalize_qk=True) -> dict:
+                 seed=0, device="cpu", lengths=None, normalize_qk=True, scalar_gate=False) -> dict:
     """Prefill inputs.  With ``lengths`` the layout is packed (B must be 1,
-    T = sum(lengths)) and ``cu_seqlens`` (int32) is included."""
+    T = sum(lengths)) and ``cu_seqlens`` (int32) is included.  With
+    ``scalar_gate`` g is [B, T, H] (Gated DeltaNet) instead of [B, T, H, dk]."""
     if lengths is not None:
         assert B == 1 and T == sum(lengths)
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -109,7 +118,8 @@ def make_prefill(B, T, H, dk, dv, dtype="bf16", g_mu=-4.0, g_sigma=1.0, s0_std=0
     k = torch.randn(shp_k, generator=gen, device=device, dtype=torch.float32)
     v = torch.randn(shp_v, generator=gen, device=device, dtype=torch.float32)
     b_logit = torch.randn((B, T, H), generator=gen, device=device, dtype=torch.float32)
-    a_logit = torch.randn(shp_k, generator=gen, device=device, dtype=torch.float32)
+    a_logit = torch.randn((B, T, H) if scalar_gate else shp_k, generator=gen, device=device,
+                          dtype=torch.float32)
     N = len(lengths) if lengths is not None else B
     if s0_std > 0:
         S0 = torch.randn((N, H, dk, dv), generator=gen, device=device, dtype=torch.float32) * s0_std
@@ -133,7 +143,7 @@ def make_prefill(B, T, H, dk, dv, dtype="bf16", g_mu=-4.0, g_sigma=1.0, s0_std=0
 
 def make_workload(w: Workload, device="cpu") -> dict:
     return make_prefill(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.g_mu, w.g_sigma, w.s0_std,
-                        w.seed, device, lengths=w.lengths)
+                        w.seed, device, lengths=w.lengths, scalar_gate=w.scalar_gate)
 
 
 def make_decode_state(N, H, dk, dv, s0_std=0.02, seed=0, device="cpu") -> torch.Tensor:
@@ -142,16 +152,17 @@ def make_decode_state(N, H, dk, dv, s0_std=0.02, seed=0, device="cpu") -> torch.
 
 
 def make_decode_steps(N, H, dk, dv, steps, dtype="bf16", g_mu=-3.0, g_sigma=1.0, seed=0,
-                      device="cpu") -> dict:
+                      device="cpu", scalar_gate=False) -> dict:
     """``steps`` consecutive single-token inputs: q, k, g [steps,N,H,dk], v [steps,N,H,dv],
-    beta [steps,N,H]; q and k unit-norm per (step, seq, head)."""
+    beta [steps,N,H]; q and k unit-norm per (step, seq, head).  With
+    ``scalar_gate`` g is [steps,N,H] (Gated DeltaNet)."""
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     gen = torch.Generator(device=device).manual_seed(seed + 7919)
     q = _unit_rows(torch.randn((steps, N, H, dk), generator=gen, device=device))
     k = _unit_rows(torch.randn((steps, N, H, dk), generator=gen, device=device))
     v = torch.randn((steps, N, H, dv), generator=gen, device=device)
     b_logit = torch.randn((steps, N, H), generator=gen, device=device)
-    a_logit = torch.randn((steps, N, H, dk), generator=gen, device=device)
+    a_logit = torch.randn((steps, N, H) if scalar_gate else (steps, N, H, dk), generator=gen, device=device)
     return dict(q=q.to(tdt).contiguous(), k=k.to(tdt).contiguous(), v=v.to(tdt).contiguous(),
                 beta=torch.sigmoid(b_logit).contiguous(),
                 g=(-F.softplus(a_logit * g_sigma + g_mu)).contiguous())
@@ -163,10 +174,11 @@ def bytes_of(*tensors) -> int:
 
 def describe(w: Workload) -> str:
     sl = f", lengths={list(w.lengths)}" if w.lengths else ""
+    gate = " per token and head" if w.scalar_gate else " per key channel"
     return (f"{w.name}: B={w.B} T={w.T} H={w.H} dk={w.dk} dv={w.dv} {w.dtype}; "
-            f"log alpha=-softplus(N({w.g_mu},{w.g_sigma})); S0 std={w.s0_std}; C={w.chunk}{sl}")
+            f"log alpha=-softplus(N({w.g_mu},{w.g_sigma})){gate}; S0 std={w.s0_std}; C={w.chunk}{sl}")
 
 
 __all__ = ["Workload", "WORKLOADS", "ORACLE_SMALL", "PREFILL_H16", "PREFILL_B8", "PREFILL_VARLEN",
-           "DECODE", "make_prefill", "make_workload", "make_decode_state", "make_decode_steps",
+           "DECODE", "GDN_PREFILL_B8", "GDN_DECODE", "make_prefill", "make_workload", "make_decode_state", "make_decode_steps",
            "cu_seqlens_of", "varlen_lengths", "bytes_of", "describe"]

@@ -36,7 +36,7 @@ KDA_BF16, KDA_F32 = 0, 1
 # Every symbol include/kda.h declares (checked by the CPU test-suite).
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_last_error", "kda_device_error", "kda_chunk_fwd_launches", "kda_profile_events",
-            "kda_version", "kda_chunk_fwd_noalloc")
+            "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -75,6 +75,10 @@ def load_library():
         lib.kda_chunk_fwd.restype = i32
         lib.kda_recurrent_step.argtypes = [vp] * 7 + [i32] * 5 + [vp]
         lib.kda_recurrent_step.restype = i32
+        lib.kda_gdn_chunk_fwd.argtypes = lib.kda_chunk_fwd.argtypes
+        lib.kda_gdn_chunk_fwd.restype = i32
+        lib.kda_gdn_recurrent_step.argtypes = lib.kda_recurrent_step.argtypes
+        lib.kda_gdn_recurrent_step.restype = i32
         lib.kda_last_error.argtypes = []
         lib.kda_last_error.restype = ctypes.c_char_p
         lib.kda_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), vp]
@@ -135,6 +139,20 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, output_
     """Chunkwise KDA prefill.  q, k, g: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H];
     S0: [N,H,dk,dv] fp32 or None; cu_seqlens: int32 [N+1] (B == 1) or None.
     Returns (o, S_out) with S_out None when output_final_state is False."""
+    return _chunk_fwd("kda_chunk_fwd", q, k, v, g, beta, S0, cu_seqlens, chunk_size, output_final_state,
+                      o, S_out, workspace)
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, output_final_state=True,
+                  o=None, S_out=None, workspace=None):
+    """Gated DeltaNet prefill: as chunk_fwd with one gate per token and head,
+    g: [B,T,H] fp32 (log alpha)."""
+    return _chunk_fwd("kda_gdn_chunk_fwd", q, k, v, g, beta, S0, cu_seqlens, chunk_size,
+                      output_final_state, o, S_out, workspace)
+
+
+def _chunk_fwd(fn, q, k, v, g, beta, S0, cu_seqlens, chunk_size, output_final_state, o, S_out,
+               workspace):
     lib = load_library()
     _need_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_out, workspace)
     B, T, H, dk = q.shape
@@ -143,6 +161,9 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, output_
     N = num_seqs if cu_seqlens is not None else B
     if g.dtype != torch.float32 or beta.dtype != torch.float32:
         raise TypeError("g and beta must be float32")
+    g_shape = (B, T, H) if fn == "kda_gdn_chunk_fwd" else (B, T, H, dk)
+    if tuple(g.shape) != g_shape or tuple(beta.shape) != (B, T, H):
+        raise ValueError(f"g must be {g_shape} and beta {(B, T, H)}, got {tuple(g.shape)}, {tuple(beta.shape)}")
     if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
         raise TypeError("cu_seqlens must be int32")
     if o is None:
@@ -153,9 +174,9 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, output_
     if workspace is None and ws_need:
         workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                           _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
-                           _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(q.device))
+    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                          _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
+                          _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(q.device))
     _check(st)
     return o, S_out
 
@@ -184,16 +205,28 @@ def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64,
 def recurrent_step(q, k, v, g, beta, S, o=None):
     """One decode token per sequence: q, k, g [N,H,dk]; v [N,H,dv]; beta [N,H];
     S [N,H,dk,dv] fp32 updated in place.  Returns o [N,H,dv]."""
+    return _recurrent_step("kda_recurrent_step", q, k, v, g, beta, S, o)
+
+
+def gdn_recurrent_step(q, k, v, g, beta, S, o=None):
+    """Gated DeltaNet decode step: as recurrent_step with g [N,H] fp32."""
+    return _recurrent_step("kda_gdn_recurrent_step", q, k, v, g, beta, S, o)
+
+
+def _recurrent_step(fn, q, k, v, g, beta, S, o):
     lib = load_library()
     _need_cuda(q, k, v, g, beta, S, o)
     N, H, dk = q.shape
     dv = v.shape[-1]
     if S.dtype != torch.float32 or g.dtype != torch.float32 or beta.dtype != torch.float32:
         raise TypeError("S, g and beta must be float32")
+    g_shape = (N, H) if fn == "kda_gdn_recurrent_step" else (N, H, dk)
+    if tuple(g.shape) != g_shape or tuple(beta.shape) != (N, H) or tuple(S.shape) != (N, H, dk, dv):
+        raise ValueError(f"g must be {g_shape}, beta {(N, H)}, S {(N, H, dk, dv)}")
     if o is None:
         o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
-    st = lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
-                                N, H, dk, dv, _dtype_code(q), _stream_handle(q.device))
+    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                          N, H, dk, dv, _dtype_code(q), _stream_handle(q.device))
     _check(st)
     return o
 
@@ -295,12 +328,16 @@ def profile_chunk_fwd(call, stream, repeats=3, dk=128, dv=128, chunk_size=64, dt
 TC_IMAGE_BYTES_PER_TOKEN_HEAD = 1160
 
 
-def algorithmic_bytes_per_launch(kernel, token_heads, units, d=128, with_state_in=False):
+def algorithmic_bytes_per_launch(kernel, token_heads, units, d=128, with_state_in=False,
+                                 gate_per_channel=True):
+    """Bytes one launch must move.  The gate is fp32, d values per token-head
+    (KDA) or one (Gated DeltaNet, gate_per_channel=False)."""
     state = d * d * 4 * units
+    gate = 4 * d if gate_per_channel else 4
     if kernel == "kda_chunk_simt_kernel":
-        return token_heads * (3 * 2 * d + 4 * d + 4 + 2 * d) + state * (2 if with_state_in else 1)
+        return token_heads * (3 * 2 * d + gate + 4 + 2 * d) + state * (2 if with_state_in else 1)
     if kernel == "kda_tc_chunk_local_kernel":
-        return token_heads * (3 * 2 * d + 4 * d + 4 + TC_IMAGE_BYTES_PER_TOKEN_HEAD)
+        return token_heads * (3 * 2 * d + gate + 4 + TC_IMAGE_BYTES_PER_TOKEN_HEAD)
     if kernel == "kda_tc_state_pass_kernel":
         return token_heads * (TC_IMAGE_BYTES_PER_TOKEN_HEAD + 2 * d) + state * (2 if with_state_in else 1)
     raise KeyError(kernel)

@@ -47,11 +47,11 @@ template <typename TIn>
 cudaError_t dispatch_chunk_simt(int dk, int C, const void* q, const void* k, const void* v,
                                 const float* g, const float* beta, const float* S0, void* o,
                                 float* S_out, const int32_t* cu, int N, int T, int H, int dv,
-                                cudaStream_t st) {
+                                int gpc, cudaStream_t st) {
 #define KDA_SIMT_CASE(D, CC)                                                                  \
   if (dk == D && C == CC)                                                                     \
     return kda::launch_chunk_simt<TIn, D, CC>(q, k, v, g, beta, S0, o, S_out, cu, N, T, H, dv, \
-                                               st);
+                                               gpc, st);
   KDA_SIMT_CASE(32, 16) KDA_SIMT_CASE(32, 32) KDA_SIMT_CASE(32, 64)
   KDA_SIMT_CASE(64, 16) KDA_SIMT_CASE(64, 32) KDA_SIMT_CASE(64, 64)
   KDA_SIMT_CASE(128, 16) KDA_SIMT_CASE(128, 32) KDA_SIMT_CASE(128, 64)
@@ -61,12 +61,109 @@ cudaError_t dispatch_chunk_simt(int dk, int C, const void* q, const void* k, con
 
 template <typename TIn>
 cudaError_t dispatch_decode(int dk, const void* q, const void* k, const void* v, const float* g,
-                            const float* beta, float* S, void* o, int N, int H,
+                            const float* beta, float* S, void* o, int N, int H, int gpc,
                             cudaStream_t st) {
-  if (dk == 32) return kda::launch_decode_step<TIn, 32, 32>(q, k, v, g, beta, S, o, N, H, st);
-  if (dk == 64) return kda::launch_decode_step<TIn, 64, 64>(q, k, v, g, beta, S, o, N, H, st);
-  if (dk == 128) return kda::launch_decode_step<TIn, 128, 128>(q, k, v, g, beta, S, o, N, H, st);
+  if (dk == 32) return kda::launch_decode_step<TIn, 32, 32>(q, k, v, g, beta, S, o, N, H, gpc, st);
+  if (dk == 64) return kda::launch_decode_step<TIn, 64, 64>(q, k, v, g, beta, S, o, N, H, gpc, st);
+  if (dk == 128) return kda::launch_decode_step<TIn, 128, 128>(q, k, v, g, beta, S, o, N, H, gpc, st);
   return cudaErrorInvalidValue;
+}
+
+// gpc: g holds one gate per key channel ([.., H, dk], KDA) or one per token
+// and head ([.., H], Gated DeltaNet).
+kda_status_t chunk_fwd_impl(const char* fn, const void* q, const void* k, const void* v,
+                            const float* g, const float* beta, const float* S0, void* o,
+                            float* S_out, const int32_t* cu_seqlens, int num_seqs, int B, int T,
+                            int H, int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                            void* workspace, size_t workspace_bytes, int gpc,
+                            cudaStream_t stream) {
+  t_err[0] = 0;
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0)
+    return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes B=%d T=%d H=%d num_seqs=%d", fn, B,
+                T, H, num_seqs);
+  if (dtype != KDA_BF16 && dtype != KDA_F32)
+    return fail(KDA_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, (int)dtype);
+  if (!supported_head(dk, dv))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: dk=%d dv=%d (need dk == dv in {32,64,128})", fn,
+                dk, dv);
+  if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64)
+    return fail(KDA_ERR_UNSUPPORTED, "%s: chunk_size=%d (need 16, 32 or 64)", fn,
+                chunk_size);
+  if (cu_seqlens) {
+    if (B != 1) return fail(KDA_ERR_INVALID_ARG, "%s: packed inputs need B == 1", fn);
+    if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "%s: cu_seqlens needs num_seqs >= 1", fn);
+  } else if (num_seqs != 0) {
+    return fail(KDA_ERR_INVALID_ARG, "%s: num_seqs=%d without cu_seqlens", fn, num_seqs);
+  }
+  const int N = cu_seqlens ? num_seqs : B;
+  const long long tokens = (long long)B * T;
+  if (N == 0) return KDA_OK;
+  if (tokens > 0 && (!q || !k || !v || !g || !beta || !o))
+    return fail(KDA_ERR_INVALID_ARG, "%s: null input/output pointer", fn);
+  const void* ptrs[] = {q, k, v, gpc ? g : nullptr, S0, o, S_out, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
+  if ((beta && !aligned_to(beta, 4)) || (cu_seqlens && !aligned_to(cu_seqlens, 4)) ||
+      (g && !aligned_to(g, 4)))
+    return fail(KDA_ERR_ALIGNMENT, "%s: beta / cu_seqlens / g not 4-byte aligned", fn);
+  if (S_out && o && (const void*)S_out == (const void*)o)
+    return fail(KDA_ERR_INVALID_ARG, "%s: o aliases S_out", fn);
+
+  const int launches = kda_chunk_fwd_launches(dk, dv, chunk_size, dtype);
+  cudaEvent_t* ev = t_prof_events;
+  if (ev && t_prof_count < launches + 1)
+    return fail(KDA_ERR_INVALID_ARG, "%s: %d profiling events, need %d", fn, t_prof_count,
+                launches + 1);
+  cudaError_t e;
+  if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return cuda_fail(e, "event record");
+  if (use_tensor_core_path(dk, dv, chunk_size, dtype)) {
+    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
+    if (need && (!workspace || workspace_bytes < need))
+      return fail(KDA_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes,
+                  need);
+    e = kda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
+                             static_cast<const __nv_bfloat16*>(k),
+                             static_cast<const __nv_bfloat16*>(v), g, beta, S0,
+                             static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H,
+                             max_chunks(B, T, num_seqs, chunk_size), workspace, gpc, ev, stream);
+  } else if (dtype == KDA_F32) {
+    e = dispatch_chunk_simt<float>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, T,
+                                   H, dv, gpc, stream);
+  } else {
+    e = dispatch_chunk_simt<__nv_bfloat16>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out,
+                                           cu_seqlens, N, T, H, dv, gpc, stream);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  if (ev && launches == 1 && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess)
+    return cuda_fail(e, "event record");
+  return KDA_OK;
+}
+
+kda_status_t recurrent_step_impl(const char* fn, const void* q, const void* k, const void* v,
+                                const float* g, const float* beta, float* S, void* o, int N, int H,
+                                int dk, int dv, kda_dtype_t dtype, int gpc, cudaStream_t stream) {
+  t_err[0] = 0;
+  if (N < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes N=%d H=%d", fn, N, H);
+  if (dtype != KDA_BF16 && dtype != KDA_F32)
+    return fail(KDA_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, (int)dtype);
+  if (!supported_head(dk, dv))
+    return fail(KDA_ERR_UNSUPPORTED,
+                "%s: dk=%d dv=%d (need dk == dv in {32,64,128})", fn, dk, dv);
+  if (N == 0) return KDA_OK;
+  if (!q || !k || !v || !g || !beta || !S || !o)
+    return fail(KDA_ERR_INVALID_ARG, "%s: null pointer", fn);
+  const unsigned esz = dtype == KDA_F32 ? 4u : 2u;
+  if (!aligned16(S)) return fail(KDA_ERR_ALIGNMENT, "%s: S %p is not 16-byte aligned", fn, (const void*)S);
+  const void* elem[] = {q, k, v, o};
+  for (const void* p : elem)
+    if (!aligned_to(p, esz)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is misaligned", fn, p);
+  if (!aligned_to(g, 4) || !aligned_to(beta, 4))
+    return fail(KDA_ERR_ALIGNMENT, "%s: g / beta not 4-byte aligned", fn);
+  cudaError_t e = dtype == KDA_F32
+                      ? dispatch_decode<float>(dk, q, k, v, g, beta, S, o, N, H, gpc, stream)
+                      : dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, N, H, gpc, stream);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return KDA_OK;
 }
 
 }  // namespace
@@ -102,92 +199,31 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
                            const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
                            int dk, int dv, int chunk_size, kda_dtype_t dtype,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  t_err[0] = 0;
-  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0)
-    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: bad sizes B=%d T=%d H=%d num_seqs=%d", B,
-                T, H, num_seqs);
-  if (dtype != KDA_BF16 && dtype != KDA_F32)
-    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd: unknown dtype %d", (int)dtype);
-  if (!supported_head(dk, dv))
-    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd: dk=%d dv=%d (need dk == dv in {32,64,128})",
-                dk, dv);
-  if (chunk_size != 16 && chunk_size != 32 && chunk_size != 64)
-    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd: chunk_size=%d (need 16, 32 or 64)",
-                chunk_size);
-  if (cu_seqlens) {
-    if (B != 1) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: packed inputs need B == 1");
-    if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: cu_seqlens needs num_seqs >= 1");
-  } else if (num_seqs != 0) {
-    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: num_seqs=%d without cu_seqlens", num_seqs);
-  }
-  const int N = cu_seqlens ? num_seqs : B;
-  const long long tokens = (long long)B * T;
-  if (N == 0) return KDA_OK;
-  if (tokens > 0 && (!q || !k || !v || !g || !beta || !o))
-    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: null input/output pointer");
-  const void* ptrs[] = {q, k, v, g, S0, o, S_out, workspace};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return fail(KDA_ERR_ALIGNMENT, "kda_chunk_fwd: pointer %p is not 16-byte aligned", p);
-  if ((beta && !aligned_to(beta, 4)) || (cu_seqlens && !aligned_to(cu_seqlens, 4)))
-    return fail(KDA_ERR_ALIGNMENT, "kda_chunk_fwd: beta / cu_seqlens not 4-byte aligned");
-  if (S_out && o && (const void*)S_out == (const void*)o)
-    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: o aliases S_out");
+  return chunk_fwd_impl("kda_chunk_fwd", q, k, v, g, beta, S0, o, S_out, cu_seqlens, num_seqs, B, T,
+                        H, dk, dv, chunk_size, dtype, workspace, workspace_bytes, 1, stream);
+}
 
-  const int launches = kda_chunk_fwd_launches(dk, dv, chunk_size, dtype);
-  cudaEvent_t* ev = t_prof_events;
-  if (ev && t_prof_count < launches + 1)
-    return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: %d profiling events, need %d", t_prof_count,
-                launches + 1);
-  cudaError_t e;
-  if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return cuda_fail(e, "event record");
-  if (use_tensor_core_path(dk, dv, chunk_size, dtype)) {
-    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
-    if (need && (!workspace || workspace_bytes < need))
-      return fail(KDA_ERR_WORKSPACE, "kda_chunk_fwd: workspace %zu bytes, need %zu", workspace_bytes,
-                  need);
-    e = kda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
-                             static_cast<const __nv_bfloat16*>(k),
-                             static_cast<const __nv_bfloat16*>(v), g, beta, S0,
-                             static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H,
-                             max_chunks(B, T, num_seqs, chunk_size), workspace, ev, stream);
-  } else if (dtype == KDA_F32) {
-    e = dispatch_chunk_simt<float>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, T,
-                                   H, dv, stream);
-  } else {
-    e = dispatch_chunk_simt<__nv_bfloat16>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out,
-                                           cu_seqlens, N, T, H, dv, stream);
-  }
-  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd launch");
-  if (ev && launches == 1 && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess)
-    return cuda_fail(e, "event record");
-  return KDA_OK;
+kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* S0, void* o, float* S_out,
+                               const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
+                               int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return chunk_fwd_impl("kda_gdn_chunk_fwd", q, k, v, g, beta, S0, o, S_out, cu_seqlens, num_seqs,
+                        B, T, H, dk, dv, chunk_size, dtype, workspace, workspace_bytes, 0, stream);
 }
 
 kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, float* S, void* o, int N, int H, int dk,
                                 int dv, kda_dtype_t dtype, cudaStream_t stream) {
-  t_err[0] = 0;
-  if (N < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_step: bad sizes N=%d H=%d", N, H);
-  if (dtype != KDA_BF16 && dtype != KDA_F32)
-    return fail(KDA_ERR_UNSUPPORTED, "kda_recurrent_step: unknown dtype %d", (int)dtype);
-  if (!supported_head(dk, dv))
-    return fail(KDA_ERR_UNSUPPORTED,
-                "kda_recurrent_step: dk=%d dv=%d (need dk == dv in {32,64,128})", dk, dv);
-  if (N == 0) return KDA_OK;
-  if (!q || !k || !v || !g || !beta || !S || !o)
-    return fail(KDA_ERR_INVALID_ARG, "kda_recurrent_step: null pointer");
-  const unsigned esz = dtype == KDA_F32 ? 4u : 2u;
-  if (!aligned16(S)) return fail(KDA_ERR_ALIGNMENT, "kda_recurrent_step: S %p is not 16-byte aligned", (const void*)S);
-  const void* elem[] = {q, k, v, o};
-  for (const void* p : elem)
-    if (!aligned_to(p, esz)) return fail(KDA_ERR_ALIGNMENT, "kda_recurrent_step: pointer %p is misaligned", p);
-  if (!aligned_to(g, 4) || !aligned_to(beta, 4))
-    return fail(KDA_ERR_ALIGNMENT, "kda_recurrent_step: g / beta not 4-byte aligned");
-  cudaError_t e = dtype == KDA_F32
-                      ? dispatch_decode<float>(dk, q, k, v, g, beta, S, o, N, H, stream)
-                      : dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, N, H, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "kda_recurrent_step launch");
-  return KDA_OK;
+  return recurrent_step_impl("kda_recurrent_step", q, k, v, g, beta, S, o, N, H, dk, dv, dtype, 1,
+                             stream);
+}
+
+kda_status_t kda_gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
+                                    const float* beta, float* S, void* o, int N, int H, int dk,
+                                    int dv, kda_dtype_t dtype, cudaStream_t stream) {
+  return recurrent_step_impl("kda_gdn_recurrent_step", q, k, v, g, beta, S, o, N, H, dk, dv, dtype,
+                             0, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(256)
                           const TIn* __restrict__ v, const float* __restrict__ g,
                           const float* __restrict__ beta, const float* __restrict__ S0,
                           TIn* __restrict__ o, float* __restrict__ S_out,
-                          const int32_t* __restrict__ cu_seqlens, int T, int H, int DV) {
+                          const int32_t* __restrict__ cu_seqlens, int T, int H, int DV, int gpc) {
   using Cfg = SimtCfg<DK, C>;
   constexpr int DVB = Cfg::DVB, NT = Cfg::NT, LD = Cfg::LD, LC = Cfg::LC, LV = Cfg::LV;
   extern __shared__ float smem[];
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256)
         const size_t off = ((size_t)(s + r) * H + h) * DK + c;
         kv = to_f32(k[off]);
         qv = to_f32(q[off]);
-        gv = g[off];
+        gv = gpc ? g[off] : g[(size_t)(s + r) * H + h];  // per channel, or one gate per token
       }
       Ks[r * LD + c] = kv;
       Qs[r * LD + c] = qv;
@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(256)
 template <typename TIn, int DK, int C>
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* g,
                               const float* beta, const float* S0, void* o, float* S_out,
-                              const int32_t* cu_seqlens, int N, int T, int H, int DV,
+                              const int32_t* cu_seqlens, int N, int T, int H, int DV, int gpc,
                               cudaStream_t stream) {
   using Cfg = SimtCfg<DK, C>;
   static bool attr_set = false;  // benign race: the attribute value is idempotent
@@ -207,7 +207,7 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
   if (grid == 0) return cudaSuccess;
   kda_chunk_simt_kernel<TIn, DK, C><<<(unsigned)grid, Cfg::NT, Cfg::smem_bytes, stream>>>(
       static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), g, beta,
-      S0, static_cast<TIn*>(o), S_out, cu_seqlens, T, H, DV);
+      S0, static_cast<TIn*>(o), S_out, cu_seqlens, T, H, DV, gpc);
   return cudaGetLastError();
 }
 

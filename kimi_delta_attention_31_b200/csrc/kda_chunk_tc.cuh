@@ -213,6 +213,9 @@ __device__ __forceinline__ void unpack8(uint4 w, float* x) {
   }
 }
 
+// kGpc: g holds one gate per key channel (KDA) or one per token and head
+// (Gated DeltaNet).
+template <bool kGpc>
 __global__ void __launch_bounds__(256, 2)
     kda_tc_chunk_local_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                               const bf16* __restrict__ v, const float* __restrict__ g,
@@ -286,8 +289,9 @@ __global__ void __launch_bounds__(256, 2)
     const long long ncps = (T + C - 1) / C, nci = nb / H, ncc = nci % ncps;
     const long long ns = (nci / ncps) * T + ncc * C;
     const int ncn = (int)min((long long)C, (long long)T - ncc * C);
-    for (int idx = tid; idx < 10 * C; idx += 256) {
-      const int r = idx / 10, l = idx % 10;
+    constexpr int lines = kGpc ? 10 : 6;  // a per-token gate is not worth a hint
+    for (int idx = tid; idx < lines * C; idx += 256) {
+      const int r = idx / lines, l = idx % lines;
       if (r < ncn) {
         const size_t off = ((size_t)(ns + r) * H + nh) * D;
         const void* pp = l < 2 ? (const void*)(k + off + 64 * l)
@@ -328,9 +332,15 @@ __global__ void __launch_bounds__(256, 2)
     const int r = 4 * rg + u;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (r < Cn) {
-      const float4* gp = reinterpret_cast<const float4*>(g + base8 + (size_t)r * rs);
-      a = gp[0];
-      b = gp[1];
+      if (kGpc) {
+        const float4* gp = reinterpret_cast<const float4*>(g + base8 + (size_t)r * rs);
+        a = gp[0];
+        b = gp[1];
+      } else {  // one gate per token (Gated DeltaNet), the same on every channel
+        const float x = g[(size_t)(s0 + r) * H + h];
+        a = make_float4(x, x, x, x);
+        b = a;
+      }
     }
     const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -956,7 +966,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
                                    const __nv_bfloat16* v, const float* g, const float* beta,
                                    const float* S0, __nv_bfloat16* o, float* S_out,
                                    const int32_t* cu_seqlens, int N, int B, int T, int H,
-                                   long long max_chunks, void* workspace, cudaEvent_t* ev,
+                                   long long max_chunks, void* workspace, int gpc, cudaEvent_t* ev,
                                    cudaStream_t stream) {
   (void)B;
   static int s_attr_device = -1;
@@ -965,7 +975,10 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (s_attr_device != dev) {
-    e = cudaFuncSetAttribute(tc::kda_tc_chunk_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tc::kda_tc_chunk_local_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc::KA_DYN);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc::kda_tc_chunk_local_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tc::KA_DYN);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc::kda_tc_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -980,8 +993,12 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   const long long items = max_chunks * H;
   if (items > 0) {
     const int gridA = (int)(items < 2LL * s_sms ? items : 2LL * s_sms);
-    tc::kda_tc_chunk_local_kernel<<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens,
-                                                                        num_seqs, T, H, items, ws);
+    if (gpc)
+      tc::kda_tc_chunk_local_kernel<true><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens,
+                                                                              num_seqs, T, H, items, ws);
+    else
+      tc::kda_tc_chunk_local_kernel<false><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens,
+                                                                               num_seqs, T, H, items, ws);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
     kda_decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                            const TIn* __restrict__ v, const float* __restrict__ g,
                            const float* __restrict__ beta, float* __restrict__ S,
-                           TIn* __restrict__ o) {
+                           TIn* __restrict__ o, int gpc) {
   using Cfg = DecodeCfg<TIn, DK, DV>;
   constexpr int DVB = Cfg::DVB, CQ = Cfg::CQ, RG = Cfg::RG, R = Cfg::R, NT = Cfg::NT,
                 NWARP = Cfg::NWARP;
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
   for (int c = tid; c < DK; c += NT) {
     s_k[c] = to_f32(k[(size_t)unit * DK + c]);
     s_q[c] = to_f32(q[(size_t)unit * DK + c]);
-    s_a[c] = expf(g[(size_t)unit * DK + c]);
+    s_a[c] = expf(gpc ? g[(size_t)unit * DK + c] : g[unit]);  // per channel, or one gate per head
   }
   __syncthreads();
   if (warp == 0) {  // k . q
@@ -127,14 +127,14 @@ __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
 
 template <typename TIn, int DK, int DV>
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, const float* g,
-                               const float* beta, float* S, void* o, int N, int H,
+                               const float* beta, float* S, void* o, int N, int H, int gpc,
                                cudaStream_t stream) {
   using Cfg = DecodeCfg<TIn, DK, DV>;
   const long long grid = (long long)N * H * Cfg::NBLK;
   if (grid == 0) return cudaSuccess;
   kda_decode_step_kernel<TIn, DK, DV><<<(unsigned)grid, Cfg::NT, 0, stream>>>(
       static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), g, beta,
-      S, static_cast<TIn*>(o));
+      S, static_cast<TIn*>(o), gpc);
   return cudaGetLastError();
 }
 

@@ -15,6 +15,8 @@ recurrent(...)  token-by-token definition ("Kimi K3 notes 1: KDA" section 4/5;
 chunk(...)      chunkwise schedule in fp64 with pairwise exponentials and plain
                 forward substitution ("Deriving KDA from scratch" section 6;
                 "Linear / sparse attention" tutorial section 6.2).
+gdn_recurrent(...)  Gated DeltaNet (one gate per token and head): the
+                recurrence above with the gate broadcast over key channels.
 
 Inputs are widened exactly to fp64 (bf16 and fp32 values are representable),
 so the rounding of the inputs the GPU sees is not counted as error.
@@ -127,6 +129,21 @@ def recurrent(q, k, v, g, beta, S0=None, cu_seqlens=None, flags=0, return_histor
     if rc != 0:
         raise ValueError(f"kda_oracle_recurrent failed with code {rc}")
     return (o, S_out, hist) if return_history else (o, S_out)
+
+
+def gdn_recurrent(q, k, v, g, beta, S0=None, cu_seqlens=None, num_threads=0):
+    """Gated DeltaNet, token by token in fp64: one decay per token and head
+    ("Kimi K3 notes 1: KDA" section 3; "Linear / sparse attention" tutorial
+    section 5.2), g: [B,T,H].  KDA with every key channel's gate equal to it,
+    so the per-channel recurrence runs on g broadcast over dk (the oracle's
+    pin 6 checks that reduction against the tutorial's own Gated DeltaNet
+    update).  Returns (o, S_out)."""
+    g = _f64(g)
+    dk = (q.shape[-1])
+    if g.ndim != 3:
+        raise ValueError("Gated DeltaNet g must be [B,T,H]")
+    g_full = np.ascontiguousarray(np.broadcast_to(g[..., None], g.shape + (dk,)))
+    return recurrent(q, k, v, g_full, beta, S0, cu_seqlens, num_threads=num_threads)
 
 
 def chunk(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=16, num_threads=0):

@@ -44,7 +44,10 @@ def gather_units(inp, units):
 def oracle_units(inp, units):
     """fp64 oracle outputs for ``units``: list of (o [T_n, dv], S [dk, dv])."""
     p, S0, cu = gather_units(inp, units)
-    o, S = oracle.recurrent(p["q"], p["k"], p["v"], p["g"], p["beta"], S0, cu_seqlens=cu)
+    if inp["g"].dim() == 3:  # Gated DeltaNet: one gate per token and head
+        o, S = oracle.gdn_recurrent(p["q"], p["k"], p["v"], p["g"], p["beta"], S0, cu_seqlens=cu)
+    else:
+        o, S = oracle.recurrent(p["q"], p["k"], p["v"], p["g"], p["beta"], S0, cu_seqlens=cu)
     return [(o[0, cu[i]:cu[i + 1], 0], S[i, 0]) for i in range(len(units))]
 
 

@@ -96,3 +96,34 @@ def test_binding_refuses_host_tensors():
     x = torch.zeros(1, 4, 1, 32)
     with pytest.raises(ValueError):
         kda.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+def test_gdn_entry_points_validate_like_kda_with_a_per_token_gate():
+    """kda_gdn_chunk_fwd takes g [B,T,H] (4-byte aligned is enough); the
+    per-channel entry point keeps its 16-byte rule for g."""
+    lib = kda.load_library()
+    f = _fake()
+
+    def call(fn, g, ws=None):
+        return fn(f, f, f, g, f, None, _fake(0x2000), _fake(0x3000), None, 0, 1, 64, 2, 128, 128, 64,
+                  kda.KDA_BF16, ws, 0, None)
+
+    # both reach the workspace check (no workspace given) only if g passed
+    assert call(lib.kda_gdn_chunk_fwd, _fake(0x1004)) == 4
+    assert "kda_gdn_chunk_fwd" in kda.last_error()
+    assert call(lib.kda_chunk_fwd, _fake(0x1004)) == 3
+    assert call(lib.kda_gdn_chunk_fwd, _fake(0x1002)) == 3
+    assert call(lib.kda_gdn_chunk_fwd, _null()) == 1
+    st = lib.kda_gdn_recurrent_step(f, f, f, f, f, f, f, 4, 2, 96, 96, kda.KDA_BF16, None)
+    assert st == 2 and kda.last_error().startswith("kda_gdn_recurrent_step")
+    assert lib.kda_gdn_recurrent_step(f, f, f, _fake(0x1002), f, f, f, 4, 2, 64, 64, 0, None) == 3
+    assert lib.kda_gdn_recurrent_step(f, f, f, f, f, f, f, 0, 2, 64, 64, 0, None) == 0
+
+
+def test_binding_checks_gate_shapes():
+    import torch
+    x = torch.zeros(1, 4, 1, 32)
+    # host tensors are refused before any shape logic; the shape rule is in the
+    # message the binding raises for device tensors, checked on the GPU suite.
+    with pytest.raises(ValueError):
+        kda.gdn_chunk_fwd(x, x, x, torch.zeros(1, 4, 1), torch.zeros(1, 4, 1))

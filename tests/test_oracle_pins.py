@@ -186,6 +186,21 @@ def test_scalar_gate_matches_gated_deltanet(scalar_gate):
     np.testing.assert_allclose(S[0, 0], ref_M.T, rtol=1e-12, atol=1e-12)
 
 
+def test_gdn_oracle_matches_gated_deltanet():
+    """oracle.gdn_recurrent (gate [B,T,H]) against the tutorial's Gated
+    DeltaNet update, per (sequence, head), two heads with different gates."""
+    rng = np.random.default_rng(16)
+    T, dk, dv, H = 20, 9, 5, 2
+    q, k, v, g, beta, S0 = rand_inputs(rng, 1, T, H, dk, dv)
+    gs = -rng.random((1, T, H)) * 2.0
+    o, S = oracle.gdn_recurrent(q, k, v, gs, beta, S0)
+    for h in range(H):
+        ref_o, ref_M = _gated_deltanet_value_by_key(k[0, :, h], v[0, :, h], q[0, :, h],
+                                                    np.exp(gs[0, :, h]), beta[0, :, h], S0[0, h].T)
+        np.testing.assert_allclose(o[0, :, h], ref_o, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(S[0, h], ref_M.T, rtol=1e-12, atol=1e-12)
+
+
 # ---- pin 7: the projection form of "Kimi K3 notes 1", section 4 ---------------
 def test_projection_form():
     """S_t = (I - beta k k^T) Diag(alpha_t) S_{t-1} + beta k v^T, o_t = S_t^T q_t."""
