@@ -6,7 +6,8 @@ q/k/v, fp32 gates and state), one prefill call per step, inputs resident in
 HBM (2.7 GB of inputs: larger than the 126 MB L2, so no flush is needed).
 Beside it: the recurrent decode (256 sequences x 32 heads, in-place fp32
 state, one token per step) as state GB/s, the Gated DeltaNet variant (one
-gate per token and head) on both shapes, the roofline fractions, the fp64
+gate per token and head) on both shapes, the prefill from raw projections
+with the input preparation fused in, the roofline fractions, the fp64
 CPU oracle timed on this host's cores, and an end-to-end figure through the
 public host-buffer API (pinned host -> device copies, prefill, copies back).
 
@@ -294,6 +295,55 @@ def gdn_leg(kda, args, world, dev, stream, peaks):
     return {"prefill": prefill_line, "decode": decode_line}
 
 
+def prep_leg(kda, args, world, dev, stream, peaks):
+    """KDA from raw projections with the preparation fused into the kernels
+    (bf16 gate logits), on the headline shape; beside it the same work done
+    unfused (torch elementwise preparation, then kda_chunk_fwd) for contrast."""
+    import torch.nn.functional as F
+    w = W.PREP_PREFILL_B8
+    inp = W.make_workload(w, dev)
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(kda.workspace_size(B, T, H, dk, dv, 0, w.chunk, torch.bfloat16), 1),
+                     dtype=torch.uint8, device=dev)
+
+    def fused():
+        kda.chunk_fwd_prep(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], None, None, w.chunk,
+                           o=o, S_out=S_out, workspace=ws)
+
+    def unfused():
+        qn = F.normalize(inp["q"].float(), dim=-1).to(torch.bfloat16)
+        kn = F.normalize(inp["k"].float(), dim=-1).to(torch.bfloat16)
+        g = -F.softplus(inp["a"].float())
+        beta = torch.sigmoid(inp["b"])
+        kda.chunk_fwd(qn, kn, inp["v"], g, beta, None, None, w.chunk, o=o, S_out=S_out, workspace=ws)
+
+    for fn in (fused, unfused):
+        for _ in range(args.warmup):
+            fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(time_launches(fused, args.steps, stream), world, dev)
+    ms_unfused = max_over_ranks(time_launches(unfused, max(1, min(args.steps, 3)), stream), world, dev)
+    kernel_ms = kda.profile_chunk_fwd(fused, stream, repeats=max(1, min(args.steps, 5)), dk=dk, dv=dv,
+                                      chunk_size=w.chunk)
+    token_heads = B * T * H
+    dom_name, dom_ms = max(kernel_ms.items(), key=lambda kv: kv[1])
+    dom_bytes = kda.algorithmic_bytes_per_launch(dom_name, token_heads, B * H, d=dk, gate_bytes=2)
+    dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
+    line = {"workload": w.name, "value": world * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "kernel_ms": kernel_ms,
+            "unfused": {"what": "torch normalize/softplus/sigmoid then kda_chunk_fwd", "ms_per_step": ms_unfused,
+                        "value": world * B * T / (ms_unfused * 1e-3)},
+            "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": dom_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": dom_gbs / peaks["hbm_gbs"], "alg_bytes_per_launch": dom_bytes,
+                         "traffic": None}}
+    del inp, o, S_out, ws
+    torch.cuda.empty_cache()
+    return line
+
+
 def run_ours(args):
     import kimi_delta_attention_31_b200 as kda
     rank, world, local = dist_setup(args.gpus)
@@ -410,6 +460,8 @@ def run_ours(args):
 
     # ---------------- Gated DeltaNet (scalar gate) ----------------
     gdn = gdn_leg(kda, args, world, dev, stream, peaks)
+    # ---------------- fused input preparation from raw projections ----------------
+    prep = prep_leg(kda, args, world, dev, stream, peaks)
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only) ----------------
     cpu = None
@@ -425,7 +477,7 @@ def run_ours(args):
                        "chunk": w.chunk, "g": f"-softplus(N({w.g_mu},{w.g_sigma}))",
                        "l2": "inputs (2.7 GB) larger than L2; no flush",
                        "parallelism": f"dp{world} (independent batches per GPU)"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "gdn": gdn,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "gdn": gdn, "prep": prep,
             "gpu_launches": gpu_launches, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -144,6 +144,33 @@ kda_status_t kda_gdn_recurrent_step(const void* q, const void* k, const void* v,
                                     int dv, kda_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * KDA from raw projections, with the input preparation fused into the
+ * kernels' load phase ("Kimi K3 notes 1: KDA" section 4: q and k are
+ * L2-normalised; "Linear / sparse attention" tutorial section 10: beta and
+ * the decay come from bounded activations, sigmoid / softplus).  Per token and
+ * head, before the recurrence:
+ *   q <- q / max(|q|_2, 1e-12),  k <- k / max(|k|_2, 1e-12)   (over dk, fp32)
+ *   log alpha = -softplus(a) = -log(1 + e^a)                   (per key channel)
+ *   beta = sigmoid(b) = 1 / (1 + e^-b)
+ * Arguments as kda_chunk_fwd / kda_recurrent_step except
+ *   a : raw gate logits, same layout as g ([B, T, H, dk] / [N, H, dk]), in
+ *       a_dtype (KDA_F32 or KDA_BF16: bf16 halves the largest input);
+ *       kda_chunk_fwd_prep needs it 16-byte aligned, the decode step
+ *       element-aligned;
+ *   b : raw beta logits, fp32, same layout as beta.
+ * q and k are read as given (unnormalised); nothing is written back to them.
+ * Same workspace, paths and exactness domain as kda_chunk_fwd.
+ */
+kda_status_t kda_chunk_fwd_prep(const void* q, const void* k, const void* v, const void* a,
+                                kda_dtype_t a_dtype, const float* b, const float* S0, void* o,
+                                float* S_out, const int32_t* cu_seqlens, int num_seqs, int B, int T,
+                                int H, int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+kda_status_t kda_recurrent_step_prep(const void* q, const void* k, const void* v, const void* a,
+                                     kda_dtype_t a_dtype, const float* b, float* S, void* o, int N,
+                                     int H, int dk, int dv, kda_dtype_t dtype, cudaStream_t stream);
+
+/*
  * kda_chunk_fwd for callers that cannot allocate device memory: the same
  * prefill, same arguments minus the workspace.  (Library plumbing: the pages
  * have no counterpart.)  Some callers get only input and output pointers
@@ -186,8 +213,8 @@ kda_status_t kda_device_error(int* code, cudaStream_t stream);
 int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype);
 
 /*
- * Measurement hook.  While set (events != NULL), each later kda_chunk_fwd or
- * kda_gdn_chunk_fwd call made by the calling thread records events[0] before its first kernel
+ * Measurement hook.  While set (events != NULL), each later kda_chunk_fwd,
+ * kda_gdn_chunk_fwd or kda_chunk_fwd_prep call made by the calling thread records events[0] before its first kernel
  * launch and events[i] after its i-th launch, on the call's stream; count
  * must be at least kda_chunk_fwd_launches(...) + 1 or the call fails with
  * KDA_ERR_INVALID_ARG.  The caller owns the events.  Pass NULL, 0 to stop.

@@ -44,6 +44,7 @@ class Workload:
     seed: int
     lengths: Optional[tuple] = None  # packed varlen sequence lengths (B == 1)
     scalar_gate: bool = False  # Gated DeltaNet: g is [B, T, H] (one gate per token and head)
+    raw_a_dtype: Optional[str] = None  # raw projections for the fused-preparation entry points
 
     @property
     def tokens(self) -> int:
@@ -87,8 +88,13 @@ GDN_PREFILL_B8 = Workload("gdn_prefill_bf16_B8_H32_T8192_d128", 8, 8192, 32, 128
 GDN_DECODE = Workload("gdn_decode_bf16_N256_H32_d128_1024steps", 256, 1024, 32, 128, 128, "bf16",
                       -3.0, 1.0, 0.02, 1, 1006, scalar_gate=True)
 
+# The headline prefill shape from raw projections: unnormalised q, k, bf16 gate
+# logits a (log alpha = -softplus(a)), fp32 beta logits b.
+PREP_PREFILL_B8 = Workload("kda_prefill_prep_bf16logits_B8_H32_T8192_d128", 8, 8192, 32, 128, 128, "bf16",
+                           -5.0, 1.5, 0.0, 64, 1007, raw_a_dtype="bf16")
+
 WORKLOADS = {w.name: w for w in (ORACLE_SMALL, PREFILL_H16, PREFILL_B8, PREFILL_VARLEN, DECODE,
-                                 GDN_PREFILL_B8, GDN_DECODE)}
+                                 GDN_PREFILL_B8, GDN_DECODE, PREP_PREFILL_B8)}
 
 
 def cu_seqlens_of(lengths, device="cpu") -> torch.Tensor:
@@ -141,7 +147,36 @@ def make_prefill(B, T, H, dk, dv, dtype="bf16", g_mu=-4.0, g_sigma=1.0, s0_std=0
     return out
 
 
+def make_prefill_raw(B, T, H, dk, dv, dtype="bf16", a_mu=-5.0, a_sigma=1.5, a_dtype="bf16",
+                     s0_std=0.0, seed=0, device="cpu", lengths=None) -> dict:
+    """Raw projections for the fused-preparation entry points.  Same draws and
+    order as make_prefill (q, k, v, beta-logit, alpha-logit, S0), but q and k
+    are not normalised, b is the beta logit itself and a = N(a_mu, a_sigma) is
+    the gate logit (log alpha = -softplus(a)), rounded to ``a_dtype``."""
+    if lengths is not None:
+        assert B == 1 and T == sum(lengths)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    adt = torch.bfloat16 if a_dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=device).manual_seed(seed)
+    q = torch.randn((B, T, H, dk), generator=gen, device=device, dtype=torch.float32)
+    k = torch.randn((B, T, H, dk), generator=gen, device=device, dtype=torch.float32)
+    v = torch.randn((B, T, H, dv), generator=gen, device=device, dtype=torch.float32)
+    b = torch.randn((B, T, H), generator=gen, device=device, dtype=torch.float32)
+    a = torch.randn((B, T, H, dk), generator=gen, device=device, dtype=torch.float32) * a_sigma + a_mu
+    N = len(lengths) if lengths is not None else B
+    S0 = (torch.randn((N, H, dk, dv), generator=gen, device=device, dtype=torch.float32) * s0_std
+          if s0_std > 0 else None)
+    out = dict(q=q.to(tdt).contiguous(), k=k.to(tdt).contiguous(), v=v.to(tdt).contiguous(),
+               a=a.to(adt).contiguous(), b=b.contiguous(), S0=S0)
+    if lengths is not None:
+        out["cu_seqlens"] = cu_seqlens_of(lengths, device)
+    return out
+
+
 def make_workload(w: Workload, device="cpu") -> dict:
+    if w.raw_a_dtype is not None:
+        return make_prefill_raw(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.g_mu, w.g_sigma, w.raw_a_dtype,
+                                w.s0_std, w.seed, device, lengths=w.lengths)
     return make_prefill(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.g_mu, w.g_sigma, w.s0_std,
                         w.seed, device, lengths=w.lengths, scalar_gate=w.scalar_gate)
 
@@ -180,5 +215,5 @@ def describe(w: Workload) -> str:
 
 
 __all__ = ["Workload", "WORKLOADS", "ORACLE_SMALL", "PREFILL_H16", "PREFILL_B8", "PREFILL_VARLEN",
-           "DECODE", "GDN_PREFILL_B8", "GDN_DECODE", "make_prefill", "make_workload", "make_decode_state", "make_decode_steps",
+           "DECODE", "GDN_PREFILL_B8", "GDN_DECODE", "PREP_PREFILL_B8", "make_prefill_raw", "make_prefill", "make_workload", "make_decode_state", "make_decode_steps",
            "cu_seqlens_of", "varlen_lengths", "bytes_of", "describe"]

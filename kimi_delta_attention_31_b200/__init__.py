@@ -36,7 +36,8 @@ KDA_BF16, KDA_F32 = 0, 1
 # Every symbol include/kda.h declares (checked by the CPU test-suite).
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_last_error", "kda_device_error", "kda_chunk_fwd_launches", "kda_profile_events",
-            "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step")
+            "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step",
+            "kda_chunk_fwd_prep", "kda_recurrent_step_prep")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -79,6 +80,10 @@ def load_library():
         lib.kda_gdn_chunk_fwd.restype = i32
         lib.kda_gdn_recurrent_step.argtypes = lib.kda_recurrent_step.argtypes
         lib.kda_gdn_recurrent_step.restype = i32
+        lib.kda_chunk_fwd_prep.argtypes = [vp] * 4 + [i32] + [vp] * 5 + [i32] * 7 + [i32, vp, szt, vp]
+        lib.kda_chunk_fwd_prep.restype = i32
+        lib.kda_recurrent_step_prep.argtypes = [vp] * 4 + [i32] + [vp] * 3 + [i32] * 5 + [vp]
+        lib.kda_recurrent_step_prep.restype = i32
         lib.kda_last_error.argtypes = []
         lib.kda_last_error.restype = ctypes.c_char_p
         lib.kda_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), vp]
@@ -151,6 +156,16 @@ def gdn_chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, out
                       output_final_state, o, S_out, workspace)
 
 
+def chunk_fwd_prep(q, k, v, a, b, S0=None, cu_seqlens=None, chunk_size=64, output_final_state=True,
+                   o=None, S_out=None, workspace=None):
+    """KDA prefill from raw projections: q, k [B,T,H,dk] unnormalised; a [B,T,H,dk]
+    raw gate logits (bf16 or fp32; log alpha = -softplus(a)); b [B,T,H] fp32 raw
+    beta logits (beta = sigmoid(b)).  q and k are L2-normalised per (token, head)
+    inside the kernels."""
+    return _chunk_fwd("kda_chunk_fwd_prep", q, k, v, a, b, S0, cu_seqlens, chunk_size, output_final_state,
+                      o, S_out, workspace)
+
+
 def _chunk_fwd(fn, q, k, v, g, beta, S0, cu_seqlens, chunk_size, output_final_state, o, S_out,
                workspace):
     lib = load_library()
@@ -159,8 +174,9 @@ def _chunk_fwd(fn, q, k, v, g, beta, S0, cu_seqlens, chunk_size, output_final_st
     dv = v.shape[-1]
     num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     N = num_seqs if cu_seqlens is not None else B
-    if g.dtype != torch.float32 or beta.dtype != torch.float32:
-        raise TypeError("g and beta must be float32")
+    prep = fn == "kda_chunk_fwd_prep"
+    if g.dtype not in ((torch.float32, torch.bfloat16) if prep else (torch.float32,)) or beta.dtype != torch.float32:
+        raise TypeError("g (a) and beta (b) must be float32 (a may be bfloat16)")
     g_shape = (B, T, H) if fn == "kda_gdn_chunk_fwd" else (B, T, H, dk)
     if tuple(g.shape) != g_shape or tuple(beta.shape) != (B, T, H):
         raise ValueError(f"g must be {g_shape} and beta {(B, T, H)}, got {tuple(g.shape)}, {tuple(beta.shape)}")
@@ -174,7 +190,8 @@ def _chunk_fwd(fn, q, k, v, g, beta, S0, cu_seqlens, chunk_size, output_final_st
     if workspace is None and ws_need:
         workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+    gargs = (_ptr(g), _dtype_code(g)) if prep else (_ptr(g),)
+    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), *gargs, _ptr(beta), _ptr(S0), _ptr(o),
                           _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
                           _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(q.device))
     _check(st)
@@ -213,19 +230,28 @@ def gdn_recurrent_step(q, k, v, g, beta, S, o=None):
     return _recurrent_step("kda_gdn_recurrent_step", q, k, v, g, beta, S, o)
 
 
+def recurrent_step_prep(q, k, v, a, b, S, o=None):
+    """Decode step from raw projections (see chunk_fwd_prep): a [N,H,dk] bf16 or
+    fp32 raw gate logits, b [N,H] fp32 raw beta logits."""
+    return _recurrent_step("kda_recurrent_step_prep", q, k, v, a, b, S, o)
+
+
 def _recurrent_step(fn, q, k, v, g, beta, S, o):
     lib = load_library()
     _need_cuda(q, k, v, g, beta, S, o)
     N, H, dk = q.shape
     dv = v.shape[-1]
-    if S.dtype != torch.float32 or g.dtype != torch.float32 or beta.dtype != torch.float32:
-        raise TypeError("S, g and beta must be float32")
+    prep = fn == "kda_recurrent_step_prep"
+    g_ok = g.dtype in ((torch.float32, torch.bfloat16) if prep else (torch.float32,))
+    if S.dtype != torch.float32 or not g_ok or beta.dtype != torch.float32:
+        raise TypeError("S, g (a) and beta (b) must be float32 (a may be bfloat16)")
     g_shape = (N, H) if fn == "kda_gdn_recurrent_step" else (N, H, dk)
     if tuple(g.shape) != g_shape or tuple(beta.shape) != (N, H) or tuple(S.shape) != (N, H, dk, dv):
         raise ValueError(f"g must be {g_shape}, beta {(N, H)}, S {(N, H, dk, dv)}")
     if o is None:
         o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
-    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+    gargs = (_ptr(g), _dtype_code(g)) if prep else (_ptr(g),)
+    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), *gargs, _ptr(beta), _ptr(S), _ptr(o),
                           N, H, dk, dv, _dtype_code(q), _stream_handle(q.device))
     _check(st)
     return o
@@ -329,11 +355,12 @@ TC_IMAGE_BYTES_PER_TOKEN_HEAD = 1160
 
 
 def algorithmic_bytes_per_launch(kernel, token_heads, units, d=128, with_state_in=False,
-                                 gate_per_channel=True):
-    """Bytes one launch must move.  The gate is fp32, d values per token-head
-    (KDA) or one (Gated DeltaNet, gate_per_channel=False)."""
+                                 gate_per_channel=True, gate_bytes=4):
+    """Bytes one launch must move.  The gate has d values per token-head (KDA)
+    or one (Gated DeltaNet, gate_per_channel=False), of gate_bytes each (4 for
+    fp32 log alpha or logits, 2 for bf16 logits)."""
     state = d * d * 4 * units
-    gate = 4 * d if gate_per_channel else 4
+    gate = gate_bytes * d if gate_per_channel else gate_bytes
     if kernel == "kda_chunk_simt_kernel":
         return token_heads * (3 * 2 * d + gate + 4 + 2 * d) + state * (2 if with_state_in else 1)
     if kernel == "kda_tc_chunk_local_kernel":

@@ -45,13 +45,13 @@ long long max_chunks(int B, int T, int num_seqs, int chunk_size) {
 
 template <typename TIn>
 cudaError_t dispatch_chunk_simt(int dk, int C, const void* q, const void* k, const void* v,
-                                const float* g, const float* beta, const float* S0, void* o,
+                                const void* g, const float* beta, const float* S0, void* o,
                                 float* S_out, const int32_t* cu, int N, int T, int H, int dv,
-                                int gpc, cudaStream_t st) {
+                                int gmode, cudaStream_t st) {
 #define KDA_SIMT_CASE(D, CC)                                                                  \
   if (dk == D && C == CC)                                                                     \
     return kda::launch_chunk_simt<TIn, D, CC>(q, k, v, g, beta, S0, o, S_out, cu, N, T, H, dv, \
-                                               gpc, st);
+                                               gmode, st);
   KDA_SIMT_CASE(32, 16) KDA_SIMT_CASE(32, 32) KDA_SIMT_CASE(32, 64)
   KDA_SIMT_CASE(64, 16) KDA_SIMT_CASE(64, 32) KDA_SIMT_CASE(64, 64)
   KDA_SIMT_CASE(128, 16) KDA_SIMT_CASE(128, 32) KDA_SIMT_CASE(128, 64)
@@ -60,22 +60,23 @@ cudaError_t dispatch_chunk_simt(int dk, int C, const void* q, const void* k, con
 }
 
 template <typename TIn>
-cudaError_t dispatch_decode(int dk, const void* q, const void* k, const void* v, const float* g,
-                            const float* beta, float* S, void* o, int N, int H, int gpc,
+cudaError_t dispatch_decode(int dk, const void* q, const void* k, const void* v, const void* g,
+                            const float* beta, float* S, void* o, int N, int H, int gmode,
                             cudaStream_t st) {
-  if (dk == 32) return kda::launch_decode_step<TIn, 32, 32>(q, k, v, g, beta, S, o, N, H, gpc, st);
-  if (dk == 64) return kda::launch_decode_step<TIn, 64, 64>(q, k, v, g, beta, S, o, N, H, gpc, st);
-  if (dk == 128) return kda::launch_decode_step<TIn, 128, 128>(q, k, v, g, beta, S, o, N, H, gpc, st);
+  if (dk == 32) return kda::launch_decode_step<TIn, 32, 32>(q, k, v, g, beta, S, o, N, H, gmode, st);
+  if (dk == 64) return kda::launch_decode_step<TIn, 64, 64>(q, k, v, g, beta, S, o, N, H, gmode, st);
+  if (dk == 128) return kda::launch_decode_step<TIn, 128, 128>(q, k, v, g, beta, S, o, N, H, gmode, st);
   return cudaErrorInvalidValue;
 }
 
-// gpc: g holds one gate per key channel ([.., H, dk], KDA) or one per token
-// and head ([.., H], Gated DeltaNet).
+// gmode (kda::GateMode): g holds log alpha per key channel ([.., H, dk], KDA)
+// or per token and head ([.., H], Gated DeltaNet), or raw per-channel logits
+// (fp32 or bf16) with q, k normalised and beta given as a logit.
 kda_status_t chunk_fwd_impl(const char* fn, const void* q, const void* k, const void* v,
-                            const float* g, const float* beta, const float* S0, void* o,
+                            const void* g, const float* beta, const float* S0, void* o,
                             float* S_out, const int32_t* cu_seqlens, int num_seqs, int B, int T,
                             int H, int dk, int dv, int chunk_size, kda_dtype_t dtype,
-                            void* workspace, size_t workspace_bytes, int gpc,
+                            void* workspace, size_t workspace_bytes, int gmode,
                             cudaStream_t stream) {
   t_err[0] = 0;
   if (B < 0 || T < 0 || H <= 0 || num_seqs < 0)
@@ -100,7 +101,7 @@ kda_status_t chunk_fwd_impl(const char* fn, const void* q, const void* k, const 
   if (N == 0) return KDA_OK;
   if (tokens > 0 && (!q || !k || !v || !g || !beta || !o))
     return fail(KDA_ERR_INVALID_ARG, "%s: null input/output pointer", fn);
-  const void* ptrs[] = {q, k, v, gpc ? g : nullptr, S0, o, S_out, workspace};
+  const void* ptrs[] = {q, k, v, gmode != kda::kGateLogTok ? g : nullptr, S0, o, S_out, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
   if ((beta && !aligned_to(beta, 4)) || (cu_seqlens && !aligned_to(cu_seqlens, 4)) ||
@@ -125,13 +126,13 @@ kda_status_t chunk_fwd_impl(const char* fn, const void* q, const void* k, const 
                              static_cast<const __nv_bfloat16*>(k),
                              static_cast<const __nv_bfloat16*>(v), g, beta, S0,
                              static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H,
-                             max_chunks(B, T, num_seqs, chunk_size), workspace, gpc, ev, stream);
+                             max_chunks(B, T, num_seqs, chunk_size), workspace, gmode, ev, stream);
   } else if (dtype == KDA_F32) {
     e = dispatch_chunk_simt<float>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, T,
-                                   H, dv, gpc, stream);
+                                   H, dv, gmode, stream);
   } else {
     e = dispatch_chunk_simt<__nv_bfloat16>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out,
-                                           cu_seqlens, N, T, H, dv, gpc, stream);
+                                           cu_seqlens, N, T, H, dv, gmode, stream);
   }
   if (e != cudaSuccess) return cuda_fail(e, fn);
   if (ev && launches == 1 && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess)
@@ -140,8 +141,8 @@ kda_status_t chunk_fwd_impl(const char* fn, const void* q, const void* k, const 
 }
 
 kda_status_t recurrent_step_impl(const char* fn, const void* q, const void* k, const void* v,
-                                const float* g, const float* beta, float* S, void* o, int N, int H,
-                                int dk, int dv, kda_dtype_t dtype, int gpc, cudaStream_t stream) {
+                                const void* g, const float* beta, float* S, void* o, int N, int H,
+                                int dk, int dv, kda_dtype_t dtype, int gmode, cudaStream_t stream) {
   t_err[0] = 0;
   if (N < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes N=%d H=%d", fn, N, H);
   if (dtype != KDA_BF16 && dtype != KDA_F32)
@@ -157,11 +158,11 @@ kda_status_t recurrent_step_impl(const char* fn, const void* q, const void* k, c
   const void* elem[] = {q, k, v, o};
   for (const void* p : elem)
     if (!aligned_to(p, esz)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is misaligned", fn, p);
-  if (!aligned_to(g, 4) || !aligned_to(beta, 4))
-    return fail(KDA_ERR_ALIGNMENT, "%s: g / beta not 4-byte aligned", fn);
+  if (!aligned_to(g, gmode == kda::kGateLogitBf16 ? 2 : 4) || !aligned_to(beta, 4))
+    return fail(KDA_ERR_ALIGNMENT, "%s: g / beta not element-aligned", fn);
   cudaError_t e = dtype == KDA_F32
-                      ? dispatch_decode<float>(dk, q, k, v, g, beta, S, o, N, H, gpc, stream)
-                      : dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, N, H, gpc, stream);
+                      ? dispatch_decode<float>(dk, q, k, v, g, beta, S, o, N, H, gmode, stream)
+                      : dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, N, H, gmode, stream);
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return KDA_OK;
 }
@@ -200,7 +201,7 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
                            int dk, int dv, int chunk_size, kda_dtype_t dtype,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   return chunk_fwd_impl("kda_chunk_fwd", q, k, v, g, beta, S0, o, S_out, cu_seqlens, num_seqs, B, T,
-                        H, dk, dv, chunk_size, dtype, workspace, workspace_bytes, 1, stream);
+                        H, dk, dv, chunk_size, dtype, workspace, workspace_bytes, kda::kGateLogCh, stream);
 }
 
 kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
@@ -209,21 +210,43 @@ kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, cons
                                int dk, int dv, int chunk_size, kda_dtype_t dtype,
                                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   return chunk_fwd_impl("kda_gdn_chunk_fwd", q, k, v, g, beta, S0, o, S_out, cu_seqlens, num_seqs,
-                        B, T, H, dk, dv, chunk_size, dtype, workspace, workspace_bytes, 0, stream);
+                        B, T, H, dk, dv, chunk_size, dtype, workspace, workspace_bytes, kda::kGateLogTok,
+                        stream);
+}
+
+kda_status_t kda_chunk_fwd_prep(const void* q, const void* k, const void* v, const void* a,
+                                kda_dtype_t a_dtype, const float* b, const float* S0, void* o,
+                                float* S_out, const int32_t* cu_seqlens, int num_seqs, int B, int T,
+                                int H, int dk, int dv, int chunk_size, kda_dtype_t dtype,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (a_dtype != KDA_BF16 && a_dtype != KDA_F32)
+    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_prep: unknown a_dtype %d", (int)a_dtype);
+  return chunk_fwd_impl("kda_chunk_fwd_prep", q, k, v, a, b, S0, o, S_out, cu_seqlens, num_seqs, B, T,
+                        H, dk, dv, chunk_size, dtype, workspace, workspace_bytes,
+                        a_dtype == KDA_BF16 ? kda::kGateLogitBf16 : kda::kGateLogitF32, stream);
 }
 
 kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, float* S, void* o, int N, int H, int dk,
                                 int dv, kda_dtype_t dtype, cudaStream_t stream) {
-  return recurrent_step_impl("kda_recurrent_step", q, k, v, g, beta, S, o, N, H, dk, dv, dtype, 1,
-                             stream);
+  return recurrent_step_impl("kda_recurrent_step", q, k, v, g, beta, S, o, N, H, dk, dv, dtype,
+                             kda::kGateLogCh, stream);
 }
 
 kda_status_t kda_gdn_recurrent_step(const void* q, const void* k, const void* v, const float* g,
                                     const float* beta, float* S, void* o, int N, int H, int dk,
                                     int dv, kda_dtype_t dtype, cudaStream_t stream) {
   return recurrent_step_impl("kda_gdn_recurrent_step", q, k, v, g, beta, S, o, N, H, dk, dv, dtype,
-                             0, stream);
+                             kda::kGateLogTok, stream);
+}
+
+kda_status_t kda_recurrent_step_prep(const void* q, const void* k, const void* v, const void* a,
+                                     kda_dtype_t a_dtype, const float* b, float* S, void* o, int N,
+                                     int H, int dk, int dv, kda_dtype_t dtype, cudaStream_t stream) {
+  if (a_dtype != KDA_BF16 && a_dtype != KDA_F32)
+    return fail(KDA_ERR_UNSUPPORTED, "kda_recurrent_step_prep: unknown a_dtype %d", (int)a_dtype);
+  return recurrent_step_impl("kda_recurrent_step_prep", q, k, v, a, b, S, o, N, H, dk, dv, dtype,
+                             a_dtype == KDA_BF16 ? kda::kGateLogitBf16 : kda::kGateLogitF32, stream);
 }
 
 // ---------------------------------------------------------------------------

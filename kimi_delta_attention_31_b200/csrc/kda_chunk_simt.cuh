@@ -49,10 +49,10 @@ __device__ __forceinline__ void seq_bounds(const int32_t* cu_seqlens, int n, int
 template <typename TIn, int DK, int C>
 __global__ void __launch_bounds__(256)
     kda_chunk_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
-                          const TIn* __restrict__ v, const float* __restrict__ g,
+                          const TIn* __restrict__ v, const void* __restrict__ gate,
                           const float* __restrict__ beta, const float* __restrict__ S0,
                           TIn* __restrict__ o, float* __restrict__ S_out,
-                          const int32_t* __restrict__ cu_seqlens, int T, int H, int DV, int gpc) {
+                          const int32_t* __restrict__ cu_seqlens, int T, int H, int DV, int gmode) {
   using Cfg = SimtCfg<DK, C>;
   constexpr int DVB = Cfg::DVB, NT = Cfg::NT, LD = Cfg::LD, LC = Cfg::LC, LV = Cfg::LV;
   extern __shared__ float smem[];
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256)
         const size_t off = ((size_t)(s + r) * H + h) * DK + c;
         kv = to_f32(k[off]);
         qv = to_f32(q[off]);
-        gv = gpc ? g[off] : g[(size_t)(s + r) * H + h];  // per channel, or one gate per token
+        gv = gate_log(gate, gmode, (size_t)(s + r) * H + h, DK, c);
       }
       Ks[r * LD + c] = kv;
       Qs[r * LD + c] = qv;
@@ -101,8 +101,29 @@ __global__ void __launch_bounds__(256)
       const int r = idx / DVB, j = idx % DVB;
       Vs[r * LV + j] = r < Cn ? to_f32(v[((size_t)(s + r) * H + h) * DV + vb * DVB + j]) : 0.f;
     }
-    for (int r = tid; r < C; r += NT) bs[r] = r < Cn ? beta[(size_t)(s + r) * H + h] : 0.f;
+    for (int r = tid; r < C; r += NT) bs[r] = r < Cn ? beta_of(beta, gmode, (size_t)(s + r) * H + h) : 0.f;
     __syncthreads();
+    if (gate_prep(gmode)) {  // L2-normalise each row of k and q over dk (a warp per row)
+      const int lane = tid & 31;
+      for (int r = tid >> 5; r < C; r += NT / 32) {
+        float sk = 0.f, sq = 0.f;
+        for (int c = lane; c < DK; c += 32) {
+          sk = fmaf(Ks[r * LD + c], Ks[r * LD + c], sk);
+          sq = fmaf(Qs[r * LD + c], Qs[r * LD + c], sq);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          sk += __shfl_xor_sync(0xffffffffu, sk, off);
+          sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        }
+        const float rk = rsqrtf(fmaxf(sk, 1e-24f)), rq = rsqrtf(fmaxf(sq, 1e-24f));
+        for (int c = lane; c < DK; c += 32) {
+          Ks[r * LD + c] *= rk;
+          Qs[r * LD + c] *= rq;
+        }
+      }
+      __syncthreads();
+    }
     // 2. cumulative log-decay per key channel
     for (int c = tid; c < DK; c += NT) {
       float acc = 0.f;
@@ -190,9 +211,9 @@ __global__ void __launch_bounds__(256)
 }
 
 template <typename TIn, int DK, int C>
-cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* g,
+cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* g,
                               const float* beta, const float* S0, void* o, float* S_out,
-                              const int32_t* cu_seqlens, int N, int T, int H, int DV, int gpc,
+                              const int32_t* cu_seqlens, int N, int T, int H, int DV, int gmode,
                               cudaStream_t stream) {
   using Cfg = SimtCfg<DK, C>;
   static bool attr_set = false;  // benign race: the attribute value is idempotent
@@ -207,7 +228,7 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
   if (grid == 0) return cudaSuccess;
   kda_chunk_simt_kernel<TIn, DK, C><<<(unsigned)grid, Cfg::NT, Cfg::smem_bytes, stream>>>(
       static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), g, beta,
-      S0, static_cast<TIn*>(o), S_out, cu_seqlens, T, H, DV, gpc);
+      S0, static_cast<TIn*>(o), S_out, cu_seqlens, T, H, DV, gmode);
   return cudaGetLastError();
 }
 

@@ -213,15 +213,27 @@ __device__ __forceinline__ void unpack8(uint4 w, float* x) {
   }
 }
 
-// kGpc: g holds one gate per key channel (KDA) or one per token and head
-// (Gated DeltaNet).
-template <bool kGpc>
+__device__ __forceinline__ void normalise_rows(float* kv, float* qv, float nk, float nq) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    kv[e] *= nk;
+    qv[e] *= nq;
+  }
+}
+
+// kGate (GateMode): what the gate argument holds -- log alpha per key channel
+// (KDA) or per token (Gated DeltaNet), or raw per-channel logits in fp32 or
+// bf16, in which case q and k rows are also L2-normalised and beta is the
+// sigmoid of the given logit.
+template <int kGate>
 __global__ void __launch_bounds__(256, 2)
     kda_tc_chunk_local_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
-                              const bf16* __restrict__ v, const float* __restrict__ g,
+                              const bf16* __restrict__ v, const void* __restrict__ gate,
                               const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                               int num_seqs, int T, int H, long long num_items, uint8_t* __restrict__ ws) {
   __shared__ __align__(16) float s_beta[C];
+  __shared__ float s_nrm[2][C];  // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
+  constexpr bool kPrep = gate_prep(kGate);
   __shared__ __align__(16) float s_Ge[4][D];  // G at the end of each 16-token block
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ uint32_t s_tmem;
@@ -289,7 +301,8 @@ __global__ void __launch_bounds__(256, 2)
     const long long ncps = (T + C - 1) / C, nci = nb / H, ncc = nci % ncps;
     const long long ns = (nci / ncps) * T + ncc * C;
     const int ncn = (int)min((long long)C, (long long)T - ncc * C);
-    constexpr int lines = kGpc ? 10 : 6;  // a per-token gate is not worth a hint
+    // 128-byte lines per row: k, q, v 2 each, then the gate (fp32 4, bf16 2, per token 0)
+    constexpr int lines = kGate == kGateLogTok ? 6 : kGate == kGateLogitBf16 ? 8 : 10;
     for (int idx = tid; idx < lines * C; idx += 256) {
       const int r = idx / lines, l = idx % lines;
       if (r < ncn) {
@@ -297,12 +310,14 @@ __global__ void __launch_bounds__(256, 2)
         const void* pp = l < 2 ? (const void*)(k + off + 64 * l)
                        : l < 4 ? (const void*)(q + off + 64 * (l - 2))
                        : l < 6 ? (const void*)(v + off + 64 * (l - 4))
-                               : (const void*)(g + off + 32 * (l - 6));
+                       : kGate == kGateLogitBf16
+                               ? (const void*)(static_cast<const bf16*>(gate) + off + 64 * (l - 6))
+                               : (const void*)(static_cast<const float*>(gate) + off + 32 * (l - 6));
         asm volatile("prefetch.global.L2 [%0];" ::"l"(pp));
       }
     }
   }
-  if (tid < C) s_beta[tid] = tid < Cn ? beta[(size_t)(s0 + tid) * H + h] : 0.f;
+  if (tid < C) s_beta[tid] = tid < Cn ? beta_of(beta, kGate, (size_t)(s0 + tid) * H + h) : 0.f;
 
   // ---- 1. loads; cumulative log-decay G (fp32); rows >= Cn contribute g = 0.
   // The k, q, v rows are loaded here, together with g, and parked in TMEM
@@ -332,19 +347,51 @@ __global__ void __launch_bounds__(256, 2)
     const int r = 4 * rg + u;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     if (r < Cn) {
-      if (kGpc) {
-        const float4* gp = reinterpret_cast<const float4*>(g + base8 + (size_t)r * rs);
-        a = gp[0];
-        b = gp[1];
-      } else {  // one gate per token (Gated DeltaNet), the same on every channel
-        const float x = g[(size_t)(s0 + r) * H + h];
+      if constexpr (kGate == kGateLogTok) {  // one gate per token, the same on every channel
+        const float x = static_cast<const float*>(gate)[(size_t)(s0 + r) * H + h];
         a = make_float4(x, x, x, x);
         b = a;
+      } else if constexpr (kGate == kGateLogitBf16) {
+        float x[8];
+        unpack8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(gate) + base8 + (size_t)r * rs), x);
+        a = make_float4(neg_softplus(x[0]), neg_softplus(x[1]), neg_softplus(x[2]), neg_softplus(x[3]));
+        b = make_float4(neg_softplus(x[4]), neg_softplus(x[5]), neg_softplus(x[6]), neg_softplus(x[7]));
+      } else {
+        const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(gate) + base8 + (size_t)r * rs);
+        a = gp[0];
+        b = gp[1];
+        if constexpr (kGate == kGateLogitF32) {
+          a = make_float4(neg_softplus(a.x), neg_softplus(a.y), neg_softplus(a.z), neg_softplus(a.w));
+          b = make_float4(neg_softplus(b.x), neg_softplus(b.y), neg_softplus(b.z), neg_softplus(b.w));
+        }
       }
     }
     const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int e = 0; e < 8; ++e) G[u][e] = (u ? G[u - 1][e] : 0.f) + x[e];
+  }
+  if constexpr (kPrep) {  // 1 / |k_r| and 1 / |q_r| over dk: the 16 lanes of a half-warp share a row
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float kx[8], qx[8];
+      unpack8(make_uint4(kst[4 * u], kst[4 * u + 1], kst[4 * u + 2], kst[4 * u + 3]), kx);
+      unpack8(make_uint4(qst[4 * u], qst[4 * u + 1], qst[4 * u + 2], qst[4 * u + 3]), qx);
+      float sk = 0.f, sq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sk = fmaf(kx[e], kx[e], sk);
+        sq = fmaf(qx[e], qx[e], sq);
+      }
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) {
+        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      }
+      if (co == 0) {
+        s_nrm[0][4 * rg + u] = rsqrtf(fmaxf(sk, 1e-24f));
+        s_nrm[1][4 * rg + u] = rsqrtf(fmaxf(sq, 1e-24f));
+      }
+    }
   }
   float* s_tot = reinterpret_cast<float*>(sm + KA_XK);  // [16][128] row-group totals (XK is built later)
   reinterpret_cast<float4*>(s_tot + rg * D + c0)[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
@@ -416,6 +463,7 @@ __global__ void __launch_bounds__(256, 2)
       float kv[8], qv[8];
       unpack8(make_uint4(kr4[0], kr4[1], kr4[2], kr4[3]), kv);
       unpack8(make_uint4(qr4[0], qr4[1], qr4[2], qr4[3]), qv);
+      if constexpr (kPrep) normalise_rows(kv, qv, s_nrm[0][r], s_nrm[1][r]);
       float o_ka[8], o_qa[8], o_kr[8], o_kb[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -464,6 +512,7 @@ __global__ void __launch_bounds__(256, 2)
       float kv[8], qv[8];
       unpack8(kw, kv);
       unpack8(qw, qv);
+      if constexpr (kPrep) normalise_rows(kv, qv, s_nrm[0][r], s_nrm[1][r]);
       float o_lk[8], o_lq[8], o_r0[8], o_r1[8], o_r2[8], o_rd[8], o_kb[8], o_xk[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -963,10 +1012,10 @@ inline size_t tc_workspace_bytes(long long max_chunks, int H, int /*N*/) {
 }
 
 inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                   const __nv_bfloat16* v, const float* g, const float* beta,
+                                   const __nv_bfloat16* v, const void* g, const float* beta,
                                    const float* S0, __nv_bfloat16* o, float* S_out,
                                    const int32_t* cu_seqlens, int N, int B, int T, int H,
-                                   long long max_chunks, void* workspace, int gpc, cudaEvent_t* ev,
+                                   long long max_chunks, void* workspace, int gmode, cudaEvent_t* ev,
                                    cudaStream_t stream) {
   (void)B;
   static int s_attr_device = -1;
@@ -975,12 +1024,14 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (s_attr_device != dev) {
-    e = cudaFuncSetAttribute(tc::kda_tc_chunk_local_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::KA_DYN);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc::kda_tc_chunk_local_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::KA_DYN);
-    if (e != cudaSuccess) return e;
+    const void* fns[] = {(const void*)tc::kda_tc_chunk_local_kernel<kGateLogCh>,
+                         (const void*)tc::kda_tc_chunk_local_kernel<kGateLogTok>,
+                         (const void*)tc::kda_tc_chunk_local_kernel<kGateLogitF32>,
+                         (const void*)tc::kda_tc_chunk_local_kernel<kGateLogitBf16>};
+    for (const void* fn : fns) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::KA_DYN);
+      if (e != cudaSuccess) return e;
+    }
     e = cudaFuncSetAttribute(tc::kda_tc_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tc::KB_DYN);
     if (e != cudaSuccess) return e;
@@ -993,12 +1044,17 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   const long long items = max_chunks * H;
   if (items > 0) {
     const int gridA = (int)(items < 2LL * s_sms ? items : 2LL * s_sms);
-    if (gpc)
-      tc::kda_tc_chunk_local_kernel<true><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens,
-                                                                              num_seqs, T, H, items, ws);
-    else
-      tc::kda_tc_chunk_local_kernel<false><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens,
-                                                                               num_seqs, T, H, items, ws);
+#define KDA_TC_LOCAL(M)                                                                            \
+  tc::kda_tc_chunk_local_kernel<M><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens, \
+                                                                       num_seqs, T, H, items, ws)
+    switch (gmode) {
+      case kGateLogCh: KDA_TC_LOCAL(kGateLogCh); break;
+      case kGateLogTok: KDA_TC_LOCAL(kGateLogTok); break;
+      case kGateLogitF32: KDA_TC_LOCAL(kGateLogitF32); break;
+      case kGateLogitBf16: KDA_TC_LOCAL(kGateLogitBf16); break;
+      default: return cudaErrorInvalidValue;
+    }
+#undef KDA_TC_LOCAL
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -28,6 +28,36 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// What the gate argument holds and how it is laid out.
+enum GateMode : int {
+  kGateLogCh = 0,      // log alpha, fp32 [.., H, dk]: one decay per key channel (KDA)
+  kGateLogTok = 1,     // log alpha, fp32 [.., H]: one decay per token and head (Gated DeltaNet)
+  kGateLogitF32 = 2,   // raw logit a, fp32 [.., H, dk]; log alpha = -softplus(a), and the
+                       // call also L2-normalises q, k and takes beta = sigmoid(b)
+  kGateLogitBf16 = 3,  // the same with a in bf16
+};
+__host__ __device__ constexpr bool gate_prep(int m) { return m >= kGateLogitF32; }
+
+// -softplus(a) = -(max(a, 0) + log(1 + e^{-|a|})), finite for every finite a.
+__device__ __forceinline__ float neg_softplus(float a) {
+  return -(fmaxf(a, 0.f) + log1pf(__expf(-fabsf(a))));
+}
+__device__ __forceinline__ float sigmoid_f(float b) { return 1.f / (1.f + __expf(-b)); }
+
+// log alpha of key channel c of token-head row `row` (row = token * H + head).
+__device__ __forceinline__ float gate_log(const void* gate, int mode, size_t row, int DK, int c) {
+  switch (mode) {
+    case kGateLogCh: return static_cast<const float*>(gate)[row * DK + c];
+    case kGateLogTok: return static_cast<const float*>(gate)[row];
+    case kGateLogitF32: return neg_softplus(static_cast<const float*>(gate)[row * DK + c]);
+    default: return neg_softplus(__bfloat162float(static_cast<const __nv_bfloat16*>(gate)[row * DK + c]));
+  }
+}
+// beta of token-head row `row`: given, or sigmoid of the given logit.
+__device__ __forceinline__ float beta_of(const float* beta, int mode, size_t row) {
+  return gate_prep(mode) ? sigmoid_f(beta[row]) : beta[row];
+}
+
 __device__ __forceinline__ float4 f4_scale(float4 a, float s) {
   return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
 }

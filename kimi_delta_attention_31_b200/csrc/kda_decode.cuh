@@ -35,9 +35,9 @@ struct DecodeCfg {
 template <typename TIn, int DK, int DV>
 __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
     kda_decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
-                           const TIn* __restrict__ v, const float* __restrict__ g,
+                           const TIn* __restrict__ v, const void* __restrict__ gate,
                            const float* __restrict__ beta, float* __restrict__ S,
-                           TIn* __restrict__ o, int gpc) {
+                           TIn* __restrict__ o, int gmode) {
   using Cfg = DecodeCfg<TIn, DK, DV>;
   constexpr int DVB = Cfg::DVB, CQ = Cfg::CQ, RG = Cfg::RG, R = Cfg::R, NT = Cfg::NT,
                 NWARP = Cfg::NWARP;
@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
   __shared__ float s_red[2][NWARP][DVB];
   __shared__ float s_e[DVB];
   __shared__ float s_kq;
+  __shared__ float s_nrm[2];
 
   const int unit = blockIdx.x / Cfg::NBLK;  // n * H + h
   const int vb = blockIdx.x % Cfg::NBLK;
@@ -61,9 +62,25 @@ __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
   for (int c = tid; c < DK; c += NT) {
     s_k[c] = to_f32(k[(size_t)unit * DK + c]);
     s_q[c] = to_f32(q[(size_t)unit * DK + c]);
-    s_a[c] = expf(gpc ? g[(size_t)unit * DK + c] : g[unit]);  // per channel, or one gate per head
+    s_a[c] = expf(gate_log(gate, gmode, unit, DK, c));
   }
   __syncthreads();
+  if (gate_prep(gmode)) {  // L2-normalise k and q over dk
+    if (warp < 2) {
+      const float* x = warp == 0 ? s_k : s_q;
+      float acc = 0.f;
+      for (int c = lane; c < DK; c += 32) acc = fmaf(x[c], x[c], acc);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) s_nrm[warp] = rsqrtf(fmaxf(acc, 1e-24f));
+    }
+    __syncthreads();
+    for (int c = tid; c < DK; c += NT) {
+      s_k[c] *= s_nrm[0];
+      s_q[c] *= s_nrm[1];
+    }
+    __syncthreads();
+  }
   if (warp == 0) {  // k . q
     float acc = 0.f;
     for (int c = lane; c < DK; c += 32) acc = fmaf(s_k[c], s_q[c], acc);
@@ -105,7 +122,7 @@ __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
       shat += s_red[1][w][tid];
     }
     const size_t vi = (size_t)unit * DV + vb * DVB + tid;
-    const float e = beta[unit] * (to_f32(v[vi]) - vhat);
+    const float e = beta_of(beta, gmode, unit) * (to_f32(v[vi]) - vhat);
     s_e[tid] = e;
     o[vi] = from_f32<TIn>(fmaf(s_kq, e, shat));
   }
@@ -126,15 +143,15 @@ __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
 }
 
 template <typename TIn, int DK, int DV>
-cudaError_t launch_decode_step(const void* q, const void* k, const void* v, const float* g,
-                               const float* beta, float* S, void* o, int N, int H, int gpc,
+cudaError_t launch_decode_step(const void* q, const void* k, const void* v, const void* gate,
+                               const float* beta, float* S, void* o, int N, int H, int gmode,
                                cudaStream_t stream) {
   using Cfg = DecodeCfg<TIn, DK, DV>;
   const long long grid = (long long)N * H * Cfg::NBLK;
   if (grid == 0) return cudaSuccess;
   kda_decode_step_kernel<TIn, DK, DV><<<(unsigned)grid, Cfg::NT, 0, stream>>>(
-      static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), g, beta,
-      S, static_cast<TIn*>(o), gpc);
+      static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), gate, beta,
+      S, static_cast<TIn*>(o), gmode);
   return cudaGetLastError();
 }
 

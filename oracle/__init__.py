@@ -17,6 +17,9 @@ chunk(...)      chunkwise schedule in fp64 with pairwise exponentials and plain
                 "Linear / sparse attention" tutorial section 6.2).
 gdn_recurrent(...)  Gated DeltaNet (one gate per token and head): the
                 recurrence above with the gate broadcast over key channels.
+prep(...)       input preparation from raw projections (q, k L2-normalised,
+                log alpha = -softplus(a), beta = sigmoid(b)); recurrent_prep
+                chains it with recurrent().
 
 Inputs are widened exactly to fp64 (bf16 and fp32 values are representable),
 so the rounding of the inputs the GPU sees is not counted as error.
@@ -144,6 +147,29 @@ def gdn_recurrent(q, k, v, g, beta, S0=None, cu_seqlens=None, num_threads=0):
         raise ValueError("Gated DeltaNet g must be [B,T,H]")
     g_full = np.ascontiguousarray(np.broadcast_to(g[..., None], g.shape + (dk,)))
     return recurrent(q, k, v, g_full, beta, S0, cu_seqlens, num_threads=num_threads)
+
+
+def prep(q, k, a, b):
+    """Input preparation in fp64, from raw projections ("Kimi K3 notes 1: KDA"
+    section 4: q and k are L2-normalised; "Linear / sparse attention" tutorial
+    section 10: beta and the decay come from bounded activations).  Per token
+    and head:
+        q / max(|q|_2, 1e-12),  k / max(|k|_2, 1e-12)   (over the last axis)
+        g = log alpha = -softplus(a) = -log(1 + e^a)
+        beta = sigmoid(b) = 1 / (1 + e^-b)
+    Returns (q, k, g, beta) as float64 arrays."""
+    q, k, a, b = (_f64(x) for x in (q, k, a, b))
+    q = q / np.maximum(np.linalg.norm(q, axis=-1, keepdims=True), 1e-12)
+    k = k / np.maximum(np.linalg.norm(k, axis=-1, keepdims=True), 1e-12)
+    g = -np.logaddexp(0.0, a)          # log(e^0 + e^a)
+    beta = 0.5 * (1.0 + np.tanh(0.5 * b))  # = 1 / (1 + e^-b), without overflow
+    return q, k, g, beta
+
+
+def recurrent_prep(q, k, v, a, b, S0=None, cu_seqlens=None, num_threads=0):
+    """prep() followed by the token-by-token recurrence.  Returns (o, S_out)."""
+    qn, kn, g, beta = prep(q, k, a, b)
+    return recurrent(qn, kn, v, g, beta, S0, cu_seqlens, num_threads=num_threads)
 
 
 def chunk(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=16, num_threads=0):

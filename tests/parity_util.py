@@ -20,9 +20,9 @@ def seq_bounds(inp, n):
     return n, 0, T
 
 
-def gather_units(inp, units):
+def gather_units(inp, units, names=("q", "k", "v", "g", "beta")):
     """Pack the selected units into a [1, sumT, 1, d] layout with cu_seqlens."""
-    cols = {n: [] for n in ("q", "k", "v", "g", "beta")}
+    cols = {n: [] for n in names}
     S0 = []
     cu = [0]
     for (n, h) in units:
@@ -36,7 +36,8 @@ def gather_units(inp, units):
     packed = {}
     for name, parts in cols.items():
         cat = torch.cat(parts, 0) if parts else torch.zeros(0)
-        packed[name] = cat.unsqueeze(0).unsqueeze(2).numpy() if name != "beta" else cat.reshape(1, -1, 1).numpy()
+        packed[name] = (cat.unsqueeze(0).unsqueeze(2).numpy() if name not in ("beta", "b")
+                        else cat.reshape(1, -1, 1).numpy())
     S0 = torch.stack(S0).unsqueeze(1).numpy() if S0 else None
     return packed, S0, np.array(cu, dtype=np.int64)
 
@@ -49,6 +50,23 @@ def oracle_units(inp, units):
     else:
         o, S = oracle.recurrent(p["q"], p["k"], p["v"], p["g"], p["beta"], S0, cu_seqlens=cu)
     return [(o[0, cu[i]:cu[i + 1], 0], S[i, 0]) for i in range(len(units))]
+
+
+def compare_units_prep(inp, o_gpu, S_gpu, units, tol):
+    """compare_units for raw projections (q, k, v, a, b): the oracle prepares
+    the selected units in fp64, then runs the recurrence."""
+    p, S0, cu = gather_units(inp, units, names=("q", "k", "v", "a", "b"))
+    o, S = oracle.recurrent_prep(p["q"], p["k"], p["v"], p["a"], p["b"], S0, cu_seqlens=cu)
+    worst_o = worst_S = 0.0
+    for i, (n, h) in enumerate(units):
+        b, t0, t1 = seq_bounds(inp, n)
+        if t1 > t0:
+            worst_o = max(worst_o, rel_rms(o_gpu[b, t0:t1, h].float().cpu().numpy(), o[0, cu[i]:cu[i + 1], 0]))
+        worst_S = max(worst_S, rel_rms(S_gpu[n, h].cpu().numpy(), S[i, 0]))
+    assert np.isfinite(worst_o) and np.isfinite(worst_S)
+    assert worst_o <= tol, f"o rel-RMS {worst_o:.3e} > {tol}"
+    assert worst_S <= tol, f"S rel-RMS {worst_S:.3e} > {tol}"
+    return worst_o, worst_S
 
 
 def rel_rms(x, ref):

@@ -127,3 +127,30 @@ def test_binding_checks_gate_shapes():
     # message the binding raises for device tensors, checked on the GPU suite.
     with pytest.raises(ValueError):
         kda.gdn_chunk_fwd(x, x, x, torch.zeros(1, 4, 1), torch.zeros(1, 4, 1))
+
+
+def test_prep_entry_points_validate_arguments():
+    """kda_chunk_fwd_prep / kda_recurrent_step_prep: same checks as the plain
+    entry points, plus the gate-logit dtype; the binding's signatures match."""
+    lib = kda.load_library()
+    f = _fake()
+
+    def chunk(a, a_dt, ws=None):
+        return lib.kda_chunk_fwd_prep(f, f, f, a, a_dt, f, None, _fake(0x2000), _fake(0x3000), None, 0, 1, 64,
+                                      2, 128, 128, 64, kda.KDA_BF16, ws, 0, None)
+
+    assert chunk(f, kda.KDA_BF16) == 4          # reached the workspace check
+    assert "kda_chunk_fwd_prep" in kda.last_error()
+    assert chunk(f, kda.KDA_F32) == 4
+    assert chunk(f, 9) == 2                     # unknown logit dtype
+    assert chunk(_fake(0x1008), kda.KDA_BF16) == 3  # logits need 16-byte alignment here
+    assert chunk(_null(), kda.KDA_F32) == 1
+
+    def step(a, a_dt, dk=64):
+        return lib.kda_recurrent_step_prep(f, f, f, a, a_dt, f, f, f, 4, 2, dk, dk, kda.KDA_BF16, None)
+
+    assert step(f, kda.KDA_BF16, dk=96) == 2
+    assert kda.last_error().startswith("kda_recurrent_step_prep")
+    assert step(_fake(0x1002), kda.KDA_BF16, dk=96) == 2   # shape is checked first
+    assert step(f, 7) == 2
+    assert lib.kda_recurrent_step_prep(f, f, f, f, kda.KDA_F32, f, f, f, 0, 2, 64, 64, 0, None) == 0
