@@ -207,6 +207,17 @@ const char* kda_last_error(void);
 kda_status_t kda_device_error(int* code, cudaStream_t stream);
 
 /*
+ * Self-check of the failure detection (library plumbing: the pages have no
+ * counterpart).  Launches one small kernel on `stream` whose single waiting
+ * thread uses the kernels' own bounded mbarrier wait on a barrier that nothing
+ * ever completes: after limit_ns (1 .. 1e9) of wall time the wait gives up,
+ * sets the device error word to KDA_ERR_DEVICE_TIMEOUT and the kernel returns
+ * normally.  A following kda_device_error() reports and clears it; the
+ * context stays usable.  Nothing faults, traps or hangs.
+ */
+kda_status_t kda_selftest_bounded_wait(unsigned long long limit_ns, cudaStream_t stream);
+
+/*
  * Number of kernels one kda_chunk_fwd call with these arguments launches
  * (1 for the fp32-arithmetic path, more for the tensor-core path).
  */

@@ -37,7 +37,7 @@ KDA_BF16, KDA_F32 = 0, 1
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_last_error", "kda_device_error", "kda_chunk_fwd_launches", "kda_profile_events",
             "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step",
-            "kda_chunk_fwd_prep", "kda_recurrent_step_prep")
+            "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -94,6 +94,8 @@ def load_library():
         lib.kda_profile_events.restype = i32
         lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 9 + [i32] * 7 + [i32, vp]
         lib.kda_chunk_fwd_noalloc.restype = i32
+        lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, vp]
+        lib.kda_selftest_bounded_wait.restype = i32
         lib.kda_version.argtypes = []
         lib.kda_version.restype = i32
         _lib = lib
@@ -260,9 +262,16 @@ def _recurrent_step(fn, q, k, v, g, beta, S, o):
 class HostPrefill:
     """chunk_fwd over pinned HOST tensors: each call copies the inputs to the
     device, runs the prefill and copies o and S_out back into pinned host
-    buffers (all on the current stream).  Device buffers are allocated once."""
+    buffers.  Device buffers are allocated once.
 
-    def __init__(self, like: dict, device="cuda", chunk_size=64):
+    Without cu_seqlens the batch is processed in `pieces` groups of rows: the
+    host->device copy of group p+1 (own stream) overlaps the prefill of group p
+    (the current stream) and the device->host copy of group p-1 (own stream),
+    so the copy engines of both directions and the kernels run together.  The
+    current stream waits for the last copy back, so synchronising it (as the
+    caller does for a one-group call) covers everything."""
+
+    def __init__(self, like: dict, device="cuda", chunk_size=64, pieces=None):
         self.device = torch.device(device)
         self.chunk_size = chunk_size
         self.dev = {n: torch.empty_like(t, device=self.device) for n, t in like.items() if t is not None}
@@ -275,8 +284,13 @@ class HostPrefill:
         self.o_dev = torch.empty_like(self.o_host, device=self.device)
         self.S_dev = torch.empty_like(self.S_host, device=self.device)
         num_seqs = 0 if cu is None else N
-        ws = workspace_size(B, T, H, dk, v.shape[-1], num_seqs, chunk_size, q.dtype)
+        self.pieces = 1 if cu is not None else max(1, min(B, pieces if pieces else 8))
+        rows = -(-B // self.pieces)
+        self.bounds = [(b, min(B, b + rows)) for b in range(0, B, rows)]
+        ws = workspace_size(rows if cu is None else B, T, H, dk, v.shape[-1], num_seqs, chunk_size, q.dtype)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=self.device) if ws else None
+        self.s_in = torch.cuda.Stream(self.device)
+        self.s_out = torch.cuda.Stream(self.device)
 
     def h2d_bytes(self, host: dict) -> int:
         return int(sum(t.numel() * t.element_size() for n, t in host.items() if t is not None and n in self.dev))
@@ -285,14 +299,30 @@ class HostPrefill:
         return int(self.o_host.numel() * self.o_host.element_size() + self.S_host.numel() * 4)
 
     def __call__(self, host: dict):
-        for n, t in host.items():
-            if t is not None and n in self.dev:
-                self.dev[n].copy_(t, non_blocking=True)
+        main = torch.cuda.current_stream(self.device)
         d = self.dev
-        chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("S0"), d.get("cu_seqlens"),
-                  self.chunk_size, o=self.o_dev, S_out=self.S_dev, workspace=self.ws)
-        self.o_host.copy_(self.o_dev, non_blocking=True)
-        self.S_host.copy_(self.S_dev, non_blocking=True)
+        packed = d.get("cu_seqlens") is not None
+        self.s_in.wait_stream(main)   # earlier work on the buffers is done
+        self.s_out.wait_stream(main)
+        for (b0, b1) in self.bounds:
+            rows = slice(None) if packed else slice(b0, b1)
+            with torch.cuda.stream(self.s_in):
+                for n, t in host.items():
+                    if t is not None and n in d:
+                        if n == "cu_seqlens" or packed:
+                            d[n].copy_(t, non_blocking=True)
+                        else:
+                            d[n][rows].copy_(t[rows], non_blocking=True)
+            main.wait_stream(self.s_in)
+            S0 = d.get("S0")
+            chunk_fwd(d["q"][rows], d["k"][rows], d["v"][rows], d["g"][rows], d["beta"][rows],
+                      None if S0 is None else S0[rows], d.get("cu_seqlens"), self.chunk_size,
+                      o=self.o_dev[rows], S_out=self.S_dev[rows], workspace=self.ws)
+            self.s_out.wait_stream(main)
+            with torch.cuda.stream(self.s_out):
+                self.o_host[rows].copy_(self.o_dev[rows], non_blocking=True)
+                self.S_host[rows].copy_(self.S_dev[rows], non_blocking=True)
+        main.wait_stream(self.s_out)
         return self.o_host, self.S_host
 
 
@@ -310,6 +340,14 @@ def device_error(device=None) -> int:
     code = ctypes.c_int(0)
     _check(lib.kda_device_error(ctypes.byref(code), _stream_handle(device)))
     return code.value
+
+
+def selftest_bounded_wait(limit_ns=50_000_000, device=None):
+    """Run the library's bounded-wait self-check on the current stream: a wait
+    that nothing completes gives up after limit_ns and sets the device error
+    word (read it with device_error())."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check(load_library().kda_selftest_bounded_wait(int(limit_ns), _stream_handle(dev)))
 
 
 def launches_per_chunk_fwd(dk, dv, chunk_size, dtype=torch.bfloat16) -> int:

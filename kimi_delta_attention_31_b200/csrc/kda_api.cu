@@ -308,6 +308,34 @@ kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, 
                        chunk_size, dtype, scratch, need, stream);
 }
 
+}  // extern "C"
+
+namespace kda {
+// One thread waits, with the kernels' own bounded wait, on an mbarrier that
+// nothing ever arrives at; the wait gives up after limit_ns and raises the
+// device error word.
+__global__ void kda_bounded_wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+    (void)ptx::mbar_wait_bounded(&bar, 0, limit_ns);
+  }
+}
+}  // namespace kda
+
+extern "C" {
+
+kda_status_t kda_selftest_bounded_wait(unsigned long long limit_ns, cudaStream_t stream) {
+  t_err[0] = 0;
+  if (limit_ns == 0 || limit_ns > 1000000000ull)
+    return fail(KDA_ERR_INVALID_ARG, "kda_selftest_bounded_wait: limit_ns=%llu (need 1 .. 1e9)", limit_ns);
+  kda::kda_bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kda_selftest_bounded_wait launch");
+  return KDA_OK;
+}
+
 kda_status_t kda_device_error(int* code, cudaStream_t stream) {
   t_err[0] = 0;
   if (!code) return fail(KDA_ERR_INVALID_ARG, "kda_device_error: null code");

@@ -154,3 +154,10 @@ def test_prep_entry_points_validate_arguments():
     assert step(_fake(0x1002), kda.KDA_BF16, dk=96) == 2   # shape is checked first
     assert step(f, 7) == 2
     assert lib.kda_recurrent_step_prep(f, f, f, f, kda.KDA_F32, f, f, f, 0, 2, 64, 64, 0, None) == 0
+
+
+def test_selftest_bounded_wait_rejects_bad_limits():
+    lib = kda.load_library()
+    assert lib.kda_selftest_bounded_wait(0, None) == 1
+    assert lib.kda_selftest_bounded_wait(2_000_000_000, None) == 1
+    assert "limit_ns" in kda.last_error()
