@@ -7,7 +7,8 @@ HBM (2.7 GB of inputs: larger than the 126 MB L2, so no flush is needed).
 Beside it: the recurrent decode (256 sequences x 32 heads, in-place fp32
 state, one token per step) as state GB/s, the Gated DeltaNet variant (one
 gate per token and head) on both shapes, the prefill from raw projections
-with the input preparation fused in, the roofline fractions, the fp64
+with the input preparation fused in, one long sequence with few heads
+(split into segments), the roofline fractions, the fp64
 CPU oracle timed on this host's cores, and an end-to-end figure through the
 public host-buffer API (pinned host -> device copies, prefill, copies back).
 
@@ -344,6 +345,40 @@ def prep_leg(kda, args, world, dev, stream, peaks):
     return line
 
 
+def long_seq_leg(kda, args, world, dev, stream):
+    """One long sequence with few heads (B1 H8 T131072): the prefill splits the
+    sequence into segments by itself; beside it the same call with segments
+    turned off."""
+    w = W.LONG_SEQ
+    inp = W.make_workload(w, dev)
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    out = {"workload": w.name, "unit": "tokens/s"}
+    for label, force in (("segmented", 0), ("unsplit", -1)):
+        kda.set_segment_chunks(force)
+        ws = torch.empty(max(kda.workspace_size(B, T, H, dk, dv, 0, w.chunk, torch.bfloat16), 1),
+                         dtype=torch.uint8, device=dev)
+
+        def prefill():
+            kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, None, w.chunk,
+                          o=o, S_out=S_out, workspace=ws)
+
+        for _ in range(args.warmup):
+            prefill()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = max_over_ranks(time_launches(prefill, max(1, min(args.steps, 5)), stream), world, dev)
+        out[label] = {"value": world * B * T / (ms * 1e-3), "ms_per_step": ms,
+                      "segment_chunks": kda.segment_chunks(B, T, H)}
+        del ws
+    kda.set_segment_chunks(0)
+    del inp, o, S_out
+    torch.cuda.empty_cache()
+    out["value"] = out["segmented"]["value"]
+    return out
+
+
 def run_ours(args):
     import kimi_delta_attention_31_b200 as kda
     rank, world, local = dist_setup(args.gpus)
@@ -462,6 +497,8 @@ def run_ours(args):
     gdn = gdn_leg(kda, args, world, dev, stream, peaks)
     # ---------------- fused input preparation from raw projections ----------------
     prep = prep_leg(kda, args, world, dev, stream, peaks)
+    # ---------------- one long sequence, few heads (sequence segments) ----------------
+    long_seq = long_seq_leg(kda, args, world, dev, stream)
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only) ----------------
     cpu = None
@@ -478,6 +515,7 @@ def run_ours(args):
                        "l2": "inputs (2.7 GB) larger than L2; no flush",
                        "parallelism": f"dp{world} (independent batches per GPU)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "gdn": gdn, "prep": prep,
+            "long_seq": long_seq,
             "gpu_launches": gpu_launches, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -218,17 +218,41 @@ kda_status_t kda_device_error(int* code, cudaStream_t stream);
 kda_status_t kda_selftest_bounded_wait(unsigned long long limit_ns, cudaStream_t stream);
 
 /*
- * Number of kernels one kda_chunk_fwd call with these arguments launches
- * (1 for the fp32-arithmetic path, more for the tensor-core path).
+ * Sequence parallelism of the tensor-core prefill (across the chunks of one
+ * sequence).  The state pass is linear in the state, so a segment of L chunks
+ * maps its entry state as S -> M S + N ("Linear / sparse attention" tutorial
+ * section 6.2: the state handed from chunk to chunk; composing those hand-offs
+ * is exact algebra).  When the (sequence, head) units are too few to fill the
+ * GPU and the sequences are long, kda_chunk_fwd (and its _gdn / _prep forms)
+ * splits each sequence into segments: the maps of all segments are formed in
+ * parallel, chained from S0 in fp32, and every segment is then run from its
+ * entry state.  Packed (cu_seqlens) inputs are not split.  The workspace size
+ * accounts for it.
+ *
+ * kda_set_segment_chunks: for the calling thread's later calls (including
+ * kda_chunk_fwd_workspace_size), 0 = choose automatically (default), L > 0 =
+ * segments of L chunks whenever a sequence has more than L chunks, < 0 = never
+ * split.  kda_segment_chunks returns the choice for these sizes on the
+ * current device (0 = not split).
+ */
+kda_status_t kda_set_segment_chunks(int chunks);
+int kda_segment_chunks(int B, int T, int H, int num_seqs);
+
+/*
+ * Number of phases one kda_chunk_fwd call with these arguments runs: 1 for
+ * the fp32-arithmetic path (one kernel); 2 for the tensor-core path (the
+ * chunk-local kernel, then the state pass -- one kernel, or three when the
+ * sequences are split into segments).
  */
 int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype);
 
 /*
  * Measurement hook.  While set (events != NULL), each later kda_chunk_fwd,
- * kda_gdn_chunk_fwd or kda_chunk_fwd_prep call made by the calling thread records events[0] before its first kernel
- * launch and events[i] after its i-th launch, on the call's stream; count
- * must be at least kda_chunk_fwd_launches(...) + 1 or the call fails with
- * KDA_ERR_INVALID_ARG.  The caller owns the events.  Pass NULL, 0 to stop.
+ * kda_gdn_chunk_fwd or kda_chunk_fwd_prep call made by the calling thread
+ * records events[0] before its first kernel launch and events[i] after its
+ * i-th phase, on the call's stream; count must be at least
+ * kda_chunk_fwd_launches(...) + 1 or the call fails with KDA_ERR_INVALID_ARG.
+ * The caller owns the events.  Pass NULL, 0 to stop.
  */
 kda_status_t kda_profile_events(cudaEvent_t* events, int count);
 

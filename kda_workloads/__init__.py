@@ -93,8 +93,13 @@ GDN_DECODE = Workload("gdn_decode_bf16_N256_H32_d128_1024steps", 256, 1024, 32, 
 PREP_PREFILL_B8 = Workload("kda_prefill_prep_bf16logits_B8_H32_T8192_d128", 8, 8192, 32, 128, 128, "bf16",
                            -5.0, 1.5, 0.0, 64, 1007, raw_a_dtype="bf16")
 
+# One long sequence with few heads: too few (sequence, head) units for the GPU,
+# the case sequence segments exist for.
+LONG_SEQ = Workload("kda_prefill_bf16_B1_H8_T131072_d128", 1, 131072, 8, 128, 128, "bf16",
+                    -5.0, 1.5, 0.0, 64, 1008)
+
 WORKLOADS = {w.name: w for w in (ORACLE_SMALL, PREFILL_H16, PREFILL_B8, PREFILL_VARLEN, DECODE,
-                                 GDN_PREFILL_B8, GDN_DECODE, PREP_PREFILL_B8)}
+                                 GDN_PREFILL_B8, GDN_DECODE, PREP_PREFILL_B8, LONG_SEQ)}
 
 
 def cu_seqlens_of(lengths, device="cpu") -> torch.Tensor:
@@ -215,5 +220,5 @@ def describe(w: Workload) -> str:
 
 
 __all__ = ["Workload", "WORKLOADS", "ORACLE_SMALL", "PREFILL_H16", "PREFILL_B8", "PREFILL_VARLEN",
-           "DECODE", "GDN_PREFILL_B8", "GDN_DECODE", "PREP_PREFILL_B8", "make_prefill_raw", "make_prefill", "make_workload", "make_decode_state", "make_decode_steps",
+           "DECODE", "GDN_PREFILL_B8", "GDN_DECODE", "PREP_PREFILL_B8", "LONG_SEQ", "make_prefill_raw", "make_prefill", "make_workload", "make_decode_state", "make_decode_steps",
            "cu_seqlens_of", "varlen_lengths", "bytes_of", "describe"]

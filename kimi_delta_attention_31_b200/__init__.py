@@ -37,7 +37,8 @@ KDA_BF16, KDA_F32 = 0, 1
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
             "kda_last_error", "kda_device_error", "kda_chunk_fwd_launches", "kda_profile_events",
             "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step",
-            "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait")
+            "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait",
+            "kda_set_segment_chunks", "kda_segment_chunks")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -94,6 +95,10 @@ def load_library():
         lib.kda_profile_events.restype = i32
         lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 9 + [i32] * 7 + [i32, vp]
         lib.kda_chunk_fwd_noalloc.restype = i32
+        lib.kda_set_segment_chunks.argtypes = [i32]
+        lib.kda_set_segment_chunks.restype = i32
+        lib.kda_segment_chunks.argtypes = [i32] * 4
+        lib.kda_segment_chunks.restype = i32
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, vp]
         lib.kda_selftest_bounded_wait.restype = i32
         lib.kda_version.argtypes = []
@@ -340,6 +345,17 @@ def device_error(device=None) -> int:
     code = ctypes.c_int(0)
     _check(lib.kda_device_error(ctypes.byref(code), _stream_handle(device)))
     return code.value
+
+
+def set_segment_chunks(chunks: int) -> None:
+    """Sequence segments of the tensor-core prefill for this thread's later
+    calls: 0 = automatic (default), L > 0 = L chunks per segment, < 0 = off."""
+    _check(load_library().kda_set_segment_chunks(int(chunks)))
+
+
+def segment_chunks(B, T, H, num_seqs=0) -> int:
+    """Chunks per segment the prefill would use for these sizes (0 = none)."""
+    return int(load_library().kda_segment_chunks(B, T, H, num_seqs))
 
 
 def selftest_bounded_wait(limit_ns=50_000_000, device=None):

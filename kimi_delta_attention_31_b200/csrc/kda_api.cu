@@ -16,6 +16,14 @@ namespace {
 thread_local char t_err[512] = "";
 thread_local cudaEvent_t* t_prof_events = nullptr;
 thread_local int t_prof_count = 0;
+thread_local int t_seg_force = 0;  // kda_set_segment_chunks: 0 auto, > 0 fixed, < 0 never
+
+int current_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
 
 kda_status_t fail(kda_status_t st, const char* fmt, ...) {
   va_list ap;
@@ -122,11 +130,12 @@ kda_status_t chunk_fwd_impl(const char* fn, const void* q, const void* k, const 
     if (need && (!workspace || workspace_bytes < need))
       return fail(KDA_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes,
                   need);
+    const int seg = kda::tc_segment_chunks(B, T, H, num_seqs, current_sms(), t_seg_force);
     e = kda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
                              static_cast<const __nv_bfloat16*>(k),
                              static_cast<const __nv_bfloat16*>(v), g, beta, S0,
                              static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H,
-                             max_chunks(B, T, num_seqs, chunk_size), workspace, gmode, ev, stream);
+                             max_chunks(B, T, num_seqs, chunk_size), workspace, gmode, seg, ev, stream);
   } else if (dtype == KDA_F32) {
     e = dispatch_chunk_simt<float>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, T,
                                    H, dv, gmode, stream);
@@ -179,6 +188,16 @@ int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype) {
   return use_tensor_core_path(dk, dv, chunk_size, dtype) ? kda::kTcLaunches : 1;
 }
 
+kda_status_t kda_set_segment_chunks(int chunks) {
+  t_err[0] = 0;
+  t_seg_force = chunks;
+  return KDA_OK;
+}
+
+int kda_segment_chunks(int B, int T, int H, int num_seqs) {
+  return kda::tc_segment_chunks(B, T, H, num_seqs, current_sms(), t_seg_force);
+}
+
 kda_status_t kda_profile_events(cudaEvent_t* events, int count) {
   t_err[0] = 0;
   if (events && count <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_profile_events: count=%d", count);
@@ -192,7 +211,8 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
   if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || chunk_size <= 0) return 0;
   if (!use_tensor_core_path(dk, dv, chunk_size, dtype)) return 0;
   const int N = num_seqs > 0 ? num_seqs : B;
-  return kda::tc_workspace_bytes(max_chunks(B, T, num_seqs, chunk_size), H, N);
+  const int seg = kda::tc_segment_chunks(B, T, H, num_seqs, current_sms(), t_seg_force);
+  return kda::tc_workspace_layout(max_chunks(B, T, num_seqs, chunk_size), H, (long long)N * H, T, seg).total;
 }
 
 kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,

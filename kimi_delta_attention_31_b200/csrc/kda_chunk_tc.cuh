@@ -36,6 +36,7 @@
 // (= k_j / a_j).  The only factor above 1 is e^{-(block log-decay)}, finite as
 // long as every channel's log-decay over one 16-token block is >= -80.
 #pragma once
+#include <algorithm>
 #include "kda_common.cuh"
 #include "tc_ptx.cuh"
 
@@ -774,6 +775,47 @@ __global__ void __launch_bounds__(256, 2)
 // Kernel 2: the state pass.  Persistent; CTA b handles units b, b + grid, ...
 // Thread t: state row c = 32 (warp mod 4) + lane, columns 64 (warp / 4) + [0, 64).
 // ---------------------------------------------------------------------------
+// State-pass passes.  A sequence split into segments of L chunks: the map
+// pass runs, for every segment but the last, the linear part M (state from I,
+// no U term) and the offset N (state from 0) of the segment's affine map
+// S -> M S + N; the combine kernel chains S0 through the maps; the final pass
+// runs every segment from its entry state and writes the outputs.
+constexpr int kPassPlain = 0, kPassMaps = 1, kPassFinal = 2;
+
+// Entry states of the segments: S_{p+1} = M_p S_p + N_p, in fp32.  One CTA per
+// (unit, 8-column block); thread t owns row t / 2, columns 4 (t mod 2) .. + 3.
+__global__ void __launch_bounds__(256)
+    kda_tc_seg_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
+                              float* __restrict__ seg_init, int P) {
+  __shared__ __align__(16) float Ss[D][8];
+  const long long u = blockIdx.x / (D / 8);
+  const int j0 = (blockIdx.x % (D / 8)) * 8;
+  const int tid = threadIdx.x, c = tid >> 1, jq = 4 * (tid & 1);
+  float4 cur = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)u * D + c) * D + j0 + jq)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  *reinterpret_cast<float4*>(&Ss[c][jq]) = cur;
+  __syncthreads();
+  for (int p = 0; p + 1 < P; ++p) {
+    const float* Nm = maps + (size_t)((u * (P - 1) + p) * 2) * D * D;
+    const float* Mrow = Nm + (size_t)D * D + (size_t)c * D;
+    float4 acc = *reinterpret_cast<const float4*>(Nm + (size_t)c * D + j0 + jq);
+#pragma unroll 4
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      const float4 m = reinterpret_cast<const float4*>(Mrow)[k4];
+      const float mk[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 sv = *reinterpret_cast<const float4*>(&Ss[4 * k4 + e][jq]);
+        acc = f4_fma(mk[e], sv, acc);
+      }
+    }
+    __syncthreads();  // every read of the old state is done
+    *reinterpret_cast<float4*>(&Ss[c][jq]) = acc;
+    *reinterpret_cast<float4*>(seg_init + ((size_t)(u * P + p + 1) * D + c) * D + j0 + jq) = acc;
+    __syncthreads();
+  }
+}
+
 __device__ __forceinline__ void store_state_bf16(uint8_t* sm, int c, int ch, const float* S) {
 #pragma unroll
   for (int k8 = 0; k8 < 8; ++k8)
@@ -783,7 +825,9 @@ __device__ __forceinline__ void store_state_bf16(uint8_t* sm, int c, int ch, con
 __global__ void __launch_bounds__(256, 1)
     kda_tc_state_pass_kernel(const uint8_t* __restrict__ ws, const float* __restrict__ S0,
                              float* __restrict__ S_out, bf16* __restrict__ o,
-                             const int32_t* __restrict__ cu_seqlens, int N, int T, int H) {
+                             const int32_t* __restrict__ cu_seqlens, int N, int T, int H,
+                             int seg_chunks, int pass, float* __restrict__ maps,
+                             const float* __restrict__ seg_init) {
   __shared__ __align__(8) uint64_t s_full[2];
   __shared__ __align__(8) uint64_t s_xbar;
   __shared__ __align__(8) uint64_t s_ybar;
@@ -831,12 +875,33 @@ __global__ void __launch_bounds__(256, 1)
   uint32_t it = 0;          // chunks consumed by this CTA; stage = it & 1
   int pending_stage = -1;   // stage with a copy in flight not yet waited for
   const long long units = (long long)N * H;
+  // Sequence segments (unpacked layout only): P segments of seg_chunks chunks.
+  const long long ncps = (T + C - 1) / C;
+  const int P = seg_chunks > 0 ? (int)((ncps + seg_chunks - 1) / seg_chunks) : 1;
+  const long long items = pass == kPassMaps ? units * (P - 1) * 2 : units * P;
   bool aborted = false;
-  for (long long u = blockIdx.x; u < units && !aborted; u += gridDim.x) {
+  for (long long item = blockIdx.x; item < items && !aborted; item += gridDim.x) {
+    // kind 1: the linear part M of a segment's map (state from I, no U term);
+    // kind 0: its offset N (state from 0), or an ordinary run.
+    long long u;
+    int p = 0, kind = 0;
+    if (pass == kPassMaps) {
+      kind = (int)(item & 1);
+      const long long r = item >> 1;
+      p = (int)(r % (P - 1));
+      u = r / (P - 1);
+    } else {
+      p = (int)(item % P);
+      u = item / P;
+    }
     const int n = (int)(u / H), h = (int)(u % H);
     long long first, start;
     int len;
-    if (cu_seqlens) {
+    if (seg_chunks > 0) {
+      first = (long long)n * ncps + (long long)p * seg_chunks;
+      start = (long long)n * T + (long long)p * seg_chunks * C;
+      len = (int)min((long long)seg_chunks * C, (long long)T - (long long)p * seg_chunks * C);
+    } else if (cu_seqlens) {
       if (warp == 0) {
         const long long f = chunks_before_warp(cu_seqlens, n);
         if (lane == 0) {
@@ -856,11 +921,17 @@ __global__ void __launch_bounds__(256, 1)
     }
     const int nc = (len + C - 1) / C;
     const size_t soff = ((size_t)u * D + c) * D + 64 * ch;
+    const float* S_src = nullptr;
+    if (pass == kPassFinal && p > 0)
+      S_src = seg_init + ((size_t)(u * P + p) * D + c) * D + 64 * ch;
+    else if (pass != kPassMaps && S0)
+      S_src = S0 + soff;
+    const bool no_u = pass == kPassMaps && kind == 1;
     float S[64];
-    if (S0) {
+    if (S_src) {
 #pragma unroll
       for (int j4 = 0; j4 < 16; ++j4) {
-        const float4 t = reinterpret_cast<const float4*>(S0 + soff)[j4];
+        const float4 t = reinterpret_cast<const float4*>(S_src)[j4];
         S[4 * j4] = t.x;
         S[4 * j4 + 1] = t.y;
         S[4 * j4 + 2] = t.z;
@@ -868,7 +939,7 @@ __global__ void __launch_bounds__(256, 1)
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) S[j] = 0.f;
+      for (int j = 0; j < 64; ++j) S[j] = (no_u && 64 * ch + j == c) ? 1.f : 0.f;
     }
     store_state_bf16(sm, c, ch, S);
     ptx::fence_proxy_async_smem();
@@ -895,18 +966,20 @@ __global__ void __launch_bounds__(256, 1)
         if (!ptx::mbar_wait_bounded(&s_full[st], (it >> 1) & 1)) s_abort = 1;
         pending_stage = (cc + 1 < nc) ? (st ^ 1) : -1;
         ptx::tc_fence_after();
-        // X = [-I; 0] U  (M=128, N=128, K=64, both K-major)
+        // X = [-I; 0] U  (M=128, N=128, K=64, both K-major); left out for a map's M part
         constexpr uint32_t id0 = ptx::idesc_bf16(128, 128, false, false);
+        if (!no_u) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_bf16(tX, ptx::sdesc_sw128(sb + KB_NEGI + kk * 32, 16, 1024),
-                        ptx::sdesc_sw128(sst + IMG_U + kk * 32, 16, 1024), id0, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_bf16(tX, ptx::sdesc_sw128(sb + KB_NEGI + kk * 32, 16, 1024),
+                          ptx::sdesc_sw128(sst + IMG_U + kk * 32, 16, 1024), id0, kk > 0);
+        }
         // X += [W; Q e^G] S  (M=128, N=128, K=128, both MN-major)
         constexpr uint32_t id1 = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + IMG_A1 + kk * 2048, 16384, 1024),
-                        ptx::sdesc_sw128(sb + KB_SB + kk * 2048, 16384, 1024), id1, 1);
+                        ptx::sdesc_sw128(sb + KB_SB + kk * 2048, 16384, 1024), id1, kk > 0 || !no_u);
         ptx::mma_commit(&s_xbar);
       }
       if (!ptx::mbar_wait_bounded(&s_xbar, it & 1)) s_abort = 1;
@@ -942,12 +1015,15 @@ __global__ void __launch_bounds__(256, 1)
           ptx::mma_bf16(tY, ptx::sdesc_sw128(sst + IMG_KB + kk * 2048, 8192, 1024),
                         ptx::sdesc_sw128(sb + KB_E + kk * 2048, 8192, 1024), id2, kk > 0);
         // X += [*; P] E: rows 64..127 become O = Q e^G S + P E (rows 0..63 are dead);
-        // A = the 8 KB in front of P (unused rows) followed by P, K-major [128][64]
+        // A = the 8 KB in front of P (unused rows) followed by P, K-major [128][64].
+        // The map pass writes no output.
         constexpr uint32_t id3 = ptx::idesc_bf16(128, 128, false, true);
+        if (pass != kPassMaps) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + IMG_P - 8192 + kk * 32, 16, 1024),
-                        ptx::sdesc_sw128(sb + KB_E + kk * 2048, 8192, 1024), id3, 1);
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + IMG_P - 8192 + kk * 32, 16, 1024),
+                          ptx::sdesc_sw128(sb + KB_E + kk * 2048, 8192, 1024), id3, 1);
+        }
         ptx::mma_commit(&s_ybar);
       }
       if (!ptx::mbar_wait_bounded(&s_ybar, it & 1)) s_abort = 1;
@@ -964,7 +1040,7 @@ __global__ void __launch_bounds__(256, 1)
       }
       store_state_bf16(sm, c, ch, S);
       // rows 64..127 of X: the chunk's outputs
-      if (qd >= 2) {
+      if (qd >= 2 && pass != kPassMaps) {
         const int r = c - 64;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -988,11 +1064,15 @@ __global__ void __launch_bounds__(256, 1)
         break;
       }
     }
-    if (!aborted && S_out) {
+    float* S_dst = nullptr;
+    if (pass == kPassMaps)
+      S_dst = maps + ((size_t)((u * (P - 1) + p) * 2 + kind) * D + c) * D + 64 * ch;
+    else if (S_out && p == P - 1)
+      S_dst = S_out + soff;
+    if (!aborted && S_dst) {
 #pragma unroll
       for (int j4 = 0; j4 < 16; ++j4)
-        reinterpret_cast<float4*>(S_out + soff)[j4] =
-            make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+        reinterpret_cast<float4*>(S_dst)[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
     }
   }
   // a copy still in flight after an abort must land before shared memory is released
@@ -1007,17 +1087,59 @@ __global__ void __launch_bounds__(256, 1)
 
 }  // namespace tc
 
-inline size_t tc_workspace_bytes(long long max_chunks, int H, int /*N*/) {
-  return (size_t)max_chunks * (size_t)H * tc::IMG_BYTES;
+// Chunks per sequence segment for the state pass, or 0 for none.  Segments
+// pay off when the (sequence, head) units are too few to fill the SMs and
+// each sequence is long: the serial chain of one unit then bounds the time.
+// Model, in chunk-step times: unsegmented ceil(units / sms) * nc; segmented
+// (P segments of L chunks) ceil(2 units (P-1) / sms) L for the maps,
+// ceil(units P / sms) L for the final pass, plus P for the combine.
+// `force` > 0 fixes L, < 0 disables segments; packed layouts are never split.
+inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int force) {
+  if (num_seqs > 0 || force < 0 || B <= 0 || T <= 0 || sms <= 0) return 0;
+  const long long nc = (T + tc::C - 1) / tc::C;
+  if (force > 0) return force < nc ? force : 0;
+  const long long units = (long long)B * H;
+  if (2 * units > sms || nc < 128) return 0;
+  auto waves = [&](long long n) { return (n + sms - 1) / sms; };
+  long long best_cost = waves(units) * nc;
+  int best_L = 0;
+  const long long pmax = std::min<long long>(nc / 16, 8LL * sms / units);
+  for (long long P = 2; P <= pmax; ++P) {
+    const long long L = (nc + P - 1) / P, Pe = (nc + L - 1) / L;
+    const long long cost = waves(2 * units * (Pe - 1)) * L + waves(units * Pe) * L + Pe;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best_L = (int)L;
+    }
+  }
+  return best_L;
+}
+
+// Workspace: the per-chunk images, then (segmented runs) the maps [N | M] of
+// every segment but the last and the entry state of every segment, fp32.
+struct TcWorkspace {
+  size_t images, maps, seg_init, total;
+};
+inline TcWorkspace tc_workspace_layout(long long max_chunks, int H, long long units, int T, int seg_chunks) {
+  TcWorkspace w{};
+  w.images = (size_t)max_chunks * (size_t)H * tc::IMG_BYTES;
+  w.maps = w.seg_init = w.total = (w.images + 255) & ~(size_t)255;
+  if (seg_chunks > 0) {
+    const long long nc = (T + tc::C - 1) / tc::C;
+    const long long P = (nc + seg_chunks - 1) / seg_chunks;
+    const size_t mat = (size_t)tc::D * tc::D * sizeof(float);
+    w.seg_init = w.maps + (size_t)units * (size_t)(P - 1) * 2 * mat;
+    w.total = w.seg_init + (size_t)units * (size_t)P * mat;
+  }
+  return w;
 }
 
 inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* k,
                                    const __nv_bfloat16* v, const void* g, const float* beta,
                                    const float* S0, __nv_bfloat16* o, float* S_out,
                                    const int32_t* cu_seqlens, int N, int B, int T, int H,
-                                   long long max_chunks, void* workspace, int gmode, cudaEvent_t* ev,
-                                   cudaStream_t stream) {
-  (void)B;
+                                   long long max_chunks, void* workspace, int gmode, int seg_chunks,
+                                   cudaEvent_t* ev, cudaStream_t stream) {
   static int s_attr_device = -1;
   static int s_sms = 0;
   int dev = 0;
@@ -1060,10 +1182,26 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   }
   if (ev && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
   const long long units = (long long)N * H;
-  if (units > 0) {
+  if (units > 0 && seg_chunks > 0 && !cu_seqlens) {
+    // segmented: maps of every segment but the last, entry states, final pass
+    const TcWorkspace lay = tc_workspace_layout(max_chunks, H, units, T, seg_chunks);
+    float* maps = reinterpret_cast<float*>(ws + lay.maps);
+    float* seg_init = reinterpret_cast<float*>(ws + lay.seg_init);
+    const long long nc = (T + tc::C - 1) / tc::C;
+    const int P = (int)((nc + seg_chunks - 1) / seg_chunks);
+    const long long map_items = units * (P - 1) * 2, fin_items = units * P;
+    tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(map_items, s_sms), 256, tc::KB_DYN, stream>>>(
+        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassMaps, maps, seg_init);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    tc::kda_tc_seg_combine_kernel<<<(unsigned)(units * (tc::D / 8)), 256, 0, stream>>>(maps, S0, seg_init, P);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(fin_items, s_sms), 256, tc::KB_DYN, stream>>>(
+        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassFinal, maps, seg_init);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else if (units > 0) {
     const int gridB = (int)(units < s_sms ? units : s_sms);
-    tc::kda_tc_state_pass_kernel<<<gridB, 256, tc::KB_DYN, stream>>>(ws, S0, S_out, o, cu_seqlens, N, T,
-                                                                      H);
+    tc::kda_tc_state_pass_kernel<<<gridB, 256, tc::KB_DYN, stream>>>(ws, S0, S_out, o, cu_seqlens, N, T, H, 0,
+                                                                      tc::kPassPlain, nullptr, nullptr);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
