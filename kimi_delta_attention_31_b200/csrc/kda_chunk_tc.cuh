@@ -76,16 +76,18 @@ constexpr uint32_t KA_BV = 90112;   // V        MN-major 2 panels [64][64]      
 constexpr uint32_t KA_BYTES = 106496;
 constexpr uint32_t KA_DYN = KA_BYTES + 1024;
 
-// state-pass kernel shared memory.  [-I; 0] is a constant K-major [128][64]
-// operand; the two image stages follow it, so that the 8 KB in front of each
-// stage's P (the zero half, or the tail of stage 0) can serve as the unused
-// upper half of the [*; P] operand.
-constexpr uint32_t KB_NEGI = 0;             // [-I; 0] K-major [128 rows][64 K]        16384
-constexpr uint32_t KB_STAGE0 = 16384;       // image stages                     2 x 75776
-constexpr uint32_t KB_STAGE = 75776;
-constexpr uint32_t KB_SB = KB_STAGE0 + 2 * KB_STAGE;  // S bf16 MN-major 2 panels [128][64] 32768
-constexpr uint32_t KB_E = KB_SB + 32768;    // E bf16 MN-major 2 panels [64][64]         16384
-constexpr uint32_t KB_BYTES = KB_E + 16384;
+// state-pass kernel shared memory (two CTAs per SM).  The image arrives in
+// three parts, each reloaded as soon as its last reader is done: [W; Q e^G]
+// (read by the first MMA), U^T (read by the first epilogue, then overwritten
+// by E), and P + Kbar + gamma (read by the second MMA group).  P sits right
+// after the state operand, whose last 8 KB serve as the unused upper half of
+// the [*; P] operand.
+constexpr uint32_t KB_SB = 0;        // S bf16 MN-major 2 panels [128 dk][64 dv]          32768
+constexpr uint32_t KB_P = 32768;     // P K-major [64 r][64 j]                             8192
+constexpr uint32_t KB_UE = 40960;    // U^T K-major [128 dv][64 j], then E MN-major 2 x [64 j][64 dv] 16384
+constexpr uint32_t KB_WQ = 57344;    // [W; Q e^G] MN-major 2 panels [128 dk][64 tok]      32768
+constexpr uint32_t KB_KG = 90112;    // Kbar MN-major 2 panels [64 tok][64 dk], gamma fp32 [128] 16896
+constexpr uint32_t KB_BYTES = KB_KG + 16896;
 constexpr uint32_t KB_DYN = KB_BYTES + 1024;
 
 // 1024-byte aligned start inside the dynamic shared buffer.  Offsetting the
@@ -816,21 +818,15 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-__device__ __forceinline__ void store_state_bf16(uint8_t* sm, int c, int ch, const float* S) {
-#pragma unroll
-  for (int k8 = 0; k8 < 8; ++k8)
-    *reinterpret_cast<uint4*>(sm + KB_SB + ch * 16384 + ptx::sw128_chunk(c, k8)) = pack8(S + 8 * k8);
-}
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
     kda_tc_state_pass_kernel(const uint8_t* __restrict__ ws, const float* __restrict__ S0,
                              float* __restrict__ S_out, bf16* __restrict__ o,
                              const int32_t* __restrict__ cu_seqlens, int N, int T, int H,
                              int seg_chunks, int pass, float* __restrict__ maps,
                              const float* __restrict__ seg_init) {
-  __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ __align__(8) uint64_t s_xbar;
-  __shared__ __align__(8) uint64_t s_ybar;
+  __shared__ __align__(8) uint64_t s_full[3];  // image parts: 0 [W; Q e^G], 1 U^T, 2 P + Kbar + gamma
+  __shared__ __align__(8) uint64_t s_mma1, s_mma2;
   __shared__ uint32_t s_tmem;
   __shared__ long long s_u_first, s_u_start;
   __shared__ int s_u_len;
@@ -841,14 +837,13 @@ __global__ void __launch_bounds__(256, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, ch = warp >> 2;
-  const int c = 32 * qd + lane;
+  const int c = 32 * qd + lane;  // state row; rows 0..63 of X are tokens (-E), 64..127 outputs
   const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
 
   if (tid == 0) {
-    ptx::mbar_init(&s_full[0], 1);
-    ptx::mbar_init(&s_full[1], 1);
-    ptx::mbar_init(&s_xbar, 1);
-    ptx::mbar_init(&s_ybar, 1);
+    for (int i = 0; i < 3; ++i) ptx::mbar_init(&s_full[i], 1);
+    ptx::mbar_init(&s_mma1, 1);
+    ptx::mbar_init(&s_mma2, 1);
     ptx::fence_mbar_init();
     s_abort = 0;
   }
@@ -856,26 +851,16 @@ __global__ void __launch_bounds__(256, 1)
     ptx::tmem_alloc(&s_tmem, 256);
     ptx::tmem_relinquish();
   }
-  // constant [-I; 0] operand (K-major [128 rows][64 K]; bf16 -1.0 = 0xBF80)
-  for (int idx = tid; idx < 1024; idx += 256) {
-    const int row = idx >> 3, chunk = idx & 7;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (row < 64 && (row >> 3) == chunk) {
-      const int e = row & 7;
-      w[e >> 1] = (e & 1) ? 0xBF800000u : 0x0000BF80u;
-    }
-    *reinterpret_cast<uint4*>(sm + KB_NEGI + ptx::sw128_chunk(row, chunk)) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tX = s_tmem, tY = s_tmem + 128;
+  // TMEM: X (columns 0..127) and the fp32 state S (columns 128..255), lane = row.
+  const uint32_t tX = s_tmem, tS = s_tmem + 128;
+  const uint32_t tXr = tX + lane_off + 64 * ch, tSr = tS + lane_off + 64 * ch;
 
-  uint32_t it = 0;          // chunks consumed by this CTA; stage = it & 1
-  int pending_stage = -1;   // stage with a copy in flight not yet waited for
+  uint32_t it = 0;  // chunks processed by this CTA: every barrier completes once per chunk
+  bool pend[3] = {false, false, false};  // (thread 0) a load in flight not yet waited for
   const long long units = (long long)N * H;
-  // Sequence segments (unpacked layout only): P segments of seg_chunks chunks.
   const long long ncps = (T + C - 1) / C;
   const int P = seg_chunks > 0 ? (int)((ncps + seg_chunks - 1) / seg_chunks) : 1;
   const long long items = pass == kPassMaps ? units * (P - 1) * 2 : units * P;
@@ -914,8 +899,9 @@ __global__ void __launch_bounds__(256, 1)
       first = s_u_first;
       start = s_u_start;
       len = s_u_len;
+      __syncthreads();  // read before warp 0 rewrites them for the next item
     } else {
-      first = (long long)n * ((T + C - 1) / C);
+      first = (long long)n * ncps;
       start = (long long)n * T;
       len = T;
     }
@@ -927,127 +913,157 @@ __global__ void __launch_bounds__(256, 1)
     else if (pass != kPassMaps && S0)
       S_src = S0 + soff;
     const bool no_u = pass == kPassMaps && kind == 1;
-    float S[64];
-    if (S_src) {
+
+    // initial state: fp32 into TMEM, bf16 into the MMA operand
 #pragma unroll
-      for (int j4 = 0; j4 < 16; ++j4) {
-        const float4 t = reinterpret_cast<const float4*>(S_src)[j4];
-        S[4 * j4] = t.x;
-        S[4 * j4 + 1] = t.y;
-        S[4 * j4 + 2] = t.z;
-        S[4 * j4 + 3] = t.w;
+    for (int q4 = 0; q4 < 4; ++q4) {
+      float x[16];
+      if (S_src) {
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+          const float4 t = reinterpret_cast<const float4*>(S_src)[4 * q4 + j4];
+          x[4 * j4] = t.x; x[4 * j4 + 1] = t.y; x[4 * j4 + 2] = t.z; x[4 * j4 + 3] = t.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = (no_u && 64 * ch + 16 * q4 + e == c) ? 1.f : 0.f;
       }
-    } else {
+      ptx::tmem_st16(tSr + 16 * q4, x);
 #pragma unroll
-      for (int j = 0; j < 64; ++j) S[j] = (no_u && 64 * ch + j == c) ? 1.f : 0.f;
+      for (int k8 = 0; k8 < 2; ++k8)
+        *reinterpret_cast<uint4*>(sm + KB_SB + ch * 16384 + ptx::sw128_chunk(c, 2 * q4 + k8)) = pack8(x + 8 * k8);
     }
-    store_state_bf16(sm, c, ch, S);
+    ptx::tmem_wait_st();
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
 
-    auto issue = [&](long long chunk_idx, int stage) {
-      ptx::mbar_arrive_expect_tx(&s_full[stage], IMG_BYTES);
-      ptx::bulk_g2s(sm + KB_STAGE0 + stage * KB_STAGE, ws + ((size_t)chunk_idx * H + h) * IMG_BYTES,
-                    IMG_BYTES, &s_full[stage]);
+    auto img_of = [&](long long chunk_idx) { return ws + ((size_t)chunk_idx * H + h) * IMG_BYTES; };
+    auto load_wq = [&](long long ci) {
+      ptx::mbar_arrive_expect_tx(&s_full[0], 32768);
+      ptx::bulk_g2s(sm + KB_WQ, img_of(ci) + IMG_A1, 32768, &s_full[0]);
+      pend[0] = true;
+    };
+    auto load_ue_pk = [&](long long ci) {
+      ptx::mbar_arrive_expect_tx(&s_full[1], 16384);
+      ptx::bulk_g2s(sm + KB_UE, img_of(ci) + IMG_U, 16384, &s_full[1]);
+      ptx::mbar_arrive_expect_tx(&s_full[2], 8192 + 16896);
+      ptx::bulk_g2s(sm + KB_P, img_of(ci) + IMG_P, 8192, &s_full[2]);
+      ptx::bulk_g2s(sm + KB_KG, img_of(ci) + IMG_KB, 16896, &s_full[2]);
+      pend[1] = pend[2] = true;
     };
     if (tid == 0 && nc > 0) {
-      issue(first, it & 1);
-      pending_stage = it & 1;
+      load_wq(first);
+      load_ue_pk(first);
     }
     for (int cc = 0; cc < nc; ++cc, ++it) {
-      const int st = it & 1;
-      uint8_t* stage = sm + KB_STAGE0 + st * KB_STAGE;
-      const uint32_t sst = sb + KB_STAGE0 + st * KB_STAGE;
+      const uint32_t ph = it & 1;
       const long long s = start + (long long)cc * C;
       const int Cn = min(C, len - cc * C);
+      // ---- X = [W; Q e^G] S_bf16  (M=128, N=128, K=128, both MN-major)
       if (tid == 0) {
-        if (cc + 1 < nc) issue(first + cc + 1, st ^ 1);
-        if (!ptx::mbar_wait_bounded(&s_full[st], (it >> 1) & 1)) s_abort = 1;
-        pending_stage = (cc + 1 < nc) ? (st ^ 1) : -1;
+        if (!ptx::mbar_wait_bounded(&s_full[0], ph)) s_abort = 1;
+        pend[0] = false;
         ptx::tc_fence_after();
-        // X = [-I; 0] U  (M=128, N=128, K=64, both K-major); left out for a map's M part
-        constexpr uint32_t id0 = ptx::idesc_bf16(128, 128, false, false);
-        if (!no_u) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            ptx::mma_bf16(tX, ptx::sdesc_sw128(sb + KB_NEGI + kk * 32, 16, 1024),
-                          ptx::sdesc_sw128(sst + IMG_U + kk * 32, 16, 1024), id0, kk > 0);
-        }
-        // X += [W; Q e^G] S  (M=128, N=128, K=128, both MN-major)
         constexpr uint32_t id1 = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + IMG_A1 + kk * 2048, 16384, 1024),
-                        ptx::sdesc_sw128(sb + KB_SB + kk * 2048, 16384, 1024), id1, kk > 0 || !no_u);
-        ptx::mma_commit(&s_xbar);
+          ptx::mma_bf16(tX, ptx::sdesc_sw128(sb + KB_WQ + kk * 2048, 16384, 1024),
+                        ptx::sdesc_sw128(sb + KB_SB + kk * 2048, 16384, 1024), id1, kk > 0);
+        ptx::mma_commit(&s_mma1);
       }
-      if (!ptx::mbar_wait_bounded(&s_xbar, it & 1)) s_abort = 1;
+      if (!ptx::mbar_wait_bounded(&s_full[1], ph)) s_abort = 1;
+      if (!ptx::mbar_wait_bounded(&s_full[2], ph)) s_abort = 1;
+      // gamma o S in TMEM (the state pass's decay), while the MMA runs
+      const float gam = reinterpret_cast<const float*>(sm + KB_KG + 16384)[c];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float x[16];
+        ptx::tmem_ld16(tSr + 16 * q4, x);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] *= gam;
+        ptx::tmem_st16(tSr + 16 * q4, x);
+      }
+      if (!ptx::mbar_wait_bounded(&s_mma1, ph)) s_abort = 1;
       ptx::tc_fence_after();
-      const float gam = reinterpret_cast<const float*>(stage + IMG_G)[c];
-      // epilogue 1: rows 0..63 -> E = -X (bf16 operand)
+      // E = U - W S for this thread's token row (rows 0..63 of X hold W S); U
+      // from U^T[dv][j]: a warp reads 32 tokens of one dv row per load.
+      uint32_t e_pk[32];
       if (qd < 2) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float x[32];
-          const uint32_t ta = tX + lane_off + 64 * ch + 32 * hh;
-          ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
-          ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+          ptx::tmem_ld16(tXr + 32 * hh, *reinterpret_cast<float(*)[16]>(x));
+          ptx::tmem_ld16(tXr + 32 * hh + 16, *reinterpret_cast<float(*)[16]>(x + 16));
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int k8 = 0; k8 < 4; ++k8) {
-            float y[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = -x[8 * k8 + e];
-            *reinterpret_cast<uint4*>(sm + KB_E + ch * 8192 + ptx::sw128_chunk(c, 4 * hh + k8)) = pack8(y);
+          for (int e = 0; e < 16; ++e) {
+            const int dv = 64 * ch + 32 * hh + 2 * e;
+            float u0 = 0.f, u1 = 0.f;
+            if (!no_u) {
+              u0 = __bfloat162float(*reinterpret_cast<const bf16*>(sm + KB_UE + ptx::sw128(dv, c)));
+              u1 = __bfloat162float(*reinterpret_cast<const bf16*>(sm + KB_UE + ptx::sw128(dv + 1, c)));
+            }
+            e_pk[16 * hh + e] = ptx::pack_bf16x2(u0 - x[2 * e], u1 - x[2 * e + 1]);
           }
         }
+      }
+      ptx::tmem_wait_st();
+      __syncthreads();  // every read of U^T is done before E overwrites it
+      if (tid == 0 && cc + 1 < nc) load_wq(first + cc + 1);  // the first MMA has read [W; Q e^G]
+      if (qd < 2) {
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8)
+          *reinterpret_cast<uint4*>(sm + KB_UE + ch * 8192 + ptx::sw128_chunk(c, k8)) =
+              make_uint4(e_pk[4 * k8], e_pk[4 * k8 + 1], e_pk[4 * k8 + 2], e_pk[4 * k8 + 3]);
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       __syncthreads();
       if (tid == 0) {
         ptx::tc_fence_after();
-        // Y = Kbar^T E  (M=128, N=128, K=64, both MN-major)
+        // S += Kbar^T E  (M=128, N=128, K=64, both MN-major), onto gamma o S
         constexpr uint32_t id2 = ptx::idesc_bf16(128, 128, true, true);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_bf16(tY, ptx::sdesc_sw128(sst + IMG_KB + kk * 2048, 8192, 1024),
-                        ptx::sdesc_sw128(sb + KB_E + kk * 2048, 8192, 1024), id2, kk > 0);
-        // X += [*; P] E: rows 64..127 become O = Q e^G S + P E (rows 0..63 are dead);
-        // A = the 8 KB in front of P (unused rows) followed by P, K-major [128][64].
+          ptx::mma_bf16(tS, ptx::sdesc_sw128(sb + KB_KG + kk * 2048, 8192, 1024),
+                        ptx::sdesc_sw128(sb + KB_UE + kk * 2048, 8192, 1024), id2, 1);
+        // X += [*; P] E: rows 64..127 become O = Q e^G S + P E (rows 0..63 are dead).
         // The map pass writes no output.
         constexpr uint32_t id3 = ptx::idesc_bf16(128, 128, false, true);
         if (pass != kPassMaps) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            ptx::mma_bf16(tX, ptx::sdesc_sw128(sst + IMG_P - 8192 + kk * 32, 16, 1024),
-                          ptx::sdesc_sw128(sb + KB_E + kk * 2048, 8192, 1024), id3, 1);
+            ptx::mma_bf16(tX, ptx::sdesc_sw128(sb + KB_P - 8192 + kk * 32, 16, 1024),
+                          ptx::sdesc_sw128(sb + KB_UE + kk * 2048, 8192, 1024), id3, 1);
         }
-        ptx::mma_commit(&s_ybar);
+        ptx::mma_commit(&s_mma2);
       }
-      if (!ptx::mbar_wait_bounded(&s_ybar, it & 1)) s_abort = 1;
+      if (!ptx::mbar_wait_bounded(&s_mma2, ph)) s_abort = 1;
       ptx::tc_fence_after();
+      if (tid == 0) {  // U^T / E, P, Kbar and gamma are all read
+        pend[1] = pend[2] = false;
+        if (cc + 1 < nc) load_ue_pk(first + cc + 1);
+      }
+      // the state operand of the next chunk
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float y[32];
-        const uint32_t ta = tY + lane_off + 64 * ch + 32 * hh;
-        ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(y));
-        ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(y + 16));
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float x[16];
+        ptx::tmem_ld16(tSr + 16 * q4, x);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) S[32 * hh + e] = fmaf(gam, S[32 * hh + e], y[e]);
+        for (int k8 = 0; k8 < 2; ++k8)
+          *reinterpret_cast<uint4*>(sm + KB_SB + ch * 16384 + ptx::sw128_chunk(c, 2 * q4 + k8)) = pack8(x + 8 * k8);
       }
-      store_state_bf16(sm, c, ch, S);
       // rows 64..127 of X: the chunk's outputs
       if (qd >= 2 && pass != kPassMaps) {
         const int r = c - 64;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float x[32];
-          const uint32_t ta = tX + lane_off + 64 * ch + 32 * hh;
-          ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
-          ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+          ptx::tmem_ld16(tXr + 32 * hh, *reinterpret_cast<float(*)[16]>(x));
+          ptx::tmem_ld16(tXr + 32 * hh + 16, *reinterpret_cast<float(*)[16]>(x + 16));
           ptx::tmem_wait_ld();
           if (r < Cn) {
             bf16* dst = o + ((size_t)(s + r) * H + h) * D + 64 * ch + 32 * hh;
@@ -1070,15 +1086,24 @@ __global__ void __launch_bounds__(256, 1)
     else if (S_out && p == P - 1)
       S_dst = S_out + soff;
     if (!aborted && S_dst) {
+      ptx::tc_fence_after();
 #pragma unroll
-      for (int j4 = 0; j4 < 16; ++j4)
-        reinterpret_cast<float4*>(S_dst)[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float x[16];
+        ptx::tmem_ld16(tSr + 16 * q4, x);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4)
+          reinterpret_cast<float4*>(S_dst)[4 * q4 + j4] = make_float4(x[4 * j4], x[4 * j4 + 1], x[4 * j4 + 2], x[4 * j4 + 3]);
+      }
     }
+    ptx::tc_fence_before();
+    __syncthreads();  // TMEM S of this item is read before the next item overwrites it
   }
-  // a copy still in flight after an abort must land before shared memory is released
-  if (tid == 0 && aborted && pending_stage >= 0) {
-    const uint32_t parity = ((it + 1) >> 1) & 1;
-    ptx::mbar_wait_bounded(&s_full[pending_stage], parity);
+  // copies still in flight after an abort must land before shared memory is released
+  if (tid == 0 && aborted) {  // they belong to the chunk after the one that gave up
+    for (int i = 0; i < 3; ++i)
+      if (pend[i]) ptx::mbar_wait_bounded(&s_full[i], (it + 1) & 1);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -1190,16 +1215,16 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     const long long nc = (T + tc::C - 1) / tc::C;
     const int P = (int)((nc + seg_chunks - 1) / seg_chunks);
     const long long map_items = units * (P - 1) * 2, fin_items = units * P;
-    tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(map_items, s_sms), 256, tc::KB_DYN, stream>>>(
+    tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(map_items, 2LL * s_sms), 256, tc::KB_DYN, stream>>>(
         ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassMaps, maps, seg_init);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     tc::kda_tc_seg_combine_kernel<<<(unsigned)(units * (tc::D / 8)), 256, 0, stream>>>(maps, S0, seg_init, P);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(fin_items, s_sms), 256, tc::KB_DYN, stream>>>(
+    tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(fin_items, 2LL * s_sms), 256, tc::KB_DYN, stream>>>(
         ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassFinal, maps, seg_init);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else if (units > 0) {
-    const int gridB = (int)(units < s_sms ? units : s_sms);
+    const int gridB = (int)(units < 2LL * s_sms ? units : 2LL * s_sms);  // two CTAs per SM
     tc::kda_tc_state_pass_kernel<<<gridB, 256, tc::KB_DYN, stream>>>(ws, S0, S_out, o, cu_seqlens, N, T, H, 0,
                                                                       tc::kPassPlain, nullptr, nullptr);
     e = cudaGetLastError();
