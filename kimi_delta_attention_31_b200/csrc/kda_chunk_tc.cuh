@@ -233,7 +233,8 @@ __global__ void __launch_bounds__(256, 2)
     kda_tc_chunk_local_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                               const bf16* __restrict__ v, const void* __restrict__ gate,
                               const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
-                              int num_seqs, int T, int H, long long num_items, uint8_t* __restrict__ ws) {
+                              int num_seqs, int T, int H, uint32_t num_items, FastDiv fdH, FastDiv fdC,
+                              uint8_t* __restrict__ ws) {
   __shared__ __align__(16) float s_beta[C];
   __shared__ float s_nrm[2][C];  // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
   constexpr bool kPrep = gate_prep(kGate);
@@ -264,9 +265,10 @@ __global__ void __launch_bounds__(256, 2)
 
   // Persistent: this CTA handles items (chunk * H + head) blockIdx.x, + gridDim.x, ...
   // Each processed item completes s_bar twice (parities 0 then 1).
-  for (long long item = blockIdx.x; item < num_items; item += gridDim.x) {
-  const int h = (int)(item % H);
-  const long long ci = item / H;
+  // item = chunk * H + head; unpacked chunk = sequence * fdC.d + chunk-in-sequence (num_items < 2^31)
+  for (uint32_t item = blockIdx.x; item < num_items; item += gridDim.x) {
+  const uint32_t ci = fdiv(item, fdH);
+  const int h = (int)(item - ci * (uint32_t)H);
 
   long long s0;
   int Cn;
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(256, 2)
     if (warp == 0) {
       long long s = 0;
       int cn = 0;
-      const bool ok = locate_chunk_warp(cu_seqlens, num_seqs, ci, &s, &cn);
+      const bool ok = locate_chunk_warp(cu_seqlens, num_seqs, (long long)ci, &s, &cn);
       if (lane == 0) {
         s_loc_s = s;
         s_loc_n = ok ? cn : -1;
@@ -284,10 +286,10 @@ __global__ void __launch_bounds__(256, 2)
     s0 = s_loc_s;
     Cn = s_loc_n;
   } else {
-    const long long cps = (T + C - 1) / C;
-    const long long cc = ci % cps;
-    s0 = (ci / cps) * T + cc * C;
-    Cn = (int)min((long long)C, (long long)T - cc * C);
+    const uint32_t bq = fdiv(ci, fdC);
+    const int cc = (int)(ci - bq * fdC.d);
+    s0 = (long long)bq * T + (long long)cc * C;
+    Cn = min(C, T - cc * C);
   }
   if (Cn <= 0) {  // uniform across the CTA: past the last chunk of a packed batch
     __syncthreads();  // everyone has read s_loc before warp 0 rewrites it
@@ -299,11 +301,13 @@ __global__ void __launch_bounds__(256, 2)
   // L2 hint for this CTA's next item (packed-free layout only): its q, k, v, g
   // rows, one 128-byte line per lane.
   if (!cu_seqlens && item + gridDim.x < num_items) {
-    const long long nb = item + gridDim.x;
-    const int nh = (int)(nb % H);
-    const long long ncps = (T + C - 1) / C, nci = nb / H, ncc = nci % ncps;
-    const long long ns = (nci / ncps) * T + ncc * C;
-    const int ncn = (int)min((long long)C, (long long)T - ncc * C);
+    const uint32_t nb = item + gridDim.x;
+    const uint32_t nci = fdiv(nb, fdH);
+    const int nh = (int)(nb - nci * (uint32_t)H);
+    const uint32_t nbq = fdiv(nci, fdC);
+    const int ncc = (int)(nci - nbq * fdC.d);
+    const long long ns = (long long)nbq * T + (long long)ncc * C;
+    const int ncn = min(C, T - ncc * C);
     // 128-byte lines per row: k, q, v 2 each, then the gate (fp32 4, bf16 2, per token 0)
     constexpr int lines = kGate == kGateLogTok ? 6 : kGate == kGateLogitBf16 ? 8 : 10;
     for (int idx = tid; idx < lines * C; idx += 256) {
@@ -470,8 +474,9 @@ __global__ void __launch_bounds__(256, 2)
       float o_ka[8], o_qa[8], o_kr[8], o_kb[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float a = __expf(G[u][e]);     // (0, 1]
-        const float rho = __expf(-G[u][e]);  // [1, e^80]
+        const float t = G[u][e] * 1.4426950408889634f;  // G log2(e), in [-115.5, 0]
+        const float a = ptx::ex2(t);     // e^G in (0, 1]
+        const float rho = ptx::ex2(-t);  // e^-G in [1, e^80]
         o_ka[e] = kv[e] * a;
         o_qa[e] = qv[e] * a;
         o_kr[e] = kv[e] * rho;
@@ -1189,11 +1194,15 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int num_seqs = cu_seqlens ? N : 0;
   const long long items = max_chunks * H;
+  if (items >= (1LL << 31)) return cudaErrorInvalidValue;  // item indices are 32-bit
+  const FastDiv fdH = make_fastdiv((uint32_t)H);
+  const FastDiv fdC = make_fastdiv((uint32_t)std::max(1, (T + tc::C - 1) / tc::C));
   if (items > 0) {
     const int gridA = (int)(items < 2LL * s_sms ? items : 2LL * s_sms);
 #define KDA_TC_LOCAL(M)                                                                            \
   tc::kda_tc_chunk_local_kernel<M><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens, \
-                                                                       num_seqs, T, H, items, ws)
+                                                                       num_seqs, T, H, (uint32_t)items, fdH, \
+                                                                       fdC, ws)
     switch (gmode) {
       case kGateLogCh: KDA_TC_LOCAL(kGateLogCh); break;
       case kGateLogTok: KDA_TC_LOCAL(kGateLogTok); break;

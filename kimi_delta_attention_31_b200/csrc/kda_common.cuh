@@ -28,6 +28,27 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Division of n < 2^31 by a fixed divisor d >= 1 with one multiply-high
+// ("division by invariant integers using multiplication", Granlund and
+// Montgomery, 1994): l = ceil(log2 d), m = ceil(2^(32+l) / d) - 2^32 (fits in
+// 32 bits), q = (umulhi(n, m) + n) >> l; n + umulhi(n, m) < 2^32 for n < 2^31.
+struct FastDiv {
+  uint32_t d, mul;
+  int shift;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{d, 0u, 0};
+  while ((1ull << f.shift) < d) ++f.shift;
+  const unsigned long long two32 = 1ull << 32;
+  // ceil(2^(32+l) / d) - 2^32 = floor((2^(32+l) - 1) / d) + 1 - 2^32
+  const unsigned long long num = (two32 << f.shift) - 1ull;  // < 2^63 for l <= 31
+  f.mul = (uint32_t)(num / d + 1ull - two32);
+  return f;
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.mul) + n) >> f.shift;
+}
+
 // What the gate argument holds and how it is laid out.
 enum GateMode : int {
   kGateLogCh = 0,      // log alpha, fp32 [.., H, dk]: one decay per key channel (KDA)

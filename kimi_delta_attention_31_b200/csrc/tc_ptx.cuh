@@ -87,6 +87,14 @@ __device__ __forceinline__ void bulk_wait_read0() {
 // ... and have completed.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// 2^x with the hardware approximation (ex2.approx.ftz.f32: relative error
+// below 2^-22; inputs here stay inside [-126, 127], away from the flushed range).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
