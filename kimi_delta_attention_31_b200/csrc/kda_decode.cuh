@@ -32,12 +32,13 @@ struct DecodeCfg {
   static_assert(DK % RG == 0 && DVB % 4 == 0 && NT % 32 == 0, "shape");
 };
 
-template <typename TIn, int DK, int DV>
+template <typename TIn, int DK, int DV, int kGate>
 __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
     kda_decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                            const TIn* __restrict__ v, const void* __restrict__ gate,
                            const float* __restrict__ beta, float* __restrict__ S,
-                           TIn* __restrict__ o, int gmode) {
+                           TIn* __restrict__ o) {
+  constexpr int gmode = kGate;  // GateMode, fixed per instantiation
   using Cfg = DecodeCfg<TIn, DK, DV>;
   constexpr int DVB = Cfg::DVB, CQ = Cfg::CQ, RG = Cfg::RG, R = Cfg::R, NT = Cfg::NT,
                 NWARP = Cfg::NWARP;
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(DecodeCfg<TIn, DK, DV>::NT)
     s_a[c] = expf(gate_log(gate, gmode, unit, DK, c));
   }
   __syncthreads();
-  if (gate_prep(gmode)) {  // L2-normalise k and q over dk
+  if constexpr (gate_prep(kGate)) {  // L2-normalise k and q over dk
     if (warp < 2) {
       const float* x = warp == 0 ? s_k : s_q;
       float acc = 0.f;
@@ -149,9 +150,18 @@ cudaError_t launch_decode_step(const void* q, const void* k, const void* v, cons
   using Cfg = DecodeCfg<TIn, DK, DV>;
   const long long grid = (long long)N * H * Cfg::NBLK;
   if (grid == 0) return cudaSuccess;
-  kda_decode_step_kernel<TIn, DK, DV><<<(unsigned)grid, Cfg::NT, 0, stream>>>(
-      static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), gate, beta,
-      S, static_cast<TIn*>(o), gmode);
+#define KDA_DECODE_LAUNCH(M)                                                                          \
+  kda_decode_step_kernel<TIn, DK, DV, M><<<(unsigned)grid, Cfg::NT, 0, stream>>>(                          \
+      static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), gate, beta, S, \
+      static_cast<TIn*>(o))
+  switch (gmode) {
+    case kGateLogCh: KDA_DECODE_LAUNCH(kGateLogCh); break;
+    case kGateLogTok: KDA_DECODE_LAUNCH(kGateLogTok); break;
+    case kGateLogitF32: KDA_DECODE_LAUNCH(kGateLogitF32); break;
+    case kGateLogitBf16: KDA_DECODE_LAUNCH(kGateLogitBf16); break;
+    default: return cudaErrorInvalidValue;
+  }
+#undef KDA_DECODE_LAUNCH
   return cudaGetLastError();
 }
 
