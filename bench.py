@@ -8,7 +8,7 @@ Beside it: the recurrent decode (256 sequences x 32 heads, in-place fp32
 state, one token per step) as state GB/s, the Gated DeltaNet variant (one
 gate per token and head) on both shapes, the prefill from raw projections
 with the input preparation fused in, one long sequence with few heads
-(split into segments), the roofline fractions, the fp64
+(split into segments), the backward pass, the roofline fractions, the fp64
 CPU oracle timed on this host's cores, and an end-to-end figure through the
 public host-buffer API (pinned host -> device copies, prefill, copies back).
 
@@ -379,6 +379,39 @@ def long_seq_leg(kda, args, world, dev, stream):
     return out
 
 
+def bwd_leg(kda, args, world, dev, stream, peaks):
+    """Backward pass on the headline shape: gradients of a loss with a random
+    dL/do (bf16) and no final-state term; tokens/s of one kda_chunk_bwd call."""
+    w = W.PREFILL_B8
+    inp = W.make_workload(w, dev)
+    B, T, H, d = w.B, w.T, w.H, w.dk
+    gen = torch.Generator(device=dev).manual_seed(w.seed + 77)
+    dout = torch.randn(inp["v"].shape, generator=gen, device=dev).to(torch.bfloat16)
+    ws = torch.empty(max(int(kda.load_library().kda_chunk_bwd_workspace_size(B, T, H, d, d, 0)), 1),
+                     dtype=torch.uint8, device=dev)
+
+    def bwd():
+        kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], dout, None, None, workspace=ws,
+                      need_dS0=False)
+
+    bwd()
+    torch.cuda.synchronize()
+    barrier(world)
+    steps = max(1, min(args.steps, 2))
+    ms = max_over_ranks(time_launches(bwd, steps, stream), world, dev)
+    th = B * T * H
+    # must move: q, k, v, do (bf16) + g, beta in; dq, dk, dv, dg (fp32) + dbeta out;
+    # plus the fp32 state checkpoint written and read once per 16-token chunk
+    alg = th * (4 * 2 * d + 4 * d + 4 + 4 * 4 * d + 4) + 2 * (th // 16) * d * d * 4
+    gbs = alg / (ms * 1e-3) / 1e9
+    del inp, dout, ws
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "value": world * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "kernel": "kda_chunk_bwd_kernel<bf16,128>",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "alg_bytes_per_launch": alg, "traffic": None}}
+
+
 def run_ours(args):
     import kimi_delta_attention_31_b200 as kda
     rank, world, local = dist_setup(args.gpus)
@@ -499,6 +532,8 @@ def run_ours(args):
     prep = prep_leg(kda, args, world, dev, stream, peaks)
     # ---------------- one long sequence, few heads (sequence segments) ----------------
     long_seq = long_seq_leg(kda, args, world, dev, stream)
+    # ---------------- backward pass ----------------
+    bwd = bwd_leg(kda, args, world, dev, stream, peaks)
 
     # ---------------- CPU oracle baseline (rank 0, N = 1 only) ----------------
     cpu = None
@@ -515,7 +550,7 @@ def run_ours(args):
                        "l2": "inputs (2.7 GB) larger than L2; no flush",
                        "parallelism": f"dp{world} (independent batches per GPU)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "gdn": gdn, "prep": prep,
-            "long_seq": long_seq,
+            "long_seq": long_seq, "bwd": bwd,
             "gpu_launches": gpu_launches, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)

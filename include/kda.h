@@ -171,6 +171,34 @@ kda_status_t kda_recurrent_step_prep(const void* q, const void* k, const void* v
                                      int H, int dk, int dv, kda_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * Backward pass of the prefill: the gradients of a scalar loss with respect
+ * to q, k, v, g (= log alpha, per key channel), beta and the initial state,
+ * given dO (the loss's gradient with respect to o) and, optionally, dS_T
+ * (with respect to the final state).  The pages describe only the forward;
+ * this is the adjoint of the chunked algebra of "Deriving Kimi Delta
+ * Attention from scratch" section 6 and the "Linear / sparse attention"
+ * tutorial sections 5.3 and 6.2, run chunk by chunk in reverse with the state
+ * gradient carried across chunks.  All arithmetic is fp32 and every decay
+ * factor is e^x with x <= 0, so it is exact for any gate.
+ *
+ *   q, k, v, dout : as kda_chunk_fwd's q, k, v and o (dtype), dout the gradient of o
+ *   g, beta, S0   : as kda_chunk_fwd (S0 may be NULL: zero initial state)
+ *   dS_T          : [N, H, dk, dv] fp32 or NULL (no loss term on the final state)
+ *   dq, dk, dv, dg: [B, T, H, d] fp32, written;  dbeta : [B, T, H] fp32, written
+ *   dS0           : [N, H, dk, dv] fp32 or NULL, written
+ *   cu_seqlens, num_seqs, B, T, H, dk, dv: as kda_chunk_fwd
+ *   workspace     : at least kda_chunk_bwd_workspace_size(...) bytes: the state
+ *                   at the start of every 16-token chunk, fp32.
+ * Alignment: every pointer element-aligned.  One CTA per (sequence, head).
+ */
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs);
+kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
+                           float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens,
+                           int num_seqs, int B, int T, int H, int dk_, int dv_, kda_dtype_t dtype,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * kda_chunk_fwd for callers that cannot allocate device memory: the same
  * prefill, same arguments minus the workspace.  (Library plumbing: the pages
  * have no counterpart.)  Some callers get only input and output pointers

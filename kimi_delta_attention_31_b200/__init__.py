@@ -38,7 +38,7 @@ EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step
             "kda_last_error", "kda_device_error", "kda_chunk_fwd_launches", "kda_profile_events",
             "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step",
             "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait",
-            "kda_set_segment_chunks", "kda_segment_chunks")
+            "kda_set_segment_chunks", "kda_segment_chunks", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -95,6 +95,10 @@ def load_library():
         lib.kda_profile_events.restype = i32
         lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 9 + [i32] * 7 + [i32, vp]
         lib.kda_chunk_fwd_noalloc.restype = i32
+        lib.kda_chunk_bwd_workspace_size.argtypes = [i32] * 6
+        lib.kda_chunk_bwd_workspace_size.restype = szt
+        lib.kda_chunk_bwd.argtypes = [vp] * 15 + [i32] * 6 + [i32, vp, szt, vp]
+        lib.kda_chunk_bwd.restype = i32
         lib.kda_set_segment_chunks.argtypes = [i32]
         lib.kda_set_segment_chunks.restype = i32
         lib.kda_segment_chunks.argtypes = [i32] * 4
@@ -241,6 +245,39 @@ def recurrent_step_prep(q, k, v, a, b, S, o=None):
     """Decode step from raw projections (see chunk_fwd_prep): a [N,H,dk] bf16 or
     fp32 raw gate logits, b [N,H] fp32 raw beta logits."""
     return _recurrent_step("kda_recurrent_step_prep", q, k, v, a, b, S, o)
+
+
+def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, cu_seqlens=None, workspace=None,
+              need_dS0=True):
+    """Backward pass of chunk_fwd: gradients of a loss L with respect to q, k,
+    v, g, beta (and S0) given dout = dL/do and dS_T = dL/dS_final (or None).
+    Returns a dict of fp32 tensors dq, dk, dv, dg [B,T,H,d], dbeta [B,T,H] and
+    dS0 [N,H,dk,dv] (None when need_dS0 is False)."""
+    lib = load_library()
+    _need_cuda(q, k, v, g, beta, dout, S0, dS_T, cu_seqlens, workspace)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = num_seqs if cu_seqlens is not None else B
+    if g.dtype != torch.float32 or beta.dtype != torch.float32 or dout.dtype != q.dtype:
+        raise TypeError("g and beta must be float32 and dout must have q's dtype")
+    if tuple(g.shape) != (B, T, H, dk) or tuple(beta.shape) != (B, T, H) or tuple(dout.shape) != (B, T, H, dv):
+        raise ValueError("g must be [B,T,H,dk], beta [B,T,H], dout [B,T,H,dv]")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+               dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty((B, T, H, dk), **f32),
+               dbeta=torch.empty((B, T, H), **f32),
+               dS0=torch.empty((N, H, dk, dv), **f32) if need_dS0 else None)
+    need = int(lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, num_seqs))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(dout), _ptr(dS_T),
+                           _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+                           _ptr(out["dS0"]), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, _dtype_code(q),
+                           _ptr(workspace), ws_bytes, _stream_handle(q.device))
+    _check(st)
+    return out
 
 
 def _recurrent_step(fn, q, k, v, g, beta, S, o):

@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include "../../include/kda.h"
+#include "kda_chunk_bwd.cuh"
 #include "kda_chunk_simt.cuh"
 #include "kda_chunk_tc.cuh"
 #include "kda_common.cuh"
@@ -186,6 +187,61 @@ int kda_version(void) { return 100; }
 
 int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype) {
   return use_tensor_core_path(dk, dv, chunk_size, dtype) ? kda::kTcLaunches : 1;
+}
+
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs) {
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || !supported_head(dk, dv)) return 0;
+  return kda::bwd::bwd_workspace_bytes(B, T, H, dk, num_seqs);
+}
+
+kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
+                           float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens,
+                           int num_seqs, int B, int T, int H, int dkh, int dvh, kda_dtype_t dtype,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const char* fn = "kda_chunk_bwd";
+  t_err[0] = 0;
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0)
+    return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes B=%d T=%d H=%d num_seqs=%d", fn, B, T, H, num_seqs);
+  if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, (int)dtype);
+  if (!supported_head(dkh, dvh))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: dk=%d dv=%d (need dk == dv in {32,64,128})", fn, dkh, dvh);
+  if (cu_seqlens) {
+    if (B != 1) return fail(KDA_ERR_INVALID_ARG, "%s: packed inputs need B == 1", fn);
+    if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "%s: cu_seqlens needs num_seqs >= 1", fn);
+  } else if (num_seqs != 0) {
+    return fail(KDA_ERR_INVALID_ARG, "%s: num_seqs=%d without cu_seqlens", fn, num_seqs);
+  }
+  const int N = cu_seqlens ? num_seqs : B;
+  if (N == 0) return KDA_OK;
+  const long long tokens = (long long)B * T;
+  if (tokens > 0 && (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta))
+    return fail(KDA_ERR_INVALID_ARG, "%s: null input/output pointer", fn);
+  const unsigned esz = dtype == KDA_F32 ? 4u : 2u;
+  const void* in_ptrs[] = {q, k, v, dout};
+  for (const void* p : in_ptrs)
+    if (p && !aligned_to(p, esz)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is misaligned", fn, p);
+  const void* f_ptrs[] = {g, beta, S0, dS_T, dq, dk, dv, dg, dbeta, dS0, cu_seqlens, workspace};
+  for (const void* p : f_ptrs)
+    if (p && !aligned_to(p, 4)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is not 4-byte aligned", fn, p);
+  const size_t need = kda_chunk_bwd_workspace_size(B, T, H, dkh, dvh, num_seqs);
+  if (need && (!workspace || workspace_bytes < need))
+    return fail(KDA_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes, need);
+  float* ck = static_cast<float*>(workspace);
+  cudaError_t e = cudaErrorInvalidValue;
+#define KDA_BWD_CASE(TT, DD)                                                                          \
+  e = kda::bwd::launch_chunk_bwd<TT, DD>(q, k, v, g, beta, S0, dout, dS_T, dq, dk, dv, dg, dbeta, dS0, \
+                                         cu_seqlens, N, T, H, ck, stream)
+  if (dtype == KDA_F32) {
+    if (dkh == 32) KDA_BWD_CASE(float, 32); else if (dkh == 64) KDA_BWD_CASE(float, 64); else KDA_BWD_CASE(float, 128);
+  } else {
+    if (dkh == 32) KDA_BWD_CASE(__nv_bfloat16, 32);
+    else if (dkh == 64) KDA_BWD_CASE(__nv_bfloat16, 64);
+    else KDA_BWD_CASE(__nv_bfloat16, 128);
+  }
+#undef KDA_BWD_CASE
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return KDA_OK;
 }
 
 kda_status_t kda_set_segment_chunks(int chunks) {

@@ -1,0 +1,437 @@
+// kda_chunk_bwd.cuh -- backward pass of the chunkwise KDA prefill: gradients
+// with respect to q, k, v, g = log alpha, beta and the initial state, in fp32
+// arithmetic on the CUDA cores.
+//
+// The pages give the forward only ("Deriving Kimi Delta Attention from
+// scratch", section 6, chunked mode; "Linear / sparse attention" tutorial,
+// sections 5.3 and 6.2).  The backward here is the adjoint of that chunk
+// algebra, chunk by chunk in reverse with the state gradient carried from
+// chunk to chunk.  Per chunk (C tokens entering with state S; G the
+// cumulative log-decay, Gam = e^G, L = e^{G_last - G}, Kb = K o L,
+// gam = e^{G_last}; M_rj = e^{G_r - G_j} per channel; X_rj = sum_c K_rc K_jc
+// M_rjc and A = beta X strictly lower; P_rj = sum_c Q_rc K_jc M_rjc lower with
+// the diagonal; T = (I + A)^{-1}; Bk = beta K o Gam, Bv = beta V; W = T Bk,
+// U = T Bv, E = U - W S), given dO and dS' (gradient of the chunk's output state):
+//   dE  = Kb dS' + P^T dO,   dKb = E dS'^T,   dOS = dO S^T
+//   dS  = gam o dS' + (Q o Gam)^T dO - W^T dE          (to the previous chunk)
+//   dP  = lower(dO E^T),  dW = -dE S^T,  dT = dE Bv^T + dW Bk^T
+//   dBv = T^T dE,  dBk = T^T dW,  dA = -T^T dT T^T (strictly lower), At = beta o dA
+//   dV  = beta o dBv;  dbeta = rowsum(dBv o V + dBk o K o Gam + dA o X)
+//   dQ  = dOS o Gam + sum_j dP_rj K_j o M_rj
+//   dK  = beta dBk o Gam + dKb o L + sum_j At_rj K_j o M_rj
+//         + sum_{r >= j} (At_rj K_r + dP_rj Q_r) o M_rj            (as a column)
+//   dG  = beta dBk o K o Gam + dOS o Q o Gam - dKb o Kb
+//         + sum_j (At_rj K_r K_j + dP_rj Q_r K_j) o M_rj   - (the same summed as a column)
+//   dG_last += sum_r dKb o Kb + gam o rowsum(dS' o S);   dg = reverse cumulative sum of dG.
+// Every decay factor is e^{x} with x <= 0, so the pass is exact for any gate.
+//
+// Work decomposition: one CTA of 4 D threads per (sequence, head).  A forward
+// sweep stores each chunk's entry state (fp32) in the workspace; the reverse
+// sweep reloads it, recomputes the chunk's A, P, T, W, E and applies the
+// equations above.  S and dS (D x D fp32) live in shared memory; loops that
+// walk them down a column start at a lane-dependent offset so that a warp's
+// loads fall in distinct banks.
+#pragma once
+#include "kda_common.cuh"
+
+namespace kda {
+namespace bwd {
+
+constexpr int C = 16;  // tokens per chunk of the backward
+
+template <int D>
+struct Cfg {
+  static constexpr int NT = 4 * D;  // threads: 4 per key channel
+  static constexpr int NTILE = 11;  // C x D tiles
+  static constexpr int NSMALL = 9;  // C x C tiles
+  static constexpr size_t smem_floats = 2 * (size_t)D * D + (size_t)NTILE * C * D + (size_t)NSMALL * C * C + 2 * C + 2 * D;
+  static constexpr size_t smem_bytes = smem_floats * sizeof(float);
+};
+
+// Checkpoint slot of chunk `ch` of sequence n: unique over the packed layout.
+__device__ __forceinline__ long long ckpt_slot(bool packed, int n, long long t0, int nch_T, int ch) {
+  return packed ? (t0 / C + ch + n) : ((long long)n * nch_T + ch);
+}
+
+template <typename TIn, int D>
+__global__ void __launch_bounds__(4 * D)
+    kda_chunk_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
+                         const float* __restrict__ g, const float* __restrict__ beta,
+                         const float* __restrict__ S0, const TIn* __restrict__ dout,
+                         const float* __restrict__ dS_T, float* __restrict__ dq, float* __restrict__ dk,
+                         float* __restrict__ dv, float* __restrict__ dg, float* __restrict__ dbeta,
+                         float* __restrict__ dS0, const int32_t* __restrict__ cu_seqlens, int T, int H,
+                         float* __restrict__ ckpt) {
+  constexpr int NT = Cfg<D>::NT;
+  extern __shared__ float smem[];
+  float* Ss = smem;             // S  [D][D]
+  float* dSs = Ss + D * D;      // dS [D][D]
+  float* Qs = dSs + D * D;      // C x D tiles
+  float* Ks = Qs + C * D;
+  float* Gs = Ks + C * D;       // cumulative log-decay
+  float* GMs = Gs + C * D;      // e^G
+  float* ELs = GMs + C * D;     // e^{G_last - G}
+  float* dOs = ELs + C * D;
+  float* Ws = dOs + C * D;      // W, later dW
+  float* Es = Ws + C * D;
+  float* dEs = Es + C * D;
+  float* R1 = dEs + C * D;      // U, later dOS
+  float* R2 = R1 + C * D;       // dKb
+  float* Xs = R2 + C * D;       // C x C tiles
+  float* As = Xs + C * C;
+  float* Ps = As + C * C;
+  float* Ts = Ps + C * C;
+  float* dPs = Ts + C * C;
+  float* dTs = dPs + C * C;
+  float* dAs = dTs + C * C;
+  float* Mt = dAs + C * C;
+  float* Ats = Mt + C * C;      // beta-scaled dA
+  float* bs = Ats + C * C;      // beta [C]
+  float* dbs = bs + C;          // dbeta accumulation [C]
+  float* gam = dbs + C;         // e^{G_last} [D]
+  float* dGl = gam + D;         // gam o rowsum(dS' o S) [D]
+
+  const int uh = blockIdx.x;  // n * H + h
+  const int h = uh % H, n = uh / H;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const bool packed = cu_seqlens != nullptr;
+  const long long t0 = packed ? (long long)cu_seqlens[n] : (long long)n * T;
+  const long long t1 = packed ? (long long)cu_seqlens[n + 1] : t0 + T;
+  const int nch = (int)((t1 - t0 + C - 1) / C);
+  const int nch_T = (T + C - 1) / C;
+  auto row_off = [&](long long t) { return ((size_t)t * H + h) * D; };
+  auto slot_ptr = [&](int ch) {
+    return ckpt + ((size_t)ckpt_slot(packed, n, t0, nch_T, ch) * H + h) * D * D;
+  };
+
+  // Chunk `ch` into shared memory (rows >= Cn are zero; g = 0 there keeps G flat).
+  auto load_chunk = [&](int ch, bool with_dout) {
+    const long long s = t0 + (long long)ch * C;
+    const int Cn = min(C, (int)(t1 - s));
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int r = idx / D, c = idx % D;
+      float qv = 0.f, kv = 0.f, gv = 0.f, ov = 0.f;
+      if (r < Cn) {
+        const size_t off = row_off(s + r) + c;
+        qv = to_f32(q[off]);
+        kv = to_f32(k[off]);
+        gv = g[off];
+        if (with_dout) ov = to_f32(dout[off]);
+      }
+      Qs[idx] = qv;
+      Ks[idx] = kv;
+      Gs[idx] = gv;
+      dOs[idx] = ov;
+    }
+    for (int r = tid; r < C; r += NT) bs[r] = r < Cn ? beta[(size_t)(s + r) * H + h] : 0.f;
+    __syncthreads();
+    for (int c = tid; c < D; c += NT) {  // cumulative sum per channel
+      float acc = 0.f;
+      for (int r = 0; r < C; ++r) {
+        acc += Gs[r * D + c];
+        Gs[r * D + c] = acc;
+      }
+      gam[c] = __expf(acc);
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int c = idx % D;
+      GMs[idx] = __expf(Gs[idx]);
+      ELs[idx] = __expf(Gs[(C - 1) * D + c] - Gs[idx]);
+    }
+    __syncthreads();
+    return Cn;
+  };
+
+  // X, A, P, T = (I + A)^{-1}, W = T Bk, U = T Bv (into R1), E = U - W S.
+  auto chunk_forward = [&](long long s, int Cn) {
+    for (int idx = tid; idx < 2 * C * C; idx += NT) {  // two lanes per pair, halves of the channels
+      const int pr = idx >> 1, half = idx & 1, r = pr / C, j = pr % C;
+      float x = 0.f, p = 0.f;
+      if (j <= r) {
+        for (int c = half * (D / 2); c < (half + 1) * (D / 2); ++c) {
+          const float kj = Ks[j * D + c] * __expf(Gs[r * D + c] - Gs[j * D + c]);
+          x = fmaf(Ks[r * D + c], kj, x);
+          p = fmaf(Qs[r * D + c], kj, p);
+        }
+      }
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      p += __shfl_xor_sync(0xffffffffu, p, 1);
+      if (half == 0) {
+        Xs[pr] = j < r ? x : 0.f;
+        As[pr] = j < r ? bs[r] * x : 0.f;
+        Ps[pr] = p;
+      }
+    }
+    __syncthreads();
+    if (tid < C) {  // forward substitution, one column per thread
+      const int j = tid;
+      float col[C];
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        float acc = (i == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < i; ++m) acc = fmaf(-As[i * C + m], col[m], acc);
+        col[i] = acc;
+      }
+#pragma unroll
+      for (int i = 0; i < C; ++i) Ts[i * C + j] = col[i];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * D; idx += NT) {  // W = T Bk, U = T Bv
+      const int r = idx / D, c = idx % D;
+      float w = 0.f, u = 0.f;
+      for (int m = 0; m <= r; ++m) {
+        const float t = Ts[r * C + m] * bs[m];
+        w = fmaf(t, Ks[m * D + c] * GMs[m * D + c], w);
+        if (m < Cn) u = fmaf(t, to_f32(v[row_off(s + m) + c]), u);
+      }
+      Ws[idx] = w;
+      R1[idx] = u;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * D; idx += NT) {  // E = U - W S
+      const int r = idx / D, j = idx % D;
+      float acc = R1[idx];
+      for (int c = 0; c < D; ++c) acc = fmaf(-Ws[r * D + c], Ss[c * D + j], acc);
+      Es[idx] = acc;
+    }
+    __syncthreads();
+  };
+
+  // ---- forward sweep: the entry state of every chunk into the workspace
+  for (int idx = tid; idx < D * D; idx += NT) Ss[idx] = S0 ? S0[(size_t)uh * D * D + idx] : 0.f;
+  __syncthreads();
+  for (int ch = 0; ch < nch; ++ch) {
+    float* slot = slot_ptr(ch);
+    for (int idx = tid; idx < D * D; idx += NT) slot[idx] = Ss[idx];
+    const long long s = t0 + (long long)ch * C;
+    const int Cn = load_chunk(ch, false);
+    chunk_forward(s, Cn);
+    for (int idx = tid; idx < D * D; idx += NT) {  // S <- gam o S + Kb^T E
+      const int c = idx / D, j = idx % D;
+      float acc = gam[c] * Ss[idx];
+      for (int r = 0; r < C; ++r) acc = fmaf(Ks[r * D + c] * ELs[r * D + c], Es[r * D + j], acc);
+      Ss[idx] = acc;
+    }
+    __syncthreads();
+  }
+
+  // ---- reverse sweep
+  for (int idx = tid; idx < D * D; idx += NT) dSs[idx] = dS_T ? dS_T[(size_t)uh * D * D + idx] : 0.f;
+  __syncthreads();
+  for (int ch = nch - 1; ch >= 0; --ch) {
+    const float* slot = slot_ptr(ch);
+    for (int idx = tid; idx < D * D; idx += NT) Ss[idx] = slot[idx];
+    const long long s = t0 + (long long)ch * C;
+    const int Cn = load_chunk(ch, true);
+    chunk_forward(s, Cn);
+
+    // 1. from the old dS': dE = Kb dS' + P^T dO, dKb = E dS'^T (R2), gam o rowsum(dS' o S)
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int r = idx / D, j = idx % D;
+      float acc = 0.f;
+      for (int c = 0; c < D; ++c) acc = fmaf(Ks[r * D + c] * ELs[r * D + c], dSs[c * D + j], acc);
+      for (int rr = r; rr < C; ++rr) acc = fmaf(Ps[rr * C + r], dOs[rr * D + j], acc);
+      dEs[idx] = acc;
+    }
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int r = idx / D, c = idx % D;
+      float acc = 0.f;
+      for (int jj = 0; jj < D; ++jj) {
+        const int j = (jj + lane) & (D - 1);  // rotated: distinct banks across the warp
+        acc = fmaf(Es[r * D + j], dSs[c * D + j], acc);
+      }
+      R2[idx] = acc;
+    }
+    for (int c = tid; c < D; c += NT) {
+      float acc = 0.f;
+      for (int j = 0; j < D; ++j) acc = fmaf(dSs[c * D + j], Ss[c * D + j], acc);
+      dGl[c] = gam[c] * acc;
+    }
+    __syncthreads();
+    // 2. dP = lower(dO E^T); dOS = dO S^T (R1, U is no longer needed)
+    for (int idx = tid; idx < C * C; idx += NT) {
+      const int r = idx / C, j = idx % C;
+      float acc = 0.f;
+      if (j <= r)
+        for (int d = 0; d < D; ++d) acc = fmaf(dOs[r * D + d], Es[j * D + d], acc);
+      dPs[idx] = acc;
+    }
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int r = idx / D, c = idx % D;
+      float acc = 0.f;
+      for (int jj = 0; jj < D; ++jj) {
+        const int j = (jj + lane) & (D - 1);
+        acc = fmaf(dOs[r * D + j], Ss[c * D + j], acc);
+      }
+      R1[idx] = acc;
+    }
+    __syncthreads();
+    // 3. dS = gam o dS' + (Q o Gam)^T dO - W^T dE  (in place: each element reads only itself of dS')
+    for (int idx = tid; idx < D * D; idx += NT) {
+      const int c = idx / D, j = idx % D;
+      float acc = gam[c] * dSs[idx];
+      for (int r = 0; r < C; ++r) {
+        acc = fmaf(Qs[r * D + c] * GMs[r * D + c], dOs[r * D + j], acc);
+        acc = fmaf(-Ws[r * D + c], dEs[r * D + j], acc);
+      }
+      dSs[idx] = acc;
+    }
+    __syncthreads();
+    // 4. dW = -dE S^T (over W)
+    for (int idx = tid; idx < C * D; idx += NT) {
+      const int r = idx / D, c = idx % D;
+      float acc = 0.f;
+      for (int jj = 0; jj < D; ++jj) {
+        const int j = (jj + lane) & (D - 1);
+        acc = fmaf(dEs[r * D + j], Ss[c * D + j], acc);
+      }
+      Ws[idx] = -acc;
+    }
+    __syncthreads();
+    // 5. dT = dE Bv^T + dW Bk^T
+    for (int idx = tid; idx < C * C; idx += NT) {
+      const int r = idx / C, j = idx % C;
+      float acc = 0.f;
+      if (j < Cn) {
+        const size_t vo = row_off(s + j);
+        for (int d = 0; d < D; ++d) {
+          acc = fmaf(dEs[r * D + d], bs[j] * to_f32(v[vo + d]), acc);
+          acc = fmaf(Ws[r * D + d], bs[j] * Ks[j * D + d] * GMs[j * D + d], acc);
+        }
+      }
+      dTs[idx] = acc;
+    }
+    __syncthreads();
+    // 6. dA = -T^T dT T^T (strictly lower): Mt = dT T^T, then -T^T Mt
+    for (int idx = tid; idx < C * C; idx += NT) {
+      const int r = idx / C, j = idx % C;
+      float acc = 0.f;
+      for (int m = 0; m < C; ++m) acc = fmaf(dTs[r * C + m], Ts[j * C + m], acc);
+      Mt[idx] = acc;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * C; idx += NT) {
+      const int r = idx / C, j = idx % C;
+      float acc = 0.f;
+      for (int m = 0; m < C; ++m) acc = fmaf(Ts[m * C + r], Mt[m * C + j], acc);
+      dAs[idx] = j < r ? -acc : 0.f;
+      Ats[idx] = j < r ? -acc * bs[r] : 0.f;
+    }
+    __syncthreads();
+    for (int r = tid; r < C; r += NT) {  // dbeta from A: rowsum(dA o X)
+      float acc = 0.f;
+      for (int j = 0; j < C; ++j) acc = fmaf(dAs[r * C + j], Xs[r * C + j], acc);
+      dbs[r] = acc;
+    }
+    __syncthreads();
+    // 7. per (row, channel) outputs.  Thread (c, part) owns channel c of rows
+    //    part, part + 4, ... both as a row (left factor) and as a column (right
+    //    factor) of the pairwise terms, so no two threads write one element.
+    {
+      const int c = tid >> 2, part = tid & 3;
+      float dQa[C / 4], dKa[C / 4], dGa[C / 4];
+      float kbsum = 0.f;  // sum over this thread's rows of dKb o Kb (for G_last)
+#pragma unroll
+      for (int i = 0; i < C / 4; ++i) {
+        const int r = part + 4 * i, e = r * D + c;
+        const float Gr = Gs[e], kr = Ks[e], qr = Qs[e];
+        // dBv, dBk for this element (T lower: rows m >= r)
+        float dbv = 0.f, dbk = 0.f;
+        for (int m = r; m < C; ++m) {
+          dbv = fmaf(Ts[m * C + r], dEs[m * D + c], dbv);
+          dbk = fmaf(Ts[m * C + r], Ws[m * D + c], dbk);
+        }
+        const float vr = r < Cn ? to_f32(v[row_off(s + r) + c]) : 0.f;
+        atomicAdd(&dbs[r], dbv * vr + dbk * kr * GMs[e]);
+        if (r < Cn) dv[row_off(s + r) + c] = bs[r] * dbv;
+        const float dos = R1[e], dkb = R2[e];
+        float dQ = dos * GMs[e];
+        float dK = bs[r] * dbk * GMs[e] + dkb * ELs[e];
+        float dG = bs[r] * dbk * kr * GMs[e] + dos * qr * GMs[e] - dkb * kr * ELs[e];
+        kbsum = fmaf(dkb, kr * ELs[e], kbsum);
+        // as a row: pairs (r, j <= r)
+        for (int j = 0; j <= r; ++j) {
+          const float kj = Ks[j * D + c], w = __expf(Gr - Gs[j * D + c]);
+          const float at = Ats[r * C + j], dp = dPs[r * C + j];
+          dQ = fmaf(dp * kj, w, dQ);
+          dK = fmaf(at * kj, w, dK);
+          dG = fmaf((at * kr + dp * qr) * kj, w, dG);
+        }
+        // as a column: pairs (rr >= r, r)
+        for (int rr = r; rr < C; ++rr) {
+          const float w = __expf(Gs[rr * D + c] - Gr);
+          const float at = Ats[rr * C + r], dp = dPs[rr * C + r];
+          const float f = at * Ks[rr * D + c] + dp * Qs[rr * D + c];
+          dK = fmaf(f, w, dK);
+          dG = fmaf(-f * kr, w, dG);
+        }
+        dQa[i] = dQ;
+        dKa[i] = dK;
+        dGa[i] = dG;
+      }
+      // G_last terms go to the chunk's last row (row C - 1, owned by part 3)
+      kbsum += __shfl_xor_sync(0xffffffffu, kbsum, 1);
+      kbsum += __shfl_xor_sync(0xffffffffu, kbsum, 2);
+      if (part == (C - 1) % 4) dGa[C / 4 - 1] += kbsum + dGl[c];
+      // dQ, dK out; dG into a tile (over dE) for the reverse cumulative sum
+#pragma unroll
+      for (int i = 0; i < C / 4; ++i) {
+        const int r = part + 4 * i;
+        if (r < Cn) {
+          const size_t o = row_off(s + r) + c;
+          dq[o] = dQa[i];
+          dk[o] = dKa[i];
+        }
+      }
+      __syncthreads();  // every read of dE is done
+#pragma unroll
+      for (int i = 0; i < C / 4; ++i) dEs[(part + 4 * i) * D + c] = dGa[i];
+      __syncthreads();
+      if (part == 0) {  // dg_i = sum_{r >= i} dG_r
+        float acc = 0.f;
+        for (int r = C - 1; r >= 0; --r) {
+          acc += dEs[r * D + c];
+          if (r < Cn) dg[row_off(s + r) + c] = acc;
+        }
+      }
+    }
+    for (int r = tid; r < Cn; r += NT) dbeta[(size_t)(s + r) * H + h] = dbs[r];
+    __syncthreads();
+  }
+  if (dS0)
+    for (int idx = tid; idx < D * D; idx += NT) dS0[(size_t)uh * D * D + idx] = dSs[idx];
+}
+
+template <typename TIn, int D>
+cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
+                             float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens, int N,
+                             int T, int H, float* ckpt, cudaStream_t stream) {
+  static int s_attr_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (s_attr_device != dev) {
+    e = cudaFuncSetAttribute(kda_chunk_bwd_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Cfg<D>::smem_bytes);
+    if (e != cudaSuccess) return e;
+    s_attr_device = dev;
+  }
+  const long long units = (long long)N * H;
+  if (units == 0) return cudaSuccess;
+  kda_chunk_bwd_kernel<TIn, D><<<(unsigned)units, Cfg<D>::NT, Cfg<D>::smem_bytes, stream>>>(
+      static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), g, beta, S0,
+      static_cast<const TIn*>(dout), dS_T, dq, dk, dv, dg, dbeta, dS0, cu_seqlens, T, H, ckpt);
+  return cudaGetLastError();
+}
+
+// Workspace (checkpoints): one D x D fp32 state per (chunk of C tokens, head).
+inline size_t bwd_workspace_bytes(int B, int T, int H, int D, int num_seqs) {
+  const long long slots = num_seqs > 0 ? (long long)T / C + num_seqs : (long long)B * ((T + C - 1) / C);
+  return (size_t)slots * H * D * D * sizeof(float);
+}
+
+}  // namespace bwd
+}  // namespace kda

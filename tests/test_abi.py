@@ -161,3 +161,25 @@ def test_selftest_bounded_wait_rejects_bad_limits():
     assert lib.kda_selftest_bounded_wait(0, None) == 1
     assert lib.kda_selftest_bounded_wait(2_000_000_000, None) == 1
     assert "limit_ns" in kda.last_error()
+
+
+def test_chunk_bwd_validates_arguments():
+    lib = kda.load_library()
+    f = _fake()
+
+    def call(dtype=kda.KDA_BF16, d=128, dq=f, ws=None, wsb=0, B=1, T=64, cu=None, ns=0, q=f):
+        return lib.kda_chunk_bwd(q, f, f, f, f, None, f, None, dq, f, f, f, f, None, cu, ns, B, T, 2, d, d,
+                                 dtype, ws, wsb, None)
+
+    assert call() == 4                                # reached the workspace check
+    assert "kda_chunk_bwd" in kda.last_error()
+    assert call(d=96) == 2
+    assert call(dtype=7) == 2
+    assert call(dq=_null()) == 1
+    assert call(dq=_fake(0x1002)) == 3                # fp32 gradients need 4-byte alignment
+    assert call(q=_fake(0x1001)) == 3                 # bf16 inputs need 2-byte alignment
+    assert call(cu=f, ns=0) == 1
+    assert call(B=0) == 0
+    need = lib.kda_chunk_bwd_workspace_size(1, 64, 2, 128, 128, 0)
+    assert need == 4 * 2 * 128 * 128 * 4              # 4 chunks of 16 tokens x 2 heads x fp32 states
+    assert call(ws=_fake(0x4000), wsb=need - 1) == 4

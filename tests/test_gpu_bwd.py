@@ -1,0 +1,100 @@
+"""GPU parity of the backward pass (kda_chunk_bwd) against the gradient
+oracle (reverse-mode differentiation of the fp64 token recurrence).  The
+kernel computes in fp32 from the same (bf16- or fp32-rounded) inputs the
+oracle widens, so both dtypes are held to 1e-4 relative RMS per (sequence,
+head) slice of every gradient."""
+import numpy as np
+import pytest
+import torch
+
+import kimi_delta_attention_31_b200 as kda
+import kda_workloads as W
+from oracle.grad import recurrent_grad
+from parity_util import rel_rms
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-4
+
+
+def _inputs(dev, B, T, H, d, dtype, seed, lengths=None, s0=True):
+    inp = W.make_prefill(B, T, H, d, d, dtype, -3.0, 1.0, 0.05 if s0 else 0.0, seed=seed, device=dev, lengths=lengths)
+    gen = torch.Generator(device=dev).manual_seed(seed + 1)
+    tdt = inp["q"].dtype
+    inp["do"] = torch.randn(inp["v"].shape, generator=gen, device=dev).to(tdt)
+    N = len(lengths) if lengths else B
+    inp["dS_T"] = torch.randn((N, H, d, d), generator=gen, device=dev) * 0.1
+    return inp
+
+
+def _check_slices(got, ref, what, tol=TOL):
+    """got, ref: [..] arrays with the (sequence, head) slice structure of the tensor."""
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    err = rel_rms(got, ref)
+    assert err <= tol, f"{what}: rel-RMS {err:.3e}"
+    return err
+
+
+def _compare(inp, out, with_s0=True):
+    cpu = {n: (t.double().cpu().numpy() if t is not None else None) for n, t in inp.items() if n != "cu_seqlens"}
+    B, T, H, d = cpu["q"].shape
+    for b in range(B):
+        for h in range(H):
+            sl = lambda x: x[b:b + 1, :, h:h + 1]
+            ref = recurrent_grad(sl(cpu["q"]), sl(cpu["k"]), sl(cpu["v"]), sl(cpu["g"]), sl(cpu["beta"]),
+                                 cpu["S0"][b:b + 1, h:h + 1] if with_s0 else None, sl(cpu["do"]),
+                                 cpu["dS_T"][b:b + 1, h:h + 1])
+            for n in ("dq", "dk", "dv", "dg", "dbeta"):
+                _check_slices(out[n][b:b + 1, :, h:h + 1].double().cpu().numpy(), ref[n], f"{n} b{b} h{h}")
+            if with_s0:
+                _check_slices(out["dS0"][b:b + 1, h:h + 1].double().cpu().numpy(), ref["dS0"], f"dS0 b{b} h{h}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("T", [1, 17, 40])
+def test_bwd_small_shapes(cuda_device, dtype, d, T):
+    inp = _inputs(cuda_device, 2, T, 2, d, dtype, seed=600 + T + d)
+    out = kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["do"], inp["S0"], inp["dS_T"])
+    torch.cuda.synchronize()
+    _compare(inp, out)
+
+
+def test_bwd_zero_initial_state_and_no_final_gradient(cuda_device):
+    inp = _inputs(cuda_device, 1, 33, 2, 64, "bf16", seed=61, s0=False)
+    out = kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["do"], None, None, need_dS0=False)
+    torch.cuda.synchronize()
+    inp["dS_T"] = torch.zeros_like(inp["dS_T"])
+    _compare(inp, out, with_s0=False)
+
+
+def test_bwd_packed_varlen(cuda_device):
+    lens = (5, 0, 33, 16)
+    inp = _inputs(cuda_device, 1, sum(lens), 2, 64, "f32", seed=62, lengths=lens)
+    out = kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["do"], inp["S0"], inp["dS_T"],
+                        cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    cu = np.cumsum((0,) + lens)
+    cpu = {n: t.double().cpu().numpy() for n, t in inp.items() if n not in ("cu_seqlens",)}
+    for s_i in range(len(lens)):
+        a, b = cu[s_i], cu[s_i + 1]
+        for h in range(2):
+            if b == a:  # empty sequence: the state gradient passes through
+                assert torch.allclose(out["dS0"][s_i, h], inp["dS_T"][s_i, h])
+                continue
+            sl = lambda x: x[:, a:b, h:h + 1]
+            ref = recurrent_grad(sl(cpu["q"]), sl(cpu["k"]), sl(cpu["v"]), sl(cpu["g"]), sl(cpu["beta"]),
+                                 cpu["S0"][s_i:s_i + 1, h:h + 1], sl(cpu["do"]), cpu["dS_T"][s_i:s_i + 1, h:h + 1])
+            for n in ("dq", "dk", "dv", "dg", "dbeta"):
+                _check_slices(out[n][:, a:b, h:h + 1].double().cpu().numpy(), ref[n], f"{n} seq{s_i} h{h}")
+            _check_slices(out["dS0"][s_i:s_i + 1, h:h + 1].double().cpu().numpy(), ref["dS0"], f"dS0 seq{s_i}")
+
+
+def test_bwd_longer_sequence_strong_decay(cuda_device):
+    """T = 300 at d = 128 with steep gates (log alpha about -2 per token): the
+    backward uses only decay factors <= 1, so any gate is exact."""
+    inp = _inputs(cuda_device, 1, 300, 1, 128, "bf16", seed=63)
+    inp["g"] = (inp["g"] * 0 - 2.0 + 0.1 * torch.rand_like(inp["g"])).contiguous()
+    out = kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["do"], inp["S0"], inp["dS_T"])
+    torch.cuda.synchronize()
+    _compare(inp, out)
