@@ -191,6 +191,14 @@ def oracle_baseline(w, target_s=15.0):
                       f"tokens/s = token-heads/s / H"}, dt
 
 
+def headline_config(w, world):
+    """The `config` of the headline line, shared by both arms."""
+    return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+            "chunk": w.chunk, "g": f"-softplus(N({w.g_mu},{w.g_sigma}))",
+            "l2": "inputs (2.7 GB) larger than L2; no flush",
+            "parallelism": f"dp{world} (independent batches per GPU)"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -211,8 +219,7 @@ def run_reference(args):
             "ms_per_step": 1e3 * total / max(args.steps, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
-                       "chunk": w.chunk},
+            "config": headline_config(w, args.gpus),
             "cpu_baseline": dict(base, value=value),
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -545,10 +552,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
-                       "chunk": w.chunk, "g": f"-softplus(N({w.g_mu},{w.g_sigma}))",
-                       "l2": "inputs (2.7 GB) larger than L2; no flush",
-                       "parallelism": f"dp{world} (independent batches per GPU)"},
+            "config": headline_config(w, world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "gdn": gdn, "prep": prep,
             "long_seq": long_seq, "bwd": bwd,
             "gpu_launches": gpu_launches, "clocks": clocks}
