@@ -48,6 +48,28 @@ struct Cfg {
   static constexpr size_t smem_bytes = smem_floats * sizeof(float);
 };
 
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float4 x) { *reinterpret_cast<float4*>(p) = x; }
+__device__ __forceinline__ float4 fma4(float a, float4 b, float4 c) {
+  return make_float4(fmaf(a, b.x, c.x), fmaf(a, b.y, c.y), fmaf(a, b.z, c.z), fmaf(a, b.w, c.w));
+}
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+}
+// sum_j X[r][j] Y[c][j] over a row of each (row length D, 16-byte groups
+// visited from a lane-dependent start so that a warp's loads of Y rows, which
+// differ per lane, fall in distinct banks).
+template <int D>
+__device__ __forceinline__ float rowdot(const float* xr, const float* yc, int lane) {
+  float acc = 0.f;
+#pragma unroll 8
+  for (int jj = 0; jj < D / 4; ++jj) {
+    const int j = 4 * ((jj + lane) & (D / 4 - 1));
+    acc = dot4(ld4(xr + j), ld4(yc + j), acc);
+  }
+  return acc;
+}
+
 // Checkpoint slot of chunk `ch` of sequence n: unique over the packed layout.
 __device__ __forceinline__ long long ckpt_slot(bool packed, int n, long long t0, int nch_T, int ch) {
   return packed ? (t0 / C + ch + n) : ((long long)n * nch_T + ch);
@@ -144,7 +166,7 @@ __global__ void __launch_bounds__(4 * D)
   };
 
   // X, A, P, T = (I + A)^{-1}, W = T Bk, U = T Bv (into R1), E = U - W S.
-  auto chunk_forward = [&](long long s, int Cn) {
+  auto chunk_forward = [&](long long s, int Cn, bool with_p) {
     for (int idx = tid; idx < 2 * C * C; idx += NT) {  // two lanes per pair, halves of the channels
       const int pr = idx >> 1, half = idx & 1, r = pr / C, j = pr % C;
       float x = 0.f, p = 0.f;
@@ -152,7 +174,7 @@ __global__ void __launch_bounds__(4 * D)
         for (int c = half * (D / 2); c < (half + 1) * (D / 2); ++c) {
           const float kj = Ks[j * D + c] * __expf(Gs[r * D + c] - Gs[j * D + c]);
           x = fmaf(Ks[r * D + c], kj, x);
-          p = fmaf(Qs[r * D + c], kj, p);
+          if (with_p) p = fmaf(Qs[r * D + c], kj, p);
         }
       }
       x += __shfl_xor_sync(0xffffffffu, x, 1);
@@ -190,11 +212,12 @@ __global__ void __launch_bounds__(4 * D)
       R1[idx] = u;
     }
     __syncthreads();
-    for (int idx = tid; idx < C * D; idx += NT) {  // E = U - W S
-      const int r = idx / D, j = idx % D;
-      float acc = R1[idx];
-      for (int c = 0; c < D; ++c) acc = fmaf(-Ws[r * D + c], Ss[c * D + j], acc);
-      Es[idx] = acc;
+    for (int idx = tid; idx < C * D / 4; idx += NT) {  // E = U - W S, four columns per thread
+      const int r = idx / (D / 4), j = 4 * (idx % (D / 4));
+      float4 acc = ld4(R1 + r * D + j);
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) acc = fma4(-Ws[r * D + c], ld4(Ss + c * D + j), acc);
+      st4(Es + r * D + j, acc);
     }
     __syncthreads();
   };
@@ -207,12 +230,14 @@ __global__ void __launch_bounds__(4 * D)
     for (int idx = tid; idx < D * D; idx += NT) slot[idx] = Ss[idx];
     const long long s = t0 + (long long)ch * C;
     const int Cn = load_chunk(ch, false);
-    chunk_forward(s, Cn);
-    for (int idx = tid; idx < D * D; idx += NT) {  // S <- gam o S + Kb^T E
-      const int c = idx / D, j = idx % D;
-      float acc = gam[c] * Ss[idx];
-      for (int r = 0; r < C; ++r) acc = fmaf(Ks[r * D + c] * ELs[r * D + c], Es[r * D + j], acc);
-      Ss[idx] = acc;
+    chunk_forward(s, Cn, false);
+    for (int idx = tid; idx < D * D / 4; idx += NT) {  // S <- gam o S + Kb^T E
+      const int c = idx / (D / 4), j = 4 * (idx % (D / 4));
+      float4 acc = ld4(Ss + c * D + j);
+      acc = make_float4(gam[c] * acc.x, gam[c] * acc.y, gam[c] * acc.z, gam[c] * acc.w);
+#pragma unroll
+      for (int r = 0; r < C; ++r) acc = fma4(Ks[r * D + c] * ELs[r * D + c], ld4(Es + r * D + j), acc);
+      st4(Ss + c * D + j, acc);
     }
     __syncthreads();
   }
@@ -225,69 +250,61 @@ __global__ void __launch_bounds__(4 * D)
     for (int idx = tid; idx < D * D; idx += NT) Ss[idx] = slot[idx];
     const long long s = t0 + (long long)ch * C;
     const int Cn = load_chunk(ch, true);
-    chunk_forward(s, Cn);
+    chunk_forward(s, Cn, true);
 
     // 1. from the old dS': dE = Kb dS' + P^T dO, dKb = E dS'^T (R2), gam o rowsum(dS' o S)
-    for (int idx = tid; idx < C * D; idx += NT) {
-      const int r = idx / D, j = idx % D;
-      float acc = 0.f;
-      for (int c = 0; c < D; ++c) acc = fmaf(Ks[r * D + c] * ELs[r * D + c], dSs[c * D + j], acc);
-      for (int rr = r; rr < C; ++rr) acc = fmaf(Ps[rr * C + r], dOs[rr * D + j], acc);
-      dEs[idx] = acc;
+    for (int idx = tid; idx < C * D / 4; idx += NT) {
+      const int r = idx / (D / 4), j = 4 * (idx % (D / 4));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) acc = fma4(Ks[r * D + c] * ELs[r * D + c], ld4(dSs + c * D + j), acc);
+      for (int rr = r; rr < C; ++rr) acc = fma4(Ps[rr * C + r], ld4(dOs + rr * D + j), acc);
+      st4(dEs + r * D + j, acc);
     }
     for (int idx = tid; idx < C * D; idx += NT) {
       const int r = idx / D, c = idx % D;
-      float acc = 0.f;
-      for (int jj = 0; jj < D; ++jj) {
-        const int j = (jj + lane) & (D - 1);  // rotated: distinct banks across the warp
-        acc = fmaf(Es[r * D + j], dSs[c * D + j], acc);
-      }
-      R2[idx] = acc;
+      R2[idx] = rowdot<D>(Es + r * D, dSs + c * D, lane);
     }
-    for (int c = tid; c < D; c += NT) {
+    {  // gam o rowsum(dS' o S): four threads per channel, a quarter of the row each
+      const int c = tid >> 2, part = tid & 3;
       float acc = 0.f;
-      for (int j = 0; j < D; ++j) acc = fmaf(dSs[c * D + j], Ss[c * D + j], acc);
-      dGl[c] = gam[c] * acc;
+      for (int j = part * (D / 4); j < (part + 1) * (D / 4); j += 4) acc = dot4(ld4(dSs + c * D + j), ld4(Ss + c * D + j), acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (part == 0) dGl[c] = gam[c] * acc;
     }
     __syncthreads();
     // 2. dP = lower(dO E^T); dOS = dO S^T (R1, U is no longer needed)
     for (int idx = tid; idx < C * C; idx += NT) {
       const int r = idx / C, j = idx % C;
-      float acc = 0.f;
-      if (j <= r)
-        for (int d = 0; d < D; ++d) acc = fmaf(dOs[r * D + d], Es[j * D + d], acc);
-      dPs[idx] = acc;
+      dPs[idx] = j <= r ? rowdot<D>(dOs + r * D, Es + j * D, lane) : 0.f;
     }
     for (int idx = tid; idx < C * D; idx += NT) {
       const int r = idx / D, c = idx % D;
-      float acc = 0.f;
-      for (int jj = 0; jj < D; ++jj) {
-        const int j = (jj + lane) & (D - 1);
-        acc = fmaf(dOs[r * D + j], Ss[c * D + j], acc);
-      }
-      R1[idx] = acc;
+      R1[idx] = rowdot<D>(dOs + r * D, Ss + c * D, lane);
     }
     __syncthreads();
     // 3. dS = gam o dS' + (Q o Gam)^T dO - W^T dE  (in place: each element reads only itself of dS')
-    for (int idx = tid; idx < D * D; idx += NT) {
-      const int c = idx / D, j = idx % D;
-      float acc = gam[c] * dSs[idx];
+    for (int idx = tid; idx < D * D / 4; idx += NT) {
+      const int c = idx / (D / 4), j = 4 * (idx % (D / 4));
+      float4 acc = ld4(dSs + c * D + j);
+      acc = make_float4(gam[c] * acc.x, gam[c] * acc.y, gam[c] * acc.z, gam[c] * acc.w);
+#pragma unroll
       for (int r = 0; r < C; ++r) {
-        acc = fmaf(Qs[r * D + c] * GMs[r * D + c], dOs[r * D + j], acc);
-        acc = fmaf(-Ws[r * D + c], dEs[r * D + j], acc);
+        acc = fma4(Qs[r * D + c] * GMs[r * D + c], ld4(dOs + r * D + j), acc);
+        acc = fma4(-Ws[r * D + c], ld4(dEs + r * D + j), acc);
       }
-      dSs[idx] = acc;
+      st4(dSs + c * D + j, acc);
     }
     __syncthreads();
     // 4. dW = -dE S^T (over W)
     for (int idx = tid; idx < C * D; idx += NT) {
       const int r = idx / D, c = idx % D;
-      float acc = 0.f;
-      for (int jj = 0; jj < D; ++jj) {
-        const int j = (jj + lane) & (D - 1);
-        acc = fmaf(dEs[r * D + j], Ss[c * D + j], acc);
-      }
-      Ws[idx] = -acc;
+      Ws[idx] = -rowdot<D>(dEs + r * D, Ss + c * D, lane);
+    }
+    for (int idx = tid; idx < C * D; idx += NT) {  // V over E (E is no longer read)
+      const int r = idx / D, c = idx % D;
+      Es[idx] = r < Cn ? to_f32(v[row_off(s + r) + c]) : 0.f;
     }
     __syncthreads();
     // 5. dT = dE Bv^T + dW Bk^T
@@ -295,11 +312,12 @@ __global__ void __launch_bounds__(4 * D)
       const int r = idx / C, j = idx % C;
       float acc = 0.f;
       if (j < Cn) {
-        const size_t vo = row_off(s + j);
-        for (int d = 0; d < D; ++d) {
-          acc = fmaf(dEs[r * D + d], bs[j] * to_f32(v[vo + d]), acc);
-          acc = fmaf(Ws[r * D + d], bs[j] * Ks[j * D + d] * GMs[j * D + d], acc);
+        for (int d = 0; d < D; d += 4) {
+          acc = dot4(ld4(dEs + r * D + d), ld4(Es + j * D + d), acc);
+          const float4 kk = ld4(Ks + j * D + d), gm = ld4(GMs + j * D + d);
+          acc = dot4(ld4(Ws + r * D + d), make_float4(kk.x * gm.x, kk.y * gm.y, kk.z * gm.z, kk.w * gm.w), acc);
         }
+        acc *= bs[j];
       }
       dTs[idx] = acc;
     }
@@ -343,7 +361,7 @@ __global__ void __launch_bounds__(4 * D)
           dbv = fmaf(Ts[m * C + r], dEs[m * D + c], dbv);
           dbk = fmaf(Ts[m * C + r], Ws[m * D + c], dbk);
         }
-        const float vr = r < Cn ? to_f32(v[row_off(s + r) + c]) : 0.f;
+        const float vr = Es[e];
         atomicAdd(&dbs[r], dbv * vr + dbk * kr * GMs[e]);
         if (r < Cn) dv[row_off(s + r) + c] = bs[r] * dbv;
         const float dos = R1[e], dkb = R2[e];
