@@ -171,7 +171,9 @@ __global__ void __launch_bounds__(4 * D)
       const int pr = idx >> 1, half = idx & 1, r = pr / C, j = pr % C;
       float x = 0.f, p = 0.f;
       if (j <= r) {
-        for (int c = half * (D / 2); c < (half + 1) * (D / 2); ++c) {
+        // the pairs of a warp differ in j (rows of K and G): start each at its own channel
+        for (int cc = 0; cc < D / 2; ++cc) {
+          const int c = half * (D / 2) + ((cc + j) & (D / 2 - 1));
           const float kj = Ks[j * D + c] * __expf(Gs[r * D + c] - Gs[j * D + c]);
           x = fmaf(Ks[r * D + c], kj, x);
           if (with_p) p = fmaf(Qs[r * D + c], kj, p);
@@ -312,7 +314,8 @@ __global__ void __launch_bounds__(4 * D)
       const int r = idx / C, j = idx % C;
       float acc = 0.f;
       if (j < Cn) {
-        for (int d = 0; d < D; d += 4) {
+        for (int dd = 0; dd < D / 4; ++dd) {
+          const int d = 4 * ((dd + lane) & (D / 4 - 1));
           acc = dot4(ld4(dEs + r * D + d), ld4(Es + j * D + d), acc);
           const float4 kk = ld4(Ks + j * D + d), gm = ld4(GMs + j * D + d);
           acc = dot4(ld4(Ws + r * D + d), make_float4(kk.x * gm.x, kk.y * gm.y, kk.z * gm.z, kk.w * gm.w), acc);
@@ -348,7 +351,8 @@ __global__ void __launch_bounds__(4 * D)
     //    part, part + 4, ... both as a row (left factor) and as a column (right
     //    factor) of the pairwise terms, so no two threads write one element.
     {
-      const int c = tid >> 2, part = tid & 3;
+      // a warp covers 32 consecutive channels of one row group: conflict-free tile accesses
+      const int c = tid % D, part = tid / D;
       float dQa[C / 4], dKa[C / 4], dGa[C / 4];
       float kbsum = 0.f;  // sum over this thread's rows of dKb o Kb (for G_last)
 #pragma unroll
@@ -389,10 +393,15 @@ __global__ void __launch_bounds__(4 * D)
         dKa[i] = dK;
         dGa[i] = dG;
       }
-      // G_last terms go to the chunk's last row (row C - 1, owned by part 3)
-      kbsum += __shfl_xor_sync(0xffffffffu, kbsum, 1);
-      kbsum += __shfl_xor_sync(0xffffffffu, kbsum, 2);
-      if (part == (C - 1) % 4) dGa[C / 4 - 1] += kbsum + dGl[c];
+      // G_last terms go to the chunk's last row (row C - 1, owned by part 3);
+      // the four parts' sums of dKb o Kb meet in shared memory (over Mt/Ats, no longer read)
+      float* kbs = Mt;  // [4][D] floats fit in the two C x C tiles Mt, Ats (2 C^2 >= 4 D for D <= 128)
+      static_assert(2 * C * C >= 4 * D, "partial sums must fit in Mt and Ats");
+      __syncthreads();  // every thread is done reading Ats
+      kbs[part * D + c] = kbsum;
+      __syncthreads();
+      if (part == (C - 1) % 4)
+        dGa[C / 4 - 1] += kbs[c] + kbs[D + c] + kbs[2 * D + c] + kbs[3 * D + c] + dGl[c];
       // dQ, dK out; dG into a tile (over dE) for the reverse cumulative sum
 #pragma unroll
       for (int i = 0; i < C / 4; ++i) {
