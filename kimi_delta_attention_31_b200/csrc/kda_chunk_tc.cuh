@@ -96,9 +96,6 @@ constexpr uint32_t KB_DYN = KB_BYTES + 1024;
 // global loads around them.
 #define KDA_ALIGNED_DSMEM(name, raw) \
   uint8_t* name = (raw) + ((1024u - (ptx::smem_u32(raw) & 1023u)) & 1023u)
-__device__ __forceinline__ void st_bf16(uint8_t* p, float x) {
-  *reinterpret_cast<bf16*>(p) = __float2bfloat16_rn(x);
-}
 __device__ __forceinline__ uint4 pack8(const float* x) {
   uint4 r;
   r.x = ptx::pack_bf16x2(x[0], x[1]);
@@ -159,9 +156,6 @@ __device__ long long chunks_before_warp(const int32_t* cu, int n) {
   return acc;
 }
 
-__device__ __forceinline__ float sel4(int i, float a0, float a1, float a2, float a3) {
-  return i == 0 ? a0 : (i == 1 ? a1 : (i == 2 ? a2 : a3));
-}
 
 // ---------------------------------------------------------------------------
 // Kernel 1: chunk-local work, one CTA (256 threads) per (chunk, head).
