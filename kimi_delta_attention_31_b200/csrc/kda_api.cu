@@ -19,12 +19,7 @@ thread_local cudaEvent_t* t_prof_events = nullptr;
 thread_local int t_prof_count = 0;
 thread_local int t_seg_force = 0;  // kda_set_segment_chunks: 0 auto, > 0 fixed, < 0 never
 
-int current_sms() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return sms;
-}
+int current_sms() { return kda::current_sm_count(); }
 
 kda_status_t fail(kda_status_t st, const char* fmt, ...) {
   va_list ap;

@@ -436,16 +436,12 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
                              const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
                              float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens, int N,
                              int T, int H, float* ckpt, cudaStream_t stream) {
-  static int s_attr_device = -1;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static PerDeviceOnce s_attrs;
+  cudaError_t e = run_once_per_device(s_attrs, [] {
+    return cudaFuncSetAttribute(kda_chunk_bwd_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Cfg<D>::smem_bytes);
+  });
   if (e != cudaSuccess) return e;
-  if (s_attr_device != dev) {
-    e = cudaFuncSetAttribute(kda_chunk_bwd_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Cfg<D>::smem_bytes);
-    if (e != cudaSuccess) return e;
-    s_attr_device = dev;
-  }
   const long long units = (long long)N * H;
   if (units == 0) return cudaSuccess;
   kda_chunk_bwd_kernel<TIn, D><<<(unsigned)units, Cfg<D>::NT, Cfg<D>::smem_bytes, stream>>>(

@@ -216,14 +216,12 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
                               const int32_t* cu_seqlens, int N, int T, int H, int DV, int gmode,
                               cudaStream_t stream) {
   using Cfg = SimtCfg<DK, C>;
-  static bool attr_set = false;  // benign race: the attribute value is idempotent
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_simt_kernel<TIn, DK, C>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Cfg::smem_bytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce s_attrs;
+  cudaError_t e = run_once_per_device(s_attrs, [] {
+    return cudaFuncSetAttribute(kda_chunk_simt_kernel<TIn, DK, C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)Cfg::smem_bytes);
+  });
+  if (e != cudaSuccess) return e;
   const long long grid = (long long)N * H * (DV / Cfg::DVB);
   if (grid == 0) return cudaSuccess;
   kda_chunk_simt_kernel<TIn, DK, C><<<(unsigned)grid, Cfg::NT, Cfg::smem_bytes, stream>>>(

@@ -1164,27 +1164,22 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
                                    const int32_t* cu_seqlens, int N, int B, int T, int H,
                                    long long max_chunks, void* workspace, int gmode, int seg_chunks,
                                    cudaEvent_t* ev, cudaStream_t stream) {
-  static int s_attr_device = -1;
-  static int s_sms = 0;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (s_attr_device != dev) {
+  static PerDeviceOnce s_attrs;
+  cudaError_t e = run_once_per_device(s_attrs, [] {
     const void* fns[] = {(const void*)tc::kda_tc_chunk_local_kernel<kGateLogCh>,
                          (const void*)tc::kda_tc_chunk_local_kernel<kGateLogTok>,
                          (const void*)tc::kda_tc_chunk_local_kernel<kGateLogitF32>,
                          (const void*)tc::kda_tc_chunk_local_kernel<kGateLogitBf16>};
     for (const void* fn : fns) {
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::KA_DYN);
-      if (e != cudaSuccess) return e;
+      cudaError_t r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::KA_DYN);
+      if (r != cudaSuccess) return r;
     }
-    e = cudaFuncSetAttribute(tc::kda_tc_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc::KB_DYN);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&s_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    s_attr_device = dev;
-  }
+    return cudaFuncSetAttribute(tc::kda_tc_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)tc::KB_DYN);
+  });
+  if (e != cudaSuccess) return e;
+  const int s_sms = current_sm_count();
+  if (s_sms <= 0) return cudaErrorInvalidDevice;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int num_seqs = cu_seqlens ? N : 0;
   const long long items = max_chunks * H;

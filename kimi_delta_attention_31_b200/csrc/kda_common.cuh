@@ -4,7 +4,44 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace kda {
+
+// Host-side, per-device one-time setup (kernel attributes), safe to call from
+// several host threads at once: `setup` runs once per device and object.
+constexpr int kMaxDevices = 64;
+struct PerDeviceOnce {
+  std::mutex mu;
+  bool done[kMaxDevices] = {};
+};
+template <typename F>
+inline cudaError_t run_once_per_device(PerDeviceOnce& once, F&& setup) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return setup();
+  std::lock_guard<std::mutex> lock(once.mu);
+  if (once.done[dev]) return cudaSuccess;
+  e = setup();
+  if (e == cudaSuccess) once.done[dev] = true;
+  return e;
+}
+// SM count of the current device (cached per device, thread-safe).
+inline int current_sm_count() {
+  static std::mutex mu;
+  static int sms[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= kMaxDevices) {
+    int n = 0;
+    return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : 0;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms[dev] = 0;
+  return sms[dev];
+}
 
 // Device-side error word.  Bounded waits set it (never trap) when they give
 // up; the host reads and clears it through kda_device_error().
