@@ -417,6 +417,10 @@ __global__ void __launch_bounds__(256, 2)
         off[4] += t1.x; off[5] += t1.y; off[6] += t1.z; off[7] += t1.w;
       }
     }
+    if constexpr (kGate == kGateLogTok) {  // one gate per token: every channel has the same G
+#pragma unroll
+      for (int e = 1; e < 8; ++e) off[e] = off[0];
+    }
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
