@@ -799,6 +799,9 @@ __global__ void __launch_bounds__(256)
   float4 cur = S0 ? *reinterpret_cast<const float4*>(S0 + ((size_t)u * D + c) * D + j0 + jq)
                   : make_float4(0.f, 0.f, 0.f, 0.f);
   *reinterpret_cast<float4*>(&Ss[c][jq]) = cur;
+  // segment 0's entry state is S0 itself; the final pass reads this copy, so
+  // that an S_out aliasing S0 may be written while other segments still run
+  *reinterpret_cast<float4*>(seg_init + ((size_t)(u * P) * D + c) * D + j0 + jq) = cur;
   __syncthreads();
   for (int p = 0; p + 1 < P; ++p) {
     const float* Nm = maps + (size_t)((u * (P - 1) + p) * 2) * D * D;
@@ -911,7 +914,7 @@ __global__ void __launch_bounds__(256, 2)
     const int nc = (len + C - 1) / C;
     const size_t soff = ((size_t)u * D + c) * D + 64 * ch;
     const float* S_src = nullptr;
-    if (pass == kPassFinal && p > 0)
+    if (pass == kPassFinal)  // every segment's entry state, segment 0's included (a copy of S0)
       S_src = seg_init + ((size_t)(u * P + p) * D + c) * D + 64 * ch;
     else if (pass != kPassMaps && S0)
       S_src = S0 + soff;

@@ -64,3 +64,16 @@ def test_no_segments_where_units_fill_the_gpu(cuda_device, segments):
     assert kda.segment_chunks(8, 8192, 32) == 0      # the headline shape
     assert kda.segment_chunks(1, 520998, 32, 16) == 0  # packed inputs are never split
     assert kda.segment_chunks(1, 4096, 4) == 0        # too short to pay off
+
+
+def test_segments_with_the_final_state_aliasing_the_initial_state(cuda_device, segments):
+    """S_out may alias S0: with segments, the last segment writes S_out while
+    other segments still run, so no segment may read S0 itself then."""
+    inp = W.make_prefill(2, 2000, 3, 128, 128, "bf16", -4.0, 1.0, 0.05, seed=83, device=cuda_device)
+    segments(4)
+    o_ref, S_ref = _run(inp)
+    S0 = inp["S0"].clone()
+    o2, S2 = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0, None, 64, S_out=S0)
+    torch.cuda.synchronize()
+    assert S2.data_ptr() == S0.data_ptr()
+    assert torch.equal(o2, o_ref) and torch.equal(S2, S_ref)
