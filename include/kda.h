@@ -189,7 +189,10 @@ kda_status_t kda_recurrent_step_prep(const void* q, const void* k, const void* v
  *   cu_seqlens, num_seqs, B, T, H, dk, dv: as kda_chunk_fwd
  *   workspace     : at least kda_chunk_bwd_workspace_size(...) bytes: the state
  *                   at the start of every 16-token chunk, fp32.
- * Alignment: every pointer element-aligned.  One CTA per (sequence, head).
+ * Alignment: every pointer element-aligned.  No output may alias an input,
+ * the workspace or another output (KDA_ERR_INVALID_ARG for identical
+ * pointers; partial overlaps are the caller's to avoid).  One CTA per
+ * (sequence, head).
  */
 size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs);
 kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,

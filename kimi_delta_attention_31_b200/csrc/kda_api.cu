@@ -219,6 +219,17 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
   const void* f_ptrs[] = {g, beta, S0, dS_T, dq, dk, dv, dg, dbeta, dS0, cu_seqlens, workspace};
   for (const void* p : f_ptrs)
     if (p && !aligned_to(p, 4)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is not 4-byte aligned", fn, p);
+  {  // outputs are written while inputs are still read (in reverse chunk order): no aliasing
+    const void* outs[] = {dq, dk, dv, dg, dbeta, dS0, workspace};
+    const void* ins[] = {q, k, v, g, beta, S0, dout, dS_T};
+    for (int i = 0; i < 7; ++i) {
+      if (!outs[i]) continue;
+      for (const void* p : ins)
+        if (p == outs[i]) return fail(KDA_ERR_INVALID_ARG, "%s: an output aliases an input (%p)", fn, p);
+      for (int j = i + 1; j < 7; ++j)
+        if (outs[j] == outs[i]) return fail(KDA_ERR_INVALID_ARG, "%s: two outputs alias (%p)", fn, outs[i]);
+    }
+  }
   const size_t need = kda_chunk_bwd_workspace_size(B, T, H, dkh, dvh, num_seqs);
   if (need && (!workspace || workspace_bytes < need))
     return fail(KDA_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes, need);

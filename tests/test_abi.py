@@ -167,8 +167,10 @@ def test_chunk_bwd_validates_arguments():
     lib = kda.load_library()
     f = _fake()
 
-    def call(dtype=kda.KDA_BF16, d=128, dq=f, ws=None, wsb=0, B=1, T=64, cu=None, ns=0, q=f):
-        return lib.kda_chunk_bwd(q, f, f, f, f, None, f, None, dq, f, f, f, f, None, cu, ns, B, T, 2, d, d,
+    o1, o2, o3, o4 = _fake(0x7000), _fake(0x7100), _fake(0x7200), _fake(0x7300)
+
+    def call(dtype=kda.KDA_BF16, d=128, dq=_fake(0x7400), ws=None, wsb=0, B=1, T=64, cu=None, ns=0, q=f):
+        return lib.kda_chunk_bwd(q, f, f, f, f, None, f, None, dq, o1, o2, o3, o4, None, cu, ns, B, T, 2, d, d,
                                  dtype, ws, wsb, None)
 
     assert call() == 4                                # reached the workspace check
@@ -180,6 +182,14 @@ def test_chunk_bwd_validates_arguments():
     assert call(q=_fake(0x1001)) == 3                 # bf16 inputs need 2-byte alignment
     assert call(cu=f, ns=0) == 1
     assert call(B=0) == 0
+    # an output that aliases an input, or another output, is rejected
+    g_ = _fake(0x5000)
+    st = lib.kda_chunk_bwd(f, f, f, g_, _fake(0x5100), None, f, None, _fake(0x6000), _fake(0x6100), _fake(0x6200),
+                           g_, _fake(0x6300), None, None, 0, 1, 64, 2, 128, 128, kda.KDA_BF16, None, 0, None)
+    assert st == 1 and "alias" in kda.last_error()
+    st = lib.kda_chunk_bwd(f, f, f, g_, _fake(0x5100), None, f, None, _fake(0x6000), _fake(0x6000), _fake(0x6200),
+                           _fake(0x6400), _fake(0x6300), None, None, 0, 1, 64, 2, 128, 128, kda.KDA_BF16, None, 0, None)
+    assert st == 1 and "alias" in kda.last_error()
     need = lib.kda_chunk_bwd_workspace_size(1, 64, 2, 128, 128, 0)
     assert need == 4 * 2 * 128 * 128 * 4              # 4 chunks of 16 tokens x 2 heads x fp32 states
     assert call(ws=_fake(0x4000), wsb=need - 1) == 4
