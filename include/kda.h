@@ -270,6 +270,22 @@ kda_status_t kda_set_segment_chunks(int chunks);
 int kda_segment_chunks(int B, int T, int H, int num_seqs);
 
 /*
+ * Which kernel forms the per-chunk operands of the tensor-core prefill
+ * ("Deriving Kimi Delta Attention from scratch", section 6: everything of a
+ * chunk that does not involve the carried state).  Two kernels compute the
+ * same result: a warp-specialised one (one CTA per SM; one warp group builds
+ * the decay-scaled operands of a chunk while the other inverts the previous
+ * chunk's I + A; inputs arrive by tensor-map TMA) and a two-CTA-per-SM one.
+ * For the calling thread's later calls: 0 (default) uses the warp-specialised
+ * kernel where it applies -- per-channel log-decay gate (kda_chunk_fwd), one
+ * sequence per batch row (cu_seqlens == NULL) -- and the two-CTA kernel for
+ * the chunks whose log-decay over the chunk falls below -80 on some channel
+ * and for every other call; 1 = the two-CTA kernel always.  Other values:
+ * KDA_ERR_INVALID_ARG, setting unchanged.
+ */
+kda_status_t kda_set_local_kernel(int variant);
+
+/*
  * Number of phases one kda_chunk_fwd call with these arguments runs: 1 for
  * the fp32-arithmetic path (one kernel); 2 for the tensor-core path (the
  * chunk-local kernel, then the state pass -- one kernel, or three when the

@@ -38,7 +38,8 @@ EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step
             "kda_last_error", "kda_device_error", "kda_chunk_fwd_launches", "kda_profile_events",
             "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step",
             "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait",
-            "kda_set_segment_chunks", "kda_segment_chunks", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size")
+            "kda_set_segment_chunks", "kda_segment_chunks", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
+            "kda_set_local_kernel")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -103,6 +104,8 @@ def load_library():
         lib.kda_set_segment_chunks.restype = i32
         lib.kda_segment_chunks.argtypes = [i32] * 4
         lib.kda_segment_chunks.restype = i32
+        lib.kda_set_local_kernel.argtypes = [i32]
+        lib.kda_set_local_kernel.restype = i32
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, vp]
         lib.kda_selftest_bounded_wait.restype = i32
         lib.kda_version.argtypes = []
@@ -388,6 +391,13 @@ def set_segment_chunks(chunks: int) -> None:
     """Sequence segments of the tensor-core prefill for this thread's later
     calls: 0 = automatic (default), L > 0 = L chunks per segment, < 0 = off."""
     _check(load_library().kda_set_segment_chunks(int(chunks)))
+
+
+def set_local_kernel(variant: int) -> None:
+    """Chunk-local kernel of the tensor-core prefill for this thread's later
+    calls: 0 = the warp-specialised kernel where it applies (default),
+    1 = the two-CTA-per-SM kernel always."""
+    _check(load_library().kda_set_local_kernel(int(variant)))
 
 
 def segment_chunks(B, T, H, num_seqs=0) -> int:

@@ -18,6 +18,7 @@ thread_local char t_err[512] = "";
 thread_local cudaEvent_t* t_prof_events = nullptr;
 thread_local int t_prof_count = 0;
 thread_local int t_seg_force = 0;  // kda_set_segment_chunks: 0 auto, > 0 fixed, < 0 never
+thread_local int t_local_kernel = 0;  // kda_set_local_kernel: 0 default, 1 two-CTA kernel only
 
 int current_sms() { return kda::current_sm_count(); }
 
@@ -131,7 +132,8 @@ kda_status_t chunk_fwd_impl(const char* fn, const void* q, const void* k, const 
                              static_cast<const __nv_bfloat16*>(k),
                              static_cast<const __nv_bfloat16*>(v), g, beta, S0,
                              static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H,
-                             max_chunks(B, T, num_seqs, chunk_size), workspace, gmode, seg, ev, stream);
+                             max_chunks(B, T, num_seqs, chunk_size), workspace, gmode, seg,
+                             t_local_kernel, ev, stream);
   } else if (dtype == KDA_F32) {
     e = dispatch_chunk_simt<float>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, T,
                                    H, dv, gmode, stream);
@@ -258,6 +260,13 @@ kda_status_t kda_set_segment_chunks(int chunks) {
 
 int kda_segment_chunks(int B, int T, int H, int num_seqs) {
   return kda::tc_segment_chunks(B, T, H, num_seqs, current_sms(), t_seg_force);
+}
+
+kda_status_t kda_set_local_kernel(int variant) {
+  t_err[0] = 0;
+  if (variant != 0 && variant != 1) return fail(KDA_ERR_INVALID_ARG, "kda_set_local_kernel: variant %d", variant);
+  t_local_kernel = variant;
+  return KDA_OK;
 }
 
 kda_status_t kda_profile_events(cudaEvent_t* events, int count) {

@@ -218,6 +218,122 @@ __device__ __forceinline__ void normalise_rows(float* kv, float* qv, float nk, f
   }
 }
 
+// Phase 4 on the single-reference path: TMEM columns [tm, tm + 64) hold, in
+// lanes 0..63, A'_rj and in lanes 64..127, P'_rj.  Writes A = beta_r A'_rj
+// (j < r, fp32, row stride AS_LD) and P (j <= r, bf16 K-major 128-byte
+// swizzled, zero above the diagonal).  Eight warps; `warp` is the warp's
+// index in the CTA (its TMEM lane quarter is warp mod 4) and `w8` its index
+// in the group of eight (which 32 columns it takes).
+__device__ __forceinline__ void scatter_single_ref(uint32_t tm, const float* s_beta, float* As, uint8_t* Pt,
+                                                   int warp, int w8, int lane) {
+  const int qd = warp & 3, ch = w8 >> 2;
+  const int rho = 32 * qd + lane, r = rho & 63, j0 = 32 * ch;
+  float x[32];
+  const uint32_t ta = tm + ((uint32_t)(32 * qd) << 16) + j0;
+  ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
+  ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+  ptx::tmem_wait_ld();
+  if (rho < 64) {  // warp-uniform
+    const float br = s_beta[r];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = (j0 + e < r) ? br * x[e] : 0.f;
+    float4* dst = reinterpret_cast<float4*>(As + r * AS_LD + j0);
+#pragma unroll
+    for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(x[4 * v4], x[4 * v4 + 1], x[4 * v4 + 2], x[4 * v4 + 3]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = (j0 + e <= r) ? x[e] : 0.f;
+#pragma unroll
+    for (int k8 = 0; k8 < 4; ++k8) *reinterpret_cast<uint4*>(Pt + ptx::sw128_chunk(r, 4 * ch + k8)) = pack8(x + 8 * k8);
+  }
+}
+
+// Phase 5: T = (I + A)^{-1} (A strictly lower, fp32 in As), blocked by 16.
+// Diagonal blocks by forward substitution in fp32, one column per 4 lanes;
+// then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ by distance below the diagonal,
+// one warp per block, TF32 warp MMAs with fp32 accumulation.  Finally
+// T diag(beta) in bf16 (K-major [64 r][64 j], 128-byte swizzle) into Tt.
+// 256 threads: t in [0, 256), w = t / 32; `sync` is their barrier.
+template <typename Sync>
+__device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* Mt, const float* s_beta, uint8_t* Tt,
+                                             int t, int w, int lane, Sync sync) {
+  {
+    const int j = t >> 2, part = t & 3;  // column j of T; this lane keeps rows 4 m + part
+    const int Ib = j >> 4, jj = j & 15, o = 16 * Ib;
+    float x[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) x[m] = (4 * m + part == jj) ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+      float acc = 0.f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if (4 * m < i) acc = fmaf(As[(o + i) * AS_LD + o + 4 * m + part], x[m], acc);  // A[i][>=i] == 0
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if ((i & 3) == part && i > jj) x[i >> 2] = -acc;
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) Ts[(o + 4 * m + part) * AS_LD + o + jj] = x[m];
+  }
+  sync();
+#pragma unroll
+  for (int dist = 1; dist <= 3; ++dist) {
+    if (w < 4 - dist) {
+      const int Jc = w, Ir = w + dist;
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int kk = 0; kk < dist; ++kk) {
+        const int K = Jc + kk;
+        warp_gemm16(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
+      }
+      float* mt = Mt + w * 16 * MT_LD;
+      warp_store16(mt, MT_LD, acc, 1.f, lane);
+      __syncwarp();
+      float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      warp_gemm16(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
+      warp_store16(Ts + 16 * Ir * AS_LD + 16 * Jc, AS_LD, acc2, -1.f, lane);
+    }
+    sync();
+  }
+  // bf16 T diag(beta); blocks above the diagonal are zero
+  for (int idx = t; idx < 512; idx += 256) {
+    const int rr = idx >> 3, k8 = idx & 7;
+    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if ((k8 >> 1) <= (rr >> 4)) {
+      const float4 t0 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8);
+      const float4 t1 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8 + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(s_beta + 8 * k8);
+      const float4 b1 = *reinterpret_cast<const float4*>(s_beta + 8 * k8 + 4);
+      y[0] = t0.x * b0.x; y[1] = t0.y * b0.y; y[2] = t0.z * b0.z; y[3] = t0.w * b0.w;
+      y[4] = t1.x * b1.x; y[5] = t1.y * b1.y; y[6] = t1.z * b1.z; y[7] = t1.w * b1.w;
+    }
+    *reinterpret_cast<uint4*>(Tt + ptx::sw128_chunk(rr, k8)) = pack8(y);
+  }
+}
+
+// Phase 6 epilogue: TMEM columns [tm, tm + 64) = W^T, [tm + 64, tm + 128) = U^T
+// (lane = channel) to bf16 K-major rows of the image staging area.  Eight
+// warps, arguments as for scatter_single_ref.
+__device__ __forceinline__ void stage_w_u(uint32_t tm, uint8_t* stage, int warp, int w8, int lane) {
+  const int qd = warp & 3, ch = w8 >> 2;
+  const int row = 32 * qd + lane;  // dk channel (W^T) or dv channel (U^T)
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float x[32];
+    const uint32_t ta = tm + ((uint32_t)(32 * qd) << 16) + 64 * ch + 32 * hh;
+    ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
+    ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int k8 = 0; k8 < 4; ++k8) {
+      const uint4 pk = pack8(x + 8 * k8);
+      const uint32_t off = ptx::sw128_chunk(row, 4 * hh + k8);
+      *reinterpret_cast<uint4*>(stage + (ch == 0 ? IMG_A1 : IMG_U) + off) = pk;
+    }
+  }
+}
+
 // kGate (GateMode): what the gate argument holds -- log alpha per key channel
 // (KDA) or per token (Gated DeltaNet), or raw per-channel logits in fp32 or
 // bf16, in which case q and k rows are also L2-normalised and beta is the
@@ -228,7 +344,8 @@ __global__ void __launch_bounds__(256, 2)
                               const bf16* __restrict__ v, const void* __restrict__ gate,
                               const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                               int num_seqs, int T, int H, uint32_t num_items, FastDiv fdH, FastDiv fdC,
-                              uint8_t* __restrict__ ws) {
+                              uint8_t* __restrict__ ws, const uint32_t* __restrict__ item_list,
+                              const uint32_t* __restrict__ item_cnt, uint32_t list_cap) {
   __shared__ __align__(16) float s_beta[C];
   __shared__ float s_nrm[2][C];  // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
   constexpr bool kPrep = gate_prep(kGate);
@@ -257,10 +374,13 @@ __global__ void __launch_bounds__(256, 2)
   ptx::tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  // Persistent: this CTA handles items (chunk * H + head) blockIdx.x, + gridDim.x, ...
-  // Each processed item completes s_bar twice (parities 0 then 1).
+  // Persistent: this CTA handles items (chunk * H + head) blockIdx.x, + gridDim.x, ...,
+  // or, given an item list, entries [0, item_cnt[b]) of list b = blockIdx.x
+  // (capacity list_cap each).  Each processed item completes s_bar twice (parities 0 then 1).
   // item = chunk * H + head; unpacked chunk = sequence * fdC.d + chunk-in-sequence (num_items < 2^31)
-  for (uint32_t item = blockIdx.x; item < num_items; item += gridDim.x) {
+  const uint32_t n_iter = item_list ? min(item_cnt[blockIdx.x], list_cap) : num_items;
+  for (uint32_t it = item_list ? 0u : blockIdx.x; it < n_iter; it += item_list ? 1u : gridDim.x) {
+  const uint32_t item = item_list ? item_list[(size_t)blockIdx.x * list_cap + it] : it;
   const uint32_t ci = fdiv(item, fdH);
   const int h = (int)(item - ci * (uint32_t)H);
 
@@ -294,7 +414,7 @@ __global__ void __launch_bounds__(256, 2)
 
   // L2 hint for this CTA's next item (packed-free layout only): its q, k, v, g
   // rows, one 128-byte line per lane.
-  if (!cu_seqlens && item + gridDim.x < num_items) {
+  if (!cu_seqlens && !item_list && item + gridDim.x < num_items) {
     const uint32_t nb = item + gridDim.x;
     const uint32_t nci = fdiv(nb, fdH);
     const int nh = (int)(nb - nci * (uint32_t)H);
@@ -592,28 +712,8 @@ __global__ void __launch_bounds__(256, 2)
   ptx::tc_fence_after();
 
   // ---- 4. scatter A (fp32, beta-scaled) and P (bf16, lower incl. diagonal, zero above)
-  if (fast) {  // TMEM columns 0..63 hold whole rows; warp half ch takes columns 32 ch ..
-    const int qd = warp & 3, ch = warp >> 2;
-    const int rho = 32 * qd + lane, r = rho & 63, j0 = 32 * ch;
-    float x[32];
-    const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + j0;
-    ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
-    ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
-    ptx::tmem_wait_ld();
-    if (rho < 64) {  // warp-uniform
-      const float br = s_beta[r];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) x[e] = (j0 + e < r) ? br * x[e] : 0.f;
-      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(sm + KA_AS) + r * AS_LD + j0);
-#pragma unroll
-      for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(x[4 * v4], x[4 * v4 + 1], x[4 * v4 + 2], x[4 * v4 + 3]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) x[e] = (j0 + e <= r) ? x[e] : 0.f;
-#pragma unroll
-      for (int k8 = 0; k8 < 4; ++k8)
-        *reinterpret_cast<uint4*>(sm + KA_PT + ptx::sw128_chunk(r, 4 * ch + k8)) = pack8(x + 8 * k8);
-    }
+  if (fast) {  // TMEM columns 0..63 hold whole rows
+    scatter_single_ref(tmem, s_beta, reinterpret_cast<float*>(sm + KA_AS), sm + KA_PT, warp, warp, lane);
   } else {
     const int qd = warp & 3, ch = warp >> 2;
     const int rho = 32 * qd + lane;
@@ -662,68 +762,10 @@ __global__ void __launch_bounds__(256, 2)
   ptx::tc_fence_before();
   __syncthreads();
 
-  // ---- 5. T = (I + A)^{-1}, blocked by 16.  Diagonal blocks: forward
-  //         substitution in fp32, one column per 4 lanes (warp shuffles).
-  //         Then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ by distance below the
-  //         diagonal, one warp per block, TF32 warp MMAs with fp32 accumulation.
-  {
-    const float* As = reinterpret_cast<const float*>(sm + KA_AS);
-    float* Ts = reinterpret_cast<float*>(sm + KA_TS);
-    float* Mt = reinterpret_cast<float*>(sm + KA_MT);
-    {
-      const int j = tid >> 2, part = tid & 3;  // column j of T; this lane keeps rows 4 m + part
-      const int Ib = j >> 4, jj = j & 15, o = 16 * Ib;
-      float x[4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) x[m] = (4 * m + part == jj) ? 1.f : 0.f;
-#pragma unroll
-      for (int i = 1; i < 16; ++i) {
-        float acc = 0.f;
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-          if (4 * m < i) acc = fmaf(As[(o + i) * AS_LD + o + 4 * m + part], x[m], acc);  // A[i][>=i] == 0
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if ((i & 3) == part && i > jj) x[i >> 2] = -acc;
-      }
-#pragma unroll
-      for (int m = 0; m < 4; ++m) Ts[(o + 4 * m + part) * AS_LD + o + jj] = x[m];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int dist = 1; dist <= 3; ++dist) {
-      if (warp < 4 - dist) {
-        const int Jc = warp, Ir = warp + dist;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int kk = 0; kk < dist; ++kk) {
-          const int K = Jc + kk;
-          warp_gemm16(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
-        }
-        float* mt = Mt + warp * 16 * MT_LD;
-        warp_store16(mt, MT_LD, acc, 1.f, lane);
-        __syncwarp();
-        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        warp_gemm16(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
-        warp_store16(Ts + 16 * Ir * AS_LD + 16 * Jc, AS_LD, acc2, -1.f, lane);
-      }
-      __syncthreads();
-    }
-    // bf16 T diag(beta) (K-major [64 r][64 j]); blocks above the diagonal are zero
-    for (int idx = tid; idx < 512; idx += 256) {
-      const int rr = idx >> 3, k8 = idx & 7;
-      float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if ((k8 >> 1) <= (rr >> 4)) {
-        const float4 t0 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8);
-        const float4 t1 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8 + 4);
-        const float4 b0 = *reinterpret_cast<const float4*>(s_beta + 8 * k8);
-        const float4 b1 = *reinterpret_cast<const float4*>(s_beta + 8 * k8 + 4);
-        y[0] = t0.x * b0.x; y[1] = t0.y * b0.y; y[2] = t0.z * b0.z; y[3] = t0.w * b0.w;
-        y[4] = t1.x * b1.x; y[5] = t1.y * b1.y; y[6] = t1.z * b1.z; y[7] = t1.w * b1.w;
-      }
-      *reinterpret_cast<uint4*>(sm + KA_TT + ptx::sw128_chunk(rr, k8)) = pack8(y);
-    }
-  }
+  // ---- 5. T = (I + A)^{-1} and T diag(beta) in bf16
+  solve_t_beta(reinterpret_cast<const float*>(sm + KA_AS), reinterpret_cast<float*>(sm + KA_TS),
+               reinterpret_cast<float*>(sm + KA_MT), s_beta, sm + KA_TT, tid, warp, lane,
+               [] { __syncthreads(); });
 
   // ---- 6. W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
   ptx::fence_proxy_async_smem();
@@ -745,24 +787,7 @@ __global__ void __launch_bounds__(256, 2)
   }
   ptx::mbar_wait_bounded(&s_bar, 1);  // second completion of this item
   ptx::tc_fence_after();
-  {
-    const int qd = warp & 3, ch = warp >> 2;
-    const int row = 32 * qd + lane;  // dk channel (W^T) or dv channel (U^T)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float x[32];
-      const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + 64 * ch + 32 * hh;
-      ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
-      ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
-      ptx::tmem_wait_ld();
-#pragma unroll
-      for (int k8 = 0; k8 < 4; ++k8) {
-        const uint4 pk = pack8(x + 8 * k8);
-        const uint32_t off = ptx::sw128_chunk(row, 4 * hh + k8);
-        *reinterpret_cast<uint4*>(sm + KA_IMG_STAGE + (ch == 0 ? IMG_A1 : IMG_U) + off) = pk;
-      }
-    }
-  }
+  stage_w_u(tmem, sm + KA_IMG_STAGE, warp, warp, lane);
 
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
@@ -1117,6 +1142,11 @@ __global__ void __launch_bounds__(256, 2)
 }
 
 }  // namespace tc
+}  // namespace kda
+
+#include "kda_chunk_ws.cuh"  // warp-specialised chunk-local kernel
+
+namespace kda {
 
 // Chunks per sequence segment for the state pass, or 0 for none.  Segments
 // pay off when the (sequence, head) units are too few to fill the SMs and
@@ -1147,21 +1177,25 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
 }
 
 // Workspace: the per-chunk images, then (segmented runs) the maps [N | M] of
-// every segment but the last and the entry state of every segment, fp32.
+// every segment but the last and the entry state of every segment, fp32,
+// then the warp-specialised kernel's per-CTA item lists (at most
+// items + kMaxListCtas entries and kMaxListCtas counts, uint32).
+constexpr int kMaxListCtas = 1024;
 struct TcWorkspace {
-  size_t images, maps, seg_init, total;
+  size_t images, maps, seg_init, lists, total;
 };
 inline TcWorkspace tc_workspace_layout(long long max_chunks, int H, long long units, int T, int seg_chunks) {
   TcWorkspace w{};
   w.images = (size_t)max_chunks * (size_t)H * tc::IMG_BYTES;
-  w.maps = w.seg_init = w.total = (w.images + 255) & ~(size_t)255;
+  w.maps = w.seg_init = w.lists = (w.images + 255) & ~(size_t)255;
   if (seg_chunks > 0) {
     const long long nc = (T + tc::C - 1) / tc::C;
     const long long P = (nc + seg_chunks - 1) / seg_chunks;
     const size_t mat = (size_t)tc::D * tc::D * sizeof(float);
     w.seg_init = w.maps + (size_t)units * (size_t)(P - 1) * 2 * mat;
-    w.total = w.seg_init + (size_t)units * (size_t)P * mat;
+    w.lists = w.seg_init + (size_t)units * (size_t)P * mat;
   }
+  w.total = w.lists + ((size_t)max_chunks * (size_t)H + 2 * kMaxListCtas) * sizeof(uint32_t);
   return w;
 }
 
@@ -1170,7 +1204,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
                                    const float* S0, __nv_bfloat16* o, float* S_out,
                                    const int32_t* cu_seqlens, int N, int B, int T, int H,
                                    long long max_chunks, void* workspace, int gmode, int seg_chunks,
-                                   cudaEvent_t* ev, cudaStream_t stream) {
+                                   int local_kernel, cudaEvent_t* ev, cudaStream_t stream) {
   static PerDeviceOnce s_attrs;
   cudaError_t e = run_once_per_device(s_attrs, [] {
     const void* fns[] = {(const void*)tc::kda_tc_chunk_local_kernel<kGateLogCh>,
@@ -1193,12 +1227,21 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   if (items >= (1LL << 31)) return cudaErrorInvalidValue;  // item indices are 32-bit
   const FastDiv fdH = make_fastdiv((uint32_t)H);
   const FastDiv fdC = make_fastdiv((uint32_t)std::max(1, (T + tc::C - 1) / tc::C));
-  if (items > 0) {
+  // The warp-specialised kernel takes per-channel log-decays on the one-row-per-
+  // sequence layout; `local_kernel` == 1 keeps every call on the two-CTA kernel.
+  const bool use_ws = items > 0 && local_kernel != 1 && gmode == kGateLogCh && !cu_seqlens &&
+                      (long long)B * T < (1LL << 31) && ws::ws_kernel_available();
+  if (use_ws) {
+    const TcWorkspace lay = tc_workspace_layout(max_chunks, H, N * (long long)H, T, seg_chunks);
+    e = ws::launch_ws_local(q, k, v, static_cast<const float*>(g), beta, B, T, H, items, fdH, fdC, ws,
+                            reinterpret_cast<uint32_t*>(ws + lay.lists), std::min(s_sms, kMaxListCtas), stream);
+    if (e != cudaSuccess) return e;
+  } else if (items > 0) {
     const int gridA = (int)(items < 2LL * s_sms ? items : 2LL * s_sms);
 #define KDA_TC_LOCAL(M)                                                                            \
   tc::kda_tc_chunk_local_kernel<M><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens, \
                                                                        num_seqs, T, H, (uint32_t)items, fdH, \
-                                                                       fdC, ws)
+                                                                       fdC, ws, nullptr, nullptr, 0u)
     switch (gmode) {
       case kGateLogCh: KDA_TC_LOCAL(kGateLogCh); break;
       case kGateLogTok: KDA_TC_LOCAL(kGateLogTok); break;

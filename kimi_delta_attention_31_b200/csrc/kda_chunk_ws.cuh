@@ -1,0 +1,526 @@
+// kda_chunk_ws.cuh -- warp-specialised chunk-local kernel for the KDA prefill
+// (bf16 q, k, v; dk = dv = 128; C = 64; per-channel log-decay gate; one
+// sequence per batch row).  It computes the same per-(chunk, head) image as
+// kda_tc_chunk_local_kernel ("Deriving Kimi Delta Attention from scratch",
+// section 6, chunked mode; "Linear / sparse attention" tutorial, section 5.3
+// WY representation): P, U^T, [W; Q e^G], Kbar and gamma, on the
+// single-reference path.
+//
+// One CTA per SM, 16 warps in two groups that work on consecutive items at
+// the same time:
+//   builder (warps 0..7): raw k, q, g rows arrive by tensor-map TMA; the
+//     group forms the cumulative log-decays G, the decay-scaled operands
+//     [K e^G; Q e^G] (double-buffered) and K e^-G, writes Kbar, Q e^G and
+//     gamma to the image, and issues the [A'; P'] MMA into one of two TMEM
+//     accumulators.  Its thread 0 starts the next item's TMA as soon as the
+//     group has read the raw rows, so that load overlaps the build.
+//   solver (warps 8..15): scatters A and P out of TMEM, inverts I + A,
+//     issues the W^T / U^T MMAs (V comes straight from TMA in the MMA's
+//     layout), stages P, U^T and W^T and stores them with one bulk copy.
+// Items whose chunk decays below the single-reference range on some channel
+// (min G_last < -80) are not built here: the builder appends them to this
+// CTA's item list, and the two-CTA kernel runs that list afterwards with the
+// 16-token block references.
+//
+// Hand-offs (all mbarriers, one completion per item unless noted):
+//   raw_full      TMA bytes of k, q, g                     builder waits
+//   v_full        TMA bytes of V                           solver thread 0 waits
+//   a_done[slot]  [A'; P'] MMA complete + builder arrive   solver waits; builder
+//                 (count 2; per slot: items n, n+2, ...)   waits item n-1's (RB reuse)
+//   b_done[slot]  W^T / U^T MMA complete (or skip arrive)  solver waits; builder
+//                 (per slot: items n, n+2, ...)            waits item n-2's (slot reuse)
+// Per-slot barriers keep every waiter at most one phase behind: the builder
+// cannot pass item n+1 before item n-1's b_done, and the solver cannot pass
+// item n-1 before item n's a_done, so b_done[slot] is never ahead of item n-2
+// when the builder waits for it, and a_done[slot] never ahead of item n when
+// the solver does.  Parity waits are therefore exact.
+// Every wait is bounded: on a timeout the CTA raises the device error word,
+// stops issuing TMA copies and MMAs, runs its remaining items through without
+// waiting, and drains what is still in flight before it exits.
+//
+// Included by kda_chunk_tc.cuh after its kernels (it uses their helpers).
+#pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace kda {
+namespace ws {
+
+using tc::C;
+using tc::D;
+using tc::IMG_A1;
+using tc::IMG_BYTES;
+using tc::IMG_G;
+using tc::IMG_KB;
+using tc::IMG_P;
+using tc::IMG_U;
+
+// shared memory (dynamic, 1024-aligned base)
+constexpr uint32_t WS_RAWK = 0;            // k rows [64 tok][128 ch] bf16, row-major        16384
+constexpr uint32_t WS_RAWQ = 16384;        // q rows                                          16384
+constexpr uint32_t WS_RAWG = 32768;        // g rows [64 tok][128 ch] fp32                    32768
+constexpr uint32_t WS_V = 65536;           // V MN-major 2 panels [64 tok][64 dv], 128-B swizzle 16384
+constexpr uint32_t WS_L3 = 81920;          // 2 slots x [K e^G; Q e^G] K-major, 2 K-panels of 128 rows 2 x 32768
+constexpr uint32_t WS_L3_SLOT = 32768;
+constexpr uint32_t WS_RB = 147456;         // K e^-G K-major 2 panels [64][64]                16384
+constexpr uint32_t WS_ST = 163840;         // staging P | U^T | W^T in image order            40960
+constexpr uint32_t WS_AS = WS_ST + 8192;   // A fp32 [64][68], over the U^T / W^T staging     17408
+constexpr uint32_t WS_TS = WS_AS + 17408;  // T fp32 [64][68]                                 17408
+constexpr uint32_t WS_MT = WS_TS + 17408;  // block products [3][16][20]                      3840
+constexpr uint32_t WS_TT = 210944;         // T diag(beta) bf16 K-major [64][64]              8192
+constexpr uint32_t WS_TOT = 219136;        // row-group totals of g [16][128] fp32            8192
+constexpr uint32_t WS_BYTES = WS_TOT + 8192;
+constexpr uint32_t WS_DYN = WS_BYTES + 1024;
+constexpr uint32_t WS_STAGE_BYTES = IMG_A1 + 16384 - IMG_P;
+static_assert(WS_MT + 3 * 16 * tc::MT_LD * 4 <= WS_TT, "solver buffers overlap");
+static_assert(WS_ST + WS_STAGE_BYTES <= WS_TS + 17408, "staging layout");
+static_assert(WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_V % 1024 == 0, "alignment");
+
+constexpr uint32_t kRawBytes = 2 * C * D * 2 + C * D * 4;  // k, q (bf16) and g (fp32)
+constexpr uint32_t kVBytes = C * D * 2;
+constexpr uint32_t kTmemCols = 256;  // [A'; P'] slot 0 | slot 1 | W^T | U^T, 64 columns each
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct ItemPos {
+  long long s0;  // first token (row of the [tokens, H, D] tensors)
+  int h, Cn;     // head, valid rows of the chunk
+};
+__device__ __forceinline__ ItemPos item_pos(uint32_t item, int T, int H, const FastDiv& fdH, const FastDiv& fdC) {
+  const uint32_t ci = fdiv(item, fdH);
+  const uint32_t bq = fdiv(ci, fdC);
+  const int cc = (int)(ci - bq * fdC.d);
+  ItemPos p;
+  p.h = (int)(item - ci * (uint32_t)H);
+  p.s0 = (long long)bq * T + (long long)cc * C;
+  p.Cn = min(C, T - cc * C);
+  return p;
+}
+
+// Bounded wait that also gives up at once when another thread of the CTA has
+// already timed out (`abort_flag`), so that a broken hand-off costs one limit,
+// not one per remaining item.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              uint64_t limit_ns = 4000000000ull) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      raise_device_error(kDevErrWaitTimeout);
+      return false;
+    }
+  }
+}
+
+template <int kGate>
+__global__ void __launch_bounds__(512, 1)
+    kda_ws_chunk_local_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                              const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
+                              const float* __restrict__ beta, int T, int H, uint32_t num_items, FastDiv fdH,
+                              FastDiv fdC, uint8_t* __restrict__ ws, uint32_t* __restrict__ steep_list,
+                              uint32_t* __restrict__ steep_cnt, uint32_t list_cap) {
+  static_assert(kGate == kGateLogCh, "the warp-specialised kernel takes per-channel log-decays");
+  __shared__ __align__(16) float s_beta[2][C];
+  __shared__ __align__(16) float s_glast[D];  // G at the chunk's last row
+  __shared__ __align__(8) uint64_t s_raw_full, s_v_full, s_a_done[2], s_b_done[2], s_drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_skip[2];
+  __shared__ int s_abort;
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
+  KDA_ALIGNED_DSMEM(sm, dsm_raw);
+  const uint32_t sb = ptx::smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = &s_abort;
+  const uint32_t grid = gridDim.x;
+
+  if (warp == 0) {
+    ptx::tmem_alloc(&s_tmem, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  if (tid == 32) {
+    ptx::mbar_init(&s_raw_full, 1);
+    ptx::mbar_init(&s_v_full, 1);
+    ptx::mbar_init(&s_a_done[0], 2);
+    ptx::mbar_init(&s_a_done[1], 2);
+    ptx::mbar_init(&s_b_done[0], 1);
+    ptx::mbar_init(&s_b_done[1], 1);
+    ptx::mbar_init(&s_drain, 2);
+    s_abort = 0;
+    s_skip[0] = s_skip[1] = 0;
+    ptx::fence_mbar_init();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  auto issue_raw = [&](uint32_t item) {
+    const ItemPos p = item_pos(item, T, H, fdH, fdC);
+    ptx::mbar_arrive_expect_tx(&s_raw_full, kRawBytes);
+    ptx::tma_load_3d(sm + WS_RAWK, &tm_k, 0, p.h, (int)p.s0, &s_raw_full);
+    ptx::tma_load_3d(sm + WS_RAWQ, &tm_q, 0, p.h, (int)p.s0, &s_raw_full);
+    ptx::tma_load_3d(sm + WS_RAWG, &tm_g, 0, p.h, (int)p.s0, &s_raw_full);
+  };
+  auto issue_v = [&](uint32_t item) {
+    const ItemPos p = item_pos(item, T, H, fdH, fdC);
+    ptx::mbar_arrive_expect_tx(&s_v_full, kVBytes);
+    ptx::tma_load_3d(sm + WS_V, &tm_v, 0, p.h, (int)p.s0, &s_v_full);
+    ptx::tma_load_3d(sm + WS_V + 8192, &tm_v, 64, p.h, (int)p.s0, &s_v_full);
+  };
+  // issued-copy counters of the two issuing threads (for the drain after a timeout)
+  uint32_t raw_issued = 0, v_issued = 0;
+
+  if (warp < 8) {
+    // ======================= builder =======================
+    // thread t owns channels 8 (t mod 16) .. + 7 of rows 4 (t / 16) .. + 3
+    const int co = tid & 15, rg = tid >> 4;
+    const int c0 = 8 * co;
+    const uint32_t kp = co >> 3, ck = co & 7;  // K-panel and 16-byte chunk of the channels
+    float* s_tot = reinterpret_cast<float*>(sm + WS_TOT);
+    if (tid == 0) {
+      ptx::prefetch_tmap(&tm_k);
+      ptx::prefetch_tmap(&tm_q);
+      ptx::prefetch_tmap(&tm_g);
+      if (blockIdx.x < num_items) {
+        issue_raw(blockIdx.x);
+        ++raw_issued;
+      }
+    }
+    uint32_t nsteep = 0;
+    uint32_t n = 0;
+    for (uint32_t item = blockIdx.x; item < num_items; item += grid, ++n) {
+      const int slot = n & 1;
+      const ItemPos p = item_pos(item, T, H, fdH, fdC);
+      float bt = 0.f;
+      if (tid < p.Cn) bt = beta[(size_t)(p.s0 + tid) * H + p.h];
+
+      // ---- raw rows to registers; rows >= Cn contribute k = q = 0, g = 0
+      wait_or_abort(&s_raw_full, n & 1, abort_flag);
+      uint32_t kst[16], qst[16];
+      float G[4][8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = 4 * rg + u;
+        uint4 kw = make_uint4(0, 0, 0, 0), qw = kw;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+        if (r < p.Cn) {
+          kw = *reinterpret_cast<const uint4*>(sm + WS_RAWK + r * 256 + 16 * co);
+          qw = *reinterpret_cast<const uint4*>(sm + WS_RAWQ + r * 256 + 16 * co);
+          // the two 16-byte halves in alternating order across the quarter-warp (no bank conflicts)
+          const float* gr = reinterpret_cast<const float*>(sm + WS_RAWG + r * 512) + c0;
+          const int sw = (co >> 2) & 1;
+          const float4 h0 = *reinterpret_cast<const float4*>(gr + 4 * sw);
+          const float4 h1 = *reinterpret_cast<const float4*>(gr + 4 - 4 * sw);
+          a = sw ? h1 : h0;
+          b = sw ? h0 : h1;
+        }
+        kst[4 * u] = kw.x; kst[4 * u + 1] = kw.y; kst[4 * u + 2] = kw.z; kst[4 * u + 3] = kw.w;
+        qst[4 * u] = qw.x; qst[4 * u + 1] = qw.y; qst[4 * u + 2] = qw.z; qst[4 * u + 3] = qw.w;
+        const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) G[u][e] = (u ? G[u - 1][e] : 0.f) + x[e];
+      }
+      reinterpret_cast<float4*>(s_tot + rg * D + c0)[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+      reinterpret_cast<float4*>(s_tot + rg * D + c0)[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
+      ptx::bar_sync(1, 256);  // raw rows consumed, row-group totals visible
+      if (tid == 0 && item + grid < num_items && !*abort_flag) {
+        issue_raw(item + grid);
+        ++raw_issued;
+      }
+      {
+        float off[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q2 = 0; q2 < 15; ++q2) {
+          if (q2 < rg) {
+            const float4 t0 = reinterpret_cast<const float4*>(s_tot + q2 * D + c0)[0];
+            const float4 t1 = reinterpret_cast<const float4*>(s_tot + q2 * D + c0)[1];
+            off[0] += t0.x; off[1] += t0.y; off[2] += t0.z; off[3] += t0.w;
+            off[4] += t1.x; off[5] += t1.y; off[6] += t1.z; off[7] += t1.w;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) G[u][e] += off[e];
+      }
+      // G is non-increasing (g <= 0), so G at the chunk's last row is each channel's minimum
+      bool steep = false;
+      if (rg == 15) {
+        reinterpret_cast<float4*>(s_glast + c0)[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+        reinterpret_cast<float4*>(s_glast + c0)[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) steep |= !(G[3][e] >= tc::kChunkRefMinG);
+      }
+      const bool fast = !ptx::bar_or(1, 256, steep);  // uniform over the group; s_glast visible
+
+      // ---- slot reuse: item n-2's W^T / U^T MMA has read L3[slot] (and the solver
+      //      is done with TMEM slot, s_beta[slot], s_skip[slot]); item n-1's
+      //      [A'; P'] MMA has read RB
+      if (n >= 2) wait_or_abort(&s_b_done[slot], ((n - 2) >> 1) & 1, abort_flag);
+      if (n >= 1) wait_or_abort(&s_a_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+
+      if (fast) {
+        // Single reference (chunk start): a = e^{G} <= 1, rho = e^{-G} >= 1.
+        uint8_t* img = ws + (size_t)item * IMG_BYTES;
+        float gl[8], gam[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          gl[e] = s_glast[c0 + e];
+          gam[e] = ptx::ex2(gl[e] * kLog2e);
+        }
+        uint8_t* l3 = sm + WS_L3 + slot * WS_L3_SLOT + kp * 16384;
+        uint8_t* rb = sm + WS_RB + kp * 8192;
+        uint32_t qgp[2][8];  // Q e^G of this thread's 4 tokens, bf16 pairs per channel
+        float qg_prev[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = 4 * rg + u;
+          float kv[8], qv[8];
+          tc::unpack8(make_uint4(kst[4 * u], kst[4 * u + 1], kst[4 * u + 2], kst[4 * u + 3]), kv);
+          tc::unpack8(make_uint4(qst[4 * u], qst[4 * u + 1], qst[4 * u + 2], qst[4 * u + 3]), qv);
+          float o_ka[8], o_qa[8], o_kr[8], o_kb[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float t = G[u][e] * kLog2e;  // G log2(e), in [-115.5, 0]
+            const float a = ptx::ex2(t);        // e^G in (0, 1]
+            const float rho = ptx::ex2(-t);     // e^-G in [1, e^80]
+            o_ka[e] = kv[e] * a;
+            o_qa[e] = qv[e] * a;
+            o_kr[e] = kv[e] * rho;
+            o_kb[e] = o_kr[e] * gam[e];  // K o e^{G_last - G}
+            if (u & 1) qgp[u >> 1][e] = ptx::pack_bf16x2(qg_prev[e], o_qa[e]);
+            else qg_prev[e] = o_qa[e];
+          }
+          *reinterpret_cast<uint4*>(l3 + ptx::sw128_chunk(r, ck)) = tc::pack8(o_ka);
+          *reinterpret_cast<uint4*>(l3 + ptx::sw128_chunk(64 + r, ck)) = tc::pack8(o_qa);
+          *reinterpret_cast<uint4*>(rb + ptx::sw128_chunk(r, ck)) = tc::pack8(o_kr);
+          *reinterpret_cast<uint4*>(img + IMG_KB + kp * 8192 + ptx::sw128_chunk(r, ck)) = tc::pack8(o_kb);
+        }
+        // Q o e^G into the lower panel of the [W; Q e^G] image (MN-major, row = channel,
+        // 64 tokens per 128-byte row): this thread's 4 tokens are 8 contiguous bytes
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = c0 + e;
+          *reinterpret_cast<uint2*>(img + IMG_A1 + 16384 + c * 128 + ((((4 * rg) >> 3) ^ c) & 7) * 16 +
+                                    8 * (rg & 1)) = make_uint2(qgp[0][e], qgp[1][e]);
+        }
+        if (rg == 0) {
+          float gm[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) gm[e] = expf(gl[e]);
+          reinterpret_cast<float4*>(img + IMG_G)[2 * co] = make_float4(gm[0], gm[1], gm[2], gm[3]);
+          reinterpret_cast<float4*>(img + IMG_G)[2 * co + 1] = make_float4(gm[4], gm[5], gm[6], gm[7]);
+        }
+      }
+      if (tid < C) s_beta[slot][tid] = bt;
+      ptx::fence_proxy_async_smem();
+      ptx::bar_sync(1, 256);  // operands, s_beta[slot] complete
+
+      if (tid == 0) {
+        const bool issue = fast && !*abort_flag;
+        if (issue) {
+          // ---- [A'; P'] = [K e^G; Q e^G] (K e^-G)^T : M=128, N=64, K=128
+          ptx::tc_fence_after();
+          constexpr uint32_t id = ptx::idesc_bf16(128, 64, false, false);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = ptx::sdesc_sw128(sb + WS_L3 + slot * WS_L3_SLOT + (kk >> 2) * 16384 + (kk & 3) * 32,
+                                                 16, 1024);
+            const uint64_t bd = ptx::sdesc_sw128(sb + WS_RB + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+            ptx::mma_bf16(tmem + 64 * slot, ad, bd, id, kk > 0);
+          }
+          ptx::mma_commit(&s_a_done[slot]);
+        }
+        if (!fast && nsteep < list_cap) steep_list[(size_t)blockIdx.x * list_cap + nsteep++] = item;
+        s_skip[slot] = fast ? 0 : 1;
+        ptx::mbar_arrive(&s_a_done[slot]);             // releases s_beta[slot], s_skip[slot]
+        if (!issue) ptx::mbar_arrive(&s_a_done[slot]);  // stands in for the MMA completion
+      }
+    }
+    if (tid == 0) steep_cnt[blockIdx.x] = nsteep;
+  } else {
+    // ======================= solver =======================
+    const int st = tid - 256, w8 = warp - 8;
+    if (st == 0) {
+      ptx::prefetch_tmap(&tm_v);
+      if (blockIdx.x < num_items) {
+        issue_v(blockIdx.x);
+        ++v_issued;
+      }
+    }
+    float* As = reinterpret_cast<float*>(sm + WS_AS);
+    uint32_t n = 0;
+    for (uint32_t item = blockIdx.x; item < num_items; item += grid, ++n) {
+      const int slot = n & 1;
+      const bool has_next = item + grid < num_items;
+      wait_or_abort(&s_a_done[slot], (n >> 1) & 1, abort_flag);
+      ptx::tc_fence_after();
+      if (st == 0) ptx::bulk_wait_read0();  // the previous image store has read the staging area
+      const bool skip = ptx::bar_or(2, 256, s_skip[slot] != 0);
+      if (!skip) {
+        // ---- scatter A (fp32, beta-scaled) and P (bf16)
+        tc::scatter_single_ref(tmem + 64 * slot, s_beta[slot], As, sm + WS_ST, warp, w8, lane);
+        ptx::tc_fence_before();
+        ptx::bar_sync(2, 256);
+        // ---- T = (I + A)^{-1}, T diag(beta) in bf16
+        tc::solve_t_beta(As, reinterpret_cast<float*>(sm + WS_TS), reinterpret_cast<float*>(sm + WS_MT),
+                         s_beta[slot], sm + WS_TT, st, w8, lane, [] { ptx::bar_sync(2, 256); });
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::bar_sync(2, 256);
+        // ---- W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
+        if (st == 0) {
+          const bool have_v = wait_or_abort(&s_v_full, n & 1, abort_flag);
+          if (have_v && !*abort_flag) {
+            ptx::tc_fence_after();
+            constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bd = ptx::sdesc_sw128(sb + WS_TT + kk * 32, 16, 1024);
+              const uint64_t xd = ptx::sdesc_sw128(sb + WS_L3 + slot * WS_L3_SLOT + kk * 2048, 16384, 1024);
+              const uint64_t vd = ptx::sdesc_sw128(sb + WS_V + kk * 2048, 8192, 1024);
+              ptx::mma_bf16(tmem + 128, xd, bd, id, kk > 0);
+              ptx::mma_bf16(tmem + 192, vd, bd, id, kk > 0);
+            }
+            ptx::mma_commit(&s_b_done[slot]);
+          } else {
+            ptx::mbar_arrive(&s_b_done[slot]);
+          }
+        }
+        wait_or_abort(&s_b_done[slot], (n >> 1) & 1, abort_flag);
+        ptx::tc_fence_after();
+        if (st == 0 && has_next && !*abort_flag) {  // V is free again: the next item's V
+          issue_v(item + grid);
+          ++v_issued;
+        }
+        tc::stage_w_u(tmem + 128, sm + WS_ST, warp, w8, lane);
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::bar_sync(2, 256);
+        if (st == 0) {
+          ptx::bulk_s2g(ws + (size_t)item * IMG_BYTES + IMG_P, sm + WS_ST, WS_STAGE_BYTES);
+          ptx::bulk_commit();
+        }
+      } else if (st == 0) {  // skipped item: keep the V and b_done phases in step
+        wait_or_abort(&s_v_full, n & 1, abort_flag);
+        ptx::mbar_arrive(&s_b_done[slot]);
+        if (has_next && !*abort_flag) {
+          issue_v(item + grid);
+          ++v_issued;
+        }
+      }
+    }
+    if (st == 0) ptx::bulk_wait0();
+  }
+
+  // After a timeout: wait (bounded again) for the copies and MMAs still in
+  // flight, so that nothing lands in shared or tensor memory after exit.
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (s_abort && (tid == 0 || tid == 256)) {
+    const uint32_t issued = tid == 0 ? raw_issued : v_issued;
+    uint64_t* bar = tid == 0 ? &s_raw_full : &s_v_full;
+    if (issued) ptx::mbar_wait_bounded(bar, (issued - 1) & 1, 1000000000ull);
+    ptx::mma_commit(&s_drain);
+    ptx::mbar_wait_bounded(&s_drain, 0, 1000000000ull);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime
+// (no link against the driver library).
+inline cudaError_t tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+  static std::mutex mu;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *out = fn;
+  return cudaSuccess;
+}
+
+// Tensor map over a [tokens, H, 128] tensor (channels contiguous) with a box of
+// `box0` channels x 1 head x 64 tokens; rows past the last token read as zero.
+inline cudaError_t encode_rows_map(PFN_cuTensorMapEncodeTiled_v12000 fn, CUtensorMap* m, const void* base,
+                                   bool f32, long long tokens, int H, uint32_t box0, bool swizzle128) {
+  const cuuint64_t elt = f32 ? 4 : 2;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * elt, (cuuint64_t)H * D * elt};
+  const cuuint32_t box[3] = {box0, 1, (cuuint32_t)C};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Whether the warp-specialised kernel fits this device (its shared memory is
+// close to the per-block limit); sets the kernel's attribute on first use.
+inline bool ws_kernel_available() {
+  static PerDeviceOnce once;
+  static bool ok[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  run_once_per_device(once, [dev] {
+    const void* fn = (const void*)kda_ws_chunk_local_kernel<kGateLogCh>;
+    int optin = 0;
+    cudaFuncAttributes fa{};
+    ok[dev] = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess &&
+              cudaFuncGetAttributes(&fa, fn) == cudaSuccess &&
+              (size_t)WS_DYN + fa.sharedSizeBytes <= (size_t)optin &&
+              cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WS_DYN) == cudaSuccess;
+    cudaGetLastError();  // an unavailable kernel is not an error of the call
+    return cudaSuccess;
+  });
+  return ok[dev];
+}
+
+// Per-CTA item lists (steep chunks) in the workspace: `grid` lists of `cap`
+// entries, then `grid` counts.
+inline uint32_t ws_list_cap(long long items, int grid) { return (uint32_t)((items + grid - 1) / grid); }
+
+// Launches the warp-specialised kernel over all items (grid = one CTA per SM)
+// and then the two-CTA kernel over the chunks it passed on.
+inline cudaError_t launch_ws_local(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                   const float* g, const float* beta, int B, int T, int H, long long items,
+                                   FastDiv fdH, FastDiv fdC, uint8_t* ws, uint32_t* lists, int sms,
+                                   cudaStream_t stream) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  cudaError_t e = tensor_map_encoder(&enc);
+  if (e != cudaSuccess) return e;
+  const long long tokens = (long long)B * T;
+  CUtensorMap mk, mq, mg, mv;
+  if ((e = encode_rows_map(enc, &mk, k, false, tokens, H, D, false)) != cudaSuccess) return e;
+  if ((e = encode_rows_map(enc, &mq, q, false, tokens, H, D, false)) != cudaSuccess) return e;
+  if ((e = encode_rows_map(enc, &mg, g, true, tokens, H, D, false)) != cudaSuccess) return e;
+  if ((e = encode_rows_map(enc, &mv, v, false, tokens, H, 64, true)) != cudaSuccess) return e;
+  const int grid = (int)std::min<long long>(items, sms);
+  const uint32_t cap = ws_list_cap(items, grid);
+  uint32_t* cnt = lists + (size_t)grid * cap;
+  kda_ws_chunk_local_kernel<kGateLogCh><<<grid, 512, WS_DYN, stream>>>(mk, mq, mg, mv, beta, T, H, (uint32_t)items,
+                                                                      fdH, fdC, ws, lists, cnt, cap);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  tc::kda_tc_chunk_local_kernel<kGateLogCh><<<grid, 256, tc::KA_DYN, stream>>>(
+      q, k, v, g, beta, nullptr, 0, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap);
+  return cudaGetLastError();
+}
+
+}  // namespace ws
+}  // namespace kda

@@ -1,0 +1,79 @@
+"""GPU parity of the two chunk-local kernels of the tensor-core prefill: the
+warp-specialised one (default for per-channel log-decay gates on the
+one-row-per-sequence layout) and the two-CTA-per-SM one (kda_set_local_kernel(1)).
+Both against the fp64 oracle, and against each other on the same inputs,
+including launches where chunks past the single-reference decay range
+(log-decay below -80 over the chunk on some channel) are mixed in at random,
+so that the warp-specialised kernel hands a scattered subset of its items to
+the two-CTA kernel's item lists.
+"""
+import pytest
+import torch
+
+import kimi_delta_attention_31_b200 as kda
+import kda_workloads as W
+from parity_util import compare_units, rel_rms
+
+pytestmark = pytest.mark.gpu
+
+
+def _both(inp):
+    outs = []
+    for variant in (0, 1):
+        kda.set_local_kernel(variant)
+        try:
+            o, S = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp.get("S0"), None, 64)
+        finally:
+            kda.set_local_kernel(0)
+        torch.cuda.synchronize()
+        assert kda.device_error() == 0
+        outs.append((o, S))
+    return outs
+
+
+def _steep_mix(inp, seed, frac):
+    """Per (batch row, chunk, head): with probability `frac` a log-decay of
+    about -1.5 per token (-96 over a full chunk), else about -0.05."""
+    B, T, H, dk = inp["g"].shape
+    dev = inp["g"].device
+    gen = torch.Generator(device=dev).manual_seed(seed)
+    nc = (T + 63) // 64
+    steep = torch.rand((B, nc, H), generator=gen, device=dev) < frac
+    rate = torch.where(steep, torch.full_like(steep, 1.5, dtype=torch.float32),
+                       torch.full_like(steep, 0.05, dtype=torch.float32))
+    rate = rate.repeat_interleave(64, dim=1)[:, :T]  # [B, T, H]
+    u = torch.rand(inp["g"].shape, generator=gen, device=dev)
+    inp["g"] = (-rate.unsqueeze(-1) * (1.0 - 0.005 * u)).contiguous()
+    return int(steep.sum())
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 1, 1), (1, 64, 2), (2, 200, 4), (3, 130, 3), (2, 1000, 5)])
+def test_local_kernels_agree(cuda_device, B, T, H):
+    inp = W.make_prefill(B, T, H, 128, 128, "bf16", -4.0, 1.0, 0.05, seed=300 + T + H, device=cuda_device)
+    (o0, S0), (o1, S1) = _both(inp)
+    units = [(n, h) for n in range(B) for h in range(H)]
+    compare_units(inp, o0, S0, units, 1e-2)
+    compare_units(inp, o1, S1, units, 1e-2)
+    assert rel_rms(o0.float().cpu(), o1.float().cpu()) < 1e-3
+    assert rel_rms(S0.cpu(), S1.cpu()) < 1e-3
+
+
+@pytest.mark.parametrize("frac", [0.1, 0.5, 0.9])
+def test_local_kernels_scattered_steep_chunks(cuda_device, frac):
+    """B4 T2048 H8: 1024 items, about 7 per CTA of the warp-specialised kernel,
+    a random subset of them steep."""
+    inp = W.make_prefill(4, 2048, 8, 128, 128, "bf16", -4.0, 1.0, 0.05, seed=41, device=cuda_device)
+    n_steep = _steep_mix(inp, seed=42 + int(frac * 10), frac=frac)
+    assert 0 < n_steep < 4 * 32 * 8
+    (o0, S0), (o1, S1) = _both(inp)
+    assert torch.isfinite(o0).all() and torch.isfinite(S0).all()
+    units = [(0, 0), (1, 3), (2, 5), (3, 7), (3, 1)]
+    compare_units(inp, o0, S0, units, 1e-2)
+    assert rel_rms(o0.float().cpu(), o1.float().cpu()) < 1e-3
+    assert rel_rms(S0.cpu(), S1.cpu()) < 1e-3
+
+
+def test_local_kernel_switch_validation():
+    with pytest.raises(kda.KDAError):
+        kda.set_local_kernel(7)
+    kda.set_local_kernel(0)
