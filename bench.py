@@ -54,8 +54,9 @@ GDN_DECODE_BYTES_PER_HEAD_STEP = 2 * STATE_BYTES + 3 * 256 + 4 + 4 + 256
 
 def profiled_traffic(kernel, unit_key):
     """DRAM bytes per unit (token-head or head-step) for `kernel` from its ncu
-    summary under profiles/, or None when there is none or when the kernel's
-    source file changed since the counters were taken (sha1 recorded there)."""
+    summary under profiles/, or None when there is none or when one of the
+    kernel's source files changed since the counters were taken (the summary
+    lists them, space-separated, with their sha1s)."""
     import glob
     import hashlib
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"{kernel}_*.md"))):
@@ -67,11 +68,14 @@ def profiled_traffic(kernel, unit_key):
         src, sha, per = fields.get("source_file"), fields.get("source_sha1"), fields.get(unit_key)
         if not (src and sha and per):
             continue
+        srcs, shas = src.split(), sha.split()
+        if len(srcs) != len(shas):
+            continue
         try:
-            cur = hashlib.sha1(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+            cur = [hashlib.sha1(open(os.path.join(ROOT, f), "rb").read()).hexdigest() for f in srcs]
         except OSError:
             continue
-        if cur == sha:
+        if cur == shas:
             return float(per), os.path.basename(path)
     return None, None
 
@@ -259,7 +263,7 @@ def gdn_leg(kda, args, world, dev, stream, peaks):
     barrier(world)
     ms = max_over_ranks(time_launches(prefill, args.steps, stream), world, dev)
     kernel_ms = kda.profile_chunk_fwd(prefill, stream, repeats=max(1, min(args.steps, 5)), dk=dk, dv=dv,
-                                      chunk_size=w.chunk)
+                                      chunk_size=w.chunk, gate="log_token")
     token_heads = B * T * H
     dom_name, dom_ms = max(kernel_ms.items(), key=lambda kv: kv[1])
     dom_bytes = kda.algorithmic_bytes_per_launch(dom_name, token_heads, B * H, d=dk, gate_per_channel=False)
@@ -335,7 +339,7 @@ def prep_leg(kda, args, world, dev, stream, peaks):
     ms = max_over_ranks(time_launches(fused, args.steps, stream), world, dev)
     ms_unfused = max_over_ranks(time_launches(unfused, max(1, min(args.steps, 3)), stream), world, dev)
     kernel_ms = kda.profile_chunk_fwd(fused, stream, repeats=max(1, min(args.steps, 5)), dk=dk, dv=dv,
-                                      chunk_size=w.chunk)
+                                      chunk_size=w.chunk, gate="logit")
     token_heads = B * T * H
     dom_name, dom_ms = max(kernel_ms.items(), key=lambda kv: kv[1])
     dom_bytes = kda.algorithmic_bytes_per_launch(dom_name, token_heads, B * H, d=dk, gate_bytes=2)
@@ -435,7 +439,9 @@ def run_ours(args):
     S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     ws_bytes = kda.workspace_size(B, T, H, dk, dv, 0, w.chunk, torch.bfloat16)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    launches_per_prefill = kda.launches_per_chunk_fwd(dk, dv, w.chunk, torch.bfloat16)
+    # every kernel one headline call launches (the warp-specialised chunk-local
+    # kernel, the two-CTA kernel over its passed-on chunks, the state pass)
+    kernels_per_prefill = kda.chunk_fwd_kernel_sequence(B, T, H, dk, dv, w.chunk, torch.bfloat16)
 
     def prefill():
         kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], None, w.chunk,
@@ -547,7 +553,7 @@ def run_ours(args):
     if world == 1 and not args.no_cpu_baseline:
         cpu, _ = oracle_baseline(w)
 
-    gpu_launches = args.steps * launches_per_prefill
+    gpu_launches = args.steps * len(kernels_per_prefill)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",

@@ -288,8 +288,11 @@ kda_status_t kda_set_local_kernel(int variant);
 /*
  * Number of phases one kda_chunk_fwd call with these arguments runs: 1 for
  * the fp32-arithmetic path (one kernel); 2 for the tensor-core path (the
- * chunk-local kernel, then the state pass -- one kernel, or three when the
- * sequences are split into segments).
+ * chunk-local phase -- one kernel, or two when the warp-specialised kernel
+ * runs and hands its steep chunks to the two-CTA kernel, see
+ * kda_set_local_kernel -- then the state pass -- one kernel, or three when the
+ * sequences are split into segments).  kda_profile_events records one event
+ * before the call and one after each phase.
  */
 int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype);
 

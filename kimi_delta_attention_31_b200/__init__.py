@@ -45,6 +45,8 @@ NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
 KERNELS_SIMT = ("kda_chunk_simt_kernel",)
 KERNELS_TC = ("kda_tc_chunk_local_kernel", "kda_tc_state_pass_kernel")
+KERNEL_WS = "kda_ws_chunk_local_kernel"
+_tls = threading.local()  # mirrors kda_set_local_kernel, which is per host thread
 
 
 class KDAError(RuntimeError):
@@ -398,6 +400,16 @@ def set_local_kernel(variant: int) -> None:
     calls: 0 = the warp-specialised kernel where it applies (default),
     1 = the two-CTA-per-SM kernel always."""
     _check(load_library().kda_set_local_kernel(int(variant)))
+    _tls.local_kernel = int(variant)
+
+
+def uses_ws_kernel(gate="log_channel", packed=False, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16) -> bool:
+    """Whether a chunk_fwd call of this kind on this thread runs the
+    warp-specialised chunk-local kernel: tensor-core path, per-channel
+    log-decay gate (gate="log_channel"; "log_token" = Gated DeltaNet,
+    "logit" = raw gate logits), one sequence per batch row."""
+    return (launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 2 and gate == "log_channel" and not packed
+            and getattr(_tls, "local_kernel", 0) == 0)
 
 
 def segment_chunks(B, T, H, num_seqs=0) -> int:
@@ -418,16 +430,35 @@ def launches_per_chunk_fwd(dk, dv, chunk_size, dtype=torch.bfloat16) -> int:
     return int(load_library().kda_chunk_fwd_launches(dk, dv, chunk_size, code))
 
 
-def kernel_names(dk, dv, chunk_size, dtype=torch.bfloat16):
+def kernel_names(dk, dv, chunk_size, dtype=torch.bfloat16, gate="log_channel", packed=False):
+    """Phases of one chunk_fwd call, named by the kernel that does each one's
+    work (the chunk-local phase of the warp-specialised path also launches the
+    two-CTA kernel over the chunks it passed on, usually none)."""
     n = launches_per_chunk_fwd(dk, dv, chunk_size, dtype)
-    return KERNELS_SIMT if n == 1 else KERNELS_TC[:n]
+    if n == 1:
+        return KERNELS_SIMT
+    first = KERNEL_WS if uses_ws_kernel(gate, packed, dk, dv, chunk_size, dtype) else KERNELS_TC[0]
+    return (first,) + KERNELS_TC[1:n]
 
 
-def profile_chunk_fwd(call, stream, repeats=3, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16):
+def chunk_fwd_kernel_sequence(B, T, H, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16, gate="log_channel",
+                              num_seqs=0):
+    """Every kernel one chunk_fwd call launches, in order."""
+    if launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 1:
+        return list(KERNELS_SIMT)
+    seq = ([KERNEL_WS, KERNELS_TC[0]] if uses_ws_kernel(gate, num_seqs > 0, dk, dv, chunk_size, dtype)
+           else [KERNELS_TC[0]])
+    if segment_chunks(B, T, H, num_seqs) > 0:
+        return seq + [KERNELS_TC[1], "kda_tc_seg_combine_kernel", KERNELS_TC[1]]
+    return seq + [KERNELS_TC[1]]
+
+
+def profile_chunk_fwd(call, stream, repeats=3, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16,
+                      gate="log_channel", packed=False):
     """Run ``call()`` (one chunk_fwd call) ``repeats`` times with the library's
-    event hook set and return {kernel name: mean ms per launch}."""
+    event hook set and return {phase's kernel name: mean ms per call}."""
     lib = load_library()
-    names = kernel_names(dk, dv, chunk_size, dtype)
+    names = kernel_names(dk, dv, chunk_size, dtype, gate, packed)
     n = len(names)
     events = [torch.cuda.Event(enable_timing=True) for _ in range((n + 1) * repeats)]
     for e in events:  # torch creates the underlying event lazily, at its first record
@@ -464,7 +495,7 @@ def algorithmic_bytes_per_launch(kernel, token_heads, units, d=128, with_state_i
     gate = gate_bytes * d if gate_per_channel else gate_bytes
     if kernel == "kda_chunk_simt_kernel":
         return token_heads * (3 * 2 * d + gate + 4 + 2 * d) + state * (2 if with_state_in else 1)
-    if kernel == "kda_tc_chunk_local_kernel":
+    if kernel in ("kda_tc_chunk_local_kernel", KERNEL_WS):
         return token_heads * (3 * 2 * d + gate + 4 + TC_IMAGE_BYTES_PER_TOKEN_HEAD)
     if kernel == "kda_tc_state_pass_kernel":
         return token_heads * (TC_IMAGE_BYTES_PER_TOKEN_HEAD + 2 * d) + state * (2 if with_state_in else 1)
@@ -477,4 +508,5 @@ def version() -> int:
 
 __all__ = ["chunk_fwd", "chunk_fwd_noalloc", "recurrent_step", "chunk_fwd_host", "HostPrefill", "workspace_size",
            "launches_per_chunk_fwd", "kernel_names", "profile_chunk_fwd", "algorithmic_bytes_per_launch",
+           "set_local_kernel", "uses_ws_kernel", "chunk_fwd_kernel_sequence",
            "last_error", "device_error", "version", "load_library", "lib_path", "KDAError", "EXPORTED"]

@@ -219,13 +219,13 @@ __device__ __forceinline__ void normalise_rows(float* kv, float* qv, float nk, f
 }
 
 // Phase 4 on the single-reference path: TMEM columns [tm, tm + 64) hold, in
-// lanes 0..63, A'_rj and in lanes 64..127, P'_rj.  Writes A = beta_r A'_rj
-// (j < r, fp32, row stride AS_LD) and P (j <= r, bf16 K-major 128-byte
-// swizzled, zero above the diagonal).  Eight warps; `warp` is the warp's
-// index in the CTA (its TMEM lane quarter is warp mod 4) and `w8` its index
-// in the group of eight (which 32 columns it takes).
+// lanes 0..63, A'_rj and in lanes 64..127, P'_rj (the other way round when
+// `p_first`).  Writes A = beta_r A'_rj (j < r, fp32, row stride AS_LD) and P
+// (j <= r, bf16 K-major 128-byte swizzled, zero above the diagonal).  Eight
+// warps; `warp` is the warp's index in the CTA (its TMEM lane quarter is
+// warp mod 4) and `w8` its index in the group of eight (which 32 columns it takes).
 __device__ __forceinline__ void scatter_single_ref(uint32_t tm, const float* s_beta, float* As, uint8_t* Pt,
-                                                   int warp, int w8, int lane) {
+                                                   int warp, int w8, int lane, bool p_first = false) {
   const int qd = warp & 3, ch = w8 >> 2;
   const int rho = 32 * qd + lane, r = rho & 63, j0 = 32 * ch;
   float x[32];
@@ -233,7 +233,7 @@ __device__ __forceinline__ void scatter_single_ref(uint32_t tm, const float* s_b
   ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
   ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
   ptx::tmem_wait_ld();
-  if (rho < 64) {  // warp-uniform
+  if ((rho < 64) != p_first) {  // warp-uniform
     const float br = s_beta[r];
 #pragma unroll
     for (int e = 0; e < 32; ++e) x[e] = (j0 + e < r) ? br * x[e] : 0.f;
@@ -249,53 +249,69 @@ __device__ __forceinline__ void scatter_single_ref(uint32_t tm, const float* s_b
 }
 
 // Phase 5: T = (I + A)^{-1} (A strictly lower, fp32 in As), blocked by 16.
-// Diagonal blocks by forward substitution in fp32, one column per 4 lanes;
-// then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ by distance below the diagonal,
-// one warp per block, TF32 warp MMAs with fp32 accumulation.  Finally
+// Diagonal blocks by forward substitution in fp32, one thread per column of T
+// holding the column's 16 rows in registers (rows of A are broadcast loads).
+// Then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ: block column J needs only the
+// blocks above it in the same column, so warp J walks down its column (warp
+// syncs only), with TF32 warp MMAs and fp32 accumulation.  Finally
 // T diag(beta) in bf16 (K-major [64 r][64 j], 128-byte swizzle) into Tt.
 // 256 threads: t in [0, 256), w = t / 32; `sync` is their barrier.
 template <typename Sync>
 __device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* Mt, const float* s_beta, uint8_t* Tt,
                                              int t, int w, int lane, Sync sync) {
-  {
-    const int j = t >> 2, part = t & 3;  // column j of T; this lane keeps rows 4 m + part
-    const int Ib = j >> 4, jj = j & 15, o = 16 * Ib;
-    float x[4];
+  if (t < 64) {
+    const int jj = t & 15, o = t & 48;  // column jj of diagonal block o / 16
+    float x[16];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) x[m] = (4 * m + part == jj) ? 1.f : 0.f;
+    for (int m = 0; m < 16; ++m) x[m] = (m == jj) ? 1.f : 0.f;
 #pragma unroll
     for (int i = 1; i < 16; ++i) {
-      float acc = 0.f;
+      const float* arow = As + (o + i) * AS_LD + o;
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-        if (4 * m < i) acc = fmaf(As[(o + i) * AS_LD + o + 4 * m + part], x[m], acc);  // A[i][>=i] == 0
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      if ((i & 3) == part && i > jj) x[i >> 2] = -acc;
+      for (int q4 = 0; q4 < 4; ++q4) {
+        if (4 * q4 < i) {
+          const float4 a4 = *reinterpret_cast<const float4*>(arow + 4 * q4);
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int m = 4 * q4 + e;
+            if (m < i) {
+              if (m & 1) acc1 = fmaf(av[e], x[m], acc1);
+              else acc0 = fmaf(av[e], x[m], acc0);
+            }
+          }
+        }
+      }
+      if (i > jj) x[i] = -(acc0 + acc1);  // rows above jj keep T's zeros, row jj its 1
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) Ts[(o + 4 * m + part) * AS_LD + o + jj] = x[m];
+    for (int i = 0; i < 16; ++i) Ts[(o + i) * AS_LD + o + jj] = x[i];
   }
   sync();
+  if (w < 3) {
+    const int Jc = w;
+    float* mt = Mt + w * 16 * MT_LD;
 #pragma unroll
-  for (int dist = 1; dist <= 3; ++dist) {
-    if (w < 4 - dist) {
-      const int Jc = w, Ir = w + dist;
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int step = 1; step <= 3; ++step) {
+      const int Ir = Jc + step;
+      if (Ir < 4) {  // warp-uniform
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int kk = 0; kk < dist; ++kk) {
-        const int K = Jc + kk;
-        warp_gemm16(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
+        for (int kk = 0; kk < step; ++kk) {
+          const int K = Jc + kk;
+          warp_gemm16(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
+        }
+        warp_store16(mt, MT_LD, acc, 1.f, lane);
+        __syncwarp();
+        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        warp_gemm16(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
+        warp_store16(Ts + 16 * Ir * AS_LD + 16 * Jc, AS_LD, acc2, -1.f, lane);
+        __syncwarp();  // block (Ir, Jc) visible to the warp's next step; mt free again
       }
-      float* mt = Mt + w * 16 * MT_LD;
-      warp_store16(mt, MT_LD, acc, 1.f, lane);
-      __syncwarp();
-      float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      warp_gemm16(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
-      warp_store16(Ts + 16 * Ir * AS_LD + 16 * Jc, AS_LD, acc2, -1.f, lane);
     }
-    sync();
   }
+  sync();
   // bf16 T diag(beta); blocks above the diagonal are zero
   for (int idx = t; idx < 512; idx += 256) {
     const int rr = idx >> 3, k8 = idx & 7;

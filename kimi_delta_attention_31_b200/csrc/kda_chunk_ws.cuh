@@ -10,13 +10,14 @@
 // the same time:
 //   builder (warps 0..7): raw k, q, g rows arrive by tensor-map TMA; the
 //     group forms the cumulative log-decays G, the decay-scaled operands
-//     [K e^G; Q e^G] (double-buffered) and K e^-G, writes Kbar, Q e^G and
+//     K e^G (double-buffered), Q e^G and K e^-G, writes Kbar, Q e^G and
 //     gamma to the image, and issues the [A'; P'] MMA into one of two TMEM
 //     accumulators.  Its thread 0 starts the next item's TMA as soon as the
-//     group has read the raw rows, so that load overlaps the build.
+//     group has read the raw rows, so that load overlaps the build, and
+//     prefetches the item after it into L2.
 //   solver (warps 8..15): scatters A and P out of TMEM, inverts I + A,
 //     issues the W^T / U^T MMAs (V comes straight from TMA in the MMA's
-//     layout), stages P, U^T and W^T and stores them with one bulk copy.
+//     layout), and stores P, then U^T and W^T, with bulk copies.
 // Items whose chunk decays below the single-reference range on some channel
 // (min G_last < -80) are not built here: the builder appends them to this
 // CTA's item list, and the two-CTA kernel runs that list afterwards with the
@@ -58,25 +59,32 @@ using tc::IMG_P;
 using tc::IMG_U;
 
 // shared memory (dynamic, 1024-aligned base)
-constexpr uint32_t WS_RAWK = 0;            // k rows [64 tok][128 ch] bf16, row-major        16384
-constexpr uint32_t WS_RAWQ = 16384;        // q rows                                          16384
-constexpr uint32_t WS_RAWG = 32768;        // g rows [64 tok][128 ch] fp32                    32768
-constexpr uint32_t WS_V = 65536;           // V MN-major 2 panels [64 tok][64 dv], 128-B swizzle 16384
-constexpr uint32_t WS_L3 = 81920;          // 2 slots x [K e^G; Q e^G] K-major, 2 K-panels of 128 rows 2 x 32768
-constexpr uint32_t WS_L3_SLOT = 32768;
-constexpr uint32_t WS_RB = 147456;         // K e^-G K-major 2 panels [64][64]                16384
-constexpr uint32_t WS_ST = 163840;         // staging P | U^T | W^T in image order            40960
-constexpr uint32_t WS_AS = WS_ST + 8192;   // A fp32 [64][68], over the U^T / W^T staging     17408
-constexpr uint32_t WS_TS = WS_AS + 17408;  // T fp32 [64][68]                                 17408
-constexpr uint32_t WS_MT = WS_TS + 17408;  // block products [3][16][20]                      3840
-constexpr uint32_t WS_TT = 210944;         // T diag(beta) bf16 K-major [64][64]              8192
-constexpr uint32_t WS_TOT = 219136;        // row-group totals of g [16][128] fp32            8192
-constexpr uint32_t WS_BYTES = WS_TOT + 8192;
+constexpr uint32_t WS_RAWK = 0;        // k rows [64 tok][128 ch] bf16, row-major             16384
+constexpr uint32_t WS_RAWQ = 16384;    // q rows                                               16384
+constexpr uint32_t WS_RAWG = 32768;    // g rows [64 tok][128 ch] fp32                         32768
+constexpr uint32_t WS_V = 65536;       // V MN-major 2 panels [64 tok][64 dv], 128-B swizzle   16384
+// Left operands, K-major, per 64-channel K-panel: K e^G of slot 0 | Q e^G | K e^G of
+// slot 1 (64 rows each).  Slot 0's [A'; P'] operand starts at its K rows, slot 1's
+// at the Q rows (so its TMEM result has P' in lanes 0..63); the W^T MMA reads K e^G
+// of the slot as an MN-major operand.
+constexpr uint32_t WS_L3 = 81920;      // 2 panels x 24576                                     49152
+constexpr uint32_t WS_L3_PANEL = 24576;
+constexpr uint32_t WS_RB = 131072;     // K e^-G K-major 2 panels [64][64]; before the build:
+                                       // warp totals of g [8][128] fp32                        16384
+constexpr uint32_t WS_UW = 147456;     // staging U^T | W^T (image order); during the solve the
+                                       // off-diagonal block products                          32768
+constexpr uint32_t WS_AS = 180224;     // A fp32 [64][68]                                      17408
+constexpr uint32_t WS_TS = WS_AS + 17408;  // T fp32 [64][68]                                  17408
+constexpr uint32_t WS_TT = 215040;     // T diag(beta) bf16 K-major [64][64]; before the solve
+                                       // the P staging                                        8192
+constexpr uint32_t WS_BYTES = WS_TT + 8192;
 constexpr uint32_t WS_DYN = WS_BYTES + 1024;
-constexpr uint32_t WS_STAGE_BYTES = IMG_A1 + 16384 - IMG_P;
-static_assert(WS_MT + 3 * 16 * tc::MT_LD * 4 <= WS_TT, "solver buffers overlap");
-static_assert(WS_ST + WS_STAGE_BYTES <= WS_TS + 17408, "staging layout");
-static_assert(WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_V % 1024 == 0, "alignment");
+static_assert(WS_TS + 17408 == WS_TT && WS_L3 + 2 * WS_L3_PANEL == WS_RB && WS_RB + 16384 == WS_UW &&
+                  WS_UW + 32768 == WS_AS, "layout");
+static_assert(3 * 16 * tc::MT_LD * 4 <= 32768 && 8 * D * 4 <= 16384, "scratch sizes");
+static_assert(WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_V % 1024 == 0 &&
+                  WS_UW % 1024 == 0, "alignment");
+static_assert(IMG_A1 - IMG_U == 16384 && IMG_U - IMG_P == 8192, "image order");
 
 constexpr uint32_t kRawBytes = 2 * C * D * 2 + C * D * 4;  // k, q (bf16) and g (fp32)
 constexpr uint32_t kVBytes = C * D * 2;
@@ -165,6 +173,14 @@ __global__ void __launch_bounds__(512, 1)
     ptx::tma_load_3d(sm + WS_RAWQ, &tm_q, 0, p.h, (int)p.s0, &s_raw_full);
     ptx::tma_load_3d(sm + WS_RAWG, &tm_g, 0, p.h, (int)p.s0, &s_raw_full);
   };
+  auto prefetch_l2 = [&](uint32_t item) {
+    const ItemPos p = item_pos(item, T, H, fdH, fdC);
+    ptx::tma_prefetch_l2_3d(&tm_k, 0, p.h, (int)p.s0);
+    ptx::tma_prefetch_l2_3d(&tm_q, 0, p.h, (int)p.s0);
+    ptx::tma_prefetch_l2_3d(&tm_g, 0, p.h, (int)p.s0);
+    ptx::tma_prefetch_l2_3d(&tm_v, 0, p.h, (int)p.s0);
+    ptx::tma_prefetch_l2_3d(&tm_v, 64, p.h, (int)p.s0);
+  };
   auto issue_v = [&](uint32_t item) {
     const ItemPos p = item_pos(item, T, H, fdH, fdC);
     ptx::mbar_arrive_expect_tx(&s_v_full, kVBytes);
@@ -180,15 +196,17 @@ __global__ void __launch_bounds__(512, 1)
     const int co = tid & 15, rg = tid >> 4;
     const int c0 = 8 * co;
     const uint32_t kp = co >> 3, ck = co & 7;  // K-panel and 16-byte chunk of the channels
-    float* s_tot = reinterpret_cast<float*>(sm + WS_TOT);
+    float* s_wtot = reinterpret_cast<float*>(sm + WS_RB);  // [8 warps][128 ch]
     if (tid == 0) {
       ptx::prefetch_tmap(&tm_k);
       ptx::prefetch_tmap(&tm_q);
       ptx::prefetch_tmap(&tm_g);
+      ptx::prefetch_tmap(&tm_v);
       if (blockIdx.x < num_items) {
         issue_raw(blockIdx.x);
         ++raw_issued;
       }
+      if (blockIdx.x + grid < num_items) prefetch_l2(blockIdx.x + grid);
     }
     uint32_t nsteep = 0;
     uint32_t n = 0;
@@ -224,23 +242,34 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) G[u][e] = (u ? G[u - 1][e] : 0.f) + x[e];
       }
-      reinterpret_cast<float4*>(s_tot + rg * D + c0)[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
-      reinterpret_cast<float4*>(s_tot + rg * D + c0)[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
-      ptx::bar_sync(1, 256);  // raw rows consumed, row-group totals visible
+      // Row-group totals: this warp holds row groups 2w (lanes 0..15) and 2w+1
+      // (lanes 16..31) of the same channels; the warp's total goes to s_wtot,
+      // which lives in RB: item n-1's [A'; P'] MMA has read RB (and Q e^G) first.
+      if (n >= 1) wait_or_abort(&s_a_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+      float lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lo[e] = __shfl_xor_sync(0xffffffffu, G[3][e], 16);
+      if (lane >= 16) {
+        reinterpret_cast<float4*>(s_wtot + warp * D + c0)[0] =
+            make_float4(G[3][0] + lo[0], G[3][1] + lo[1], G[3][2] + lo[2], G[3][3] + lo[3]);
+        reinterpret_cast<float4*>(s_wtot + warp * D + c0)[1] =
+            make_float4(G[3][4] + lo[4], G[3][5] + lo[5], G[3][6] + lo[6], G[3][7] + lo[7]);
+      }
+      ptx::bar_sync(1, 256);  // raw rows consumed, warp totals visible
       if (tid == 0 && item + grid < num_items && !*abort_flag) {
         issue_raw(item + grid);
         ++raw_issued;
+        if (item + 2 * grid < num_items) prefetch_l2(item + 2 * grid);
       }
       {
-        float off[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float off[8];
 #pragma unroll
-        for (int q2 = 0; q2 < 15; ++q2) {
-          if (q2 < rg) {
-            const float4 t0 = reinterpret_cast<const float4*>(s_tot + q2 * D + c0)[0];
-            const float4 t1 = reinterpret_cast<const float4*>(s_tot + q2 * D + c0)[1];
-            off[0] += t0.x; off[1] += t0.y; off[2] += t0.z; off[3] += t0.w;
-            off[4] += t1.x; off[5] += t1.y; off[6] += t1.z; off[7] += t1.w;
-          }
+        for (int e = 0; e < 8; ++e) off[e] = lane >= 16 ? lo[e] : 0.f;
+        for (int w2 = 0; w2 < warp; ++w2) {  // warp-uniform
+          const float4 t0 = reinterpret_cast<const float4*>(s_wtot + w2 * D + c0)[0];
+          const float4 t1 = reinterpret_cast<const float4*>(s_wtot + w2 * D + c0)[1];
+          off[0] += t0.x; off[1] += t0.y; off[2] += t0.z; off[3] += t0.w;
+          off[4] += t1.x; off[5] += t1.y; off[6] += t1.z; off[7] += t1.w;
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -257,11 +286,9 @@ __global__ void __launch_bounds__(512, 1)
       }
       const bool fast = !ptx::bar_or(1, 256, steep);  // uniform over the group; s_glast visible
 
-      // ---- slot reuse: item n-2's W^T / U^T MMA has read L3[slot] (and the solver
-      //      is done with TMEM slot, s_beta[slot], s_skip[slot]); item n-1's
-      //      [A'; P'] MMA has read RB
+      // ---- slot reuse: item n-2's W^T / U^T MMA has read K e^G of this slot (and
+      //      the solver is done with TMEM slot, s_beta[slot], s_skip[slot])
       if (n >= 2) wait_or_abort(&s_b_done[slot], ((n - 2) >> 1) & 1, abort_flag);
-      if (n >= 1) wait_or_abort(&s_a_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
 
       if (fast) {
         // Single reference (chunk start): a = e^{G} <= 1, rho = e^{-G} >= 1.
@@ -272,7 +299,8 @@ __global__ void __launch_bounds__(512, 1)
           gl[e] = s_glast[c0 + e];
           gam[e] = ptx::ex2(gl[e] * kLog2e);
         }
-        uint8_t* l3 = sm + WS_L3 + slot * WS_L3_SLOT + kp * 16384;
+        uint8_t* l3k = sm + WS_L3 + kp * WS_L3_PANEL + (slot ? 16384 : 0);
+        uint8_t* l3q = sm + WS_L3 + kp * WS_L3_PANEL + 8192;
         uint8_t* rb = sm + WS_RB + kp * 8192;
         uint32_t qgp[2][8];  // Q e^G of this thread's 4 tokens, bf16 pairs per channel
         float qg_prev[8];
@@ -295,8 +323,8 @@ __global__ void __launch_bounds__(512, 1)
             if (u & 1) qgp[u >> 1][e] = ptx::pack_bf16x2(qg_prev[e], o_qa[e]);
             else qg_prev[e] = o_qa[e];
           }
-          *reinterpret_cast<uint4*>(l3 + ptx::sw128_chunk(r, ck)) = tc::pack8(o_ka);
-          *reinterpret_cast<uint4*>(l3 + ptx::sw128_chunk(64 + r, ck)) = tc::pack8(o_qa);
+          *reinterpret_cast<uint4*>(l3k + ptx::sw128_chunk(r, ck)) = tc::pack8(o_ka);
+          *reinterpret_cast<uint4*>(l3q + ptx::sw128_chunk(r, ck)) = tc::pack8(o_qa);
           *reinterpret_cast<uint4*>(rb + ptx::sw128_chunk(r, ck)) = tc::pack8(o_kr);
           *reinterpret_cast<uint4*>(img + IMG_KB + kp * 8192 + ptx::sw128_chunk(r, ck)) = tc::pack8(o_kb);
         }
@@ -323,13 +351,13 @@ __global__ void __launch_bounds__(512, 1)
       if (tid == 0) {
         const bool issue = fast && !*abort_flag;
         if (issue) {
-          // ---- [A'; P'] = [K e^G; Q e^G] (K e^-G)^T : M=128, N=64, K=128
+          // ---- [A'; P'] = [K e^G; Q e^G] (K e^-G)^T : M=128, N=64, K=128 (slot 1: [P'; A'])
           ptx::tc_fence_after();
           constexpr uint32_t id = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = ptx::sdesc_sw128(sb + WS_L3 + slot * WS_L3_SLOT + (kk >> 2) * 16384 + (kk & 3) * 32,
-                                                 16, 1024);
+            const uint64_t ad =
+                ptx::sdesc_sw128(sb + WS_L3 + (kk >> 2) * WS_L3_PANEL + (slot ? 8192 : 0) + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = ptx::sdesc_sw128(sb + WS_RB + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
             ptx::mma_bf16(tmem + 64 * slot, ad, bd, id, kk > 0);
           }
@@ -359,16 +387,26 @@ __global__ void __launch_bounds__(512, 1)
       const bool has_next = item + grid < num_items;
       wait_or_abort(&s_a_done[slot], (n >> 1) & 1, abort_flag);
       ptx::tc_fence_after();
-      if (st == 0) ptx::bulk_wait_read0();  // the previous image store has read the staging area
       const bool skip = ptx::bar_or(2, 256, s_skip[slot] != 0);
       if (!skip) {
-        // ---- scatter A (fp32, beta-scaled) and P (bf16)
-        tc::scatter_single_ref(tmem + 64 * slot, s_beta[slot], As, sm + WS_ST, warp, w8, lane);
+        // ---- scatter A (fp32, beta-scaled) and P (bf16, staged in the T diag(beta) buffer)
+        tc::scatter_single_ref(tmem + 64 * slot, s_beta[slot], As, sm + WS_TT, warp, w8, lane, slot == 1);
+        ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::bar_sync(2, 256);
-        // ---- T = (I + A)^{-1}, T diag(beta) in bf16
-        tc::solve_t_beta(As, reinterpret_cast<float*>(sm + WS_TS), reinterpret_cast<float*>(sm + WS_MT),
-                         s_beta[slot], sm + WS_TT, st, w8, lane, [] { ptx::bar_sync(2, 256); });
+        if (st == 0) {
+          ptx::bulk_s2g(ws + (size_t)item * IMG_BYTES + IMG_P, sm + WS_TT, 8192);
+          ptx::bulk_commit();
+        }
+        // ---- T = (I + A)^{-1}, T diag(beta) in bf16.  At each barrier thread 0
+        //      first waits for its stores to have read shared memory: the block
+        //      products reuse the U^T / W^T staging (stored at the end of the
+        //      previous item), T diag(beta) the P staging.
+        tc::solve_t_beta(As, reinterpret_cast<float*>(sm + WS_TS), reinterpret_cast<float*>(sm + WS_UW),
+                         s_beta[slot], sm + WS_TT, st, w8, lane, [st] {
+                           if (st == 0) ptx::bulk_wait_read0();
+                           ptx::bar_sync(2, 256);
+                         });
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::bar_sync(2, 256);
@@ -381,7 +419,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t bd = ptx::sdesc_sw128(sb + WS_TT + kk * 32, 16, 1024);
-              const uint64_t xd = ptx::sdesc_sw128(sb + WS_L3 + slot * WS_L3_SLOT + kk * 2048, 16384, 1024);
+              const uint64_t xd = ptx::sdesc_sw128(sb + WS_L3 + (slot ? 16384 : 0) + kk * 2048, WS_L3_PANEL, 1024);
               const uint64_t vd = ptx::sdesc_sw128(sb + WS_V + kk * 2048, 8192, 1024);
               ptx::mma_bf16(tmem + 128, xd, bd, id, kk > 0);
               ptx::mma_bf16(tmem + 192, vd, bd, id, kk > 0);
@@ -397,12 +435,12 @@ __global__ void __launch_bounds__(512, 1)
           issue_v(item + grid);
           ++v_issued;
         }
-        tc::stage_w_u(tmem + 128, sm + WS_ST, warp, w8, lane);
+        tc::stage_w_u(tmem + 128, sm + WS_UW - IMG_U, warp, w8, lane);  // U^T at WS_UW, W^T after it
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::bar_sync(2, 256);
         if (st == 0) {
-          ptx::bulk_s2g(ws + (size_t)item * IMG_BYTES + IMG_P, sm + WS_ST, WS_STAGE_BYTES);
+          ptx::bulk_s2g(ws + (size_t)item * IMG_BYTES + IMG_U, sm + WS_UW, 32768);
           ptx::bulk_commit();
         }
       } else if (st == 0) {  // skipped item: keep the V and b_done phases in step

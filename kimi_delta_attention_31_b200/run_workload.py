@@ -2,6 +2,7 @@
 synthetic inputs), e.g. to profile one kernel with Nsight Compute:
 
     python -m kimi_delta_attention_31_b200.run_workload --op prefill --B 2 --T 8192 --H 32 --iters 3
+    python -m kimi_delta_attention_31_b200.run_workload --op prefill --B 2 --T 8192 --H 32 --local-kernel 1
     python -m kimi_delta_attention_31_b200.run_workload --op decode --N 64 --H 32 --iters 5
 
 Prints the mean CUDA-event time per call.
@@ -33,7 +34,10 @@ def main(argv=None):
     ap.add_argument("--chunk", type=int, default=64)
     ap.add_argument("--dtype", choices=["bf16", "f32"], default="bf16")
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--local-kernel", type=int, choices=[0, 1], default=0,
+                    help="chunk-local kernel of the prefill: 0 warp-specialised (default), 1 two-CTA")
     a = ap.parse_args(argv)
+    kda.set_local_kernel(a.local_kernel)
     dev = torch.device("cuda:0")
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if a.op == "prefill":
