@@ -404,11 +404,13 @@ def set_local_kernel(variant: int) -> None:
 
 
 def uses_ws_kernel(gate="log_channel", packed=False, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16) -> bool:
-    """Whether a chunk_fwd call of this kind on this thread runs the
-    warp-specialised chunk-local kernel: tensor-core path, per-channel
-    log-decay gate (gate="log_channel"; "log_token" = Gated DeltaNet,
-    "logit" = raw gate logits), one sequence per batch row."""
-    return (launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 2 and gate == "log_channel" and not packed
+    """Whether a prefill call of this kind on this thread runs the
+    warp-specialised chunk-local kernel: tensor-core path, one sequence per
+    batch row, any gate ("log_channel" = KDA, "log_token" = Gated DeltaNet,
+    "logit" = raw gate logits with the preparation fused)."""
+    if gate not in ("log_channel", "log_token", "logit"):
+        raise ValueError(f"gate {gate!r}")
+    return (launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 2 and not packed
             and getattr(_tls, "local_kernel", 0) == 0)
 
 

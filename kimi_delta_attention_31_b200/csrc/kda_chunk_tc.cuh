@@ -1243,14 +1243,15 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   if (items >= (1LL << 31)) return cudaErrorInvalidValue;  // item indices are 32-bit
   const FastDiv fdH = make_fastdiv((uint32_t)H);
   const FastDiv fdC = make_fastdiv((uint32_t)std::max(1, (T + tc::C - 1) / tc::C));
-  // The warp-specialised kernel takes per-channel log-decays on the one-row-per-
-  // sequence layout; `local_kernel` == 1 keeps every call on the two-CTA kernel.
-  const bool use_ws = items > 0 && local_kernel != 1 && gmode == kGateLogCh && !cu_seqlens &&
-                      (long long)B * T < (1LL << 31) && ws::ws_kernel_available();
+  // The warp-specialised kernel takes the one-row-per-sequence layout (every
+  // gate mode); `local_kernel` == 1 keeps every call on the two-CTA kernel.
+  const bool use_ws = items > 0 && local_kernel != 1 && !cu_seqlens && (long long)B * T < (1LL << 31) &&
+                      ws::ws_kernel_available();
   if (use_ws) {
     const TcWorkspace lay = tc_workspace_layout(max_chunks, H, N * (long long)H, T, seg_chunks);
-    e = ws::launch_ws_local(q, k, v, static_cast<const float*>(g), beta, B, T, H, items, fdH, fdC, ws,
-                            reinterpret_cast<uint32_t*>(ws + lay.lists), std::min(s_sms, kMaxListCtas), stream);
+    e = ws::launch_ws_local(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws,
+                            reinterpret_cast<uint32_t*>(ws + lay.lists), std::min(s_sms, kMaxListCtas), gmode,
+                            stream);
     if (e != cudaSuccess) return e;
   } else if (items > 0) {
     const int gridA = (int)(items < 2LL * s_sms ? items : 2LL * s_sms);

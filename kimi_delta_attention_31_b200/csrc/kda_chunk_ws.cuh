@@ -1,6 +1,7 @@
 // kda_chunk_ws.cuh -- warp-specialised chunk-local kernel for the KDA prefill
-// (bf16 q, k, v; dk = dv = 128; C = 64; per-channel log-decay gate; one
-// sequence per batch row).  It computes the same per-(chunk, head) image as
+// (bf16 q, k, v; dk = dv = 128; C = 64; one sequence per batch row; every gate
+// mode: per-channel log-decay, per-token log-decay (Gated DeltaNet), or raw
+// per-channel gate logits with the input preparation fused).  It computes the same per-(chunk, head) image as
 // kda_tc_chunk_local_kernel ("Deriving Kimi Delta Attention from scratch",
 // section 6, chunked mode; "Linear / sparse attention" tutorial, section 5.3
 // WY representation): P, U^T, [W; Q e^G], Kbar and gamma, on the
@@ -86,7 +87,13 @@ static_assert(WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_
                   WS_UW % 1024 == 0, "alignment");
 static_assert(IMG_A1 - IMG_U == 16384 && IMG_U - IMG_P == 8192, "image order");
 
-constexpr uint32_t kRawBytes = 2 * C * D * 2 + C * D * 4;  // k, q (bf16) and g (fp32)
+// Bytes of one item's raw rows: k, q (bf16) and g -- fp32 per channel, bf16 per
+// channel, or none (a per-token gate is read with plain loads: its box would be
+// 4 bytes wide, below the 16-byte minimum of a tensor copy).
+template <int kGate>
+constexpr uint32_t raw_bytes() {
+  return 2 * C * D * 2 + (kGate == kGateLogTok ? 0u : kGate == kGateLogitBf16 ? C * D * 2 : C * D * 4);
+}
 constexpr uint32_t kVBytes = C * D * 2;
 constexpr uint32_t kTmemCols = 256;  // [A'; P'] slot 0 | slot 1 | W^T | U^T, 64 columns each
 constexpr float kLog2e = 1.4426950408889634f;
@@ -128,10 +135,12 @@ template <int kGate>
 __global__ void __launch_bounds__(512, 1)
     kda_ws_chunk_local_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
-                              const float* __restrict__ beta, int T, int H, uint32_t num_items, FastDiv fdH,
+                              const void* __restrict__ gate, const float* __restrict__ beta, int T, int H,
+                              uint32_t num_items, FastDiv fdH,
                               FastDiv fdC, uint8_t* __restrict__ ws, uint32_t* __restrict__ steep_list,
                               uint32_t* __restrict__ steep_cnt, uint32_t list_cap) {
-  static_assert(kGate == kGateLogCh, "the warp-specialised kernel takes per-channel log-decays");
+  constexpr bool kPrep = gate_prep(kGate);
+  constexpr bool kTmaGate = kGate != kGateLogTok;
   __shared__ __align__(16) float s_beta[2][C];
   __shared__ __align__(16) float s_glast[D];  // G at the chunk's last row
   __shared__ __align__(8) uint64_t s_raw_full, s_v_full, s_a_done[2], s_b_done[2], s_drain;
@@ -168,16 +177,16 @@ __global__ void __launch_bounds__(512, 1)
 
   auto issue_raw = [&](uint32_t item) {
     const ItemPos p = item_pos(item, T, H, fdH, fdC);
-    ptx::mbar_arrive_expect_tx(&s_raw_full, kRawBytes);
+    ptx::mbar_arrive_expect_tx(&s_raw_full, raw_bytes<kGate>());
     ptx::tma_load_3d(sm + WS_RAWK, &tm_k, 0, p.h, (int)p.s0, &s_raw_full);
     ptx::tma_load_3d(sm + WS_RAWQ, &tm_q, 0, p.h, (int)p.s0, &s_raw_full);
-    ptx::tma_load_3d(sm + WS_RAWG, &tm_g, 0, p.h, (int)p.s0, &s_raw_full);
+    if constexpr (kTmaGate) ptx::tma_load_3d(sm + WS_RAWG, &tm_g, 0, p.h, (int)p.s0, &s_raw_full);
   };
   auto prefetch_l2 = [&](uint32_t item) {
     const ItemPos p = item_pos(item, T, H, fdH, fdC);
     ptx::tma_prefetch_l2_3d(&tm_k, 0, p.h, (int)p.s0);
     ptx::tma_prefetch_l2_3d(&tm_q, 0, p.h, (int)p.s0);
-    ptx::tma_prefetch_l2_3d(&tm_g, 0, p.h, (int)p.s0);
+    if constexpr (kTmaGate) ptx::tma_prefetch_l2_3d(&tm_g, 0, p.h, (int)p.s0);
     ptx::tma_prefetch_l2_3d(&tm_v, 0, p.h, (int)p.s0);
     ptx::tma_prefetch_l2_3d(&tm_v, 64, p.h, (int)p.s0);
   };
@@ -200,7 +209,7 @@ __global__ void __launch_bounds__(512, 1)
     if (tid == 0) {
       ptx::prefetch_tmap(&tm_k);
       ptx::prefetch_tmap(&tm_q);
-      ptx::prefetch_tmap(&tm_g);
+      if constexpr (kTmaGate) ptx::prefetch_tmap(&tm_g);
       ptx::prefetch_tmap(&tm_v);
       if (blockIdx.x < num_items) {
         issue_raw(blockIdx.x);
@@ -214,7 +223,13 @@ __global__ void __launch_bounds__(512, 1)
       const int slot = n & 1;
       const ItemPos p = item_pos(item, T, H, fdH, fdC);
       float bt = 0.f;
-      if (tid < p.Cn) bt = beta[(size_t)(p.s0 + tid) * H + p.h];
+      if (tid < p.Cn) bt = beta_of(beta, kGate, (size_t)(p.s0 + tid) * H + p.h);
+      float gtok[4] = {0.f, 0.f, 0.f, 0.f};  // per-token gate of this thread's rows
+      if constexpr (kGate == kGateLogTok) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (4 * rg + u < p.Cn) gtok[u] = static_cast<const float*>(gate)[(size_t)(p.s0 + 4 * rg + u) * H + p.h];
+      }
 
       // ---- raw rows to registers; rows >= Cn contribute k = q = 0, g = 0
       wait_or_abort(&s_raw_full, n & 1, abort_flag);
@@ -228,19 +243,57 @@ __global__ void __launch_bounds__(512, 1)
         if (r < p.Cn) {
           kw = *reinterpret_cast<const uint4*>(sm + WS_RAWK + r * 256 + 16 * co);
           qw = *reinterpret_cast<const uint4*>(sm + WS_RAWQ + r * 256 + 16 * co);
-          // the two 16-byte halves in alternating order across the quarter-warp (no bank conflicts)
-          const float* gr = reinterpret_cast<const float*>(sm + WS_RAWG + r * 512) + c0;
-          const int sw = (co >> 2) & 1;
-          const float4 h0 = *reinterpret_cast<const float4*>(gr + 4 * sw);
-          const float4 h1 = *reinterpret_cast<const float4*>(gr + 4 - 4 * sw);
-          a = sw ? h1 : h0;
-          b = sw ? h0 : h1;
+          if constexpr (kGate == kGateLogTok) {
+            a = make_float4(gtok[u], gtok[u], gtok[u], gtok[u]);
+            b = a;
+          } else if constexpr (kGate == kGateLogitBf16) {
+            float x[8];
+            tc::unpack8(*reinterpret_cast<const uint4*>(sm + WS_RAWG + r * 256 + 16 * co), x);
+            a = make_float4(neg_softplus(x[0]), neg_softplus(x[1]), neg_softplus(x[2]), neg_softplus(x[3]));
+            b = make_float4(neg_softplus(x[4]), neg_softplus(x[5]), neg_softplus(x[6]), neg_softplus(x[7]));
+          } else {
+            // the two 16-byte halves in alternating order across the quarter-warp (no bank conflicts)
+            const float* gr = reinterpret_cast<const float*>(sm + WS_RAWG + r * 512) + c0;
+            const int sw = (co >> 2) & 1;
+            const float4 h0 = *reinterpret_cast<const float4*>(gr + 4 * sw);
+            const float4 h1 = *reinterpret_cast<const float4*>(gr + 4 - 4 * sw);
+            a = sw ? h1 : h0;
+            b = sw ? h0 : h1;
+            if constexpr (kGate == kGateLogitF32) {
+              a = make_float4(neg_softplus(a.x), neg_softplus(a.y), neg_softplus(a.z), neg_softplus(a.w));
+              b = make_float4(neg_softplus(b.x), neg_softplus(b.y), neg_softplus(b.z), neg_softplus(b.w));
+            }
+          }
         }
         kst[4 * u] = kw.x; kst[4 * u + 1] = kw.y; kst[4 * u + 2] = kw.z; kst[4 * u + 3] = kw.w;
         qst[4 * u] = qw.x; qst[4 * u + 1] = qw.y; qst[4 * u + 2] = qw.z; qst[4 * u + 3] = qw.w;
         const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) G[u][e] = (u ? G[u - 1][e] : 0.f) + x[e];
+      }
+      // 1 / |k_r| and 1 / |q_r| over dk (only when the call normalises): the 16
+      // lanes of a half-warp hold one row
+      float nk[4] = {1.f, 1.f, 1.f, 1.f}, nq[4] = {1.f, 1.f, 1.f, 1.f};
+      if constexpr (kPrep) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float kx[8], qx[8];
+          tc::unpack8(make_uint4(kst[4 * u], kst[4 * u + 1], kst[4 * u + 2], kst[4 * u + 3]), kx);
+          tc::unpack8(make_uint4(qst[4 * u], qst[4 * u + 1], qst[4 * u + 2], qst[4 * u + 3]), qx);
+          float sk = 0.f, sq = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            sk = fmaf(kx[e], kx[e], sk);
+            sq = fmaf(qx[e], qx[e], sq);
+          }
+#pragma unroll
+          for (int off = 1; off < 16; off <<= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+          }
+          nk[u] = rsqrtf(fmaxf(sk, 1e-24f));
+          nq[u] = rsqrtf(fmaxf(sq, 1e-24f));
+        }
       }
       // Row-group totals: this warp holds row groups 2w (lanes 0..15) and 2w+1
       // (lanes 16..31) of the same channels; the warp's total goes to s_wtot,
@@ -270,6 +323,10 @@ __global__ void __launch_bounds__(512, 1)
           const float4 t1 = reinterpret_cast<const float4*>(s_wtot + w2 * D + c0)[1];
           off[0] += t0.x; off[1] += t0.y; off[2] += t0.z; off[3] += t0.w;
           off[4] += t1.x; off[5] += t1.y; off[6] += t1.z; off[7] += t1.w;
+        }
+        if constexpr (kGate == kGateLogTok) {  // one gate per token: every channel has the same G
+#pragma unroll
+          for (int e = 1; e < 8; ++e) off[e] = off[0];
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -310,6 +367,7 @@ __global__ void __launch_bounds__(512, 1)
           float kv[8], qv[8];
           tc::unpack8(make_uint4(kst[4 * u], kst[4 * u + 1], kst[4 * u + 2], kst[4 * u + 3]), kv);
           tc::unpack8(make_uint4(qst[4 * u], qst[4 * u + 1], qst[4 * u + 2], qst[4 * u + 3]), qv);
+          if constexpr (kPrep) tc::normalise_rows(kv, qv, nk[u], nq[u]);
           float o_ka[8], o_qa[8], o_kr[8], o_kb[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -517,13 +575,19 @@ inline bool ws_kernel_available() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   run_once_per_device(once, [dev] {
-    const void* fn = (const void*)kda_ws_chunk_local_kernel<kGateLogCh>;
+    const void* fns[] = {(const void*)kda_ws_chunk_local_kernel<kGateLogCh>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogTok>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogitF32>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogitBf16>};
     int optin = 0;
-    cudaFuncAttributes fa{};
-    ok[dev] = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess &&
-              cudaFuncGetAttributes(&fa, fn) == cudaSuccess &&
-              (size_t)WS_DYN + fa.sharedSizeBytes <= (size_t)optin &&
-              cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WS_DYN) == cudaSuccess;
+    bool all = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
+    for (const void* fn : fns) {
+      cudaFuncAttributes fa{};
+      all = all && cudaFuncGetAttributes(&fa, fn) == cudaSuccess &&
+            (size_t)WS_DYN + fa.sharedSizeBytes <= (size_t)optin &&
+            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WS_DYN) == cudaSuccess;
+    }
+    ok[dev] = all;
     cudaGetLastError();  // an unavailable kernel is not an error of the call
     return cudaSuccess;
   });
@@ -536,10 +600,11 @@ inline uint32_t ws_list_cap(long long items, int grid) { return (uint32_t)((item
 
 // Launches the warp-specialised kernel over all items (grid = one CTA per SM)
 // and then the two-CTA kernel over the chunks it passed on.
-inline cudaError_t launch_ws_local(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                                   const float* g, const float* beta, int B, int T, int H, long long items,
-                                   FastDiv fdH, FastDiv fdC, uint8_t* ws, uint32_t* lists, int sms,
-                                   cudaStream_t stream) {
+template <int kGate>
+inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                     const void* g, const float* beta, int B, int T, int H, long long items,
+                                     FastDiv fdH, FastDiv fdC, uint8_t* ws, uint32_t* lists, int sms,
+                                     cudaStream_t stream) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   cudaError_t e = tensor_map_encoder(&enc);
   if (e != cudaSuccess) return e;
@@ -547,17 +612,39 @@ inline cudaError_t launch_ws_local(const __nv_bfloat16* q, const __nv_bfloat16* 
   CUtensorMap mk, mq, mg, mv;
   if ((e = encode_rows_map(enc, &mk, k, false, tokens, H, D, false)) != cudaSuccess) return e;
   if ((e = encode_rows_map(enc, &mq, q, false, tokens, H, D, false)) != cudaSuccess) return e;
-  if ((e = encode_rows_map(enc, &mg, g, true, tokens, H, D, false)) != cudaSuccess) return e;
   if ((e = encode_rows_map(enc, &mv, v, false, tokens, H, 64, true)) != cudaSuccess) return e;
+  if constexpr (kGate == kGateLogTok) {
+    mg = mk;  // not read: a per-token gate takes plain loads
+  } else {
+    if ((e = encode_rows_map(enc, &mg, g, kGate != kGateLogitBf16, tokens, H, D, false)) != cudaSuccess) return e;
+  }
   const int grid = (int)std::min<long long>(items, sms);
   const uint32_t cap = ws_list_cap(items, grid);
   uint32_t* cnt = lists + (size_t)grid * cap;
-  kda_ws_chunk_local_kernel<kGateLogCh><<<grid, 512, WS_DYN, stream>>>(mk, mq, mg, mv, beta, T, H, (uint32_t)items,
-                                                                      fdH, fdC, ws, lists, cnt, cap);
+  kda_ws_chunk_local_kernel<kGate><<<grid, 512, WS_DYN, stream>>>(mk, mq, mg, mv, g, beta, T, H, (uint32_t)items,
+                                                                  fdH, fdC, ws, lists, cnt, cap);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc::kda_tc_chunk_local_kernel<kGateLogCh><<<grid, 256, tc::KA_DYN, stream>>>(
+  tc::kda_tc_chunk_local_kernel<kGate><<<grid, 256, tc::KA_DYN, stream>>>(
       q, k, v, g, beta, nullptr, 0, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap);
   return cudaGetLastError();
+}
+
+inline cudaError_t launch_ws_local(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                   const void* g, const float* beta, int B, int T, int H, long long items,
+                                   FastDiv fdH, FastDiv fdC, uint8_t* ws, uint32_t* lists, int sms, int gmode,
+                                   cudaStream_t stream) {
+  switch (gmode) {
+    case kGateLogCh:
+      return launch_ws_local_t<kGateLogCh>(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws, lists, sms, stream);
+    case kGateLogTok:
+      return launch_ws_local_t<kGateLogTok>(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws, lists, sms, stream);
+    case kGateLogitF32:
+      return launch_ws_local_t<kGateLogitF32>(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws, lists, sms, stream);
+    case kGateLogitBf16:
+      return launch_ws_local_t<kGateLogitBf16>(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws, lists, sms, stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace ws

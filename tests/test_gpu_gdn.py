@@ -47,23 +47,26 @@ def test_gdn_prefill_varlen_small(cuda_device, dtype, d):
 @pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 32)])
 def test_gdn_equals_kda_with_broadcast_gate(cuda_device, dtype, d):
     """The scalar-gate entry point reads g[t, h] where the per-channel one reads
-    g[t, h, c]; fed the broadcast gate, the same kernels give the same bits.
-    (The per-channel call's default chunk-local kernel on the tensor-core path
-    is the warp-specialised one, which sums G in another order: the same bits
-    come from the two-CTA kernel, and the default agrees to rounding.)"""
+    g[t, h, c]; fed the broadcast gate, the same kernel gives the same bits --
+    for each of the two chunk-local kernels of the tensor-core path (the
+    warp-specialised default and the two-CTA one), which agree with each
+    other to rounding (they sum G in different orders)."""
     inp = W.make_prefill(2, 150, 4, d, d, dtype, -3.0, 1.0, 0.05, seed=32, device=cuda_device,
                          scalar_gate=True)
-    o1, S1 = _gdn(inp, 64)
     g_full = inp["g"].unsqueeze(-1).expand(2, 150, 4, d).contiguous()
-    kda.set_local_kernel(1)
-    try:
-        o2, S2 = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], g_full, inp["beta"], inp["S0"], None, 64)
-    finally:
-        kda.set_local_kernel(0)
-    o3, S3 = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], g_full, inp["beta"], inp["S0"], None, 64)
-    torch.cuda.synchronize()
-    assert torch.equal(o1, o2) and torch.equal(S1, S2)
-    assert rel_rms(o3.float().cpu(), o1.float().cpu()) < 1e-3 and rel_rms(S3.cpu(), S1.cpu()) < 1e-3
+    res = []
+    for variant in (0, 1):
+        kda.set_local_kernel(variant)
+        try:
+            o1, S1 = _gdn(inp, 64)
+            o2, S2 = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], g_full, inp["beta"], inp["S0"], None, 64)
+        finally:
+            kda.set_local_kernel(0)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(S1, S2)
+        res.append((o1, S1))
+    (oa, Sa), (ob, Sb) = res
+    assert rel_rms(oa.float().cpu(), ob.float().cpu()) < 1e-3 and rel_rms(Sa.cpu(), Sb.cpu()) < 1e-3
 
 
 def test_gdn_prefill_b8_sampled(cuda_device):

@@ -12,7 +12,7 @@ import torch
 
 import kimi_delta_attention_31_b200 as kda
 import kda_workloads as W
-from parity_util import compare_units, rel_rms
+from parity_util import compare_units, compare_units_prep, rel_rms
 
 pytestmark = pytest.mark.gpu
 
@@ -77,3 +77,45 @@ def test_local_kernel_switch_validation():
     with pytest.raises(kda.KDAError):
         kda.set_local_kernel(7)
     kda.set_local_kernel(0)
+
+
+def _both_fn(fn):
+    outs = []
+    for variant in (0, 1):
+        kda.set_local_kernel(variant)
+        try:
+            o, S = fn()
+        finally:
+            kda.set_local_kernel(0)
+        torch.cuda.synchronize()
+        assert kda.device_error() == 0
+        outs.append((o, S))
+    return outs
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 64, 2), (2, 200, 4), (2, 1000, 5)])
+def test_local_kernels_agree_gdn(cuda_device, B, T, H):
+    """Per-token gate (Gated DeltaNet): the warp-specialised kernel reads it
+    with plain loads (no tensor copy)."""
+    inp = W.make_prefill(B, T, H, 128, 128, "bf16", -3.0, 1.0, 0.05, seed=340 + T, device=cuda_device,
+                         scalar_gate=True)
+    (o0, S0), (o1, S1) = _both_fn(lambda: kda.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                                            inp["S0"], None, 64))
+    units = [(n, h) for n in range(B) for h in range(H)]
+    compare_units(inp, o0, S0, units, 1e-2)
+    assert rel_rms(o0.float().cpu(), o1.float().cpu()) < 1e-3
+    assert rel_rms(S0.cpu(), S1.cpu()) < 1e-3
+
+
+@pytest.mark.parametrize("a_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B,T,H", [(1, 65, 2), (2, 1000, 5)])
+def test_local_kernels_agree_prep(cuda_device, a_dtype, B, T, H):
+    """Raw projections: q, k normalised, -softplus of the gate logits and the
+    sigmoid of beta's logits inside the kernels."""
+    inp = W.make_prefill_raw(B, T, H, 128, 128, "bf16", -3.0, 1.0, a_dtype, 0.05, seed=360 + T,
+                             device=cuda_device)
+    (o0, S0), (o1, S1) = _both_fn(lambda: kda.chunk_fwd_prep(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"],
+                                                             inp["S0"], None, 64))
+    compare_units_prep(inp, o0, S0, [(n, h) for n in range(B) for h in range(H)], 1e-2)
+    assert rel_rms(o0.float().cpu(), o1.float().cpu()) < 1e-3
+    assert rel_rms(S0.cpu(), S1.cpu()) < 1e-3
