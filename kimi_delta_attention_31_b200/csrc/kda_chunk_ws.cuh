@@ -14,11 +14,12 @@
 //     K e^G (double-buffered), Q e^G and K e^-G, writes Kbar, Q e^G and
 //     gamma to the image, and issues the [A'; P'] MMA into one of two TMEM
 //     accumulators.  Its thread 0 starts the next item's TMA as soon as the
-//     group has read the raw rows, so that load overlaps the build, and
-//     prefetches the item after it into L2.
+//     group has read the raw rows, so that load overlaps the build.
 //   solver (warps 8..15): scatters A and P out of TMEM, inverts I + A,
 //     issues the W^T / U^T MMAs (V comes straight from TMA in the MMA's
-//     layout), and stores P, then U^T and W^T, with bulk copies.
+//     layout), and stores P, then U^T and W^T, with bulk copies.  One solver
+//     thread outside the solve's serial chains issues its copies and stores,
+//     and the L2 prefetch of the item after next.
 // Items whose chunk decays below the single-reference range on some channel
 // (min G_last < -80) are not built here: the builder appends them to this
 // CTA's item list, and the two-CTA kernel runs that list afterwards with the
@@ -215,7 +216,6 @@ __global__ void __launch_bounds__(512, 1)
         issue_raw(blockIdx.x);
         ++raw_issued;
       }
-      if (blockIdx.x + grid < num_items) prefetch_l2(blockIdx.x + grid);
     }
     uint32_t nsteep = 0;
     uint32_t n = 0;
@@ -312,7 +312,6 @@ __global__ void __launch_bounds__(512, 1)
       if (tid == 0 && item + grid < num_items && !*abort_flag) {
         issue_raw(item + grid);
         ++raw_issued;
-        if (item + 2 * grid < num_items) prefetch_l2(item + 2 * grid);
       }
       {
         float off[8];
@@ -431,7 +430,11 @@ __global__ void __launch_bounds__(512, 1)
   } else {
     // ======================= solver =======================
     const int st = tid - 256, w8 = warp - 8;
-    if (st == 0) {
+    // Solver thread 0 issues the MMAs; thread kIo (warp 11, which has no part in
+    // the solve's serial chains) issues the copies and stores, so that an issue
+    // waiting for room in the copy queue never holds up those chains.
+    constexpr int kIo = 96;
+    if (st == kIo) {
       ptx::prefetch_tmap(&tm_v);
       if (blockIdx.x < num_items) {
         issue_v(blockIdx.x);
@@ -452,17 +455,17 @@ __global__ void __launch_bounds__(512, 1)
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::bar_sync(2, 256);
-        if (st == 0) {
+        if (st == kIo) {
           ptx::bulk_s2g(ws + (size_t)item * IMG_BYTES + IMG_P, sm + WS_TT, 8192);
           ptx::bulk_commit();
         }
-        // ---- T = (I + A)^{-1}, T diag(beta) in bf16.  At each barrier thread 0
+        // ---- T = (I + A)^{-1}, T diag(beta) in bf16.  At each barrier thread kIo
         //      first waits for its stores to have read shared memory: the block
         //      products reuse the U^T / W^T staging (stored at the end of the
         //      previous item), T diag(beta) the P staging.
         tc::solve_t_beta(As, reinterpret_cast<float*>(sm + WS_TS), reinterpret_cast<float*>(sm + WS_UW),
                          s_beta[slot], sm + WS_TT, st, w8, lane, [st] {
-                           if (st == 0) ptx::bulk_wait_read0();
+                           if (st == kIo) ptx::bulk_wait_read0();
                            ptx::bar_sync(2, 256);
                          });
         ptx::fence_proxy_async_smem();
@@ -489,7 +492,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         wait_or_abort(&s_b_done[slot], (n >> 1) & 1, abort_flag);
         ptx::tc_fence_after();
-        if (st == 0 && has_next && !*abort_flag) {  // V is free again: the next item's V
+        if (st == kIo && has_next && !*abort_flag) {  // V is free again: the next item's V
           issue_v(item + grid);
           ++v_issued;
         }
@@ -497,11 +500,11 @@ __global__ void __launch_bounds__(512, 1)
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::bar_sync(2, 256);
-        if (st == 0) {
+        if (st == kIo) {
           ptx::bulk_s2g(ws + (size_t)item * IMG_BYTES + IMG_U, sm + WS_UW, 32768);
           ptx::bulk_commit();
         }
-      } else if (st == 0) {  // skipped item: keep the V and b_done phases in step
+      } else if (st == kIo) {  // skipped item: keep the V and b_done phases in step
         wait_or_abort(&s_v_full, n & 1, abort_flag);
         ptx::mbar_arrive(&s_b_done[slot]);
         if (has_next && !*abort_flag) {
@@ -510,19 +513,22 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-    if (st == 0) ptx::bulk_wait0();
+    if (st == kIo) ptx::bulk_wait0();
   }
 
   // After a timeout: wait (bounded again) for the copies and MMAs still in
   // flight, so that nothing lands in shared or tensor memory after exit.
   ptx::tc_fence_before();
   __syncthreads();
-  if (s_abort && (tid == 0 || tid == 256)) {
-    const uint32_t issued = tid == 0 ? raw_issued : v_issued;
-    uint64_t* bar = tid == 0 ? &s_raw_full : &s_v_full;
-    if (issued) ptx::mbar_wait_bounded(bar, (issued - 1) & 1, 1000000000ull);
-    ptx::mma_commit(&s_drain);
-    ptx::mbar_wait_bounded(&s_drain, 0, 1000000000ull);
+  if (s_abort) {
+    // copies: the builder's thread 0 (raw rows), solver thread 96 (V);
+    // MMAs: the builder's thread 0 ([A'; P']) and solver thread 0 (W^T, U^T)
+    if (tid == 0 && raw_issued) ptx::mbar_wait_bounded(&s_raw_full, (raw_issued - 1) & 1, 1000000000ull);
+    if (tid == 256 + 96 && v_issued) ptx::mbar_wait_bounded(&s_v_full, (v_issued - 1) & 1, 1000000000ull);
+    if (tid == 0 || tid == 256) {
+      ptx::mma_commit(&s_drain);
+      ptx::mbar_wait_bounded(&s_drain, 0, 1000000000ull);
+    }
   }
   ptx::tc_fence_before();
   __syncthreads();
