@@ -405,13 +405,13 @@ def set_local_kernel(variant: int) -> None:
 
 def uses_ws_kernel(gate="log_channel", packed=False, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16) -> bool:
     """Whether a prefill call of this kind on this thread runs the
-    warp-specialised chunk-local kernel: tensor-core path, one sequence per
-    batch row, any gate ("log_channel" = KDA, "log_token" = Gated DeltaNet,
-    "logit" = raw gate logits with the preparation fused)."""
+    warp-specialised chunk-local kernel: tensor-core path, any layout (packed
+    sequences first build a chunk table), any gate ("log_channel" = KDA,
+    "log_token" = Gated DeltaNet, "logit" = raw gate logits with the
+    preparation fused)."""
     if gate not in ("log_channel", "log_token", "logit"):
         raise ValueError(f"gate {gate!r}")
-    return (launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 2 and not packed
-            and getattr(_tls, "local_kernel", 0) == 0)
+    return launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 2 and getattr(_tls, "local_kernel", 0) == 0
 
 
 def segment_chunks(B, T, H, num_seqs=0) -> int:
@@ -448,8 +448,10 @@ def chunk_fwd_kernel_sequence(B, T, H, dk=128, dv=128, chunk_size=64, dtype=torc
     """Every kernel one chunk_fwd call launches, in order."""
     if launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 1:
         return list(KERNELS_SIMT)
-    seq = ([KERNEL_WS, KERNELS_TC[0]] if uses_ws_kernel(gate, num_seqs > 0, dk, dv, chunk_size, dtype)
-           else [KERNELS_TC[0]])
+    if uses_ws_kernel(gate, num_seqs > 0, dk, dv, chunk_size, dtype):
+        seq = (["kda_ws_chunk_table_kernel"] if num_seqs > 0 else []) + [KERNEL_WS, KERNELS_TC[0]]
+    else:
+        seq = [KERNELS_TC[0]]
     if segment_chunks(B, T, H, num_seqs) > 0:
         return seq + [KERNELS_TC[1], "kda_tc_seg_combine_kernel", KERNELS_TC[1]]
     return seq + [KERNELS_TC[1]]

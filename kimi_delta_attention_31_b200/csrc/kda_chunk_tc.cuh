@@ -1195,10 +1195,11 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
 // Workspace: the per-chunk images, then (segmented runs) the maps [N | M] of
 // every segment but the last and the entry state of every segment, fp32,
 // then the warp-specialised kernel's per-CTA item lists (at most
-// items + kMaxListCtas entries and kMaxListCtas counts, uint32).
+// items + kMaxListCtas entries and kMaxListCtas counts, uint32), then (packed
+// sequences) its chunk table, {first token, rows} per chunk, and the count.
 constexpr int kMaxListCtas = 1024;
 struct TcWorkspace {
-  size_t images, maps, seg_init, lists, total;
+  size_t images, maps, seg_init, lists, table, total;
 };
 inline TcWorkspace tc_workspace_layout(long long max_chunks, int H, long long units, int T, int seg_chunks) {
   TcWorkspace w{};
@@ -1211,7 +1212,8 @@ inline TcWorkspace tc_workspace_layout(long long max_chunks, int H, long long un
     w.seg_init = w.maps + (size_t)units * (size_t)(P - 1) * 2 * mat;
     w.lists = w.seg_init + (size_t)units * (size_t)P * mat;
   }
-  w.total = w.lists + ((size_t)max_chunks * (size_t)H + 2 * kMaxListCtas) * sizeof(uint32_t);
+  w.table = (w.lists + ((size_t)max_chunks * (size_t)H + 2 * kMaxListCtas) * sizeof(uint32_t) + 255) & ~(size_t)255;
+  w.total = w.table + (size_t)max_chunks * sizeof(int2) + 16;
   return w;
 }
 
@@ -1243,14 +1245,15 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   if (items >= (1LL << 31)) return cudaErrorInvalidValue;  // item indices are 32-bit
   const FastDiv fdH = make_fastdiv((uint32_t)H);
   const FastDiv fdC = make_fastdiv((uint32_t)std::max(1, (T + tc::C - 1) / tc::C));
-  // The warp-specialised kernel takes the one-row-per-sequence layout (every
-  // gate mode); `local_kernel` == 1 keeps every call on the two-CTA kernel.
-  const bool use_ws = items > 0 && local_kernel != 1 && !cu_seqlens && (long long)B * T < (1LL << 31) &&
-                      ws::ws_kernel_available();
+  // The warp-specialised kernel takes every layout and gate mode;
+  // `local_kernel` == 1 keeps every call on the two-CTA kernel.
+  const bool use_ws = items > 0 && local_kernel != 1 && (long long)B * T < (1LL << 31) && ws::ws_kernel_available();
   if (use_ws) {
     const TcWorkspace lay = tc_workspace_layout(max_chunks, H, N * (long long)H, T, seg_chunks);
-    e = ws::launch_ws_local(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws,
-                            reinterpret_cast<uint32_t*>(ws + lay.lists), std::min(s_sms, kMaxListCtas), gmode,
+    int2* table = reinterpret_cast<int2*>(ws + lay.table);
+    e = ws::launch_ws_local(q, k, v, g, beta, cu_seqlens, num_seqs, B, T, H, items, fdH, fdC, ws,
+                            reinterpret_cast<uint32_t*>(ws + lay.lists), table,
+                            reinterpret_cast<int*>(table + max_chunks), std::min(s_sms, kMaxListCtas), gmode,
                             stream);
     if (e != cudaSuccess) return e;
   } else if (items > 0) {

@@ -1,7 +1,8 @@
 // kda_chunk_ws.cuh -- warp-specialised chunk-local kernel for the KDA prefill
-// (bf16 q, k, v; dk = dv = 128; C = 64; one sequence per batch row; every gate
-// mode: per-channel log-decay, per-token log-decay (Gated DeltaNet), or raw
-// per-channel gate logits with the input preparation fused).  It computes the same per-(chunk, head) image as
+// (bf16 q, k, v; dk = dv = 128; C = 64; one sequence per batch row or packed
+// sequences; every gate mode: per-channel log-decay, per-token log-decay
+// (Gated DeltaNet), or raw per-channel gate logits with the input preparation
+// fused).  It computes the same per-(chunk, head) image as
 // kda_tc_chunk_local_kernel ("Deriving Kimi Delta Attention from scratch",
 // section 6, chunked mode; "Linear / sparse attention" tutorial, section 5.3
 // WY representation): P, U^T, [W; Q e^G], Kbar and gamma, on the
@@ -103,15 +104,72 @@ struct ItemPos {
   long long s0;  // first token (row of the [tokens, H, D] tensors)
   int h, Cn;     // head, valid rows of the chunk
 };
-__device__ __forceinline__ ItemPos item_pos(uint32_t item, int T, int H, const FastDiv& fdH, const FastDiv& fdC) {
+// item = chunk * H + head.  One sequence per batch row: chunk = row * fdC.d +
+// chunk-in-row.  Packed sequences: chunk_table[chunk] = {first token, rows}.
+__device__ __forceinline__ ItemPos item_pos(uint32_t item, int T, int H, const FastDiv& fdH, const FastDiv& fdC,
+                                            const int2* chunk_table) {
   const uint32_t ci = fdiv(item, fdH);
-  const uint32_t bq = fdiv(ci, fdC);
-  const int cc = (int)(ci - bq * fdC.d);
   ItemPos p;
   p.h = (int)(item - ci * (uint32_t)H);
-  p.s0 = (long long)bq * T + (long long)cc * C;
-  p.Cn = min(C, T - cc * C);
+  if (chunk_table) {
+    const int2 e = chunk_table[ci];
+    p.s0 = e.x;
+    p.Cn = e.y;
+  } else {
+    const uint32_t bq = fdiv(ci, fdC);
+    const int cc = (int)(ci - bq * fdC.d);
+    p.s0 = (long long)bq * T + (long long)cc * C;
+    p.Cn = min(C, T - cc * C);
+  }
   return p;
+}
+
+// Chunk table of packed sequences (one CTA of 1024 threads): for every chunk of
+// every sequence in order, {first token, rows}; *total = the number of chunks.
+// A block-wide exclusive scan of the per-sequence chunk counts, 1024 sequences
+// at a time.
+__global__ void __launch_bounds__(1024)
+    kda_ws_chunk_table_kernel(const int32_t* __restrict__ cu_seqlens, int num_seqs, int2* __restrict__ table,
+                              int* __restrict__ total) {
+  __shared__ int s_warp[32];
+  __shared__ int s_carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  for (int base = 0; base < num_seqs; base += 1024) {
+    const int i = base + tid;
+    int st = 0, len = 0;
+    if (i < num_seqs) {
+      st = cu_seqlens[i];
+      len = cu_seqlens[i + 1] - st;
+    }
+    const int nch = len > 0 ? (len + C - 1) / C : 0;
+    int incl = nch;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = s_warp[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w += t;
+      }
+      s_warp[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int carry = s_carry;
+    const int excl = carry + (warp ? s_warp[warp - 1] : 0) + incl - nch;
+    for (int c = 0; c < nch; ++c) table[excl + c] = make_int2(st + c * C, min(C, len - c * C));
+    __syncthreads();  // everyone has read s_carry and s_warp
+    if (tid == 0) s_carry = carry + s_warp[31];
+    __syncthreads();
+  }
+  if (tid == 0) *total = s_carry;
 }
 
 // Bounded wait that also gives up at once when another thread of the CTA has
@@ -139,7 +197,8 @@ __global__ void __launch_bounds__(512, 1)
                               const void* __restrict__ gate, const float* __restrict__ beta, int T, int H,
                               uint32_t num_items, FastDiv fdH,
                               FastDiv fdC, uint8_t* __restrict__ ws, uint32_t* __restrict__ steep_list,
-                              uint32_t* __restrict__ steep_cnt, uint32_t list_cap) {
+                              uint32_t* __restrict__ steep_cnt, uint32_t list_cap,
+                              const int2* __restrict__ chunk_table, const int* __restrict__ chunk_total) {
   constexpr bool kPrep = gate_prep(kGate);
   constexpr bool kTmaGate = kGate != kGateLogTok;
   __shared__ __align__(16) float s_beta[2][C];
@@ -154,6 +213,8 @@ __global__ void __launch_bounds__(512, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort_flag = &s_abort;
   const uint32_t grid = gridDim.x;
+  // packed sequences: the exact item count (num_items is the host's upper bound)
+  if (chunk_table) num_items = min(num_items, (uint32_t)max(*chunk_total, 0) * (uint32_t)H);
 
   if (warp == 0) {
     ptx::tmem_alloc(&s_tmem, kTmemCols);
@@ -177,14 +238,14 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = s_tmem;
 
   auto issue_raw = [&](uint32_t item) {
-    const ItemPos p = item_pos(item, T, H, fdH, fdC);
+    const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
     ptx::mbar_arrive_expect_tx(&s_raw_full, raw_bytes<kGate>());
     ptx::tma_load_3d(sm + WS_RAWK, &tm_k, 0, p.h, (int)p.s0, &s_raw_full);
     ptx::tma_load_3d(sm + WS_RAWQ, &tm_q, 0, p.h, (int)p.s0, &s_raw_full);
     if constexpr (kTmaGate) ptx::tma_load_3d(sm + WS_RAWG, &tm_g, 0, p.h, (int)p.s0, &s_raw_full);
   };
   auto prefetch_l2 = [&](uint32_t item) {
-    const ItemPos p = item_pos(item, T, H, fdH, fdC);
+    const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
     ptx::tma_prefetch_l2_3d(&tm_k, 0, p.h, (int)p.s0);
     ptx::tma_prefetch_l2_3d(&tm_q, 0, p.h, (int)p.s0);
     if constexpr (kTmaGate) ptx::tma_prefetch_l2_3d(&tm_g, 0, p.h, (int)p.s0);
@@ -192,7 +253,7 @@ __global__ void __launch_bounds__(512, 1)
     ptx::tma_prefetch_l2_3d(&tm_v, 64, p.h, (int)p.s0);
   };
   auto issue_v = [&](uint32_t item) {
-    const ItemPos p = item_pos(item, T, H, fdH, fdC);
+    const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
     ptx::mbar_arrive_expect_tx(&s_v_full, kVBytes);
     ptx::tma_load_3d(sm + WS_V, &tm_v, 0, p.h, (int)p.s0, &s_v_full);
     ptx::tma_load_3d(sm + WS_V + 8192, &tm_v, 64, p.h, (int)p.s0, &s_v_full);
@@ -221,7 +282,7 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t n = 0;
     for (uint32_t item = blockIdx.x; item < num_items; item += grid, ++n) {
       const int slot = n & 1;
-      const ItemPos p = item_pos(item, T, H, fdH, fdC);
+      const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
       float bt = 0.f;
       if (tid < p.Cn) bt = beta_of(beta, kGate, (size_t)(p.s0 + tid) * H + p.h);
       float gtok[4] = {0.f, 0.f, 0.f, 0.f};  // per-token gate of this thread's rows
@@ -606,11 +667,13 @@ inline uint32_t ws_list_cap(long long items, int grid) { return (uint32_t)((item
 
 // Launches the warp-specialised kernel over all items (grid = one CTA per SM)
 // and then the two-CTA kernel over the chunks it passed on.
+// Packed sequences (cu_seqlens != NULL): first the chunk table, then the
+// kernels look positions up in it.
 template <int kGate>
 inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                                     const void* g, const float* beta, int B, int T, int H, long long items,
-                                     FastDiv fdH, FastDiv fdC, uint8_t* ws, uint32_t* lists, int sms,
-                                     cudaStream_t stream) {
+                                     const void* g, const float* beta, const int32_t* cu_seqlens, int num_seqs,
+                                     int B, int T, int H, long long items, FastDiv fdH, FastDiv fdC, uint8_t* ws,
+                                     uint32_t* lists, int2* table, int* table_total, int sms, cudaStream_t stream) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   cudaError_t e = tensor_map_encoder(&enc);
   if (e != cudaSuccess) return e;
@@ -624,33 +687,40 @@ inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16
   } else {
     if ((e = encode_rows_map(enc, &mg, g, kGate != kGateLogitBf16, tokens, H, D, false)) != cudaSuccess) return e;
   }
+  if (cu_seqlens) {
+    kda_ws_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, table, table_total);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   const int grid = (int)std::min<long long>(items, sms);
   const uint32_t cap = ws_list_cap(items, grid);
   uint32_t* cnt = lists + (size_t)grid * cap;
-  kda_ws_chunk_local_kernel<kGate><<<grid, 512, WS_DYN, stream>>>(mk, mq, mg, mv, g, beta, T, H, (uint32_t)items,
-                                                                  fdH, fdC, ws, lists, cnt, cap);
+  kda_ws_chunk_local_kernel<kGate><<<grid, 512, WS_DYN, stream>>>(
+      mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap,
+      cu_seqlens ? table : nullptr, cu_seqlens ? table_total : nullptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   tc::kda_tc_chunk_local_kernel<kGate><<<grid, 256, tc::KA_DYN, stream>>>(
-      q, k, v, g, beta, nullptr, 0, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap);
+      q, k, v, g, beta, cu_seqlens, cu_seqlens ? num_seqs : 0, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap);
   return cudaGetLastError();
 }
 
 inline cudaError_t launch_ws_local(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                                   const void* g, const float* beta, int B, int T, int H, long long items,
-                                   FastDiv fdH, FastDiv fdC, uint8_t* ws, uint32_t* lists, int sms, int gmode,
+                                   const void* g, const float* beta, const int32_t* cu_seqlens, int num_seqs, int B,
+                                   int T, int H, long long items, FastDiv fdH, FastDiv fdC, uint8_t* ws,
+                                   uint32_t* lists, int2* table, int* table_total, int sms, int gmode,
                                    cudaStream_t stream) {
+#define KDA_WS_CASE(M)                                                                                     \
+  case M:                                                                                                  \
+    return launch_ws_local_t<M>(q, k, v, g, beta, cu_seqlens, num_seqs, B, T, H, items, fdH, fdC, ws, lists, \
+                                table, table_total, sms, stream)
   switch (gmode) {
-    case kGateLogCh:
-      return launch_ws_local_t<kGateLogCh>(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws, lists, sms, stream);
-    case kGateLogTok:
-      return launch_ws_local_t<kGateLogTok>(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws, lists, sms, stream);
-    case kGateLogitF32:
-      return launch_ws_local_t<kGateLogitF32>(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws, lists, sms, stream);
-    case kGateLogitBf16:
-      return launch_ws_local_t<kGateLogitBf16>(q, k, v, g, beta, B, T, H, items, fdH, fdC, ws, lists, sms, stream);
+    KDA_WS_CASE(kGateLogCh);
+    KDA_WS_CASE(kGateLogTok);
+    KDA_WS_CASE(kGateLogitF32);
+    KDA_WS_CASE(kGateLogitBf16);
     default:
       return cudaErrorInvalidValue;
   }
+#undef KDA_WS_CASE
 }
 
 }  // namespace ws

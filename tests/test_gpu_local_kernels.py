@@ -119,3 +119,42 @@ def test_local_kernels_agree_prep(cuda_device, a_dtype, B, T, H):
     compare_units_prep(inp, o0, S0, [(n, h) for n in range(B) for h in range(H)], 1e-2)
     assert rel_rms(o0.float().cpu(), o1.float().cpu()) < 1e-3
     assert rel_rms(S0.cpu(), S1.cpu()) < 1e-3
+
+
+@pytest.mark.parametrize("lens", [(0, 1, 17, 64, 65, 100, 3), (130,) * 40 + (0, 7), (4096, 1, 2000, 64)])
+def test_local_kernels_agree_packed(cuda_device, lens):
+    """Packed sequences (cu_seqlens): the warp-specialised kernel looks chunk
+    positions up in a table a one-CTA kernel builds from cu_seqlens, and stops
+    at the exact chunk count read on the device (the host's item count is an
+    upper bound)."""
+    inp = W.make_prefill(1, sum(lens), 3, 128, 128, "bf16", -4.0, 1.0, 0.05, seed=380 + len(lens),
+                         device=cuda_device, lengths=lens)
+    (o0, S0), (o1, S1) = _both_fn(lambda: kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                                        inp["S0"], inp["cu_seqlens"], 64))
+    units = [(n, h) for n in range(len(lens)) for h in range(3)][:24]
+    compare_units(inp, o0, S0, units, 1e-2)
+    assert rel_rms(o0.float().cpu(), o1.float().cpu()) < 1e-3
+    assert rel_rms(S0.cpu(), S1.cpu()) < 1e-3
+    for n, L in enumerate(lens):  # an empty sequence hands its state through
+        if L == 0:
+            assert torch.equal(S0[n], inp["S0"][n])
+
+
+def test_local_kernels_packed_steep_mix(cuda_device):
+    """Packed sequences with steep chunks mixed in: the item lists hold
+    packed-layout items that the two-CTA kernel locates from cu_seqlens."""
+    lens = (700, 64, 1000, 5, 300)
+    inp = W.make_prefill(1, sum(lens), 4, 128, 128, "bf16", -4.0, 1.0, 0.05, seed=391, device=cuda_device,
+                         lengths=lens)
+    gen = torch.Generator(device=cuda_device).manual_seed(392)
+    # sequences 0 and 2 decay by about -1.5 per token (-96 over a full chunk:
+    # past the single-reference range), the others by about -0.05
+    rate = torch.cat([torch.full((L,), 1.5 if n in (0, 2) else 0.05) for n, L in enumerate(lens)])
+    rate = rate.to(cuda_device).view(1, -1, 1, 1)
+    inp["g"] = (-rate * (1.0 - 0.005 * torch.rand(inp["g"].shape, generator=gen, device=cuda_device))).contiguous()
+    (o0, S0), (o1, S1) = _both_fn(lambda: kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                                        inp["S0"], inp["cu_seqlens"], 64))
+    assert torch.isfinite(o0).all() and torch.isfinite(S0).all()
+    compare_units(inp, o0, S0, [(0, 0), (1, 1), (2, 2), (3, 3), (4, 0)], 1e-2)
+    assert rel_rms(o0.float().cpu(), o1.float().cpu()) < 1e-3
+    assert rel_rms(S0.cpu(), S1.cpu()) < 1e-3
