@@ -278,11 +278,11 @@ int kda_segment_chunks(int B, int T, int H, int num_seqs);
  * chunk's I + A; inputs arrive by tensor-map TMA) and a two-CTA-per-SM one.
  * For the calling thread's later calls (kda_chunk_fwd, kda_gdn_chunk_fwd,
  * kda_chunk_fwd_prep on the tensor-core path): 0 (default) uses the
- * warp-specialised kernel when there is one sequence per batch row
- * (cu_seqlens == NULL), with the two-CTA kernel for the chunks whose
- * log-decay over the chunk falls below -80 on some channel, and the two-CTA
- * kernel for packed sequences; 1 = the two-CTA kernel always.  Other values:
- * KDA_ERR_INVALID_ARG, setting unchanged.
+ * warp-specialised kernel (packed sequences: after a one-CTA kernel has built
+ * a chunk table from cu_seqlens in the workspace), with the two-CTA kernel for
+ * the chunks whose log-decay over the chunk falls below -80 on some channel;
+ * 1 = the two-CTA kernel always.  Other values: KDA_ERR_INVALID_ARG, setting
+ * unchanged.
  */
 kda_status_t kda_set_local_kernel(int variant);
 
