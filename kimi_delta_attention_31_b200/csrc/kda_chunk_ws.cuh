@@ -19,8 +19,7 @@
 //   solver (warps 8..15): scatters A and P out of TMEM, inverts I + A,
 //     issues the W^T / U^T MMAs (V comes straight from TMA in the MMA's
 //     layout), and stores P, then U^T and W^T, with bulk copies.  One solver
-//     thread outside the solve's serial chains issues its copies and stores,
-//     and the L2 prefetch of the item after next.
+//     thread outside the solve's serial chains issues its copies and stores.
 // Items whose chunk decays below the single-reference range on some channel
 // (min G_last < -80) are not built here: the builder appends them to this
 // CTA's item list, and the two-CTA kernel runs that list afterwards with the
@@ -28,7 +27,9 @@
 //
 // Hand-offs (all mbarriers, one completion per item unless noted):
 //   raw_full      TMA bytes of k, q, g                     builder waits
-//   v_full        TMA bytes of V                           solver thread 0 waits
+//   v_full        TMA bytes of V                           solver thread 0 (before the
+//                                                          W^T / U^T MMA) or, for a
+//                                                          skipped item, the copy thread
 //   a_done[slot]  [A'; P'] MMA complete + builder arrive   solver waits; builder
 //                 (count 2; per slot: items n, n+2, ...)   waits item n-1's (RB reuse)
 //   b_done[slot]  W^T / U^T MMA complete (or skip arrive)  solver waits; builder
@@ -243,14 +244,6 @@ __global__ void __launch_bounds__(512, 1)
     ptx::tma_load_3d(sm + WS_RAWK, &tm_k, 0, p.h, (int)p.s0, &s_raw_full);
     ptx::tma_load_3d(sm + WS_RAWQ, &tm_q, 0, p.h, (int)p.s0, &s_raw_full);
     if constexpr (kTmaGate) ptx::tma_load_3d(sm + WS_RAWG, &tm_g, 0, p.h, (int)p.s0, &s_raw_full);
-  };
-  auto prefetch_l2 = [&](uint32_t item) {
-    const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
-    ptx::tma_prefetch_l2_3d(&tm_k, 0, p.h, (int)p.s0);
-    ptx::tma_prefetch_l2_3d(&tm_q, 0, p.h, (int)p.s0);
-    if constexpr (kTmaGate) ptx::tma_prefetch_l2_3d(&tm_g, 0, p.h, (int)p.s0);
-    ptx::tma_prefetch_l2_3d(&tm_v, 0, p.h, (int)p.s0);
-    ptx::tma_prefetch_l2_3d(&tm_v, 64, p.h, (int)p.s0);
   };
   auto issue_v = [&](uint32_t item) {
     const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
