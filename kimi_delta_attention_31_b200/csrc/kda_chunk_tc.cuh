@@ -376,6 +376,8 @@ __global__ void __launch_bounds__(256, 2)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t rs = (size_t)H * D;  // elements between consecutive tokens
+  // an empty item list (the usual case): nothing to set up
+  if (item_list && item_cnt[blockIdx.x] == 0) return;
 
   if (warp == 0) {
     ptx::tmem_alloc(&s_tmem, 256);
