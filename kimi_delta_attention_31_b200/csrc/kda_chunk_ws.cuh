@@ -107,12 +107,13 @@ struct ItemPos {
 };
 // item = chunk * H + head.  One sequence per batch row: chunk = row * fdC.d +
 // chunk-in-row.  Packed sequences: chunk_table[chunk] = {first token, rows}.
+template <bool kPacked>
 __device__ __forceinline__ ItemPos item_pos(uint32_t item, int T, int H, const FastDiv& fdH, const FastDiv& fdC,
                                             const int2* chunk_table) {
   const uint32_t ci = fdiv(item, fdH);
   ItemPos p;
   p.h = (int)(item - ci * (uint32_t)H);
-  if (chunk_table) {
+  if constexpr (kPacked) {
     const int2 e = chunk_table[ci];
     p.s0 = e.x;
     p.Cn = e.y;
@@ -191,7 +192,9 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   }
 }
 
-template <int kGate>
+// kPacked: positions from the chunk table of packed sequences (a template
+// parameter, so that the one-row-per-sequence form carries none of it).
+template <int kGate, bool kPacked>
 __global__ void __launch_bounds__(512, 1)
     kda_ws_chunk_local_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
@@ -204,6 +207,7 @@ __global__ void __launch_bounds__(512, 1)
   constexpr bool kTmaGate = kGate != kGateLogTok;
   __shared__ __align__(16) float s_beta[2][C];
   __shared__ __align__(16) float s_glast[D];  // G at the chunk's last row
+  __shared__ float s_nrm[2][C];               // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
   __shared__ __align__(8) uint64_t s_raw_full, s_v_full, s_a_done[2], s_b_done[2], s_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_skip[2];
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(512, 1)
   volatile int* abort_flag = &s_abort;
   const uint32_t grid = gridDim.x;
   // packed sequences: the exact item count (num_items is the host's upper bound)
-  if (chunk_table) num_items = min(num_items, (uint32_t)max(*chunk_total, 0) * (uint32_t)H);
+  if constexpr (kPacked) num_items = min(num_items, (uint32_t)max(*chunk_total, 0) * (uint32_t)H);
 
   if (warp == 0) {
     ptx::tmem_alloc(&s_tmem, kTmemCols);
@@ -239,14 +243,14 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = s_tmem;
 
   auto issue_raw = [&](uint32_t item) {
-    const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
+    const ItemPos p = item_pos<kPacked>(item, T, H, fdH, fdC, chunk_table);
     ptx::mbar_arrive_expect_tx(&s_raw_full, raw_bytes<kGate>());
     ptx::tma_load_3d(sm + WS_RAWK, &tm_k, 0, p.h, (int)p.s0, &s_raw_full);
     ptx::tma_load_3d(sm + WS_RAWQ, &tm_q, 0, p.h, (int)p.s0, &s_raw_full);
     if constexpr (kTmaGate) ptx::tma_load_3d(sm + WS_RAWG, &tm_g, 0, p.h, (int)p.s0, &s_raw_full);
   };
   auto issue_v = [&](uint32_t item) {
-    const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
+    const ItemPos p = item_pos<kPacked>(item, T, H, fdH, fdC, chunk_table);
     ptx::mbar_arrive_expect_tx(&s_v_full, kVBytes);
     ptx::tma_load_3d(sm + WS_V, &tm_v, 0, p.h, (int)p.s0, &s_v_full);
     ptx::tma_load_3d(sm + WS_V + 8192, &tm_v, 64, p.h, (int)p.s0, &s_v_full);
@@ -275,7 +279,7 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t n = 0;
     for (uint32_t item = blockIdx.x; item < num_items; item += grid, ++n) {
       const int slot = n & 1;
-      const ItemPos p = item_pos(item, T, H, fdH, fdC, chunk_table);
+      const ItemPos p = item_pos<kPacked>(item, T, H, fdH, fdC, chunk_table);
       float bt = 0.f;
       if (tid < p.Cn) bt = beta_of(beta, kGate, (size_t)(p.s0 + tid) * H + p.h);
       float gtok[4] = {0.f, 0.f, 0.f, 0.f};  // per-token gate of this thread's rows
@@ -326,8 +330,9 @@ __global__ void __launch_bounds__(512, 1)
         for (int e = 0; e < 8; ++e) G[u][e] = (u ? G[u - 1][e] : 0.f) + x[e];
       }
       // 1 / |k_r| and 1 / |q_r| over dk (only when the call normalises): the 16
-      // lanes of a half-warp hold one row
-      float nk[4] = {1.f, 1.f, 1.f, 1.f}, nq[4] = {1.f, 1.f, 1.f, 1.f};
+      // lanes of a half-warp hold one row.  Kept in shared memory, not in
+      // registers: written before the group's next barrier, read in the build,
+      // and not rewritten before the item's last barrier.
       if constexpr (kPrep) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -345,8 +350,10 @@ __global__ void __launch_bounds__(512, 1)
             sk += __shfl_xor_sync(0xffffffffu, sk, off);
             sq += __shfl_xor_sync(0xffffffffu, sq, off);
           }
-          nk[u] = rsqrtf(fmaxf(sk, 1e-24f));
-          nq[u] = rsqrtf(fmaxf(sq, 1e-24f));
+          if (co == 0) {
+            s_nrm[0][4 * rg + u] = rsqrtf(fmaxf(sk, 1e-24f));
+            s_nrm[1][4 * rg + u] = rsqrtf(fmaxf(sq, 1e-24f));
+          }
         }
       }
       // Row-group totals: this warp holds row groups 2w (lanes 0..15) and 2w+1
@@ -420,7 +427,7 @@ __global__ void __launch_bounds__(512, 1)
           float kv[8], qv[8];
           tc::unpack8(make_uint4(kst[4 * u], kst[4 * u + 1], kst[4 * u + 2], kst[4 * u + 3]), kv);
           tc::unpack8(make_uint4(qst[4 * u], qst[4 * u + 1], qst[4 * u + 2], qst[4 * u + 3]), qv);
-          if constexpr (kPrep) tc::normalise_rows(kv, qv, nk[u], nq[u]);
+          if constexpr (kPrep) tc::normalise_rows(kv, qv, s_nrm[0][r], s_nrm[1][r]);
           float o_ka[8], o_qa[8], o_kr[8], o_kb[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -635,10 +642,14 @@ inline bool ws_kernel_available() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   run_once_per_device(once, [dev] {
-    const void* fns[] = {(const void*)kda_ws_chunk_local_kernel<kGateLogCh>,
-                         (const void*)kda_ws_chunk_local_kernel<kGateLogTok>,
-                         (const void*)kda_ws_chunk_local_kernel<kGateLogitF32>,
-                         (const void*)kda_ws_chunk_local_kernel<kGateLogitBf16>};
+    const void* fns[] = {(const void*)kda_ws_chunk_local_kernel<kGateLogCh, false>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogTok, false>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogitF32, false>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogitBf16, false>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogCh, true>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogTok, true>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogitF32, true>,
+                         (const void*)kda_ws_chunk_local_kernel<kGateLogitBf16, true>};
     int optin = 0;
     bool all = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
     for (const void* fn : fns) {
@@ -687,9 +698,12 @@ inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16
   const int grid = (int)std::min<long long>(items, sms);
   const uint32_t cap = ws_list_cap(items, grid);
   uint32_t* cnt = lists + (size_t)grid * cap;
-  kda_ws_chunk_local_kernel<kGate><<<grid, 512, WS_DYN, stream>>>(
-      mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap,
-      cu_seqlens ? table : nullptr, cu_seqlens ? table_total : nullptr);
+  if (cu_seqlens)
+    kda_ws_chunk_local_kernel<kGate, true><<<grid, 512, WS_DYN, stream>>>(
+        mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap, table, table_total);
+  else
+    kda_ws_chunk_local_kernel<kGate, false><<<grid, 512, WS_DYN, stream>>>(
+        mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap, nullptr, nullptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   tc::kda_tc_chunk_local_kernel<kGate><<<grid, 256, tc::KA_DYN, stream>>>(
       q, k, v, g, beta, cu_seqlens, cu_seqlens ? num_seqs : 0, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap);
