@@ -193,3 +193,24 @@ def test_chunk_bwd_validates_arguments():
     need = lib.kda_chunk_bwd_workspace_size(1, 64, 2, 128, 128, 0)
     assert need == 4 * 2 * 128 * 128 * 4              # 4 chunks of 16 tokens x 2 heads x fp32 states
     assert call(ws=_fake(0x4000), wsb=need - 1) == 4
+
+
+def test_local_kernel_switch():
+    """kda_set_local_kernel takes 0 (warp-specialised where it applies) or 1
+    (two-CTA kernel); anything else is KDA_ERR_INVALID_ARG and leaves the
+    setting unchanged.  The binding mirrors the setting per thread."""
+    lib = kda.load_library()
+    assert lib.kda_set_local_kernel(7) == 1
+    assert "variant" in kda.last_error()
+    kda.set_local_kernel(1)
+    try:
+        assert not kda.uses_ws_kernel()
+        assert kda.chunk_fwd_kernel_sequence(2, 128, 4) == ["kda_tc_chunk_local_kernel", "kda_tc_state_pass_kernel"]
+    finally:
+        kda.set_local_kernel(0)
+    assert kda.uses_ws_kernel("log_token") and kda.uses_ws_kernel("logit", packed=True)
+    assert kda.chunk_fwd_kernel_sequence(2, 128, 4) == ["kda_ws_chunk_local_kernel", "kda_tc_chunk_local_kernel",
+                                                        "kda_tc_state_pass_kernel"]
+    assert kda.chunk_fwd_kernel_sequence(1, 300, 4, num_seqs=3)[0] == "kda_ws_chunk_table_kernel"
+    with pytest.raises(ValueError):
+        kda.uses_ws_kernel("per_head")

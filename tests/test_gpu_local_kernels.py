@@ -73,12 +73,6 @@ def test_local_kernels_scattered_steep_chunks(cuda_device, frac):
     assert rel_rms(S0.cpu(), S1.cpu()) < 1e-3
 
 
-def test_local_kernel_switch_validation():
-    with pytest.raises(kda.KDAError):
-        kda.set_local_kernel(7)
-    kda.set_local_kernel(0)
-
-
 def _both_fn(fn):
     outs = []
     for variant in (0, 1):
