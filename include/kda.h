@@ -86,8 +86,14 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
  *   S_out : [N, H, dk, dv] fp32, or NULL; may alias S0
  *   cu_seqlens : device int32 [num_seqs + 1] (packed varlen layout, B == 1,
  *           T == total tokens, cu_seqlens[0] == 0, non-decreasing,
- *           cu_seqlens[num_seqs] == T; the library trusts these values) or
- *           NULL, in which case num_seqs must be 0 and N = B.
+ *           cu_seqlens[num_seqs] == T) or NULL, in which case num_seqs must
+ *           be 0 and N = B.  The values live on the device, so they are
+ *           checked there: a table that breaks these rules sets the device
+ *           error word (kda_device_error reports KDA_ERR_INVALID_ARG) and no
+ *           read or write leaves the buffers' bounds.  The tensor-core path
+ *           then writes nothing at all (o and S_out keep their contents); the
+ *           fp32 path treats each sequence whose own range [cu[n], cu[n+1])
+ *           is not inside [0, T] as empty (its S_out is its S0).
  *   chunk_size : 16, 32 or 64.  The tensor-core path (bf16, dk == dv == 128)
  *           runs with 64; other combinations run the fp32-arithmetic path.
  *   workspace : device buffer of at least kda_chunk_fwd_workspace_size(...)
@@ -202,6 +208,42 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * kda_chunk_fwd from HOST buffers (library plumbing around the prefill of
+ * "Deriving Kimi Delta Attention from scratch" section 6, chunked mode; the
+ * pages have no host interface).  q, k, v, g, beta, S0 (or NULL), cu_seqlens
+ * (or NULL) are read from host memory and o, S_out (or NULL) written to host
+ * memory, with the layouts, sizes and meaning of kda_chunk_fwd (KDA gates, one
+ * per key channel).  Use page-locked (pinned) host memory: with pageable
+ * memory the copies still happen but do not overlap anything.
+ *
+ * The batch is processed in `pieces` groups of rows (packed inputs: one
+ * group): the host->device copies of group p+1 run on `copy_in`, the prefill
+ * of group p on `compute` and the device->host copies of group p-1 on
+ * `copy_out`, so both copy directions and the kernels work at once.  The three
+ * streams may be the same stream (no overlap then).  Ordering: the copies
+ * start after the work already queued on `compute`, and `compute` waits for
+ * the last copy back, so synchronising `compute` covers the whole call.
+ *
+ *   device_buffer : device memory of at least kda_chunk_fwd_host_buffer_size
+ *     (same sizes, same pieces) bytes, 256-byte aligned; the library keeps the
+ *     device copies of every tensor and the prefill's workspace there.  Its
+ *     contents are scratch; it must not be used by anything else until
+ *     `compute` has passed the call.
+ * Errors: as kda_chunk_fwd (KDA_ERR_WORKSPACE when device_buffer is too
+ * small).  The host buffers must stay valid until `compute` has passed the
+ * call.  Uses three CUDA events per host thread and device, created on the
+ * first call and kept.
+ */
+size_t kda_chunk_fwd_host_buffer_size(int B, int T, int H, int dk, int dv, int num_seqs, int chunk_size,
+                                      kda_dtype_t dtype, int pieces);
+kda_status_t kda_chunk_fwd_host(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, const float* S0, void* o, float* S_out,
+                                const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dk,
+                                int dv, int chunk_size, kda_dtype_t dtype, int pieces,
+                                void* device_buffer, size_t device_buffer_bytes, cudaStream_t compute,
+                                cudaStream_t copy_in, cudaStream_t copy_out);
+
+/*
  * kda_chunk_fwd for callers that cannot allocate device memory: the same
  * prefill, same arguments minus the workspace.  (Library plumbing: the pages
  * have no counterpart.)  Some callers get only input and output pointers
@@ -215,7 +257,10 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
  * KDA_ERR_WORKSPACE (64 MiB holds 903 (chunk, head) pairs of the tensor-core
  * path, e.g. B=1, H=8, T=7168; the fp32-arithmetic path needs none).
  * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * that device current) and remembers it together with the CUDA context that
+ * was current; a call from another context on that device (a driver-API
+ * context, or the primary context re-created after cudaDeviceReset) looks it
+ * up again.  Make the first call in each context before any stream capture.
  * All calls share the one array: calls whose executions overlap on the GPU
  * (other streams, other threads) race and corrupt each other's results.
  * Nothing in it has to start at zero: each call writes every byte it reads.
@@ -231,9 +276,11 @@ kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, 
 const char* kda_last_error(void);
 
 /*
- * Reads and clears the device-side error word that bounded waits inside the
- * kernels set when they give up (KDA_ERR_DEVICE_TIMEOUT).  Synchronises
- * `stream` first.  *code receives 0 when no wait gave up.
+ * Reads and clears the device-side error word.  Kernels set it, never trap:
+ * KDA_ERR_DEVICE_TIMEOUT when a bounded wait gives up, KDA_ERR_INVALID_ARG
+ * when a cu_seqlens table fails its device-side check (see kda_chunk_fwd).
+ * The first error since the last read is kept.  Synchronises `stream` first.
+ * *code receives 0 when nothing was raised.
  */
 kda_status_t kda_device_error(int* code, cudaStream_t stream);
 

@@ -39,7 +39,7 @@ EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step
             "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step",
             "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait",
             "kda_set_segment_chunks", "kda_segment_chunks", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
-            "kda_set_local_kernel")
+            "kda_set_local_kernel", "kda_chunk_fwd_host", "kda_chunk_fwd_host_buffer_size")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -96,6 +96,10 @@ def load_library():
         lib.kda_chunk_fwd_launches.restype = i32
         lib.kda_profile_events.argtypes = [vp, i32]
         lib.kda_profile_events.restype = i32
+        lib.kda_chunk_fwd_host_buffer_size.argtypes = [i32] * 9
+        lib.kda_chunk_fwd_host_buffer_size.restype = szt
+        lib.kda_chunk_fwd_host.argtypes = [vp] * 9 + [i32] * 7 + [i32, i32, vp, szt, vp, vp, vp]
+        lib.kda_chunk_fwd_host.restype = i32
         lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 9 + [i32] * 7 + [i32, vp]
         lib.kda_chunk_fwd_noalloc.restype = i32
         lib.kda_chunk_bwd_workspace_size.argtypes = [i32] * 6
@@ -142,12 +146,53 @@ def _dtype_code(t):
 
 
 def _need_cuda(*ts):
+    dev = None
     for t in ts:
         if t is not None:
             if not t.is_cuda:
                 raise ValueError("tensors must be on a CUDA device (use chunk_fwd_host for host buffers)")
             if not t.is_contiguous():
                 raise ValueError("tensors must be contiguous")
+            if dev is None:
+                dev = t.device
+            elif t.device != dev:
+                raise ValueError(f"tensors on different devices ({dev} and {t.device})")
+
+
+def _prefill_shapes(fn, q, k, v, g, beta, S0, cu_seqlens, o=None, S_out=None):
+    """Checks every prefill argument's dtype and shape against q's [B,T,H,dk]
+    and v's dv (the C ABI sees only pointers and sizes, so a wrong dtype or
+    shape here would be read past its end on the device), then that all are
+    contiguous CUDA tensors on one device.  Returns (B, T, H, dk, dv,
+    num_seqs, N)."""
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError(f"q, k must be [B,T,H,dk] and v [B,T,H,dv], got {tuple(q.shape)}, {tuple(k.shape)}, "
+                         f"{tuple(v.shape)}")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError(f"q, k, v must share one dtype, got {q.dtype}, {k.dtype}, {v.dtype}")
+    _dtype_code(q)
+    prep = fn == "kda_chunk_fwd_prep"
+    if g.dtype not in ((torch.float32, torch.bfloat16) if prep else (torch.float32,)) or beta.dtype != torch.float32:
+        raise TypeError("g (a) and beta (b) must be float32 (a may be bfloat16)")
+    g_shape = (B, T, H) if fn == "kda_gdn_chunk_fwd" else (B, T, H, dk)
+    if tuple(g.shape) != g_shape or tuple(beta.shape) != (B, T, H):
+        raise ValueError(f"g must be {g_shape} and beta {(B, T, H)}, got {tuple(g.shape)}, {tuple(beta.shape)}")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise TypeError("cu_seqlens must be a 1-D int32 tensor of num_seqs + 1 entries")
+        if B != 1:
+            raise ValueError("packed sequences (cu_seqlens) need B == 1")
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = num_seqs if cu_seqlens is not None else B
+    for name, t in (("S0", S0), ("S_out", S_out)):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != (N, H, dk, dv)):
+            raise ValueError(f"{name} must be float32 {(N, H, dk, dv)}, got {t.dtype} {tuple(t.shape)}")
+    if o is not None and (o.dtype != q.dtype or tuple(o.shape) != (B, T, H, dv)):
+        raise ValueError(f"o must be {q.dtype} {(B, T, H, dv)}, got {o.dtype} {tuple(o.shape)}")
+    _need_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_out)
+    return B, T, H, dk, dv, num_seqs, N
 
 
 def workspace_size(B, T, H, dk, dv, num_seqs=0, chunk_size=64, dtype=torch.bfloat16) -> int:
@@ -185,31 +230,22 @@ def chunk_fwd_prep(q, k, v, a, b, S0=None, cu_seqlens=None, chunk_size=64, outpu
 def _chunk_fwd(fn, q, k, v, g, beta, S0, cu_seqlens, chunk_size, output_final_state, o, S_out,
                workspace):
     lib = load_library()
-    _need_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_out, workspace)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    N = num_seqs if cu_seqlens is not None else B
+    B, T, H, dk, dv, num_seqs, N = _prefill_shapes(fn, q, k, v, g, beta, S0, cu_seqlens, o, S_out)
+    _need_cuda(workspace, q)
     prep = fn == "kda_chunk_fwd_prep"
-    if g.dtype not in ((torch.float32, torch.bfloat16) if prep else (torch.float32,)) or beta.dtype != torch.float32:
-        raise TypeError("g (a) and beta (b) must be float32 (a may be bfloat16)")
-    g_shape = (B, T, H) if fn == "kda_gdn_chunk_fwd" else (B, T, H, dk)
-    if tuple(g.shape) != g_shape or tuple(beta.shape) != (B, T, H):
-        raise ValueError(f"g must be {g_shape} and beta {(B, T, H)}, got {tuple(g.shape)}, {tuple(beta.shape)}")
-    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
-        raise TypeError("cu_seqlens must be int32")
-    if o is None:
-        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
-    if S_out is None and output_final_state:
-        S_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
-    ws_need = workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, q.dtype)
-    if workspace is None and ws_need:
-        workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    gargs = (_ptr(g), _dtype_code(g)) if prep else (_ptr(g),)
-    st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), *gargs, _ptr(beta), _ptr(S0), _ptr(o),
-                          _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
-                          _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(q.device))
+    with torch.cuda.device(q.device):
+        if o is None:
+            o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+        if S_out is None and output_final_state:
+            S_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+        ws_need = workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, q.dtype)
+        if workspace is None and ws_need:
+            workspace = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        gargs = (_ptr(g), _dtype_code(g)) if prep else (_ptr(g),)
+        st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), *gargs, _ptr(beta), _ptr(S0), _ptr(o),
+                              _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
+                              _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(q.device))
     _check(st)
     return o, S_out
 
@@ -217,20 +253,20 @@ def _chunk_fwd(fn, q, k, v, g, beta, S0, cu_seqlens, chunk_size, output_final_st
 def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, chunk_size=64, o=None, S_out=None):
     """chunk_fwd through kda_chunk_fwd_noalloc: no workspace is passed or
     allocated (the library's built-in scratch array is used; o and S_out are
-    allocated here only when not given).  Returns (o, S_out)."""
+    allocated here only when not given).  The arguments are checked exactly as
+    chunk_fwd checks them, and the call runs with q's device current (the
+    library looks up the built-in array of the current device).  Returns
+    (o, S_out)."""
     lib = load_library()
-    _need_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_out)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    N = num_seqs if cu_seqlens is not None else B
-    if o is None:
-        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
-    if S_out is None:
-        S_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
-    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                                   _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
-                                   _dtype_code(q), _stream_handle(q.device))
+    B, T, H, dk, dv, num_seqs, N = _prefill_shapes("kda_chunk_fwd", q, k, v, g, beta, S0, cu_seqlens, o, S_out)
+    with torch.cuda.device(q.device):
+        if o is None:
+            o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+        if S_out is None:
+            S_out = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+        st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                       _ptr(S_out), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, chunk_size,
+                                       _dtype_code(q), _stream_handle(q.device))
     _check(st)
     return o, S_out
 
@@ -307,69 +343,58 @@ def _recurrent_step(fn, q, k, v, g, beta, S, o):
 
 
 class HostPrefill:
-    """chunk_fwd over pinned HOST tensors: each call copies the inputs to the
-    device, runs the prefill and copies o and S_out back into pinned host
-    buffers.  Device buffers are allocated once.
-
-    Without cu_seqlens the batch is processed in `pieces` groups of rows: the
-    host->device copy of group p+1 (own stream) overlaps the prefill of group p
-    (the current stream) and the device->host copy of group p-1 (own stream),
-    so the copy engines of both directions and the kernels run together.  The
-    current stream waits for the last copy back, so synchronising it (as the
-    caller does for a one-group call) covers everything."""
+    """chunk_fwd over HOST tensors through the C ABI's kda_chunk_fwd_host: the
+    library copies the inputs to the device, runs the prefill and copies o and
+    S_out back into host buffers, pipelined over `pieces` groups of batch rows
+    on three streams (host->device copies, the prefill on the current stream,
+    device->host copies).  This class only keeps the device buffer the library
+    asks for, the two copy streams and the pinned output buffers; the current
+    stream waits for the last copy back, so synchronising it covers the call.
+    Host inputs should be pinned (page-locked) for the copies to overlap."""
 
     def __init__(self, like: dict, device="cuda", chunk_size=64, pieces=None):
         self.device = torch.device(device)
         self.chunk_size = chunk_size
-        self.dev = {n: torch.empty_like(t, device=self.device) for n, t in like.items() if t is not None}
         q, v = like["q"], like["v"]
         B, T, H, dk = q.shape
         cu = like.get("cu_seqlens")
-        N = cu.numel() - 1 if cu is not None else B
+        self.num_seqs = 0 if cu is None else cu.numel() - 1
+        N = self.num_seqs if cu is not None else B
+        self.shape = (B, T, H, dk, v.shape[-1])
+        self.dtype = q.dtype
+        self.pieces = max(1, min(B, pieces if pieces else 8))
         self.o_host = torch.empty((B, T, H, v.shape[-1]), dtype=q.dtype, pin_memory=True)
         self.S_host = torch.empty((N, H, dk, v.shape[-1]), dtype=torch.float32, pin_memory=True)
-        self.o_dev = torch.empty_like(self.o_host, device=self.device)
-        self.S_dev = torch.empty_like(self.S_host, device=self.device)
-        num_seqs = 0 if cu is None else N
-        self.pieces = 1 if cu is not None else max(1, min(B, pieces if pieces else 8))
-        rows = -(-B // self.pieces)
-        self.bounds = [(b, min(B, b + rows)) for b in range(0, B, rows)]
-        ws = workspace_size(rows if cu is None else B, T, H, dk, v.shape[-1], num_seqs, chunk_size, q.dtype)
-        self.ws = torch.empty(ws, dtype=torch.uint8, device=self.device) if ws else None
+        lib = load_library()
+        nbytes = int(lib.kda_chunk_fwd_host_buffer_size(B, T, H, dk, v.shape[-1], self.num_seqs, chunk_size,
+                                                         _dtype_code(q), self.pieces))
+        self.buf = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=self.device)
+        self.buf_bytes = nbytes
         self.s_in = torch.cuda.Stream(self.device)
         self.s_out = torch.cuda.Stream(self.device)
 
     def h2d_bytes(self, host: dict) -> int:
-        return int(sum(t.numel() * t.element_size() for n, t in host.items() if t is not None and n in self.dev))
+        names = ("q", "k", "v", "g", "beta", "S0", "cu_seqlens")
+        return int(sum(t.numel() * t.element_size() for n, t in host.items() if t is not None and n in names))
 
     def d2h_bytes(self) -> int:
         return int(self.o_host.numel() * self.o_host.element_size() + self.S_host.numel() * 4)
 
     def __call__(self, host: dict):
-        main = torch.cuda.current_stream(self.device)
-        d = self.dev
-        packed = d.get("cu_seqlens") is not None
-        self.s_in.wait_stream(main)   # earlier work on the buffers is done
-        self.s_out.wait_stream(main)
-        for (b0, b1) in self.bounds:
-            rows = slice(None) if packed else slice(b0, b1)
-            with torch.cuda.stream(self.s_in):
-                for n, t in host.items():
-                    if t is not None and n in d:
-                        if n == "cu_seqlens" or packed:
-                            d[n].copy_(t, non_blocking=True)
-                        else:
-                            d[n][rows].copy_(t[rows], non_blocking=True)
-            main.wait_stream(self.s_in)
-            S0 = d.get("S0")
-            chunk_fwd(d["q"][rows], d["k"][rows], d["v"][rows], d["g"][rows], d["beta"][rows],
-                      None if S0 is None else S0[rows], d.get("cu_seqlens"), self.chunk_size,
-                      o=self.o_dev[rows], S_out=self.S_dev[rows], workspace=self.ws)
-            self.s_out.wait_stream(main)
-            with torch.cuda.stream(self.s_out):
-                self.o_host[rows].copy_(self.o_dev[rows], non_blocking=True)
-                self.S_host[rows].copy_(self.S_dev[rows], non_blocking=True)
-        main.wait_stream(self.s_out)
+        lib = load_library()
+        B, T, H, dk, dv = self.shape
+        for n in ("q", "k", "v", "g", "beta", "S0", "cu_seqlens"):
+            t = host.get(n)
+            if t is not None and (t.is_cuda or not t.is_contiguous()):
+                raise ValueError(f"{n} must be a contiguous host tensor")
+        with torch.cuda.device(self.device):
+            st = lib.kda_chunk_fwd_host(
+                _ptr(host["q"]), _ptr(host["k"]), _ptr(host["v"]), _ptr(host["g"]), _ptr(host["beta"]),
+                _ptr(host.get("S0")), _ptr(self.o_host), _ptr(self.S_host), _ptr(host.get("cu_seqlens")),
+                self.num_seqs, B, T, H, dk, dv, self.chunk_size, _dtype_code(host["q"]), self.pieces,
+                _ptr(self.buf), self.buf_bytes, _stream_handle(self.device),
+                ctypes.c_void_p(self.s_in.cuda_stream), ctypes.c_void_p(self.s_out.cuda_stream))
+        _check(st)
         return self.o_host, self.S_host
 
 

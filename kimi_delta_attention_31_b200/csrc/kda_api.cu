@@ -11,6 +11,7 @@
 #include "kda_chunk_tc.cuh"
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
+#include "kda_host.cuh"
 
 namespace {
 
@@ -341,6 +342,131 @@ kda_status_t kda_recurrent_step_prep(const void* q, const void* k, const void* v
 }
 
 // ---------------------------------------------------------------------------
+// Prefill from host buffers.
+// ---------------------------------------------------------------------------
+namespace {
+// Rows of one pipeline group and the device workspace a group needs (the
+// largest over the group sizes that occur: a smaller group may take another
+// path).
+struct HostPlan {
+  int pieces, rows, last_rows;
+  size_t ws;
+};
+HostPlan host_plan(int B, int T, int H, int dk, int dv, int num_seqs, int chunk_size, kda_dtype_t dtype,
+                   int pieces) {
+  HostPlan p;
+  p.pieces = num_seqs > 0 || B <= 1 ? 1 : std::max(1, std::min(pieces, B));
+  p.rows = num_seqs > 0 ? B : (B + p.pieces - 1) / p.pieces;
+  p.pieces = num_seqs > 0 ? 1 : (B + p.rows - 1) / std::max(p.rows, 1);
+  p.last_rows = B - (p.pieces - 1) * p.rows;
+  p.ws = std::max(kda_chunk_fwd_workspace_size(p.rows, T, H, dk, dv, num_seqs, chunk_size, dtype),
+                  kda_chunk_fwd_workspace_size(p.last_rows, T, H, dk, dv, num_seqs, chunk_size, dtype));
+  return p;
+}
+}  // namespace
+
+size_t kda_chunk_fwd_host_buffer_size(int B, int T, int H, int dk, int dv, int num_seqs, int chunk_size,
+                                      kda_dtype_t dtype, int pieces) {
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || pieces < 1 || !supported_head(dk, dv)) return 0;
+  if (dtype != KDA_BF16 && dtype != KDA_F32) return 0;
+  const int N = num_seqs > 0 ? num_seqs : B;
+  const HostPlan plan = host_plan(B, T, H, dk, dv, num_seqs, chunk_size, dtype, pieces);
+  const size_t esz = dtype == KDA_F32 ? 4 : 2;
+  return kda::host::host_layout(kda::host::host_sizes(B, T, H, dk, dv, N, num_seqs, esz), plan.ws).total;
+}
+
+kda_status_t kda_chunk_fwd_host(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, const float* S0, void* o, float* S_out,
+                                const int32_t* cu_seqlens, int num_seqs, int B, int T, int H, int dk,
+                                int dv, int chunk_size, kda_dtype_t dtype, int pieces,
+                                void* device_buffer, size_t device_buffer_bytes, cudaStream_t compute,
+                                cudaStream_t copy_in, cudaStream_t copy_out) {
+  const char* fn = "kda_chunk_fwd_host";
+  t_err[0] = 0;
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || pieces < 1)
+    return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes B=%d T=%d H=%d num_seqs=%d pieces=%d", fn, B, T, H,
+                num_seqs, pieces);
+  if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, (int)dtype);
+  if (!supported_head(dk, dv))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: dk=%d dv=%d (need dk == dv in {32,64,128})", fn, dk, dv);
+  if (cu_seqlens ? (B != 1 || num_seqs < 1) : num_seqs != 0)
+    return fail(KDA_ERR_INVALID_ARG, "%s: cu_seqlens needs B == 1 and num_seqs >= 1 (num_seqs=0 without)", fn);
+  const int N = cu_seqlens ? num_seqs : B;
+  if (N == 0) return KDA_OK;
+  const long long tokens = (long long)B * T;
+  if (tokens > 0 && (!q || !k || !v || !g || !beta || !o))
+    return fail(KDA_ERR_INVALID_ARG, "%s: null host input/output pointer", fn);
+  if (!device_buffer || (reinterpret_cast<uintptr_t>(device_buffer) & (kda::host::kAlign - 1)))
+    return fail(KDA_ERR_ALIGNMENT, "%s: device_buffer must be a %zu-byte aligned device pointer", fn,
+                kda::host::kAlign);
+  const HostPlan plan = host_plan(B, T, H, dk, dv, num_seqs, chunk_size, dtype, pieces);
+  const size_t esz = dtype == KDA_F32 ? 4 : 2;
+  const kda::host::HostSizes sz = kda::host::host_sizes(B, T, H, dk, dv, N, num_seqs, esz);
+  const kda::host::HostLayout L = kda::host::host_layout(sz, plan.ws);
+  if (device_buffer_bytes < L.total)
+    return fail(KDA_ERR_WORKSPACE, "%s: device_buffer %zu bytes, need %zu (kda_chunk_fwd_host_buffer_size)", fn,
+                device_buffer_bytes, L.total);
+  kda::host::HostEvents* ev = nullptr;
+  cudaError_t e = kda::host::host_events(&ev);
+  if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_host: events");
+  uint8_t* base = static_cast<uint8_t*>(device_buffer);
+  // the inner prefill calls record no profiling events of the caller's
+  cudaEvent_t* saved_ev = t_prof_events;
+  const int saved_cnt = t_prof_count;
+  t_prof_events = nullptr;
+  t_prof_count = 0;
+  kda_status_t st = KDA_OK;
+  auto h2d = [&](size_t off, const void* src, size_t bytes) {
+    if (e == cudaSuccess && bytes) e = cudaMemcpyAsync(base + off, src, bytes, cudaMemcpyHostToDevice, copy_in);
+  };
+  auto d2h = [&](void* dst, size_t off, size_t bytes) {
+    if (e == cudaSuccess && bytes) e = cudaMemcpyAsync(dst, base + off, bytes, cudaMemcpyDeviceToHost, copy_out);
+  };
+  auto cu8 = [](const void* p) { return static_cast<const uint8_t*>(p); };
+  // earlier work on `compute` (which may still use the buffer) comes first
+  if ((e = cudaEventRecord(ev->done, compute)) == cudaSuccess) e = cudaStreamWaitEvent(copy_in, ev->done, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(copy_out, ev->done, 0);
+  h2d(L.cu, cu_seqlens, sz.cu);
+  // per-row strides of every tensor (rows = batch rows; packed: one row)
+  const size_t row_q = sz.q / std::max(B, 1), row_v = sz.v / std::max(B, 1), row_g = sz.g / std::max(B, 1);
+  const size_t row_b = sz.beta / std::max(B, 1), row_s = sz.state / N;
+  for (int p = 0; p < plan.pieces && e == cudaSuccess && st == KDA_OK; ++p) {
+    const int b0 = p * plan.rows, nb = std::min(plan.rows, B - b0);
+    // states: packed inputs have N = num_seqs state rows, all in the one group
+    const int s0r = cu_seqlens ? 0 : b0, ns = cu_seqlens ? N : nb;
+    h2d(L.q + b0 * row_q, cu8(q) + b0 * row_q, nb * row_q);
+    h2d(L.k + b0 * row_q, cu8(k) + b0 * row_q, nb * row_q);
+    h2d(L.v + b0 * row_v, cu8(v) + b0 * row_v, nb * row_v);
+    h2d(L.g + b0 * row_g, cu8(g) + b0 * row_g, nb * row_g);
+    h2d(L.beta + b0 * row_b, cu8(beta) + b0 * row_b, nb * row_b);
+    if (S0) h2d(L.S0 + s0r * row_s, cu8(S0) + s0r * row_s, ns * row_s);
+    if (e == cudaSuccess) e = cudaEventRecord(ev->in, copy_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(compute, ev->in, 0);
+    if (e != cudaSuccess) break;
+    st = kda_chunk_fwd(base + L.q + b0 * row_q, base + L.k + b0 * row_q, base + L.v + b0 * row_v,
+                       reinterpret_cast<const float*>(base + L.g + b0 * row_g),
+                       reinterpret_cast<const float*>(base + L.beta + b0 * row_b),
+                       S0 ? reinterpret_cast<const float*>(base + L.S0 + s0r * row_s) : nullptr,
+                       base + L.o + b0 * row_v,
+                       S_out ? reinterpret_cast<float*>(base + L.S_out + s0r * row_s) : nullptr,
+                       cu_seqlens ? reinterpret_cast<const int32_t*>(base + L.cu) : nullptr, num_seqs, nb, T, H,
+                       dk, dv, chunk_size, dtype, plan.ws ? base + L.ws : nullptr, plan.ws, compute);
+    if (st != KDA_OK) break;
+    if ((e = cudaEventRecord(ev->done, compute)) == cudaSuccess) e = cudaStreamWaitEvent(copy_out, ev->done, 0);
+    d2h(static_cast<uint8_t*>(o) + b0 * row_v, L.o + b0 * row_v, nb * row_v);
+    if (S_out) d2h(reinterpret_cast<uint8_t*>(S_out) + s0r * row_s, L.S_out + s0r * row_s, ns * row_s);
+  }
+  // the caller synchronises `compute` to see everything, the copies back included
+  if (e == cudaSuccess && st == KDA_OK && (e = cudaEventRecord(ev->out, copy_out)) == cudaSuccess)
+    e = cudaStreamWaitEvent(compute, ev->out, 0);
+  t_prof_events = saved_ev;
+  t_prof_count = saved_cnt;
+  if (st != KDA_OK) return st;
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return KDA_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Prefill without any caller-provided workspace.
 //
 // Some callers cannot allocate device memory: a plug-in that receives only
@@ -354,23 +480,62 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[KDA_NOALLOC_SCR
 
 namespace {
 std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[256] = {};  // device address of g_noalloc_scratch, per device ordinal
+// Device address of g_noalloc_scratch, per device ordinal, with the context
+// that was current when it was looked up: the address belongs to the module
+// instance of that context, so a different context on the same ordinal (a
+// non-primary context, or the primary one re-created after cudaDeviceReset)
+// looks it up again.
+struct NoallocEntry {
+  void* ctx;
+  void* ptr;
+};
+NoallocEntry g_noalloc[256] = {};
+
+// cuCtxGetCurrent, fetched once from the driver through the runtime (no link
+// against the driver library).
+typedef int (*CtxGetCurrentFn)(void**);
+CtxGetCurrentFn ctx_get_current() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
 
 // Host code only ever sees a host-side stand-in for g_noalloc_scratch, so the
-// real device address is looked up once per device, with that device current.
+// real device address is looked up with the device current, once per device
+// and context.
 kda_status_t noalloc_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetDevice");
   if (dev < 0 || dev >= 256) return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_noalloc: device %d", dev);
+  void* ctx = nullptr;
+  const CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return fail(KDA_ERR_CUDA, "kda_chunk_fwd_noalloc: cuCtxGetCurrent unavailable");
+  if (get(&ctx) != 0 || !ctx) {
+    // No context current on this thread yet: cudaSetDevice (CUDA 12+) makes the
+    // device's primary context current (the device itself does not change).  A
+    // context the caller made current is never replaced.
+    e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaSetDevice");
+    if (get(&ctx) != 0 || !ctx) return fail(KDA_ERR_CUDA, "kda_chunk_fwd_noalloc: no current CUDA context");
+  }
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocEntry& ent = g_noalloc[dev];
+  if (!ent.ptr || ent.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetSymbolAddress");
-    g_noalloc_ptr[dev] = p;
+    ent.ctx = ctx;
+    ent.ptr = p;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = ent.ptr;
   return KDA_OK;
 }
 }  // namespace

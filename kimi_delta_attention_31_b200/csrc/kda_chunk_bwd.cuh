@@ -117,8 +117,8 @@ __global__ void __launch_bounds__(4 * D)
   const int h = uh % H, n = uh / H;
   const int tid = threadIdx.x, lane = tid & 31;
   const bool packed = cu_seqlens != nullptr;
-  const long long t0 = packed ? (long long)cu_seqlens[n] : (long long)n * T;
-  const long long t1 = packed ? (long long)cu_seqlens[n + 1] : t0 + T;
+  long long t0 = (long long)n * T, t1 = t0 + T;
+  if (packed) checked_seq_range(cu_seqlens, n, T, &t0, &t1);  // T = total tokens when packed
   const int nch = (int)((t1 - t0 + C - 1) / C);
   const int nch_T = (T + C - 1) / C;
   auto row_off = [&](long long t) { return ((size_t)t * H + h) * D; };

@@ -38,8 +38,7 @@ struct SimtCfg {
 __device__ __forceinline__ void seq_bounds(const int32_t* cu_seqlens, int n, int T, long long* t0,
                                            long long* t1) {
   if (cu_seqlens) {
-    *t0 = cu_seqlens[n];
-    *t1 = cu_seqlens[n + 1];
+    checked_seq_range(cu_seqlens, n, T, t0, t1);  // T = total tokens when packed
   } else {
     *t0 = (long long)n * T;
     *t1 = (long long)(n + 1) * T;

@@ -361,7 +361,8 @@ __global__ void __launch_bounds__(256, 2)
                               const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                               int num_seqs, int T, int H, uint32_t num_items, FastDiv fdH, FastDiv fdC,
                               uint8_t* __restrict__ ws, const uint32_t* __restrict__ item_list,
-                              const uint32_t* __restrict__ item_cnt, uint32_t list_cap) {
+                              const uint32_t* __restrict__ item_cnt, uint32_t list_cap,
+                              const int* __restrict__ chunk_total) {
   __shared__ __align__(16) float s_beta[C];
   __shared__ float s_nrm[2][C];  // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
   constexpr bool kPrep = gate_prep(kGate);
@@ -378,6 +379,8 @@ __global__ void __launch_bounds__(256, 2)
   const size_t rs = (size_t)H * D;  // elements between consecutive tokens
   // an empty item list (the usual case): nothing to set up
   if (item_list && item_cnt[blockIdx.x] == 0) return;
+  // packed sequences whose cu_seqlens the chunk-table kernel rejected: no work
+  if (cu_seqlens && chunk_total && *chunk_total < 0) return;
 
   if (warp == 0) {
     ptx::tmem_alloc(&s_tmem, 256);
@@ -873,7 +876,7 @@ __global__ void __launch_bounds__(256, 2)
                              float* __restrict__ S_out, bf16* __restrict__ o,
                              const int32_t* __restrict__ cu_seqlens, int N, int T, int H,
                              int seg_chunks, int pass, float* __restrict__ maps,
-                             const float* __restrict__ seg_init) {
+                             const float* __restrict__ seg_init, const int* __restrict__ chunk_total) {
   __shared__ __align__(8) uint64_t s_full[3];  // image parts: 0 [W; Q e^G], 1 U^T, 2 P + Kbar + gamma
   __shared__ __align__(8) uint64_t s_mma1, s_mma2;
   __shared__ uint32_t s_tmem;
@@ -884,6 +887,9 @@ __global__ void __launch_bounds__(256, 2)
   KDA_ALIGNED_DSMEM(sm, dsm_raw);
   const uint32_t sb = ptx::smem_u32(sm);
 
+  // packed sequences whose cu_seqlens the chunk-table kernel rejected: the
+  // outputs are left untouched
+  if (cu_seqlens && chunk_total && *chunk_total < 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, ch = warp >> 2;
   const int c = 32 * qd + lane;  // state row; rows 0..63 of X are tokens (-E), 64..127 outputs
@@ -939,9 +945,14 @@ __global__ void __launch_bounds__(256, 2)
       if (warp == 0) {
         const long long f = chunks_before_warp(cu_seqlens, n);
         if (lane == 0) {
-          s_u_first = f;
-          s_u_start = cu_seqlens[n];
-          s_u_len = cu_seqlens[n + 1] - cu_seqlens[n];
+          long long t0, t1;
+          checked_seq_range(cu_seqlens, n, T, &t0, &t1);  // T = total tokens when packed
+          // the unit's images must lie inside the workspace (T / C + N chunks)
+          const bool in_ws = f >= 0 && f + (t1 - t0 + C - 1) / C <= (long long)T / C + N;
+          if (!in_ws) raise_device_error(kDevErrBadSeqlens);
+          s_u_first = in_ws ? f : 0;
+          s_u_start = t0;
+          s_u_len = in_ws ? (int)(t1 - t0) : 0;
         }
       }
       __syncthreads();
@@ -1250,20 +1261,27 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   // The warp-specialised kernel takes every layout and gate mode;
   // `local_kernel` == 1 keeps every call on the two-CTA kernel.
   const bool use_ws = items > 0 && local_kernel != 1 && (long long)B * T < (1LL << 31) && ws::ws_kernel_available();
+  const TcWorkspace lay = tc_workspace_layout(max_chunks, H, N * (long long)H, T, seg_chunks);
+  int2* table = reinterpret_cast<int2*>(ws + lay.table);
+  int* chunk_total = reinterpret_cast<int*>(table + max_chunks);
+  if (cu_seqlens) {
+    // validates cu_seqlens (a malformed table: total = -1 and every later kernel
+    // skips its work) and builds the chunk table of packed sequences
+    ws::kda_ws_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, table, chunk_total);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   if (use_ws) {
-    const TcWorkspace lay = tc_workspace_layout(max_chunks, H, N * (long long)H, T, seg_chunks);
-    int2* table = reinterpret_cast<int2*>(ws + lay.table);
     e = ws::launch_ws_local(q, k, v, g, beta, cu_seqlens, num_seqs, B, T, H, items, fdH, fdC, ws,
-                            reinterpret_cast<uint32_t*>(ws + lay.lists), table,
-                            reinterpret_cast<int*>(table + max_chunks), std::min(s_sms, kMaxListCtas), gmode,
-                            stream);
+                            reinterpret_cast<uint32_t*>(ws + lay.lists), table, chunk_total,
+                            std::min(s_sms, kMaxListCtas), gmode, stream);
     if (e != cudaSuccess) return e;
   } else if (items > 0) {
     const int gridA = (int)(items < 2LL * s_sms ? items : 2LL * s_sms);
 #define KDA_TC_LOCAL(M)                                                                            \
   tc::kda_tc_chunk_local_kernel<M><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens, \
                                                                        num_seqs, T, H, (uint32_t)items, fdH, \
-                                                                       fdC, ws, nullptr, nullptr, 0u)
+                                                                       fdC, ws, nullptr, nullptr, 0u, \
+                                                                       cu_seqlens ? chunk_total : nullptr)
     switch (gmode) {
       case kGateLogCh: KDA_TC_LOCAL(kGateLogCh); break;
       case kGateLogTok: KDA_TC_LOCAL(kGateLogTok); break;
@@ -1286,17 +1304,18 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
     const int P = (int)((nc + seg_chunks - 1) / seg_chunks);
     const long long map_items = units * (P - 1) * 2, fin_items = units * P;
     tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(map_items, 2LL * s_sms), 256, tc::KB_DYN, stream>>>(
-        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassMaps, maps, seg_init);
+        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassMaps, maps, seg_init, nullptr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     tc::kda_tc_seg_combine_kernel<<<(unsigned)(units * (tc::D / 8)), 256, 0, stream>>>(maps, S0, seg_init, P);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(fin_items, 2LL * s_sms), 256, tc::KB_DYN, stream>>>(
-        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassFinal, maps, seg_init);
+        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassFinal, maps, seg_init, nullptr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else if (units > 0) {
     const int gridB = (int)(units < 2LL * s_sms ? units : 2LL * s_sms);  // two CTAs per SM
     tc::kda_tc_state_pass_kernel<<<gridB, 256, tc::KB_DYN, stream>>>(ws, S0, S_out, o, cu_seqlens, N, T, H, 0,
-                                                                      tc::kPassPlain, nullptr, nullptr);
+                                                                      tc::kPassPlain, nullptr, nullptr,
+                                                                      cu_seqlens ? chunk_total : nullptr);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

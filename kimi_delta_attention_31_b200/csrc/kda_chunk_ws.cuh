@@ -129,13 +129,26 @@ __device__ __forceinline__ ItemPos item_pos(uint32_t item, int T, int H, const F
 // Chunk table of packed sequences (one CTA of 1024 threads): for every chunk of
 // every sequence in order, {first token, rows}; *total = the number of chunks.
 // A block-wide exclusive scan of the per-sequence chunk counts, 1024 sequences
-// at a time.
+// at a time.  First it checks the table it is given: cu_seqlens[0] == 0,
+// non-decreasing, cu_seqlens[num_seqs] == T (the total tokens).  A table that
+// fails raises the device error word (KDA_ERR_INVALID_ARG) and sets
+// *total = -1, which every later kernel of the call reads as "no work"; with a
+// valid table the chunk count is at most T / C + num_seqs, the table's capacity.
 __global__ void __launch_bounds__(1024)
-    kda_ws_chunk_table_kernel(const int32_t* __restrict__ cu_seqlens, int num_seqs, int2* __restrict__ table,
-                              int* __restrict__ total) {
+    kda_ws_chunk_table_kernel(const int32_t* __restrict__ cu_seqlens, int num_seqs, int T,
+                              int2* __restrict__ table, int* __restrict__ total) {
   __shared__ int s_warp[32];
   __shared__ int s_carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  bool bad = tid == 0 && (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T);
+  for (int i = tid; i < num_seqs; i += 1024) bad |= cu_seqlens[i + 1] < cu_seqlens[i];
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) {
+      raise_device_error(kDevErrBadSeqlens);
+      *total = -1;
+    }
+    return;
+  }
   if (tid == 0) s_carry = 0;
   __syncthreads();
   for (int base = 0; base < num_seqs; base += 1024) {
@@ -677,7 +690,8 @@ template <int kGate>
 inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                      const void* g, const float* beta, const int32_t* cu_seqlens, int num_seqs,
                                      int B, int T, int H, long long items, FastDiv fdH, FastDiv fdC, uint8_t* ws,
-                                     uint32_t* lists, int2* table, int* table_total, int sms, cudaStream_t stream) {
+                                     uint32_t* lists, const int2* table, const int* table_total, int sms,
+                                     cudaStream_t stream) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   cudaError_t e = tensor_map_encoder(&enc);
   if (e != cudaSuccess) return e;
@@ -691,10 +705,6 @@ inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16
   } else {
     if ((e = encode_rows_map(enc, &mg, g, kGate != kGateLogitBf16, tokens, H, D, false)) != cudaSuccess) return e;
   }
-  if (cu_seqlens) {
-    kda_ws_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, table, table_total);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
   const int grid = (int)std::min<long long>(items, sms);
   const uint32_t cap = ws_list_cap(items, grid);
   uint32_t* cnt = lists + (size_t)grid * cap;
@@ -706,14 +716,15 @@ inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16
         mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap, nullptr, nullptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   tc::kda_tc_chunk_local_kernel<kGate><<<grid, 256, tc::KA_DYN, stream>>>(
-      q, k, v, g, beta, cu_seqlens, cu_seqlens ? num_seqs : 0, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap);
+      q, k, v, g, beta, cu_seqlens, cu_seqlens ? num_seqs : 0, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap,
+      cu_seqlens ? table_total : nullptr);
   return cudaGetLastError();
 }
 
 inline cudaError_t launch_ws_local(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                    const void* g, const float* beta, const int32_t* cu_seqlens, int num_seqs, int B,
                                    int T, int H, long long items, FastDiv fdH, FastDiv fdC, uint8_t* ws,
-                                   uint32_t* lists, int2* table, int* table_total, int sms, int gmode,
+                                   uint32_t* lists, const int2* table, const int* table_total, int sms, int gmode,
                                    cudaStream_t stream) {
 #define KDA_WS_CASE(M)                                                                                     \
   case M:                                                                                                  \

@@ -47,9 +47,27 @@ inline int current_sm_count() {
 // up; the host reads and clears it through kda_device_error().
 __device__ int g_device_error;
 
-enum : int { kDevErrNone = 0, kDevErrWaitTimeout = 6 };
+// Codes match kda_status_t: a malformed cu_seqlens table seen on the device
+// (KDA_ERR_INVALID_ARG), a bounded wait that gave up (KDA_ERR_DEVICE_TIMEOUT).
+enum : int { kDevErrNone = 0, kDevErrBadSeqlens = 1, kDevErrWaitTimeout = 6 };
 
 __device__ __forceinline__ void raise_device_error(int code) { atomicCAS(&g_device_error, 0, code); }
+
+// Token range [t0, t1) of packed sequence n, checked: a sequence whose range
+// is not inside [0, total] with t0 <= t1 raises the device error word and is
+// treated as empty (the caller then reads and writes nothing for it).
+__device__ __forceinline__ bool checked_seq_range(const int32_t* cu, int n, long long total, long long* t0,
+                                                  long long* t1) {
+  const long long a = cu[n], b = cu[n + 1];
+  if (a < 0 || b < a || b > total) {
+    raise_device_error(kDevErrBadSeqlens);
+    *t0 = *t1 = 0;
+    return false;
+  }
+  *t0 = a;
+  *t1 = b;
+  return true;
+}
 
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);

@@ -3,12 +3,28 @@
 the max-over-slices relative RMS error."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
 import oracle
 
 TOL = {torch.bfloat16: 1e-2, torch.float32: 1e-4}
+
+
+def record_margin(worst_o, worst_S, tol, units):
+    """Appends the worst errors of one comparison to the JSON-lines file named
+    by the environment variable KDA_PARITY_LOG (when it is set), so that the
+    margin under each tolerance is on record, not only pass or fail."""
+    path = os.environ.get("KDA_PARITY_LOG")
+    if not path:
+        return
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    with open(path, "a") as f:
+        f.write(json.dumps({"test": test, "worst_o": float(worst_o), "worst_S": float(worst_S), "tol": tol,
+                            "units": int(units)}) + "\n")
 
 
 def seq_bounds(inp, n):
@@ -63,6 +79,7 @@ def compare_units_prep(inp, o_gpu, S_gpu, units, tol):
         if t1 > t0:
             worst_o = max(worst_o, rel_rms(o_gpu[b, t0:t1, h].float().cpu().numpy(), o[0, cu[i]:cu[i + 1], 0]))
         worst_S = max(worst_S, rel_rms(S_gpu[n, h].cpu().numpy(), S[i, 0]))
+    record_margin(worst_o, worst_S, tol, len(units))
     assert np.isfinite(worst_o) and np.isfinite(worst_S)
     assert worst_o <= tol, f"o rel-RMS {worst_o:.3e} > {tol}"
     assert worst_S <= tol, f"S rel-RMS {worst_S:.3e} > {tol}"
@@ -90,6 +107,7 @@ def compare_units(inp, o_gpu, S_gpu, units, tol):
             worst_o = max(worst_o, rel_rms(og, o_ref))
         if S_gpu is not None:
             worst_S = max(worst_S, rel_rms(S_gpu[n, h].cpu().numpy(), S_ref))
+    record_margin(worst_o, worst_S, tol, len(units))
     assert np.isfinite(worst_o) and np.isfinite(worst_S)
     assert worst_o <= tol, f"o rel-RMS {worst_o:.3e} > {tol}"
     assert worst_S <= tol, f"S rel-RMS {worst_S:.3e} > {tol}"

@@ -214,3 +214,49 @@ def test_local_kernel_switch():
     assert kda.chunk_fwd_kernel_sequence(1, 300, 4, num_seqs=3)[0] == "kda_ws_chunk_table_kernel"
     with pytest.raises(ValueError):
         kda.uses_ws_kernel("per_head")
+
+
+def test_noalloc_binding_checks_arguments_before_any_launch():
+    """chunk_fwd_noalloc checks dtypes and shapes exactly as chunk_fwd does:
+    the C ABI sees only pointers, so a wrong dtype or shape would otherwise be
+    read past its end on the device.  These fail before any CUDA call."""
+    import torch
+    B, T, H, d = 1, 8, 2, 32
+    q = torch.zeros(B, T, H, d, dtype=torch.bfloat16)
+    g = torch.zeros(B, T, H, d)
+    beta = torch.zeros(B, T, H)
+    for fn in (kda.chunk_fwd, kda.chunk_fwd_noalloc):
+        with pytest.raises(TypeError):
+            fn(q, q, q, g.to(torch.bfloat16), beta)           # bf16 g
+        with pytest.raises(ValueError):
+            fn(q, q, q, g[..., 0].contiguous(), beta)          # g of shape [B,T,H]
+        with pytest.raises(ValueError):
+            fn(q, q, q, g, torch.zeros(B, T, H + 1))           # beta of the wrong shape
+        with pytest.raises(TypeError):
+            fn(q, q, q, g, beta, cu_seqlens=torch.tensor([0, T], dtype=torch.int64))
+        with pytest.raises(ValueError):
+            fn(q, q, q, g, beta)                               # right shapes, host tensors
+
+
+def test_host_entry_point_sizes_and_argument_checks():
+    """kda_chunk_fwd_host: its device buffer holds a copy of every tensor plus
+    the workspace, and bad arguments are refused before any copy is queued."""
+    lib = kda.load_library()
+    B, T, H, d = 4, 96, 2, 64
+    tensors = 2 * B * T * H * d * 4 + B * T * H * d * 4 + B * T * H * d * 4 + B * T * H * 4 + 2 * B * H * d * d * 4
+    size = lib.kda_chunk_fwd_host_buffer_size(B, T, H, d, d, 0, 32, kda.KDA_F32, 2)
+    assert size >= tensors
+    assert lib.kda_chunk_fwd_host_buffer_size(B, T, H, 96, 96, 0, 32, kda.KDA_F32, 2) == 0
+    assert lib.kda_chunk_fwd_host_buffer_size(B, T, H, d, d, 0, 32, kda.KDA_F32, 0) == 0
+    f = _fake()
+
+    def call(dk=d, buf=0x10000, nbytes=None, pieces=2):
+        nb = size if nbytes is None else nbytes
+        return lib.kda_chunk_fwd_host(f, f, f, f, f, None, f, f, None, 0, B, T, H, dk, dk, 32, kda.KDA_F32,
+                                      pieces, ctypes.c_void_p(buf), nb, None, None, None)
+
+    assert call(dk=80) == 2
+    assert call(pieces=0) == 1
+    assert call(buf=0x10010) == 3          # device buffer not 256-byte aligned
+    assert call(nbytes=size - 1) == 4      # too small
+    assert "kda_chunk_fwd_host" in kda.last_error()

@@ -11,7 +11,7 @@ import torch
 import kimi_delta_attention_31_b200 as kda
 import kda_workloads as W
 import oracle
-from parity_util import TOL, compare_units, oracle_units, rel_rms, sample_units
+from parity_util import TOL, compare_units, oracle_units, record_margin, rel_rms, sample_units
 
 pytestmark = pytest.mark.gpu
 
@@ -133,25 +133,28 @@ def test_prefill_h16_full(cuda_device):
 
 
 def test_prefill_b8_sampled(cuda_device):
-    """bf16 B8 H32 T8192 d128 (the benchmark workload, same launch): 12 sampled units."""
+    """bf16 B8 H32 T8192 d128 (the benchmark workload, same launch): 40 seeded
+    units, the first and the last always included."""
     w = W.PREFILL_B8
     inp = W.make_workload(w, cuda_device)
     o, S = _run_prefill(inp, w.chunk)
     torch.cuda.synchronize()
-    units = sample_units(w.B, w.H, 12, seed=11, must=[(0, 0), (w.B - 1, w.H - 1)])
+    units = sample_units(w.B, w.H, 40, seed=11, must=[(0, 0), (w.B - 1, w.H - 1)])
     compare_units(inp, o, S, units, 1e-2)
     assert torch.isfinite(o).all() and torch.isfinite(S).all()
 
 
 def test_prefill_varlen_sampled(cuda_device):
-    """16 packed sequences (~512K tokens), H32: longest, shortest + sampled units."""
+    """16 packed sequences (~512K tokens), H32: the longest and the shortest
+    sequence on four heads each, plus seeded units (40 in all)."""
     w = W.PREFILL_VARLEN
     inp = W.make_workload(w, cuda_device)
     o, S = _run_prefill(inp, w.chunk)
     torch.cuda.synchronize()
     lens = list(w.lengths)
     longest, shortest = int(np.argmax(lens)), int(np.argmin(lens))
-    units = sample_units(w.num_seqs, w.H, 6, seed=12, must=[(longest, 3), (shortest, 17)])
+    must = [(longest, h) for h in (0, 3, 17, 31)] + [(shortest, h) for h in (0, 9, 17, 30)]
+    units = sample_units(w.num_seqs, w.H, 40, seed=12, must=must)
     compare_units(inp, o, S, units, 1e-2)
     assert torch.isfinite(o).all() and torch.isfinite(S).all()
 
@@ -178,35 +181,38 @@ def test_decode_small(cuda_device, dtype, d):
     assert oracle.rel_rms_per_slice(S.cpu().numpy(), rS) <= tol
 
 
-def test_decode_full_sampled(cuda_device):
-    """256 sequences x 32 heads, d128, 1024 in-place steps (the benchmark's decode
-    launch): o at steps 1, 2, 8, 64, 1024 and the final state of sampled units."""
+def test_decode_full_all_units(cuda_device):
+    """256 sequences x 32 heads, d128, 1024 in-place steps (the benchmark's
+    decode launch, same inputs): every one of the 8,192 units, o at steps 1,
+    2, 8, 64 and 1024 and the final state, against the oracle run on the same
+    steps as one prefill per unit (in batches of units, to bound host memory)."""
     w = W.DECODE
     N, H, d, steps = w.B, w.H, w.dk, w.T
     S = W.make_decode_state(N, H, d, d, w.s0_std, seed=w.seed, device=cuda_device)
-    units = sample_units(N, H, 16, seed=13, must=[(0, 0), (N - 1, H - 1)])
-    ui = torch.tensor([n for n, _ in units], device=cuda_device)
-    hi = torch.tensor([h for _, h in units], device=cuda_device)
-    S0_sel = S[ui, hi].cpu()
-    keep_steps = {0, 1, 7, 63, steps - 1}
-    hist = {n: [] for n in ("q", "k", "v", "g", "beta")}
+    S0 = S.clone()
+    xs = W.make_decode_steps(N, H, d, d, steps, w.dtype, w.g_mu, w.g_sigma, seed=w.seed, device=cuda_device)
+    keep_steps = (0, 1, 7, 63, steps - 1)
     o_kept = {}
     for t in range(steps):
-        x = W.make_decode_steps(N, H, d, d, 1, w.dtype, w.g_mu, w.g_sigma, seed=w.seed * 10000 + t,
-                                device=cuda_device)
-        x = {n: v[0] for n, v in x.items()}
-        o = kda.recurrent_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S)
-        for n in hist:
-            hist[n].append(x[n][ui, hi].cpu())
+        o = kda.recurrent_step(xs["q"][t], xs["k"][t], xs["v"][t], xs["g"][t], xs["beta"][t], S)
         if t in keep_steps:
-            o_kept[t] = o[ui, hi].float().cpu()
+            o_kept[t] = o.float().cpu()
     torch.cuda.synchronize()
-    seq = {n: torch.stack(v, 1).unsqueeze(2) for n, v in hist.items()}  # [U, steps, 1, ...]
-    ro, rS = oracle.recurrent(seq["q"], seq["k"], seq["v"], seq["g"], seq["beta"],
-                              S0_sel.unsqueeze(1))
-    for t, og in o_kept.items():
-        assert rel_rms(og.numpy(), ro[:, t, 0]) <= 1e-2, t
-    assert oracle.rel_rms_per_slice(S[ui, hi].cpu().unsqueeze(1).numpy(), rS) <= 1e-2
+    S_gpu = S.cpu()
+    worst_o = worst_S = 0.0
+    batch = 256
+    flat = lambda x: x.reshape(steps, N * H, *x.shape[3:])  # [steps, units, ...]
+    for u0 in range(0, N * H, batch):
+        sel = slice(u0, u0 + batch)
+        seq = {n: flat(xs[n])[:, sel].transpose(0, 1).unsqueeze(2).cpu() for n in ("q", "k", "v", "g", "beta")}
+        S0_b = S0.reshape(N * H, d, d)[sel].unsqueeze(1).cpu()
+        ro, rS = oracle.recurrent(seq["q"], seq["k"], seq["v"], seq["g"], seq["beta"], S0_b)
+        for t in keep_steps:
+            og = o_kept[t].reshape(N * H, d)[sel].numpy()
+            worst_o = max(worst_o, oracle.rel_rms_per_slice(og[:, None, None, :], ro[:, t:t + 1]))
+        worst_S = max(worst_S, oracle.rel_rms_per_slice(S_gpu.reshape(N * H, d, d)[sel].unsqueeze(1).numpy(), rS))
+    record_margin(worst_o, worst_S, 1e-2, N * H)
+    assert worst_o <= 1e-2 and worst_S <= 1e-2, (worst_o, worst_S)
 
 
 def test_decode_equals_prefill(cuda_device):

@@ -1,8 +1,10 @@
 """kda_chunk_fwd_noalloc: the prefill for callers that cannot allocate device
 memory (for example a plug-in handed only input and output pointers by a host
-framework that owns the device memory pool).  It must give the same results
-as kda_chunk_fwd with a caller-allocated workspace, call after call (its
-built-in scratch array is reused), and refuse sizes its array cannot hold.
+framework that owns the device memory pool).  It runs the very same kernels as
+kda_chunk_fwd with a caller-allocated workspace, so its results must be
+bit-for-bit the same, call after call (its built-in scratch array is reused
+and keeps the previous call's contents); it must refuse sizes its array cannot
+hold and check its arguments exactly as chunk_fwd does.
 
 This file is named so that pytest collects it last."""
 import pytest
@@ -10,40 +12,48 @@ import torch
 
 import kimi_delta_attention_31_b200 as kda
 import kda_workloads as W
-from parity_util import rel_rms
 
 pytestmark = pytest.mark.gpu
 
-TOL = 1e-2  # the bf16 tolerance of the parity tests
+
+def _same(x, ref_o, ref_S, o, S):
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
+    assert torch.equal(o, ref_o) and torch.equal(S, ref_S)
 
 
-def _inputs(seed, device):
-    # tensor-core shape (bf16, d=128, C=64), ragged last chunk, random initial state:
-    # 2 x 11 chunks x 8 heads = 176 (chunk, head) images, well inside the built-in array
-    return W.make_prefill(2, 700, 8, 128, 128, "bf16", -4.0, 1.0, 0.02, seed=seed, device=device)
+def _both(x, cu=None, C=64):
+    ref_o, ref_S = kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], cu, C)
+    o, S = kda.chunk_fwd_noalloc(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], cu, C)
+    torch.cuda.synchronize()
+    return ref_o, ref_S, o, S
 
 
 def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
-    for call, seed in enumerate((901, 902)):
-        x = _inputs(seed, cuda_device)
-        ref_o, ref_S = kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], None, 64)
-        o, S = kda.chunk_fwd_noalloc(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], None, 64)
-        torch.cuda.synchronize()
-        assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
-        eo = rel_rms(o.float().cpu().numpy(), ref_o.float().cpu().numpy())
-        eS = rel_rms(S.cpu().numpy(), ref_S.cpu().numpy())
-        assert eo <= TOL and eS <= TOL, f"call {call}: o {eo:.3e}, S {eS:.3e}"
+    # tensor-core shape (bf16, d=128, C=64), ragged last chunk, random initial state
+    for seed in (901, 902):
+        x = W.make_prefill(2, 700, 8, 128, 128, "bf16", -4.0, 1.0, 0.02, seed=seed, device=cuda_device)
+        _same(x, *_both(x))
 
 
 def test_noalloc_packed_sequences(cuda_device):
     lens = (64, 1, 130, 0, 77)
     x = W.make_prefill(1, sum(lens), 4, 128, 128, "bf16", -4.0, 1.0, 0.02, seed=903, device=cuda_device,
                        lengths=lens)
-    ref_o, ref_S = kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], 64)
-    o, S = kda.chunk_fwd_noalloc(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], 64)
-    torch.cuda.synchronize()
-    assert rel_rms(o.float().cpu().numpy(), ref_o.float().cpu().numpy()) <= TOL
-    assert rel_rms(S.cpu().numpy(), ref_S.cpu().numpy()) <= TOL
+    _same(x, *_both(x, x["cu_seqlens"]))
+
+
+def test_noalloc_at_its_documented_limit(cuda_device):
+    # B=1, H=8, T=7168: 112 chunks x 8 heads, the largest case named in kda.h
+    need = kda.workspace_size(1, 7168, 8, 128, 128, 0, 64, torch.bfloat16)
+    assert 0 < need <= kda.NOALLOC_SCRATCH_BYTES
+    x = W.make_prefill(1, 7168, 8, 128, 128, "bf16", -4.0, 1.0, 0.02, seed=905, device=cuda_device)
+    _same(x, *_both(x))
+
+
+def test_noalloc_fp32_path_needs_no_scratch(cuda_device):
+    assert kda.workspace_size(2, 100, 3, 64, 64, 0, 32, torch.float32) == 0
+    x = W.make_prefill(2, 100, 3, 64, 64, "f32", -3.0, 1.0, 0.05, seed=906, device=cuda_device)
+    _same(x, *_both(x, None, 32))
 
 
 def test_noalloc_rejects_sizes_beyond_its_array(cuda_device):
