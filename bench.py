@@ -319,7 +319,7 @@ def gdn_leg(kda, args, world, dev, stream, peaks):
     barrier(world)
     ms = max_over_ranks(time_launches(prefill, args.steps, stream), world, dev)
     kernel_ms = kda.profile_chunk_fwd(prefill, stream, repeats=max(1, min(args.steps, 5)), dk=dk, dv=dv,
-                                      chunk_size=w.chunk, gate="log_token")
+                                      chunk_size=w.chunk, gate="log_token", shape=(B, T, H, 0))
     token_heads = B * T * H
     dom_name, dom_ms = max(kernel_ms.items(), key=lambda kv: kv[1])
     alg_bytes = token_heads * GDN_PREFILL_BYTES_PER_TOKEN_HEAD + B * H * STATE_BYTES
@@ -397,7 +397,7 @@ def prep_leg(kda, args, world, dev, stream, peaks):
     ms = max_over_ranks(time_launches(fused, args.steps, stream), world, dev)
     ms_unfused = max_over_ranks(time_launches(unfused, max(1, min(args.steps, 3)), stream), world, dev)
     kernel_ms = kda.profile_chunk_fwd(fused, stream, repeats=max(1, min(args.steps, 5)), dk=dk, dv=dv,
-                                      chunk_size=w.chunk, gate="logit")
+                                      chunk_size=w.chunk, gate="logit", shape=(B, T, H, 0))
     token_heads = B * T * H
     dom_name, dom_ms = max(kernel_ms.items(), key=lambda kv: kv[1])
     # q, k, v, o bf16 + bf16 gate logits + fp32 beta logit per token-head, + the final state
@@ -554,7 +554,8 @@ def prefill_leg(kda, w, args, world, dev, stream, peaks, peak_src, sample_clocks
     try:
         ms = time_launches(call, args.steps, stream)
         kernel_ms = kda.profile_chunk_fwd(call, stream, repeats=max(1, min(args.steps, 5)), dk=dk, dv=dv,
-                                          chunk_size=w.chunk, dtype=tdt, packed=cu is not None)
+                                          chunk_size=w.chunk, dtype=tdt, packed=cu is not None,
+                                          shape=(B, T, H, num_seqs))
     finally:
         if clk:
             clk.__exit__(None, None, None)
@@ -567,6 +568,28 @@ def prefill_leg(kda, w, args, world, dev, stream, peaks, peak_src, sample_clocks
             "roofline": prefill_roofline(kda, w, ms, kernel_ms, peaks, peak_src, inp["S0"] is not None)}
     if clk:
         line["clocks"] = clk.summary()
+    if tdt == torch.bfloat16 and dk == 128:
+        # the same calls on the other tensor-core path, for comparison
+        other = kda.PATH_TWO_KERNEL if kda.uses_fused_kernel(B, T, H, num_seqs) else kda.PATH_FUSED
+        kda.set_prefill_path(other)
+        try:
+            ws2 = torch.empty(max(kda.workspace_size(B, T, H, dk, dv, num_seqs, w.chunk, tdt), 1),
+                              dtype=torch.uint8, device=dev)
+
+            def call2():
+                kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], cu, w.chunk,
+                              o=o, S_out=S_out, workspace=ws2)
+
+            for _ in range(args.warmup):
+                call2()
+            torch.cuda.synchronize()
+            barrier(world)
+            ms2 = max_over_ranks(time_launches(call2, max(1, min(args.steps, 5)), stream), world, dev)
+            line["other_path"] = {"path": "two kernels" if other == kda.PATH_TWO_KERNEL else "single pass",
+                                  "ms_per_step": ms2, "value": world * w.tokens / (ms2 * 1e-3)}
+            del ws2
+        finally:
+            kda.set_prefill_path(kda.PATH_AUTO)
     del inp, o, S_out, ws
     torch.cuda.empty_cache()
     if cpu and world == 1 and not args.no_cpu_baseline:

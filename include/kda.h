@@ -334,13 +334,40 @@ int kda_segment_chunks(int B, int T, int H, int num_seqs);
 kda_status_t kda_set_local_kernel(int variant);
 
 /*
- * Number of phases one kda_chunk_fwd call with these arguments runs: 1 for
- * the fp32-arithmetic path (one kernel); 2 for the tensor-core path (the
- * chunk-local phase -- one kernel, or two when the warp-specialised kernel
- * runs and hands its steep chunks to the two-CTA kernel, see
- * kda_set_local_kernel -- then the state pass -- one kernel, or three when the
- * sequences are split into segments).  kda_profile_events records one event
- * before the call and one after each phase.
+ * Which tensor-core prefill runs (bf16, dk == dv == 128, chunk 64), for the
+ * calling thread's later calls (kda_chunk_fwd, kda_gdn_chunk_fwd,
+ * kda_chunk_fwd_prep, their workspace sizes and kda_chunk_fwd_phases).  Both
+ * compute the chunked form of "Deriving Kimi Delta Attention from scratch"
+ * section 6:
+ *   1 = single pass: one persistent kernel, one CTA per SM, each CTA taking
+ *       whole (sequence, head) units (packed sequences longest first) and
+ *       carrying the state from chunk to chunk in tensor memory; nothing of a
+ *       chunk goes to HBM but its outputs; its workspace is a few hundred bytes;
+ *   2 = two kernels: every chunk's operands built in parallel into a per-chunk
+ *       workspace image, then a state pass over the chunks of each unit (the
+ *       path that also splits long sequences into segments);
+ *   0 = automatic (default): the single pass unless the sequences are split
+ *       into segments (see kda_set_segment_chunks), then the two kernels.
+ * Other values: KDA_ERR_INVALID_ARG, setting unchanged.
+ */
+kda_status_t kda_set_prefill_path(int path);
+
+/*
+ * Phases of one kda_chunk_fwd call with these sizes on the current device and
+ * the calling thread's settings: 1 for the fp32-arithmetic path and for the
+ * single-pass tensor-core prefill, 2 for the two-kernel one (the chunk-local
+ * phase, then the state pass).  kda_profile_events records one event before
+ * the call and one after each phase.
+ */
+int kda_chunk_fwd_phases(int B, int T, int H, int num_seqs, int dk, int dv, int chunk_size, kda_dtype_t dtype);
+
+/*
+ * Largest number of phases any kda_chunk_fwd call with these head and chunk
+ * sizes can run: 1 for the fp32-arithmetic path (one kernel); 2 for the
+ * tensor-core path, whose two-kernel form runs the chunk-local phase (one
+ * kernel, or two when the warp-specialised kernel hands its steep chunks to
+ * the two-CTA kernel, see kda_set_local_kernel) and then the state pass (one
+ * kernel, or three when the sequences are split into segments).
  */
 int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype);
 
@@ -349,7 +376,8 @@ int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype);
  * kda_gdn_chunk_fwd or kda_chunk_fwd_prep call made by the calling thread
  * records events[0] before its first kernel launch and events[i] after its
  * i-th phase, on the call's stream; count must be at least
- * kda_chunk_fwd_launches(...) + 1 or the call fails with KDA_ERR_INVALID_ARG.
+ * kda_chunk_fwd_phases(...) + 1 for the call's sizes (kda_chunk_fwd_launches(...) + 1
+ * always suffices) or the call fails with KDA_ERR_INVALID_ARG.
  * The caller owns the events.  Pass NULL, 0 to stop.
  */
 kda_status_t kda_profile_events(cudaEvent_t* events, int count);

@@ -39,14 +39,17 @@ EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step
             "kda_version", "kda_chunk_fwd_noalloc", "kda_gdn_chunk_fwd", "kda_gdn_recurrent_step",
             "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait",
             "kda_set_segment_chunks", "kda_segment_chunks", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
-            "kda_set_local_kernel", "kda_chunk_fwd_host", "kda_chunk_fwd_host_buffer_size")
+            "kda_set_local_kernel", "kda_chunk_fwd_host", "kda_chunk_fwd_host_buffer_size",
+            "kda_set_prefill_path", "kda_chunk_fwd_phases")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
 KERNELS_SIMT = ("kda_chunk_simt_kernel",)
 KERNELS_TC = ("kda_tc_chunk_local_kernel", "kda_tc_state_pass_kernel")
 KERNEL_WS = "kda_ws_chunk_local_kernel"
-_tls = threading.local()  # mirrors kda_set_local_kernel, which is per host thread
+KERNEL_FUSED = "kda_fused_prefill_kernel"
+PATH_AUTO, PATH_FUSED, PATH_TWO_KERNEL = 0, 1, 2
+_tls = threading.local()  # mirrors kda_set_local_kernel / kda_set_prefill_path, which are per host thread
 
 
 class KDAError(RuntimeError):
@@ -112,6 +115,10 @@ def load_library():
         lib.kda_segment_chunks.restype = i32
         lib.kda_set_local_kernel.argtypes = [i32]
         lib.kda_set_local_kernel.restype = i32
+        lib.kda_set_prefill_path.argtypes = [i32]
+        lib.kda_set_prefill_path.restype = i32
+        lib.kda_chunk_fwd_phases.argtypes = [i32] * 8
+        lib.kda_chunk_fwd_phases.restype = i32
         lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, vp]
         lib.kda_selftest_bounded_wait.restype = i32
         lib.kda_version.argtypes = []
@@ -428,6 +435,28 @@ def set_local_kernel(variant: int) -> None:
     _tls.local_kernel = int(variant)
 
 
+def set_prefill_path(path: int) -> None:
+    """Tensor-core prefill for this thread's later calls: 0 = automatic
+    (default), 1 = the single-pass kernel, 2 = the two-kernel path."""
+    _check(load_library().kda_set_prefill_path(int(path)))
+    _tls.prefill_path = int(path)
+
+
+def prefill_phases(B, T, H, num_seqs=0, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16) -> int:
+    """Phases of one chunk_fwd call with these sizes on the current device and
+    this thread's settings (1: one kernel does the work; 2: chunk-local phase
+    and state pass)."""
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(load_library().kda_chunk_fwd_phases(B, T, H, num_seqs, dk, dv, chunk_size, code))
+
+
+def uses_fused_kernel(B, T, H, num_seqs=0, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16) -> bool:
+    """Whether a prefill call of these sizes on this thread runs the
+    single-pass kernel."""
+    return (launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 2
+            and prefill_phases(B, T, H, num_seqs, dk, dv, chunk_size, dtype) == 1)
+
+
 def uses_ws_kernel(gate="log_channel", packed=False, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16) -> bool:
     """Whether a prefill call of this kind on this thread runs the
     warp-specialised chunk-local kernel: tensor-core path, any layout (packed
@@ -457,13 +486,17 @@ def launches_per_chunk_fwd(dk, dv, chunk_size, dtype=torch.bfloat16) -> int:
     return int(load_library().kda_chunk_fwd_launches(dk, dv, chunk_size, code))
 
 
-def kernel_names(dk, dv, chunk_size, dtype=torch.bfloat16, gate="log_channel", packed=False):
+def kernel_names(dk, dv, chunk_size, dtype=torch.bfloat16, gate="log_channel", packed=False, shape=None):
     """Phases of one chunk_fwd call, named by the kernel that does each one's
-    work (the chunk-local phase of the warp-specialised path also launches the
+    work.  ``shape`` = (B, T, H, num_seqs) selects the path those sizes take
+    (single pass or two kernels); without it the two-kernel names are given
+    (the chunk-local phase of the warp-specialised path also launches the
     two-CTA kernel over the chunks it passed on, usually none)."""
     n = launches_per_chunk_fwd(dk, dv, chunk_size, dtype)
     if n == 1:
         return KERNELS_SIMT
+    if shape is not None and uses_fused_kernel(*shape, dk=dk, dv=dv, chunk_size=chunk_size, dtype=dtype):
+        return (KERNEL_FUSED,)
     first = KERNEL_WS if uses_ws_kernel(gate, packed, dk, dv, chunk_size, dtype) else KERNELS_TC[0]
     return (first,) + KERNELS_TC[1:n]
 
@@ -473,21 +506,25 @@ def chunk_fwd_kernel_sequence(B, T, H, dk=128, dv=128, chunk_size=64, dtype=torc
     """Every kernel one chunk_fwd call launches, in order."""
     if launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 1:
         return list(KERNELS_SIMT)
+    if uses_fused_kernel(B, T, H, num_seqs, dk, dv, chunk_size, dtype):
+        return ["kda_fused_setup_kernel", KERNEL_FUSED]
+    seq = ["kda_ws_chunk_table_kernel"] if num_seqs > 0 else []
     if uses_ws_kernel(gate, num_seqs > 0, dk, dv, chunk_size, dtype):
-        seq = (["kda_ws_chunk_table_kernel"] if num_seqs > 0 else []) + [KERNEL_WS, KERNELS_TC[0]]
+        seq += [KERNEL_WS, KERNELS_TC[0]]
     else:
-        seq = [KERNELS_TC[0]]
+        seq += [KERNELS_TC[0]]
     if segment_chunks(B, T, H, num_seqs) > 0:
         return seq + [KERNELS_TC[1], "kda_tc_seg_combine_kernel", KERNELS_TC[1]]
     return seq + [KERNELS_TC[1]]
 
 
 def profile_chunk_fwd(call, stream, repeats=3, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16,
-                      gate="log_channel", packed=False):
+                      gate="log_channel", packed=False, shape=None):
     """Run ``call()`` (one chunk_fwd call) ``repeats`` times with the library's
-    event hook set and return {phase's kernel name: mean ms per call}."""
+    event hook set and return {phase's kernel name: mean ms per call}.
+    ``shape`` = (B, T, H, num_seqs) of the call (selects its path)."""
     lib = load_library()
-    names = kernel_names(dk, dv, chunk_size, dtype, gate, packed)
+    names = kernel_names(dk, dv, chunk_size, dtype, gate, packed, shape)
     n = len(names)
     events = [torch.cuda.Event(enable_timing=True) for _ in range((n + 1) * repeats)]
     for e in events:  # torch creates the underlying event lazily, at its first record
@@ -524,6 +561,8 @@ def algorithmic_bytes_per_launch(kernel, token_heads, units, d=128, with_state_i
     gate = gate_bytes * d if gate_per_channel else gate_bytes
     if kernel == "kda_chunk_simt_kernel":
         return token_heads * (3 * 2 * d + gate + 4 + 2 * d) + state * (2 if with_state_in else 1)
+    if kernel == KERNEL_FUSED:
+        return token_heads * (3 * 2 * d + gate + 4 + 2 * d) + state * (2 if with_state_in else 1)
     if kernel in ("kda_tc_chunk_local_kernel", KERNEL_WS):
         return token_heads * (3 * 2 * d + gate + 4 + TC_IMAGE_BYTES_PER_TOKEN_HEAD)
     if kernel == "kda_tc_state_pass_kernel":
@@ -537,5 +576,6 @@ def version() -> int:
 
 __all__ = ["chunk_fwd", "chunk_fwd_noalloc", "recurrent_step", "chunk_fwd_host", "HostPrefill", "workspace_size",
            "launches_per_chunk_fwd", "kernel_names", "profile_chunk_fwd", "algorithmic_bytes_per_launch",
-           "set_local_kernel", "uses_ws_kernel", "chunk_fwd_kernel_sequence",
+           "set_local_kernel", "uses_ws_kernel", "chunk_fwd_kernel_sequence", "set_prefill_path",
+           "prefill_phases", "uses_fused_kernel",
            "last_error", "device_error", "version", "load_library", "lib_path", "KDAError", "EXPORTED"]

@@ -20,6 +20,7 @@ thread_local cudaEvent_t* t_prof_events = nullptr;
 thread_local int t_prof_count = 0;
 thread_local int t_seg_force = 0;  // kda_set_segment_chunks: 0 auto, > 0 fixed, < 0 never
 thread_local int t_local_kernel = 0;  // kda_set_local_kernel: 0 default, 1 two-CTA kernel only
+thread_local int t_prefill_path = 0;  // kda_set_prefill_path: 0 automatic, 1 single pass, 2 two kernels
 
 int current_sms() { return kda::current_sm_count(); }
 
@@ -47,6 +48,23 @@ bool use_tensor_core_path(int dk, int dv, int chunk_size, kda_dtype_t dt) {
 long long max_chunks(int B, int T, int num_seqs, int chunk_size) {
   if (num_seqs > 0) return (long long)T / chunk_size + num_seqs;
   return (long long)B * ((T + chunk_size - 1) / chunk_size);
+}
+
+// The tensor-core prefill's choices for these sizes on the current device and
+// this thread's settings: sequence segments (two-kernel path only) and the path.
+struct TcPlan {
+  int seg;
+  bool fused;
+};
+TcPlan tc_plan(int B, int T, int H, int num_seqs) {
+  const int sms = current_sms();
+  TcPlan p;
+  p.seg = kda::tc_segment_chunks(B, T, H, num_seqs, sms, t_seg_force);
+  p.fused = kda::tc_use_fused(B, T, H, num_seqs, sms, t_prefill_path == kda::kPathFused ? 0 : p.seg,
+                              t_prefill_path) &&
+            kda::fu::fused_kernel_available();
+  if (p.fused) p.seg = 0;
+  return p;
 }
 
 template <typename TIn>
@@ -116,25 +134,34 @@ kda_status_t chunk_fwd_impl(const char* fn, const void* q, const void* k, const 
   if (S_out && o && (const void*)S_out == (const void*)o)
     return fail(KDA_ERR_INVALID_ARG, "%s: o aliases S_out", fn);
 
-  const int launches = kda_chunk_fwd_launches(dk, dv, chunk_size, dtype);
+  const bool tc_path = use_tensor_core_path(dk, dv, chunk_size, dtype);
+  const TcPlan plan = tc_path ? tc_plan(B, T, H, num_seqs) : TcPlan{0, false};
+  const int launches = !tc_path ? 1 : plan.fused ? 1 : kda::kTcLaunches;
   cudaEvent_t* ev = t_prof_events;
   if (ev && t_prof_count < launches + 1)
     return fail(KDA_ERR_INVALID_ARG, "%s: %d profiling events, need %d", fn, t_prof_count,
                 launches + 1);
   cudaError_t e;
   if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return cuda_fail(e, "event record");
-  if (use_tensor_core_path(dk, dv, chunk_size, dtype)) {
+  if (tc_path) {
     const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
     if (need && (!workspace || workspace_bytes < need))
       return fail(KDA_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes,
                   need);
-    const int seg = kda::tc_segment_chunks(B, T, H, num_seqs, current_sms(), t_seg_force);
-    e = kda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
-                             static_cast<const __nv_bfloat16*>(k),
-                             static_cast<const __nv_bfloat16*>(v), g, beta, S0,
-                             static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H,
-                             max_chunks(B, T, num_seqs, chunk_size), workspace, gmode, seg,
-                             t_local_kernel, ev, stream);
+    if (plan.fused) {
+      e = kda::fu::launch_fused(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                static_cast<const __nv_bfloat16*>(v), g, beta, S0,
+                                static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H, workspace,
+                                current_sms(), gmode, stream);
+      if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], stream);
+    } else {
+      e = kda::launch_chunk_tc(static_cast<const __nv_bfloat16*>(q),
+                               static_cast<const __nv_bfloat16*>(k),
+                               static_cast<const __nv_bfloat16*>(v), g, beta, S0,
+                               static_cast<__nv_bfloat16*>(o), S_out, cu_seqlens, N, B, T, H,
+                               max_chunks(B, T, num_seqs, chunk_size), workspace, gmode, plan.seg,
+                               t_local_kernel, ev, stream);
+    }
   } else if (dtype == KDA_F32) {
     e = dispatch_chunk_simt<float>(dk, chunk_size, q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, T,
                                    H, dv, gmode, stream);
@@ -260,7 +287,20 @@ kda_status_t kda_set_segment_chunks(int chunks) {
 }
 
 int kda_segment_chunks(int B, int T, int H, int num_seqs) {
-  return kda::tc_segment_chunks(B, T, H, num_seqs, current_sms(), t_seg_force);
+  return tc_plan(B, T, H, num_seqs).seg;
+}
+
+kda_status_t kda_set_prefill_path(int path) {
+  t_err[0] = 0;
+  if (path != kda::kPathAuto && path != kda::kPathFused && path != kda::kPathTwoKernel)
+    return fail(KDA_ERR_INVALID_ARG, "kda_set_prefill_path: path %d", path);
+  t_prefill_path = path;
+  return KDA_OK;
+}
+
+int kda_chunk_fwd_phases(int B, int T, int H, int num_seqs, int dk, int dv, int chunk_size, kda_dtype_t dtype) {
+  if (!use_tensor_core_path(dk, dv, chunk_size, dtype)) return 1;
+  return tc_plan(B, T, H, num_seqs).fused ? 1 : kda::kTcLaunches;
 }
 
 kda_status_t kda_set_local_kernel(int variant) {
@@ -283,8 +323,9 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
   if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || chunk_size <= 0) return 0;
   if (!use_tensor_core_path(dk, dv, chunk_size, dtype)) return 0;
   const int N = num_seqs > 0 ? num_seqs : B;
-  const int seg = kda::tc_segment_chunks(B, T, H, num_seqs, current_sms(), t_seg_force);
-  return kda::tc_workspace_layout(max_chunks(B, T, num_seqs, chunk_size), H, (long long)N * H, T, seg).total;
+  const TcPlan plan = tc_plan(B, T, H, num_seqs);
+  if (plan.fused) return kda::fu::fused_workspace_bytes(num_seqs);
+  return kda::tc_workspace_layout(max_chunks(B, T, num_seqs, chunk_size), H, (long long)N * H, T, plan.seg).total;
 }
 
 kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,

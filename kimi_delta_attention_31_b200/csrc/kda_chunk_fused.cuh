@@ -1,0 +1,1002 @@
+// kda_chunk_fused.cuh -- single-pass tensor-core prefill (bf16 q, k, v;
+// dk = dv = 128; C = 64): the chunk-local work and the state hand-off of
+// every chunk in one persistent kernel, with the carried state kept on chip
+// ("Deriving Kimi Delta Attention from scratch", section 6, chunked mode;
+// "Linear / sparse attention" tutorial, section 6.2: per chunk an intra term,
+// an inter term through the state, and the state handed to the next chunk).
+//
+// Within a chunk entering with state S (fp32, dk x dv), chunk-relative
+// cumulative log-decays G (fp32) and T = (I + A)^{-1} as in kda_chunk_tc.cuh,
+// the kernel evaluates
+//   R = V - (K o e^G) S,           E = T diag(beta) R             (= U - W S)
+//   O = (Q o e^G) S + P E,          S <- (S + (K o e^-G)^T E) o e^{G_last}
+// (the last line is Diag(e^{G_last}) S + (K o e^{G_last - G})^T E with the
+// decay applied after the sum; chunks whose decay leaves that range use
+// Kbar = K o e^{G_last - G} and decay first).  Nothing of a chunk goes to HBM
+// except o, and the final state per (sequence, head) unit.
+//
+// One CTA per SM (640 threads, ~223 KB of shared memory, all 512 TMEM
+// columns).  CTAs take whole units from a counter in the workspace (packed
+// sequences longest first) and walk their chunks in order; three warp groups
+// work on consecutive chunks at once:
+//   builder (warps 0..7)   chunk n+2: cumulative log-decays, the decay-scaled
+//                          operands [K e^G; Q e^G] (written over the raw k, q
+//                          rows in place) and K e^-G, the [A'; P'] MMA.
+//   solver  (warps 8..15)  chunk n+1: A and P out of TMEM, T = (I + A)^{-1},
+//                          T diag(beta) in bf16.
+//   state   (warps 16..19) chunk n: the state in TMEM, TRANSPOSED (lane = value
+//                          channel), so that every state-side product is an MMA
+//                          whose A operand sits in TMEM:
+//       X^T   = S^T [K e^G; Q e^G]^T          (M=128, N=128, K=128)
+//       R^T   = V^T - X^T[:, 0:64]            (threads, fp32 -> bf16 hi + lo)
+//       E^T   = R^T (T diag(beta))^T          (N=64, K=64, hi and lo)
+//       S^T  += E^T (K e^-G),  X^T[:, 64:128] += E^T P^T  (hi and lo)
+//       S^T  *= e^{G_last} per key channel;  o = X^T[:, 64:128]
+// R and E enter the MMAs as a bf16 pair hi + lo (lo = the rounding error of
+// hi), so their fp32 values are used to about 2^-16; S enters in bf16.
+//
+// TMEM columns: [A'; P'] slot 0 (0..63) | slot 1 (64..127) | X^T (128..255:
+// (K e^G S)^T in 128..191, where E^T lands next, and (Q e^G S)^T -> O^T in
+// 192..255) | bf16 hi | lo of R^T, then of E^T (256..319) | S^T bf16
+// (320..383) | S^T fp32 (384..511).
+//
+// Hand-offs (mbarriers; slot = chunk index mod 2):
+//   g_full        TMA of the raw gate rows (issued by builder thread 0 for the
+//                 next chunk once the group has read the current one)
+//   kqv_full[s]   TMA of k, q (128-byte swizzled, straight into the operand
+//                 panels) and V; issued by the state thread for chunk n+2 as
+//                 soon as chunk n's X^T MMA has read the panels and R^T is
+//                 formed; waited by the builder (k, q) and the state (V)
+//   a_done[s]     [A'; P'] MMA complete + builder arrive        -> solver
+//   s_ready[s]    solver done (P, T diag(beta) in shared memory)  -> state,
+//                 and -> builder (TMEM slot free for chunk n+2)
+//   rb_free[s]    state done with chunk n (MMAs read K e^-G, P; gamma read)
+//                 -> builder (K e^-G, gamma of chunk n+2), solver (P of n+2)
+//   e_done        the E MMA of the previous chunk done -> solver may rewrite
+//                 T diag(beta)
+//   m1, m3, st    MMA completions inside one group.
+// Chunk descriptors travel in an 8-entry ring written by builder thread 0
+// three chunks ahead.  Every wait is bounded; after a timeout every group
+// leaves its loop, the copies still in flight are waited for (bounded), TMEM
+// is freed and the kernel returns with the device error word set.
+//
+// Included by kda_chunk_tc.cuh after the warp-specialised kernel (it uses
+// the tensor-map helpers and the shared solve).
+#pragma once
+
+namespace kda {
+namespace fu {
+
+using tc::bf16;
+using tc::C;
+using tc::D;
+using ws::wait_or_abort;
+
+// ---------------------------------------------------------- shared memory
+constexpr uint32_t FU_L3 = 0;          // 2 slots x 32768: [K e^G; Q e^G] K-major, 2 panels [128 rows][128 B]
+constexpr uint32_t FU_L3_SLOT = 32768;
+constexpr uint32_t FU_RB = 65536;      // 2 slots x 16384: K e^-G (or Kbar) K-major, 2 panels [64 rows][128 B]
+constexpr uint32_t FU_V = 98304;       // 2 slots x 16384: V [64 tokens][128 dv] bf16 row-major
+constexpr uint32_t FU_P = 131072;      // 2 slots x 8192: P bf16 K-major [64 r][64 j]
+constexpr uint32_t FU_RAWG = 147456;   // raw gate rows [64][128] fp32 (bf16 logits: 16 KB); then the
+                                       // group's warp totals [8][128] fp32; steep chunks: left operand
+constexpr uint32_t FU_AS = 180224;     // A fp32 [64][68]
+constexpr uint32_t FU_TS = 197632;     // T fp32 [64][68]; after the solve the lo part of T diag(beta)
+constexpr uint32_t FU_TT = 215040;     // T diag(beta) bf16 (hi) K-major [64][64]; block products during the solve
+constexpr uint32_t FU_GAM = 223232;    // 2 slots x 512: gamma = e^{G_last} fp32 [128]
+constexpr uint32_t FU_BYTES = 224256;
+constexpr uint32_t FU_DYN = FU_BYTES + 1024;
+static_assert(FU_L3 + 2 * FU_L3_SLOT == FU_RB && FU_RB + 2 * 16384 == FU_V && FU_V + 2 * 16384 == FU_P &&
+                  FU_P + 2 * 8192 == FU_RAWG && FU_RAWG + 32768 == FU_AS && FU_AS + 17408 == FU_TS &&
+                  FU_TS + 17408 == FU_TT && FU_TT + 8192 == FU_GAM && FU_GAM + 1024 == FU_BYTES,
+              "layout");
+static_assert(FU_RB % 1024 == 0 && FU_P % 1024 == 0 && FU_RAWG % 1024 == 0 && FU_TT % 1024 == 0, "alignment");
+static_assert(3 * 16 * tc::MT_LD * 4 <= 8192 && 8 * D * 4 <= 32768, "scratch sizes");
+
+// ------------------------------------------------------------------ TMEM
+constexpr uint32_t kTmCols = 512;
+constexpr uint32_t kTmX = 128;   // X^T = S^T [K e^G; Q e^G]^T; E^T (fp32) then lands in its first 64 columns
+constexpr uint32_t kTmO = 192;   // (Q e^G S)^T, then O^T
+constexpr uint32_t kTmHL = 256;  // bf16 hi (256..287) and lo (288..319) of R^T, then of E^T
+constexpr uint32_t kTmSb = 320;  // S^T bf16
+constexpr uint32_t kTmS = 384;   // S^T fp32
+
+constexpr int kThreads = 640;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Chunk descriptor.
+enum : int { kItFirst = 1, kItLast = 2, kItEmpty = 4, kItEnd = 8, kItSteep = 16 };
+struct FuItem {
+  long long s0;  // first token (row of the [tokens, H, D] tensors)
+  int unit;      // sequence * H + head
+  int Cn;        // valid rows (0 for an empty sequence)
+  int flags;
+  int pad;
+};
+
+template <int kGate>
+constexpr uint32_t g_bytes() {
+  return kGate == kGateLogTok ? 0u : kGate == kGateLogitBf16 ? C * D * 2 : C * D * 4;
+}
+constexpr uint32_t kKqvBytes = 4 * 8192 + 16384;
+
+// The two bf16 of a 32-bit word as floats (element 2i in the low half).
+__device__ __forceinline__ float2 bf2(uint32_t w) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+}
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// One 32-column TMEM load into registers (two 16-column loads).
+__device__ __forceinline__ void ld32(uint32_t ta, float* x) {
+  ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
+  ptx::tmem_ld16(ta + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+}
+
+// Splits x[0..31] (fp32, tokens 32h .. 32h + 31) into bf16 hi + lo pairs and
+// stores them, two tokens per column (token 2i in the low half), at columns
+// [base + 16h, +16) (hi) and [base + 32 + 16h, +16) (lo): after both halves
+// the 64 tokens' hi parts fill [base, base + 32) and the lo parts the next 32.
+__device__ __forceinline__ void store_hi_lo32(uint32_t base, int h, const float* x) {
+  uint32_t hi[16], lo[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = x[2 * i], b = x[2 * i + 1];
+    const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+    const float2 f = __bfloat1622float2(p);
+    hi[i] = *reinterpret_cast<const uint32_t*>(&p);
+    lo[i] = ptx::pack_bf16x2(a - f.x, b - f.y);
+  }
+  ptx::tmem_st16u(base + 16 * h, hi);
+  ptx::tmem_st16u(base + 32 + 16 * h, lo);
+}
+
+template <int kGate, bool kPacked>
+__global__ void __launch_bounds__(kThreads, 1)
+    kda_fused_prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                             const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
+                             const void* __restrict__ gate, const float* __restrict__ beta,
+                             const float* __restrict__ S0, bf16* __restrict__ o, float* __restrict__ S_out,
+                             const int32_t* __restrict__ cu_seqlens, int N, int T, int H,
+                             int* __restrict__ unit_ctr, const int* __restrict__ seq_order,
+                             const int* __restrict__ seq_status) {
+  constexpr bool kPrep = gate_prep(kGate);
+  constexpr bool kTmaGate = kGate != kGateLogTok;
+  __shared__ __align__(16) float s_beta[2][C];
+  __shared__ __align__(16) float s_glast[D];     // G at the chunk's last row
+  __shared__ __align__(16) float s_gref[4][D];   // G at the end of each 16-token block (steep chunks)
+  __shared__ float s_nrm[2][C];                  // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
+  __shared__ FuItem s_ring[8];
+  __shared__ __align__(8) uint64_t s_g_full, s_kqv_full[2], s_a_done[2], s_s_ready[2], s_rb_free[2];
+  __shared__ __align__(8) uint64_t s_e_done, s_m1, s_m3, s_st, s_drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  // packed sequences whose cu_seqlens the set-up kernel rejected: no work at all
+  if (kPacked && *seq_status < 0) return;
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
+  KDA_ALIGNED_DSMEM(sm, dsm_raw);
+  const uint32_t sb = ptx::smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = &s_abort;
+  const int units = N * H;
+
+  // chunk generator (builder thread 0 only): whole units from the counter.
+  // Its state lives in shared memory, so that it holds no registers in the
+  // other threads of the group.
+  __shared__ struct {
+    long long t0;
+    int c, nc, len, unit, done;
+  } s_gen;
+  int& g_c = s_gen.c;
+  int& g_nc = s_gen.nc;
+  int& g_len = s_gen.len;
+  int& g_unit = s_gen.unit;
+  int& g_done = s_gen.done;
+  long long& g_t0 = s_gen.t0;
+  auto gen = [&](FuItem& it) {
+    it.pad = 0;
+    if (g_done) {
+      it.flags = kItEnd;
+      return;
+    }
+    if (g_c >= g_nc) {
+      const int u = atomicAdd(unit_ctr, 1);
+      if (u >= units) {
+        g_done = 1;
+        it.flags = kItEnd;
+        return;
+      }
+      const int rank = u / H, hh = u - rank * H;
+      const int seq = seq_order ? seq_order[rank] : rank;
+      g_unit = seq * H + hh;
+      if constexpr (kPacked) {
+        long long a, b;
+        checked_seq_range(cu_seqlens, seq, T, &a, &b);
+        g_t0 = a;
+        g_len = (int)(b - a);
+      } else {
+        g_t0 = (long long)seq * T;
+        g_len = T;
+      }
+      g_nc = (g_len + C - 1) / C;
+      g_c = 0;
+      if (g_nc == 0) {  // an empty sequence: one descriptor, S_out = S0
+        it.s0 = g_t0;
+        it.unit = g_unit;
+        it.Cn = 0;
+        it.flags = kItFirst | kItLast | kItEmpty;
+        return;
+      }
+    }
+    it.s0 = g_t0 + (long long)g_c * C;
+    it.unit = g_unit;
+    it.Cn = min(C, g_len - g_c * C);
+    it.flags = (g_c == 0 ? kItFirst : 0) | (g_c == g_nc - 1 ? kItLast : 0);
+    ++g_c;
+  };
+
+  if (warp == 0) {
+    ptx::tmem_alloc(&s_tmem, kTmCols);
+    ptx::tmem_relinquish();
+  }
+  if (tid == 0) {
+    ptx::mbar_init(&s_g_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&s_kqv_full[i], 1);
+      ptx::mbar_init(&s_a_done[i], 2);
+      ptx::mbar_init(&s_s_ready[i], 1);
+      ptx::mbar_init(&s_rb_free[i], 1);
+    }
+    ptx::mbar_init(&s_e_done, 1);
+    ptx::mbar_init(&s_m1, 1);
+    ptx::mbar_init(&s_m3, 1);
+    ptx::mbar_init(&s_st, 1);
+    ptx::mbar_init(&s_drain, 2);
+    s_abort = 0;
+    ptx::fence_mbar_init();
+    g_c = g_nc = g_len = g_unit = g_done = 0;
+    g_t0 = 0;
+    for (int i = 0; i < 3; ++i) gen(s_ring[i]);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  // TMA of chunk item n's k, q (two 64-channel boxes each, swizzled into the
+  // operand panels) and V into slot n & 1; an empty chunk completes the phase
+  // with a plain arrive, the end of the work issues nothing.
+  auto issue_kqv = [&](uint32_t n, uint32_t* issued) {
+    const FuItem it = s_ring[n & 7];
+    if (it.flags & kItEnd) return;
+    const int s = n & 1;
+    ++issued[s];
+    if ((it.flags & kItEmpty) || *abort_flag) {
+      ptx::mbar_arrive(&s_kqv_full[s]);
+      return;
+    }
+    const int h = it.unit % H;
+    uint8_t* l3 = sm + FU_L3 + s * FU_L3_SLOT;
+    ptx::mbar_arrive_expect_tx(&s_kqv_full[s], kKqvBytes);
+    ptx::tma_load_3d(l3, &tm_k, 0, h, (int)it.s0, &s_kqv_full[s]);
+    ptx::tma_load_3d(l3 + 16384, &tm_k, 64, h, (int)it.s0, &s_kqv_full[s]);
+    ptx::tma_load_3d(l3 + 8192, &tm_q, 0, h, (int)it.s0, &s_kqv_full[s]);
+    ptx::tma_load_3d(l3 + 16384 + 8192, &tm_q, 64, h, (int)it.s0, &s_kqv_full[s]);
+    ptx::tma_load_3d(sm + FU_V + s * 16384, &tm_v, 0, h, (int)it.s0, &s_kqv_full[s]);
+  };
+  // TMA of item n's raw gate rows (per-channel gates only).
+  auto issue_g = [&](uint32_t n, uint32_t* issued) {
+    if constexpr (kTmaGate) {
+      const FuItem it = s_ring[n & 7];
+      if (it.flags & kItEnd) return;
+      ++*issued;
+      if ((it.flags & kItEmpty) || *abort_flag) {
+        ptx::mbar_arrive(&s_g_full);
+        return;
+      }
+      ptx::mbar_arrive_expect_tx(&s_g_full, g_bytes<kGate>());
+      ptx::tma_load_3d(sm + FU_RAWG, &tm_g, 0, it.unit % H, (int)it.s0, &s_g_full);
+    }
+  };
+  uint32_t g_issued = 0, kqv_issued[2] = {0u, 0u};
+  bool mma_issued = false;  // by this thread (builder thread 0, state thread 0)
+
+  if (warp < 8) {
+    // ============================== builder ==============================
+    // thread t owns channels 8 (t mod 16) .. + 7 of rows 4 (t / 16) .. + 3
+    const int co = tid & 15, rg = tid >> 4;
+    const int c0 = 8 * co;
+    const uint32_t kp = co >> 3, ck = co & 7;  // 64-channel panel and 16-byte chunk of the channels
+    float* s_wtot = reinterpret_cast<float*>(sm + FU_RAWG);  // [8 warps][128 ch]
+    if (tid == 0) {
+      ptx::prefetch_tmap(&tm_k);
+      ptx::prefetch_tmap(&tm_q);
+      if constexpr (kTmaGate) ptx::prefetch_tmap(&tm_g);
+      ptx::prefetch_tmap(&tm_v);
+      issue_g(0, &g_issued);
+    }
+    uint32_t st_round = 0;  // completions of s_st
+    for (uint32_t n = 0;; ++n) {
+      const int s = n & 1;
+      if (tid == 0) gen(s_ring[(n + 3) & 7]);
+      const FuItem it = s_ring[n & 7];
+      if (it.flags & kItEnd) {
+        if (tid == 0) {
+          ptx::mbar_arrive(&s_a_done[s]);
+          ptx::mbar_arrive(&s_a_done[s]);
+        }
+        break;
+      }
+      if (it.flags & kItEmpty) {  // keep the per-chunk phases in step; nothing to build
+        bool okE = true;
+        if constexpr (kTmaGate) okE = wait_or_abort(&s_g_full, n & 1, abort_flag);
+        if (ptx::bar_or(1, 256, !okE || *abort_flag)) break;  // uniform over the group
+        if (tid == 0) {
+          issue_g(n + 1, &g_issued);
+          ptx::mbar_arrive(&s_a_done[s]);
+          ptx::mbar_arrive(&s_a_done[s]);
+        }
+        continue;
+      }
+      const int h = it.unit % H;
+      const long long s0 = it.s0;
+      const int Cn = it.Cn;
+      uint8_t* l3 = sm + FU_L3 + s * FU_L3_SLOT;
+      uint8_t* rb = sm + FU_RB + s * 16384;
+      float bt = 0.f;
+      if (tid < Cn) bt = beta_of(beta, kGate, (size_t)(s0 + tid) * H + h);
+      float gtok[4] = {0.f, 0.f, 0.f, 0.f};  // per-token gate of this thread's rows
+      if constexpr (kGate == kGateLogTok) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (4 * rg + u < Cn) gtok[u] = static_cast<const float*>(gate)[(size_t)(s0 + 4 * rg + u) * H + h];
+      }
+      // Every wait is followed by a group-wide vote before anything depends on
+      // it, so that the whole group leaves together after a timeout.
+      bool ok = true;
+      if constexpr (kTmaGate) ok = wait_or_abort(&s_g_full, n & 1, abort_flag);
+      if constexpr (kPrep) ok = ok && wait_or_abort(&s_kqv_full[s], (n >> 1) & 1, abort_flag);
+
+      // ---- raw gate rows -> local cumulative sums; rows >= Cn contribute g = 0
+      float G[4][8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = 4 * rg + u;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+        if (r < Cn) {
+          if constexpr (kGate == kGateLogTok) {
+            a = make_float4(gtok[u], gtok[u], gtok[u], gtok[u]);
+            b = a;
+          } else if constexpr (kGate == kGateLogitBf16) {
+            float x[8];
+            tc::unpack8(*reinterpret_cast<const uint4*>(sm + FU_RAWG + r * 256 + 16 * co), x);
+            a = make_float4(neg_softplus(x[0]), neg_softplus(x[1]), neg_softplus(x[2]), neg_softplus(x[3]));
+            b = make_float4(neg_softplus(x[4]), neg_softplus(x[5]), neg_softplus(x[6]), neg_softplus(x[7]));
+          } else {
+            // the two 16-byte halves in alternating order across the quarter-warp (no bank conflicts)
+            const float* gr = reinterpret_cast<const float*>(sm + FU_RAWG + r * 512) + c0;
+            const int sw = (co >> 2) & 1;
+            const float4 h0 = *reinterpret_cast<const float4*>(gr + 4 * sw);
+            const float4 h1 = *reinterpret_cast<const float4*>(gr + 4 - 4 * sw);
+            a = sw ? h1 : h0;
+            b = sw ? h0 : h1;
+            if constexpr (kGate == kGateLogitF32) {
+              a = make_float4(neg_softplus(a.x), neg_softplus(a.y), neg_softplus(a.z), neg_softplus(a.w));
+              b = make_float4(neg_softplus(b.x), neg_softplus(b.y), neg_softplus(b.z), neg_softplus(b.w));
+            }
+          }
+        }
+        const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) G[u][e] = (u ? G[u - 1][e] : 0.f) + x[e];
+      }
+      // 1 / |k_r| and 1 / |q_r| over dk (only when the call normalises): the 16
+      // lanes of a half-warp hold one row; k and q are read from their panels.
+      if constexpr (kPrep) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = 4 * rg + u;
+          float kx[8], qx[8];
+          tc::unpack8(*reinterpret_cast<const uint4*>(l3 + kp * 16384 + ptx::sw128_chunk(r, ck)), kx);
+          tc::unpack8(*reinterpret_cast<const uint4*>(l3 + kp * 16384 + 8192 + ptx::sw128_chunk(r, ck)), qx);
+          float sk = 0.f, sq = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            sk = fmaf(kx[e], kx[e], sk);
+            sq = fmaf(qx[e], qx[e], sq);
+          }
+#pragma unroll
+          for (int off = 1; off < 16; off <<= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+          }
+          if (co == 0) {
+            s_nrm[0][r] = rsqrtf(fmaxf(sk, 1e-24f));
+            s_nrm[1][r] = rsqrtf(fmaxf(sq, 1e-24f));
+          }
+        }
+      }
+      // Row-group totals: this warp holds row groups 2w (lanes 0..15) and 2w+1
+      // (lanes 16..31) of the same channels; the warp's total goes to s_wtot,
+      // which lives over the raw gate rows once every thread has read its own.
+      float lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lo[e] = __shfl_xor_sync(0xffffffffu, G[3][e], 16);
+      if (ptx::bar_or(1, 256, !ok || *abort_flag)) break;  // raw gate rows consumed
+      if (lane >= 16) {
+        reinterpret_cast<float4*>(s_wtot + warp * D + c0)[0] =
+            make_float4(G[3][0] + lo[0], G[3][1] + lo[1], G[3][2] + lo[2], G[3][3] + lo[3]);
+        reinterpret_cast<float4*>(s_wtot + warp * D + c0)[1] =
+            make_float4(G[3][4] + lo[4], G[3][5] + lo[5], G[3][6] + lo[6], G[3][7] + lo[7]);
+      }
+      ptx::bar_sync(1, 256);  // warp totals visible
+      {
+        float off[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) off[e] = lane >= 16 ? lo[e] : 0.f;
+        for (int w2 = 0; w2 < warp; ++w2) {  // warp-uniform
+          const float4 t0 = reinterpret_cast<const float4*>(s_wtot + w2 * D + c0)[0];
+          const float4 t1 = reinterpret_cast<const float4*>(s_wtot + w2 * D + c0)[1];
+          off[0] += t0.x; off[1] += t0.y; off[2] += t0.z; off[3] += t0.w;
+          off[4] += t1.x; off[5] += t1.y; off[6] += t1.z; off[7] += t1.w;
+        }
+        if constexpr (kGate == kGateLogTok) {  // one gate per token: every channel has the same G
+#pragma unroll
+          for (int e = 1; e < 8; ++e) off[e] = off[0];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) G[u][e] += off[e];
+      }
+      // G is non-increasing (g <= 0): G at the chunk's last row is each channel's
+      // minimum; G at the last row of blocks 0..2 are the block references.
+      bool steep = false;
+      if (rg == 15) {
+        reinterpret_cast<float4*>(s_glast + c0)[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+        reinterpret_cast<float4*>(s_glast + c0)[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) steep |= !(G[3][e] >= tc::kChunkRefMinG);
+      }
+      if ((rg & 3) == 3 && rg < 15) {
+        reinterpret_cast<float4*>(&s_gref[(rg + 1) >> 2][c0])[0] = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
+        reinterpret_cast<float4*>(&s_gref[(rg + 1) >> 2][c0])[1] = make_float4(G[3][4], G[3][5], G[3][6], G[3][7]);
+      }
+      // uniform over the group; s_glast, s_gref visible; s_wtot (the raw gate buffer) read
+      const bool fast = !ptx::bar_or(1, 256, steep);
+      if (fast && tid == 0) issue_g(n + 1, &g_issued);
+
+      ok = true;
+      if constexpr (!kPrep) ok = wait_or_abort(&s_kqv_full[s], (n >> 1) & 1, abort_flag);
+      // K e^-G, gamma of this slot: the state is done with chunk n-2
+      if (n >= 2) ok = ok && wait_or_abort(&s_rb_free[s], ((n - 2) >> 1) & 1, abort_flag);
+      if (ptx::bar_or(1, 256, !ok || *abort_flag)) break;
+      if (tid < C) s_beta[s][tid] = bt;  // the solver is done with chunk n-2's
+
+      if (fast) {
+        // Single reference (chunk start): a = e^{G} <= 1, rho = e^{-G} <= e^80.
+        // Each 16-byte piece (8 channels of one row) is rewritten in place.
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = 4 * rg + u;
+          uint8_t* pk = l3 + kp * 16384 + ptx::sw128_chunk(r, ck);
+          uint8_t* pq = pk + 8192;
+          uint4 kw = *reinterpret_cast<const uint4*>(pk), qw = *reinterpret_cast<const uint4*>(pq);
+          if (r >= Cn) kw = qw = make_uint4(0u, 0u, 0u, 0u);
+          const float nk = kPrep ? s_nrm[0][r] : 1.f, nq = kPrep ? s_nrm[1][r] : 1.f;
+          uint32_t ka[4], qa[4], kr[4];
+#pragma unroll
+          for (int p2 = 0; p2 < 4; ++p2) {
+            float2 kf = bf2(word(kw, p2)), qf = bf2(word(qw, p2));
+            if constexpr (kPrep) {
+              kf.x *= nk; kf.y *= nk;
+              qf.x *= nq; qf.y *= nq;
+            }
+            const float t0 = G[u][2 * p2] * kLog2e, t1 = G[u][2 * p2 + 1] * kLog2e;  // in [-115.5, 0]
+            const float a0 = ptx::ex2(t0), a1 = ptx::ex2(t1);
+            ka[p2] = ptx::pack_bf16x2(kf.x * a0, kf.y * a1);
+            qa[p2] = ptx::pack_bf16x2(qf.x * a0, qf.y * a1);
+            kr[p2] = ptx::pack_bf16x2(kf.x * ptx::ex2(-t0), kf.y * ptx::ex2(-t1));
+          }
+          *reinterpret_cast<uint4*>(pk) = make_uint4(ka[0], ka[1], ka[2], ka[3]);
+          *reinterpret_cast<uint4*>(pq) = make_uint4(qa[0], qa[1], qa[2], qa[3]);
+          *reinterpret_cast<uint4*>(rb + kp * 8192 + ptx::sw128_chunk(r, ck)) = make_uint4(kr[0], kr[1], kr[2], kr[3]);
+        }
+      } else {
+        // Steep chunk: some channel decays by more than 80 over the chunk.  [A'; P']
+        // is accumulated from four MMAs, one per 16-row block I, with the block's
+        // reference rho_I = G at the end of block I-1 (0 for I = 0): left rows of
+        // block I scaled by e^{G - rho_I} <= 1 (other rows zero), right rows
+        // j <= end of block I scaled by e^{rho_I - G_j} (<= e^80 inside block I,
+        // <= 1 before it; later rows zero).  The left operand sits over the raw
+        // gate rows, whose next load waits until the four MMAs are done.
+        if (tid == 0 && n >= 2) wait_or_abort(&s_s_ready[s], ((n - 2) >> 1) & 1, abort_flag);
+        uint8_t* lft = sm + FU_RAWG;
+        bool quit = false;
+        for (int I = 0; I < 4; ++I) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = 4 * rg + u, blk = rg >> 2;
+            uint4 kw = *reinterpret_cast<const uint4*>(l3 + kp * 16384 + ptx::sw128_chunk(r, ck));
+            uint4 qw = *reinterpret_cast<const uint4*>(l3 + kp * 16384 + 8192 + ptx::sw128_chunk(r, ck));
+            if (r >= Cn) kw = qw = make_uint4(0u, 0u, 0u, 0u);
+            const float nk = kPrep ? s_nrm[0][r] : 1.f, nq = kPrep ? s_nrm[1][r] : 1.f;
+            uint32_t lk[4], lq[4], rr[4];
+#pragma unroll
+            for (int p2 = 0; p2 < 4; ++p2) {
+              float2 kf = bf2(word(kw, p2)), qf = bf2(word(qw, p2));
+              if constexpr (kPrep) {
+                kf.x *= nk; kf.y *= nk;
+                qf.x *= nq; qf.y *= nq;
+              }
+              const float2 ref = I ? *reinterpret_cast<const float2*>(&s_gref[I][c0 + 2 * p2]) : make_float2(0.f, 0.f);
+              // d <= 0 for rows in or after block I, >= 0 before it
+              const float d0 = (G[u][2 * p2] - ref.x) * kLog2e, d1 = (G[u][2 * p2 + 1] - ref.y) * kLog2e;
+              const float a0 = blk == I ? ptx::ex2(d0) : 0.f, a1 = blk == I ? ptx::ex2(d1) : 0.f;
+              lk[p2] = ptx::pack_bf16x2(kf.x * a0, kf.y * a1);
+              lq[p2] = ptx::pack_bf16x2(qf.x * a0, qf.y * a1);
+              rr[p2] = blk <= I ? ptx::pack_bf16x2(kf.x * ptx::ex2(-d0), kf.y * ptx::ex2(-d1)) : 0u;
+            }
+            *reinterpret_cast<uint4*>(lft + kp * 16384 + ptx::sw128_chunk(r, ck)) = make_uint4(lk[0], lk[1], lk[2], lk[3]);
+            *reinterpret_cast<uint4*>(lft + kp * 16384 + ptx::sw128_chunk(64 + r, ck)) =
+                make_uint4(lq[0], lq[1], lq[2], lq[3]);
+            *reinterpret_cast<uint4*>(rb + kp * 8192 + ptx::sw128_chunk(r, ck)) = make_uint4(rr[0], rr[1], rr[2], rr[3]);
+          }
+          ptx::fence_proxy_async_smem();
+          if (ptx::bar_or(1, 256, *abort_flag != 0)) {
+            quit = true;
+            break;
+          }
+          if (tid == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t id = ptx::idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t ad = ptx::sdesc_sw128(sb + FU_RAWG + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = ptx::sdesc_sw128(sb + FU_RB + s * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+              ptx::mma_bf16(tmem + 64 * s, ad, bd, id, (I > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_issued = true;
+            ptx::mma_commit(&s_st);
+          }
+          // the operands are rewritten by the next round: wait for this MMA
+          wait_or_abort(&s_st, st_round & 1, abort_flag);
+          ++st_round;
+        }
+        if (quit || ptx::bar_or(1, 256, *abort_flag != 0)) break;
+        // the state's operands: K e^G, Q e^G (chunk start, in place), Kbar = K e^{G_last - G}
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = 4 * rg + u;
+          uint8_t* pk = l3 + kp * 16384 + ptx::sw128_chunk(r, ck);
+          uint8_t* pq = pk + 8192;
+          uint4 kw = *reinterpret_cast<const uint4*>(pk), qw = *reinterpret_cast<const uint4*>(pq);
+          if (r >= Cn) kw = qw = make_uint4(0u, 0u, 0u, 0u);
+          const float nk = kPrep ? s_nrm[0][r] : 1.f, nq = kPrep ? s_nrm[1][r] : 1.f;
+          uint32_t ka[4], qa[4], kb[4];
+#pragma unroll
+          for (int p2 = 0; p2 < 4; ++p2) {
+            float2 kf = bf2(word(kw, p2)), qf = bf2(word(qw, p2));
+            if constexpr (kPrep) {
+              kf.x *= nk; kf.y *= nk;
+              qf.x *= nq; qf.y *= nq;
+            }
+            const float2 gl2 = *reinterpret_cast<const float2*>(&s_glast[c0 + 2 * p2]);
+            const float a0 = ptx::ex2(G[u][2 * p2] * kLog2e), a1 = ptx::ex2(G[u][2 * p2 + 1] * kLog2e);
+            ka[p2] = ptx::pack_bf16x2(kf.x * a0, kf.y * a1);
+            qa[p2] = ptx::pack_bf16x2(qf.x * a0, qf.y * a1);
+            kb[p2] = ptx::pack_bf16x2(kf.x * ptx::ex2((gl2.x - G[u][2 * p2]) * kLog2e),
+                                      kf.y * ptx::ex2((gl2.y - G[u][2 * p2 + 1]) * kLog2e));
+          }
+          *reinterpret_cast<uint4*>(pk) = make_uint4(ka[0], ka[1], ka[2], ka[3]);
+          *reinterpret_cast<uint4*>(pq) = make_uint4(qa[0], qa[1], qa[2], qa[3]);
+          *reinterpret_cast<uint4*>(rb + kp * 8192 + ptx::sw128_chunk(r, ck)) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
+        }
+      }
+      if (rg == 0) {
+        float gm[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gm[e] = expf(s_glast[c0 + e]);
+        float* gam = reinterpret_cast<float*>(sm + FU_GAM + s * 512);
+        reinterpret_cast<float4*>(gam)[2 * co] = make_float4(gm[0], gm[1], gm[2], gm[3]);
+        reinterpret_cast<float4*>(gam)[2 * co + 1] = make_float4(gm[4], gm[5], gm[6], gm[7]);
+      }
+      if (tid == 0 && !fast) s_ring[n & 7].flags |= kItSteep;
+      ptx::fence_proxy_async_smem();
+      ptx::bar_sync(1, 256);  // operands, s_beta[s], gamma complete
+
+      if (tid == 0) {
+        if (fast) {
+          // TMEM slot s: the solver is done with chunk n-2
+          const bool go = !*abort_flag && (n < 2 || wait_or_abort(&s_s_ready[s], ((n - 2) >> 1) & 1, abort_flag));
+          if (go) {
+            // [A'; P'] = [K e^G; Q e^G] (K e^-G)^T : M=128, N=64, K=128
+            ptx::tc_fence_after();
+            constexpr uint32_t id = ptx::idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t ad = ptx::sdesc_sw128(sb + FU_L3 + s * FU_L3_SLOT + (kk >> 2) * 16384 + (kk & 3) * 32,
+                                                   16, 1024);
+              const uint64_t bd = ptx::sdesc_sw128(sb + FU_RB + s * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+              ptx::mma_bf16(tmem + 64 * s, ad, bd, id, kk > 0);
+            }
+            mma_issued = true;
+            ptx::mma_commit(&s_a_done[s]);
+          } else {
+            ptx::mbar_arrive(&s_a_done[s]);
+          }
+        } else {
+          ptx::mbar_arrive(&s_a_done[s]);  // the block MMAs have completed already
+          issue_g(n + 1, &g_issued);       // the raw gate buffer is free again
+        }
+        ptx::mbar_arrive(&s_a_done[s]);  // releases s_beta[s] and the descriptor's flags
+      }
+    }
+  } else if (warp < 16) {
+    // ============================== solver ==============================
+    const int st = tid - 256, w8 = warp - 8;
+    float* As = reinterpret_cast<float*>(sm + FU_AS);
+    uint32_t real = 0;  // chunks solved (E MMAs to wait for)
+    for (uint32_t n = 0;; ++n) {
+      const int s = n & 1;
+      bool ok = wait_or_abort(&s_a_done[s], (n >> 1) & 1, abort_flag);
+      // P of this slot: the state is done with chunk n-2
+      if (n >= 2) ok = ok && wait_or_abort(&s_rb_free[s], ((n - 2) >> 1) & 1, abort_flag);
+      if (ptx::bar_or(2, 256, !ok || *abort_flag)) break;  // uniform over the group
+      ptx::tc_fence_after();
+      const FuItem it = s_ring[n & 7];
+      if (!(it.flags & (kItEnd | kItEmpty))) {
+        // scatter A (fp32, beta-scaled) and P (bf16) out of TMEM slot s
+        tc::scatter_single_ref(tmem + 64 * s, s_beta[s], As, sm + FU_P + s * 8192, warp, w8, lane, false);
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        // T diag(beta) and the block products (both in FU_TT): the E MMA of the
+        // previous chunk has read T diag(beta)
+        ok = real == 0 || wait_or_abort(&s_e_done, (real - 1) & 1, abort_flag);
+        if (ptx::bar_or(2, 256, !ok || *abort_flag)) break;
+        // T = (I + A)^{-1}, T diag(beta) as bf16 hi (FU_TT) + lo (over T, FU_TS)
+        tc::solve_t_beta(As, reinterpret_cast<float*>(sm + FU_TS), reinterpret_cast<float*>(sm + FU_TT),
+                         s_beta[s], sm + FU_TT, st, w8, lane, [] { ptx::bar_sync(2, 256); },
+                         [](bool p) { return ptx::bar_or(2, 256, p); }, sm + FU_TS);
+        ptx::fence_proxy_async_smem();
+        ptx::bar_sync(2, 256);
+        ++real;
+      }
+      if (st == 0) ptx::mbar_arrive(&s_s_ready[s]);
+      if (it.flags & kItEnd) break;
+    }
+  } else {
+    // ============================== state ==============================
+    const int st = tid - 512, qd = warp & 3;
+    const int dv = 32 * qd + lane;  // this thread's value channel = its TMEM lane
+    const uint32_t lo_lane = (uint32_t)(32 * qd) << 16;
+    if (st == 0) {
+      issue_kqv(0, kqv_issued);
+      issue_kqv(1, kqv_issued);
+    }
+    uint32_t real = 0;  // chunks with MMAs (phases of m1, e_done, m3)
+    for (uint32_t n = 0;; ++n) {
+      const int s = n & 1;
+      const bool okr = wait_or_abort(&s_s_ready[s], (n >> 1) & 1, abort_flag);
+      if (ptx::bar_or(3, 128, !okr || *abort_flag)) break;  // uniform over the group
+      ptx::tc_fence_after();
+      const FuItem it = s_ring[n & 7];
+      if (it.flags & kItEnd) break;
+      const size_t urow = (size_t)it.unit * D;  // first state row of the unit
+      if (it.flags & kItEmpty) {  // an empty sequence hands its initial state through
+        if (S_out)
+          for (int c = 0; c < D; ++c) S_out[(urow + c) * D + dv] = S0 ? S0[(urow + c) * D + dv] : 0.f;
+        if (st == 0) {
+          issue_kqv(n + 2, kqv_issued);
+          ptx::mbar_arrive(&s_rb_free[s]);
+        }
+        continue;
+      }
+      const bool steep = (it.flags & kItSteep) != 0;
+      if (it.flags & kItFirst) {  // the unit's initial state, transposed: row dv of S^T
+#pragma unroll 1
+        for (int c16 = 0; c16 < D; c16 += 16) {
+          float x[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) x[e] = S0 ? S0[(urow + c16 + e) * D + dv] : 0.f;
+          ptx::tmem_st16(tmem + lo_lane + kTmS + c16, x);
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[i] = ptx::pack_bf16x2(x[2 * i], x[2 * i + 1]);
+          ptx::tmem_st8u(tmem + lo_lane + kTmSb + c16 / 2, w);
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::bar_sync(3, 128);
+      }
+      // ---- X^T = S^T [K e^G; Q e^G]^T  (M=128, N=128, K=128; A in TMEM)
+      if (st == 0) {
+        ptx::tc_fence_after();
+        constexpr uint32_t id = ptx::idesc_bf16(128, 128, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::mma_bf16_ts(tmem + kTmX, tmem + kTmSb + 8 * kk,
+                           ptx::sdesc_sw128(sb + FU_L3 + s * FU_L3_SLOT + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                           id, kk > 0);
+        mma_issued = true;
+        ptx::mma_commit(&s_m1);
+      }
+      const float* gam = reinterpret_cast<const float*>(sm + FU_GAM + s * 512);
+      if (steep) {  // Kbar form: decay the state first (the MMA above reads only the bf16 copy)
+#pragma unroll 1
+        for (int c32 = 0; c32 < D; c32 += 32) {
+          float x[32];
+          ld32(tmem + lo_lane + kTmS + c32, x);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= gam[c32 + e];
+          ptx::tmem_st16(tmem + lo_lane + kTmS + c32, *reinterpret_cast<float(*)[16]>(x));
+          ptx::tmem_st16(tmem + lo_lane + kTmS + c32 + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+        }
+      }
+      bool ok = wait_or_abort(&s_m1, real & 1, abort_flag);
+      ok = ok && wait_or_abort(&s_kqv_full[s], (n >> 1) & 1, abort_flag);  // V
+      ptx::tc_fence_after();
+      // ---- R^T = V^T - (K e^G S)^T in fp32 (tokens j >= Cn zero) as bf16 hi | lo
+      const bf16* vs = reinterpret_cast<const bf16*>(sm + FU_V + s * 16384) + dv;
+#pragma unroll 1
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float x[32];
+        ld32(tmem + lo_lane + kTmX + 32 * h2, x);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = 32 * h2 + e;
+          x[e] = j < it.Cn ? __bfloat162float(vs[j * D]) - x[e] : 0.f;
+        }
+        store_hi_lo32(tmem + lo_lane + kTmHL, h2, x);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      if (ptx::bar_or(3, 128, !ok || *abort_flag)) break;  // R^T stored; this slot's panels and V are free
+      if (st == 0) {
+        issue_kqv(n + 2, kqv_issued);
+        // ---- E^T = R^T (T diag(beta))^T  (N=64, K=64), over (K e^G S)^T, from
+        //      the hi + lo pairs: R_hi T_hi + R_lo T_hi + R_hi T_lo
+        ptx::tc_fence_after();
+        constexpr uint32_t id = ptx::idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int i = 0; i < 12; ++i) {
+          const uint32_t rcol = (i >> 2) == 1 ? 32 : 0;        // R lo for the second group
+          const uint32_t tsm = (i >> 2) == 2 ? FU_TS : FU_TT;   // T lo for the third group
+          ptx::mma_bf16_ts(tmem + kTmX, tmem + kTmHL + rcol + 8 * (i & 3),
+                           ptx::sdesc_sw128(sb + tsm + (i & 3) * 32, 16, 1024), id, i > 0);
+        }
+        ptx::mma_commit(&s_e_done);
+      }
+      ok = wait_or_abort(&s_e_done, real & 1, abort_flag);
+      ptx::tc_fence_after();
+#pragma unroll 1
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float x[32];
+        ld32(tmem + lo_lane + kTmX + 32 * h2, x);
+        ptx::tmem_wait_ld();
+        store_hi_lo32(tmem + lo_lane + kTmHL, h2, x);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      if (ptx::bar_or(3, 128, !ok || *abort_flag)) break;
+      if (st == 0) {
+        ptx::tc_fence_after();
+        // S^T += E^T (K e^-G) (Kbar for a steep chunk): N=128, K=64, B MN-major
+        constexpr uint32_t id2 = ptx::idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          ptx::mma_bf16_ts(tmem + kTmS, tmem + kTmHL + (i >> 2) * 32 + 8 * (i & 3),
+                           ptx::sdesc_sw128(sb + FU_RB + s * 16384 + (i & 3) * 2048, 8192, 1024), id2, 1);
+        // X^T[:, 64:128] += E^T P^T: N=64, K=64, B K-major
+        constexpr uint32_t id3 = ptx::idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          ptx::mma_bf16_ts(tmem + kTmO, tmem + kTmHL + (i >> 2) * 32 + 8 * (i & 3),
+                           ptx::sdesc_sw128(sb + FU_P + s * 8192 + (i & 3) * 32, 16, 1024), id3, 1);
+        ptx::mma_commit(&s_m3);
+      }
+      ok = wait_or_abort(&s_m3, real & 1, abort_flag);
+      if (ptx::bar_or(3, 128, !ok || *abort_flag)) break;
+      ptx::tc_fence_after();
+      // ---- decay (single-reference chunks), the next chunk's bf16 operand, the outputs
+#pragma unroll 1
+      for (int c32 = 0; c32 < D; c32 += 32) {
+        float x[32];
+        ld32(tmem + lo_lane + kTmS + c32, x);
+        ptx::tmem_wait_ld();
+        if (!steep) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= gam[c32 + e];
+          ptx::tmem_st16(tmem + lo_lane + kTmS + c32, *reinterpret_cast<float(*)[16]>(x));
+          ptx::tmem_st16(tmem + lo_lane + kTmS + c32 + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = ptx::pack_bf16x2(x[2 * i], x[2 * i + 1]);
+        ptx::tmem_st16u(tmem + lo_lane + kTmSb + c32 / 2, w);
+      }
+      float ov[64];
+      ld32(tmem + lo_lane + kTmO, ov);
+      ld32(tmem + lo_lane + kTmO + 32, ov + 32);
+      ptx::tmem_wait_ld();
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::bar_sync(3, 128);  // every read of this slot's K e^-G, P, gamma and of X^T done
+      if (st == 0) ptx::mbar_arrive(&s_rb_free[s]);
+      const int h = it.unit % H;
+      bf16* orow = o + ((size_t)it.s0 * H + h) * D + dv;
+      const size_t ostride = (size_t)H * D;
+#pragma unroll
+      for (int r = 0; r < 64; ++r)
+        if (r < it.Cn) orow[r * ostride] = __float2bfloat16_rn(ov[r]);
+      if ((it.flags & kItLast) && S_out) {
+#pragma unroll 1
+        for (int c32 = 0; c32 < D; c32 += 32) {
+          float x[32];
+          ld32(tmem + lo_lane + kTmS + c32, x);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) S_out[(urow + c32 + e) * D + dv] = x[e];
+        }
+      }
+      ++real;
+    }
+  }
+
+  // After a timeout: wait (bounded again) for the copies and MMAs still in
+  // flight, so that nothing lands in shared or tensor memory after exit.
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (s_abort) {
+    if (tid == 0 && g_issued) ptx::mbar_wait_bounded(&s_g_full, (g_issued - 1) & 1, 1000000000ull);
+    if (tid == 512)
+      for (int i = 0; i < 2; ++i)
+        if (kqv_issued[i]) ptx::mbar_wait_bounded(&s_kqv_full[i], (kqv_issued[i] - 1) & 1, 1000000000ull);
+  }
+  __syncthreads();
+  if (s_abort && (tid == 0 || tid == 512)) {  // the two MMA-issuing threads
+    if (mma_issued) ptx::mma_commit(&s_drain);
+    else ptx::mbar_arrive(&s_drain);
+    ptx::mbar_wait_bounded(&s_drain, 0, 1000000000ull);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 0) ptx::tmem_dealloc(tmem, kTmCols);
+}
+
+// Set-up of one call (one CTA of 1024 threads): zeroes the unit counter and,
+// for packed sequences, checks cu_seqlens (cu[0] == 0, non-decreasing,
+// cu[num_seqs] == T) -- a bad table raises the device error word and sets
+// *status = -1, so the prefill kernel does nothing -- then orders the
+// sequences longest first (rank by length, ties by index) when there are at
+// most kSortMax of them; longer lists keep their order.
+constexpr int kSortMax = 2048;
+__global__ void __launch_bounds__(1024)
+    kda_fused_setup_kernel(const int32_t* __restrict__ cu_seqlens, int num_seqs, int T, int* __restrict__ ctr,
+                           int* __restrict__ status, int* __restrict__ order) {
+  __shared__ int s_len[kSortMax];
+  const int tid = threadIdx.x;
+  if (tid == 0) *ctr = 0;
+  if (!cu_seqlens) return;
+  bool bad = tid == 0 && (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T);
+  for (int i = tid; i < num_seqs; i += 1024) bad |= cu_seqlens[i + 1] < cu_seqlens[i];
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) {
+      raise_device_error(kDevErrBadSeqlens);
+      *status = -1;
+    }
+    return;
+  }
+  if (tid == 0) *status = 0;
+  if (num_seqs > kSortMax) {
+    for (int i = tid; i < num_seqs; i += 1024) order[i] = i;
+    return;
+  }
+  for (int i = tid; i < num_seqs; i += 1024) s_len[i] = cu_seqlens[i + 1] - cu_seqlens[i];
+  __syncthreads();
+  for (int i = tid; i < num_seqs; i += 1024) {
+    const int li = s_len[i];
+    int rank = 0;
+    for (int j = 0; j < num_seqs; ++j) {
+      const int lj = s_len[j];
+      rank += (lj > li) || (lj == li && j < i);
+    }
+    order[rank] = i;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+// Workspace: the unit counter, the table check's status, the sequence order.
+inline size_t fused_workspace_bytes(int num_seqs) { return 256 + (size_t)std::max(num_seqs, 0) * sizeof(int); }
+
+inline bool fused_kernel_available() {
+  static PerDeviceOnce once;
+  static bool ok[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  run_once_per_device(once, [dev] {
+    const void* fns[] = {(const void*)kda_fused_prefill_kernel<kGateLogCh, false>,
+                         (const void*)kda_fused_prefill_kernel<kGateLogTok, false>,
+                         (const void*)kda_fused_prefill_kernel<kGateLogitF32, false>,
+                         (const void*)kda_fused_prefill_kernel<kGateLogitBf16, false>,
+                         (const void*)kda_fused_prefill_kernel<kGateLogCh, true>,
+                         (const void*)kda_fused_prefill_kernel<kGateLogTok, true>,
+                         (const void*)kda_fused_prefill_kernel<kGateLogitF32, true>,
+                         (const void*)kda_fused_prefill_kernel<kGateLogitBf16, true>};
+    int optin = 0;
+    bool all = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
+    for (const void* fn : fns) {
+      cudaFuncAttributes fa{};
+      all = all && cudaFuncGetAttributes(&fa, fn) == cudaSuccess &&
+            (size_t)FU_DYN + fa.sharedSizeBytes <= (size_t)optin &&
+            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FU_DYN) == cudaSuccess;
+    }
+    ok[dev] = all;
+    cudaGetLastError();  // an unavailable kernel is not an error of the call
+    return cudaSuccess;
+  });
+  return ok[dev];
+}
+
+template <int kGate>
+inline cudaError_t launch_fused_t(const bf16* q, const bf16* k, const bf16* v, const void* g, const float* beta,
+                                  const float* S0, bf16* o, float* S_out, const int32_t* cu_seqlens, int N,
+                                  int B, int T, int H, void* workspace, int sms, cudaStream_t stream) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  cudaError_t e = ws::tensor_map_encoder(&enc);
+  if (e != cudaSuccess) return e;
+  const long long tokens = (long long)B * T;
+  CUtensorMap mk, mq, mg, mv;
+  if ((e = ws::encode_rows_map(enc, &mk, k, false, tokens, H, 64, true)) != cudaSuccess) return e;
+  if ((e = ws::encode_rows_map(enc, &mq, q, false, tokens, H, 64, true)) != cudaSuccess) return e;
+  if ((e = ws::encode_rows_map(enc, &mv, v, false, tokens, H, D, false)) != cudaSuccess) return e;
+  if constexpr (kGate == kGateLogTok) {
+    mg = mk;  // not read: a per-token gate takes plain loads
+  } else {
+    if ((e = ws::encode_rows_map(enc, &mg, g, kGate != kGateLogitBf16, tokens, H, D, false)) != cudaSuccess) return e;
+  }
+  int* wsi = static_cast<int*>(workspace);
+  int* ctr = wsi;
+  int* status = wsi + 1;
+  int* order = wsi + 64;
+  kda_fused_setup_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, cu_seqlens ? N : 0, T, ctr, status, order);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const long long units = (long long)N * H;
+  const int grid = (int)std::min<long long>(units, sms);
+  if (grid <= 0) return cudaSuccess;
+  if (cu_seqlens)
+    kda_fused_prefill_kernel<kGate, true><<<grid, kThreads, FU_DYN, stream>>>(
+        mk, mq, mg, mv, g, beta, S0, o, S_out, cu_seqlens, N, T, H, ctr, order, status);
+  else
+    kda_fused_prefill_kernel<kGate, false><<<grid, kThreads, FU_DYN, stream>>>(
+        mk, mq, mg, mv, g, beta, S0, o, S_out, nullptr, N, T, H, ctr, nullptr, status);
+  return cudaGetLastError();
+}
+
+inline cudaError_t launch_fused(const bf16* q, const bf16* k, const bf16* v, const void* g, const float* beta,
+                                const float* S0, bf16* o, float* S_out, const int32_t* cu_seqlens, int N, int B,
+                                int T, int H, void* workspace, int sms, int gmode, cudaStream_t stream) {
+  switch (gmode) {
+    case kGateLogCh:
+      return launch_fused_t<kGateLogCh>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms, stream);
+    case kGateLogTok:
+      return launch_fused_t<kGateLogTok>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms, stream);
+    case kGateLogitF32:
+      return launch_fused_t<kGateLogitF32>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms,
+                                           stream);
+    case kGateLogitBf16:
+      return launch_fused_t<kGateLogitBf16>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms,
+                                            stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace fu
+}  // namespace kda

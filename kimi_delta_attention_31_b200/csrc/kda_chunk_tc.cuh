@@ -189,6 +189,40 @@ __device__ __forceinline__ void warp_gemm16(float (&acc)[2][4], const float* xp,
     }
   }
 }
+// The same product with each operand split as tf32 hi + lo (x = hi + lo to
+// about 2^-22): acc += Xlo Yhi + Xhi Ylo + Xhi Yhi, three TF32 MMAs per step,
+// about fp32 accuracy.  For blocks of A whose entries are large (near-parallel
+// keys), where the block products cancel and TF32 rounding would not average out.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = ptx::to_tf32(x);
+  lo = ptx::to_tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void warp_gemm16_3x(float (&acc)[2][4], const float* xp, int ldx, const float* yp,
+                                               int ldy, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int kh = 0; kh < 2; ++kh) {
+    uint32_t ah[4], al[4];
+    split_tf32(xp[g * ldx + 8 * kh + t], ah[0], al[0]);
+    split_tf32(xp[(g + 8) * ldx + 8 * kh + t], ah[1], al[1]);
+    split_tf32(xp[g * ldx + 8 * kh + t + 4], ah[2], al[2]);
+    split_tf32(xp[(g + 8) * ldx + 8 * kh + t + 4], ah[3], al[3]);
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+      uint32_t bh[2], bl[2];
+      split_tf32(yp[(8 * kh + t) * ldy + 8 * nh + g], bh[0], bl[0]);
+      split_tf32(yp[(8 * kh + t + 4) * ldy + 8 * nh + g], bh[1], bl[1]);
+      ptx::mma_tf32_m16n8k8(acc[nh], al, bh);
+      ptx::mma_tf32_m16n8k8(acc[nh], ah, bl);
+      ptx::mma_tf32_m16n8k8(acc[nh], ah, bh);
+    }
+  }
+}
+// An entry of A at least this large switches the chunk's block products to
+// warp_gemm16_3x (keys this close to parallel do not occur by chance in 128
+// dimensions; repeated or near-duplicate keys do).
+constexpr float kSolveAccurateA = 0.5f;
+
 __device__ __forceinline__ void warp_store16(float* dp, int ldd, const float (&acc)[2][4], float scale, int lane) {
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -255,10 +289,26 @@ __device__ __forceinline__ void scatter_single_ref(uint32_t tm, const float* s_b
 // blocks above it in the same column, so warp J walks down its column (warp
 // syncs only), with TF32 warp MMAs and fp32 accumulation.  Finally
 // T diag(beta) in bf16 (K-major [64 r][64 j], 128-byte swizzle) into Tt.
-// 256 threads: t in [0, 256), w = t / 32; `sync` is their barrier.
-template <typename Sync>
+// 256 threads: t in [0, 256), w = t / 32; `sync` is their barrier and
+// `sync_or(p)` the same barrier returning the OR of p over them.  When some
+// |A_rj| >= kSolveAccurateA the block products run in split TF32.
+// With Tlo given, T diag(beta) is also split as hi + lo, hi = bf16(x) into Tt
+// and lo = bf16(x - hi) into Tlo (same layout), so that a pair of bf16 MMAs
+// uses it to about 2^-16; Tlo may overlap Ts (it is written after a barrier
+// that follows the last read of Ts).
+template <typename Sync, typename SyncOr>
 __device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* Mt, const float* s_beta, uint8_t* Tt,
-                                             int t, int w, int lane, Sync sync) {
+                                             int t, int w, int lane, Sync sync, SyncOr sync_or,
+                                             uint8_t* Tlo = nullptr) {
+  bool big = false;  // this thread's 16 entries of A (rows t / 4, columns 16 (t mod 4) ..)
+  {
+    const float4* a4 = reinterpret_cast<const float4*>(As + (t >> 2) * AS_LD + 16 * (t & 3));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 a = a4[i];
+      big |= fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))) >= kSolveAccurateA;
+    }
+  }
   if (t < 64) {
     const int jj = t & 15, o = t & 48;  // column jj of diagonal block o / 16
     float x[16];
@@ -288,7 +338,7 @@ __device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* 
 #pragma unroll
     for (int i = 0; i < 16; ++i) Ts[(o + i) * AS_LD + o + jj] = x[i];
   }
-  sync();
+  const bool accurate = sync_or(big);
   if (w < 3) {
     const int Jc = w;
     float* mt = Mt + w * 16 * MT_LD;
@@ -300,12 +350,18 @@ __device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* 
 #pragma unroll
         for (int kk = 0; kk < step; ++kk) {
           const int K = Jc + kk;
-          warp_gemm16(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
+          if (accurate)
+            warp_gemm16_3x(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
+          else
+            warp_gemm16(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
         }
         warp_store16(mt, MT_LD, acc, 1.f, lane);
         __syncwarp();
         float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        warp_gemm16(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
+        if (accurate)
+          warp_gemm16_3x(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
+        else
+          warp_gemm16(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
         warp_store16(Ts + 16 * Ir * AS_LD + 16 * Jc, AS_LD, acc2, -1.f, lane);
         __syncwarp();  // block (Ir, Jc) visible to the warp's next step; mt free again
       }
@@ -313,7 +369,8 @@ __device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* 
   }
   sync();
   // bf16 T diag(beta); blocks above the diagonal are zero
-  for (int idx = t; idx < 512; idx += 256) {
+  uint4 lo_w[2];
+  for (int i = 0, idx = t; idx < 512; ++i, idx += 256) {
     const int rr = idx >> 3, k8 = idx & 7;
     float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if ((k8 >> 1) <= (rr >> 4)) {
@@ -324,7 +381,20 @@ __device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* 
       y[0] = t0.x * b0.x; y[1] = t0.y * b0.y; y[2] = t0.z * b0.z; y[3] = t0.w * b0.w;
       y[4] = t1.x * b1.x; y[5] = t1.y * b1.y; y[6] = t1.z * b1.z; y[7] = t1.w * b1.w;
     }
-    *reinterpret_cast<uint4*>(Tt + ptx::sw128_chunk(rr, k8)) = pack8(y);
+    const uint4 hi = pack8(y);
+    *reinterpret_cast<uint4*>(Tt + ptx::sw128_chunk(rr, k8)) = hi;
+    if (Tlo) {
+      float r[8];
+      unpack8(hi, r);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r[e] = y[e] - r[e];
+      lo_w[i] = pack8(r);
+    }
+  }
+  if (Tlo) {
+    sync();  // every read of Ts is done
+    for (int i = 0, idx = t; idx < 512; ++i, idx += 256)
+      *reinterpret_cast<uint4*>(Tlo + ptx::sw128_chunk(idx >> 3, idx & 7)) = lo_w[i];
   }
 }
 
@@ -786,7 +856,7 @@ __global__ void __launch_bounds__(256, 2)
   // ---- 5. T = (I + A)^{-1} and T diag(beta) in bf16
   solve_t_beta(reinterpret_cast<const float*>(sm + KA_AS), reinterpret_cast<float*>(sm + KA_TS),
                reinterpret_cast<float*>(sm + KA_MT), s_beta, sm + KA_TT, tid, warp, lane,
-               [] { __syncthreads(); });
+               [] { __syncthreads(); }, [](bool p) { return __syncthreads_or(p) != 0; });
 
   // ---- 6. W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
   ptx::fence_proxy_async_smem();
@@ -1173,7 +1243,8 @@ __global__ void __launch_bounds__(256, 2)
 }  // namespace tc
 }  // namespace kda
 
-#include "kda_chunk_ws.cuh"  // warp-specialised chunk-local kernel
+#include "kda_chunk_ws.cuh"     // warp-specialised chunk-local kernel
+#include "kda_chunk_fused.cuh"  // single-pass kernel
 
 namespace kda {
 
@@ -1203,6 +1274,21 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
     }
   }
   return best_L;
+}
+
+// Which tensor-core prefill runs: the single-pass kernel (one CTA per SM takes
+// whole (sequence, head) units) or the two-kernel path (chunk-local kernel over
+// all chunks at once, then the state pass), which alone carries the sequence
+// segments that long sequences with too few units for the GPU need.  `force`:
+// 0 automatic (the single pass unless segments were chosen), 1 single pass,
+// 2 two kernels.  Returns true for the single pass.
+constexpr int kPathAuto = 0, kPathFused = 1, kPathTwoKernel = 2;
+inline bool tc_use_fused(int B, int T, int H, int num_seqs, int sms, int seg_chunks, int force) {
+  if (force == kPathTwoKernel || seg_chunks > 0 || sms <= 0) return false;
+  const long long N = num_seqs > 0 ? num_seqs : B;
+  const long long tokens = (long long)B * T;
+  if (tokens >= (1LL << 31) || N * H >= (1LL << 31)) return false;
+  return force == kPathFused || N * H >= 1;
 }
 
 // Workspace: the per-chunk images, then (segmented runs) the maps [N | M] of

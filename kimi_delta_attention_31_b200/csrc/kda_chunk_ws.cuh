@@ -541,6 +541,10 @@ __global__ void __launch_bounds__(512, 1)
                          s_beta[slot], sm + WS_TT, st, w8, lane, [st] {
                            if (st == kIo) ptx::bulk_wait_read0();
                            ptx::bar_sync(2, 256);
+                         },
+                         [st](bool p) {
+                           if (st == kIo) ptx::bulk_wait_read0();
+                           return ptx::bar_or(2, 256, p);
                          });
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();

@@ -70,13 +70,12 @@ def test_full_replacement_with_repeated_keys(cuda_device, dtype, d, C):
     inp["g"].zero_()
     o, S = _run(inp, C)
     torch.cuda.synchronize()
-    # Conditioning of this case on the bf16 tensor-core path: with one key, beta = 1
-    # and no decay, W = 0 after the first row and each output is the telescoping sum
-    # o_r = (q_r . k) sum_{j <= r} bf16(v_j - v_{j-1}) within a chunk, so the bf16
-    # rounding errors of U add up like a random walk over up to 64 terms:
-    # sqrt(64) * 2^-9 * sqrt(2) ~ 2.2e-2 relative.  The fp32 path keeps 1e-4.
-    tol = 3e-2 if dtype == "bf16" else TOL[inp["q"].dtype]
-    compare_units(inp, o, S, [(0, 0)], tol)
+    # With one key every entry below the diagonal of A is |k|^2, so every
+    # subdiagonal entry of T diag(beta) is the same -|k|^2 and the outputs are
+    # telescoping sums over up to 64 rows: a rounding of T diag(beta) or of the
+    # corrected errors to bf16 would add up coherently.  The tensor-core prefill
+    # feeds both to its MMAs as bf16 hi + lo pairs, so the bf16 tolerance holds.
+    compare_units(inp, o, S, [(0, 0)], TOL[inp["q"].dtype])
     kk = inp["k"][0, 0, 0].float()
     readback = S[0, 0].T @ kk * (1.0 / (kk @ kk))  # S^T k / |k|^2 with |k| ~ 1 after rounding
     ref = inp["v"][0, -1, 0].float()

@@ -1,6 +1,6 @@
-"""GPU parity of the two chunk-local kernels of the tensor-core prefill: the
-warp-specialised one (default for per-channel log-decay gates on the
-one-row-per-sequence layout) and the two-CTA-per-SM one (kda_set_local_kernel(1)).
+"""GPU parity of the two chunk-local kernels of the two-kernel tensor-core
+prefill (kda_set_prefill_path(2)): the warp-specialised one (its default) and
+the two-CTA-per-SM one (kda_set_local_kernel(1)).
 Both against the fp64 oracle, and against each other on the same inputs,
 including launches where chunks past the single-reference decay range
 (log-decay below -80 over the chunk on some channel) are mixed in at random,
@@ -21,10 +21,12 @@ def _both(inp):
     outs = []
     for variant in (0, 1):
         kda.set_local_kernel(variant)
+        kda.set_prefill_path(kda.PATH_TWO_KERNEL)
         try:
             o, S = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp.get("S0"), None, 64)
         finally:
             kda.set_local_kernel(0)
+            kda.set_prefill_path(kda.PATH_AUTO)
         torch.cuda.synchronize()
         assert kda.device_error() == 0
         outs.append((o, S))
@@ -77,10 +79,12 @@ def _both_fn(fn):
     outs = []
     for variant in (0, 1):
         kda.set_local_kernel(variant)
+        kda.set_prefill_path(kda.PATH_TWO_KERNEL)
         try:
             o, S = fn()
         finally:
             kda.set_local_kernel(0)
+            kda.set_prefill_path(kda.PATH_AUTO)
         torch.cuda.synchronize()
         assert kda.device_error() == 0
         outs.append((o, S))
