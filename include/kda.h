@@ -254,8 +254,11 @@ kda_status_t kda_chunk_fwd_host(const void* q, const void* k, const void* v, con
  * Its scratch is a fixed array inside the library, KDA_NOALLOC_SCRATCH_BYTES
  * bytes on every GPU that loads the library, held until process exit.  Sizes
  * whose kda_chunk_fwd_workspace_size(...) exceeds it are rejected with
- * KDA_ERR_WORKSPACE (64 MiB holds 903 (chunk, head) pairs of the tensor-core
- * path, e.g. B=1, H=8, T=7168; the fp32-arithmetic path needs none).
+ * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill needs 256 + 4 *
+ * num_seqs bytes, the fp32-arithmetic path none; only the two-kernel path
+ * (long sequences split into segments, or kda_set_prefill_path(2)) keeps a
+ * per-chunk image and can exceed it: 64 MiB hold 903 of its (chunk, head)
+ * pairs, e.g. B=1, H=8, T=7168.
  * The first call on each device looks up the array's device address (with
  * that device current) and remembers it together with the CUDA context that
  * was current; a call from another context on that device (a driver-API

@@ -43,10 +43,12 @@
 // Hand-offs (mbarriers; slot = chunk index mod 2):
 //   g_full        TMA of the raw gate rows (issued by builder thread 0 for the
 //                 next chunk once the group has read the current one)
-//   kqv_full[s]   TMA of k, q (128-byte swizzled, straight into the operand
-//                 panels) and V; issued by the state thread for chunk n+2 as
-//                 soon as chunk n's X^T MMA has read the panels and R^T is
-//                 formed; waited by the builder (k, q) and the state (V)
+//   kq_full[s]    TMA of k, q (128-byte swizzled, straight into the operand
+//                 panels), issued by the state thread for chunk n+2 as soon as
+//                 chunk n's X^T MMA has read the panels; waited by the builder
+//   v_full[s]     TMA of V, issued by the state thread for chunk n+1 at the
+//                 start of chunk n (the slot held chunk n-1's V and then its
+//                 output tile, whose stores have read it by then)
 //   a_done[s]     [A'; P'] MMA complete + builder arrive        -> solver
 //   s_ready[s]    solver done (P, T diag(beta) in shared memory)  -> state,
 //                 and -> builder (TMEM slot free for chunk n+2)
@@ -76,7 +78,8 @@ using ws::wait_or_abort;
 constexpr uint32_t FU_L3 = 0;          // 2 slots x 32768: [K e^G; Q e^G] K-major, 2 panels [128 rows][128 B]
 constexpr uint32_t FU_L3_SLOT = 32768;
 constexpr uint32_t FU_RB = 65536;      // 2 slots x 16384: K e^-G (or Kbar) K-major, 2 panels [64 rows][128 B]
-constexpr uint32_t FU_V = 98304;       // 2 slots x 16384: V [64 tokens][128 dv] bf16 row-major
+constexpr uint32_t FU_V = 98304;       // 2 slots x 16384: V [64 tokens][128 dv] bf16 row-major; after R
+                                       // the chunk's output tile (same layout), stored row by row
 constexpr uint32_t FU_P = 131072;      // 2 slots x 8192: P bf16 K-major [64 r][64 j]
 constexpr uint32_t FU_RAWG = 147456;   // raw gate rows [64][128] fp32 (bf16 logits: 16 KB); then the
                                        // group's warp totals [8][128] fp32; steep chunks: left operand
@@ -118,7 +121,7 @@ template <int kGate>
 constexpr uint32_t g_bytes() {
   return kGate == kGateLogTok ? 0u : kGate == kGateLogitBf16 ? C * D * 2 : C * D * 4;
 }
-constexpr uint32_t kKqvBytes = 4 * 8192 + 16384;
+constexpr uint32_t kKqBytes = 4 * 8192, kVBytes = 16384;
 
 // The two bf16 of a 32-bit word as floats (element 2i in the low half).
 __device__ __forceinline__ float2 bf2(uint32_t w) {
@@ -156,6 +159,7 @@ template <int kGate, bool kPacked>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fused_prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
+                             const __grid_constant__ CUtensorMap tm_o,
                              const void* __restrict__ gate, const float* __restrict__ beta,
                              const float* __restrict__ S0, bf16* __restrict__ o, float* __restrict__ S_out,
                              const int32_t* __restrict__ cu_seqlens, int N, int T, int H,
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(16) float s_gref[4][D];   // G at the end of each 16-token block (steep chunks)
   __shared__ float s_nrm[2][C];                  // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
   __shared__ FuItem s_ring[8];
-  __shared__ __align__(8) uint64_t s_g_full, s_kqv_full[2], s_a_done[2], s_s_ready[2], s_rb_free[2];
+  __shared__ __align__(8) uint64_t s_g_full, s_kq_full[2], s_v_full[2], s_a_done[2], s_s_ready[2], s_rb_free[2];
   __shared__ __align__(8) uint64_t s_e_done, s_m1, s_m3, s_st, s_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -243,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     ptx::mbar_init(&s_g_full, 1);
     for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&s_kqv_full[i], 1);
+      ptx::mbar_init(&s_kq_full[i], 1);
+      ptx::mbar_init(&s_v_full[i], 1);
       ptx::mbar_init(&s_a_done[i], 2);
       ptx::mbar_init(&s_s_ready[i], 1);
       ptx::mbar_init(&s_rb_free[i], 1);
@@ -265,25 +270,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s_tmem;
 
   // TMA of chunk item n's k, q (two 64-channel boxes each, swizzled into the
-  // operand panels) and V into slot n & 1; an empty chunk completes the phase
-  // with a plain arrive, the end of the work issues nothing.
-  auto issue_kqv = [&](uint32_t n, uint32_t* issued) {
+  // operand panels of slot n & 1), and of its V (slot n & 1); an empty chunk
+  // completes the phase with a plain arrive, the end of the work issues nothing.
+  auto issue_kq = [&](uint32_t n, uint32_t* issued) {
     const FuItem it = s_ring[n & 7];
     if (it.flags & kItEnd) return;
     const int s = n & 1;
     ++issued[s];
     if ((it.flags & kItEmpty) || *abort_flag) {
-      ptx::mbar_arrive(&s_kqv_full[s]);
+      ptx::mbar_arrive(&s_kq_full[s]);
       return;
     }
     const int h = it.unit % H;
     uint8_t* l3 = sm + FU_L3 + s * FU_L3_SLOT;
-    ptx::mbar_arrive_expect_tx(&s_kqv_full[s], kKqvBytes);
-    ptx::tma_load_3d(l3, &tm_k, 0, h, (int)it.s0, &s_kqv_full[s]);
-    ptx::tma_load_3d(l3 + 16384, &tm_k, 64, h, (int)it.s0, &s_kqv_full[s]);
-    ptx::tma_load_3d(l3 + 8192, &tm_q, 0, h, (int)it.s0, &s_kqv_full[s]);
-    ptx::tma_load_3d(l3 + 16384 + 8192, &tm_q, 64, h, (int)it.s0, &s_kqv_full[s]);
-    ptx::tma_load_3d(sm + FU_V + s * 16384, &tm_v, 0, h, (int)it.s0, &s_kqv_full[s]);
+    ptx::mbar_arrive_expect_tx(&s_kq_full[s], kKqBytes);
+    ptx::tma_load_3d(l3, &tm_k, 0, h, (int)it.s0, &s_kq_full[s]);
+    ptx::tma_load_3d(l3 + 16384, &tm_k, 64, h, (int)it.s0, &s_kq_full[s]);
+    ptx::tma_load_3d(l3 + 8192, &tm_q, 0, h, (int)it.s0, &s_kq_full[s]);
+    ptx::tma_load_3d(l3 + 16384 + 8192, &tm_q, 64, h, (int)it.s0, &s_kq_full[s]);
+  };
+  auto issue_v = [&](uint32_t n, uint32_t* issued) {
+    const FuItem it = s_ring[n & 7];
+    if (it.flags & kItEnd) return;
+    const int s = n & 1;
+    ++issued[s];
+    if ((it.flags & kItEmpty) || *abort_flag) {
+      ptx::mbar_arrive(&s_v_full[s]);
+      return;
+    }
+    ptx::mbar_arrive_expect_tx(&s_v_full[s], kVBytes);
+    ptx::tma_load_3d(sm + FU_V + s * 16384, &tm_v, 0, it.unit % H, (int)it.s0, &s_v_full[s]);
   };
   // TMA of item n's raw gate rows (per-channel gates only).
   auto issue_g = [&](uint32_t n, uint32_t* issued) {
@@ -299,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tma_load_3d(sm + FU_RAWG, &tm_g, 0, it.unit % H, (int)it.s0, &s_g_full);
     }
   };
-  uint32_t g_issued = 0, kqv_issued[2] = {0u, 0u};
+  uint32_t g_issued = 0, kq_issued[2] = {0u, 0u}, v_issued[2] = {0u, 0u};
   bool mma_issued = false;  // by this thread (builder thread 0, state thread 0)
 
   if (warp < 8) {
@@ -356,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // it, so that the whole group leaves together after a timeout.
       bool ok = true;
       if constexpr (kTmaGate) ok = wait_or_abort(&s_g_full, n & 1, abort_flag);
-      if constexpr (kPrep) ok = ok && wait_or_abort(&s_kqv_full[s], (n >> 1) & 1, abort_flag);
+      if constexpr (kPrep) ok = ok && wait_or_abort(&s_kq_full[s], (n >> 1) & 1, abort_flag);
 
       // ---- raw gate rows -> local cumulative sums; rows >= Cn contribute g = 0
       float G[4][8];
@@ -468,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (fast && tid == 0) issue_g(n + 1, &g_issued);
 
       ok = true;
-      if constexpr (!kPrep) ok = wait_or_abort(&s_kqv_full[s], (n >> 1) & 1, abort_flag);
+      if constexpr (!kPrep) ok = wait_or_abort(&s_kq_full[s], (n >> 1) & 1, abort_flag);
       // K e^-G, gamma of this slot: the state is done with chunk n-2
       if (n >= 2) ok = ok && wait_or_abort(&s_rb_free[s], ((n - 2) >> 1) & 1, abort_flag);
       if (ptx::bar_or(1, 256, !ok || *abort_flag)) break;
@@ -672,15 +688,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int dv = 32 * qd + lane;  // this thread's value channel = its TMEM lane
     const uint32_t lo_lane = (uint32_t)(32 * qd) << 16;
     if (st == 0) {
-      issue_kqv(0, kqv_issued);
-      issue_kqv(1, kqv_issued);
+      issue_kq(0, kq_issued);
+      issue_kq(1, kq_issued);
+      issue_v(0, v_issued);
+      issue_v(1, v_issued);
     }
     uint32_t real = 0;  // chunks with MMAs (phases of m1, e_done, m3)
     for (uint32_t n = 0;; ++n) {
       const int s = n & 1;
       const bool okr = wait_or_abort(&s_s_ready[s], (n >> 1) & 1, abort_flag);
+      ptx::bulk_wait_read0();  // this thread's output-row stores of chunk n-1 have read the V slot
       if (ptx::bar_or(3, 128, !okr || *abort_flag)) break;  // uniform over the group
       ptx::tc_fence_after();
+      if (st == 0 && n >= 1) issue_v(n + 1, v_issued);  // into chunk n-1's slot
       const FuItem it = s_ring[n & 7];
       if (it.flags & kItEnd) break;
       const size_t urow = (size_t)it.unit * D;  // first state row of the unit
@@ -688,7 +708,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (S_out)
           for (int c = 0; c < D; ++c) S_out[(urow + c) * D + dv] = S0 ? S0[(urow + c) * D + dv] : 0.f;
         if (st == 0) {
-          issue_kqv(n + 2, kqv_issued);
+          issue_kq(n + 2, kq_issued);
           ptx::mbar_arrive(&s_rb_free[s]);
         }
         continue;
@@ -736,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       bool ok = wait_or_abort(&s_m1, real & 1, abort_flag);
-      ok = ok && wait_or_abort(&s_kqv_full[s], (n >> 1) & 1, abort_flag);  // V
+      ok = ok && wait_or_abort(&s_v_full[s], (n >> 1) & 1, abort_flag);
       ptx::tc_fence_after();
       // ---- R^T = V^T - (K e^G S)^T in fp32 (tokens j >= Cn zero) as bf16 hi | lo
       const bf16* vs = reinterpret_cast<const bf16*>(sm + FU_V + s * 16384) + dv;
@@ -756,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       if (ptx::bar_or(3, 128, !ok || *abort_flag)) break;  // R^T stored; this slot's panels and V are free
       if (st == 0) {
-        issue_kqv(n + 2, kqv_issued);
+        issue_kq(n + 2, kq_issued);
         // ---- E^T = R^T (T diag(beta))^T  (N=64, K=64), over (K e^G S)^T, from
         //      the hi + lo pairs: R_hi T_hi + R_lo T_hi + R_hi T_lo
         ptx::tc_fence_after();
@@ -818,20 +838,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 16; ++i) w[i] = ptx::pack_bf16x2(x[2 * i], x[2 * i + 1]);
         ptx::tmem_st16u(tmem + lo_lane + kTmSb + c32 / 2, w);
       }
-      float ov[64];
-      ld32(tmem + lo_lane + kTmO, ov);
-      ld32(tmem + lo_lane + kTmO + 32, ov + 32);
-      ptx::tmem_wait_ld();
+      // the output tile, [64 tokens][128 dv] bf16, over this slot's V (read by R)
+      bf16* otile = reinterpret_cast<bf16*>(sm + FU_V + s * 16384);
+#pragma unroll 1
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float x[32];
+        ld32(tmem + lo_lane + kTmO + 32 * h2, x);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) otile[(32 * h2 + e) * D + dv] = __float2bfloat16_rn(x[e]);
+      }
+      ptx::fence_proxy_async_smem();
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::bar_sync(3, 128);  // every read of this slot's K e^-G, P, gamma and of X^T done
+      ptx::bar_sync(3, 128);  // every read of this slot's K e^-G, P, gamma and of X^T done; tile complete
       if (st == 0) ptx::mbar_arrive(&s_rb_free[s]);
-      const int h = it.unit % H;
-      bf16* orow = o + ((size_t)it.s0 * H + h) * D + dv;
-      const size_t ostride = (size_t)H * D;
-#pragma unroll
-      for (int r = 0; r < 64; ++r)
-        if (r < it.Cn) orow[r * ostride] = __float2bfloat16_rn(ov[r]);
+      if (it.Cn == C) {  // a whole chunk: one tensor store
+        if (st == 0) {
+          ptx::tma_store_3d(&tm_o, 0, it.unit % H, (int)it.s0, otile);
+          ptx::bulk_commit();
+        }
+      } else if (st < it.Cn) {  // the ragged last chunk of a sequence: one 256-byte row per thread
+        ptx::bulk_s2g(o + ((size_t)(it.s0 + st) * H + it.unit % H) * D, otile + st * D, D * 2);
+        ptx::bulk_commit();
+      }
       if ((it.flags & kItLast) && S_out) {
 #pragma unroll 1
         for (int c32 = 0; c32 < D; c32 += 32) {
@@ -844,6 +874,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++real;
     }
+    ptx::bulk_wait0();  // the output rows have landed
   }
 
   // After a timeout: wait (bounded again) for the copies and MMAs still in
@@ -853,8 +884,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (s_abort) {
     if (tid == 0 && g_issued) ptx::mbar_wait_bounded(&s_g_full, (g_issued - 1) & 1, 1000000000ull);
     if (tid == 512)
-      for (int i = 0; i < 2; ++i)
-        if (kqv_issued[i]) ptx::mbar_wait_bounded(&s_kqv_full[i], (kqv_issued[i] - 1) & 1, 1000000000ull);
+      for (int i = 0; i < 2; ++i) {
+        if (kq_issued[i]) ptx::mbar_wait_bounded(&s_kq_full[i], (kq_issued[i] - 1) & 1, 1000000000ull);
+        if (v_issued[i]) ptx::mbar_wait_bounded(&s_v_full[i], (v_issued[i] - 1) & 1, 1000000000ull);
+      }
   }
   __syncthreads();
   if (s_abort && (tid == 0 || tid == 512)) {  // the two MMA-issuing threads
@@ -952,7 +985,8 @@ inline cudaError_t launch_fused_t(const bf16* q, const bf16* k, const bf16* v, c
   cudaError_t e = ws::tensor_map_encoder(&enc);
   if (e != cudaSuccess) return e;
   const long long tokens = (long long)B * T;
-  CUtensorMap mk, mq, mg, mv;
+  CUtensorMap mk, mq, mg, mv, mo;
+  if ((e = ws::encode_rows_map(enc, &mo, o, false, tokens, H, D, false)) != cudaSuccess) return e;
   if ((e = ws::encode_rows_map(enc, &mk, k, false, tokens, H, 64, true)) != cudaSuccess) return e;
   if ((e = ws::encode_rows_map(enc, &mq, q, false, tokens, H, 64, true)) != cudaSuccess) return e;
   if ((e = ws::encode_rows_map(enc, &mv, v, false, tokens, H, D, false)) != cudaSuccess) return e;
@@ -972,10 +1006,10 @@ inline cudaError_t launch_fused_t(const bf16* q, const bf16* k, const bf16* v, c
   if (grid <= 0) return cudaSuccess;
   if (cu_seqlens)
     kda_fused_prefill_kernel<kGate, true><<<grid, kThreads, FU_DYN, stream>>>(
-        mk, mq, mg, mv, g, beta, S0, o, S_out, cu_seqlens, N, T, H, ctr, order, status);
+        mk, mq, mg, mv, mo, g, beta, S0, o, S_out, cu_seqlens, N, T, H, ctr, order, status);
   else
     kda_fused_prefill_kernel<kGate, false><<<grid, kThreads, FU_DYN, stream>>>(
-        mk, mq, mg, mv, g, beta, S0, o, S_out, nullptr, N, T, H, ctr, nullptr, status);
+        mk, mq, mg, mv, mo, g, beta, S0, o, S_out, nullptr, N, T, H, ctr, nullptr, status);
   return cudaGetLastError();
 }
 

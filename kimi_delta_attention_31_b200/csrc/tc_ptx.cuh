@@ -118,6 +118,14 @@ __device__ __forceinline__ void bulk_s2g(void* dst_gmem, const void* src_smem, u
                "r"(smem_u32(src_smem)), "r"(bytes)
                : "memory");
 }
+// Tiled tensor copy shared -> global through a tensor map (bulk-group
+// completion), three coordinates, innermost first; elements outside the
+// tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const void* tmap, int c0, int c1, int c2, const void* src_smem) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(tmap),
+               "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(src_smem))
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // The issuing thread's bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read0() {

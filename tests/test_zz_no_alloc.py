@@ -43,10 +43,22 @@ def test_noalloc_packed_sequences(cuda_device):
 
 
 def test_noalloc_at_its_documented_limit(cuda_device):
-    # B=1, H=8, T=7168: 112 chunks x 8 heads, the largest case named in kda.h
-    need = kda.workspace_size(1, 7168, 8, 128, 128, 0, 64, torch.bfloat16)
-    assert 0 < need <= kda.NOALLOC_SCRATCH_BYTES
-    x = W.make_prefill(1, 7168, 8, 128, 128, "bf16", -4.0, 1.0, 0.02, seed=905, device=cuda_device)
+    # the two-kernel path keeps a per-chunk image: B=1, H=8, T=7168 (112 chunks x
+    # 8 heads) is the largest case kda.h names for it
+    kda.set_prefill_path(kda.PATH_TWO_KERNEL)
+    try:
+        need = kda.workspace_size(1, 7168, 8, 128, 128, 0, 64, torch.bfloat16)
+        assert 0 < need <= kda.NOALLOC_SCRATCH_BYTES
+        x = W.make_prefill(1, 7168, 8, 128, 128, "bf16", -4.0, 1.0, 0.02, seed=905, device=cuda_device)
+        _same(x, *_both(x))
+    finally:
+        kda.set_prefill_path(kda.PATH_AUTO)
+
+
+def test_noalloc_single_pass_at_the_benchmark_size(cuda_device):
+    # the single-pass prefill needs only a unit counter: B8 H32 T8192 fits easily
+    assert kda.workspace_size(8, 8192, 32, 128, 128, 0, 64, torch.bfloat16) <= 4096
+    x = W.make_prefill(8, 8192, 32, 128, 128, "bf16", -5.0, 1.5, 0.0, seed=907, device=cuda_device)
     _same(x, *_both(x))
 
 
