@@ -8,8 +8,8 @@
 // Within a chunk entering with state S (fp32, dk x dv), chunk-relative
 // cumulative log-decays G (fp32) and T = (I + A)^{-1} as in kda_chunk_tc.cuh,
 // the kernel evaluates
-//   R = V - (K o e^G) S,           E = T diag(beta) R             (= U - W S)
-//   O = (Q o e^G) S + P E,          S <- (S + (K o e^-G)^T E) o e^{G_last}
+//   W = T diag(beta) (K o e^G),  U = T diag(beta) V,  E = U - W S   (the WY form)
+//   O = (Q o e^G) S + P E,       S <- (S + (K o e^-G)^T E) o e^{G_last}
 // (the last line is Diag(e^{G_last}) S + (K o e^{G_last - G})^T E with the
 // decay applied after the sum; chunks whose decay leaves that range use
 // Kbar = K o e^{G_last - G} and decay first).  Nothing of a chunk goes to HBM
@@ -23,44 +23,48 @@
 //                          operands [K e^G; Q e^G] (written over the raw k, q
 //                          rows in place) and K e^-G, the [A'; P'] MMA.
 //   solver  (warps 8..15)  chunk n+1: A and P out of TMEM, T = (I + A)^{-1},
-//                          T diag(beta) in bf16.
+//                          T diag(beta) as a bf16 pair hi + lo, then two MMA
+//                          groups: W^T into the chunk's [A'; P'] columns (read
+//                          back and written, negated, in bf16 over the K e^G
+//                          rows) and U^T straight into the state's columns.
 //   state   (warps 16..19) chunk n: the state in TMEM, TRANSPOSED (lane = value
 //                          channel), so that every state-side product is an MMA
 //                          whose A operand sits in TMEM:
-//       X^T   = S^T [K e^G; Q e^G]^T          (M=128, N=128, K=128)
-//       R^T   = V^T - X^T[:, 0:64]            (threads, fp32 -> bf16 hi + lo)
-//       E^T   = R^T (T diag(beta))^T          (N=64, K=64, hi and lo)
-//       S^T  += E^T (K e^-G),  X^T[:, 64:128] += E^T P^T  (hi and lo)
-//       S^T  *= e^{G_last} per key channel;  o = X^T[:, 64:128]
-// R and E enter the MMAs as a bf16 pair hi + lo (lo = the rounding error of
-// hi), so their fp32 values are used to about 2^-16; S enters in bf16.
+//       E^T   = U^T + S^T (-W)^T,  (Q e^G S)^T    (N=64 each, K=128)
+//       S^T  += E^T (K e^-G),  (Q e^G S)^T += E^T P^T   (E as bf16 hi + lo)
+//       S^T  *= e^{G_last} per key channel;  o = the second product
+// E enters the MMAs as a bf16 pair hi + lo (lo = the rounding error of hi),
+// so its fp32 value is used to about 2^-16; U is exact to fp32 accumulation;
+// W and S enter in bf16.
 //
-// TMEM columns: [A'; P'] slot 0 (0..63) | slot 1 (64..127) | X^T (128..255:
-// (K e^G S)^T in 128..191, where E^T lands next, and (Q e^G S)^T -> O^T in
-// 192..255) | bf16 hi | lo of R^T, then of E^T (256..319) | S^T bf16
-// (320..383) | S^T fp32 (384..511).
+// TMEM columns: [A'; P'] slot 0 (0..63) | slot 1 (64..127) (also the W^T
+// accumulator) | U^T -> E^T (128..191) | (Q e^G S)^T -> O^T (192..255) | bf16
+// hi | lo of E^T (256..319) | S^T bf16 (320..383) | S^T fp32 (384..511).
 //
 // Hand-offs (mbarriers; slot = chunk index mod 2):
 //   g_full        TMA of the raw gate rows (issued by builder thread 0 for the
 //                 next chunk once the group has read the current one)
 //   kq_full[s]    TMA of k, q (128-byte swizzled, straight into the operand
 //                 panels), issued by the state thread for chunk n+2 as soon as
-//                 chunk n's X^T MMA has read the panels; waited by the builder
+//                 chunk n's E MMA has read the panels; waited by the builder
 //   v_full[s]     TMA of V, issued by the state thread for chunk n+1 at the
 //                 start of chunk n (the slot held chunk n-1's V and then its
-//                 output tile, whose stores have read it by then)
+//                 output tile, whose stores have read it by then); waited by
+//                 the solver before the U MMA
 //   a_done[s]     [A'; P'] MMA complete + builder arrive        -> solver
-//   s_ready[s]    solver done (P, T diag(beta) in shared memory)  -> state,
+//   s_ready[s]    solver done (P, -W in shared memory, U^T in TMEM) -> state,
 //                 and -> builder (TMEM slot free for chunk n+2)
-//   rb_free[s]    state done with chunk n (MMAs read K e^-G, P; gamma read)
-//                 -> builder (K e^-G, gamma of chunk n+2), solver (P of n+2)
-//   e_done        the E MMA of the previous chunk done -> solver may rewrite
-//                 T diag(beta)
-//   m1, m3, st    MMA completions inside one group.
+//   rb_free[s]    state's MMAs of chunk n done (K e^-G and P read) -> builder
+//                 (K e^-G of chunk n+2), solver (P of n+2); gamma has four
+//                 slots, so the builder of chunk n+2 never meets chunk n's
+//   x_free        the state has read chunk n's E^T -> the solver's U MMA of
+//                 the next chunk may write those columns
+//   uw_done, m1, m3, st   MMA completions inside one group.
 // Chunk descriptors travel in an 8-entry ring written by builder thread 0
-// three chunks ahead.  Every wait is bounded; after a timeout every group
-// leaves its loop, the copies still in flight are waited for (bounded), TMEM
-// is freed and the kernel returns with the device error word set.
+// three chunks ahead.  Every wait is bounded, and every group leaves its loop
+// by a group-wide vote, so that after a timeout the whole group stops
+// together; the copies still in flight are then waited for (bounded), TMEM is
+// freed and the kernel returns with the device error word set.
 //
 // Included by kda_chunk_tc.cuh after the warp-specialised kernel (it uses
 // the tensor-map helpers and the shared solve).
@@ -78,23 +82,26 @@ using ws::wait_or_abort;
 constexpr uint32_t FU_L3 = 0;          // 2 slots x 32768: [K e^G; Q e^G] K-major, 2 panels [128 rows][128 B]
 constexpr uint32_t FU_L3_SLOT = 32768;
 constexpr uint32_t FU_RB = 65536;      // 2 slots x 16384: K e^-G (or Kbar) K-major, 2 panels [64 rows][128 B]
-constexpr uint32_t FU_V = 98304;       // 2 slots x 16384: V [64 tokens][128 dv] bf16 row-major; after R
-                                       // the chunk's output tile (same layout), stored row by row
-constexpr uint32_t FU_P = 131072;      // 2 slots x 8192: P bf16 K-major [64 r][64 j]
+constexpr uint32_t FU_V = 98304;       // 2 slots x 16384: V, two 64-channel panels [64 tokens][128 B]
+constexpr uint32_t FU_P = 131072;      // 2 slots x 8192: P bf16 K-major [64 r][64 j]; once read, the
+                                       // chunk's output tile, value channels 0..63 ([64 tokens][128 B])
 constexpr uint32_t FU_RAWG = 147456;   // raw gate rows [64][128] fp32 (bf16 logits: 16 KB); then the
                                        // group's warp totals [8][128] fp32; steep chunks: left operand
-constexpr uint32_t FU_AS = 180224;     // A fp32 [64][68]
-constexpr uint32_t FU_TS = 197632;     // T fp32 [64][68]; after the solve the lo part of T diag(beta)
-constexpr uint32_t FU_TT = 215040;     // T diag(beta) bf16 (hi) K-major [64][64]; block products during the solve
-constexpr uint32_t FU_GAM = 223232;    // 2 slots x 512: gamma = e^{G_last} fp32 [128]
+constexpr uint32_t FU_AS = 180224;     // A fp32 [64][68], then T over it
+constexpr uint32_t FU_TLO = 197632;    // T diag(beta) bf16, lo part, K-major [64][64]
+constexpr uint32_t FU_TT = 205824;     // T diag(beta) bf16, hi part, K-major [64][64]
+constexpr uint32_t FU_GAM = 214016;    // 4 slots x 512: gamma = e^{G_last} fp32 [128] (chunk n in slot n mod 4)
+constexpr uint32_t FU_OST = 216064;    // the output tile, value channels 64..127 ([64 tokens][128 B])
 constexpr uint32_t FU_BYTES = 224256;
 constexpr uint32_t FU_DYN = FU_BYTES + 1024;
 static_assert(FU_L3 + 2 * FU_L3_SLOT == FU_RB && FU_RB + 2 * 16384 == FU_V && FU_V + 2 * 16384 == FU_P &&
-                  FU_P + 2 * 8192 == FU_RAWG && FU_RAWG + 32768 == FU_AS && FU_AS + 17408 == FU_TS &&
-                  FU_TS + 17408 == FU_TT && FU_TT + 8192 == FU_GAM && FU_GAM + 1024 == FU_BYTES,
+                  FU_P + 2 * 8192 == FU_RAWG && FU_RAWG + 32768 == FU_AS && FU_AS + 17408 == FU_TLO &&
+                  FU_TLO + 8192 == FU_TT && FU_TT + 8192 == FU_GAM && FU_GAM + 2048 == FU_OST &&
+                  FU_OST + 8192 == FU_BYTES,
               "layout");
-static_assert(FU_RB % 1024 == 0 && FU_P % 1024 == 0 && FU_RAWG % 1024 == 0 && FU_TT % 1024 == 0, "alignment");
-static_assert(3 * 16 * tc::MT_LD * 4 <= 8192 && 8 * D * 4 <= 32768, "scratch sizes");
+static_assert(FU_RB % 1024 == 0 && FU_P % 1024 == 0 && FU_RAWG % 1024 == 0 && FU_TLO % 1024 == 0 &&
+                  FU_TT % 1024 == 0 && FU_OST % 1024 == 0, "alignment");
+static_assert(8 * D * 4 <= 32768, "scratch sizes");
 
 // ------------------------------------------------------------------ TMEM
 constexpr uint32_t kTmCols = 512;
@@ -104,7 +111,7 @@ constexpr uint32_t kTmHL = 256;  // bf16 hi (256..287) and lo (288..319) of R^T,
 constexpr uint32_t kTmSb = 320;  // S^T bf16
 constexpr uint32_t kTmS = 384;   // S^T fp32
 
-constexpr int kThreads = 640;
+constexpr int kThreads = 640;  // builder 256, solver 256, state 128
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Chunk descriptor.
@@ -155,6 +162,15 @@ __device__ __forceinline__ void store_hi_lo32(uint32_t base, int h, const float*
   ptx::tmem_st16u(base + 32 + 16 * h, lo);
 }
 
+// Zeroes 64 fp32 TMEM columns [ta, ta + 64) of the calling warp's 32 lanes.
+__device__ __forceinline__ void zero_cols64(uint32_t ta) {
+  float z[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) z[i] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ptx::tmem_st16(ta + 16 * i, z);
+}
+
 template <int kGate, bool kPacked>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fused_prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -173,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ float s_nrm[2][C];                  // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
   __shared__ FuItem s_ring[8];
   __shared__ __align__(8) uint64_t s_g_full, s_kq_full[2], s_v_full[2], s_a_done[2], s_s_ready[2], s_rb_free[2];
-  __shared__ __align__(8) uint64_t s_e_done, s_m1, s_m3, s_st, s_drain;
+  __shared__ __align__(8) uint64_t s_x_free, s_uw_done, s_m1, s_m3, s_st, s_drain, s_p_free[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   // packed sequences whose cu_seqlens the set-up kernel rejected: no work at all
@@ -252,12 +268,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&s_a_done[i], 2);
       ptx::mbar_init(&s_s_ready[i], 1);
       ptx::mbar_init(&s_rb_free[i], 1);
+      ptx::mbar_init(&s_p_free[i], 1);
     }
-    ptx::mbar_init(&s_e_done, 1);
+    ptx::mbar_init(&s_x_free, 1);
+    ptx::mbar_init(&s_uw_done, 1);
     ptx::mbar_init(&s_m1, 1);
     ptx::mbar_init(&s_m3, 1);
     ptx::mbar_init(&s_st, 1);
-    ptx::mbar_init(&s_drain, 2);
+    ptx::mbar_init(&s_drain, 3);
     s_abort = 0;
     ptx::fence_mbar_init();
     g_c = g_nc = g_len = g_unit = g_done = 0;
@@ -300,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::mbar_arrive_expect_tx(&s_v_full[s], kVBytes);
     ptx::tma_load_3d(sm + FU_V + s * 16384, &tm_v, 0, it.unit % H, (int)it.s0, &s_v_full[s]);
+    ptx::tma_load_3d(sm + FU_V + s * 16384 + 8192, &tm_v, 64, it.unit % H, (int)it.s0, &s_v_full[s]);
   };
   // TMA of item n's raw gate rows (per-channel gates only).
   auto issue_g = [&](uint32_t n, uint32_t* issued) {
@@ -315,8 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tma_load_3d(sm + FU_RAWG, &tm_g, 0, it.unit % H, (int)it.s0, &s_g_full);
     }
   };
+  bool mma_issued = false;  // by this thread (builder, solver, state thread 0)
+  // copies issued per barrier phase stream (builder thread 0: g; state thread 0: k, q;
+  // solver thread 224: V)
   uint32_t g_issued = 0, kq_issued[2] = {0u, 0u}, v_issued[2] = {0u, 0u};
-  bool mma_issued = false;  // by this thread (builder thread 0, state thread 0)
 
   if (warp < 8) {
     // ============================== builder ==============================
@@ -330,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm_q);
       if constexpr (kTmaGate) ptx::prefetch_tmap(&tm_g);
       ptx::prefetch_tmap(&tm_v);
+      ptx::prefetch_tmap(&tm_o);
       issue_g(0, &g_issued);
     }
     uint32_t st_round = 0;  // completions of s_st
@@ -481,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // uniform over the group; s_glast, s_gref visible; s_wtot (the raw gate buffer) read
       const bool fast = !ptx::bar_or(1, 256, steep);
-      if (fast && tid == 0) issue_g(n + 1, &g_issued);
+      if (fast && tid == 0) issue_g(n + 1, &g_issued);  // the raw gate buffer is free
 
       ok = true;
       if constexpr (!kPrep) ok = wait_or_abort(&s_kq_full[s], (n >> 1) & 1, abort_flag);
@@ -614,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float gm[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) gm[e] = expf(s_glast[c0 + e]);
-        float* gam = reinterpret_cast<float*>(sm + FU_GAM + s * 512);
+        float* gam = reinterpret_cast<float*>(sm + FU_GAM + (n & 3) * 512);
         reinterpret_cast<float4*>(gam)[2 * co] = make_float4(gm[0], gm[1], gm[2], gm[3]);
         reinterpret_cast<float4*>(gam)[2 * co + 1] = make_float4(gm[4], gm[5], gm[6], gm[7]);
       }
@@ -652,32 +674,87 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 16) {
     // ============================== solver ==============================
     const int st = tid - 256, w8 = warp - 8;
+    const int qd = warp & 3, ch = w8 >> 2;  // TMEM lane quarter; 32-column half
     float* As = reinterpret_cast<float*>(sm + FU_AS);
-    uint32_t real = 0;  // chunks solved (E MMAs to wait for)
+    constexpr int kVIssuer = 224;  // warp 7 of the group: idle in the middle of the solve
+    if (st == kVIssuer) {
+      ptx::prefetch_tmap(&tm_v);
+      issue_v(0, v_issued);
+    }
+    uint32_t real = 0;  // chunks solved (phases of uw_done and of the state's x_free)
     for (uint32_t n = 0;; ++n) {
       const int s = n & 1;
       bool ok = wait_or_abort(&s_a_done[s], (n >> 1) & 1, abort_flag);
-      // P of this slot: the state is done with chunk n-2
-      if (n >= 2) ok = ok && wait_or_abort(&s_rb_free[s], ((n - 2) >> 1) & 1, abort_flag);
+      // P of this slot: the state is done with chunk n-2's P and output tile
+      if (n >= 2) ok = ok && wait_or_abort(&s_p_free[s], ((n - 2) >> 1) & 1, abort_flag);
       if (ptx::bar_or(2, 256, !ok || *abort_flag)) break;  // uniform over the group
       ptx::tc_fence_after();
       const FuItem it = s_ring[n & 7];
       if (!(it.flags & (kItEnd | kItEmpty))) {
+        uint8_t* l3 = sm + FU_L3 + s * FU_L3_SLOT;
         // scatter A (fp32, beta-scaled) and P (bf16) out of TMEM slot s
-        tc::scatter_single_ref(tmem + 64 * s, s_beta[s], As, sm + FU_P + s * 8192, warp, w8, lane, false);
+        const bool big =
+            tc::scatter_single_ref(tmem + 64 * s, s_beta[s], As, sm + FU_P + s * 8192, warp, w8, lane, false);
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
-        // T diag(beta) and the block products (both in FU_TT): the E MMA of the
-        // previous chunk has read T diag(beta)
-        ok = real == 0 || wait_or_abort(&s_e_done, (real - 1) & 1, abort_flag);
-        if (ptx::bar_or(2, 256, !ok || *abort_flag)) break;
-        // T = (I + A)^{-1}, T diag(beta) as bf16 hi (FU_TT) + lo (over T, FU_TS)
-        tc::solve_t_beta(As, reinterpret_cast<float*>(sm + FU_TS), reinterpret_cast<float*>(sm + FU_TT),
-                         s_beta[s], sm + FU_TT, st, w8, lane, [] { ptx::bar_sync(2, 256); },
-                         [](bool p) { return ptx::bar_or(2, 256, p); }, sm + FU_TS);
+        const bool accurate = ptx::bar_or(2, 256, big);
+        // T = (I + A)^{-1} over A, T diag(beta) as bf16 hi (FU_TT) + lo (FU_TLO)
+        // (V of chunk n+1 into the other slot, whose V chunk n-1's U MMA has read,
+        // from the warp that is idle at that point of the solve)
+        tc::solve_t_beta(As, s_beta[s], sm + FU_TT, sm + FU_TLO, accurate, st, w8, lane,
+                         [] { ptx::bar_sync(2, 256); }, [&] {
+                           if (lane == 0) issue_v(n + 1, v_issued);
+                         });
         ptx::fence_proxy_async_smem();
         ptx::bar_sync(2, 256);
+        // ---- W^T = (K e^G)^T (T diag(beta))^T into TMEM slot s (free since the
+        //      scatter), U^T = V^T (T diag(beta))^T into the state's X^T columns
+        //      (free once the state has split chunk n-1's E): M=128, N=64, K=64,
+        //      T diag(beta) as hi then lo.
+        if (st == 0) {
+          bool go = wait_or_abort(&s_v_full[s], (n >> 1) & 1, abort_flag);
+          go = go && (real == 0 || wait_or_abort(&s_x_free, (real - 1) & 1, abort_flag));
+          if (go) {
+            ptx::tc_fence_after();
+            constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              ptx::mma_bf16(tmem + 64 * s,
+                            ptx::sdesc_sw128(sb + FU_L3 + s * FU_L3_SLOT + (i & 3) * 2048, 16384, 1024),
+                            ptx::sdesc_sw128(sb + (i < 4 ? FU_TT : FU_TLO) + (i & 3) * 32, 16, 1024), id, i > 0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              ptx::mma_bf16(tmem + kTmX, ptx::sdesc_sw128(sb + FU_V + s * 16384 + (i & 3) * 2048, 8192, 1024),
+                            ptx::sdesc_sw128(sb + (i < 4 ? FU_TT : FU_TLO) + (i & 3) * 32, 16, 1024), id, i > 0);
+            mma_issued = true;
+            ptx::mma_commit(&s_uw_done);
+          } else {
+            ptx::mbar_arrive(&s_uw_done);
+          }
+        }
+        ok = wait_or_abort(&s_uw_done, real & 1, abort_flag);
+        ptx::tc_fence_after();
+        // ---- -W (bf16) over the K e^G rows of the slot, in their layout (K-major:
+        //      row = token, key channels 0..63 | 64..127 in the two panels), so that
+        //      the state's first MMA reads [-W; Q e^G] as one 128-row operand
+        {
+          const int c = 32 * qd + lane;  // key channel = TMEM lane
+          float x[32];
+          ld32(tmem + ((uint32_t)(32 * qd) << 16) + 64 * s + 32 * ch, x);
+          ptx::tmem_wait_ld();
+          uint8_t* wcol = l3 + (c >> 6) * 16384 + (c & 7) * 2;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int r = 32 * ch + e;  // token
+            *reinterpret_cast<bf16*>(wcol + r * 128 + (((((c & 63) >> 3) ^ r) & 7) << 4)) = __float2bfloat16_rn(-x[e]);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        if (ptx::bar_or(2, 256, !ok || *abort_flag)) break;
         ++real;
+      } else if (st == kVIssuer) {  // keep V's per-chunk phases in step
+        issue_v(n + 1, v_issued);
       }
       if (st == 0) ptx::mbar_arrive(&s_s_ready[s]);
       if (it.flags & kItEnd) break;
@@ -690,24 +767,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (st == 0) {
       issue_kq(0, kq_issued);
       issue_kq(1, kq_issued);
-      issue_v(0, v_issued);
-      issue_v(1, v_issued);
     }
-    uint32_t real = 0;  // chunks with MMAs (phases of m1, e_done, m3)
+    zero_cols64(tmem + lo_lane + kTmO);  // the first MMA accumulates O onto zeros
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    uint32_t real = 0;  // chunks with MMAs (phases of m1, m3, x_free)
     for (uint32_t n = 0;; ++n) {
       const int s = n & 1;
       const bool okr = wait_or_abort(&s_s_ready[s], (n >> 1) & 1, abort_flag);
-      ptx::bulk_wait_read0();  // this thread's output-row stores of chunk n-1 have read the V slot
+      if (st == 0 && n >= 1) {  // chunk n-1's output tile is read: its P slot and FU_OST are free
+        ptx::bulk_wait_read0();
+        ptx::mbar_arrive(&s_p_free[(n - 1) & 1]);
+      }
       if (ptx::bar_or(3, 128, !okr || *abort_flag)) break;  // uniform over the group
       ptx::tc_fence_after();
-      if (st == 0 && n >= 1) issue_v(n + 1, v_issued);  // into chunk n-1's slot
       const FuItem it = s_ring[n & 7];
       if (it.flags & kItEnd) break;
       const size_t urow = (size_t)it.unit * D;  // first state row of the unit
       if (it.flags & kItEmpty) {  // an empty sequence hands its initial state through
         if (S_out)
           for (int c = 0; c < D; ++c) S_out[(urow + c) * D + dv] = S0 ? S0[(urow + c) * D + dv] : 0.f;
-        if (st == 0) {
+        if (st == 0) {  // keep the per-chunk phases in step
           issue_kq(n + 2, kq_issued);
           ptx::mbar_arrive(&s_rb_free[s]);
         }
@@ -730,20 +810,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_before();
         ptx::bar_sync(3, 128);
       }
-      // ---- X^T = S^T [K e^G; Q e^G]^T  (M=128, N=128, K=128; A in TMEM)
+      // ---- [E^T | (Q e^G S)^T] = [U^T | 0] + S^T [-W; Q e^G]^T  (N=128, K=128: the
+      //      slot's panel rows are -W (tokens 0..63) and Q e^G (64..127), K-major;
+      //      the E half accumulates onto the solver's U^T, the other onto zeros)
       if (st == 0) {
         ptx::tc_fence_after();
         constexpr uint32_t id = ptx::idesc_bf16(128, 128, false, false);
+        const uint32_t l3s = sb + FU_L3 + s * FU_L3_SLOT;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           ptx::mma_bf16_ts(tmem + kTmX, tmem + kTmSb + 8 * kk,
-                           ptx::sdesc_sw128(sb + FU_L3 + s * FU_L3_SLOT + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                           id, kk > 0);
+                           ptx::sdesc_sw128(l3s + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id, 1);
         mma_issued = true;
         ptx::mma_commit(&s_m1);
       }
-      const float* gam = reinterpret_cast<const float*>(sm + FU_GAM + s * 512);
-      if (steep) {  // Kbar form: decay the state first (the MMA above reads only the bf16 copy)
+      const float* gam = reinterpret_cast<const float*>(sm + FU_GAM + (n & 3) * 512);
+      if (steep) {  // Kbar form: decay the state first (the MMAs above read only the bf16 copy)
 #pragma unroll 1
         for (int c32 = 0; c32 < D; c32 += 32) {
           float x[32];
@@ -756,42 +838,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       bool ok = wait_or_abort(&s_m1, real & 1, abort_flag);
-      ok = ok && wait_or_abort(&s_v_full[s], (n >> 1) & 1, abort_flag);
       ptx::tc_fence_after();
-      // ---- R^T = V^T - (K e^G S)^T in fp32 (tokens j >= Cn zero) as bf16 hi | lo
-      const bf16* vs = reinterpret_cast<const bf16*>(sm + FU_V + s * 16384) + dv;
-#pragma unroll 1
-      for (int h2 = 0; h2 < 2; ++h2) {
-        float x[32];
-        ld32(tmem + lo_lane + kTmX + 32 * h2, x);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int j = 32 * h2 + e;
-          x[e] = j < it.Cn ? __bfloat162float(vs[j * D]) - x[e] : 0.f;
-        }
-        store_hi_lo32(tmem + lo_lane + kTmHL, h2, x);
-      }
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      if (ptx::bar_or(3, 128, !ok || *abort_flag)) break;  // R^T stored; this slot's panels and V are free
-      if (st == 0) {
-        issue_kq(n + 2, kq_issued);
-        // ---- E^T = R^T (T diag(beta))^T  (N=64, K=64), over (K e^G S)^T, from
-        //      the hi + lo pairs: R_hi T_hi + R_lo T_hi + R_hi T_lo
-        ptx::tc_fence_after();
-        constexpr uint32_t id = ptx::idesc_bf16(128, 64, false, false);
-#pragma unroll
-        for (int i = 0; i < 12; ++i) {
-          const uint32_t rcol = (i >> 2) == 1 ? 32 : 0;        // R lo for the second group
-          const uint32_t tsm = (i >> 2) == 2 ? FU_TS : FU_TT;   // T lo for the third group
-          ptx::mma_bf16_ts(tmem + kTmX, tmem + kTmHL + rcol + 8 * (i & 3),
-                           ptx::sdesc_sw128(sb + tsm + (i & 3) * 32, 16, 1024), id, i > 0);
-        }
-        ptx::mma_commit(&s_e_done);
-      }
-      ok = wait_or_abort(&s_e_done, real & 1, abort_flag);
-      ptx::tc_fence_after();
+      if (st == 0) issue_kq(n + 2, kq_issued);  // the slot's panels are read: chunk n+2's k, q may land
+      // ---- E (fp32) as bf16 hi | lo
 #pragma unroll 1
       for (int h2 = 0; h2 < 2; ++h2) {
         float x[32];
@@ -803,6 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       if (ptx::bar_or(3, 128, !ok || *abort_flag)) break;
       if (st == 0) {
+        ptx::mbar_arrive(&s_x_free);  // E^T's columns are read: the next U^T may land there
         ptx::tc_fence_after();
         // S^T += E^T (K e^-G) (Kbar for a steep chunk): N=128, K=64, B MN-major
         constexpr uint32_t id2 = ptx::idesc_bf16(128, 128, false, true);
@@ -810,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 8; ++i)
           ptx::mma_bf16_ts(tmem + kTmS, tmem + kTmHL + (i >> 2) * 32 + 8 * (i & 3),
                            ptx::sdesc_sw128(sb + FU_RB + s * 16384 + (i & 3) * 2048, 8192, 1024), id2, 1);
-        // X^T[:, 64:128] += E^T P^T: N=64, K=64, B K-major
+        // (Q e^G S)^T += E^T P^T: N=64, K=64, B K-major
         constexpr uint32_t id3 = ptx::idesc_bf16(128, 64, false, false);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
@@ -821,6 +871,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait_or_abort(&s_m3, real & 1, abort_flag);
       if (ptx::bar_or(3, 128, !ok || *abort_flag)) break;
       ptx::tc_fence_after();
+      // K e^-G and P of this slot are read; gamma has a slot of its own per chunk mod 4
+      if (st == 0) ptx::mbar_arrive(&s_rb_free[s]);
       // ---- decay (single-reference chunks), the next chunk's bf16 operand, the outputs
 #pragma unroll 1
       for (int c32 = 0; c32 < D; c32 += 32) {
@@ -838,29 +890,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 16; ++i) w[i] = ptx::pack_bf16x2(x[2 * i], x[2 * i + 1]);
         ptx::tmem_st16u(tmem + lo_lane + kTmSb + c32 / 2, w);
       }
-      // the output tile, [64 tokens][128 dv] bf16, over this slot's V (read by R)
-      bf16* otile = reinterpret_cast<bf16*>(sm + FU_V + s * 16384);
+      // the output tile, two 64-channel panels [64 tokens][128 B], 128-byte
+      // swizzled: value channels 0..63 over this slot's P (read by the MMAs
+      // above), 64..127 in FU_OST (read by chunk n-1's store)
+      uint8_t* opan[2] = {sm + FU_P + s * 8192, sm + FU_OST};
+      uint8_t* ocol = opan[dv >> 6] + (dv & 7) * 2;
 #pragma unroll 1
       for (int h2 = 0; h2 < 2; ++h2) {
         float x[32];
         ld32(tmem + lo_lane + kTmO + 32 * h2, x);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) otile[(32 * h2 + e) * D + dv] = __float2bfloat16_rn(x[e]);
+        for (int e = 0; e < 32; ++e) {
+          const int r = 32 * h2 + e;
+          *reinterpret_cast<bf16*>(ocol + r * 128 + (((((dv & 63) >> 3) ^ r) & 7) << 4)) = __float2bfloat16_rn(x[e]);
+        }
       }
+      zero_cols64(tmem + lo_lane + kTmO);  // the next chunk's first MMA accumulates O onto zeros
       ptx::fence_proxy_async_smem();
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::bar_sync(3, 128);  // every read of this slot's K e^-G, P, gamma and of X^T done; tile complete
-      if (st == 0) ptx::mbar_arrive(&s_rb_free[s]);
-      if (it.Cn == C) {  // a whole chunk: one tensor store
+      ptx::bar_sync(3, 128);  // every read of X^T done; tile complete
+      const int h = it.unit % H;
+      if (it.Cn == C) {  // a whole chunk: two tensor stores
         if (st == 0) {
-          ptx::tma_store_3d(&tm_o, 0, it.unit % H, (int)it.s0, otile);
+          ptx::tma_store_3d(&tm_o, 0, h, (int)it.s0, opan[0]);
+          ptx::tma_store_3d(&tm_o, 64, h, (int)it.s0, opan[1]);
           ptx::bulk_commit();
         }
-      } else if (st < it.Cn) {  // the ragged last chunk of a sequence: one 256-byte row per thread
-        ptx::bulk_s2g(o + ((size_t)(it.s0 + st) * H + it.unit % H) * D, otile + st * D, D * 2);
-        ptx::bulk_commit();
+      } else {  // the ragged last chunk of a sequence: 16-byte pieces of its rows
+#pragma unroll 1
+        for (int piece = st; piece < C * 16; piece += 128) {
+          const int r = piece >> 4, c16 = piece & 15;
+          if (r < it.Cn) {
+            const uint4 val =
+                *reinterpret_cast<const uint4*>(opan[c16 >> 3] + r * 128 + ((((c16 & 7) ^ r) & 7) << 4));
+            *reinterpret_cast<uint4*>(o + ((size_t)(it.s0 + r) * H + h) * D + 8 * c16) = val;
+          }
+        }
+        ptx::bar_sync(3, 128);  // the tile is read
       }
       if ((it.flags & kItLast) && S_out) {
 #pragma unroll 1
@@ -874,7 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++real;
     }
-    ptx::bulk_wait0();  // the output rows have landed
+    if (st == 0) ptx::bulk_wait0();  // the output tiles have landed
   }
 
   // After a timeout: wait (bounded again) for the copies and MMAs still in
@@ -884,13 +952,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (s_abort) {
     if (tid == 0 && g_issued) ptx::mbar_wait_bounded(&s_g_full, (g_issued - 1) & 1, 1000000000ull);
     if (tid == 512)
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < 2; ++i)
         if (kq_issued[i]) ptx::mbar_wait_bounded(&s_kq_full[i], (kq_issued[i] - 1) & 1, 1000000000ull);
+    if (tid == 256 + 224)
+      for (int i = 0; i < 2; ++i)
         if (v_issued[i]) ptx::mbar_wait_bounded(&s_v_full[i], (v_issued[i] - 1) & 1, 1000000000ull);
-      }
   }
-  __syncthreads();
-  if (s_abort && (tid == 0 || tid == 512)) {  // the two MMA-issuing threads
+  if (s_abort && (tid == 0 || tid == 256 || tid == 512)) {  // the three MMA-issuing threads
     if (mma_issued) ptx::mma_commit(&s_drain);
     else ptx::mbar_arrive(&s_drain);
     ptx::mbar_wait_bounded(&s_drain, 0, 1000000000ull);
@@ -986,10 +1054,10 @@ inline cudaError_t launch_fused_t(const bf16* q, const bf16* k, const bf16* v, c
   if (e != cudaSuccess) return e;
   const long long tokens = (long long)B * T;
   CUtensorMap mk, mq, mg, mv, mo;
-  if ((e = ws::encode_rows_map(enc, &mo, o, false, tokens, H, D, false)) != cudaSuccess) return e;
+  if ((e = ws::encode_rows_map(enc, &mo, o, false, tokens, H, 64, true)) != cudaSuccess) return e;
   if ((e = ws::encode_rows_map(enc, &mk, k, false, tokens, H, 64, true)) != cudaSuccess) return e;
   if ((e = ws::encode_rows_map(enc, &mq, q, false, tokens, H, 64, true)) != cudaSuccess) return e;
-  if ((e = ws::encode_rows_map(enc, &mv, v, false, tokens, H, D, false)) != cudaSuccess) return e;
+  if ((e = ws::encode_rows_map(enc, &mv, v, false, tokens, H, 64, true)) != cudaSuccess) return e;
   if constexpr (kGate == kGateLogTok) {
     mg = mk;  // not read: a per-token gate takes plain loads
   } else {

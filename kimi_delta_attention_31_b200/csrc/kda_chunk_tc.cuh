@@ -162,13 +162,10 @@ __device__ long long chunks_before_warp(const int32_t* cu, int n) {
 // Operand building: thread t owns channels 8 (t mod 16) .. + 7 of rows
 // 4 (t / 16) .. + 3, so every global load and shared store moves 16 bytes.
 // ---------------------------------------------------------------------------
-constexpr uint32_t KA_TS = 50176;  // after the first MMA: T fp32 [64][68] (over RB) 17408
-constexpr uint32_t KA_MT = 67584;  //                      block products [3][16][20] 3840
 // A chunk whose every channel keeps its log-decay over the whole chunk above
 // this bound takes the single-reference form (left K o e^{G}, right K o e^{-G}):
 // both factors and every product stay inside the fp32 / bf16 exponent range.
 constexpr float kChunkRefMinG = -80.f;
-constexpr int MT_LD = 20;          // row stride (floats) of a block product
 constexpr int AS_LD = 68;          // row stride (floats) of A and T in fp32
 
 // acc (16 x 16 as two m16n8 halves) += X (16 x 16, fp32, row stride ldx) * Y (16 x 16,
@@ -255,10 +252,11 @@ __device__ __forceinline__ void normalise_rows(float* kv, float* qv, float nk, f
 // Phase 4 on the single-reference path: TMEM columns [tm, tm + 64) hold, in
 // lanes 0..63, A'_rj and in lanes 64..127, P'_rj (the other way round when
 // `p_first`).  Writes A = beta_r A'_rj (j < r, fp32, row stride AS_LD) and P
-// (j <= r, bf16 K-major 128-byte swizzled, zero above the diagonal).  Eight
+// (j <= r, bf16 K-major 128-byte swizzled, zero above the diagonal).  Returns
+// whether some |A_rj| this thread wrote is at least kSolveAccurateA.  Eight
 // warps; `warp` is the warp's index in the CTA (its TMEM lane quarter is
 // warp mod 4) and `w8` its index in the group of eight (which 32 columns it takes).
-__device__ __forceinline__ void scatter_single_ref(uint32_t tm, const float* s_beta, float* As, uint8_t* Pt,
+__device__ __forceinline__ bool scatter_single_ref(uint32_t tm, const float* s_beta, float* As, uint8_t* Pt,
                                                    int warp, int w8, int lane, bool p_first = false) {
   const int qd = warp & 3, ch = w8 >> 2;
   const int rho = 32 * qd + lane, r = rho & 63, j0 = 32 * ch;
@@ -272,45 +270,103 @@ __device__ __forceinline__ void scatter_single_ref(uint32_t tm, const float* s_b
 #pragma unroll
     for (int e = 0; e < 32; ++e) x[e] = (j0 + e < r) ? br * x[e] : 0.f;
     float4* dst = reinterpret_cast<float4*>(As + r * AS_LD + j0);
+    float mx = 0.f;
 #pragma unroll
-    for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(x[4 * v4], x[4 * v4 + 1], x[4 * v4 + 2], x[4 * v4 + 3]);
+    for (int v4 = 0; v4 < 8; ++v4) {
+      dst[v4] = make_float4(x[4 * v4], x[4 * v4 + 1], x[4 * v4 + 2], x[4 * v4 + 3]);
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x[4 * v4]), fabsf(x[4 * v4 + 1])), fmaxf(fabsf(x[4 * v4 + 2]), fabsf(x[4 * v4 + 3]))));
+    }
+    return mx >= kSolveAccurateA;
   } else {
 #pragma unroll
     for (int e = 0; e < 32; ++e) x[e] = (j0 + e <= r) ? x[e] : 0.f;
 #pragma unroll
     for (int k8 = 0; k8 < 4; ++k8) *reinterpret_cast<uint4*>(Pt + ptx::sw128_chunk(r, 4 * ch + k8)) = pack8(x + 8 * k8);
+    return false;
   }
 }
 
-// Phase 5: T = (I + A)^{-1} (A strictly lower, fp32 in As), blocked by 16.
-// Diagonal blocks by forward substitution in fp32, one thread per column of T
-// holding the column's 16 rows in registers (rows of A are broadcast loads).
-// Then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ: block column J needs only the
-// blocks above it in the same column, so warp J walks down its column (warp
-// syncs only), with TF32 warp MMAs and fp32 accumulation.  Finally
-// T diag(beta) in bf16 (K-major [64 r][64 j], 128-byte swizzle) into Tt.
-// 256 threads: t in [0, 256), w = t / 32; `sync` is their barrier and
-// `sync_or(p)` the same barrier returning the OR of p over them.  When some
-// |A_rj| >= kSolveAccurateA the block products run in split TF32.
-// With Tlo given, T diag(beta) is also split as hi + lo, hi = bf16(x) into Tt
-// and lo = bf16(x - hi) into Tlo (same layout), so that a pair of bf16 MMAs
-// uses it to about 2^-16; Tlo may overlap Ts (it is written after a barrier
-// that follows the last read of Ts).
-template <typename Sync, typename SyncOr>
-__device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* Mt, const float* s_beta, uint8_t* Tt,
-                                             int t, int w, int lane, Sync sync, SyncOr sync_or,
-                                             uint8_t* Tlo = nullptr) {
-  bool big = false;  // this thread's 16 entries of A (rows t / 4, columns 16 (t mod 4) ..)
-  {
-    const float4* a4 = reinterpret_cast<const float4*>(As + (t >> 2) * AS_LD + 16 * (t & 3));
+// acc <- the 16 x 16 fp32 block at dp (row stride ldd), in the C-fragment
+// layout of warp_gemm16.
+__device__ __forceinline__ void warp_load16(float (&acc)[2][4], const float* dp, int ldd, int lane) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 a = a4[i];
-      big |= fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))) >= kSolveAccurateA;
+  for (int nh = 0; nh < 2; ++nh) {
+    const float2 a = *reinterpret_cast<const float2*>(dp + g * ldd + 8 * nh + 2 * t);
+    const float2 b = *reinterpret_cast<const float2*>(dp + (g + 8) * ldd + 8 * nh + 2 * t);
+    acc[nh][0] = a.x;
+    acc[nh][1] = a.y;
+    acc[nh][2] = b.x;
+    acc[nh][3] = b.y;
+  }
+}
+// Block (I, J) of T diag(beta), T_IJ = scale * acc (C-fragment layout): bf16
+// hi into Tt (K-major [64 r][64 j], 128-byte swizzle), and lo = bf16(x - hi)
+// returned in lo[] (the words t_beta_store_lo writes) when the caller keeps a
+// lo part.
+__device__ __forceinline__ void t_beta_hi(const float (&acc)[2][4], float scale, const float* s_beta, int I, int J,
+                                          uint8_t* Tt, uint32_t (&lo)[4], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nh = 0; nh < 2; ++nh) {
+    const float2 b = *reinterpret_cast<const float2*>(s_beta + 16 * J + 8 * nh + 2 * t);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int r = 16 * I + g + 8 * hh;
+      const float x0 = scale * acc[nh][2 * hh] * b.x, x1 = scale * acc[nh][2 * hh + 1] * b.y;
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+      const float2 hf = __bfloat1622float2(h);
+      *reinterpret_cast<__nv_bfloat162*>(Tt + r * 128 + ((((2 * J + nh) ^ r) & 7) << 4) + 4 * t) = h;
+      lo[2 * nh + hh] = ptx::pack_bf16x2(x0 - hf.x, x1 - hf.y);
     }
   }
-  if (t < 64) {
-    const int jj = t & 15, o = t & 48;  // column jj of diagonal block o / 16
+}
+__device__ __forceinline__ void t_beta_store_lo(const uint32_t (&lo)[4], int I, int J, uint8_t* Tlo, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nh = 0; nh < 2; ++nh)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int r = 16 * I + g + 8 * hh;
+      *reinterpret_cast<uint32_t*>(Tlo + r * 128 + ((((2 * J + nh) ^ r) & 7) << 4) + 4 * t) = lo[2 * nh + hh];
+    }
+}
+// Zeroes the 16 x 16 bf16 block (I, J) of a K-major [64][64] swizzled tile (one warp).
+__device__ __forceinline__ void zero_block16(uint8_t* Tx, int I, int J, int lane) {
+  *reinterpret_cast<uint4*>(Tx + ptx::sw128_chunk(16 * I + (lane >> 1), 2 * J + (lane & 1))) =
+      make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Phase 5: T = (I + A)^{-1} (A strictly lower, fp32 in As, row stride AS_LD),
+// blocked by 16, computed in place over A, and T diag(beta) in bf16 (K-major
+// [64 r][64 j], 128-byte swizzle) into Tt.  The diagonal blocks by forward
+// substitution in fp32, one thread per column of T holding the column's 16
+// rows in registers (rows of A are broadcast loads).  The off-diagonal blocks
+// by levels over eight warps: with the 32 x 32 halves TA = T[0:32, 0:32] and
+// TB = T[32:64, 32:64] (the inverse of a block lower-triangular matrix),
+//   level 1   T10 = -T11 A10 T00,  T32 = -T33 A32 T22,  and A20 T00, A30 T00,
+//             A21 T11, A31 T11
+//   level 2   X = A[32:64, 0:32] TA (its other two blocks), T21 = -T22 X21,
+//             T31 = -(T32 X21 + T33 X31)
+//   level 3   T20 = -T22 X20,  T30 = -(T32 X20 + T33 X30)
+// so that no chain is longer than two 16 x 16 products per level.  Only the
+// diagonal blocks, T10 and T32 are read again: they overwrite their blocks of
+// A once no other warp reads those; the intermediate blocks live in the upper
+// blocks of As.  The products are TF32 warp MMAs with fp32 accumulation, in
+// split TF32 (about fp32 accuracy) when `accurate` (some |A_rj| >=
+// kSolveAccurateA, voted by the caller).  Each block of T diag(beta) goes to
+// bf16 as soon as it is final.  With Tlo given (its own buffer), T diag(beta)
+// is also split as hi + lo, hi = bf16(x) into Tt and lo = bf16(x - hi) into
+// Tlo (same layout), so that a pair of bf16 MMAs uses it to about 2^-16.
+// 256 threads: t in [0, 256), w = t / 32; `sync` is their barrier.  Tt and
+// Tlo are first written after the first barrier; the caller's barrier after
+// the call makes everything visible.  Warp 7 calls `idle()` (all its lanes)
+// after its level-1 work: it has nothing more to do in the call.
+template <typename Sync, typename Idle>
+__device__ __forceinline__ void solve_t_beta(float* As, const float* s_beta, uint8_t* Tt, uint8_t* Tlo,
+                                             bool accurate, int t, int w, int lane, Sync sync, Idle idle) {
+  if (t < 64) {  // diagonal blocks: forward substitution, one thread per column
+    const int jj = t & 15, o = t & 48;
     float x[16];
 #pragma unroll
     for (int m = 0; m < 16; ++m) x[m] = (m == jj) ? 1.f : 0.f;
@@ -333,68 +389,96 @@ __device__ __forceinline__ void solve_t_beta(const float* As, float* Ts, float* 
           }
         }
       }
-      if (i > jj) x[i] = -(acc0 + acc1);  // rows above jj keep T's zeros, row jj its 1
+      if (i > jj) x[i] = -(acc0 + acc1);
     }
+    __syncwarp();  // the block's 16 threads (one half-warp) have read its rows of A
 #pragma unroll
-    for (int i = 0; i < 16; ++i) Ts[(o + i) * AS_LD + o + jj] = x[i];
+    for (int i = 0; i < 16; ++i) As[(o + i) * AS_LD + o + jj] = x[i];
   }
-  const bool accurate = sync_or(big);
-  if (w < 3) {
-    const int Jc = w;
-    float* mt = Mt + w * 16 * MT_LD;
+  sync();  // diagonal blocks of T visible
+  auto gemm = [&](float (&acc)[2][4], const float* xp, const float* yp) {
+    if (accurate) warp_gemm16_3x(acc, xp, AS_LD, yp, AS_LD, lane);
+    else warp_gemm16(acc, xp, AS_LD, yp, AS_LD, lane);
+  };
+  auto blk = [As](int I, int J) { return As + 16 * I * AS_LD + 16 * J; };
+  auto clear = [](float (&acc)[2][4]) {
 #pragma unroll
-    for (int step = 1; step <= 3; ++step) {
-      const int Ir = Jc + step;
-      if (Ir < 4) {  // warp-uniform
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int kk = 0; kk < step; ++kk) {
-          const int K = Jc + kk;
-          if (accurate)
-            warp_gemm16_3x(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
-          else
-            warp_gemm16(acc, As + 16 * Ir * AS_LD + 16 * K, AS_LD, Ts + 16 * K * AS_LD + 16 * Jc, AS_LD, lane);
-        }
-        warp_store16(mt, MT_LD, acc, 1.f, lane);
-        __syncwarp();
-        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        if (accurate)
-          warp_gemm16_3x(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
-        else
-          warp_gemm16(acc2, Ts + 16 * Ir * AS_LD + 16 * Ir, AS_LD, mt, MT_LD, lane);
-        warp_store16(Ts + 16 * Ir * AS_LD + 16 * Jc, AS_LD, acc2, -1.f, lane);
-        __syncwarp();  // block (Ir, Jc) visible to the warp's next step; mt free again
-      }
-    }
+      for (int k = 0; k < 4; ++k) acc[i][k] = 0.f;
+  };
+  auto final_block = [&](const float (&acc)[2][4], float scale, int I, int J) {
+    uint32_t lo[4];
+    t_beta_hi(acc, scale, s_beta, I, J, Tt, lo, lane);
+    if (Tlo) t_beta_store_lo(lo, I, J, Tlo, lane);
+  };
+  // intermediate blocks, in the upper blocks of As
+  float* m10 = blk(0, 1);  // A10 T00
+  float* m32 = blk(2, 3);  // A32 T22
+  float* x20 = blk(0, 2);  // A20 T00, then X20 = A20 T00 + A21 T10
+  float* x30 = blk(0, 3);  // A30 T00, then X30 = A30 T00 + A31 T10
+  float* x21 = blk(1, 2);  // X21 = A21 T11
+  float* x31 = blk(1, 3);  // X31 = A31 T11
+  float acc[2][4];
+  // ---- level 1
+  if (w < 2) {  // T10 (w = 0), T32 (w = 1), each over its block of A
+    const int I = 2 * w + 1, J = 2 * w;
+    float* mt = w ? m32 : m10;
+    clear(acc);
+    gemm(acc, blk(I, J), blk(J, J));
+    warp_store16(mt, AS_LD, acc, 1.f, lane);
+    __syncwarp();
+    clear(acc);
+    gemm(acc, blk(I, I), mt);
+    warp_store16(blk(I, J), AS_LD, acc, -1.f, lane);
+    final_block(acc, -1.f, I, J);
+  } else if (w < 6) {  // A20 T00, A30 T00, A21 T11, A31 T11
+    const int I = 2 + (w & 1), J = (w - 2) >> 1;
+    clear(acc);
+    gemm(acc, blk(I, J), blk(J, J));
+    warp_store16(w == 2 ? x20 : w == 3 ? x30 : w == 4 ? x21 : x31, AS_LD, acc, 1.f, lane);
+  } else {  // the diagonal blocks of T diag(beta)
+    const int b0 = 2 * (w - 6);
+    warp_load16(acc, blk(b0, b0), AS_LD, lane);
+    final_block(acc, 1.f, b0, b0);
+    warp_load16(acc, blk(b0 + 1, b0 + 1), AS_LD, lane);
+    final_block(acc, 1.f, b0 + 1, b0 + 1);
+  }
+  if (w >= 2) {  // blocks above the diagonal: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+    const int zi = w - 2;
+    const int I = zi < 3 ? 0 : zi < 5 ? 1 : 2, J = zi < 3 ? zi + 1 : zi < 5 ? zi - 1 : 3;
+    zero_block16(Tt, I, J, lane);
+    if (Tlo) zero_block16(Tlo, I, J, lane);
+  }
+  if (w == 7) idle();
+  sync();
+  // ---- level 2
+  if (w < 2) {  // X20 = A20 T00 + A21 T10 (w = 0), X30 = A30 T00 + A31 T10 (w = 1)
+    float* xp = w ? x30 : x20;
+    warp_load16(acc, xp, AS_LD, lane);
+    gemm(acc, blk(2 + w, 1), blk(1, 0));
+    warp_store16(xp, AS_LD, acc, 1.f, lane);
+  } else if (w == 2) {  // T21 = -T22 X21
+    clear(acc);
+    gemm(acc, blk(2, 2), x21);
+    final_block(acc, -1.f, 2, 1);
+  } else if (w == 3) {  // T31 = -(T32 X21 + T33 X31)
+    clear(acc);
+    gemm(acc, blk(3, 2), x21);
+    gemm(acc, blk(3, 3), x31);
+    final_block(acc, -1.f, 3, 1);
   }
   sync();
-  // bf16 T diag(beta); blocks above the diagonal are zero
-  uint4 lo_w[2];
-  for (int i = 0, idx = t; idx < 512; ++i, idx += 256) {
-    const int rr = idx >> 3, k8 = idx & 7;
-    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if ((k8 >> 1) <= (rr >> 4)) {
-      const float4 t0 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8);
-      const float4 t1 = *reinterpret_cast<const float4*>(Ts + rr * AS_LD + 8 * k8 + 4);
-      const float4 b0 = *reinterpret_cast<const float4*>(s_beta + 8 * k8);
-      const float4 b1 = *reinterpret_cast<const float4*>(s_beta + 8 * k8 + 4);
-      y[0] = t0.x * b0.x; y[1] = t0.y * b0.y; y[2] = t0.z * b0.z; y[3] = t0.w * b0.w;
-      y[4] = t1.x * b1.x; y[5] = t1.y * b1.y; y[6] = t1.z * b1.z; y[7] = t1.w * b1.w;
-    }
-    const uint4 hi = pack8(y);
-    *reinterpret_cast<uint4*>(Tt + ptx::sw128_chunk(rr, k8)) = hi;
-    if (Tlo) {
-      float r[8];
-      unpack8(hi, r);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) r[e] = y[e] - r[e];
-      lo_w[i] = pack8(r);
-    }
-  }
-  if (Tlo) {
-    sync();  // every read of Ts is done
-    for (int i = 0, idx = t; idx < 512; ++i, idx += 256)
-      *reinterpret_cast<uint4*>(Tlo + ptx::sw128_chunk(idx >> 3, idx & 7)) = lo_w[i];
+  // ---- level 3
+  if (w == 4) {  // T20 = -T22 X20
+    clear(acc);
+    gemm(acc, blk(2, 2), x20);
+    final_block(acc, -1.f, 2, 0);
+  } else if (w == 5) {  // T30 = -(T32 X20 + T33 X30)
+    clear(acc);
+    gemm(acc, blk(3, 2), x20);
+    gemm(acc, blk(3, 3), x30);
+    final_block(acc, -1.f, 3, 0);
   }
 }
 
@@ -803,8 +887,9 @@ __global__ void __launch_bounds__(256, 2)
   ptx::tc_fence_after();
 
   // ---- 4. scatter A (fp32, beta-scaled) and P (bf16, lower incl. diagonal, zero above)
+  bool big = false;  // some |A_rj| this thread wrote >= kSolveAccurateA
   if (fast) {  // TMEM columns 0..63 hold whole rows
-    scatter_single_ref(tmem, s_beta, reinterpret_cast<float*>(sm + KA_AS), sm + KA_PT, warp, warp, lane);
+    big = scatter_single_ref(tmem, s_beta, reinterpret_cast<float*>(sm + KA_AS), sm + KA_PT, warp, warp, lane);
   } else {
     const int qd = warp & 3, ch = warp >> 2;
     const int rho = 32 * qd + lane;
@@ -836,7 +921,10 @@ __global__ void __launch_bounds__(256, 2)
       if (isK) {
         if (use) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) x[e] = (!diag || 16 * Jb + e < r) ? br * x[e] : 0.f;
+          for (int e = 0; e < 16; ++e) {
+            x[e] = (!diag || 16 * Jb + e < r) ? br * x[e] : 0.f;
+            big |= fabsf(x[e]) >= kSolveAccurateA;
+          }
           float4* dst = reinterpret_cast<float4*>(As + r * AS_LD + 16 * Jb);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
@@ -851,12 +939,11 @@ __global__ void __launch_bounds__(256, 2)
     }
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  const bool accurate = __syncthreads_or(big) != 0;
 
   // ---- 5. T = (I + A)^{-1} and T diag(beta) in bf16
-  solve_t_beta(reinterpret_cast<const float*>(sm + KA_AS), reinterpret_cast<float*>(sm + KA_TS),
-               reinterpret_cast<float*>(sm + KA_MT), s_beta, sm + KA_TT, tid, warp, lane,
-               [] { __syncthreads(); }, [](bool p) { return __syncthreads_or(p) != 0; });
+  solve_t_beta(reinterpret_cast<float*>(sm + KA_AS), s_beta, sm + KA_TT, nullptr, accurate, tid, warp, lane,
+               [] { __syncthreads(); }, [] {});
 
   // ---- 6. W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
   ptx::fence_proxy_async_smem();
@@ -1284,11 +1371,10 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
 // 2 two kernels.  Returns true for the single pass.
 constexpr int kPathAuto = 0, kPathFused = 1, kPathTwoKernel = 2;
 inline bool tc_use_fused(int B, int T, int H, int num_seqs, int sms, int seg_chunks, int force) {
-  if (force == kPathTwoKernel || seg_chunks > 0 || sms <= 0) return false;
+  if (force != kPathFused || seg_chunks > 0 || sms <= 0) return false;
   const long long N = num_seqs > 0 ? num_seqs : B;
   const long long tokens = (long long)B * T;
-  if (tokens >= (1LL << 31) || N * H >= (1LL << 31)) return false;
-  return force == kPathFused || N * H >= 1;
+  return tokens < (1LL << 31) && N * H < (1LL << 31);
 }
 
 // Workspace: the per-chunk images, then (segmented runs) the maps [N | M] of

@@ -75,17 +75,16 @@ constexpr uint32_t WS_L3 = 81920;      // 2 panels x 24576                      
 constexpr uint32_t WS_L3_PANEL = 24576;
 constexpr uint32_t WS_RB = 131072;     // K e^-G K-major 2 panels [64][64]; before the build:
                                        // warp totals of g [8][128] fp32                        16384
-constexpr uint32_t WS_UW = 147456;     // staging U^T | W^T (image order); during the solve the
-                                       // off-diagonal block products                          32768
-constexpr uint32_t WS_AS = 180224;     // A fp32 [64][68]                                      17408
-constexpr uint32_t WS_TS = WS_AS + 17408;  // T fp32 [64][68]                                  17408
+constexpr uint32_t WS_UW = 147456;     // staging U^T | W^T (image order)                       32768
+constexpr uint32_t WS_AS = 180224;     // A fp32 [64][68], then T over it                      17408
+                                       // (free)                                               17408
 constexpr uint32_t WS_TT = 215040;     // T diag(beta) bf16 K-major [64][64]; before the solve
                                        // the P staging                                        8192
 constexpr uint32_t WS_BYTES = WS_TT + 8192;
 constexpr uint32_t WS_DYN = WS_BYTES + 1024;
-static_assert(WS_TS + 17408 == WS_TT && WS_L3 + 2 * WS_L3_PANEL == WS_RB && WS_RB + 16384 == WS_UW &&
+static_assert(WS_AS + 2 * 17408 == WS_TT && WS_L3 + 2 * WS_L3_PANEL == WS_RB && WS_RB + 16384 == WS_UW &&
                   WS_UW + 32768 == WS_AS, "layout");
-static_assert(3 * 16 * tc::MT_LD * 4 <= 32768 && 8 * D * 4 <= 16384, "scratch sizes");
+static_assert(8 * D * 4 <= 16384, "scratch sizes");
 static_assert(WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_V % 1024 == 0 &&
                   WS_UW % 1024 == 0, "alignment");
 static_assert(IMG_A1 - IMG_U == 16384 && IMG_U - IMG_P == 8192, "image order");
@@ -525,27 +524,22 @@ __global__ void __launch_bounds__(512, 1)
       const bool skip = ptx::bar_or(2, 256, s_skip[slot] != 0);
       if (!skip) {
         // ---- scatter A (fp32, beta-scaled) and P (bf16, staged in the T diag(beta) buffer)
-        tc::scatter_single_ref(tmem + 64 * slot, s_beta[slot], As, sm + WS_TT, warp, w8, lane, slot == 1);
+        const bool big = tc::scatter_single_ref(tmem + 64 * slot, s_beta[slot], As, sm + WS_TT, warp, w8, lane,
+                                                slot == 1);
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
-        ptx::bar_sync(2, 256);
+        const bool accurate = ptx::bar_or(2, 256, big);
         if (st == kIo) {
           ptx::bulk_s2g(ws + (size_t)item * IMG_BYTES + IMG_P, sm + WS_TT, 8192);
           ptx::bulk_commit();
         }
         // ---- T = (I + A)^{-1}, T diag(beta) in bf16.  At each barrier thread kIo
-        //      first waits for its stores to have read shared memory: the block
-        //      products reuse the U^T / W^T staging (stored at the end of the
-        //      previous item), T diag(beta) the P staging.
-        tc::solve_t_beta(As, reinterpret_cast<float*>(sm + WS_TS), reinterpret_cast<float*>(sm + WS_UW),
-                         s_beta[slot], sm + WS_TT, st, w8, lane, [st] {
-                           if (st == kIo) ptx::bulk_wait_read0();
-                           ptx::bar_sync(2, 256);
-                         },
-                         [st](bool p) {
-                           if (st == kIo) ptx::bulk_wait_read0();
-                           return ptx::bar_or(2, 256, p);
-                         });
+        //      first waits for its stores to have read shared memory: T diag(beta)
+        //      reuses the P staging (written after the first barrier).
+        tc::solve_t_beta(As, s_beta[slot], sm + WS_TT, nullptr, accurate, st, w8, lane, [st] {
+          if (st == kIo) ptx::bulk_wait_read0();
+          ptx::bar_sync(2, 256);
+        }, [] {});
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::bar_sync(2, 256);

@@ -57,9 +57,13 @@ def test_noalloc_at_its_documented_limit(cuda_device):
 
 def test_noalloc_single_pass_at_the_benchmark_size(cuda_device):
     # the single-pass prefill needs only a unit counter: B8 H32 T8192 fits easily
-    assert kda.workspace_size(8, 8192, 32, 128, 128, 0, 64, torch.bfloat16) <= 4096
-    x = W.make_prefill(8, 8192, 32, 128, 128, "bf16", -5.0, 1.5, 0.0, seed=907, device=cuda_device)
-    _same(x, *_both(x))
+    kda.set_prefill_path(kda.PATH_FUSED)
+    try:
+        assert kda.workspace_size(8, 8192, 32, 128, 128, 0, 64, torch.bfloat16) <= 4096
+        x = W.make_prefill(8, 8192, 32, 128, 128, "bf16", -5.0, 1.5, 0.0, seed=907, device=cuda_device)
+        _same(x, *_both(x))
+    finally:
+        kda.set_prefill_path(kda.PATH_AUTO)
 
 
 def test_noalloc_fp32_path_needs_no_scratch(cuda_device):
