@@ -254,9 +254,9 @@ kda_status_t kda_chunk_fwd_host(const void* q, const void* k, const void* v, con
  * Its scratch is a fixed array inside the library, KDA_NOALLOC_SCRATCH_BYTES
  * bytes on every GPU that loads the library, held until process exit.  Sizes
  * whose kda_chunk_fwd_workspace_size(...) exceeds it are rejected with
- * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill
- * (kda_set_prefill_path(1)) needs 256 + 4 * num_seqs bytes, the
- * fp32-arithmetic path none; the two-kernel path (the default) keeps a
+ * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill needs 256 + 4 *
+ * num_seqs bytes, the fp32-arithmetic path none; only the two-kernel path
+ * (long sequences split into segments, or kda_set_prefill_path(2)) keeps a
  * per-chunk image and can exceed it: 64 MiB hold 903 of its (chunk, head)
  * pairs, e.g. B=1, H=8, T=7168.
  * The first call on each device looks up the array's device address (with
@@ -349,9 +349,8 @@ kda_status_t kda_set_local_kernel(int variant);
  *   2 = two kernels: every chunk's operands built in parallel into a per-chunk
  *       workspace image, then a state pass over the chunks of each unit (the
  *       path that also splits long sequences into segments);
- *   0 = automatic (default): the two kernels, which are faster than the
- *       single pass on every shape measured so far; the single pass runs only
- *       when asked for.
+ *   0 = automatic (default): the single pass unless the sequences are split
+ *       into segments (see kda_set_segment_chunks), then the two kernels.
  * Other values: KDA_ERR_INVALID_ARG, setting unchanged.
  */
 kda_status_t kda_set_prefill_path(int path);

@@ -67,10 +67,11 @@ constexpr uint32_t KA_L3 = 0;       // [K a; Q a]  K-major [128][128] (2 K-panel
 constexpr uint32_t KA_RB = 32768;   // right operands K-major [160][128]          40960
 constexpr uint32_t KA_TT = 8192;    // after the first MMA: T diag(beta) bf16 (Q part of panel 0) 8192
 constexpr uint32_t KA_PT = 24576;   //                      P bf16 K-major (Q part of panel 1)  8192
-// P, U^T and W^T are staged at KA_PT .. KA_PT + 40960 (U^T and W^T over A and T,
+// P, U^T and W^T are staged at KA_PT .. KA_PT + 40960 (U^T and W^T over A, T and T lo,
 // after the second MMA) in image order and leave in one bulk store.
 constexpr uint32_t KA_IMG_STAGE = KA_PT;
-constexpr uint32_t KA_AS = 32768;   //                      A fp32 [64][68] (over RB)  17408
+constexpr uint32_t KA_AS = 32768;   //                      A fp32 [64][68], then T (over RB)  17408
+constexpr uint32_t KA_TLO = 50176;  //                      T diag(beta) bf16 lo part (over RB) 8192
 constexpr uint32_t KA_XK = 73728;   // K o e^G  MN-major 2 panels [64][64] (block path) 16384
 constexpr uint32_t KA_BV = 90112;   // V        MN-major 2 panels [64][64]       16384
 constexpr uint32_t KA_BYTES = 106496;
@@ -942,10 +943,11 @@ __global__ void __launch_bounds__(256, 2)
   const bool accurate = __syncthreads_or(big) != 0;
 
   // ---- 5. T = (I + A)^{-1} and T diag(beta) in bf16
-  solve_t_beta(reinterpret_cast<float*>(sm + KA_AS), s_beta, sm + KA_TT, nullptr, accurate, tid, warp, lane,
+  solve_t_beta(reinterpret_cast<float*>(sm + KA_AS), s_beta, sm + KA_TT, sm + KA_TLO, accurate, tid, warp, lane,
                [] { __syncthreads(); }, [] {});
 
-  // ---- 6. W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
+  // ---- 6. W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64,
+  //      T diag(beta) as its bf16 hi part, then its lo part
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
@@ -953,13 +955,14 @@ __global__ void __launch_bounds__(256, 2)
     ptx::tc_fence_after();
     constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint64_t bd = ptx::sdesc_sw128(sb + KA_TT + kk * 32, 16, 1024);
+    for (int i = 0; i < 8; ++i) {
+      const int kk = i & 3;
+      const uint64_t bd = ptx::sdesc_sw128(sb + (i < 4 ? KA_TT : KA_TLO) + kk * 32, 16, 1024);
       // K o e^G: the K part of L3 (panel stride 16 KB) on the single-reference path
       const uint64_t xd = fast ? ptx::sdesc_sw128(sb + KA_L3 + kk * 2048, 16384, 1024)
                                : ptx::sdesc_sw128(sb + KA_XK + kk * 2048, 8192, 1024);
-      ptx::mma_bf16(tmem + 0, xd, bd, id, kk > 0);
-      ptx::mma_bf16(tmem + 64, ptx::sdesc_sw128(sb + KA_BV + kk * 2048, 8192, 1024), bd, id, kk > 0);
+      ptx::mma_bf16(tmem + 0, xd, bd, id, i > 0);
+      ptx::mma_bf16(tmem + 64, ptx::sdesc_sw128(sb + KA_BV + kk * 2048, 8192, 1024), bd, id, i > 0);
     }
     ptx::mma_commit(&s_bar);
   }
@@ -1371,7 +1374,7 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
 // 2 two kernels.  Returns true for the single pass.
 constexpr int kPathAuto = 0, kPathFused = 1, kPathTwoKernel = 2;
 inline bool tc_use_fused(int B, int T, int H, int num_seqs, int sms, int seg_chunks, int force) {
-  if (force != kPathFused || seg_chunks > 0 || sms <= 0) return false;
+  if (force == kPathTwoKernel || seg_chunks > 0 || sms <= 0) return false;
   const long long N = num_seqs > 0 ? num_seqs : B;
   const long long tokens = (long long)B * T;
   return tokens < (1LL << 31) && N * H < (1LL << 31);

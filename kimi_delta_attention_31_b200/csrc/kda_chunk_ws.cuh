@@ -77,7 +77,8 @@ constexpr uint32_t WS_RB = 131072;     // K e^-G K-major 2 panels [64][64]; befo
                                        // warp totals of g [8][128] fp32                        16384
 constexpr uint32_t WS_UW = 147456;     // staging U^T | W^T (image order)                       32768
 constexpr uint32_t WS_AS = 180224;     // A fp32 [64][68], then T over it                      17408
-                                       // (free)                                               17408
+constexpr uint32_t WS_TLO = WS_AS + 17408;  // T diag(beta) bf16 lo part K-major [64][64]       8192
+                                       // (free)                                                9216
 constexpr uint32_t WS_TT = 215040;     // T diag(beta) bf16 K-major [64][64]; before the solve
                                        // the P staging                                        8192
 constexpr uint32_t WS_BYTES = WS_TT + 8192;
@@ -85,7 +86,7 @@ constexpr uint32_t WS_DYN = WS_BYTES + 1024;
 static_assert(WS_AS + 2 * 17408 == WS_TT && WS_L3 + 2 * WS_L3_PANEL == WS_RB && WS_RB + 16384 == WS_UW &&
                   WS_UW + 32768 == WS_AS, "layout");
 static_assert(8 * D * 4 <= 16384, "scratch sizes");
-static_assert(WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_V % 1024 == 0 &&
+static_assert(WS_TLO % 1024 == 0 && WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_V % 1024 == 0 &&
                   WS_UW % 1024 == 0, "alignment");
 static_assert(IMG_A1 - IMG_U == 16384 && IMG_U - IMG_P == 8192, "image order");
 
@@ -536,26 +537,28 @@ __global__ void __launch_bounds__(512, 1)
         // ---- T = (I + A)^{-1}, T diag(beta) in bf16.  At each barrier thread kIo
         //      first waits for its stores to have read shared memory: T diag(beta)
         //      reuses the P staging (written after the first barrier).
-        tc::solve_t_beta(As, s_beta[slot], sm + WS_TT, nullptr, accurate, st, w8, lane, [st] {
+        tc::solve_t_beta(As, s_beta[slot], sm + WS_TT, sm + WS_TLO, accurate, st, w8, lane, [st] {
           if (st == kIo) ptx::bulk_wait_read0();
           ptx::bar_sync(2, 256);
         }, [] {});
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::bar_sync(2, 256);
-        // ---- W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
+        // ---- W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64,
+        //      T diag(beta) as its bf16 hi part, then its lo part
         if (st == 0) {
           const bool have_v = wait_or_abort(&s_v_full, n & 1, abort_flag);
           if (have_v && !*abort_flag) {
             ptx::tc_fence_after();
             constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bd = ptx::sdesc_sw128(sb + WS_TT + kk * 32, 16, 1024);
+            for (int i = 0; i < 8; ++i) {
+              const int kk = i & 3;
+              const uint64_t bd = ptx::sdesc_sw128(sb + (i < 4 ? WS_TT : WS_TLO) + kk * 32, 16, 1024);
               const uint64_t xd = ptx::sdesc_sw128(sb + WS_L3 + (slot ? 16384 : 0) + kk * 2048, WS_L3_PANEL, 1024);
               const uint64_t vd = ptx::sdesc_sw128(sb + WS_V + kk * 2048, 8192, 1024);
-              ptx::mma_bf16(tmem + 128, xd, bd, id, kk > 0);
-              ptx::mma_bf16(tmem + 192, vd, bd, id, kk > 0);
+              ptx::mma_bf16(tmem + 128, xd, bd, id, i > 0);
+              ptx::mma_bf16(tmem + 192, vd, bd, id, i > 0);
             }
             ptx::mma_commit(&s_b_done[slot]);
           } else {
