@@ -254,9 +254,9 @@ kda_status_t kda_chunk_fwd_host(const void* q, const void* k, const void* v, con
  * Its scratch is a fixed array inside the library, KDA_NOALLOC_SCRATCH_BYTES
  * bytes on every GPU that loads the library, held until process exit.  Sizes
  * whose kda_chunk_fwd_workspace_size(...) exceeds it are rejected with
- * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill needs 256 + 4 *
- * num_seqs bytes, the fp32-arithmetic path none; only the two-kernel path
- * (long sequences split into segments, or kda_set_prefill_path(2)) keeps a
+ * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill
+ * (kda_set_prefill_path(1)) needs 256 + 4 * num_seqs bytes, the
+ * fp32-arithmetic path none; the two-kernel path (the default) keeps a
  * per-chunk image and can exceed it: 64 MiB hold 903 of its (chunk, head)
  * pairs, e.g. B=1, H=8, T=7168.
  * The first call on each device looks up the array's device address (with
@@ -349,8 +349,13 @@ kda_status_t kda_set_local_kernel(int variant);
  *   2 = two kernels: every chunk's operands built in parallel into a per-chunk
  *       workspace image, then a state pass over the chunks of each unit (the
  *       path that also splits long sequences into segments);
- *   0 = automatic (default): the single pass unless the sequences are split
- *       into segments (see kda_set_segment_chunks), then the two kernels.
+ *   0 = automatic (default): the two kernels, faster on every shape measured.
+ * The two-kernel path keeps U and E in bf16 and T diag(beta) without its lo
+ * part, which is accurate unless a chunk has near-parallel keys (some
+ * |A_rj| >= 0.5, e.g. a key repeated within a chunk): its chunk-local kernels
+ * then raise a flag in the workspace, its state pass does nothing, and the
+ * single-pass kernel, launched last in every two-kernel call (it returns at
+ * once when the flag is clear), recomputes the whole call in its precise form.
  * Other values: KDA_ERR_INVALID_ARG, setting unchanged.
  */
 kda_status_t kda_set_prefill_path(int path);
@@ -367,10 +372,12 @@ int kda_chunk_fwd_phases(int B, int T, int H, int num_seqs, int dk, int dv, int 
 /*
  * Largest number of phases any kda_chunk_fwd call with these head and chunk
  * sizes can run: 1 for the fp32-arithmetic path (one kernel); 2 for the
- * tensor-core path, whose two-kernel form runs the chunk-local phase (one
- * kernel, or two when the warp-specialised kernel hands its steep chunks to
- * the two-CTA kernel, see kda_set_local_kernel) and then the state pass (one
- * kernel, or three when the sequences are split into segments).
+ * tensor-core path, whose two-kernel form runs the chunk-local phase (the
+ * precise fallback's set-up kernel, then one kernel, or two when the
+ * warp-specialised kernel hands its steep chunks to the two-CTA kernel, see
+ * kda_set_local_kernel) and then the state pass (one kernel, or three when the
+ * sequences are split into segments) followed by the precise fallback's
+ * single-pass kernel (see kda_set_prefill_path).
  */
 int kda_chunk_fwd_launches(int dk, int dv, int chunk_size, kda_dtype_t dtype);
 

@@ -508,14 +508,16 @@ def chunk_fwd_kernel_sequence(B, T, H, dk=128, dv=128, chunk_size=64, dtype=torc
         return list(KERNELS_SIMT)
     if uses_fused_kernel(B, T, H, num_seqs, dk, dv, chunk_size, dtype):
         return ["kda_fused_setup_kernel", KERNEL_FUSED]
-    seq = ["kda_ws_chunk_table_kernel"] if num_seqs > 0 else []
+    # the precise fallback's set-up first and its single-pass kernel last (it
+    # returns at once unless a chunk-local kernel met near-parallel keys)
+    seq = ["kda_fused_setup_kernel"] + (["kda_ws_chunk_table_kernel"] if num_seqs > 0 else [])
     if uses_ws_kernel(gate, num_seqs > 0, dk, dv, chunk_size, dtype):
         seq += [KERNEL_WS, KERNELS_TC[0]]
     else:
         seq += [KERNELS_TC[0]]
     if segment_chunks(B, T, H, num_seqs) > 0:
-        return seq + [KERNELS_TC[1], "kda_tc_seg_combine_kernel", KERNELS_TC[1]]
-    return seq + [KERNELS_TC[1]]
+        return seq + [KERNELS_TC[1], "kda_tc_seg_combine_kernel", KERNELS_TC[1], KERNEL_FUSED]
+    return seq + [KERNELS_TC[1], KERNEL_FUSED]
 
 
 def profile_chunk_fwd(call, stream, repeats=3, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16,

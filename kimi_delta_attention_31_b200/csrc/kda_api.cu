@@ -325,7 +325,8 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
   const int N = num_seqs > 0 ? num_seqs : B;
   const TcPlan plan = tc_plan(B, T, H, num_seqs);
   if (plan.fused) return kda::fu::fused_workspace_bytes(num_seqs);
-  return kda::tc_workspace_layout(max_chunks(B, T, num_seqs, chunk_size), H, (long long)N * H, T, plan.seg).total;
+  return kda::tc_workspace_layout(max_chunks(B, T, num_seqs, chunk_size), H, (long long)N * H, T, plan.seg,
+                                  num_seqs).total;
 }
 
 kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,

@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              const float* __restrict__ S0, bf16* __restrict__ o, float* __restrict__ S_out,
                              const int32_t* __restrict__ cu_seqlens, int N, int T, int H,
                              int* __restrict__ unit_ctr, const int* __restrict__ seq_order,
-                             const int* __restrict__ seq_status) {
+                             const int* __restrict__ seq_status, const int* __restrict__ esc_flag) {
   constexpr bool kPrep = gate_prep(kGate);
   constexpr bool kTmaGate = kGate != kGateLogTok;
   __shared__ __align__(16) float s_beta[2][C];
@@ -194,6 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_abort;
   // packed sequences whose cu_seqlens the set-up kernel rejected: no work at all
   if (kPacked && *seq_status < 0) return;
+  // run as the two-kernel path's precise fallback: nothing to do unless one of
+  // its chunk-local kernels met near-parallel keys
+  if (esc_flag && *esc_flag == 0) return;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   KDA_ALIGNED_DSMEM(sm, dsm_raw);
   const uint32_t sb = ptx::smem_u32(sm);
@@ -698,34 +701,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         const bool accurate = ptx::bar_or(2, 256, big);
-        // T = (I + A)^{-1} over A, T diag(beta) as bf16 hi (FU_TT) + lo (FU_TLO)
-        // (V of chunk n+1 into the other slot, whose V chunk n-1's U MMA has read,
-        // from the warp that is idle at that point of the solve)
-        tc::solve_t_beta(As, s_beta[s], sm + FU_TT, sm + FU_TLO, accurate, st, w8, lane,
-                         [] { ptx::bar_sync(2, 256); }, [&] {
-                           if (lane == 0) issue_v(n + 1, v_issued);
-                         });
+        // T = (I + A)^{-1} over A, T diag(beta) as bf16 hi (FU_TT), and for a chunk
+        // with near-parallel keys also its lo part (FU_TLO).  V of chunk n+1 goes
+        // into the other slot (its V, chunk n-1's, is read) from the warp that is
+        // idle at that point of the solve.
+        auto sync2 = [] { ptx::bar_sync(2, 256); };
+        auto idle = [&] {
+          if (lane == 0) issue_v(n + 1, v_issued);
+        };
+        if (accurate) tc::solve_t_beta_precise(As, s_beta[s], sm + FU_TT, sm + FU_TLO, st, w8, lane, sync2, idle);
+        else tc::solve_t_beta<false>(As, s_beta[s], sm + FU_TT, nullptr, st, w8, lane, sync2, idle);
         ptx::fence_proxy_async_smem();
         ptx::bar_sync(2, 256);
         // ---- W^T = (K e^G)^T (T diag(beta))^T into TMEM slot s (free since the
         //      scatter), U^T = V^T (T diag(beta))^T into the state's X^T columns
         //      (free once the state has split chunk n-1's E): M=128, N=64, K=64,
-        //      T diag(beta) as hi then lo.
+        //      T diag(beta) as hi, then (near-parallel keys) lo.
         if (st == 0) {
           bool go = wait_or_abort(&s_v_full[s], (n >> 1) & 1, abort_flag);
           go = go && (real == 0 || wait_or_abort(&s_x_free, (real - 1) & 1, abort_flag));
           if (go) {
             ptx::tc_fence_after();
             constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
+            const uint32_t kg = sb + FU_L3 + s * FU_L3_SLOT, vs = sb + FU_V + s * 16384;
+            const int parts = accurate ? 2 : 1;
+#pragma unroll 1
+            for (int part = 0; part < parts; ++part) {
+              const uint32_t tb = sb + (part ? FU_TLO : FU_TT);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              ptx::mma_bf16(tmem + 64 * s,
-                            ptx::sdesc_sw128(sb + FU_L3 + s * FU_L3_SLOT + (i & 3) * 2048, 16384, 1024),
-                            ptx::sdesc_sw128(sb + (i < 4 ? FU_TT : FU_TLO) + (i & 3) * 32, 16, 1024), id, i > 0);
+              for (int i = 0; i < 4; ++i)
+                ptx::mma_bf16(tmem + 64 * s, ptx::sdesc_sw128(kg + i * 2048, 16384, 1024),
+                              ptx::sdesc_sw128(tb + i * 32, 16, 1024), id, (part | i) > 0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              ptx::mma_bf16(tmem + kTmX, ptx::sdesc_sw128(sb + FU_V + s * 16384 + (i & 3) * 2048, 8192, 1024),
-                            ptx::sdesc_sw128(sb + (i < 4 ? FU_TT : FU_TLO) + (i & 3) * 32, 16, 1024), id, i > 0);
+              for (int i = 0; i < 4; ++i)
+                ptx::mma_bf16(tmem + kTmX, ptx::sdesc_sw128(vs + i * 2048, 8192, 1024),
+                              ptx::sdesc_sw128(tb + i * 32, 16, 1024), id, (part | i) > 0);
+            }
             mma_issued = true;
             ptx::mma_commit(&s_uw_done);
           } else {
@@ -969,7 +980,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) ptx::tmem_dealloc(tmem, kTmCols);
 }
 
-// Set-up of one call (one CTA of 1024 threads): zeroes the unit counter and,
+// Set-up of one call (one CTA of 1024 threads): zeroes the unit counter (and,
+// when the two-kernel path runs this kernel as its precise fallback, the flag
+// its chunk-local kernels raise) and,
 // for packed sequences, checks cu_seqlens (cu[0] == 0, non-decreasing,
 // cu[num_seqs] == T) -- a bad table raises the device error word and sets
 // *status = -1, so the prefill kernel does nothing -- then orders the
@@ -978,10 +991,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kSortMax = 2048;
 __global__ void __launch_bounds__(1024)
     kda_fused_setup_kernel(const int32_t* __restrict__ cu_seqlens, int num_seqs, int T, int* __restrict__ ctr,
-                           int* __restrict__ status, int* __restrict__ order) {
+                           int* __restrict__ status, int* __restrict__ order, int* __restrict__ esc_flag) {
   __shared__ int s_len[kSortMax];
   const int tid = threadIdx.x;
-  if (tid == 0) *ctr = 0;
+  if (tid == 0) {
+    *ctr = 0;
+    if (esc_flag) *esc_flag = 0;
+  }
   if (!cu_seqlens) return;
   bool bad = tid == 0 && (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T);
   for (int i = tid; i < num_seqs; i += 1024) bad |= cu_seqlens[i + 1] < cu_seqlens[i];
@@ -1045,10 +1061,17 @@ inline bool fused_kernel_available() {
   return ok[dev];
 }
 
+// Launches the set-up kernel (phase & kFusedSetup) and the prefill kernel
+// (phase & kFusedMain).  With esc_flag the pair is the two-kernel path's
+// precise fallback: the set-up kernel zeroes *esc_flag, and the prefill kernel
+// (launched after the two-kernel path's state pass) does the call's work only
+// if a chunk-local kernel has raised it meanwhile.
+constexpr int kFusedSetup = 1, kFusedMain = 2;
 template <int kGate>
 inline cudaError_t launch_fused_t(const bf16* q, const bf16* k, const bf16* v, const void* g, const float* beta,
                                   const float* S0, bf16* o, float* S_out, const int32_t* cu_seqlens, int N,
-                                  int B, int T, int H, void* workspace, int sms, cudaStream_t stream) {
+                                  int B, int T, int H, void* workspace, int sms, cudaStream_t stream,
+                                  int phase, int* esc_flag) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   cudaError_t e = ws::tensor_map_encoder(&enc);
   if (e != cudaSuccess) return e;
@@ -1067,37 +1090,39 @@ inline cudaError_t launch_fused_t(const bf16* q, const bf16* k, const bf16* v, c
   int* ctr = wsi;
   int* status = wsi + 1;
   int* order = wsi + 64;
-  kda_fused_setup_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, cu_seqlens ? N : 0, T, ctr, status, order);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (phase & kFusedSetup) {
+    kda_fused_setup_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, cu_seqlens ? N : 0, T, ctr, status, order, esc_flag);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   const long long units = (long long)N * H;
   const int grid = (int)std::min<long long>(units, sms);
-  if (grid <= 0) return cudaSuccess;
+  if (grid <= 0 || !(phase & kFusedMain)) return cudaSuccess;
   if (cu_seqlens)
     kda_fused_prefill_kernel<kGate, true><<<grid, kThreads, FU_DYN, stream>>>(
-        mk, mq, mg, mv, mo, g, beta, S0, o, S_out, cu_seqlens, N, T, H, ctr, order, status);
+        mk, mq, mg, mv, mo, g, beta, S0, o, S_out, cu_seqlens, N, T, H, ctr, order, status, esc_flag);
   else
     kda_fused_prefill_kernel<kGate, false><<<grid, kThreads, FU_DYN, stream>>>(
-        mk, mq, mg, mv, mo, g, beta, S0, o, S_out, nullptr, N, T, H, ctr, nullptr, status);
+        mk, mq, mg, mv, mo, g, beta, S0, o, S_out, nullptr, N, T, H, ctr, nullptr, status, esc_flag);
   return cudaGetLastError();
 }
 
 inline cudaError_t launch_fused(const bf16* q, const bf16* k, const bf16* v, const void* g, const float* beta,
                                 const float* S0, bf16* o, float* S_out, const int32_t* cu_seqlens, int N, int B,
-                                int T, int H, void* workspace, int sms, int gmode, cudaStream_t stream) {
+                                int T, int H, void* workspace, int sms, int gmode, cudaStream_t stream,
+                                int phase = kFusedSetup | kFusedMain, int* esc_flag = nullptr) {
+#define KDA_FU_CASE(M)                                                                                          \
+  case M:                                                                                                       \
+    return launch_fused_t<M>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms, stream, \
+                             phase, esc_flag)
   switch (gmode) {
-    case kGateLogCh:
-      return launch_fused_t<kGateLogCh>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms, stream);
-    case kGateLogTok:
-      return launch_fused_t<kGateLogTok>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms, stream);
-    case kGateLogitF32:
-      return launch_fused_t<kGateLogitF32>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms,
-                                           stream);
-    case kGateLogitBf16:
-      return launch_fused_t<kGateLogitBf16>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms,
-                                            stream);
+    KDA_FU_CASE(kGateLogCh);
+    KDA_FU_CASE(kGateLogTok);
+    KDA_FU_CASE(kGateLogitF32);
+    KDA_FU_CASE(kGateLogitBf16);
     default:
       return cudaErrorInvalidValue;
   }
+#undef KDA_FU_CASE
 }
 
 }  // namespace fu

@@ -67,11 +67,10 @@ constexpr uint32_t KA_L3 = 0;       // [K a; Q a]  K-major [128][128] (2 K-panel
 constexpr uint32_t KA_RB = 32768;   // right operands K-major [160][128]          40960
 constexpr uint32_t KA_TT = 8192;    // after the first MMA: T diag(beta) bf16 (Q part of panel 0) 8192
 constexpr uint32_t KA_PT = 24576;   //                      P bf16 K-major (Q part of panel 1)  8192
-// P, U^T and W^T are staged at KA_PT .. KA_PT + 40960 (U^T and W^T over A, T and T lo,
+// P, U^T and W^T are staged at KA_PT .. KA_PT + 40960 (U^T and W^T over A and T,
 // after the second MMA) in image order and leave in one bulk store.
 constexpr uint32_t KA_IMG_STAGE = KA_PT;
 constexpr uint32_t KA_AS = 32768;   //                      A fp32 [64][68], then T (over RB)  17408
-constexpr uint32_t KA_TLO = 50176;  //                      T diag(beta) bf16 lo part (over RB) 8192
 constexpr uint32_t KA_XK = 73728;   // K o e^G  MN-major 2 panels [64][64] (block path) 16384
 constexpr uint32_t KA_BV = 90112;   // V        MN-major 2 panels [64][64]       16384
 constexpr uint32_t KA_BYTES = 106496;
@@ -190,7 +189,8 @@ __device__ __forceinline__ void warp_gemm16(float (&acc)[2][4], const float* xp,
 // The same product with each operand split as tf32 hi + lo (x = hi + lo to
 // about 2^-22): acc += Xlo Yhi + Xhi Ylo + Xhi Yhi, three TF32 MMAs per step,
 // about fp32 accuracy.  For blocks of A whose entries are large (near-parallel
-// keys), where the block products cancel and TF32 rounding would not average out.
+// keys), where the block products cancel and TF32 rounding would not average
+// out.
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
   hi = ptx::to_tf32(x);
   lo = ptx::to_tf32(x - __uint_as_float(hi));
@@ -356,16 +356,19 @@ __device__ __forceinline__ void zero_block16(uint8_t* Tx, int I, int J, int lane
 // blocks of As.  The products are TF32 warp MMAs with fp32 accumulation, in
 // split TF32 (about fp32 accuracy) when `accurate` (some |A_rj| >=
 // kSolveAccurateA, voted by the caller).  Each block of T diag(beta) goes to
-// bf16 as soon as it is final.  With Tlo given (its own buffer), T diag(beta)
-// is also split as hi + lo, hi = bf16(x) into Tt and lo = bf16(x - hi) into
-// Tlo (same layout), so that a pair of bf16 MMAs uses it to about 2^-16.
+// bf16 as soon as it is final.  kPrecise (for chunks where some |A_rj| >=
+// kSolveAccurateA, see solve_t_beta_precise) adds two things: split-TF32
+// products (about fp32 accuracy), and T diag(beta) split as hi + lo,
+// hi = bf16(x) into Tt and lo = bf16(x - hi) into Tlo (its own buffer, same
+// layout), so that a pair of bf16 MMAs uses it to about 2^-16.  Without it the
+// products are plain TF32 and only hi is written (Tlo is not touched).
 // 256 threads: t in [0, 256), w = t / 32; `sync` is their barrier.  Tt and
 // Tlo are first written after the first barrier; the caller's barrier after
 // the call makes everything visible.  Warp 7 calls `idle()` (all its lanes)
 // after its level-1 work: it has nothing more to do in the call.
-template <typename Sync, typename Idle>
-__device__ __forceinline__ void solve_t_beta(float* As, const float* s_beta, uint8_t* Tt, uint8_t* Tlo,
-                                             bool accurate, int t, int w, int lane, Sync sync, Idle idle) {
+template <bool kPrecise, typename Sync, typename Idle>
+__device__ __forceinline__ void solve_t_beta(float* As, const float* s_beta, uint8_t* Tt, uint8_t* Tlo, int t,
+                                             int w, int lane, Sync sync, Idle idle) {
   if (t < 64) {  // diagonal blocks: forward substitution, one thread per column
     const int jj = t & 15, o = t & 48;
     float x[16];
@@ -397,8 +400,8 @@ __device__ __forceinline__ void solve_t_beta(float* As, const float* s_beta, uin
     for (int i = 0; i < 16; ++i) As[(o + i) * AS_LD + o + jj] = x[i];
   }
   sync();  // diagonal blocks of T visible
-  auto gemm = [&](float (&acc)[2][4], const float* xp, const float* yp) {
-    if (accurate) warp_gemm16_3x(acc, xp, AS_LD, yp, AS_LD, lane);
+  auto gemm = [&](float (&acc)[2][4], const float* xp, const float* yp) {  // acc += X Y
+    if (kPrecise) warp_gemm16_3x(acc, xp, AS_LD, yp, AS_LD, lane);
     else warp_gemm16(acc, xp, AS_LD, yp, AS_LD, lane);
   };
   auto blk = [As](int I, int J) { return As + 16 * I * AS_LD + 16 * J; };
@@ -411,7 +414,7 @@ __device__ __forceinline__ void solve_t_beta(float* As, const float* s_beta, uin
   auto final_block = [&](const float (&acc)[2][4], float scale, int I, int J) {
     uint32_t lo[4];
     t_beta_hi(acc, scale, s_beta, I, J, Tt, lo, lane);
-    if (Tlo) t_beta_store_lo(lo, I, J, Tlo, lane);
+    if (kPrecise) t_beta_store_lo(lo, I, J, Tlo, lane);
   };
   // intermediate blocks, in the upper blocks of As
   float* m10 = blk(0, 1);  // A10 T00
@@ -449,7 +452,7 @@ __device__ __forceinline__ void solve_t_beta(float* As, const float* s_beta, uin
     const int zi = w - 2;
     const int I = zi < 3 ? 0 : zi < 5 ? 1 : 2, J = zi < 3 ? zi + 1 : zi < 5 ? zi - 1 : 3;
     zero_block16(Tt, I, J, lane);
-    if (Tlo) zero_block16(Tlo, I, J, lane);
+    if (kPrecise) zero_block16(Tlo, I, J, lane);
   }
   if (w == 7) idle();
   sync();
@@ -481,6 +484,14 @@ __device__ __forceinline__ void solve_t_beta(float* As, const float* s_beta, uin
     gemm(acc, blk(3, 3), x30);
     final_block(acc, -1.f, 3, 0);
   }
+}
+
+// The solve of a chunk with near-parallel keys (some |A_rj| >= kSolveAccurateA):
+// solve_t_beta<true>.
+template <typename Sync, typename Idle>
+__device__ __forceinline__ void solve_t_beta_precise(float* As, const float* s_beta, uint8_t* Tt, uint8_t* Tlo, int t,
+                                                  int w, int lane, Sync sync, Idle idle) {
+  solve_t_beta<true>(As, s_beta, Tt, Tlo, t, w, lane, sync, idle);
 }
 
 // Phase 6 epilogue: TMEM columns [tm, tm + 64) = W^T, [tm + 64, tm + 128) = U^T
@@ -517,7 +528,7 @@ __global__ void __launch_bounds__(256, 2)
                               int num_seqs, int T, int H, uint32_t num_items, FastDiv fdH, FastDiv fdC,
                               uint8_t* __restrict__ ws, const uint32_t* __restrict__ item_list,
                               const uint32_t* __restrict__ item_cnt, uint32_t list_cap,
-                              const int* __restrict__ chunk_total) {
+                              const int* __restrict__ chunk_total, int* __restrict__ esc_flag) {
   __shared__ __align__(16) float s_beta[C];
   __shared__ float s_nrm[2][C];  // 1 / |k_r|, 1 / |q_r| (only when the call normalises)
   constexpr bool kPrep = gate_prep(kGate);
@@ -940,14 +951,15 @@ __global__ void __launch_bounds__(256, 2)
     }
   }
   ptx::tc_fence_before();
-  const bool accurate = __syncthreads_or(big) != 0;
+  // near-parallel keys: this call's result is recomputed by the single-pass
+  // kernel in its precise form (launch_chunk_tc)
+  if (__syncthreads_or(big) && tid == 0) *esc_flag = 1;
 
   // ---- 5. T = (I + A)^{-1} and T diag(beta) in bf16
-  solve_t_beta(reinterpret_cast<float*>(sm + KA_AS), s_beta, sm + KA_TT, sm + KA_TLO, accurate, tid, warp, lane,
-               [] { __syncthreads(); }, [] {});
+  solve_t_beta<false>(reinterpret_cast<float*>(sm + KA_AS), s_beta, sm + KA_TT, nullptr, tid, warp, lane,
+                      [] { __syncthreads(); }, [] {});
 
-  // ---- 6. W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64,
-  //      T diag(beta) as its bf16 hi part, then its lo part
+  // ---- 6. W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
@@ -955,14 +967,13 @@ __global__ void __launch_bounds__(256, 2)
     ptx::tc_fence_after();
     constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int kk = i & 3;
-      const uint64_t bd = ptx::sdesc_sw128(sb + (i < 4 ? KA_TT : KA_TLO) + kk * 32, 16, 1024);
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t bd = ptx::sdesc_sw128(sb + KA_TT + kk * 32, 16, 1024);
       // K o e^G: the K part of L3 (panel stride 16 KB) on the single-reference path
       const uint64_t xd = fast ? ptx::sdesc_sw128(sb + KA_L3 + kk * 2048, 16384, 1024)
                                : ptx::sdesc_sw128(sb + KA_XK + kk * 2048, 8192, 1024);
-      ptx::mma_bf16(tmem + 0, xd, bd, id, i > 0);
-      ptx::mma_bf16(tmem + 64, ptx::sdesc_sw128(sb + KA_BV + kk * 2048, 8192, 1024), bd, id, i > 0);
+      ptx::mma_bf16(tmem + 0, xd, bd, id, kk > 0);
+      ptx::mma_bf16(tmem + 64, ptx::sdesc_sw128(sb + KA_BV + kk * 2048, 8192, 1024), bd, id, kk > 0);
     }
     ptx::mma_commit(&s_bar);
   }
@@ -997,7 +1008,8 @@ constexpr int kPassPlain = 0, kPassMaps = 1, kPassFinal = 2;
 // (unit, 8-column block); thread t owns row t / 2, columns 4 (t mod 2) .. + 3.
 __global__ void __launch_bounds__(256)
     kda_tc_seg_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
-                              float* __restrict__ seg_init, int P) {
+                              float* __restrict__ seg_init, int P, const int* __restrict__ esc_flag) {
+  if (*esc_flag) return;  // the single-pass kernel recomputes the call
   __shared__ __align__(16) float Ss[D][8];
   const long long u = blockIdx.x / (D / 8);
   const int j0 = (blockIdx.x % (D / 8)) * 8;
@@ -1036,7 +1048,8 @@ __global__ void __launch_bounds__(256, 2)
                              float* __restrict__ S_out, bf16* __restrict__ o,
                              const int32_t* __restrict__ cu_seqlens, int N, int T, int H,
                              int seg_chunks, int pass, float* __restrict__ maps,
-                             const float* __restrict__ seg_init, const int* __restrict__ chunk_total) {
+                             const float* __restrict__ seg_init, const int* __restrict__ chunk_total,
+                             const int* __restrict__ esc_flag) {
   __shared__ __align__(8) uint64_t s_full[3];  // image parts: 0 [W; Q e^G], 1 U^T, 2 P + Kbar + gamma
   __shared__ __align__(8) uint64_t s_mma1, s_mma2;
   __shared__ uint32_t s_tmem;
@@ -1050,6 +1063,8 @@ __global__ void __launch_bounds__(256, 2)
   // packed sequences whose cu_seqlens the chunk-table kernel rejected: the
   // outputs are left untouched
   if (cu_seqlens && chunk_total && *chunk_total < 0) return;
+  // a chunk with near-parallel keys: the single-pass kernel recomputes the call
+  if (*esc_flag) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, ch = warp >> 2;
   const int c = 32 * qd + lane;  // state row; rows 0..63 of X are tokens (-E), 64..127 outputs
@@ -1373,8 +1388,11 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
 // 0 automatic (the single pass unless segments were chosen), 1 single pass,
 // 2 two kernels.  Returns true for the single pass.
 constexpr int kPathAuto = 0, kPathFused = 1, kPathTwoKernel = 2;
+// The single pass runs when asked for (kda_set_prefill_path(1)); the
+// automatic choice is the two-kernel path, faster on every measured shape and,
+// with its precise fallback, as accurate.
 inline bool tc_use_fused(int B, int T, int H, int num_seqs, int sms, int seg_chunks, int force) {
-  if (force == kPathTwoKernel || seg_chunks > 0 || sms <= 0) return false;
+  if (force != kPathFused || seg_chunks > 0 || sms <= 0) return false;
   const long long N = num_seqs > 0 ? num_seqs : B;
   const long long tokens = (long long)B * T;
   return tokens < (1LL << 31) && N * H < (1LL << 31);
@@ -1384,12 +1402,14 @@ inline bool tc_use_fused(int B, int T, int H, int num_seqs, int sms, int seg_chu
 // every segment but the last and the entry state of every segment, fp32,
 // then the warp-specialised kernel's per-CTA item lists (at most
 // items + kMaxListCtas entries and kMaxListCtas counts, uint32), then (packed
-// sequences) its chunk table, {first token, rows} per chunk, and the count.
+// sequences) its chunk table, {first token, rows} per chunk, and the count,
+// then the precise-fallback flag and the single-pass kernel's own workspace.
 constexpr int kMaxListCtas = 1024;
 struct TcWorkspace {
-  size_t images, maps, seg_init, lists, table, total;
+  size_t images, maps, seg_init, lists, table, esc, fused, total;
 };
-inline TcWorkspace tc_workspace_layout(long long max_chunks, int H, long long units, int T, int seg_chunks) {
+inline TcWorkspace tc_workspace_layout(long long max_chunks, int H, long long units, int T, int seg_chunks,
+                                       int num_seqs) {
   TcWorkspace w{};
   w.images = (size_t)max_chunks * (size_t)H * tc::IMG_BYTES;
   w.maps = w.seg_init = w.lists = (w.images + 255) & ~(size_t)255;
@@ -1401,7 +1421,9 @@ inline TcWorkspace tc_workspace_layout(long long max_chunks, int H, long long un
     w.lists = w.seg_init + (size_t)units * (size_t)P * mat;
   }
   w.table = (w.lists + ((size_t)max_chunks * (size_t)H + 2 * kMaxListCtas) * sizeof(uint32_t) + 255) & ~(size_t)255;
-  w.total = w.table + (size_t)max_chunks * sizeof(int2) + 16;
+  w.esc = (w.table + (size_t)max_chunks * sizeof(int2) + 16 + 255) & ~(size_t)255;
+  w.fused = w.esc + 256;
+  w.total = w.fused + fu::fused_workspace_bytes(num_seqs);
   return w;
 }
 
@@ -1436,9 +1458,20 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   // The warp-specialised kernel takes every layout and gate mode;
   // `local_kernel` == 1 keeps every call on the two-CTA kernel.
   const bool use_ws = items > 0 && local_kernel != 1 && (long long)B * T < (1LL << 31) && ws::ws_kernel_available();
-  const TcWorkspace lay = tc_workspace_layout(max_chunks, H, N * (long long)H, T, seg_chunks);
+  const TcWorkspace lay = tc_workspace_layout(max_chunks, H, N * (long long)H, T, seg_chunks, num_seqs);
   int2* table = reinterpret_cast<int2*>(ws + lay.table);
   int* chunk_total = reinterpret_cast<int*>(table + max_chunks);
+  // Precise fallback.  These kernels keep U and E in bf16 and T diag(beta)
+  // without its lo part, which is accurate unless some chunk has near-parallel
+  // keys (|A_rj| >= kSolveAccurateA: then U's rows telescope and their bf16
+  // roundings add up).  The chunk-local kernels raise *esc on such a chunk; the
+  // state pass then does nothing and the single-pass kernel, which handles
+  // those chunks in its precise form, recomputes the whole call.
+  int* esc = reinterpret_cast<int*>(ws + lay.esc);
+  if (!fu::fused_kernel_available()) return cudaErrorNotSupported;
+  e = fu::launch_fused(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, ws + lay.fused, s_sms, gmode,
+                       stream, fu::kFusedSetup, esc);
+  if (e != cudaSuccess) return e;
   if (cu_seqlens) {
     // validates cu_seqlens (a malformed table: total = -1 and every later kernel
     // skips its work) and builds the chunk table of packed sequences
@@ -1447,7 +1480,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   }
   if (use_ws) {
     e = ws::launch_ws_local(q, k, v, g, beta, cu_seqlens, num_seqs, B, T, H, items, fdH, fdC, ws,
-                            reinterpret_cast<uint32_t*>(ws + lay.lists), table, chunk_total,
+                            reinterpret_cast<uint32_t*>(ws + lay.lists), table, chunk_total, esc,
                             std::min(s_sms, kMaxListCtas), gmode, stream);
     if (e != cudaSuccess) return e;
   } else if (items > 0) {
@@ -1456,7 +1489,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   tc::kda_tc_chunk_local_kernel<M><<<gridA, 256, tc::KA_DYN, stream>>>(q, k, v, g, beta, cu_seqlens, \
                                                                        num_seqs, T, H, (uint32_t)items, fdH, \
                                                                        fdC, ws, nullptr, nullptr, 0u, \
-                                                                       cu_seqlens ? chunk_total : nullptr)
+                                                                       cu_seqlens ? chunk_total : nullptr, esc)
     switch (gmode) {
       case kGateLogCh: KDA_TC_LOCAL(kGateLogCh); break;
       case kGateLogTok: KDA_TC_LOCAL(kGateLogTok); break;
@@ -1472,26 +1505,31 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   const long long units = (long long)N * H;
   if (units > 0 && seg_chunks > 0 && !cu_seqlens) {
     // segmented: maps of every segment but the last, entry states, final pass
-    const TcWorkspace lay = tc_workspace_layout(max_chunks, H, units, T, seg_chunks);
     float* maps = reinterpret_cast<float*>(ws + lay.maps);
     float* seg_init = reinterpret_cast<float*>(ws + lay.seg_init);
     const long long nc = (T + tc::C - 1) / tc::C;
     const int P = (int)((nc + seg_chunks - 1) / seg_chunks);
     const long long map_items = units * (P - 1) * 2, fin_items = units * P;
     tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(map_items, 2LL * s_sms), 256, tc::KB_DYN, stream>>>(
-        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassMaps, maps, seg_init, nullptr);
+        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassMaps, maps, seg_init, nullptr, esc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    tc::kda_tc_seg_combine_kernel<<<(unsigned)(units * (tc::D / 8)), 256, 0, stream>>>(maps, S0, seg_init, P);
+    tc::kda_tc_seg_combine_kernel<<<(unsigned)(units * (tc::D / 8)), 256, 0, stream>>>(maps, S0, seg_init, P,
+                                                                                        esc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     tc::kda_tc_state_pass_kernel<<<(int)std::min<long long>(fin_items, 2LL * s_sms), 256, tc::KB_DYN, stream>>>(
-        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassFinal, maps, seg_init, nullptr);
+        ws, S0, S_out, o, nullptr, B, T, H, seg_chunks, tc::kPassFinal, maps, seg_init, nullptr, esc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else if (units > 0) {
     const int gridB = (int)(units < 2LL * s_sms ? units : 2LL * s_sms);  // two CTAs per SM
     tc::kda_tc_state_pass_kernel<<<gridB, 256, tc::KB_DYN, stream>>>(ws, S0, S_out, o, cu_seqlens, N, T, H, 0,
                                                                       tc::kPassPlain, nullptr, nullptr,
-                                                                      cu_seqlens ? chunk_total : nullptr);
+                                                                      cu_seqlens ? chunk_total : nullptr, esc);
     e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (units > 0) {
+    e = fu::launch_fused(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, ws + lay.fused, s_sms, gmode,
+                         stream, fu::kFusedMain, esc);
     if (e != cudaSuccess) return e;
   }
   if (ev && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;

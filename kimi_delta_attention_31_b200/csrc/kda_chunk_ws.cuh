@@ -77,8 +77,7 @@ constexpr uint32_t WS_RB = 131072;     // K e^-G K-major 2 panels [64][64]; befo
                                        // warp totals of g [8][128] fp32                        16384
 constexpr uint32_t WS_UW = 147456;     // staging U^T | W^T (image order)                       32768
 constexpr uint32_t WS_AS = 180224;     // A fp32 [64][68], then T over it                      17408
-constexpr uint32_t WS_TLO = WS_AS + 17408;  // T diag(beta) bf16 lo part K-major [64][64]       8192
-                                       // (free)                                                9216
+                                       // (free)                                               17408
 constexpr uint32_t WS_TT = 215040;     // T diag(beta) bf16 K-major [64][64]; before the solve
                                        // the P staging                                        8192
 constexpr uint32_t WS_BYTES = WS_TT + 8192;
@@ -86,7 +85,7 @@ constexpr uint32_t WS_DYN = WS_BYTES + 1024;
 static_assert(WS_AS + 2 * 17408 == WS_TT && WS_L3 + 2 * WS_L3_PANEL == WS_RB && WS_RB + 16384 == WS_UW &&
                   WS_UW + 32768 == WS_AS, "layout");
 static_assert(8 * D * 4 <= 16384, "scratch sizes");
-static_assert(WS_TLO % 1024 == 0 && WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_V % 1024 == 0 &&
+static_assert(WS_TT % 1024 == 0 && WS_RB % 1024 == 0 && WS_L3 % 1024 == 0 && WS_V % 1024 == 0 &&
                   WS_UW % 1024 == 0, "alignment");
 static_assert(IMG_A1 - IMG_U == 16384 && IMG_U - IMG_P == 8192, "image order");
 
@@ -215,7 +214,8 @@ __global__ void __launch_bounds__(512, 1)
                               uint32_t num_items, FastDiv fdH,
                               FastDiv fdC, uint8_t* __restrict__ ws, uint32_t* __restrict__ steep_list,
                               uint32_t* __restrict__ steep_cnt, uint32_t list_cap,
-                              const int2* __restrict__ chunk_table, const int* __restrict__ chunk_total) {
+                              const int2* __restrict__ chunk_table, const int* __restrict__ chunk_total,
+                              int* __restrict__ esc_flag) {
   constexpr bool kPrep = gate_prep(kGate);
   constexpr bool kTmaGate = kGate != kGateLogTok;
   __shared__ __align__(16) float s_beta[2][C];
@@ -525,11 +525,13 @@ __global__ void __launch_bounds__(512, 1)
       const bool skip = ptx::bar_or(2, 256, s_skip[slot] != 0);
       if (!skip) {
         // ---- scatter A (fp32, beta-scaled) and P (bf16, staged in the T diag(beta) buffer)
-        const bool big = tc::scatter_single_ref(tmem + 64 * slot, s_beta[slot], As, sm + WS_TT, warp, w8, lane,
-                                                slot == 1);
+        const bool big =
+            tc::scatter_single_ref(tmem + 64 * slot, s_beta[slot], As, sm + WS_TT, warp, w8, lane, slot == 1);
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
-        const bool accurate = ptx::bar_or(2, 256, big);
+        // near-parallel keys: this call's result is recomputed by the single-pass
+        // kernel in its precise form (kda_chunk_tc.cuh, launch_chunk_tc)
+        if (ptx::bar_or(2, 256, big) && st == 0) *esc_flag = 1;
         if (st == kIo) {
           ptx::bulk_s2g(ws + (size_t)item * IMG_BYTES + IMG_P, sm + WS_TT, 8192);
           ptx::bulk_commit();
@@ -537,28 +539,26 @@ __global__ void __launch_bounds__(512, 1)
         // ---- T = (I + A)^{-1}, T diag(beta) in bf16.  At each barrier thread kIo
         //      first waits for its stores to have read shared memory: T diag(beta)
         //      reuses the P staging (written after the first barrier).
-        tc::solve_t_beta(As, s_beta[slot], sm + WS_TT, sm + WS_TLO, accurate, st, w8, lane, [st] {
+        tc::solve_t_beta<false>(As, s_beta[slot], sm + WS_TT, nullptr, st, w8, lane, [st] {
           if (st == kIo) ptx::bulk_wait_read0();
           ptx::bar_sync(2, 256);
         }, [] {});
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::bar_sync(2, 256);
-        // ---- W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64,
-        //      T diag(beta) as its bf16 hi part, then its lo part
+        // ---- W^T = (K e^G)^T (T diag(beta))^T, U^T = V^T (T diag(beta))^T : M=128, N=64, K=64
         if (st == 0) {
           const bool have_v = wait_or_abort(&s_v_full, n & 1, abort_flag);
           if (have_v && !*abort_flag) {
             ptx::tc_fence_after();
             constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int kk = i & 3;
-              const uint64_t bd = ptx::sdesc_sw128(sb + (i < 4 ? WS_TT : WS_TLO) + kk * 32, 16, 1024);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bd = ptx::sdesc_sw128(sb + WS_TT + kk * 32, 16, 1024);
               const uint64_t xd = ptx::sdesc_sw128(sb + WS_L3 + (slot ? 16384 : 0) + kk * 2048, WS_L3_PANEL, 1024);
               const uint64_t vd = ptx::sdesc_sw128(sb + WS_V + kk * 2048, 8192, 1024);
-              ptx::mma_bf16(tmem + 128, xd, bd, id, i > 0);
-              ptx::mma_bf16(tmem + 192, vd, bd, id, i > 0);
+              ptx::mma_bf16(tmem + 128, xd, bd, id, kk > 0);
+              ptx::mma_bf16(tmem + 192, vd, bd, id, kk > 0);
             }
             ptx::mma_commit(&s_b_done[slot]);
           } else {
@@ -691,8 +691,8 @@ template <int kGate>
 inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                      const void* g, const float* beta, const int32_t* cu_seqlens, int num_seqs,
                                      int B, int T, int H, long long items, FastDiv fdH, FastDiv fdC, uint8_t* ws,
-                                     uint32_t* lists, const int2* table, const int* table_total, int sms,
-                                     cudaStream_t stream) {
+                                     uint32_t* lists, const int2* table, const int* table_total, int* esc_flag,
+                                     int sms, cudaStream_t stream) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   cudaError_t e = tensor_map_encoder(&enc);
   if (e != cudaSuccess) return e;
@@ -711,26 +711,27 @@ inline cudaError_t launch_ws_local_t(const __nv_bfloat16* q, const __nv_bfloat16
   uint32_t* cnt = lists + (size_t)grid * cap;
   if (cu_seqlens)
     kda_ws_chunk_local_kernel<kGate, true><<<grid, 512, WS_DYN, stream>>>(
-        mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap, table, table_total);
+        mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap, table, table_total,
+        esc_flag);
   else
     kda_ws_chunk_local_kernel<kGate, false><<<grid, 512, WS_DYN, stream>>>(
-        mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap, nullptr, nullptr);
+        mk, mq, mg, mv, g, beta, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap, nullptr, nullptr, esc_flag);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   tc::kda_tc_chunk_local_kernel<kGate><<<grid, 256, tc::KA_DYN, stream>>>(
       q, k, v, g, beta, cu_seqlens, cu_seqlens ? num_seqs : 0, T, H, (uint32_t)items, fdH, fdC, ws, lists, cnt, cap,
-      cu_seqlens ? table_total : nullptr);
+      cu_seqlens ? table_total : nullptr, esc_flag);
   return cudaGetLastError();
 }
 
 inline cudaError_t launch_ws_local(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                    const void* g, const float* beta, const int32_t* cu_seqlens, int num_seqs, int B,
                                    int T, int H, long long items, FastDiv fdH, FastDiv fdC, uint8_t* ws,
-                                   uint32_t* lists, const int2* table, const int* table_total, int sms, int gmode,
-                                   cudaStream_t stream) {
+                                   uint32_t* lists, const int2* table, const int* table_total, int* esc_flag,
+                                   int sms, int gmode, cudaStream_t stream) {
 #define KDA_WS_CASE(M)                                                                                     \
   case M:                                                                                                  \
     return launch_ws_local_t<M>(q, k, v, g, beta, cu_seqlens, num_seqs, B, T, H, items, fdH, fdC, ws, lists, \
-                                table, table_total, sms, stream)
+                                table, table_total, esc_flag, sms, stream)
   switch (gmode) {
     KDA_WS_CASE(kGateLogCh);
     KDA_WS_CASE(kGateLogTok);

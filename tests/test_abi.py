@@ -205,13 +205,17 @@ def test_local_kernel_switch():
     kda.set_local_kernel(1)
     try:
         assert not kda.uses_ws_kernel()
-        assert kda.chunk_fwd_kernel_sequence(2, 128, 4) == ["kda_tc_chunk_local_kernel", "kda_tc_state_pass_kernel"]
+        assert kda.chunk_fwd_kernel_sequence(2, 128, 4) == ["kda_fused_setup_kernel", "kda_tc_chunk_local_kernel",
+                                                            "kda_tc_state_pass_kernel", "kda_fused_prefill_kernel"]
     finally:
         kda.set_local_kernel(0)
     assert kda.uses_ws_kernel("log_token") and kda.uses_ws_kernel("logit", packed=True)
-    assert kda.chunk_fwd_kernel_sequence(2, 128, 4) == ["kda_ws_chunk_local_kernel", "kda_tc_chunk_local_kernel",
-                                                        "kda_tc_state_pass_kernel"]
-    assert kda.chunk_fwd_kernel_sequence(1, 300, 4, num_seqs=3)[0] == "kda_ws_chunk_table_kernel"
+    # the precise fallback's set-up kernel first, its single-pass kernel last
+    assert kda.chunk_fwd_kernel_sequence(2, 128, 4) == ["kda_fused_setup_kernel", "kda_ws_chunk_local_kernel",
+                                                        "kda_tc_chunk_local_kernel", "kda_tc_state_pass_kernel",
+                                                        "kda_fused_prefill_kernel"]
+    assert kda.chunk_fwd_kernel_sequence(1, 300, 4, num_seqs=3)[:2] == ["kda_fused_setup_kernel",
+                                                                       "kda_ws_chunk_table_kernel"]
     with pytest.raises(ValueError):
         kda.uses_ws_kernel("per_head")
 

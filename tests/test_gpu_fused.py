@@ -5,7 +5,8 @@ in tensor memory.  Against the fp64 oracle at the bf16 tolerance, and against
 the two-kernel path on the same inputs, across shapes with ragged chunks,
 packed sequences (empty ones included), chunks past the single-reference decay
 range, the per-token gate, raw projections, S_out aliasing S0, and more units
-than SMs (the dynamic unit schedule)."""
+than SMs (the dynamic unit schedule); and in its role as the two-kernel
+path's precise fallback for chunks with near-parallel keys."""
 import numpy as np
 import pytest
 import torch
@@ -135,3 +136,39 @@ def test_fused_workspace_is_small(cuda_device):
         assert kda.prefill_phases(8, 8192, 32) == 1
     finally:
         kda.set_prefill_path(kda.PATH_AUTO)
+
+
+def _repeated_key_input(B, T, H, seed, device):
+    inp = W.make_prefill(B, T, H, 128, 128, "bf16", -3.0, 1.0, 0.0, seed=seed, device=device)
+    inp["k"][:] = inp["k"][:, :1]
+    inp["beta"].fill_(1.0)
+    inp["g"].zero_()
+    return inp
+
+
+@pytest.mark.parametrize("segments", [0, 4])
+def test_two_kernel_path_falls_back_on_near_parallel_keys(cuda_device, segments):
+    """One repeated key makes every entry of A about 1: the two-kernel path's
+    chunk-local kernels raise the fallback flag, its state pass stands down and
+    the single-pass kernel recomputes the call, so the two-kernel call returns
+    exactly the single pass's result (and meets the bf16 tolerance), with or
+    without sequence segments."""
+    inp = _repeated_key_input(1, 2048, 2, 571, cuda_device)
+    kda.set_segment_chunks(segments if segments else -1)
+    try:
+        (o1, S1), (o2, S2) = _both_paths(_prefill(inp))
+        if segments:
+            assert kda.segment_chunks(1, 2048, 2) == segments
+    finally:
+        kda.set_segment_chunks(0)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    compare_units(inp, o2, S2, [(0, 0), (0, 1)], 1e-2)
+
+
+def test_two_kernel_path_keeps_its_own_result_on_ordinary_keys(cuda_device):
+    """Random unit keys never reach |A| >= 0.5 here: the fallback stays idle and
+    the two paths' (different) roundings give different bits."""
+    inp = W.make_prefill(2, 512, 4, 128, 128, "bf16", -4.0, 1.0, 0.02, seed=572, device=cuda_device)
+    (o1, S1), (o2, S2) = _both_paths(_prefill(inp))
+    assert not torch.equal(o1, o2)
+    assert rel_rms(o1.float().cpu().numpy(), o2.float().cpu().numpy()) < 1e-2
