@@ -255,10 +255,11 @@ kda_status_t kda_chunk_fwd_host(const void* q, const void* k, const void* v, con
  * bytes on every GPU that loads the library, held until process exit.  Sizes
  * whose kda_chunk_fwd_workspace_size(...) exceeds it are rejected with
  * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill
- * (kda_set_prefill_path(1)) needs 256 + 4 * num_seqs bytes, the
- * fp32-arithmetic path none; the two-kernel path (the default) keeps a
- * per-chunk image and can exceed it: 64 MiB hold 903 of its (chunk, head)
- * pairs, e.g. B=1, H=8, T=7168.
+ * (the default for packed sequences with at least one unit per SM, or
+ * kda_set_prefill_path(1)) needs 256 + 4 * num_seqs bytes, the
+ * fp32-arithmetic path none; the two-kernel path keeps a per-chunk image and
+ * can exceed it: 64 MiB hold 903 of its (chunk, head) pairs, e.g. B=1, H=8,
+ * T=7168.
  * The first call on each device looks up the array's device address (with
  * that device current) and remembers it together with the CUDA context that
  * was current; a call from another context on that device (a driver-API
@@ -349,7 +350,9 @@ kda_status_t kda_set_local_kernel(int variant);
  *   2 = two kernels: every chunk's operands built in parallel into a per-chunk
  *       workspace image, then a state pass over the chunks of each unit (the
  *       path that also splits long sequences into segments);
- *   0 = automatic (default): the two kernels, faster on every shape measured.
+ *   0 = automatic (default): the single pass for packed sequences with at
+ *       least one (sequence, head) unit per SM (it balances unequal lengths
+ *       longest first), the two kernels otherwise.
  * The two-kernel path keeps U and E in bf16 and T diag(beta) without its lo
  * part, which is accurate unless a chunk has near-parallel keys (some
  * |A_rj| >= 0.5, e.g. a key repeated within a chunk): its chunk-local kernels

@@ -1388,14 +1388,20 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
 // 0 automatic (the single pass unless segments were chosen), 1 single pass,
 // 2 two kernels.  Returns true for the single pass.
 constexpr int kPathAuto = 0, kPathFused = 1, kPathTwoKernel = 2;
-// The single pass runs when asked for (kda_set_prefill_path(1)); the
-// automatic choice is the two-kernel path, faster on every measured shape and,
-// with its precise fallback, as accurate.
+// Which tensor-core prefill a call runs.  Automatic: the single pass for packed
+// sequences with at least one (sequence, head) unit per SM -- its CTAs take
+// whole units longest first, where the two-kernel state pass deals them out in
+// order, and sequence lengths that differ by 64x leave its SMs idle (16
+// sequences of 1 K to 64 K tokens, 32 heads: 11.7 against 15.6 ms); the
+// two-kernel path otherwise (uniform batches: 1.71 against 1.80 ms at B8 H32
+// T8192; few units: sequence segments).  With its precise fallback the
+// two-kernel path is as accurate as the single pass.
 inline bool tc_use_fused(int B, int T, int H, int num_seqs, int sms, int seg_chunks, int force) {
-  if (force != kPathFused || seg_chunks > 0 || sms <= 0) return false;
+  if (force == kPathTwoKernel || seg_chunks > 0 || sms <= 0) return false;
   const long long N = num_seqs > 0 ? num_seqs : B;
   const long long tokens = (long long)B * T;
-  return tokens < (1LL << 31) && N * H < (1LL << 31);
+  if (tokens >= (1LL << 31) || N * H >= (1LL << 31)) return false;
+  return force == kPathFused || (num_seqs > 0 && N * H >= sms);
 }
 
 // Workspace: the per-chunk images, then (segmented runs) the maps [N | M] of
