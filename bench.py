@@ -696,6 +696,7 @@ def run_ours(args):
             "config": headline_config(w, world),
             "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": e2e,
             "workspace_bytes": head["workspace_bytes"], "kernels_per_call": head["kernels_per_call"],
+            "other_path": head.get("other_path"),
             "cfg1": cfg1, "cfg2": cfg2, "cfg4": cfg4, "decode": decode, "gdn": gdn, "prep": prep,
             "long_seq": long_seq, "bwd": bwd,
             "gpu_launches": gpu_launches, "clocks": clocks}

@@ -254,9 +254,8 @@ kda_status_t kda_chunk_fwd_host(const void* q, const void* k, const void* v, con
  * Its scratch is a fixed array inside the library, KDA_NOALLOC_SCRATCH_BYTES
  * bytes on every GPU that loads the library, held until process exit.  Sizes
  * whose kda_chunk_fwd_workspace_size(...) exceeds it are rejected with
- * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill
- * (the default for packed sequences with at least one unit per SM, or
- * kda_set_prefill_path(1)) needs 256 + 4 * num_seqs bytes, the
+ * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill (see
+ * kda_set_prefill_path) needs 256 + 4 * (num_seqs + N * H) bytes, the
  * fp32-arithmetic path none; the two-kernel path keeps a per-chunk image and
  * can exceed it: 64 MiB hold 903 of its (chunk, head) pairs, e.g. B=1, H=8,
  * T=7168.
@@ -352,7 +351,13 @@ kda_status_t kda_set_local_kernel(int variant);
  *       path that also splits long sequences into segments);
  *   0 = automatic (default): the single pass for packed sequences with at
  *       least one (sequence, head) unit per SM (it balances unequal lengths
- *       longest first), the two kernels otherwise.
+ *       longest first) and for batches whose units fill their waves (one
+ *       unit per SM) to at least 80% (on 148 SMs: 128 or 256 units, e.g.
+ *       B8 H32), with at least 16 chunks per sequence; the two kernels
+ *       otherwise.
+ * The single pass runs a plain instance and then a precise one, which
+ * recomputes only the units where the plain one met near-parallel keys (some
+ * |A_rj| >= 0.5) and returns at once when there are none.
  * The two-kernel path keeps U and E in bf16 and T diag(beta) without its lo
  * part, which is accurate unless a chunk has near-parallel keys (some
  * |A_rj| >= 0.5, e.g. a key repeated within a chunk): its chunk-local kernels

@@ -507,7 +507,9 @@ def chunk_fwd_kernel_sequence(B, T, H, dk=128, dv=128, chunk_size=64, dtype=torc
     if launches_per_chunk_fwd(dk, dv, chunk_size, dtype) == 1:
         return list(KERNELS_SIMT)
     if uses_fused_kernel(B, T, H, num_seqs, dk, dv, chunk_size, dtype):
-        return ["kda_fused_setup_kernel", KERNEL_FUSED]
+        # the plain instance, then the precise one (it returns at once unless the
+        # plain one marked a unit with near-parallel keys)
+        return ["kda_fused_setup_kernel", KERNEL_FUSED, KERNEL_FUSED]
     # the precise fallback's set-up first and its single-pass kernel last (it
     # returns at once unless a chunk-local kernel met near-parallel keys)
     seq = ["kda_fused_setup_kernel"] + (["kda_ws_chunk_table_kernel"] if num_seqs > 0 else [])

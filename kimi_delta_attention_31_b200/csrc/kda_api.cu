@@ -324,7 +324,7 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
   if (!use_tensor_core_path(dk, dv, chunk_size, dtype)) return 0;
   const int N = num_seqs > 0 ? num_seqs : B;
   const TcPlan plan = tc_plan(B, T, H, num_seqs);
-  if (plan.fused) return kda::fu::fused_workspace_bytes(num_seqs);
+  if (plan.fused) return kda::fu::fused_workspace_bytes(num_seqs, (long long)N * H);
   return kda::tc_workspace_layout(max_chunks(B, T, num_seqs, chunk_size), H, (long long)N * H, T, plan.seg,
                                   num_seqs).total;
 }

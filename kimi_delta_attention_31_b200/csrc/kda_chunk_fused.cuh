@@ -121,7 +121,7 @@ struct FuItem {
   int unit;      // sequence * H + head
   int Cn;        // valid rows (0 for an empty sequence)
   int flags;
-  int pad;
+  int ord;       // the unit's ordinal among this CTA's units
 };
 
 template <int kGate>
@@ -171,7 +171,7 @@ __device__ __forceinline__ void zero_cols64(uint32_t ta) {
   for (int i = 0; i < 4; ++i) ptx::tmem_st16(ta + 16 * i, z);
 }
 
-template <int kGate, bool kPacked>
+template <int kGate, bool kPacked, bool kPrecise>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_fused_prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
@@ -180,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                              const float* __restrict__ S0, bf16* __restrict__ o, float* __restrict__ S_out,
                              const int32_t* __restrict__ cu_seqlens, int N, int T, int H,
                              int* __restrict__ unit_ctr, const int* __restrict__ seq_order,
-                             const int* __restrict__ seq_status, const int* __restrict__ esc_flag) {
+                             const int* __restrict__ seq_status, const int* __restrict__ esc_flag,
+                             int* __restrict__ unit_mark, int* __restrict__ any_mark) {
   constexpr bool kPrep = gate_prep(kGate);
   constexpr bool kTmaGate = kGate != kGateLogTok;
   __shared__ __align__(16) float s_beta[2][C];
@@ -192,10 +193,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t s_x_free, s_uw_done, s_m1, s_m3, s_st, s_drain, s_p_free[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ int s_doom[4];  // plain instance: unit (ordinal mod 4) met a chunk with near-parallel keys
   // packed sequences whose cu_seqlens the set-up kernel rejected: no work at all
   if (kPacked && *seq_status < 0) return;
-  // run as the two-kernel path's precise fallback: nothing to do unless one of
-  // its chunk-local kernels met near-parallel keys
+  // the precise instance, run after the plain one (or after the two-kernel
+  // path): nothing to do unless a chunk with near-parallel keys was met
   if (esc_flag && *esc_flag == 0) return;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   KDA_ALIGNED_DSMEM(sm, dsm_raw);
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // other threads of the group.
   __shared__ struct {
     long long t0;
-    int c, nc, len, unit, done;
+    int c, nc, len, unit, done, ord;
   } s_gen;
   int& g_c = s_gen.c;
   int& g_nc = s_gen.nc;
@@ -218,21 +220,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   int& g_done = s_gen.done;
   long long& g_t0 = s_gen.t0;
   auto gen = [&](FuItem& it) {
-    it.pad = 0;
     if (g_done) {
       it.flags = kItEnd;
       return;
     }
     if (g_c >= g_nc) {
-      const int u = atomicAdd(unit_ctr, 1);
-      if (u >= units) {
-        g_done = 1;
-        it.flags = kItEnd;
-        return;
+      int seq;
+      for (;;) {
+        const int u = atomicAdd(unit_ctr, 1);
+        if (u >= units) {
+          g_done = 1;
+          it.flags = kItEnd;
+          return;
+        }
+        const int rank = u / H, hh = u - rank * H;
+        seq = seq_order ? seq_order[rank] : rank;
+        g_unit = seq * H + hh;
+        // the precise instance after the plain one takes only the units it marked
+        if (!kPrecise || !unit_mark || unit_mark[g_unit]) break;
       }
-      const int rank = u / H, hh = u - rank * H;
-      const int seq = seq_order ? seq_order[rank] : rank;
-      g_unit = seq * H + hh;
+      ++s_gen.ord;
       if constexpr (kPacked) {
         long long a, b;
         checked_seq_range(cu_seqlens, seq, T, &a, &b);
@@ -249,11 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         it.unit = g_unit;
         it.Cn = 0;
         it.flags = kItFirst | kItLast | kItEmpty;
+        it.ord = s_gen.ord;
         return;
       }
     }
     it.s0 = g_t0 + (long long)g_c * C;
     it.unit = g_unit;
+    it.ord = s_gen.ord;
     it.Cn = min(C, g_len - g_c * C);
     it.flags = (g_c == 0 ? kItFirst : 0) | (g_c == g_nc - 1 ? kItLast : 0);
     ++g_c;
@@ -282,6 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_abort = 0;
     ptx::fence_mbar_init();
     g_c = g_nc = g_len = g_unit = g_done = 0;
+    s_gen.ord = 0;
+    for (int i = 0; i < 4; ++i) s_doom[i] = 0;
     g_t0 = 0;
     for (int i = 0; i < 3; ++i) gen(s_ring[i]);
   }
@@ -701,6 +712,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         const bool accurate = ptx::bar_or(2, 256, big);
+        // the plain instance leaves such a chunk to the precise one: it marks the unit
+        if (!kPrecise && accurate && st == 0) s_doom[it.ord & 3] = 1;
         // T = (I + A)^{-1} over A, T diag(beta) as bf16 hi (FU_TT), and for a chunk
         // with near-parallel keys also its lo part (FU_TLO).  V of chunk n+1 goes
         // into the other slot (its V, chunk n-1's, is read) from the warp that is
@@ -709,8 +722,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto idle = [&] {
           if (lane == 0) issue_v(n + 1, v_issued);
         };
-        if (accurate) tc::solve_t_beta_precise(As, s_beta[s], sm + FU_TT, sm + FU_TLO, st, w8, lane, sync2, idle);
-        else tc::solve_t_beta<false>(As, s_beta[s], sm + FU_TT, nullptr, st, w8, lane, sync2, idle);
+        if (kPrecise && accurate)
+          tc::solve_t_beta_precise(As, s_beta[s], sm + FU_TT, sm + FU_TLO, st, w8, lane, sync2, idle);
+        else
+          tc::solve_t_beta<false>(As, s_beta[s], sm + FU_TT, nullptr, st, w8, lane, sync2, idle);
         ptx::fence_proxy_async_smem();
         ptx::bar_sync(2, 256);
         // ---- W^T = (K e^G)^T (T diag(beta))^T into TMEM slot s (free since the
@@ -724,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             constexpr uint32_t id = ptx::idesc_bf16(128, 64, true, false);
             const uint32_t kg = sb + FU_L3 + s * FU_L3_SLOT, vs = sb + FU_V + s * 16384;
-            const int parts = accurate ? 2 : 1;
+            const int parts = kPrecise && accurate ? 2 : 1;
 #pragma unroll 1
             for (int part = 0; part < parts; ++part) {
               const uint32_t tb = sb + (part ? FU_TLO : FU_TT);
@@ -918,10 +933,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       zero_cols64(tmem + lo_lane + kTmO);  // the next chunk's first MMA accumulates O onto zeros
+      // plain instance, the unit's last chunk: a unit that met near-parallel keys
+      // is left to the precise instance (its state is not written, so an S_out
+      // aliasing S0 keeps S0; its output rows are written again)
+      const bool doomed = !kPrecise && (it.flags & kItLast) && s_doom[it.ord & 3] != 0;
       ptx::fence_proxy_async_smem();
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::bar_sync(3, 128);  // every read of X^T done; tile complete
+      if (doomed && st == 0) {
+        s_doom[it.ord & 3] = 0;
+        unit_mark[it.unit] = 1;
+        *any_mark = 1;
+      }
       const int h = it.unit % H;
       if (it.Cn == C) {  // a whole chunk: two tensor stores
         if (st == 0) {
@@ -941,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::bar_sync(3, 128);  // the tile is read
       }
-      if ((it.flags & kItLast) && S_out) {
+      if ((it.flags & kItLast) && S_out && !doomed) {
 #pragma unroll 1
         for (int c32 = 0; c32 < D; c32 += 32) {
           float x[32];
@@ -980,9 +1004,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) ptx::tmem_dealloc(tmem, kTmCols);
 }
 
-// Set-up of one call (one CTA of 1024 threads): zeroes the unit counter (and,
-// when the two-kernel path runs this kernel as its precise fallback, the flag
-// its chunk-local kernels raise) and,
+// Set-up of one call (one CTA of 1024 threads): zeroes the unit counters, the
+// unit marks (and, when the two-kernel path runs the precise instance as its
+// fallback, the flag its chunk-local kernels raise) and,
 // for packed sequences, checks cu_seqlens (cu[0] == 0, non-decreasing,
 // cu[num_seqs] == T) -- a bad table raises the device error word and sets
 // *status = -1, so the prefill kernel does nothing -- then orders the
@@ -991,13 +1015,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kSortMax = 2048;
 __global__ void __launch_bounds__(1024)
     kda_fused_setup_kernel(const int32_t* __restrict__ cu_seqlens, int num_seqs, int T, int* __restrict__ ctr,
-                           int* __restrict__ status, int* __restrict__ order, int* __restrict__ esc_flag) {
+                           int* __restrict__ status, int* __restrict__ order, int* __restrict__ esc_flag,
+                           int* __restrict__ unit_mark, int units) {
   __shared__ int s_len[kSortMax];
   const int tid = threadIdx.x;
   if (tid == 0) {
-    *ctr = 0;
+    ctr[0] = ctr[1] = ctr[2] = 0;  // the plain and precise instances' unit counters, the any-unit mark
     if (esc_flag) *esc_flag = 0;
   }
+  for (int i = tid; i < units; i += 1024) unit_mark[i] = 0;
   if (!cu_seqlens) return;
   bool bad = tid == 0 && (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T);
   for (int i = tid; i < num_seqs; i += 1024) bad |= cu_seqlens[i + 1] < cu_seqlens[i];
@@ -1029,8 +1055,12 @@ __global__ void __launch_bounds__(1024)
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-// Workspace: the unit counter, the table check's status, the sequence order.
-inline size_t fused_workspace_bytes(int num_seqs) { return 256 + (size_t)std::max(num_seqs, 0) * sizeof(int); }
+// Workspace: the plain and precise instances' unit counters, the any-unit
+// mark, the table check's status (ints 0..3), the sequence order (from byte
+// 256), then one mark per (sequence, head) unit.
+inline size_t fused_workspace_bytes(int num_seqs, long long units) {
+  return 256 + ((size_t)std::max(num_seqs, 0) + (size_t)std::max(units, 0LL)) * sizeof(int);
+}
 
 inline bool fused_kernel_available() {
   static PerDeviceOnce once;
@@ -1038,14 +1068,14 @@ inline bool fused_kernel_available() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   run_once_per_device(once, [dev] {
-    const void* fns[] = {(const void*)kda_fused_prefill_kernel<kGateLogCh, false>,
-                         (const void*)kda_fused_prefill_kernel<kGateLogTok, false>,
-                         (const void*)kda_fused_prefill_kernel<kGateLogitF32, false>,
-                         (const void*)kda_fused_prefill_kernel<kGateLogitBf16, false>,
-                         (const void*)kda_fused_prefill_kernel<kGateLogCh, true>,
-                         (const void*)kda_fused_prefill_kernel<kGateLogTok, true>,
-                         (const void*)kda_fused_prefill_kernel<kGateLogitF32, true>,
-                         (const void*)kda_fused_prefill_kernel<kGateLogitBf16, true>};
+    const void* fns[] = {
+#define KDA_FU_FN(M) (const void*)kda_fused_prefill_kernel<M, false, false>,                                      \
+                     (const void*)kda_fused_prefill_kernel<M, true, false>,                                       \
+                     (const void*)kda_fused_prefill_kernel<M, false, true>,                                       \
+                     (const void*)kda_fused_prefill_kernel<M, true, true>
+        KDA_FU_FN(kGateLogCh), KDA_FU_FN(kGateLogTok), KDA_FU_FN(kGateLogitF32), KDA_FU_FN(kGateLogitBf16)
+#undef KDA_FU_FN
+    };
     int optin = 0;
     bool all = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
     for (const void* fn : fns) {
@@ -1061,12 +1091,15 @@ inline bool fused_kernel_available() {
   return ok[dev];
 }
 
-// Launches the set-up kernel (phase & kFusedSetup) and the prefill kernel
-// (phase & kFusedMain).  With esc_flag the pair is the two-kernel path's
-// precise fallback: the set-up kernel zeroes *esc_flag, and the prefill kernel
-// (launched after the two-kernel path's state pass) does the call's work only
-// if a chunk-local kernel has raised it meanwhile.
-constexpr int kFusedSetup = 1, kFusedMain = 2;
+// Launches the set-up kernel (phase & kFusedSetup), the plain instance of the
+// prefill kernel (phase & kFusedMain) and its precise instance (phase &
+// kFusedPrecise).  After the plain instance, the precise one recomputes only
+// the units the plain one marked (those with a chunk of near-parallel keys)
+// and returns at once when there are none.  With esc_flag the set-up kernel
+// and the precise instance are the two-kernel path's precise fallback: the
+// set-up kernel zeroes *esc_flag, and the precise instance (launched after the
+// state pass) recomputes the whole call only if a chunk-local kernel raised it.
+constexpr int kFusedSetup = 1, kFusedMain = 2, kFusedPrecise = 4;
 template <int kGate>
 inline cudaError_t launch_fused_t(const bf16* q, const bf16* k, const bf16* v, const void* g, const float* beta,
                                   const float* S0, bf16* o, float* S_out, const int32_t* cu_seqlens, int N,
@@ -1086,30 +1119,54 @@ inline cudaError_t launch_fused_t(const bf16* q, const bf16* k, const bf16* v, c
   } else {
     if ((e = ws::encode_rows_map(enc, &mg, g, kGate != kGateLogitBf16, tokens, H, D, false)) != cudaSuccess) return e;
   }
+  const long long units = (long long)N * H;
   int* wsi = static_cast<int*>(workspace);
-  int* ctr = wsi;
-  int* status = wsi + 1;
+  int* ctr_plain = wsi;
+  int* ctr_precise = wsi + 1;
+  int* any_mark = wsi + 2;
+  int* status = wsi + 3;
   int* order = wsi + 64;
+  int* marks = wsi + 64 + (cu_seqlens ? N : 0);
   if (phase & kFusedSetup) {
-    kda_fused_setup_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, cu_seqlens ? N : 0, T, ctr, status, order, esc_flag);
+    kda_fused_setup_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, cu_seqlens ? N : 0, T, ctr_plain, status, order,
+                                                   esc_flag, marks, (int)units);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const long long units = (long long)N * H;
   const int grid = (int)std::min<long long>(units, sms);
-  if (grid <= 0 || !(phase & kFusedMain)) return cudaSuccess;
-  if (cu_seqlens)
-    kda_fused_prefill_kernel<kGate, true><<<grid, kThreads, FU_DYN, stream>>>(
-        mk, mq, mg, mv, mo, g, beta, S0, o, S_out, cu_seqlens, N, T, H, ctr, order, status, esc_flag);
-  else
-    kda_fused_prefill_kernel<kGate, false><<<grid, kThreads, FU_DYN, stream>>>(
-        mk, mq, mg, mv, mo, g, beta, S0, o, S_out, nullptr, N, T, H, ctr, nullptr, status, esc_flag);
-  return cudaGetLastError();
+  if (grid <= 0) return cudaSuccess;
+  const int* ord = cu_seqlens ? order : nullptr;
+  if (phase & kFusedMain) {
+    if (cu_seqlens)
+      kda_fused_prefill_kernel<kGate, true, false><<<grid, kThreads, FU_DYN, stream>>>(
+          mk, mq, mg, mv, mo, g, beta, S0, o, S_out, cu_seqlens, N, T, H, ctr_plain, ord, status, nullptr, marks,
+          any_mark);
+    else
+      kda_fused_prefill_kernel<kGate, false, false><<<grid, kThreads, FU_DYN, stream>>>(
+          mk, mq, mg, mv, mo, g, beta, S0, o, S_out, nullptr, N, T, H, ctr_plain, ord, status, nullptr, marks,
+          any_mark);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (phase & kFusedPrecise) {
+    // after the plain instance: its marked units; as the two-kernel fallback: all
+    const int* gate_flag = esc_flag ? esc_flag : any_mark;
+    int* filter = esc_flag ? nullptr : marks;
+    if (cu_seqlens)
+      kda_fused_prefill_kernel<kGate, true, true><<<grid, kThreads, FU_DYN, stream>>>(
+          mk, mq, mg, mv, mo, g, beta, S0, o, S_out, cu_seqlens, N, T, H, ctr_precise, ord, status, gate_flag,
+          filter, any_mark);
+    else
+      kda_fused_prefill_kernel<kGate, false, true><<<grid, kThreads, FU_DYN, stream>>>(
+          mk, mq, mg, mv, mo, g, beta, S0, o, S_out, nullptr, N, T, H, ctr_precise, ord, status, gate_flag,
+          filter, any_mark);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 inline cudaError_t launch_fused(const bf16* q, const bf16* k, const bf16* v, const void* g, const float* beta,
                                 const float* S0, bf16* o, float* S_out, const int32_t* cu_seqlens, int N, int B,
                                 int T, int H, void* workspace, int sms, int gmode, cudaStream_t stream,
-                                int phase = kFusedSetup | kFusedMain, int* esc_flag = nullptr) {
+                                int phase = kFusedSetup | kFusedMain | kFusedPrecise, int* esc_flag = nullptr) {
 #define KDA_FU_CASE(M)                                                                                          \
   case M:                                                                                                       \
     return launch_fused_t<M>(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, workspace, sms, stream, \

@@ -1388,20 +1388,29 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
 // 0 automatic (the single pass unless segments were chosen), 1 single pass,
 // 2 two kernels.  Returns true for the single pass.
 constexpr int kPathAuto = 0, kPathFused = 1, kPathTwoKernel = 2;
-// Which tensor-core prefill a call runs.  Automatic: the single pass for packed
-// sequences with at least one (sequence, head) unit per SM -- its CTAs take
-// whole units longest first, where the two-kernel state pass deals them out in
-// order, and sequence lengths that differ by 64x leave its SMs idle (16
-// sequences of 1 K to 64 K tokens, 32 heads: 11.7 against 15.6 ms); the
-// two-kernel path otherwise (uniform batches: 1.71 against 1.80 ms at B8 H32
-// T8192; few units: sequence segments).  With its precise fallback the
-// two-kernel path is as accurate as the single pass.
+// Which tensor-core prefill a call runs.  The single pass keeps one
+// (sequence, head) unit per SM, so its time goes in whole waves of units; the
+// two-kernel path spreads the chunk-local work over every SM.  Measured
+// (B200, 148 SMs): B4 H32 T4096 (128 units, one wave) 0.39 against 0.50 ms;
+// B8 H32 T8192 (256 units, two waves) 1.63 against 1.70 ms; B16 H32 T8192
+// (512 units, four waves) 3.06 against 3.38 ms; B1 H16 T4096 (16 units) 0.34
+// against 0.24 ms; 16 packed sequences of 1 K to 64 K tokens, 32 heads: 11.7
+// against 15.6 ms (its CTAs take whole units longest first, where the
+// two-kernel state pass deals them out in order).  Automatic choice: the
+// single pass for packed sequences with at least one unit per SM, and for
+// batches whose units fill their waves to 80% or more; the two-kernel path
+// otherwise (with sequence segments for few, long sequences).  Both paths
+// meet the same tolerance (the two-kernel path through its precise fallback).
 inline bool tc_use_fused(int B, int T, int H, int num_seqs, int sms, int seg_chunks, int force) {
   if (force == kPathTwoKernel || seg_chunks > 0 || sms <= 0) return false;
   const long long N = num_seqs > 0 ? num_seqs : B;
   const long long tokens = (long long)B * T;
   if (tokens >= (1LL << 31) || N * H >= (1LL << 31)) return false;
-  return force == kPathFused || (num_seqs > 0 && N * H >= sms);
+  if (force == kPathFused) return true;
+  const long long units = N * H;
+  if (num_seqs > 0) return units >= sms;
+  const long long waves = (units + sms - 1) / sms;
+  return units * 10 >= waves * sms * 8 && (T + tc::C - 1) / tc::C >= 16;
 }
 
 // Workspace: the per-chunk images, then (segmented runs) the maps [N | M] of
@@ -1429,7 +1438,7 @@ inline TcWorkspace tc_workspace_layout(long long max_chunks, int H, long long un
   w.table = (w.lists + ((size_t)max_chunks * (size_t)H + 2 * kMaxListCtas) * sizeof(uint32_t) + 255) & ~(size_t)255;
   w.esc = (w.table + (size_t)max_chunks * sizeof(int2) + 16 + 255) & ~(size_t)255;
   w.fused = w.esc + 256;
-  w.total = w.fused + fu::fused_workspace_bytes(num_seqs);
+  w.total = w.fused + fu::fused_workspace_bytes(num_seqs, units);
   return w;
 }
 
@@ -1535,7 +1544,7 @@ inline cudaError_t launch_chunk_tc(const __nv_bfloat16* q, const __nv_bfloat16* 
   }
   if (units > 0) {
     e = fu::launch_fused(q, k, v, g, beta, S0, o, S_out, cu_seqlens, N, B, T, H, ws + lay.fused, s_sms, gmode,
-                         stream, fu::kFusedMain, esc);
+                         stream, fu::kFusedPrecise, esc);
     if (e != cudaSuccess) return e;
   }
   if (ev && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;

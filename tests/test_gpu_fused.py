@@ -172,3 +172,32 @@ def test_two_kernel_path_keeps_its_own_result_on_ordinary_keys(cuda_device):
     (o1, S1), (o2, S2) = _both_paths(_prefill(inp))
     assert not torch.equal(o1, o2)
     assert rel_rms(o1.float().cpu().numpy(), o2.float().cpu().numpy()) < 1e-2
+
+
+def test_single_pass_precise_instance_keeps_aliased_state(cuda_device):
+    """The plain instance leaves a unit with near-parallel keys to the precise
+    one without writing its state, so an S_out aliasing S0 still holds S0 when
+    the precise instance starts from it."""
+    inp = _repeated_key_input(2, 300, 2, 573, cuda_device)
+    inp["S0"] = 0.05 * torch.randn((2, 2, 128, 128), generator=torch.Generator(device=cuda_device).manual_seed(5),
+                                   device=cuda_device)
+    o_ref, S_ref = _on_path(kda.PATH_FUSED, _prefill(inp))
+    S0 = inp["S0"].clone()
+    o2, S2 = _on_path(kda.PATH_FUSED, _prefill(dict(inp, S0=S0), S_out=S0))
+    assert S2.data_ptr() == S0.data_ptr()
+    assert torch.equal(o2, o_ref) and torch.equal(S2, S_ref)
+    compare_units(inp, o_ref, S_ref, [(n, h) for n in range(2) for h in range(2)], 1e-2)
+
+
+def test_single_pass_recomputes_only_marked_units(cuda_device):
+    """Head 0 repeats one key (its unit is marked and recomputed by the precise
+    instance), head 1 has random keys: head 1's result is bit for bit the one
+    of a call in which no unit is marked."""
+    rnd = W.make_prefill(1, 512, 2, 128, 128, "bf16", -3.0, 1.0, 0.0, seed=574, device=cuda_device)
+    mixed = {k: (v.clone() if torch.is_tensor(v) else v) for k, v in rnd.items()}
+    mixed["k"][:, :, 0] = mixed["k"][:, :1, 0]
+    mixed["beta"][:, :, 0] = 1.0
+    o_r, S_r = _on_path(kda.PATH_FUSED, _prefill(rnd))
+    o_m, S_m = _on_path(kda.PATH_FUSED, _prefill(mixed))
+    assert torch.equal(o_m[:, :, 1], o_r[:, :, 1]) and torch.equal(S_m[:, 1], S_r[:, 1])
+    compare_units(mixed, o_m, S_m, [(0, 0), (0, 1)], 1e-2)
