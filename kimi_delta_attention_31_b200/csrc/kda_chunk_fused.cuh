@@ -22,41 +22,54 @@
 //   builder (warps 0..7)   chunk n+2: cumulative log-decays, the decay-scaled
 //                          operands [K e^G; Q e^G] (written over the raw k, q
 //                          rows in place) and K e^-G, the [A'; P'] MMA.
-//   solver  (warps 8..15)  chunk n+1: A and P out of TMEM, T = (I + A)^{-1},
-//                          T diag(beta) as a bf16 pair hi + lo, then two MMA
-//                          groups: W^T into the chunk's [A'; P'] columns (read
+//   solver  (warps 8..15)  chunk n+1: A and P out of TMEM and the |A| vote,
+//                          T = (I + A)^{-1} and T diag(beta) in bf16, then the
+//                          W^T MMA (into the chunk's [A'; P'] columns; read
 //                          back and written, negated, in bf16 over the K e^G
-//                          rows) and U^T straight into the state's columns.
+//                          rows in their own K-major layout) and the U^T MMA
+//                          (straight into the state's columns).
 //   state   (warps 16..19) chunk n: the state in TMEM, TRANSPOSED (lane = value
 //                          channel), so that every state-side product is an MMA
 //                          whose A operand sits in TMEM:
-//       E^T   = U^T + S^T (-W)^T,  (Q e^G S)^T    (N=64 each, K=128)
-//       S^T  += E^T (K e^-G),  (Q e^G S)^T += E^T P^T   (E as bf16 hi + lo)
+//       [E^T | (Q e^G S)^T] = [U^T | 0] + S^T [-W; Q e^G]^T  (one N=128 group, K=128)
+//       S^T  += E^T (K e^-G),  (Q e^G S)^T += E^T P^T          (E as bf16 hi + lo)
 //       S^T  *= e^{G_last} per key channel;  o = the second product
 // E enters the MMAs as a bf16 pair hi + lo (lo = the rounding error of hi),
 // so its fp32 value is used to about 2^-16; U is exact to fp32 accumulation;
 // W and S enter in bf16.
 //
+// Two instances.  The plain one (kPrecise = false) runs every chunk with plain
+// TF32 block products and T diag(beta) in bf16.  A chunk whose |A| vote fires
+// (some |A_rj| >= kSolveAccurateA: near-parallel keys) needs more: there the
+// plain instance marks the unit, and at the unit's end it does not write the
+// unit's state (an S_out aliasing S0 keeps S0).  The precise instance, launched
+// next, returns at once when no unit is marked and otherwise recomputes the
+// marked units, their voted chunks with split-TF32 block products and
+// T diag(beta) as a bf16 pair hi + lo (the W and U MMAs run on hi, then lo).
+// The precise instance is also the two-kernel path's fallback for the whole
+// call (kda_chunk_tc.cuh).
+//
 // TMEM columns: [A'; P'] slot 0 (0..63) | slot 1 (64..127) (also the W^T
 // accumulator) | U^T -> E^T (128..191) | (Q e^G S)^T -> O^T (192..255) | bf16
 // hi | lo of E^T (256..319) | S^T bf16 (320..383) | S^T fp32 (384..511).
 //
+// Copies: builder thread 0 issues the raw gate rows of chunk n+1 once the
+// group has read chunk n's; state thread 0 issues k, q of chunk n+2 once chunk
+// n's first state MMA has read its panel, and the output tile's two tensor
+// stores; solver warp 7, idle in the middle of the solve, issues V of chunk
+// n+1 (the slot's V, chunk n-1's, is read by then).  The output tile is staged
+// over the chunk's P slot (channels 0..63) and an 8 KB panel (64..127).
+//
 // Hand-offs (mbarriers; slot = chunk index mod 2):
-//   g_full        TMA of the raw gate rows (issued by builder thread 0 for the
-//                 next chunk once the group has read the current one)
-//   kq_full[s]    TMA of k, q (128-byte swizzled, straight into the operand
-//                 panels), issued by the state thread for chunk n+2 as soon as
-//                 chunk n's E MMA has read the panels; waited by the builder
-//   v_full[s]     TMA of V, issued by the state thread for chunk n+1 at the
-//                 start of chunk n (the slot held chunk n-1's V and then its
-//                 output tile, whose stores have read it by then); waited by
-//                 the solver before the U MMA
+//   g_full, kq_full[s], v_full[s]   the copies above (bytes)
 //   a_done[s]     [A'; P'] MMA complete + builder arrive        -> solver
 //   s_ready[s]    solver done (P, -W in shared memory, U^T in TMEM) -> state,
 //                 and -> builder (TMEM slot free for chunk n+2)
-//   rb_free[s]    state's MMAs of chunk n done (K e^-G and P read) -> builder
-//                 (K e^-G of chunk n+2), solver (P of n+2); gamma has four
-//                 slots, so the builder of chunk n+2 never meets chunk n's
+//   rb_free[s]    state's MMAs of chunk n done (K e^-G read) -> builder
+//                 (K e^-G of chunk n+2); gamma has four slots, so the builder
+//                 of chunk n+2 never meets chunk n's
+//   p_free[s]     chunk n's output tile is read (its P slot and the 8 KB panel
+//                 are free) -> solver (P of chunk n+2)
 //   x_free        the state has read chunk n's E^T -> the solver's U MMA of
 //                 the next chunk may write those columns
 //   uw_done, m1, m3, st   MMA completions inside one group.
