@@ -201,3 +201,27 @@ def test_single_pass_recomputes_only_marked_units(cuda_device):
     o_m, S_m = _on_path(kda.PATH_FUSED, _prefill(mixed))
     assert torch.equal(o_m[:, :, 1], o_r[:, :, 1]) and torch.equal(S_m[:, 1], S_r[:, 1])
     compare_units(mixed, o_m, S_m, [(0, 0), (0, 1)], 1e-2)
+
+
+@pytest.mark.parametrize("path", ["single", "two"])
+def test_packed_sequences_with_near_parallel_keys(cuda_device, path):
+    """Packed sequences (an empty one, ragged tails) where two of them repeat
+    one key: the single pass marks those units and its precise instance
+    recomputes them; the two-kernel path hands the call to its fallback.
+    Either way every unit meets the bf16 tolerance, and S_out may alias S0."""
+    lens = (300, 0, 129, 64, 450)
+    inp = W.make_prefill(1, sum(lens), 3, 128, 128, "bf16", -3.0, 1.0, 0.05, seed=575, device=cuda_device,
+                         lengths=lens)
+    cu = inp["cu_seqlens"]
+    for seq in (0, 4):  # sequences 0 and 4: one key repeated over the whole sequence, beta = 1
+        t0, t1 = int(cu[seq]), int(cu[seq + 1])
+        inp["k"][:, t0:t1] = inp["k"][:, t0:t0 + 1]
+        inp["beta"][:, t0:t1] = 1.0
+    p = kda.PATH_FUSED if path == "single" else kda.PATH_TWO_KERNEL
+    o_ref, S_ref = _on_path(p, _prefill(inp, cu))
+    units = [(n, h) for n in range(len(lens)) for h in range(3)]
+    compare_units(inp, o_ref, S_ref, units, 1e-2)
+    S0 = inp["S0"].clone()
+    o2, S2 = _on_path(p, _prefill(dict(inp, S0=S0), cu, S_out=S0))
+    assert S2.data_ptr() == S0.data_ptr()
+    assert torch.equal(o2, o_ref) and torch.equal(S2, S_ref)
