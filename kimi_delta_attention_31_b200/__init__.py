@@ -437,15 +437,19 @@ def set_local_kernel(variant: int) -> None:
 
 def set_prefill_path(path: int) -> None:
     """Tensor-core prefill for this thread's later calls: 0 = automatic
-    (default), 1 = the single-pass kernel, 2 = the two-kernel path."""
+    (default: the single pass when the (sequence, head) units fill their waves
+    of one unit per SM to 80%, or for packed sequences with a unit per SM; the
+    two-kernel path otherwise), 1 = the single-pass kernel, 2 = the two-kernel
+    path."""
     _check(load_library().kda_set_prefill_path(int(path)))
     _tls.prefill_path = int(path)
 
 
 def prefill_phases(B, T, H, num_seqs=0, dk=128, dv=128, chunk_size=64, dtype=torch.bfloat16) -> int:
     """Phases of one chunk_fwd call with these sizes on the current device and
-    this thread's settings (1: one kernel does the work; 2: chunk-local phase
-    and state pass)."""
+    this thread's settings (1: the fp32 path, or the single pass: its set-up
+    kernel and its plain and precise instances; 2: the two-kernel path's
+    chunk-local phase, then its state pass with the precise fallback)."""
     code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
     return int(load_library().kda_chunk_fwd_phases(B, T, H, num_seqs, dk, dv, chunk_size, code))
 
