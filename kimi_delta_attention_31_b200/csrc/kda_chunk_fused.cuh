@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_doom[4];  // plain instance: unit (ordinal mod 4) met a chunk with near-parallel keys
+  __shared__ int s_kq_mode;  // the state's k, q copies of the coming chunk: 1 = the four copies are armed
   // packed sequences whose cu_seqlens the set-up kernel rejected: no work at all
   if (kPacked && *seq_status < 0) return;
   // the precise instance, run after the plain one (or after the two-kernel
@@ -333,6 +334,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tma_load_3d(l3 + 16384, &tm_k, 64, h, (int)it.s0, &s_kq_full[s]);
     ptx::tma_load_3d(l3 + 8192, &tm_q, 0, h, (int)it.s0, &s_kq_full[s]);
     ptx::tma_load_3d(l3 + 16384 + 8192, &tm_q, 64, h, (int)it.s0, &s_kq_full[s]);
+  };
+  // The same copies in two steps: arm_kq (one thread) arms the barrier, or
+  // completes the phase with a plain arrive when there is nothing to copy, and
+  // returns 1 when the four copies are to follow; issue_kq_part(n, p) issues
+  // copy p (k or q, channels 0..63 or 64..127).
+  auto arm_kq = [&](uint32_t n, uint32_t* issued) -> int {
+    const FuItem it = s_ring[n & 7];
+    if (it.flags & kItEnd) return 0;
+    const int s = n & 1;
+    ++issued[s];
+    if ((it.flags & kItEmpty) || *abort_flag) {
+      ptx::mbar_arrive(&s_kq_full[s]);
+      return 0;
+    }
+    ptx::mbar_arrive_expect_tx(&s_kq_full[s], kKqBytes);
+    return 1;
+  };
+  auto issue_kq_part = [&](uint32_t n, int p) {
+    const FuItem it = s_ring[n & 7];
+    const int s = n & 1;
+    uint8_t* l3 = sm + FU_L3 + s * FU_L3_SLOT;
+    ptx::tma_load_3d(l3 + (p & 1) * 16384 + (p >> 1) * 8192, (p >> 1) ? &tm_q : &tm_k, 64 * (p & 1), it.unit % H,
+                     (int)it.s0, &s_kq_full[s]);
   };
   auto issue_v = [&](uint32_t n, uint32_t* issued) {
     const FuItem it = s_ring[n & 7];
@@ -810,14 +834,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     zero_cols64(tmem + lo_lane + kTmO);  // the first MMA accumulates O onto zeros
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
+    // chunk m's output tile is read by its tensor stores (issued by this thread):
+    // the tile's P slot and the 8 KB panel are free
+    auto release_tile = [&](uint32_t m) {
+      ptx::bulk_wait_read0();
+      ptx::mbar_arrive(&s_p_free[m & 1]);
+    };
     uint32_t real = 0;  // chunks with MMAs (phases of m1, m3, x_free)
     for (uint32_t n = 0;; ++n) {
       const int s = n & 1;
       const bool okr = wait_or_abort(&s_s_ready[s], (n >> 1) & 1, abort_flag);
-      if (st == 0 && n >= 1) {  // chunk n-1's output tile is read: its P slot and FU_OST are free
-        ptx::bulk_wait_read0();
-        ptx::mbar_arrive(&s_p_free[(n - 1) & 1]);
-      }
       if (ptx::bar_or(3, 128, !okr || *abort_flag)) break;  // uniform over the group
       ptx::tc_fence_after();
       const FuItem it = s_ring[n & 7];
@@ -827,6 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (S_out)
           for (int c = 0; c < D; ++c) S_out[(urow + c) * D + dv] = S0 ? S0[(urow + c) * D + dv] : 0.f;
         if (st == 0) {  // keep the per-chunk phases in step
+          if (n >= 1) release_tile(n - 1);
           issue_kq(n + 2, kq_issued);
           ptx::mbar_arrive(&s_rb_free[s]);
         }
@@ -862,6 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            ptx::sdesc_sw128(l3s + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id, 1);
         mma_issued = true;
         ptx::mma_commit(&s_m1);
+        if (n >= 1) release_tile(n - 1);  // while the MMAs run
       }
       const float* gam = reinterpret_cast<const float*>(sm + FU_GAM + (n & 3) * 512);
       if (steep) {  // Kbar form: decay the state first (the MMAs above read only the bf16 copy)
@@ -878,7 +906,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       bool ok = wait_or_abort(&s_m1, real & 1, abort_flag);
       ptx::tc_fence_after();
-      if (st == 0) issue_kq(n + 2, kq_issued);  // the slot's panels are read: chunk n+2's k, q may land
+      // the slot's panels are read: chunk n+2's k, q may land.  Thread 0 arms the
+      // barrier now; after the group barrier below each warp's lane 0 issues one
+      // of the four tensor copies, so that no thread issues all four.
+      if (st == 0) s_kq_mode = arm_kq(n + 2, kq_issued);
       // ---- E (fp32) as bf16 hi | lo
 #pragma unroll 1
       for (int h2 = 0; h2 < 2; ++h2) {
@@ -890,6 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       if (ptx::bar_or(3, 128, !ok || *abort_flag)) break;
+      if (lane == 0 && s_kq_mode) issue_kq_part(n + 2, qd);
       if (st == 0) {
         ptx::mbar_arrive(&s_x_free);  // E^T's columns are read: the next U^T may land there
         ptx::tc_fence_after();
