@@ -638,6 +638,47 @@ def decode_leg(kda, args, world, dev, stream, peaks, peak_src):
     return line
 
 
+def packed_shard_leg(kda, w, args, world, rank, dev, stream):
+    """The packed workload split across the ranks (N > 1 only): each rank
+    takes its longest-first share of the sequences (balanced by token count),
+    re-packs them contiguously, and runs kda_chunk_fwd on them alone.  The
+    time is the max over ranks, so the value is strong scaling of one fixed
+    workload; no collective touches the data."""
+    if world <= 1:
+        return None
+    from kimi_delta_attention_31_b200.sharding import assign_sequences_lpt, packed_subset
+    inp = W.make_workload(w, dev)
+    mine = assign_sequences_lpt(w.lengths, world)[rank]
+    ranges, cu = packed_subset(w.lengths, mine)
+    tokens = cu[-1]
+    run = None
+    if tokens > 0:
+        idx = torch.cat([torch.arange(a, b, dtype=torch.long) for a, b in ranges]).to(dev)
+        sub = {n: inp[n].index_select(1, idx).contiguous() for n in ("q", "k", "v", "g", "beta")}
+        S0 = inp["S0"][torch.tensor(mine, dtype=torch.long, device=dev)].contiguous() \
+            if inp["S0"] is not None else None
+        cu_t = torch.tensor(cu, dtype=torch.int32, device=dev)
+        o = torch.empty((1, tokens, w.H, w.dv), dtype=w.torch_dtype, device=dev)
+        S_out = torch.empty((len(mine), w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(kda.workspace_size(1, tokens, w.H, w.dk, w.dv, len(mine), w.chunk, w.torch_dtype), 1),
+                         dtype=torch.uint8, device=dev)
+
+        def run():
+            kda.chunk_fwd(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], S0, cu_t, w.chunk,
+                          o=o, S_out=S_out, workspace=ws)
+        for _ in range(args.warmup):
+            run()
+    del inp
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = time_launches(run, max(1, min(args.steps, 5)), stream) if run else 0.0
+    ms_max = max_over_ranks(ms, world, dev)
+    torch.cuda.synchronize()
+    return {"workload": w.name, "split": "sequences, longest first, by token count",
+            "value": w.tokens / (ms_max * 1e-3), "unit": "tokens/s", "ms_per_step": ms_max,
+            "scaling": "strong", "rank0_sequences": len(mine) if rank == 0 else None}
+
+
 def e2e_leg(kda, w, args, world, dev, stream):
     """The headline prefill end to end through the C ABI's host-buffer call
     (kda_chunk_fwd_host, wrapped by HostPrefill): every step copies the pinned
@@ -678,6 +719,9 @@ def run_ours(args):
     cfg1 = prefill_leg(kda, W.ORACLE_SMALL, args, world, dev, stream, peaks, peak_src, cpu_target_s=3.0)
     cfg2 = prefill_leg(kda, W.PREFILL_H16, args, world, dev, stream, peaks, peak_src, cpu_target_s=5.0)
     cfg4 = prefill_leg(kda, W.PREFILL_VARLEN, args, world, dev, stream, peaks, peak_src, cpu_target_s=8.0)
+    cfg4_split = packed_shard_leg(kda, W.PREFILL_VARLEN, args, world, rank, dev, stream)
+    if cfg4_split is not None:
+        cfg4["split_over_ranks"] = cfg4_split
     # ---------------- end to end through the host-buffer C call ----------------
     e2e = e2e_leg(kda, w, args, world, dev, stream)
     # ---------------- decode (config 5) ----------------
