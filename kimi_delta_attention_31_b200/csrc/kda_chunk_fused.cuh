@@ -151,6 +151,35 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
+// A block of 32 channels x 32 tokens of a transposed tile in TMEM (lane =
+// channel, column = token; `ta` = the warp's first lane and the block's first
+// column), times `sign`, as bf16 into a K-major tile in shared memory at
+// `tile`: row = token, 128-byte rows of 64 channels with the 128-byte swizzle,
+// channels 64..127 `panel` bytes further.  c0 and t0 are the block's first
+// channel and token in the tile.  8 x 8 pieces go through stmatrix with
+// transposition, so that each token's 8 channels are one 16-byte store.  One
+// warp; the roundings are those of a per-element bf16 conversion.
+__device__ __forceinline__ void store_tile_t(uint32_t ta, uint32_t tile, int c0, int t0, uint32_t panel, float sign,
+                                             int lane) {
+  const int piece = lane >> 3, row = lane & 7;  // the row of stmatrix piece `piece` this thread addresses
+#pragma unroll
+  for (int hl = 0; hl < 2; ++hl) {  // channels c0 + 16 hl .. + 15
+    float x[16];
+    ptx::tmem_ld16x256b_x4(ta + ((uint32_t)(16 * hl) << 16), x);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {  // tokens t0 + 16 hf .. + 15: pieces (8 tokens) x (channels +0, +8)
+      const int c = c0 + 16 * hl + 8 * (piece & 1);
+      const int t = t0 + 16 * hf + 8 * (piece >> 1) + row;
+      const uint32_t addr = tile + (uint32_t)(c >> 6) * panel + t * 128 + (((((c & 63) >> 3) ^ t) & 7) << 4);
+      const float* y = x + 8 * hf;
+      ptx::stmatrix_x4_trans(addr, ptx::pack_bf16x2(sign * y[0], sign * y[1]),
+                             ptx::pack_bf16x2(sign * y[2], sign * y[3]), ptx::pack_bf16x2(sign * y[4], sign * y[5]),
+                             ptx::pack_bf16x2(sign * y[6], sign * y[7]));
+    }
+  }
+}
+
 // One 32-column TMEM load into registers (two 16-column loads).
 __device__ __forceinline__ void ld32(uint32_t ta, float* x) {
   ptx::tmem_ld16(ta, *reinterpret_cast<float(*)[16]>(x));
@@ -800,18 +829,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- -W (bf16) over the K e^G rows of the slot, in their layout (K-major:
         //      row = token, key channels 0..63 | 64..127 in the two panels), so that
         //      the state's first MMA reads [-W; Q e^G] as one 128-row operand
-        {
-          const int c = 32 * qd + lane;  // key channel = TMEM lane
-          float x[32];
-          ld32(tmem + ((uint32_t)(32 * qd) << 16) + 64 * s + 32 * ch, x);
-          ptx::tmem_wait_ld();
-          uint8_t* wcol = l3 + (c >> 6) * 16384 + (c & 7) * 2;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int r = 32 * ch + e;  // token
-            *reinterpret_cast<bf16*>(wcol + r * 128 + (((((c & 63) >> 3) ^ r) & 7) << 4)) = __float2bfloat16_rn(-x[e]);
-          }
-        }
+        store_tile_t(tmem + ((uint32_t)(32 * qd) << 16) + 64 * s + 32 * ch, ptx::smem_u32(l3), 32 * qd, 32 * ch,
+                     16384, -1.f, lane);
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         if (ptx::bar_or(2, 256, !ok || *abort_flag)) break;
@@ -965,18 +984,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // swizzled: value channels 0..63 over this slot's P (read by the MMAs
       // above), 64..127 in FU_OST (read by chunk n-1's store)
       uint8_t* opan[2] = {sm + FU_P + s * 8192, sm + FU_OST};
-      uint8_t* ocol = opan[dv >> 6] + (dv & 7) * 2;
 #pragma unroll 1
-      for (int h2 = 0; h2 < 2; ++h2) {
-        float x[32];
-        ld32(tmem + lo_lane + kTmO + 32 * h2, x);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int r = 32 * h2 + e;
-          *reinterpret_cast<bf16*>(ocol + r * 128 + (((((dv & 63) >> 3) ^ r) & 7) << 4)) = __float2bfloat16_rn(x[e]);
-        }
-      }
+      for (int h2 = 0; h2 < 2; ++h2)
+        store_tile_t(tmem + lo_lane + kTmO + 32 * h2, ptx::smem_u32(opan[qd >> 1]), 32 * (qd & 1), 32 * h2, 0, 1.f,
+                     lane);
       zero_cols64(tmem + lo_lane + kTmO);  // the next chunk's first MMA accumulates O onto zeros
       // plain instance, the unit's last chunk: a unit that met near-parallel keys
       // is left to the precise instance (its state is not written, so an S_out

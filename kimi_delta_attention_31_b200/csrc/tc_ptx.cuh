@@ -260,6 +260,34 @@ __device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&v)[8]
       "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
       : "memory");
 }
+// 16 lanes x 32 consecutive 32-bit columns in the m16n8 accumulator layout:
+// for each group j of 8 columns, thread i receives v[4j], v[4j+1] = lane
+// (taddr.lane + i/4), columns 8j + 2(i%4) + {0, 1}, and v[4j+2], v[4j+3] =
+// the same columns of lane (taddr.lane + 8 + i/4).  taddr.lane is the first
+// or the middle lane of the warp's quarter.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// Four 8 x 8 bf16 tiles stored transposed: word j of thread i holds tile j's
+// elements (row i/4, columns 2(i%4) and 2(i%4)+1, the first in the low half);
+// column r of tile j (8 elements, 16 bytes) goes to the shared address that
+// thread 8j + r passes (16-byte aligned).
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t w0, uint32_t w1, uint32_t w2,
+                                                  uint32_t w3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(w0),
+               "r"(w1), "r"(w2), "r"(w3)
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
