@@ -25,17 +25,32 @@ def recurrent_grad(q, k, v, g, beta, S0, do, dS_T=None):
     the final state) [B,H,dk,dv] or None.  Returns a dict of float64 numpy
     arrays dq, dk, dv, dg, dbeta, dS0 (dS0 is None when S0 is None) and the
     forward o, S_T."""
+    return _grad(q, k, v, g, beta, S0, do, dS_T, scalar_gate=False)
+
+
+def gdn_recurrent_grad(q, k, v, g, beta, S0, do, dS_T=None):
+    """Gated DeltaNet: one decay per token and head ("Kimi K3 notes 1: KDA"
+    section 3; "Linear / sparse attention" tutorial section 5.2), g [B,T,H],
+    so the loop decays the whole state by the scalar e^{g_t}:
+        S~ = e^{g_t} S;  then the same delta-rule write and read.
+    Arguments and result as recurrent_grad, with dg [B,T,H]."""
+    return _grad(q, k, v, g, beta, S0, do, dS_T, scalar_gate=True)
+
+
+def _grad(q, k, v, g, beta, S0, do, dS_T, scalar_gate):
     t64 = lambda x: torch.as_tensor(np.asarray(x if not hasattr(x, "detach") else x.detach().cpu(),
                                                dtype=np.float64)).clone()
     q, k, v, g, beta = (t64(x).requires_grad_(True) for x in (q, k, v, g, beta))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    if g.shape != ((B, T, H) if scalar_gate else (B, T, H, dk)):
+        raise ValueError("g must be [B,T,H] for a scalar gate and [B,T,H,dk] otherwise")
     S = (t64(S0) if S0 is not None else torch.zeros(B, H, dk, dv, dtype=torch.float64)).requires_grad_(S0 is not None)
     S_init = S
     outs = []
     for t in range(T):
-        a = torch.exp(g[:, t])                                # [B,H,dk]
-        St = a.unsqueeze(-1) * S                              # S~
+        a = torch.exp(g[:, t])                                # [B,H] or [B,H,dk]
+        St = (a[..., None, None] if scalar_gate else a.unsqueeze(-1)) * S  # S~
         vh = torch.einsum("bhcj,bhc->bhj", St, k[:, t])
         e = beta[:, t].unsqueeze(-1) * (v[:, t] - vh)
         S = St + k[:, t].unsqueeze(-1) * e.unsqueeze(-2)

@@ -1,11 +1,12 @@
-"""Pins of the gradient oracle (oracle.grad.recurrent_grad): central finite
-differences of the fp64 recurrence itself, a closed form for the gradient of
-a single step, and consistency of the forward it differentiates with the
-pinned recurrence."""
+"""Pins of the gradient oracle (oracle.grad.recurrent_grad and
+gdn_recurrent_grad): central finite differences of the fp64 recurrences
+themselves, a closed form for the gradient of a single step, consistency of
+the forwards they differentiate with the pinned recurrences, and the chain
+rule that ties the Gated DeltaNet gate's gradient to the per-channel one."""
 import numpy as np
 
 import oracle
-from oracle.grad import recurrent_grad
+from oracle.grad import gdn_recurrent_grad, recurrent_grad
 
 
 def _inputs(rng, B, T, H, dk, dv):
@@ -68,3 +69,57 @@ def test_single_step_closed_form():
     D = np.exp(g[0, 0, 0])
     ref = D[:, None] * (np.outer(q[0, 0, 0], do[0, 0, 0]) - b * kq * np.outer(k[0, 0, 0], do[0, 0, 0]))
     np.testing.assert_allclose(r["dS0"][0, 0], ref, rtol=1e-12, atol=1e-14)
+
+
+def _gdn_inputs(rng, B, T, H, dk, dv):
+    q, k, v, g, beta, S0, do, dS = _inputs(rng, B, T, H, dk, dv)
+    return q, k, v, g[..., 0].copy(), beta, S0, do, dS  # one gate per token and head
+
+
+def _gdn_loss(q, k, v, g, beta, S0, do, dS):
+    o, S = oracle.gdn_recurrent(q, k, v, g, beta, S0)
+    return float((o * do).sum() + (S * dS).sum())
+
+
+def test_gdn_forward_matches_the_pinned_gdn_recurrence():
+    rng = np.random.default_rng(93)
+    q, k, v, g, beta, S0, do, dS = _gdn_inputs(rng, 2, 9, 2, 5, 4)
+    r = gdn_recurrent_grad(q, k, v, g, beta, S0, do, dS)
+    o, S = oracle.gdn_recurrent(q, k, v, g, beta, S0)
+    np.testing.assert_allclose(r["o"], o, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(r["S_T"], S, rtol=1e-12, atol=1e-13)
+
+
+def test_gdn_gradients_match_central_differences():
+    """Finite differences of the pinned Gated DeltaNet forward (oracle.gdn_recurrent)."""
+    rng = np.random.default_rng(94)
+    args = list(_gdn_inputs(rng, 1, 6, 2, 4, 3))
+    r = gdn_recurrent_grad(*args)
+    h = 1e-6
+    for i, n in enumerate(["q", "k", "v", "g", "beta", "S0"]):
+        x = args[i]
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = x[idx]
+            x[idx] = old + h
+            lp = _gdn_loss(*args)
+            x[idx] = old - h
+            lm = _gdn_loss(*args)
+            x[idx] = old
+            fd = (lp - lm) / (2 * h)
+            assert abs(r["d" + n][idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (n, idx, r["d" + n][idx], fd)
+
+
+def test_gdn_gate_gradient_is_the_sum_over_channels():
+    """Every key channel decays by the one g_t, so by the chain rule dL/dg_t is
+    the per-channel gradient (of the same inputs with g repeated over dk)
+    summed over the channels; the other gradients are the per-channel ones."""
+    rng = np.random.default_rng(95)
+    q, k, v, g, beta, S0, do, dS = _gdn_inputs(rng, 2, 7, 3, 5, 4)
+    r = gdn_recurrent_grad(q, k, v, g, beta, S0, do, dS)
+    g_full = np.repeat(g[..., None], q.shape[-1], axis=-1)
+    rk = recurrent_grad(q, k, v, g_full, beta, S0, do, dS)
+    np.testing.assert_allclose(r["dg"], rk["dg"].sum(-1), rtol=1e-11, atol=1e-12)
+    for n in ("dq", "dk", "dv", "dbeta", "dS0"):
+        np.testing.assert_allclose(r[n], rk[n], rtol=1e-11, atol=1e-12)
