@@ -208,6 +208,22 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Backward pass of the Gated DeltaNet prefill (kda_gdn_chunk_fwd: one decay
+ * alpha_t = e^{g_t} per token and head, "Kimi K3 notes 1: KDA" section 3;
+ * "Linear / sparse attention" tutorial section 5.2).  Arguments, workspace
+ * (kda_chunk_bwd_workspace_size), alignment, aliasing rules and errors as
+ * kda_chunk_bwd except
+ *   g  : [B, T, H] fp32 log alpha, one per token and head;
+ *   dg : [B, T, H] fp32, written: dL/dg_t, which is the sum over the key
+ *        channels of the per-channel gradient (every channel decays by g_t).
+ */
+kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                               const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
+                               float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens,
+                               int num_seqs, int B, int T, int H, int dk_, int dv_, kda_dtype_t dtype,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * kda_chunk_fwd from HOST buffers (library plumbing around the prefill of
  * "Deriving Kimi Delta Attention from scratch" section 6, chunked mode; the
  * pages have no host interface).  q, k, v, g, beta, S0 (or NULL), cu_seqlens

@@ -40,7 +40,7 @@ EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step
             "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait",
             "kda_set_segment_chunks", "kda_segment_chunks", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
             "kda_set_local_kernel", "kda_chunk_fwd_host", "kda_chunk_fwd_host_buffer_size",
-            "kda_set_prefill_path", "kda_chunk_fwd_phases")
+            "kda_set_prefill_path", "kda_chunk_fwd_phases", "kda_gdn_chunk_bwd")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -109,6 +109,8 @@ def load_library():
         lib.kda_chunk_bwd_workspace_size.restype = szt
         lib.kda_chunk_bwd.argtypes = [vp] * 15 + [i32] * 6 + [i32, vp, szt, vp]
         lib.kda_chunk_bwd.restype = i32
+        lib.kda_gdn_chunk_bwd.argtypes = lib.kda_chunk_bwd.argtypes
+        lib.kda_gdn_chunk_bwd.restype = i32
         lib.kda_set_segment_chunks.argtypes = [i32]
         lib.kda_set_segment_chunks.restype = i32
         lib.kda_segment_chunks.argtypes = [i32] * 4
@@ -301,29 +303,42 @@ def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, cu_seqlens=None, works
     v, g, beta (and S0) given dout = dL/do and dS_T = dL/dS_final (or None).
     Returns a dict of fp32 tensors dq, dk, dv, dg [B,T,H,d], dbeta [B,T,H] and
     dS0 [N,H,dk,dv] (None when need_dS0 is False)."""
+    return _chunk_bwd("kda_chunk_bwd", q, k, v, g, beta, dout, S0, dS_T, cu_seqlens, workspace, need_dS0)
+
+
+def gdn_chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, cu_seqlens=None, workspace=None,
+                  need_dS0=True):
+    """Backward pass of gdn_chunk_fwd (one gate per token and head): as
+    chunk_bwd with g [B,T,H] fp32, and dg [B,T,H]."""
+    return _chunk_bwd("kda_gdn_chunk_bwd", q, k, v, g, beta, dout, S0, dS_T, cu_seqlens, workspace, need_dS0)
+
+
+def _chunk_bwd(fn, q, k, v, g, beta, dout, S0, dS_T, cu_seqlens, workspace, need_dS0):
     lib = load_library()
-    _need_cuda(q, k, v, g, beta, dout, S0, dS_T, cu_seqlens, workspace)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     N = num_seqs if cu_seqlens is not None else B
     if g.dtype != torch.float32 or beta.dtype != torch.float32 or dout.dtype != q.dtype:
         raise TypeError("g and beta must be float32 and dout must have q's dtype")
-    if tuple(g.shape) != (B, T, H, dk) or tuple(beta.shape) != (B, T, H) or tuple(dout.shape) != (B, T, H, dv):
-        raise ValueError("g must be [B,T,H,dk], beta [B,T,H], dout [B,T,H,dv]")
+    g_shape = (B, T, H) if fn == "kda_gdn_chunk_bwd" else (B, T, H, dk)
+    if tuple(g.shape) != g_shape or tuple(beta.shape) != (B, T, H) or tuple(dout.shape) != (B, T, H, dv):
+        raise ValueError(f"g must be {list(g_shape)}, beta [B,T,H], dout [B,T,H,dv]")
+    _need_cuda(q, k, v, g, beta, dout, S0, dS_T, cu_seqlens, workspace)
     f32 = dict(dtype=torch.float32, device=q.device)
-    out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
-               dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty((B, T, H, dk), **f32),
-               dbeta=torch.empty((B, T, H), **f32),
-               dS0=torch.empty((N, H, dk, dv), **f32) if need_dS0 else None)
-    need = int(lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, num_seqs))
-    if workspace is None and need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(dout), _ptr(dS_T),
-                           _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
-                           _ptr(out["dS0"]), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, _dtype_code(q),
-                           _ptr(workspace), ws_bytes, _stream_handle(q.device))
+    with torch.cuda.device(q.device):
+        out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+                   dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty(g_shape, **f32),
+                   dbeta=torch.empty((B, T, H), **f32),
+                   dS0=torch.empty((N, H, dk, dv), **f32) if need_dS0 else None)
+        need = int(lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, num_seqs))
+        if workspace is None and need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(dout), _ptr(dS_T),
+                              _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                              _ptr(out["dbeta"]), _ptr(out["dS0"]), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv,
+                              _dtype_code(q), _ptr(workspace), ws_bytes, _stream_handle(q.device))
     _check(st)
     return out
 

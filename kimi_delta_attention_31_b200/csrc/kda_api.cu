@@ -219,12 +219,14 @@ size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num
   return kda::bwd::bwd_workspace_bytes(B, T, H, dk, num_seqs);
 }
 
-kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                           const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
-                           float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens,
-                           int num_seqs, int B, int T, int H, int dkh, int dvh, kda_dtype_t dtype,
-                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  const char* fn = "kda_chunk_bwd";
+// The backward of both gate layouts: gate = kGateLogCh (g, dg [.., H, dk]) or
+// kGateLogTok (g, dg [.., H]).
+static kda_status_t chunk_bwd_impl(const char* fn, int gate, const void* q, const void* k, const void* v,
+                                   const float* g, const float* beta, const float* S0, const void* dout,
+                                   const float* dS_T, float* dq, float* dk, float* dv, float* dg, float* dbeta,
+                                   float* dS0, const int32_t* cu_seqlens, int num_seqs, int B, int T, int H,
+                                   int dkh, int dvh, kda_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
   t_err[0] = 0;
   if (B < 0 || T < 0 || H <= 0 || num_seqs < 0)
     return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes B=%d T=%d H=%d num_seqs=%d", fn, B, T, H, num_seqs);
@@ -265,9 +267,14 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
     return fail(KDA_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes, need);
   float* ck = static_cast<float*>(workspace);
   cudaError_t e = cudaErrorInvalidValue;
-#define KDA_BWD_CASE(TT, DD)                                                                          \
-  e = kda::bwd::launch_chunk_bwd<TT, DD>(q, k, v, g, beta, S0, dout, dS_T, dq, dk, dv, dg, dbeta, dS0, \
-                                         cu_seqlens, N, T, H, ck, stream)
+#define KDA_BWD_CASE(TT, DD)                                                                            \
+  e = gate == kda::kGateLogTok                                                                           \
+          ? kda::bwd::launch_chunk_bwd<TT, DD, kda::kGateLogTok>(q, k, v, g, beta, S0, dout, dS_T, dq, dk, \
+                                                                 dv, dg, dbeta, dS0, cu_seqlens, N, T, H,  \
+                                                                 ck, stream)                               \
+          : kda::bwd::launch_chunk_bwd<TT, DD, kda::kGateLogCh>(q, k, v, g, beta, S0, dout, dS_T, dq, dk,  \
+                                                                dv, dg, dbeta, dS0, cu_seqlens, N, T, H,   \
+                                                                ck, stream)
   if (dtype == KDA_F32) {
     if (dkh == 32) KDA_BWD_CASE(float, 32); else if (dkh == 64) KDA_BWD_CASE(float, 64); else KDA_BWD_CASE(float, 128);
   } else {
@@ -278,6 +285,26 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
 #undef KDA_BWD_CASE
   if (e != cudaSuccess) return cuda_fail(e, fn);
   return KDA_OK;
+}
+
+kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
+                           float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens,
+                           int num_seqs, int B, int T, int H, int dkh, int dvh, kda_dtype_t dtype,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return chunk_bwd_impl("kda_chunk_bwd", kda::kGateLogCh, q, k, v, g, beta, S0, dout, dS_T, dq, dk, dv, dg,
+                        dbeta, dS0, cu_seqlens, num_seqs, B, T, H, dkh, dvh, dtype, workspace, workspace_bytes,
+                        stream);
+}
+
+kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                               const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
+                               float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens,
+                               int num_seqs, int B, int T, int H, int dkh, int dvh, kda_dtype_t dtype,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return chunk_bwd_impl("kda_gdn_chunk_bwd", kda::kGateLogTok, q, k, v, g, beta, S0, dout, dS_T, dq, dk, dv, dg,
+                        dbeta, dS0, cu_seqlens, num_seqs, B, T, H, dkh, dvh, dtype, workspace, workspace_bytes,
+                        stream);
 }
 
 kda_status_t kda_set_segment_chunks(int chunks) {

@@ -1,6 +1,8 @@
 // kda_chunk_bwd.cuh -- backward pass of the chunkwise KDA prefill: gradients
 // with respect to q, k, v, g = log alpha, beta and the initial state, in fp32
-// arithmetic on the CUDA cores.
+// arithmetic on the CUDA cores.  kGate selects the gate: one per key channel
+// (KDA) or one per token and head (Gated DeltaNet, whose dg is the sum over
+// channels of the per-channel dg).
 //
 // The pages give the forward only ("Deriving Kimi Delta Attention from
 // scratch", section 6, chunked mode; "Linear / sparse attention" tutorial,
@@ -75,7 +77,7 @@ __device__ __forceinline__ long long ckpt_slot(bool packed, int n, long long t0,
   return packed ? (t0 / C + ch + n) : ((long long)n * nch_T + ch);
 }
 
-template <typename TIn, int D>
+template <typename TIn, int D, int kGate>
 __global__ void __launch_bounds__(4 * D)
     kda_chunk_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                          const float* __restrict__ g, const float* __restrict__ beta,
@@ -115,7 +117,8 @@ __global__ void __launch_bounds__(4 * D)
 
   const int uh = blockIdx.x;  // n * H + h
   const int h = uh % H, n = uh / H;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  static_assert(kGate == kGateLogCh || kGate == kGateLogTok, "log-decay gates only");
   const bool packed = cu_seqlens != nullptr;
   long long t0 = (long long)n * T, t1 = t0 + T;
   if (packed) checked_seq_range(cu_seqlens, n, T, &t0, &t1);  // T = total tokens when packed
@@ -137,7 +140,7 @@ __global__ void __launch_bounds__(4 * D)
         const size_t off = row_off(s + r) + c;
         qv = to_f32(q[off]);
         kv = to_f32(k[off]);
-        gv = g[off];
+        gv = kGate == kGateLogTok ? g[(size_t)(s + r) * H + h] : g[off];
         if (with_dout) ov = to_f32(dout[off]);
       }
       Qs[idx] = qv;
@@ -416,7 +419,28 @@ __global__ void __launch_bounds__(4 * D)
 #pragma unroll
       for (int i = 0; i < C / 4; ++i) dEs[(part + 4 * i) * D + c] = dGa[i];
       __syncthreads();
-      if (part == 0) {  // dg_i = sum_{r >= i} dG_r
+      if constexpr (kGate == kGateLogTok) {
+        // one gate per token and head (Gated DeltaNet: every key channel decays
+        // by the same g_t), so dL/dg_t is the sum over channels of the
+        // per-channel gradient: the row sums of dG, then the same reverse
+        // cumulative sum (the two sums commute)
+        float* rsum = Mt;  // C floats (Mt is no longer read in this chunk)
+        for (int r = warp; r < C; r += NT / 32) {
+          float acc = 0.f;
+          for (int cc = lane; cc < D; cc += 32) acc += dEs[r * D + cc];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (lane == 0) rsum[r] = acc;
+        }
+        __syncthreads();
+        if (tid == 0) {
+          float acc = 0.f;
+          for (int r = C - 1; r >= 0; --r) {
+            acc += rsum[r];
+            if (r < Cn) dg[(size_t)(s + r) * H + h] = acc;
+          }
+        }
+      } else if (part == 0) {  // dg_i = sum_{r >= i} dG_r
         float acc = 0.f;
         for (int r = C - 1; r >= 0; --r) {
           acc += dEs[r * D + c];
@@ -431,20 +455,20 @@ __global__ void __launch_bounds__(4 * D)
     for (int idx = tid; idx < D * D; idx += NT) dS0[(size_t)uh * D * D + idx] = dSs[idx];
 }
 
-template <typename TIn, int D>
+template <typename TIn, int D, int kGate>
 cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                              const float* S0, const void* dout, const float* dS_T, float* dq, float* dk,
                              float* dv, float* dg, float* dbeta, float* dS0, const int32_t* cu_seqlens, int N,
                              int T, int H, float* ckpt, cudaStream_t stream) {
   static PerDeviceOnce s_attrs;
   cudaError_t e = run_once_per_device(s_attrs, [] {
-    return cudaFuncSetAttribute(kda_chunk_bwd_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(kda_chunk_bwd_kernel<TIn, D, kGate>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)Cfg<D>::smem_bytes);
   });
   if (e != cudaSuccess) return e;
   const long long units = (long long)N * H;
   if (units == 0) return cudaSuccess;
-  kda_chunk_bwd_kernel<TIn, D><<<(unsigned)units, Cfg<D>::NT, Cfg<D>::smem_bytes, stream>>>(
+  kda_chunk_bwd_kernel<TIn, D, kGate><<<(unsigned)units, Cfg<D>::NT, Cfg<D>::smem_bytes, stream>>>(
       static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), g, beta, S0,
       static_cast<const TIn*>(dout), dS_T, dq, dk, dv, dg, dbeta, dS0, cu_seqlens, T, H, ckpt);
   return cudaGetLastError();

@@ -242,6 +242,24 @@ def test_noalloc_binding_checks_arguments_before_any_launch():
             fn(q, q, q, g, beta)                               # right shapes, host tensors
 
 
+def test_backward_bindings_check_the_gate_layout_before_any_launch():
+    """chunk_bwd takes one gate per key channel and gdn_chunk_bwd one per token
+    and head; the C ABI sees only pointers, so the bindings refuse the other
+    layout (and a non-fp32 gate) before any CUDA call."""
+    import torch
+    B, T, H, d = 1, 8, 2, 32
+    q = torch.zeros(B, T, H, d, dtype=torch.bfloat16)
+    beta = torch.zeros(B, T, H)
+    g_ch, g_tok = torch.zeros(B, T, H, d), torch.zeros(B, T, H)
+    for fn, good, other in ((kda.chunk_bwd, g_ch, g_tok), (kda.gdn_chunk_bwd, g_tok, g_ch)):
+        with pytest.raises(TypeError):
+            fn(q, q, q, good.to(torch.bfloat16), beta, q)      # bf16 gate
+        with pytest.raises(ValueError):
+            fn(q, q, q, other, beta, q)                        # the other gate layout
+        with pytest.raises(ValueError):
+            fn(q, q, q, good, beta, q)                         # right shapes, host tensors
+
+
 def test_host_entry_point_sizes_and_argument_checks():
     """kda_chunk_fwd_host: its device buffer holds a copy of every tensor plus
     the workspace, and bad arguments are refused before any copy is queued."""

@@ -1,5 +1,6 @@
-"""GPU parity of the backward pass (kda_chunk_bwd) against the gradient
-oracle (reverse-mode differentiation of the fp64 token recurrence).  The
+"""GPU parity of the backward pass (kda_chunk_bwd, and kda_gdn_chunk_bwd for
+one gate per token and head) against the gradient oracle (reverse-mode
+differentiation of the fp64 token recurrence).  The
 kernel computes in fp32 from the same (bf16- or fp32-rounded) inputs the
 oracle widens, so both dtypes are held to 1e-4 relative RMS per (sequence,
 head) slice of every gradient."""
@@ -9,7 +10,7 @@ import torch
 
 import kimi_delta_attention_31_b200 as kda
 import kda_workloads as W
-from oracle.grad import recurrent_grad
+from oracle.grad import gdn_recurrent_grad, recurrent_grad
 from parity_util import rel_rms
 
 pytestmark = pytest.mark.gpu
@@ -17,8 +18,9 @@ pytestmark = pytest.mark.gpu
 TOL = 1e-4
 
 
-def _inputs(dev, B, T, H, d, dtype, seed, lengths=None, s0=True):
-    inp = W.make_prefill(B, T, H, d, d, dtype, -3.0, 1.0, 0.05 if s0 else 0.0, seed=seed, device=dev, lengths=lengths)
+def _inputs(dev, B, T, H, d, dtype, seed, lengths=None, s0=True, scalar_gate=False):
+    inp = W.make_prefill(B, T, H, d, d, dtype, -3.0, 1.0, 0.05 if s0 else 0.0, seed=seed, device=dev, lengths=lengths,
+                         scalar_gate=scalar_gate)
     gen = torch.Generator(device=dev).manual_seed(seed + 1)
     tdt = inp["q"].dtype
     inp["do"] = torch.randn(inp["v"].shape, generator=gen, device=dev).to(tdt)
@@ -35,13 +37,13 @@ def _check_slices(got, ref, what, tol=TOL):
     return err
 
 
-def _compare(inp, out, with_s0=True):
+def _compare(inp, out, with_s0=True, grad=recurrent_grad):
     cpu = {n: (t.double().cpu().numpy() if t is not None else None) for n, t in inp.items() if n != "cu_seqlens"}
     B, T, H, d = cpu["q"].shape
     for b in range(B):
         for h in range(H):
             sl = lambda x: x[b:b + 1, :, h:h + 1]
-            ref = recurrent_grad(sl(cpu["q"]), sl(cpu["k"]), sl(cpu["v"]), sl(cpu["g"]), sl(cpu["beta"]),
+            ref = grad(sl(cpu["q"]), sl(cpu["k"]), sl(cpu["v"]), sl(cpu["g"]), sl(cpu["beta"]),
                                  cpu["S0"][b:b + 1, h:h + 1] if with_s0 else None, sl(cpu["do"]),
                                  cpu["dS_T"][b:b + 1, h:h + 1])
             for n in ("dq", "dk", "dv", "dg", "dbeta"):
@@ -98,3 +100,55 @@ def test_bwd_longer_sequence_strong_decay(cuda_device):
     out = kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["do"], inp["S0"], inp["dS_T"])
     torch.cuda.synchronize()
     _compare(inp, out)
+
+
+# ---- Gated DeltaNet (one gate per token and head)
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 128])
+@pytest.mark.parametrize("T", [17, 40])
+def test_gdn_bwd_small_shapes(cuda_device, dtype, d, T):
+    inp = _inputs(cuda_device, 2, T, 2, d, dtype, seed=700 + T + d, scalar_gate=True)
+    out = kda.gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["do"], inp["S0"], inp["dS_T"])
+    torch.cuda.synchronize()
+    assert kda.device_error() == 0
+    assert tuple(out["dg"].shape) == tuple(inp["g"].shape)
+    _compare(inp, out, grad=gdn_recurrent_grad)
+
+
+def test_gdn_bwd_packed_varlen(cuda_device):
+    lens = (5, 0, 33, 16)
+    inp = _inputs(cuda_device, 1, sum(lens), 2, 64, "f32", seed=72, lengths=lens, scalar_gate=True)
+    out = kda.gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["do"], inp["S0"],
+                            inp["dS_T"], cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    cu = np.cumsum((0,) + lens)
+    cpu = {n: t.double().cpu().numpy() for n, t in inp.items() if n not in ("cu_seqlens",)}
+    for s_i in range(len(lens)):
+        a, b = cu[s_i], cu[s_i + 1]
+        for h in range(2):
+            if b == a:  # empty sequence: the state gradient passes through
+                assert torch.allclose(out["dS0"][s_i, h], inp["dS_T"][s_i, h])
+                continue
+            sl = lambda x: x[:, a:b, h:h + 1]
+            ref = gdn_recurrent_grad(sl(cpu["q"]), sl(cpu["k"]), sl(cpu["v"]), sl(cpu["g"]), sl(cpu["beta"]),
+                                     cpu["S0"][s_i:s_i + 1, h:h + 1], sl(cpu["do"]), cpu["dS_T"][s_i:s_i + 1, h:h + 1])
+            for n in ("dq", "dk", "dv", "dg", "dbeta"):
+                _check_slices(out[n][:, a:b, h:h + 1].double().cpu().numpy(), ref[n], f"{n} seq{s_i} h{h}")
+            _check_slices(out["dS0"][s_i:s_i + 1, h:h + 1].double().cpu().numpy(), ref["dS0"], f"dS0 seq{s_i}")
+
+
+def test_gdn_bwd_equals_the_per_channel_bwd_on_the_repeated_gate(cuda_device):
+    """The scalar-gate backward reads the one gate where the per-channel one
+    reads its copies and does the same arithmetic, so every gradient but dg
+    agrees to fp32 rounding; dg is the per-channel dg summed over channels
+    (up to fp32 summation order)."""
+    inp = _inputs(cuda_device, 2, 70, 3, 64, "bf16", seed=73, scalar_gate=True)
+    g_full = inp["g"][..., None].expand(*inp["g"].shape, 64).contiguous()
+    out = kda.gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["do"], inp["S0"], inp["dS_T"])
+    ref = kda.chunk_bwd(inp["q"], inp["k"], inp["v"], g_full, inp["beta"], inp["do"], inp["S0"], inp["dS_T"])
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "dbeta", "dS0"):
+        assert rel_rms(out[n].double().cpu().numpy(), ref[n].double().cpu().numpy()) <= 1e-6, n
+    err = rel_rms(out["dg"].double().cpu().numpy(), ref["dg"].sum(-1).double().cpu().numpy())
+    assert err <= 1e-6, err
