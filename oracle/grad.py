@@ -37,7 +37,17 @@ def gdn_recurrent_grad(q, k, v, g, beta, S0, do, dS_T=None):
     return _grad(q, k, v, g, beta, S0, do, dS_T, scalar_gate=True)
 
 
-def _grad(q, k, v, g, beta, S0, do, dS_T, scalar_gate):
+def recurrent_prep_grad(q, k, v, a, b, S0, do, dS_T=None):
+    """The recurrence fed by the input preparation of oracle.prep (q, k
+    L2-normalised with the norm clamped at 1e-12, log alpha = -softplus(a),
+    beta = sigmoid(b); "Kimi K3 notes 1: KDA" section 4, "Linear / sparse
+    attention" tutorial section 10), differentiated with respect to the RAW
+    q, k, a [B,T,H,dk] and b [B,T,H].  Returns the dict of recurrent_grad with
+    dq, dk, da, db (gradients of the raw inputs) in place of dq, dk, dg, dbeta."""
+    return _grad(q, k, v, a, b, S0, do, dS_T, scalar_gate=False, prep=True)
+
+
+def _grad(q, k, v, g, beta, S0, do, dS_T, scalar_gate, prep=False):
     t64 = lambda x: torch.as_tensor(np.asarray(x if not hasattr(x, "detach") else x.detach().cpu(),
                                                dtype=np.float64)).clone()
     q, k, v, g, beta = (t64(x).requires_grad_(True) for x in (q, k, v, g, beta))
@@ -47,6 +57,12 @@ def _grad(q, k, v, g, beta, S0, do, dS_T, scalar_gate):
         raise ValueError("g must be [B,T,H] for a scalar gate and [B,T,H,dk] otherwise")
     S = (t64(S0) if S0 is not None else torch.zeros(B, H, dk, dv, dtype=torch.float64)).requires_grad_(S0 is not None)
     S_init = S
+    qr, kr, ar, br = q, k, g, beta  # the leaves
+    if prep:  # raw projections: the preparation first, in the leaves' graph
+        q = q / q.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+        k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+        g = -torch.logaddexp(torch.zeros_like(g), g)
+        beta = torch.sigmoid(beta)
     outs = []
     for t in range(T):
         a = torch.exp(g[:, t])                                # [B,H] or [B,H,dk]
@@ -59,9 +75,10 @@ def _grad(q, k, v, g, beta, S0, do, dS_T, scalar_gate):
     loss = (o * t64(do)).sum()
     if dS_T is not None:
         loss = loss + (S * t64(dS_T)).sum()
-    leaves = [q, k, v, g, beta] + ([S_init] if S0 is not None else [])
+    leaves = [qr, kr, v, ar, br] + ([S_init] if S0 is not None else [])
     grads = torch.autograd.grad(loss, leaves)
-    res = {n: x.numpy() for n, x in zip(("dq", "dk", "dv", "dg", "dbeta"), grads[:5])}
+    names = ("dq", "dk", "dv", "da", "db") if prep else ("dq", "dk", "dv", "dg", "dbeta")
+    res = {n: x.numpy() for n, x in zip(names, grads[:5])}
     res["dS0"] = grads[5].numpy() if S0 is not None else None
     res["o"] = o.detach().numpy()
     res["S_T"] = S.detach().numpy()
