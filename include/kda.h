@@ -224,6 +224,35 @@ kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v, cons
                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Backward pass of the prefill from raw projections (kda_chunk_fwd_prep: q, k
+ * L2-normalised per token and head, log alpha = -softplus(a), beta =
+ * sigmoid(b); "Kimi K3 notes 1: KDA" section 4 and the "Linear / sparse
+ * attention" tutorial section 10 for the preparation).  The gradients are
+ * those of kda_chunk_bwd, taken on the prepared inputs in fp32, composed
+ * with the preparation's Jacobians:
+ *   dq = (dq^ - q^ (q^ . dq^)) / |q|  (dq^ / 1e-12 where |q| < 1e-12), dk alike,
+ *   da = -sigmoid(a) dg,  db = beta (1 - beta) dbeta.
+ * Arguments as kda_chunk_bwd except
+ *   q, k           : the raw (unnormalised) projections, dtype;
+ *   a, a_dtype     : raw gate logits [B, T, H, dk], KDA_F32 or KDA_BF16, element-aligned;
+ *   b              : raw beta logits [B, T, H] fp32;
+ *   dq, dk         : [B, T, H, dk] fp32, written: gradients of the RAW q, k;
+ *   da             : [B, T, H, dk] fp32, written: gradient of a;
+ *   db             : [B, T, H] fp32, written: gradient of b;
+ *   workspace      : at least kda_chunk_bwd_prep_workspace_size(...) bytes: the
+ *                    checkpoints of kda_chunk_bwd, then fp32 copies of the
+ *                    prepared q, k, of v, dO and of the gates (20 B per
+ *                    token, head and channel, and 12 B per token-head row, more).
+ * Three launches: the preparation, the backward kernel, the chain rule.
+ */
+size_t kda_chunk_bwd_prep_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs);
+kda_status_t kda_chunk_bwd_prep(const void* q, const void* k, const void* v, const void* a, kda_dtype_t a_dtype,
+                                const float* b, const float* S0, const void* dout, const float* dS_T, float* dq,
+                                float* dk, float* dv, float* da, float* db, float* dS0, const int32_t* cu_seqlens,
+                                int num_seqs, int B, int T, int H, int dk_, int dv_, kda_dtype_t dtype,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * kda_chunk_fwd from HOST buffers (library plumbing around the prefill of
  * "Deriving Kimi Delta Attention from scratch" section 6, chunked mode; the
  * pages have no host interface).  q, k, v, g, beta, S0 (or NULL), cu_seqlens

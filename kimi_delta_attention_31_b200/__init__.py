@@ -40,7 +40,8 @@ EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step
             "kda_chunk_fwd_prep", "kda_recurrent_step_prep", "kda_selftest_bounded_wait",
             "kda_set_segment_chunks", "kda_segment_chunks", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
             "kda_set_local_kernel", "kda_chunk_fwd_host", "kda_chunk_fwd_host_buffer_size",
-            "kda_set_prefill_path", "kda_chunk_fwd_phases", "kda_gdn_chunk_bwd")
+            "kda_set_prefill_path", "kda_chunk_fwd_phases", "kda_gdn_chunk_bwd", "kda_chunk_bwd_prep",
+            "kda_chunk_bwd_prep_workspace_size")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # Kernels of one kda_chunk_fwd call, in launch order, per path.
@@ -111,6 +112,10 @@ def load_library():
         lib.kda_chunk_bwd.restype = i32
         lib.kda_gdn_chunk_bwd.argtypes = lib.kda_chunk_bwd.argtypes
         lib.kda_gdn_chunk_bwd.restype = i32
+        lib.kda_chunk_bwd_prep_workspace_size.argtypes = [i32] * 6
+        lib.kda_chunk_bwd_prep_workspace_size.restype = szt
+        lib.kda_chunk_bwd_prep.argtypes = [vp] * 4 + [i32] + [vp] * 11 + [i32] * 6 + [i32, vp, szt, vp]
+        lib.kda_chunk_bwd_prep.restype = i32
         lib.kda_set_segment_chunks.argtypes = [i32]
         lib.kda_set_segment_chunks.restype = i32
         lib.kda_segment_chunks.argtypes = [i32] * 4
@@ -311,6 +316,41 @@ def gdn_chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, cu_seqlens=None, w
     """Backward pass of gdn_chunk_fwd (one gate per token and head): as
     chunk_bwd with g [B,T,H] fp32, and dg [B,T,H]."""
     return _chunk_bwd("kda_gdn_chunk_bwd", q, k, v, g, beta, dout, S0, dS_T, cu_seqlens, workspace, need_dS0)
+
+
+def chunk_bwd_prep(q, k, v, a, b, dout, S0=None, dS_T=None, cu_seqlens=None, workspace=None, need_dS0=True):
+    """Backward pass of chunk_fwd_prep (raw projections): gradients of a loss L
+    with respect to the RAW q, k [B,T,H,dk], v, the gate logits a [B,T,H,dk]
+    (bf16 or fp32) and the beta logits b [B,T,H] fp32 (and S0), given dout =
+    dL/do and dS_T = dL/dS_final (or None).  Returns a dict of fp32 tensors dq,
+    dk, dv, da, db and dS0 (None when need_dS0 is False)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = num_seqs if cu_seqlens is not None else B
+    if a.dtype not in (torch.float32, torch.bfloat16) or b.dtype != torch.float32 or dout.dtype != q.dtype:
+        raise TypeError("a must be float32 or bfloat16, b float32, and dout must have q's dtype")
+    if tuple(a.shape) != (B, T, H, dk) or tuple(b.shape) != (B, T, H) or tuple(dout.shape) != (B, T, H, dv):
+        raise ValueError("a must be [B,T,H,dk], b [B,T,H], dout [B,T,H,dv]")
+    _need_cuda(q, k, v, a, b, dout, S0, dS_T, cu_seqlens, workspace)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+                   dv=torch.empty((B, T, H, dv), **f32), da=torch.empty((B, T, H, dk), **f32),
+                   db=torch.empty((B, T, H), **f32),
+                   dS0=torch.empty((N, H, dk, dv), **f32) if need_dS0 else None)
+        need = int(lib.kda_chunk_bwd_prep_workspace_size(B, T, H, dk, dv, num_seqs))
+        if workspace is None and need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib.kda_chunk_bwd_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _dtype_code(a), _ptr(b), _ptr(S0),
+                                    _ptr(dout), _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                    _ptr(out["da"]), _ptr(out["db"]), _ptr(out["dS0"]), _ptr(cu_seqlens), num_seqs,
+                                    B, T, H, dk, dv, _dtype_code(q), _ptr(workspace), ws_bytes,
+                                    _stream_handle(q.device))
+    _check(st)
+    return out
 
 
 def _chunk_bwd(fn, q, k, v, g, beta, dout, S0, dS_T, cu_seqlens, workspace, need_dS0):

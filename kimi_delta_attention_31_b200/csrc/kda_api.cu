@@ -307,6 +307,78 @@ kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v, cons
                         stream);
 }
 
+size_t kda_chunk_bwd_prep_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs) {
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || !supported_head(dk, dv)) return 0;
+  const size_t ck = kda::bwd::bwd_workspace_bytes(B, T, H, dk, num_seqs);
+  return kda::bwd::prep_bwd_layout(ck, (long long)B * T * H, dk).total;
+}
+
+kda_status_t kda_chunk_bwd_prep(const void* q, const void* k, const void* v, const void* a, kda_dtype_t a_dtype,
+                                const float* b, const float* S0, const void* dout, const float* dS_T, float* dq,
+                                float* dk, float* dv, float* da, float* db, float* dS0, const int32_t* cu_seqlens,
+                                int num_seqs, int B, int T, int H, int dkh, int dvh, kda_dtype_t dtype,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const char* fn = "kda_chunk_bwd_prep";
+  t_err[0] = 0;
+  if (B < 0 || T < 0 || H <= 0 || num_seqs < 0)
+    return fail(KDA_ERR_INVALID_ARG, "%s: bad sizes B=%d T=%d H=%d num_seqs=%d", fn, B, T, H, num_seqs);
+  if (dtype != KDA_BF16 && dtype != KDA_F32) return fail(KDA_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, (int)dtype);
+  if (a_dtype != KDA_BF16 && a_dtype != KDA_F32)
+    return fail(KDA_ERR_UNSUPPORTED, "%s: unknown a_dtype %d", fn, (int)a_dtype);
+  if (!supported_head(dkh, dvh))
+    return fail(KDA_ERR_UNSUPPORTED, "%s: dk=%d dv=%d (need dk == dv in {32,64,128})", fn, dkh, dvh);
+  if (cu_seqlens) {
+    if (B != 1) return fail(KDA_ERR_INVALID_ARG, "%s: packed inputs need B == 1", fn);
+    if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "%s: cu_seqlens needs num_seqs >= 1", fn);
+  } else if (num_seqs != 0) {
+    return fail(KDA_ERR_INVALID_ARG, "%s: num_seqs=%d without cu_seqlens", fn, num_seqs);
+  }
+  const int N = cu_seqlens ? num_seqs : B;
+  if (N == 0) return KDA_OK;
+  const long long tokens = (long long)B * T;
+  if (tokens > 0 && (!q || !k || !v || !a || !b || !dout || !dq || !dk || !dv || !da || !db))
+    return fail(KDA_ERR_INVALID_ARG, "%s: null input/output pointer", fn);
+  const unsigned esz = dtype == KDA_F32 ? 4u : 2u, aesz = a_dtype == KDA_F32 ? 4u : 2u;
+  const void* in_ptrs[] = {q, k, v, dout};
+  for (const void* p : in_ptrs)
+    if (p && !aligned_to(p, esz)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is misaligned", fn, p);
+  if (a && !aligned_to(a, aesz)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is misaligned", fn, a);
+  const void* f_ptrs[] = {b, S0, dS_T, dq, dk, dv, da, db, dS0, cu_seqlens, workspace};
+  for (const void* p : f_ptrs)
+    if (p && !aligned_to(p, 4)) return fail(KDA_ERR_ALIGNMENT, "%s: pointer %p is not 4-byte aligned", fn, p);
+  {  // outputs are written while inputs are still read: no aliasing
+    const void* outs[] = {dq, dk, dv, da, db, dS0, workspace};
+    const void* ins[] = {q, k, v, a, b, S0, dout, dS_T};
+    for (int i = 0; i < 7; ++i) {
+      if (!outs[i]) continue;
+      for (const void* p : ins)
+        if (p == outs[i]) return fail(KDA_ERR_INVALID_ARG, "%s: an output aliases an input (%p)", fn, p);
+      for (int j = i + 1; j < 7; ++j)
+        if (outs[j] == outs[i]) return fail(KDA_ERR_INVALID_ARG, "%s: two outputs alias (%p)", fn, outs[i]);
+    }
+  }
+  const size_t need = kda_chunk_bwd_prep_workspace_size(B, T, H, dkh, dvh, num_seqs);
+  if (need && (!workspace || workspace_bytes < need))
+    return fail(KDA_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", fn, workspace_bytes, need);
+  const size_t ck = kda::bwd::bwd_workspace_bytes(B, T, H, dkh, num_seqs);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int a_bf16 = a_dtype == KDA_BF16;
+  cudaError_t e = cudaErrorInvalidValue;
+#define KDA_BWD_PREP_CASE(TT, DD)                                                                           \
+  e = kda::bwd::launch_chunk_bwd_prep<TT, DD>(q, k, v, a, a_bf16, b, S0, dout, dS_T, dq, dk, dv, da, db, dS0, \
+                                              cu_seqlens, N, B, T, H, ck, ws, stream)
+  if (dtype == KDA_F32) {
+    if (dkh == 32) KDA_BWD_PREP_CASE(float, 32); else if (dkh == 64) KDA_BWD_PREP_CASE(float, 64); else KDA_BWD_PREP_CASE(float, 128);
+  } else {
+    if (dkh == 32) KDA_BWD_PREP_CASE(__nv_bfloat16, 32);
+    else if (dkh == 64) KDA_BWD_PREP_CASE(__nv_bfloat16, 64);
+    else KDA_BWD_PREP_CASE(__nv_bfloat16, 128);
+  }
+#undef KDA_BWD_PREP_CASE
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return KDA_OK;
+}
+
 kda_status_t kda_set_segment_chunks(int chunks) {
   t_err[0] = 0;
   t_seg_force = chunks;

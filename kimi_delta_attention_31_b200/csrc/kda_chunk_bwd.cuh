@@ -480,5 +480,162 @@ inline size_t bwd_workspace_bytes(int B, int T, int H, int D, int num_seqs) {
   return (size_t)slots * H * D * D * sizeof(float);
 }
 
+// ---- backward of the prefill from raw projections (kda_chunk_fwd_prep).
+// The preparation of that entry point, per token-head row:
+//   q^ = q / max(|q|, 1e-12),  k^ likewise,  g = -softplus(a),  beta = sigmoid(b)
+// composed with the recurrence, so its gradients are the recurrence's (taken
+// on the prepared inputs in fp32) through the preparation's Jacobians:
+//   dq = (dq^ - q^ (q^ . dq^)) / |q|   (dq^ / 1e-12 where the clamp holds)
+//   da = -sigmoid(a) dg,   db = beta (1 - beta) dbeta.
+
+// Workspace after the checkpoints: fp32 q^, k^ [rows][D], v, dO [rows][D],
+// g [rows][D], beta [rows], and the rows' sums of squares of q and k.
+struct PrepBwdLayout {
+  size_t qn, kn, vf, dof, g, beta, sq, sk, total;
+};
+inline PrepBwdLayout prep_bwd_layout(size_t ckpt_bytes, long long rows, int D) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  PrepBwdLayout L;
+  const size_t mat = up((size_t)rows * D * sizeof(float)), vec = up((size_t)rows * sizeof(float));
+  L.qn = up(ckpt_bytes);
+  L.kn = L.qn + mat;
+  L.vf = L.kn + mat;
+  L.dof = L.vf + mat;
+  L.g = L.dof + mat;
+  L.beta = L.g + mat;
+  L.sq = L.beta + vec;
+  L.sk = L.sq + vec;
+  L.total = L.sk + vec;
+  return L;
+}
+
+// The preparation, one warp per token-head row, in the forward's arithmetic
+// (rsqrt of the clamped sum of squares, the same -softplus and sigmoid).
+template <typename TIn, int D>
+__global__ void __launch_bounds__(256)
+    kda_bwd_prep_in_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
+                           const TIn* __restrict__ dout, const void* __restrict__ a, int a_bf16,
+                           const float* __restrict__ b, float* __restrict__ qn, float* __restrict__ kn,
+                           float* __restrict__ vf, float* __restrict__ dof, float* __restrict__ g,
+                           float* __restrict__ beta, float* __restrict__ sq, float* __restrict__ sk,
+                           long long rows) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows; row += warps) {
+    const size_t base = (size_t)row * D;
+    float xq[D / 32], xk[D / 32], ssq = 0.f, ssk = 0.f;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      xq[i] = to_f32(q[base + lane + 32 * i]);
+      xk[i] = to_f32(k[base + lane + 32 * i]);
+      ssq = fmaf(xq[i], xq[i], ssq);
+      ssk = fmaf(xk[i], xk[i], ssk);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+      ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
+    }
+    const float rq = rsqrtf(fmaxf(ssq, 1e-24f)), rk = rsqrtf(fmaxf(ssk, 1e-24f));
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const size_t e = base + lane + 32 * i;
+      qn[e] = xq[i] * rq;
+      kn[e] = xk[i] * rk;
+      vf[e] = to_f32(v[e]);
+      dof[e] = to_f32(dout[e]);
+      const float av = a_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a)[e]) : static_cast<const float*>(a)[e];
+      g[e] = neg_softplus(av);
+    }
+    if (lane == 0) {
+      beta[row] = sigmoid_f(b[row]);
+      sq[row] = ssq;
+      sk[row] = ssk;
+    }
+  }
+}
+
+// The chain rule through the preparation, in place over the recurrence's
+// gradients: dq, dk (with respect to q^, k^), da (holding dg) and db (holding
+// dbeta).  One warp per token-head row.
+template <int D>
+__global__ void __launch_bounds__(256)
+    kda_bwd_prep_out_kernel(const float* __restrict__ qn, const float* __restrict__ kn,
+                            const float* __restrict__ sq, const float* __restrict__ sk, const void* __restrict__ a,
+                            int a_bf16, const float* __restrict__ beta, float* __restrict__ dq,
+                            float* __restrict__ dk, float* __restrict__ da, float* __restrict__ db, long long rows) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows; row += warps) {
+    const size_t base = (size_t)row * D;
+    float dqv[D / 32], dkv[D / 32], pq = 0.f, pk = 0.f;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const size_t e = base + lane + 32 * i;
+      dqv[i] = dq[e];
+      dkv[i] = dk[e];
+      pq = fmaf(qn[e], dqv[i], pq);
+      pk = fmaf(kn[e], dkv[i], pk);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      pq += __shfl_xor_sync(0xffffffffu, pq, o);
+      pk += __shfl_xor_sync(0xffffffffu, pk, o);
+    }
+    const float ssq = sq[row], ssk = sk[row];
+    const float rq = rsqrtf(fmaxf(ssq, 1e-24f)), rk = rsqrtf(fmaxf(ssk, 1e-24f));
+    // where the clamp holds, q^ = q / 1e-12 is linear in q: no projection
+    if (!(ssq > 1e-24f)) pq = 0.f;
+    if (!(ssk > 1e-24f)) pk = 0.f;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const size_t e = base + lane + 32 * i;
+      dq[e] = (dqv[i] - qn[e] * pq) * rq;
+      dk[e] = (dkv[i] - kn[e] * pk) * rk;
+      const float av = a_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a)[e]) : static_cast<const float*>(a)[e];
+      da[e] = -sigmoid_f(av) * da[e];
+    }
+    if (lane == 0) {
+      const float bt = beta[row];
+      db[row] = bt * (1.f - bt) * db[row];
+    }
+  }
+}
+
+// The three launches of the raw-projection backward; ws = the workspace
+// (checkpoints first, then the layout above).
+template <typename TIn, int D>
+cudaError_t launch_chunk_bwd_prep(const void* q, const void* k, const void* v, const void* a, int a_bf16,
+                                  const float* b, const float* S0, const void* dout, const float* dS_T, float* dq,
+                                  float* dk, float* dv, float* da, float* db, float* dS0,
+                                  const int32_t* cu_seqlens, int N, int B, int T, int H, size_t ckpt_bytes,
+                                  uint8_t* ws, cudaStream_t stream) {
+  const long long rows = (long long)B * T * H;
+  const PrepBwdLayout L = prep_bwd_layout(ckpt_bytes, rows, D);
+  float* qn = reinterpret_cast<float*>(ws + L.qn);
+  float* kn = reinterpret_cast<float*>(ws + L.kn);
+  float* vf = reinterpret_cast<float*>(ws + L.vf);
+  float* dof = reinterpret_cast<float*>(ws + L.dof);
+  float* g = reinterpret_cast<float*>(ws + L.g);
+  float* beta = reinterpret_cast<float*>(ws + L.beta);
+  float* sq = reinterpret_cast<float*>(ws + L.sq);
+  float* sk = reinterpret_cast<float*>(ws + L.sk);
+  if (rows > 0) {
+    const unsigned blocks = (unsigned)std::min<long long>((rows + 7) / 8, 148LL * 16);
+    kda_bwd_prep_in_kernel<TIn, D><<<blocks, 256, 0, stream>>>(
+        static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v),
+        static_cast<const TIn*>(dout), a, a_bf16, b, qn, kn, vf, dof, g, beta, sq, sk, rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = launch_chunk_bwd<float, D, kGateLogCh>(qn, kn, vf, g, beta, S0, dof, dS_T, dq, dk, dv, da, db,
+                                                         dS0, cu_seqlens, N, T, H,
+                                                         reinterpret_cast<float*>(ws), stream);
+  if (e != cudaSuccess || rows == 0) return e;
+  const unsigned blocks = (unsigned)std::min<long long>((rows + 7) / 8, 148LL * 16);
+  kda_bwd_prep_out_kernel<D><<<blocks, 256, 0, stream>>>(qn, kn, sq, sk, a, a_bf16, beta, dq, dk, da, db, rows);
+  return cudaGetLastError();
+}
+
 }  // namespace bwd
 }  // namespace kda

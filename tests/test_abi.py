@@ -258,6 +258,13 @@ def test_backward_bindings_check_the_gate_layout_before_any_launch():
             fn(q, q, q, other, beta, q)                        # the other gate layout
         with pytest.raises(ValueError):
             fn(q, q, q, good, beta, q)                         # right shapes, host tensors
+    a = torch.zeros(B, T, H, d, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        kda.chunk_bwd_prep(q, q, q, a.to(torch.float16), beta, q)   # half-precision gate logits
+    with pytest.raises(ValueError):
+        kda.chunk_bwd_prep(q, q, q, a[..., 0].contiguous(), beta, q)  # a of shape [B,T,H]
+    with pytest.raises(ValueError):
+        kda.chunk_bwd_prep(q, q, q, a, beta, q)                   # right shapes, host tensors
 
 
 def test_host_entry_point_sizes_and_argument_checks():

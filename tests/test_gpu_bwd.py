@@ -1,5 +1,6 @@
-"""GPU parity of the backward pass (kda_chunk_bwd, and kda_gdn_chunk_bwd for
-one gate per token and head) against the gradient oracle (reverse-mode
+"""GPU parity of the backward pass (kda_chunk_bwd; kda_gdn_chunk_bwd for one
+gate per token and head; kda_chunk_bwd_prep from raw projections) against
+the gradient oracle (reverse-mode
 differentiation of the fp64 token recurrence).  The
 kernel computes in fp32 from the same (bf16- or fp32-rounded) inputs the
 oracle widens, so both dtypes are held to 1e-4 relative RMS per (sequence,
@@ -10,7 +11,7 @@ import torch
 
 import kimi_delta_attention_31_b200 as kda
 import kda_workloads as W
-from oracle.grad import gdn_recurrent_grad, recurrent_grad
+from oracle.grad import gdn_recurrent_grad, recurrent_grad, recurrent_prep_grad
 from parity_util import rel_rms
 
 pytestmark = pytest.mark.gpu
@@ -152,3 +153,60 @@ def test_gdn_bwd_equals_the_per_channel_bwd_on_the_repeated_gate(cuda_device):
         assert rel_rms(out[n].double().cpu().numpy(), ref[n].double().cpu().numpy()) <= 1e-6, n
     err = rel_rms(out["dg"].double().cpu().numpy(), ref["dg"].sum(-1).double().cpu().numpy())
     assert err <= 1e-6, err
+
+
+# ---- from raw projections (q, k unnormalised; gate and beta logits)
+
+def _raw(dev, B, T, H, d, dtype, a_dtype, seed, lengths=None):
+    inp = W.make_prefill_raw(B, T, H, d, d, dtype, -5.0, 1.5, a_dtype, 0.05, seed=seed, device=dev, lengths=lengths)
+    gen = torch.Generator(device=dev).manual_seed(seed + 1)
+    inp["do"] = torch.randn(inp["v"].shape, generator=gen, device=dev).to(inp["q"].dtype)
+    N = len(lengths) if lengths else B
+    inp["dS_T"] = torch.randn((N, H, d, d), generator=gen, device=dev) * 0.1
+    return inp
+
+
+def _compare_prep(inp, out, seqs):
+    """seqs: list of (batch row, token range) per sequence."""
+    cpu = {n: t.double().cpu().numpy() for n, t in inp.items() if n != "cu_seqlens" and t is not None}
+    H = cpu["q"].shape[2]
+    for s_i, (b, a0, a1) in enumerate(seqs):
+        for h in range(H):
+            sl = lambda x: x[b:b + 1, a0:a1, h:h + 1]
+            ref = recurrent_prep_grad(sl(cpu["q"]), sl(cpu["k"]), sl(cpu["v"]), sl(cpu["a"]), sl(cpu["b"]),
+                                      cpu["S0"][s_i:s_i + 1, h:h + 1], sl(cpu["do"]), cpu["dS_T"][s_i:s_i + 1, h:h + 1])
+            for n in ("dq", "dk", "dv", "da", "db"):
+                _check_slices(out[n][b:b + 1, a0:a1, h:h + 1].double().cpu().numpy(), ref[n], f"{n} seq{s_i} h{h}")
+            _check_slices(out["dS0"][s_i:s_i + 1, h:h + 1].double().cpu().numpy(), ref["dS0"], f"dS0 seq{s_i}")
+
+
+@pytest.mark.parametrize("dtype,a_dtype,d,T", [("f32", "f32", 64, 40), ("bf16", "bf16", 64, 40),
+                                               ("bf16", "f32", 32, 17), ("bf16", "bf16", 128, 33)])
+def test_prep_bwd_matches_the_oracle(cuda_device, dtype, a_dtype, d, T):
+    inp = _raw(cuda_device, 2, T, 2, d, dtype, a_dtype, seed=800 + d + T)
+    out = kda.chunk_bwd_prep(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["do"], inp["S0"], inp["dS_T"])
+    torch.cuda.synchronize()
+    assert kda.device_error() == 0
+    _compare_prep(inp, out, [(b, 0, T) for b in range(2)])
+
+
+def test_prep_bwd_packed_and_a_zero_query_row(cuda_device):
+    """Packed sequences (one empty), and one token whose q is all zeros: its
+    norm is clamped at 1e-12, where the normalisation is linear."""
+    lens = (9, 0, 40, 16)
+    inp = _raw(cuda_device, 1, sum(lens), 2, 64, "f32", "f32", seed=81, lengths=lens)
+    inp["q"][0, 3, 1].zero_()
+    out = kda.chunk_bwd_prep(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["do"], inp["S0"], inp["dS_T"],
+                             cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    cu = np.cumsum((0,) + lens)
+    for s_i in range(len(lens)):
+        if lens[s_i] == 0:
+            assert torch.allclose(out["dS0"][s_i], inp["dS_T"][s_i])
+    seqs = [(0, cu[i], cu[i + 1]) for i in range(len(lens))]
+    keep = [i for i in range(len(lens)) if lens[i] > 0]
+    sub = dict(inp)
+    sub["S0"], sub["dS_T"] = inp["S0"][keep], inp["dS_T"][keep]
+    out_sub = dict(out)
+    out_sub["dS0"] = out["dS0"][keep]
+    _compare_prep(sub, out_sub, [seqs[i] for i in keep])
