@@ -477,12 +477,38 @@ def bwd_leg(kda, args, world, dev, stream, peaks):
     # plus the fp32 state checkpoint written and read once per 16-token chunk
     alg = th * (4 * 2 * d + 4 * d + 4 + 4 * 4 * d + 4) + 2 * (th // 16) * d * d * 4
     gbs = alg / (ms * 1e-3) / 1e9
-    del inp, dout, ws
+    del inp
     torch.cuda.empty_cache()
-    return {"workload": w.name, "value": world * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+    line = {"workload": w.name, "value": world * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "kernel": "kda_chunk_bwd_kernel<bf16,128>",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "alg_bytes_per_launch": alg, "traffic": None}}
+
+    # the same shape in the Gated DeltaNet form and from raw projections (one
+    # timed call each, after one untimed)
+    def timed_once(fn):
+        fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(time_launches(fn, 1, stream), world, dev)
+
+    gw = W.GDN_PREFILL_B8
+    ginp = W.make_workload(gw, dev)
+    gms = timed_once(lambda: kda.gdn_chunk_bwd(ginp["q"], ginp["k"], ginp["v"], ginp["g"], ginp["beta"], dout,
+                                               None, None, workspace=ws, need_dS0=False))
+    line["gdn"] = {"workload": gw.name, "value": world * B * T / (gms * 1e-3), "ms_per_step": gms}
+    del ginp, ws
+    torch.cuda.empty_cache()
+    pw = W.PREP_PREFILL_B8
+    pinp = W.make_workload(pw, dev)
+    pws = torch.empty(max(int(kda.load_library().kda_chunk_bwd_prep_workspace_size(B, T, H, d, d, 0)), 1),
+                      dtype=torch.uint8, device=dev)
+    pms = timed_once(lambda: kda.chunk_bwd_prep(pinp["q"], pinp["k"], pinp["v"], pinp["a"], pinp["b"], dout,
+                                                None, None, workspace=pws, need_dS0=False))
+    line["prep"] = {"workload": pw.name, "value": world * B * T / (pms * 1e-3), "ms_per_step": pms}
+    del pinp, pws, dout
+    torch.cuda.empty_cache()
+    return line
 
 
 def prefill_roofline(kda, w, ms, kernel_ms, peaks, peak_src, with_state_in):
