@@ -474,7 +474,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // it, so that the whole group leaves together after a timeout.
       bool ok = true;
       if constexpr (kTmaGate) ok = wait_or_abort(&s_g_full, n & 1, abort_flag);
-      if constexpr (kPrep) ok = ok && wait_or_abort(&s_kq_full[s], (n >> 1) & 1, abort_flag);
 
       // ---- raw gate rows -> local cumulative sums; rows >= Cn contribute g = 0
       float G[4][8];
@@ -508,32 +507,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) G[u][e] = (u ? G[u - 1][e] : 0.f) + x[e];
-      }
-      // 1 / |k_r| and 1 / |q_r| over dk (only when the call normalises): the 16
-      // lanes of a half-warp hold one row; k and q are read from their panels.
-      if constexpr (kPrep) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int r = 4 * rg + u;
-          float kx[8], qx[8];
-          tc::unpack8(*reinterpret_cast<const uint4*>(l3 + kp * 16384 + ptx::sw128_chunk(r, ck)), kx);
-          tc::unpack8(*reinterpret_cast<const uint4*>(l3 + kp * 16384 + 8192 + ptx::sw128_chunk(r, ck)), qx);
-          float sk = 0.f, sq = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            sk = fmaf(kx[e], kx[e], sk);
-            sq = fmaf(qx[e], qx[e], sq);
-          }
-#pragma unroll
-          for (int off = 1; off < 16; off <<= 1) {
-            sk += __shfl_xor_sync(0xffffffffu, sk, off);
-            sq += __shfl_xor_sync(0xffffffffu, sq, off);
-          }
-          if (co == 0) {
-            s_nrm[0][r] = rsqrtf(fmaxf(sk, 1e-24f));
-            s_nrm[1][r] = rsqrtf(fmaxf(sq, 1e-24f));
-          }
-        }
       }
       // Row-group totals: this warp holds row groups 2w (lanes 0..15) and 2w+1
       // (lanes 16..31) of the same channels; the warp's total goes to s_wtot,
@@ -585,10 +558,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool fast = !ptx::bar_or(1, 256, steep);
       if (fast && tid == 0) issue_g(n + 1, &g_issued);  // the raw gate buffer is free
 
-      ok = true;
-      if constexpr (!kPrep) ok = wait_or_abort(&s_kq_full[s], (n >> 1) & 1, abort_flag);
+      ok = wait_or_abort(&s_kq_full[s], (n >> 1) & 1, abort_flag);
       // K e^-G, gamma of this slot: the state is done with chunk n-2
       if (n >= 2) ok = ok && wait_or_abort(&s_rb_free[s], ((n - 2) >> 1) & 1, abort_flag);
+      // 1 / |k_r| and 1 / |q_r| over dk (only when the call normalises), once k
+      // and q have landed (the gate phase above overlaps their copy): the 16
+      // lanes of a half-warp hold one row; k and q are read from their panels.
+      if constexpr (kPrep) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = 4 * rg + u;
+          float kx[8], qx[8];
+          tc::unpack8(*reinterpret_cast<const uint4*>(l3 + kp * 16384 + ptx::sw128_chunk(r, ck)), kx);
+          tc::unpack8(*reinterpret_cast<const uint4*>(l3 + kp * 16384 + 8192 + ptx::sw128_chunk(r, ck)), qx);
+          float sk = 0.f, sq = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            sk = fmaf(kx[e], kx[e], sk);
+            sq = fmaf(qx[e], qx[e], sq);
+          }
+#pragma unroll
+          for (int off = 1; off < 16; off <<= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+          }
+          if (co == 0) {
+            s_nrm[0][r] = rsqrtf(fmaxf(sk, 1e-24f));
+            s_nrm[1][r] = rsqrtf(fmaxf(sq, 1e-24f));
+          }
+        }
+      }
       if (ptx::bar_or(1, 256, !ok || *abort_flag)) break;
       if (tid < C) s_beta[s][tid] = bt;  // the solver is done with chunk n-2's
 
