@@ -299,7 +299,9 @@ kda_status_t kda_chunk_fwd_host(const void* q, const void* k, const void* v, con
  * Its scratch is a fixed array inside the library, KDA_NOALLOC_SCRATCH_BYTES
  * bytes on every GPU that loads the library, held until process exit.  Sizes
  * whose kda_chunk_fwd_workspace_size(...) exceeds it are rejected with
- * KDA_ERR_WORKSPACE.  The single-pass tensor-core prefill (see
+ * KDA_ERR_WORKSPACE, except that where the automatic sequence segments
+ * (kda_set_segment_chunks, left at 0) make the difference, the call runs
+ * without them.  The single-pass tensor-core prefill (see
  * kda_set_prefill_path) needs 256 + 4 * (num_seqs + N * H) bytes, the
  * fp32-arithmetic path none; the two-kernel path keeps a per-chunk image and
  * can exceed it: 64 MiB hold 903 of its (chunk, head) pairs, e.g. B=1, H=8,

@@ -690,19 +690,33 @@ kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, 
   if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || chunk_size <= 0)
     return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_noalloc: bad sizes B=%d T=%d H=%d num_seqs=%d", B, T,
                 H, num_seqs);
-  const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
-  if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES)
+  size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
+  // The automatic sequence segments are a speed choice whose state maps take
+  // scratch too: where they would not fit, this call runs without them.
+  const int seg_setting = t_seg_force;
+  if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES && seg_setting == 0) {
+    t_seg_force = -1;
+    need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
+  }
+  if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES) {
+    t_seg_force = seg_setting;
     return fail(KDA_ERR_WORKSPACE,
                 "kda_chunk_fwd_noalloc: these sizes need %zu bytes of scratch, more than the built-in "
                 "%zu-byte array; use kda_chunk_fwd with a caller-provided workspace",
                 need, (size_t)KDA_NOALLOC_SCRATCH_BYTES);
+  }
   void* scratch = nullptr;
   if (need > 0) {
     const kda_status_t st = noalloc_scratch(&scratch);
-    if (st != KDA_OK) return st;
+    if (st != KDA_OK) {
+      t_seg_force = seg_setting;
+      return st;
+    }
   }
-  return kda_chunk_fwd(q, k, v, g, beta, S0, o, S_out, cu_seqlens, num_seqs, B, T, H, dk, dv,
-                       chunk_size, dtype, scratch, need, stream);
+  const kda_status_t st = kda_chunk_fwd(q, k, v, g, beta, S0, o, S_out, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                                        chunk_size, dtype, scratch, need, stream);
+  t_seg_force = seg_setting;
+  return st;
 }
 
 }  // extern "C"

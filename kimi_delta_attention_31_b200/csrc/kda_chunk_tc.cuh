@@ -1365,7 +1365,7 @@ inline int tc_segment_chunks(int B, int T, int H, int num_seqs, int sms, int for
   const long long nc = (T + tc::C - 1) / tc::C;
   if (force > 0) return force < nc ? force : 0;
   const long long units = (long long)B * H;
-  if (2 * units > sms || nc < 128) return 0;
+  if (2 * units > sms || nc < 64) return 0;
   auto waves = [&](long long n) { return (n + sms - 1) / sms; };
   long long best_cost = waves(units) * nc;
   int best_L = 0;

@@ -63,7 +63,9 @@ def test_no_segments_where_units_fill_the_gpu(cuda_device, segments):
     segments(0)
     assert kda.segment_chunks(8, 8192, 32) == 0      # the headline shape
     assert kda.segment_chunks(1, 520998, 32, 16) == 0  # packed inputs are never split
-    assert kda.segment_chunks(1, 4096, 4) == 0        # too short to pay off
+    assert kda.segment_chunks(1, 2048, 4) == 0        # 32 chunks: too short to pay off
+    assert kda.segment_chunks(1, 4096, 16) == 16      # 64 chunks, 16 units: measured 0.247 -> 0.185 ms
+    assert kda.segment_chunks(4, 4096, 16) == 0       # 64 units: measured no gain
 
 
 def test_segments_with_the_final_state_aliasing_the_initial_state(cuda_device, segments):

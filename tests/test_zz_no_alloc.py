@@ -1,8 +1,9 @@
 """kda_chunk_fwd_noalloc: the prefill for callers that cannot allocate device
 memory (for example a plug-in handed only input and output pointers by a host
 framework that owns the device memory pool).  It runs the very same kernels as
-kda_chunk_fwd with a caller-allocated workspace, so its results must be
-bit-for-bit the same, call after call (its built-in scratch array is reused
+kda_chunk_fwd with a caller-allocated workspace (without the automatic
+sequence segments where their maps would not fit its array), so its results
+must be bit-for-bit the same, call after call (its built-in scratch array is reused
 and keeps the previous call's contents); it must refuse sizes its array cannot
 hold and check its arguments exactly as chunk_fwd does.
 
@@ -44,14 +45,26 @@ def test_noalloc_packed_sequences(cuda_device):
 
 def test_noalloc_at_its_documented_limit(cuda_device):
     # the two-kernel path keeps a per-chunk image: B=1, H=8, T=7168 (112 chunks x
-    # 8 heads) is the largest case kda.h names for it
+    # 8 heads) is the largest case kda.h names for it.  Its automatic sequence
+    # segments add state maps; where those would not fit the array, the
+    # no-alloc call runs without them, so the reference runs the same way.
+    sizes = (1, 7168, 8, 128, 128, 0, 64, torch.bfloat16)
     kda.set_prefill_path(kda.PATH_TWO_KERNEL)
     try:
-        need = kda.workspace_size(1, 7168, 8, 128, 128, 0, 64, torch.bfloat16)
-        assert 0 < need <= kda.NOALLOC_SCRATCH_BYTES
+        need_auto = kda.workspace_size(*sizes)
+        kda.set_segment_chunks(-1)
+        need_plain = kda.workspace_size(*sizes)
+        assert 0 < need_plain <= kda.NOALLOC_SCRATCH_BYTES
         x = W.make_prefill(1, 7168, 8, 128, 128, "bf16", -4.0, 1.0, 0.02, seed=905, device=cuda_device)
-        _same(x, *_both(x))
+        kda.set_segment_chunks(-1 if need_auto > kda.NOALLOC_SCRATCH_BYTES else 0)
+        ref_o, ref_S = kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], None, 64)
+        kda.set_segment_chunks(0)  # the no-alloc call decides for itself
+        o, S = kda.chunk_fwd_noalloc(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], None, 64)
+        torch.cuda.synchronize()
+        _same(x, ref_o, ref_S, o, S)
+        assert kda.device_error() == 0
     finally:
+        kda.set_segment_chunks(0)
         kda.set_prefill_path(kda.PATH_AUTO)
 
 
