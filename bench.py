@@ -672,17 +672,13 @@ def packed_shard_leg(kda, w, args, world, rank, dev, stream):
     workload; no collective touches the data."""
     if world <= 1:
         return None
-    from kimi_delta_attention_31_b200.sharding import assign_sequences_lpt, packed_subset
+    from kimi_delta_attention_31_b200.sharding import rank_share
     inp = W.make_workload(w, dev)
-    mine = assign_sequences_lpt(w.lengths, world)[rank]
-    ranges, cu = packed_subset(w.lengths, mine)
+    sub, mine, cu = rank_share(inp, w.lengths, world, rank)
     tokens = cu[-1]
     run = None
     if tokens > 0:
-        idx = torch.cat([torch.arange(a, b, dtype=torch.long) for a, b in ranges]).to(dev)
-        sub = {n: inp[n].index_select(1, idx).contiguous() for n in ("q", "k", "v", "g", "beta")}
-        S0 = inp["S0"][torch.tensor(mine, dtype=torch.long, device=dev)].contiguous() \
-            if inp["S0"] is not None else None
+        S0 = sub["S0"]
         cu_t = torch.tensor(cu, dtype=torch.int32, device=dev)
         o = torch.empty((1, tokens, w.H, w.dv), dtype=w.torch_dtype, device=dev)
         S_out = torch.empty((len(mine), w.H, w.dk, w.dv), dtype=torch.float32, device=dev)

@@ -3,8 +3,8 @@
 Every (sequence, head) unit of the recurrence is independent of every other
 one, in the prefill and in decode, so the work splits across ranks with no
 exchange on the data path: each rank runs the kernels on its own sequences
-(or heads) and owns their outputs and final states.  This module only
-decides who gets what.
+(or heads) and owns their outputs and final states.  This module decides who
+gets what, and gathers a rank's share of a packed batch on its own device.
 """
 from __future__ import annotations
 
@@ -48,3 +48,23 @@ def packed_subset(lengths: Sequence[int], seqs: Sequence[int]):
     for a, b in ranges:
         cu.append(cu[-1] + (b - a))
     return ranges, cu
+
+
+def rank_share(tensors, lengths: Sequence[int], world: int, rank: int):
+    """One rank's share of a packed batch: the sequences assign_sequences_lpt
+    gives it, re-packed contiguously along the token axis (axis 1 of q, k, v,
+    g and beta, each [1, T, ...]), with the rows of S0 ([N, ...], optional)
+    that belong to them.  `tensors` maps those names to torch tensors on one
+    device.  Returns (share, seqs, cu): the re-packed tensors, the sequence
+    indices in their original order, and the share's cu_seqlens as a list."""
+    import torch
+    seqs = assign_sequences_lpt(lengths, world)[rank]
+    ranges, cu = packed_subset(lengths, seqs)
+    dev = tensors["q"].device
+    idx = (torch.cat([torch.arange(a, b, dtype=torch.long) for a, b in ranges]) if ranges
+           else torch.zeros(0, dtype=torch.long)).to(dev)
+    share = {n: tensors[n].index_select(1, idx).contiguous() for n in ("q", "k", "v", "g", "beta")}
+    S0 = tensors.get("S0")
+    share["S0"] = (S0.index_select(0, torch.tensor(seqs, dtype=torch.long, device=dev)).contiguous()
+                   if S0 is not None else None)
+    return share, seqs, cu

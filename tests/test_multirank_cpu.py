@@ -12,7 +12,7 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from kimi_delta_attention_31_b200.sharding import assign_sequences_lpt, packed_subset, shard_range
+from kimi_delta_attention_31_b200.sharding import assign_sequences_lpt, packed_subset, rank_share, shard_range
 
 
 def test_lpt_assignment_partitions_and_balances():
@@ -41,11 +41,15 @@ def _rank_main(rank, world, init_file, lengths, out_file):
         v = rng.standard_normal((1, T, H, d))
         g = -rng.random((1, T, H, d))
         beta = rng.random((1, T, H))
-        mine = assign_sequences_lpt(lengths, world)[rank]
-        ranges, cu = packed_subset(lengths, mine)
+        # the benchmark's own gathering of a rank's share (torch tensors)
+        share, mine, cu = rank_share({"q": torch.from_numpy(q), "k": torch.from_numpy(k), "v": torch.from_numpy(v),
+                                      "g": torch.from_numpy(g), "beta": torch.from_numpy(beta), "S0": None},
+                                     lengths, world, rank)
+        ranges, cu2 = packed_subset(lengths, mine)
+        assert cu == cu2 and share["S0"] is None
         idx = np.concatenate([np.arange(a, b) for a, b in ranges]) if ranges else np.zeros(0, int)
-        sub = lambda x: x[:, idx]
-        o, S = oracle.recurrent(sub(q), sub(k), sub(v), sub(g), sub(beta), cu_seqlens=np.array(cu))
+        o, S = oracle.recurrent(share["q"].numpy(), share["k"].numpy(), share["v"].numpy(), share["g"].numpy(),
+                                share["beta"].numpy(), cu_seqlens=np.array(cu))
         # max over ranks of a per-rank "time", as the benchmark reports it
         t = torch.tensor([float(rank + 1)], dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -74,3 +78,26 @@ def test_two_gloo_ranks_shard_sequences_without_exchange():
         mp.start_processes(_rank_main, args=(2, init_file, lengths, out_file), nprocs=2, join=True,
                            start_method="spawn")
         assert open(out_file).read() == "ok"
+
+
+def test_rank_share_repacks_tokens_and_initial_states():
+    """Each rank's share holds exactly its sequences' tokens, in order, and
+    their rows of S0; together the shares cover the batch once."""
+    lengths = [13, 40, 7, 0, 25, 31]
+    T, H, d = sum(lengths), 2, 4
+    gen = torch.Generator().manual_seed(5)
+    full = {n: torch.randn((1, T, H, d), generator=gen) for n in ("q", "k", "v", "g")}
+    full["beta"] = torch.rand((1, T, H), generator=gen)
+    full["S0"] = torch.randn((len(lengths), H, d, d), generator=gen)
+    starts = np.cumsum([0] + lengths)
+    seen = []
+    for rank in range(3):
+        share, seqs, cu = rank_share(full, lengths, 3, rank)
+        assert cu[-1] == sum(lengths[s] for s in seqs) == share["q"].shape[1]
+        for j, s_i in enumerate(seqs):
+            a, b = starts[s_i], starts[s_i + 1]
+            for n in ("q", "k", "v", "g", "beta"):
+                assert torch.equal(share[n][:, cu[j]:cu[j + 1]], full[n][:, a:b])
+            assert torch.equal(share["S0"][j], full["S0"][s_i])
+        seen += seqs
+    assert sorted(seen) == list(range(len(lengths)))
