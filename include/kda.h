@@ -351,7 +351,8 @@ kda_status_t kda_selftest_bounded_wait(unsigned long long limit_ns, cudaStream_t
  * maps its entry state as S -> M S + N ("Linear / sparse attention" tutorial
  * section 6.2: the state handed from chunk to chunk; composing those hand-offs
  * is exact algebra).  When the (sequence, head) units are too few to fill the
- * GPU and the sequences are long, kda_chunk_fwd (and its _gdn / _prep forms)
+ * GPU and the sequences are long (64 chunks or more, when a wave-count model
+ * of the two schedules says it pays), kda_chunk_fwd (and its _gdn / _prep forms)
  * splits each sequence into segments: the maps of all segments are formed in
  * parallel, chained from S0 in fp32, and every segment is then run from its
  * entry state.  Packed (cu_seqlens) inputs are not split.  The workspace size
