@@ -126,19 +126,6 @@ constexpr uint32_t kTmS = 384;   // S^T fp32
 
 constexpr int kThreads = 640;  // builder 256, solver 256, state 128
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-
-// -softplus(a) = -(max(a, 0) + log(1 + y)), y = e^{-|a|} in (0, 1], on the
-// SFU's exp2 and log2 instead of log1pf: log(1 + y) directly when y >= 2^-8
-// (1 + y then rounds by at most 2^-24 of itself), else the series
-// y - y^2/2 + y^3/3, whose error is below y^4/4 < 2^-34.  A chunk's gate sum
-// (at most 64 terms) then carries an absolute error of a few 1e-6 at most,
-// far inside the tolerance of this bf16 path.
-__device__ __forceinline__ float neg_softplus_sfu(float a) {
-  const float y = ptx::ex2(-fabsf(a) * kLog2e);
-  const float l = y >= 0.00390625f ? __log2f(1.f + y) * kLn2 : y * (1.f - y * (0.5f - y * (1.f / 3.f)));
-  return -(fmaxf(a, 0.f) + l);
-}
 
 // Chunk descriptor.
 enum : int { kItFirst = 1, kItLast = 2, kItEmpty = 4, kItEnd = 8, kItSteep = 16 };
@@ -501,8 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else if constexpr (kGate == kGateLogitBf16) {
             float x[8];
             tc::unpack8(*reinterpret_cast<const uint4*>(sm + FU_RAWG + r * 256 + 16 * co), x);
-            a = make_float4(neg_softplus_sfu(x[0]), neg_softplus_sfu(x[1]), neg_softplus_sfu(x[2]), neg_softplus_sfu(x[3]));
-            b = make_float4(neg_softplus_sfu(x[4]), neg_softplus_sfu(x[5]), neg_softplus_sfu(x[6]), neg_softplus_sfu(x[7]));
+            a = make_float4(tc::neg_softplus_sfu(x[0]), tc::neg_softplus_sfu(x[1]), tc::neg_softplus_sfu(x[2]), tc::neg_softplus_sfu(x[3]));
+            b = make_float4(tc::neg_softplus_sfu(x[4]), tc::neg_softplus_sfu(x[5]), tc::neg_softplus_sfu(x[6]), tc::neg_softplus_sfu(x[7]));
           } else {
             // the two 16-byte halves in alternating order across the quarter-warp (no bank conflicts)
             const float* gr = reinterpret_cast<const float*>(sm + FU_RAWG + r * 512) + c0;
@@ -512,8 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             a = sw ? h1 : h0;
             b = sw ? h0 : h1;
             if constexpr (kGate == kGateLogitF32) {
-              a = make_float4(neg_softplus_sfu(a.x), neg_softplus_sfu(a.y), neg_softplus_sfu(a.z), neg_softplus_sfu(a.w));
-              b = make_float4(neg_softplus_sfu(b.x), neg_softplus_sfu(b.y), neg_softplus_sfu(b.z), neg_softplus_sfu(b.w));
+              a = make_float4(tc::neg_softplus_sfu(a.x), tc::neg_softplus_sfu(a.y), tc::neg_softplus_sfu(a.z), tc::neg_softplus_sfu(a.w));
+              b = make_float4(tc::neg_softplus_sfu(b.x), tc::neg_softplus_sfu(b.y), tc::neg_softplus_sfu(b.z), tc::neg_softplus_sfu(b.w));
             }
           }
         }

@@ -51,6 +51,21 @@ using bf16 = __nv_bfloat16;
 constexpr int C = 64;   // tokens per chunk
 constexpr int D = 128;  // dk = dv
 
+// -softplus(a) = -(max(a, 0) + log(1 + y)), y = e^{-|a|} in (0, 1], on the
+// SFU's exp2 and log2 instead of log1pf, for the bf16 tensor-core kernels'
+// gate logits: log(1 + y) directly when y >= 2^-8 (1 + y then rounds by at
+// most 2^-24 of itself), else the series y - y^2/2 + y^3/3, whose error is
+// below y^4/4 < 2^-34.  Its largest absolute error over a in [-40, 40] is
+// about 5e-7, so a chunk's gate sum (at most 64 terms) is off by a few 1e-6
+// at most, far inside those kernels' tolerance.  The fp32 path and the
+// backward keep log1pf.
+__device__ __forceinline__ float neg_softplus_sfu(float a) {
+  constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
+  const float y = ptx::ex2(-fabsf(a) * kLog2e);
+  const float l = y >= 0.00390625f ? __log2f(1.f + y) * kLn2 : y * (1.f - y * (0.5f - y * (1.f / 3.f)));
+  return -(fmaxf(a, 0.f) + l);
+}
+
 // Per (chunk, head) image: written by the chunk-local kernel, copied in one
 // piece by the state pass.  Offsets in bytes; every piece 1024-aligned.
 constexpr uint32_t IMG_P = 0;       // P     K-major [64 r][64 j]                 8192
@@ -662,15 +677,15 @@ __global__ void __launch_bounds__(256, 2)
       } else if constexpr (kGate == kGateLogitBf16) {
         float x[8];
         unpack8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(gate) + base8 + (size_t)r * rs), x);
-        a = make_float4(neg_softplus(x[0]), neg_softplus(x[1]), neg_softplus(x[2]), neg_softplus(x[3]));
-        b = make_float4(neg_softplus(x[4]), neg_softplus(x[5]), neg_softplus(x[6]), neg_softplus(x[7]));
+        a = make_float4(neg_softplus_sfu(x[0]), neg_softplus_sfu(x[1]), neg_softplus_sfu(x[2]), neg_softplus_sfu(x[3]));
+        b = make_float4(neg_softplus_sfu(x[4]), neg_softplus_sfu(x[5]), neg_softplus_sfu(x[6]), neg_softplus_sfu(x[7]));
       } else {
         const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(gate) + base8 + (size_t)r * rs);
         a = gp[0];
         b = gp[1];
         if constexpr (kGate == kGateLogitF32) {
-          a = make_float4(neg_softplus(a.x), neg_softplus(a.y), neg_softplus(a.z), neg_softplus(a.w));
-          b = make_float4(neg_softplus(b.x), neg_softplus(b.y), neg_softplus(b.z), neg_softplus(b.w));
+          a = make_float4(neg_softplus_sfu(a.x), neg_softplus_sfu(a.y), neg_softplus_sfu(a.z), neg_softplus_sfu(a.w));
+          b = make_float4(neg_softplus_sfu(b.x), neg_softplus_sfu(b.y), neg_softplus_sfu(b.z), neg_softplus_sfu(b.w));
         }
       }
     }

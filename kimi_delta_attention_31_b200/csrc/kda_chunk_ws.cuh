@@ -320,8 +320,8 @@ __global__ void __launch_bounds__(512, 1)
           } else if constexpr (kGate == kGateLogitBf16) {
             float x[8];
             tc::unpack8(*reinterpret_cast<const uint4*>(sm + WS_RAWG + r * 256 + 16 * co), x);
-            a = make_float4(neg_softplus(x[0]), neg_softplus(x[1]), neg_softplus(x[2]), neg_softplus(x[3]));
-            b = make_float4(neg_softplus(x[4]), neg_softplus(x[5]), neg_softplus(x[6]), neg_softplus(x[7]));
+            a = make_float4(tc::neg_softplus_sfu(x[0]), tc::neg_softplus_sfu(x[1]), tc::neg_softplus_sfu(x[2]), tc::neg_softplus_sfu(x[3]));
+            b = make_float4(tc::neg_softplus_sfu(x[4]), tc::neg_softplus_sfu(x[5]), tc::neg_softplus_sfu(x[6]), tc::neg_softplus_sfu(x[7]));
           } else {
             // the two 16-byte halves in alternating order across the quarter-warp (no bank conflicts)
             const float* gr = reinterpret_cast<const float*>(sm + WS_RAWG + r * 512) + c0;
@@ -331,8 +331,8 @@ __global__ void __launch_bounds__(512, 1)
             a = sw ? h1 : h0;
             b = sw ? h0 : h1;
             if constexpr (kGate == kGateLogitF32) {
-              a = make_float4(neg_softplus(a.x), neg_softplus(a.y), neg_softplus(a.z), neg_softplus(a.w));
-              b = make_float4(neg_softplus(b.x), neg_softplus(b.y), neg_softplus(b.z), neg_softplus(b.w));
+              a = make_float4(tc::neg_softplus_sfu(a.x), tc::neg_softplus_sfu(a.y), tc::neg_softplus_sfu(a.z), tc::neg_softplus_sfu(a.w));
+              b = make_float4(tc::neg_softplus_sfu(b.x), tc::neg_softplus_sfu(b.y), tc::neg_softplus_sfu(b.z), tc::neg_softplus_sfu(b.w));
             }
           }
         }
